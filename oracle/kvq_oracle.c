@@ -1,0 +1,496 @@
+/*
+ * kvq_oracle.c -- plain, slow, obviously-correct CPU oracle for the rotated
+ * INT2 KV-cache hot path (rotate -> quantize -> append, and decode attention
+ * over the packed cache).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file.  Only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or constant
+ * generator with the CUDA library: every formula below is written out again
+ * from the method description and from the cache-format specification.
+ *
+ * What the method computes (sources are the pages on the subject):
+ *   - "Output-Aware Rotation for INT2 KV-Cache Quantization", section
+ *     "Key Details": each head has an orthogonal rotation, applied to the
+ *     cache before INT2 quantization and removed after the attention
+ *     computation.  Section "Why It Matters": the inference (attention)
+ *     kernel itself is unchanged.
+ *   - "RotateKV: Accurate and Robust 2-Bit KV Cache Quantization ..."
+ *     abstract, item (i): the rotation is a channel reordering followed by a
+ *     fast Walsh-Hadamard transform; item (iii): attention sinks are
+ *     protected from 2-bit quantization.
+ *   - "KVLinC : KV Cache Quantization with Hadamard Rotation and Linear
+ *     Correction", abstract: a Hadamard rotation of the values.
+ * The pages fix the 2-bit width only.  The group of 32 along head_dim, the
+ * asymmetric min/max grid with an fp16 scale and fp16 zero per group, and the
+ * packed cache layout are this library's format; they are restated here as
+ * the format specification describes them.
+ *
+ * Precision: rotations and attention in fp64; the quantizer in exact IEEE
+ * fp32 with no contraction (build with -ffp-contract=off, no fast-math).
+ *
+ * Parity pins for every function are in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define D 128      /* head_dim */
+#define GS 32      /* quantization group size along head_dim */
+#define NG 4       /* groups per row */
+#define BLK_TOK 16 /* tokens per cache block */
+#define BLK_BYTES 1536
+
+/* status bits (same meaning as the library's device status word) */
+#define ST_CAPACITY 1
+#define ST_BAD_LEN 2
+
+/* ------------------------------------------------------------------------ */
+/* IEEE binary16 <-> binary32, written from the IEEE 754 encoding.            */
+/* ------------------------------------------------------------------------ */
+
+/* binary32 -> binary16, round to nearest, ties to even; overflow -> +-inf. */
+uint16_t orc_f32_to_f16(float f) {
+    uint32_t x;
+    memcpy(&x, &f, 4);
+    uint32_t sign = (x >> 16) & 0x8000u;
+    uint32_t ax = x & 0x7fffffffu;
+    if (ax >= 0x7f800000u) {                   /* inf / nan */
+        if (ax == 0x7f800000u) return (uint16_t)(sign | 0x7c00u);
+        return (uint16_t)(sign | 0x7e00u);     /* quiet nan */
+    }
+    if (ax >= 0x477ff000u) return (uint16_t)(sign | 0x7c00u); /* >= 65520 */
+    if (ax >= 0x38800000u) {                   /* half normal range */
+        uint32_t e = (ax >> 23) - 127u + 15u;
+        uint32_t m = ax & 0x7fffffu;
+        uint32_t hm = m >> 13, rem = m & 0x1fffu;
+        uint32_t h = (e << 10) | hm;
+        if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h += 1u;
+        return (uint16_t)(sign | h);
+    }
+    if (ax <= 0x33000000u) return (uint16_t)sign; /* <= 2^-25 -> 0 */
+    {                                          /* half subnormal */
+        uint32_t e = ax >> 23;                 /* 102..112 */
+        uint32_t m = (ax & 0x7fffffu) | 0x800000u;
+        uint32_t shift = 126u - e;             /* 14..24 */
+        uint32_t hm = m >> shift;
+        uint32_t rem = m & ((1u << shift) - 1u);
+        uint32_t half = 1u << (shift - 1u);
+        if (rem > half || (rem == half && (hm & 1u))) hm += 1u;
+        return (uint16_t)(sign | hm);
+    }
+}
+
+float orc_f16_to_f32(uint16_t h) {
+    uint32_t sign = ((uint32_t)h & 0x8000u) << 16;
+    uint32_t e = ((uint32_t)h >> 10) & 0x1fu;
+    uint32_t m = (uint32_t)h & 0x3ffu;
+    uint32_t x;
+    if (e == 0x1fu) {
+        x = sign | 0x7f800000u | (m << 13);
+    } else if (e != 0) {
+        x = sign | ((e - 15u + 127u) << 23) | (m << 13);
+    } else if (m == 0) {
+        x = sign;
+    } else {                                   /* subnormal: m * 2^-24 */
+        float v = (float)m * 5.9604644775390625e-08f;
+        memcpy(&x, &v, 4);
+        x |= sign;
+    }
+    float f;
+    memcpy(&f, &x, 4);
+    return f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rotations (fp64).                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* In-place unnormalised Walsh-Hadamard transform in Sylvester (natural)
+ * order: H[i][j] = (-1)^popcount(i & j).  Butterfly (a, b) -> (a+b, a-b)
+ * at strides 1, 2, 4, ... n/2.  RotateKV abstract, item (i) (FWHT). */
+void orc_fwht_f64(double *y, int n) {
+    for (int s = 1; s < n; s <<= 1)
+        for (int i = 0; i < n; i++)
+            if ((i & s) == 0) {
+                double a = y[i], b = y[i + s];
+                y[i] = a + b;
+                y[i + s] = a - b;
+            }
+}
+
+/* x_rot = x . R (row-vector convention, R row-major R[i][j]), or in FWHT
+ * mode x_rot = FWHT(y)/sqrt(128) with y[i] = x[perm[i]] (channel reordering
+ * then Hadamard; RotateKV item (i), KVLinC abstract).  fp64 throughout. */
+static void rotate_f64(const double *x, int mode, const float *R,
+                       const int32_t *perm, double *out) {
+    if (mode == 0) {
+        for (int j = 0; j < D; j++) {
+            double acc = 0.0;
+            for (int i = 0; i < D; i++) acc += x[i] * (double)R[i * D + j];
+            out[j] = acc;
+        }
+    } else {
+        for (int i = 0; i < D; i++) out[i] = x[perm[i]];
+        orc_fwht_f64(out, D);
+        double sc = 1.0 / sqrt((double)D);
+        for (int i = 0; i < D; i++) out[i] *= sc;
+    }
+}
+
+/* Inverse rotation, o . R^T (the rotation "removed after the attention
+ * computation", OptR page, "Key Details").  FWHT mode: y = FWHT(o)/sqrt(128),
+ * out[perm[i]] = y[i]. */
+static void unrotate_f64(const double *o, int mode, const float *R,
+                         const int32_t *perm, double *out) {
+    if (mode == 0) {
+        for (int i = 0; i < D; i++) {
+            double acc = 0.0;
+            for (int j = 0; j < D; j++) acc += o[j] * (double)R[i * D + j];
+            out[i] = acc;
+        }
+    } else {
+        double y[D];
+        for (int i = 0; i < D; i++) y[i] = o[i];
+        orc_fwht_f64(y, D);
+        double sc = 1.0 / sqrt((double)D);
+        for (int i = 0; i < D; i++) out[perm[i]] = y[i] * sc;
+    }
+}
+
+/* fp64 rotation of fp64 rows, exported for the invariance pins. */
+void orc_rotate_f64_rows(const double *x, int64_t n, int mode, const float *R,
+                         const int32_t *perm, double *out) {
+    for (int64_t r = 0; r < n; r++) rotate_f64(x + r * D, mode, R, perm, out + r * D);
+}
+
+void orc_unrotate_f64_rows(const double *o, int64_t n, int mode, const float *R,
+                           const int32_t *perm, double *out) {
+    for (int64_t r = 0; r < n; r++) unrotate_f64(o + r * D, mode, R, perm, out + r * D);
+}
+
+/* Rotate fp16 rows into "the rotated fp32 input" of the quantizer: fp64
+ * rotation of the exactly widened fp16 row, rounded once to fp32. */
+void orc_rotate_rows_f32(const uint16_t *x, int64_t n, int mode, const float *R,
+                         const int32_t *perm, float *out) {
+    double xin[D], xo[D];
+    for (int64_t r = 0; r < n; r++) {
+        for (int i = 0; i < D; i++) xin[i] = (double)orc_f16_to_f32(x[r * D + i]);
+        rotate_f64(xin, mode, R, perm, xo);
+        for (int i = 0; i < D; i++) out[r * D + i] = (float)xo[i];
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT2 quantizer (exact fp32).                                              */
+/* ------------------------------------------------------------------------ */
+
+/* One row of 128 rotated fp32 values -> 128 codes in {0,1,2,3} and, per group
+ * of 32 consecutive elements, an fp16 scale s and fp16 zero z:
+ *   mn, mx = min, max of the group
+ *   s = half(fp32((mx - mn) / 3)),  z = half(mn)       (a zero is stored +0)
+ *   inv = (s == 0) ? 0 : fp32(1 / float(s))
+ *   c = clamp(rint_even(fp32(fp32(x - float(z)) * inv)), 0, 3)
+ * Dequantised value: c * s + z.  Four levels = INT2 (OptR page, intro and
+ * "Key Details"; RotateKV abstract, "2-bit"). */
+void orc_quantize_row(const float *x, uint8_t *codes, uint16_t *s_out, uint16_t *z_out) {
+    for (int g = 0; g < NG; g++) {
+        const float *xg = x + g * GS;
+        float mn = xg[0], mx = xg[0];
+        for (int e = 1; e < GS; e++) {
+            if (xg[e] < mn) mn = xg[e];
+            if (xg[e] > mx) mx = xg[e];
+        }
+        float r = mx - mn;
+        float sf = r / 3.0f;
+        uint16_t s = orc_f32_to_f16(sf + 0.0f);
+        uint16_t z = orc_f32_to_f16(mn + 0.0f);
+        float sF = orc_f16_to_f32(s), zF = orc_f16_to_f32(z);
+        float inv = (sF == 0.0f) ? 0.0f : 1.0f / sF;
+        for (int e = 0; e < GS; e++) {
+            float d = xg[e] - zF;
+            float t = d * inv;
+            float rt = rintf(t);
+            int c = (rt < 0.0f) ? 0 : (rt > 3.0f ? 3 : (int)rt);
+            codes[g * GS + e] = (uint8_t)c;
+        }
+        s_out[g] = s;
+        z_out[g] = z;
+    }
+}
+
+void orc_quantize_rows(const float *x, int64_t n, uint8_t *codes, uint16_t *s, uint16_t *z) {
+    for (int64_t r = 0; r < n; r++)
+        orc_quantize_row(x + r * D, codes + r * D, s + r * NG, z + r * NG);
+}
+
+/* Logical packing, 4 codes per byte: the code of element j goes to byte
+ * (j mod 32), bits 2*(j div 32) .. 2*(j div 32)+1.  So byte e carries the
+ * element e of each of the 4 groups. */
+void orc_pack_row(const uint8_t *codes, uint8_t *bytes) {
+    for (int e = 0; e < 32; e++) {
+        uint8_t b = 0;
+        for (int g = 0; g < NG; g++) b |= (uint8_t)((codes[g * GS + e] & 3u) << (2 * g));
+        bytes[e] = b;
+    }
+}
+
+void orc_unpack_row(const uint8_t *bytes, uint8_t *codes) {
+    for (int j = 0; j < D; j++) codes[j] = (uint8_t)((bytes[j % 32] >> (2 * (j / 32))) & 3u);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Physical cache block (16 tokens, 1536 bytes), restated from the format     */
+/* specification.  tau = token index in the block, r = tau mod 8,             */
+/* th = tau div 8.                                                            */
+/*   K codes  [0,512):    logical 32-bit word wi (bytes 4wi..4wi+3) at        */
+/*                        16*(4r + wi%4) + 4*(2*th + wi/4)                    */
+/*   V codes  [512,1024): token pair p = tau/2, side = tau%2; logical 16-bit  */
+/*                        piece w (bytes 2w, 2w+1) at                         */
+/*                        512 + 16*(4*(w%8) + p%4) + 4*(2*(p/4) + w/8) + 2*side*/
+/*   K meta   [1024,1280): group g {s, z} (two fp16, s first) at              */
+/*                        1024 + 8*(4r + g) + 4*th                            */
+/*   V scale  [1280,1408): group g scale at                                   */
+/*                        1280 + 8*(4*(p%4) + g) + 4*(p/4) + 2*side           */
+/*   V zero   [1408,1536): same offset + 128                                  */
+/* ------------------------------------------------------------------------ */
+
+static size_t off_kword(int tau, int wi) {
+    int r = tau % 8, th = tau / 8;
+    return (size_t)(16 * (4 * r + wi % 4) + 4 * (2 * th + wi / 4));
+}
+static size_t off_vpiece(int tau, int w) {
+    int p = tau / 2, side = tau % 2;
+    return (size_t)(512 + 16 * (4 * (w % 8) + p % 4) + 4 * (2 * (p / 4) + w / 8) + 2 * side);
+}
+static size_t off_kmeta(int tau, int g) {
+    int r = tau % 8, th = tau / 8;
+    return (size_t)(1024 + 8 * (4 * r + g) + 4 * th);
+}
+static size_t off_vscale(int tau, int g) {
+    int p = tau / 2, side = tau % 2;
+    return (size_t)(1280 + 8 * (4 * (p % 4) + g) + 4 * (p / 4) + 2 * side);
+}
+
+static void put16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)(v & 0xff); p[1] = (uint8_t)(v >> 8); }
+static uint16_t get16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+
+/* Store one token's packed K and V rows and their metadata into a block. */
+void orc_store_token(uint8_t *block, int tau, const uint8_t *kbytes, const uint8_t *vbytes,
+                     const uint16_t *ks, const uint16_t *kz, const uint16_t *vs,
+                     const uint16_t *vz) {
+    for (int wi = 0; wi < 8; wi++) memcpy(block + off_kword(tau, wi), kbytes + 4 * wi, 4);
+    for (int w = 0; w < 16; w++) memcpy(block + off_vpiece(tau, w), vbytes + 2 * w, 2);
+    for (int g = 0; g < NG; g++) {
+        put16(block + off_kmeta(tau, g), ks[g]);
+        put16(block + off_kmeta(tau, g) + 2, kz[g]);
+        put16(block + off_vscale(tau, g), vs[g]);
+        put16(block + off_vscale(tau, g) + 128, vz[g]);
+    }
+}
+
+void orc_load_token(const uint8_t *block, int tau, uint8_t *kbytes, uint8_t *vbytes,
+                    uint16_t *ks, uint16_t *kz, uint16_t *vs, uint16_t *vz) {
+    for (int wi = 0; wi < 8; wi++) memcpy(kbytes + 4 * wi, block + off_kword(tau, wi), 4);
+    for (int w = 0; w < 16; w++) memcpy(vbytes + 2 * w, block + off_vpiece(tau, w), 2);
+    for (int g = 0; g < NG; g++) {
+        ks[g] = get16(block + off_kmeta(tau, g));
+        kz[g] = get16(block + off_kmeta(tau, g) + 2);
+        vs[g] = get16(block + off_vscale(tau, g));
+        vz[g] = get16(block + off_vscale(tau, g) + 128);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rotate -> quantize -> append.                                              */
+/* ------------------------------------------------------------------------ */
+
+/* K, V: fp16 [B][T][Hkv][128].  R_k, R_v: fp32 [Hkv][128][128] (dense mode).
+ * perm: int32 [2][Hkv][128] (FWHT mode; plane 0 keys, plane 1 values).
+ * blocks: [B][Hkv][capacity/16][1536].  k_sink, v_sink: fp16 [B][Hkv][S][128].
+ * seq_lens[b] (in: old length, out: old + T).  Position p = seq_lens[b] + t
+ * with p < S is an attention sink (RotateKV item (iii)): stored as the fp16
+ * rounding of its rotated fp32 row; its code and meta slots are zeroed.
+ * A sequence whose new length would exceed capacity is skipped whole and
+ * flags ST_CAPACITY.  Returns the status bits. */
+int orc_append(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int mode,
+               const float *R_k, const float *R_v, const int32_t *perm, int capacity, int S,
+               uint8_t *blocks, uint16_t *k_sink, uint16_t *v_sink, int32_t *seq_lens) {
+    int status = 0;
+    const int nblk = capacity / BLK_TOK;
+    for (int b = 0; b < B; b++) {
+        int L0 = seq_lens[b];
+        if (L0 < 0 || (int64_t)L0 + T > capacity) {
+            status |= (L0 < 0) ? ST_BAD_LEN : ST_CAPACITY;
+            continue;
+        }
+        for (int t = 0; t < T; t++) {
+            int p = L0 + t;
+            for (int h = 0; h < Hkv; h++) {
+                const size_t src = (((size_t)b * T + t) * Hkv + h) * D;
+                float kr[D], vr[D];
+                orc_rotate_rows_f32(K + src, 1, mode, mode == 0 ? R_k + (size_t)h * D * D : NULL,
+                                    mode == 1 ? perm + (size_t)h * D : NULL, kr);
+                orc_rotate_rows_f32(V + src, 1, mode, mode == 0 ? R_v + (size_t)h * D * D : NULL,
+                                    mode == 1 ? perm + ((size_t)Hkv + h) * D : NULL, vr);
+                uint8_t *block = blocks + (((size_t)b * Hkv + h) * nblk + p / BLK_TOK) * BLK_BYTES;
+                uint8_t kc[D], vc[D], kb[32], vb[32];
+                uint16_t ks[NG], kz[NG], vs[NG], vz[NG];
+                if (p < S) {
+                    uint16_t *ksr = k_sink + (((size_t)b * Hkv + h) * S + p) * D;
+                    uint16_t *vsr = v_sink + (((size_t)b * Hkv + h) * S + p) * D;
+                    for (int i = 0; i < D; i++) {
+                        ksr[i] = orc_f32_to_f16(kr[i]);
+                        vsr[i] = orc_f32_to_f16(vr[i]);
+                    }
+                    memset(kb, 0, 32);
+                    memset(vb, 0, 32);
+                    memset(ks, 0, sizeof ks);
+                    memset(kz, 0, sizeof kz);
+                    memset(vs, 0, sizeof vs);
+                    memset(vz, 0, sizeof vz);
+                } else {
+                    orc_quantize_row(kr, kc, ks, kz);
+                    orc_quantize_row(vr, vc, vs, vz);
+                    orc_pack_row(kc, kb);
+                    orc_pack_row(vc, vb);
+                }
+                orc_store_token(block, p % BLK_TOK, kb, vb, ks, kz, vs, vz);
+            }
+        }
+        seq_lens[b] = L0 + T;
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention over the packed cache (fp64).                            */
+/* ------------------------------------------------------------------------ */
+
+/* Dequantise token t of unit (b, h) into fp64 rotated K and V rows. */
+static void dequant_token(const uint8_t *unit_blocks, const uint16_t *ksink_u,
+                          const uint16_t *vsink_u, int S, int t, double *k, double *v) {
+    if (t < S) {
+        for (int i = 0; i < D; i++) {
+            k[i] = (double)orc_f16_to_f32(ksink_u[(size_t)t * D + i]);
+            v[i] = (double)orc_f16_to_f32(vsink_u[(size_t)t * D + i]);
+        }
+        return;
+    }
+    const uint8_t *block = unit_blocks + (size_t)(t / BLK_TOK) * BLK_BYTES;
+    uint8_t kb[32], vb[32], kc[D], vc[D];
+    uint16_t ks[NG], kz[NG], vs[NG], vz[NG];
+    orc_load_token(block, t % BLK_TOK, kb, vb, ks, kz, vs, vz);
+    orc_unpack_row(kb, kc);
+    orc_unpack_row(vb, vc);
+    for (int j = 0; j < D; j++) {
+        int g = j / GS;
+        k[j] = (double)kc[j] * (double)orc_f16_to_f32(ks[g]) + (double)orc_f16_to_f32(kz[g]);
+        v[j] = (double)vc[j] * (double)orc_f16_to_f32(vs[g]) + (double)orc_f16_to_f32(vz[g]);
+    }
+}
+
+/* One (b, query head): q_rot = q . R_k, scores s_t = q_rot . k_t / sqrt(128)
+ * over t in [0, L), softmax, o_rot = sum p_t v_t, out = o_rot . R_v^T.
+ * Query head h uses KV head h / G (contiguous GQA grouping). */
+static void decode_one(const uint16_t *q, int mode, const float *Rk, const float *Rv,
+                       const int32_t *pk, const int32_t *pv, const uint8_t *unit_blocks,
+                       const uint16_t *ksink_u, const uint16_t *vsink_u, int S, int L,
+                       double *out) {
+    double qin[D], qr[D], k[D], v[D], o[D];
+    for (int i = 0; i < D; i++) qin[i] = (double)orc_f16_to_f32(q[i]);
+    rotate_f64(qin, mode, Rk, pk, qr);
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    const double scale = 1.0 / sqrt((double)D);
+    double m = -INFINITY;
+    for (int t = 0; t < L; t++) {
+        dequant_token(unit_blocks, ksink_u, vsink_u, S, t, k, v);
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += qr[i] * k[i];
+        s[t] = acc * scale;
+        if (s[t] > m) m = s[t];
+    }
+    double l = 0.0;
+    for (int i = 0; i < D; i++) o[i] = 0.0;
+    for (int t = 0; t < L; t++) {
+        double p = exp(s[t] - m);
+        l += p;
+        dequant_token(unit_blocks, ksink_u, vsink_u, S, t, k, v);
+        for (int i = 0; i < D; i++) o[i] += p * v[i];
+    }
+    for (int i = 0; i < D; i++) o[i] /= l;
+    unrotate_f64(o, mode, Rv, pv, out);
+    free(s);
+}
+
+/* Q: fp16 [B][Hq][128].  out: fp64 [B][Hq][128].  Units with an invalid
+ * length (L < 1 or L > capacity) get out = 0 and flag ST_BAD_LEN.
+ * only_b / only_h >= 0 restrict the work to one sequence / KV head (used to
+ * sample large workloads); other outputs are left untouched.
+ * n_threads > 1 runs (b, query head) pairs on that many OpenMP threads. */
+int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
+               const float *R_v, const int32_t *perm, int capacity, int S,
+               const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
+               const int32_t *seq_lens, int only_b, int only_h, int n_threads, double *out) {
+    int status = 0;
+    const int G = Hq / Hkv;
+    const int nblk = capacity / BLK_TOK;
+    for (int b = 0; b < B; b++) {
+        int L = seq_lens[b];
+        if ((only_b < 0 || b == only_b) && (L < 1 || L > capacity)) status |= ST_BAD_LEN;
+    }
+    const int64_t npairs = (int64_t)B * Hq;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int64_t bh = 0; bh < npairs; bh++) {
+        int b = (int)(bh / Hq), hq = (int)(bh % Hq), h = hq / G;
+        if (only_b >= 0 && b != only_b) continue;
+        if (only_h >= 0 && h != only_h) continue;
+        double *o = out + (size_t)bh * D;
+        int L = seq_lens[b];
+        if (L < 1 || L > capacity) {
+            for (int i = 0; i < D; i++) o[i] = 0.0;
+            continue;
+        }
+        const size_t u = (size_t)b * Hkv + h;
+        decode_one(Q + (size_t)bh * D, mode, mode == 0 ? R_k + (size_t)h * D * D : NULL,
+                   mode == 0 ? R_v + (size_t)h * D * D : NULL,
+                   mode == 1 ? perm + (size_t)h * D : NULL,
+                   mode == 1 ? perm + ((size_t)Hkv + h) * D : NULL,
+                   blocks + u * (size_t)nblk * BLK_BYTES,
+                   S > 0 ? k_sink + u * (size_t)S * D : NULL,
+                   S > 0 ? v_sink + u * (size_t)S * D : NULL, S, L, o);
+    }
+    return status;
+}
+
+/* Attention over explicit fp64 rows (no cache, no quantization), used by the
+ * rotation-invariance pin: out = softmax(q . K^T / sqrt(128)) V. */
+void orc_attention_f64(const double *q, const double *K, const double *V, int L, double *out) {
+    const double scale = 1.0 / sqrt((double)D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    double m = -INFINITY, l = 0.0;
+    for (int t = 0; t < L; t++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += q[i] * K[(size_t)t * D + i];
+        s[t] = acc * scale;
+        if (s[t] > m) m = s[t];
+    }
+    for (int i = 0; i < D; i++) out[i] = 0.0;
+    for (int t = 0; t < L; t++) {
+        double p = exp(s[t] - m);
+        l += p;
+        for (int i = 0; i < D; i++) out[i] += p * V[(size_t)t * D + i];
+    }
+    for (int i = 0; i < D; i++) out[i] /= l;
+    free(s);
+}
+
+/* Array forms of the binary16 conversions (one call per array). */
+void orc_f32_to_f16_array(const float *x, int64_t n, uint16_t *out) {
+    for (int64_t i = 0; i < n; i++) out[i] = orc_f32_to_f16(x[i]);
+}
+
+void orc_f16_to_f32_array(const uint16_t *x, int64_t n, float *out) {
+    for (int64_t i = 0; i < n; i++) out[i] = orc_f16_to_f32(x[i]);
+}

@@ -1,0 +1,436 @@
+"""Pins of the CPU oracle against facts fixed outside it: IEEE binary16,
+closed forms, library routines (scipy Hadamard, scipy softmax), invariants of
+orthogonal rotations, hand-derived worked values (tests/golden) and a second,
+independently written numpy oracle.  CPU only."""
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+
+from oracle import np_mini
+from oracle import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quantizer_worked.json")
+D = 128
+
+
+def rand_orth(rng):
+    q, r = np.linalg.qr(rng.standard_normal((D, D)))
+    return (q * np.sign(np.diag(r))[None, :]).astype(np.float32)
+
+
+# --- binary16 ----------------------------------------------------------------------------
+
+def test_f16_to_f32_exhaustive():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = orc.f16_bits_to_f32(bits)
+    ref = bits.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_f32_to_f16_matches_numpy():
+    rng = np.random.default_rng(0)
+    parts = [
+        rng.standard_normal(200000).astype(np.float32) * 10,
+        (rng.standard_normal(100000) * 1e-5).astype(np.float32),      # subnormal halves
+        (rng.standard_normal(50000) * 1e-7).astype(np.float32),       # underflow region
+        rng.uniform(6e4, 7e4, 20000).astype(np.float32),               # overflow edge
+        np.array([65504, 65519.99, 65520, -65520, 2**-25, 2**-24, 3 * 2**-26, 0.0, -0.0,
+                  np.inf, -np.inf], np.float32),
+    ]
+    # exact midpoints between consecutive halves (ties), normal and subnormal
+    h = np.arange(0, 0x7bff, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float64)
+    hi = (h + 1).view(np.float16).astype(np.float64)
+    parts.append(((lo + hi) / 2).astype(np.float32))
+    parts.append(-((lo + hi) / 2).astype(np.float32))
+    x = np.concatenate(parts)
+    got = orc.f32_to_f16_bits(x)
+    ref = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# --- FWHT and rotations -------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64, 128])
+def test_fwht_equals_sylvester_matrix(n):
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((5, n))
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    for r in range(5):
+        assert np.allclose(orc.fwht_f64(x[r]), H @ x[r], rtol=0, atol=1e-12)
+
+
+def test_fwht_orthogonality_and_involution():
+    I = np.eye(D)
+    H = np.stack([orc.fwht_f64(I[i]) for i in range(D)])
+    assert np.array_equal(H @ H.T, D * np.eye(D))
+    x = np.random.default_rng(1).standard_normal(D)
+    assert np.allclose(orc.fwht_f64(orc.fwht_f64(x)) / D, x, atol=1e-13)
+
+
+def test_dense_rotation_is_row_vector_convention():
+    """x_rot = x . R: the basis vector e_i must rotate to row i of R."""
+    R = rand_orth(np.random.default_rng(2))
+    out = orc.rotate_f64(np.eye(D), 0, R=R)
+    assert np.array_equal(out, R.astype(np.float64))
+    back = orc.unrotate_f64(np.eye(D), 0, R=R)          # e_j . R^T = column j of R
+    assert np.array_equal(back, R.astype(np.float64).T)
+
+
+def test_perm_fwht_equals_explicit_matrix():
+    """FWHT mode equals the dense rotation R[perm[i], :] = H[i, :]/sqrt(128),
+    which is orthogonal; its inverse undoes it."""
+    rng = np.random.default_rng(3)
+    perm = rng.permutation(D).astype(np.int32)
+    H = scipy.linalg.hadamard(D) / np.sqrt(D)
+    R = np.zeros((D, D))
+    R[perm, :] = H
+    assert np.allclose(R @ R.T, np.eye(D), atol=1e-14)
+    x = rng.standard_normal((7, D))
+    got = orc.rotate_f64(x, 1, perm=perm)
+    assert np.allclose(got, x @ R, atol=1e-12)
+    assert np.allclose(orc.unrotate_f64(got, 1, perm=perm), x, atol=1e-12)
+    dense = orc.rotate_f64(x, 0, R=R.astype(np.float32))
+    assert np.allclose(dense, got, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_rotation_invariance_of_attention(mode):
+    """Attention over (qR, KR, VR) followed by R_v^T equals attention over
+    (q, K, V) in fp64: the rotation applied before quantization and removed
+    after attention changes nothing but the quantization error."""
+    rng = np.random.default_rng(4 + mode)
+    L = 37
+    q = rng.standard_normal(D)
+    K = rng.standard_normal((L, D)) * 2
+    V = rng.standard_normal((L, D))
+    if mode == 0:
+        kw = dict(R=rand_orth(rng))
+        vw = dict(R=rand_orth(rng))
+    else:
+        kw = dict(perm=rng.permutation(D).astype(np.int32))
+        vw = dict(perm=rng.permutation(D).astype(np.int32))
+    ref = orc.attention_f64(q, K, V)
+    rot = orc.attention_f64(orc.rotate_f64(q, mode, **kw)[0], orc.rotate_f64(K, mode, **kw),
+                            orc.rotate_f64(V, mode, **vw))
+    back = orc.unrotate_f64(rot, mode, **vw)[0]
+    assert np.max(np.abs(back - ref)) <= 1e-5 * np.linalg.norm(ref)
+    # a dense fp32 R is orthogonal only to fp32 precision; FWHT is exact
+    assert np.max(np.abs(back - ref)) <= (1e-6 if mode == 0 else 1e-12)
+
+
+def test_attention_f64_against_scipy_softmax():
+    rng = np.random.default_rng(5)
+    L = 9
+    q, K, V = rng.standard_normal(D), rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    p = scipy.special.softmax(K @ q / np.sqrt(D))
+    assert np.allclose(orc.attention_f64(q, K, V), p @ V, atol=1e-13)
+
+
+# --- quantizer ----------------------------------------------------------------------------
+
+def golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def test_quantizer_worked_groups():
+    for case in golden()["groups"]:
+        row = np.zeros(D, np.float32)
+        for g in range(4):            # same group in all 4 slots
+            row[g * 32:(g + 1) * 32] = np.array(case["x"], np.float32)
+        codes, s, z = orc.quantize_rows(row)
+        for g in range(4):
+            assert list(codes[0, g * 32:(g + 1) * 32]) == case["codes"], case["name"]
+            assert s[0, g] == case["s_bits"] and z[0, g] == case["z_bits"], case["name"]
+
+
+def test_quantizer_grid_round_trip():
+    """x = z + c*s with z an fp16 value, s a power of two and c covering all
+    four levels: codes recover c exactly and dequantisation returns x."""
+    rng = np.random.default_rng(6)
+    for _ in range(200):
+        row = np.zeros(D, np.float32)
+        want = np.zeros(D, np.uint8)
+        zs, ss = [], []
+        for g in range(4):
+            s = np.float32(2.0 ** rng.integers(-8, 4))
+            z = np.float32(np.float16(rng.uniform(-4, 4)))
+            c = rng.integers(0, 4, 32)
+            c[:4] = [0, 1, 2, 3]
+            rng.shuffle(c)
+            row[g * 32:(g + 1) * 32] = z + c.astype(np.float32) * s
+            want[g * 32:(g + 1) * 32] = c
+            zs.append(z)
+            ss.append(s)
+        codes, s_bits, z_bits = orc.quantize_rows(row)
+        assert np.array_equal(codes[0], want)
+        assert np.array_equal(orc.f16_bits_to_f32(s_bits[0]), np.array(ss, np.float32))
+        assert np.array_equal(orc.f16_bits_to_f32(z_bits[0]), np.array(zs, np.float32))
+        deq = np_mini.dequant(codes[0], s_bits[0], z_bits[0])
+        assert np.array_equal(deq, row.astype(np.float64))
+
+
+def test_quantizer_error_bound():
+    """Every element that is not clamped lies within half a step of its
+    dequantised value; clamped ones only spill by the fp16 rounding of z/s."""
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((500, D)) * rng.uniform(0.1, 30, (500, 1))).astype(np.float32)
+    codes, s_bits, z_bits = orc.quantize_rows(x)
+    s = orc.f16_bits_to_f32(s_bits).astype(np.float64)
+    z = orc.f16_bits_to_f32(z_bits).astype(np.float64)
+    g = np.arange(D) // 32
+    xhat = codes * s[:, g] + z[:, g]
+    err = np.abs(x - xhat)
+    t = (x - z[:, g]) / s[:, g]
+    inner = (t >= -0.5) & (t <= 3.5)
+    assert np.all(err[inner] <= 0.5 * s[:, g][inner] * (1 + 2e-6) + 1e-30)
+    # outside the grid only by the rounding of z and s (far below one step)
+    assert np.all(np.abs(t[~inner] - np.clip(t[~inner], -0.5, 3.5)) < 0.01)
+    # every level is used and the extremes land on 0 and 3
+    assert set(np.unique(codes)) == {0, 1, 2, 3}
+
+
+def test_quantizer_matches_numpy_mini_oracle():
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((300, D)) * rng.uniform(0.01, 50, (300, 1))).astype(np.float32)
+    x[0, :32] = 1.5                       # constant group
+    x[1, :32] = np.linspace(0, 3, 32)     # exact grid with ties
+    a = orc.quantize_rows(x)
+    b = np_mini.quantize_rows(x)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+# --- packing and the cache block format -------------------------------------------------------
+
+def test_pack_worked_bytes():
+    for case in golden()["pack"]:
+        codes = np.zeros(D, np.uint8)
+        for g, c in enumerate(case["codes_g0_g1_g2_g3"]):
+            codes[g * 32 + 5] = c                      # element 5 of each group
+        b = orc.pack_row(codes)
+        assert b[5] == case["byte"] and b.sum() == case["byte"]
+
+
+def test_pack_unpack_round_trip():
+    rng = np.random.default_rng(9)
+    for _ in range(50):
+        c = rng.integers(0, 4, D).astype(np.uint8)
+        assert np.array_equal(orc.unpack_row(orc.pack_row(c)), c)
+
+
+def test_block_layout_is_a_bijection():
+    """The 16 tokens' fields tile the 1536-byte block exactly once."""
+    owner = np.full(orc.BLK_BYTES, -1)
+    for tau in range(16):
+        block = np.zeros(orc.BLK_BYTES, np.uint8)
+        ff = np.full(32, 0xFF, np.uint8)
+        f16 = np.full(4, 0xFFFF, np.uint16)
+        orc.store_token(block, tau, ff, ff, f16, f16, f16, f16)
+        hit = np.nonzero(block)[0]
+        assert len(hit) == 96                        # 32 + 32 + 16 + 16 bytes per token
+        assert np.all(owner[hit] == -1)
+        owner[hit] = tau
+    assert np.all(owner >= 0)
+
+
+def test_block_layout_worked_offsets():
+    lay = golden()["layout"]
+    for c in lay["k_word"]:
+        block = np.zeros(orc.BLK_BYTES, np.uint8)
+        kb = np.zeros(32, np.uint8)
+        kb[4 * c["wi"]:4 * c["wi"] + 4] = [1, 2, 3, 4]
+        z32, z4 = np.zeros(32, np.uint8), np.zeros(4, np.uint16)
+        orc.store_token(block, c["tau"], kb, z32, z4, z4, z4, z4)
+        assert list(block[c["offset"]:c["offset"] + 4]) == [1, 2, 3, 4]
+    for c in lay["v_piece"]:
+        block = np.zeros(orc.BLK_BYTES, np.uint8)
+        vb = np.zeros(32, np.uint8)
+        vb[2 * c["w"]:2 * c["w"] + 2] = [7, 9]
+        z32, z4 = np.zeros(32, np.uint8), np.zeros(4, np.uint16)
+        orc.store_token(block, c["tau"], z32, vb, z4, z4, z4, z4)
+        assert list(block[c["offset"]:c["offset"] + 2]) == [7, 9]
+    for c in lay["k_meta"]:
+        block = np.zeros(orc.BLK_BYTES, np.uint8)
+        ks, kz = np.zeros(4, np.uint16), np.zeros(4, np.uint16)
+        ks[c["g"]], kz[c["g"]] = 0x1234, 0x5678
+        z32, z4 = np.zeros(32, np.uint8), np.zeros(4, np.uint16)
+        orc.store_token(block, c["tau"], z32, z32, ks, kz, z4, z4)
+        assert list(block[c["offset"]:c["offset"] + 4]) == [0x34, 0x12, 0x78, 0x56]
+    for c in lay["v_scale"]:
+        block = np.zeros(orc.BLK_BYTES, np.uint8)
+        vs, vz = np.zeros(4, np.uint16), np.zeros(4, np.uint16)
+        vs[c["g"]], vz[c["g"]] = 0x1111, 0x2222
+        z32, z4 = np.zeros(32, np.uint8), np.zeros(4, np.uint16)
+        orc.store_token(block, c["tau"], z32, z32, z4, z4, vs, vz)
+        assert list(block[c["offset"]:c["offset"] + 2]) == [0x11, 0x11]
+        assert list(block[c["offset"] + 128:c["offset"] + 130]) == [0x22, 0x22]
+
+
+# --- append / decode ----------------------------------------------------------------------------
+
+def f16(x):
+    return np.asarray(x, np.float16).view(np.uint16)
+
+
+def grid_rows(rng, n):
+    """fp16 rows whose every group of 32 is an exact 4-level grid z + c*s."""
+    rows = np.zeros((n, D), np.float32)
+    for r in range(n):
+        for g in range(4):
+            s = np.float32(2.0 ** rng.integers(-3, 1))
+            z = np.float32(rng.integers(-16, 16) / 8.0)     # multiples of 1/8: fp16-exact
+            c = rng.integers(0, 4, 32)
+            c[:4] = [0, 1, 2, 3]
+            rng.shuffle(c)
+            rows[r, g * 32:(g + 1) * 32] = z + c * s
+    assert np.array_equal(rows.astype(np.float16).astype(np.float32), rows)
+    return rows
+
+
+def test_decode_exact_on_grid_values_with_identity_rotation():
+    """With R = I and K/V on exact 4-level grids, quantization is lossless and
+    the decode equals exact fp64 attention (scipy softmax)."""
+    rng = np.random.default_rng(10)
+    L, Hkv = 37, 2
+    K = grid_rows(rng, L * Hkv).reshape(1, L, Hkv, D)
+    V = grid_rows(rng, L * Hkv).reshape(1, L, Hkv, D)
+    I = np.stack([np.eye(D, dtype=np.float32)] * Hkv)
+    cache = orc.Cache(1, Hkv, 48, 0)
+    sl = np.zeros(1, np.int32)
+    assert orc.append(cache, f16(K), f16(V), 0, I, I, None, sl) == 0
+    assert sl[0] == L
+    Q = rng.standard_normal((1, 2 * Hkv, D)).astype(np.float16)
+    out, st = orc.decode(cache, Q.view(np.uint16), 0, I, I, None, sl)
+    assert st == 0
+    for hq in range(2 * Hkv):
+        h = hq // 2
+        q = Q[0, hq].astype(np.float64)
+        Kh, Vh = K[0, :, h].astype(np.float64), V[0, :, h].astype(np.float64)
+        p = scipy.special.softmax(Kh @ q / np.sqrt(D))
+        assert np.allclose(out[0, hq], p @ Vh, rtol=0, atol=1e-12)
+
+
+def test_decode_zero_query_is_mean_of_values():
+    """q = 0 gives equal scores: the output is the mean of the dequantised V
+    rows (decoded here by the numpy mini-oracle), rotated back."""
+    rng = np.random.default_rng(11)
+    L = 21
+    R = np.stack([rand_orth(rng)])
+    K = rng.standard_normal((1, L, 1, D)).astype(np.float16)
+    V = rng.standard_normal((1, L, 1, D)).astype(np.float16)
+    cache = orc.Cache(1, 1, 32, 0)
+    sl = np.zeros(1, np.int32)
+    orc.append(cache, K.view(np.uint16), V.view(np.uint16), 0, R, R, None, sl)
+    out, _ = orc.decode(cache, np.zeros((1, 1, D), np.uint16), 0, R, R, None, sl)
+    vrows = []
+    for t in range(L):
+        _, vb, _, _, vs, vz = orc.load_token(cache.blocks[0, 0, t // 16], t % 16)
+        vrows.append(np_mini.dequant(orc.unpack_row(vb), vs, vz))
+    ref = np.mean(vrows, axis=0) @ R[0].astype(np.float64).T
+    assert np.allclose(out[0, 0], ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode,S,G", [(0, 0, 1), (0, 4, 4), (1, 0, 2), (1, 3, 1)])
+def test_c_oracle_matches_numpy_mini_oracle(mode, S, G):
+    """Two independent oracles: bit-exact codes and metadata from the same
+    rotated fp32 rows, <= 1e-12 on the decoded output."""
+    rng = np.random.default_rng(12 + mode + S)
+    B, T, Hkv = 2, 41, 2
+    Hq = Hkv * G
+    K = (rng.standard_normal((B, T, Hkv, D)) * 3).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    if mode == 0:
+        Rk = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        Rv = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        perm = None
+        kw = lambda h, kind: dict(R=(Rk if kind == 0 else Rv)[h])
+    else:
+        Rk = Rv = None
+        perm = np.stack([np.stack([rng.permutation(D) for _ in range(Hkv)])
+                         for _ in range(2)]).astype(np.int32)
+        kw = lambda h, kind: dict(perm=perm[kind, h])
+    cache = orc.Cache(B, Hkv, 48, S)
+    sl = np.array([0, 5], np.int32)
+    assert orc.append(cache, K.view(np.uint16), V.view(np.uint16), mode, Rk, Rv, perm, sl) == 0
+    Q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    out, st = orc.decode(cache, Q.view(np.uint16), mode, Rk, Rv, perm, sl)
+    assert st == 0
+    for b in range(B):
+        L0 = [0, 5][b]
+        for h in range(Hkv):
+            khat, vhat = [], []
+            for kind, X in ((0, K), (1, V)):
+                xr_c = orc.rotate_rows_f32(X[b, :, h].view(np.uint16), mode, **kw(h, kind))
+                xr_n = np_mini.rotate_rows_f32(X[b, :, h], mode, **kw(h, kind))
+                assert np.max(np.abs(xr_c - xr_n) / (np.abs(xr_n) + 1e-3)) < 1e-6
+                codes, s, z = np_mini.quantize_rows(xr_c)
+                rows = []
+                for t in range(L0 + T):
+                    p = t
+                    if p < L0:                      # never written: zero block -> value 0
+                        rows.append(np.zeros(D))
+                        continue
+                    if p < S:
+                        rows.append(xr_c[p - L0].astype(np.float16).astype(np.float64))
+                        continue
+                    blk = cache.blocks[b, h, p // 16]
+                    kb, vb, ks, kz, vs, vz = orc.load_token(blk, p % 16)
+                    bb, ss, zz = (kb, ks, kz) if kind == 0 else (vb, vs, vz)
+                    assert np.array_equal(orc.unpack_row(bb), codes[p - L0])
+                    assert np.array_equal(ss, s[p - L0]) and np.array_equal(zz, z[p - L0])
+                    rows.append(np_mini.dequant(codes[p - L0], s[p - L0], z[p - L0]))
+                (khat if kind == 0 else vhat).append(np.array(rows))
+            for hq in range(h * G, (h + 1) * G):
+                ref = np_mini.decode_one(Q[b, hq], khat[0], vhat[0], mode,
+                                         Rk[h] if mode == 0 else None,
+                                         Rv[h] if mode == 0 else None,
+                                         perm[0, h] if mode == 1 else None,
+                                         perm[1, h] if mode == 1 else None)
+                assert np.allclose(out[b, hq], ref, rtol=0, atol=1e-12)
+
+
+def test_sinks_are_rotated_fp16_rows_and_leave_slots_zero():
+    rng = np.random.default_rng(13)
+    S, T = 4, 6
+    R = np.stack([rand_orth(rng)])
+    K = rng.standard_normal((1, T, 1, D)).astype(np.float16)
+    V = rng.standard_normal((1, T, 1, D)).astype(np.float16)
+    cache = orc.Cache(1, 1, 16, S)
+    cache.blocks[:] = 0xAB
+    sl = np.zeros(1, np.int32)
+    orc.append(cache, K.view(np.uint16), V.view(np.uint16), 0, R, R, None, sl)
+    kr = np_mini.rotate_rows_f32(K[0, :, 0], 0, R=R[0])
+    assert np.array_equal(cache.k_sink[0, 0], kr[:S].astype(np.float16).view(np.uint16))
+    for tau in range(S):
+        fields = orc.load_token(cache.blocks[0, 0, 0], tau)
+        assert all(not np.any(f) for f in fields)
+    kb = orc.load_token(cache.blocks[0, 0, 0], S)[0]
+    assert np.array_equal(orc.unpack_row(kb), np_mini.quantize_rows(kr[S:S + 1])[0][0])
+
+
+def test_capacity_overflow_skips_sequence():
+    rng = np.random.default_rng(14)
+    cache = orc.Cache(2, 1, 16, 0)
+    K = rng.standard_normal((2, 5, 1, D)).astype(np.float16)
+    R = np.stack([np.eye(D, dtype=np.float32)])
+    sl = np.array([12, 3], np.int32)
+    st = orc.append(cache, K.view(np.uint16), K.view(np.uint16), 0, R, R, None, sl)
+    assert st == orc.ST_CAPACITY
+    assert list(sl) == [12, 8]
+    assert not cache.blocks[0].any() and cache.blocks[1].any()
+
+
+def test_decode_bad_length_gives_zero_and_status():
+    cache = orc.Cache(2, 1, 16, 0)
+    R = np.stack([np.eye(D, dtype=np.float32)])
+    Q = np.ones((2, 1, D), np.float16).view(np.uint16)
+    out, st = orc.decode(cache, Q, 0, R, R, None, np.array([0, 17], np.int32))
+    assert st == orc.ST_BAD_LEN and not out.any()
