@@ -1,0 +1,189 @@
+/*
+ * kvq.h -- C ABI of libkvq, a B200 (sm_100a) library for rotated INT2
+ * KV caches: rotate -> quantize -> append, and decode attention over the
+ * packed cache.
+ *
+ * The method (pages on the subject):
+ *   "Output-Aware Rotation for INT2 KV-Cache Quantization" (OptR), section
+ *   "Key Details": every head owns an orthogonal rotation that is applied to
+ *   the cache before INT2 quantization and removed after the attention
+ *   computation; section "Why It Matters": the attention kernel itself is
+ *   unchanged.  "RotateKV: Accurate and Robust 2-Bit KV Cache Quantization for
+ *   LLMs via Outlier-Aware Adaptive Rotations", abstract: (i) channel
+ *   reordering followed by a fast Walsh-Hadamard transform, (iii) attention
+ *   sinks protected from 2-bit quantization.  "KVLinC : KV Cache Quantization
+ *   with Hadamard Rotation and Linear Correction", abstract: Hadamard rotation
+ *   of the values.  The rotation itself is learned or chosen offline and is an
+ *   input here.
+ *
+ * Conventions
+ *   - head_dim is 128; quantization groups are 32 consecutive elements of
+ *     head_dim (4 per row); each group stores an fp16 scale s and fp16 zero z.
+ *   - fp16 values cross the ABI as uint16_t bit patterns (IEEE binary16).
+ *   - Row-vector convention: x_rot = x . R with R row-major, R[i][j] at
+ *     R + i*128 + j.  FWHT mode: y[i] = x[perm[i]], x_rot = FWHT(y)/sqrt(128),
+ *     FWHT in Sylvester order, H[i][j] = (-1)^popcount(i & j).
+ *   - Every pointer argument except the descriptor itself and kvq_get_status's
+ *     host_out is DEVICE memory owned by the caller.  The library never
+ *     allocates or frees memory and keeps no state between calls (it caches
+ *     per-device attributes only).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Compute
+ *     calls are asynchronous on it; argument errors are reported before any
+ *     launch and nothing is launched then.
+ *   - Device-detected errors never trap: they OR a bit into *cache->status
+ *     (see KVQ_DEV_*) and the affected work is skipped.
+ *
+ * Quantizer (exact IEEE fp32, no contraction), per group of 32 values x:
+ *   mn = min x, mx = max x
+ *   s  = fp16_rn((mx - mn) / 3)          z = fp16_rn(mn)    (zeros stored +0)
+ *   inv = (s == 0) ? 0 : fp32(1 / s)
+ *   c  = clamp(rint_even(fp32(fp32(x - z) * inv)), 0, 3)
+ *   dequantised value: c * s + z
+ * Logical packing: the code of element j is byte (j % 32), bits 2*(j/32).
+ *
+ * Cache layout.  One cache holds B sequences x Hkv KV heads; each (b, h)
+ * "unit" owns capacity/16 blocks of 16 tokens, 1536 bytes each:
+ *   blocks + ((b*Hkv + h) * (capacity/16) + p/16) * 1536   for position p.
+ * Inside a block, with tau = p % 16, r = tau % 8, th = tau / 8,
+ * pair q = tau / 2, side = tau % 2 (all offsets in bytes):
+ *   K codes  [0,512)     logical 32-bit word wi (bytes 4wi..4wi+3 of the
+ *                        token's 32 code bytes) at 16*(4r + wi%4) + 4*(2th + wi/4)
+ *   V codes  [512,1024)  logical 16-bit piece w (bytes 2w, 2w+1) at
+ *                        512 + 16*(4*(w%8) + q%4) + 4*(2*(q/4) + w/8) + 2*side
+ *   K meta   [1024,1280) group g: fp16 s then fp16 z at 1024 + 8*(4r + g) + 4*th
+ *   V scales [1280,1408) group g: fp16 s at 1280 + 8*(4*(q%4) + g) + 4*(q/4) + 2*side
+ *   V zeros  [1408,1536) same offset + 128
+ * This order is the operand order of the decode kernel's tensor-core
+ * fragments, so one warp reads each 512-byte region as 32 x 16 contiguous
+ * bytes.  The 96 bytes per token-head (3 bits per element) are the whole
+ * cache read of a decode step.
+ * Sinks: positions p < sink_fp16 are kept as fp16 rotated rows in
+ *   k_sink / v_sink [B][Hkv][sink_fp16][128]; their block slots are zeroed.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, mode/pointer mismatch */
+    KVQ_ERR_UNSUPPORTED = 2,  /* head_dim != 128, group != 32, misalignment   */
+    KVQ_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed          */
+    KVQ_ERR_CAPACITY = 4,     /* reserved: capacity errors are device-side     */
+    KVQ_ERR_WORKSPACE = 5     /* decode workspace too small                    */
+} kvq_status;
+
+typedef enum {
+    KVQ_ROT_DENSE = 0,        /* per-head dense 128x128 orthogonal R (OptR)     */
+    KVQ_ROT_PERM_FWHT = 1     /* per-head channel permutation + FWHT (RotateKV) */
+} kvq_rot_mode;
+
+/* Bits ORed into *status by device code. */
+#define KVQ_DEV_CAPACITY 1    /* append would exceed capacity: sequence skipped */
+#define KVQ_DEV_BAD_LEN 2     /* seq_lens[b] < 0 (append) or not in [1, capacity]
+                                 (decode): skipped, decode output row is 0      */
+#define KVQ_DEV_TIMEOUT 4     /* a bounded pipeline wait gave up: output invalid */
+
+typedef struct {
+    int32_t B;                /* sequences                                      */
+    int32_t Hkv;              /* KV heads                                       */
+    int32_t head_dim;         /* must be 128                                    */
+    int32_t group;            /* must be 32                                     */
+    int32_t capacity;         /* tokens per sequence, multiple of 16            */
+    int32_t sink_fp16;        /* leading positions kept in fp16 (0..64)         */
+    void *blocks;             /* [B][Hkv][capacity/16][1536] bytes, 16-B aligned */
+    uint16_t *k_sink;         /* [B][Hkv][sink_fp16][128] fp16, or NULL if 0     */
+    uint16_t *v_sink;         /* same                                           */
+    int32_t *status;          /* one device word, sticky error bits (KVQ_DEV_*) */
+} kvq_cache_desc;
+
+/* Bytes of the blocks array for a cache of this shape (0 on bad arguments). */
+KVQ_API size_t kvq_cache_bytes(int32_t B, int32_t Hkv, int32_t capacity);
+
+/*
+ * Rotate, quantize and append T tokens to every sequence.
+ *   K, V      fp16 [B][T][Hkv][128] (post-RoPE keys, values), 16-B aligned.
+ *   mode      KVQ_ROT_DENSE: R_k, R_v fp32 [Hkv][128][128] required, perm ignored.
+ *             KVQ_ROT_PERM_FWHT: perm int32 [2][Hkv][128] required (plane 0
+ *             keys, plane 1 values; each row a permutation of 0..127),
+ *             R_k / R_v ignored.
+ *   seq_lens  int32 [B]: in = current length, out = length + T.  Positions
+ *             seq_lens[b] .. seq_lens[b]+T-1 are written.  If that exceeds
+ *             capacity (or seq_lens[b] < 0) the sequence is left untouched
+ *             and a KVQ_DEV_* bit is set.
+ * Rotation: OptR page "Key Details"; RotateKV abstract item (i); KVLinC
+ * abstract.  Sinks: RotateKV abstract item (iii).
+ */
+KVQ_API kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int32_t T,
+                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                      const int32_t *perm, const kvq_cache_desc *cache,
+                                      int32_t *seq_lens, void *stream);
+
+/* Workspace bytes needed by kvq_decode_attention for these sizes on a GPU
+ * with sm_count SMs (0 on bad arguments). */
+KVQ_API size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max_ctx,
+                                 int32_t sm_count);
+
+/*
+ * Decode attention of one query per query head over the packed cache.
+ *   Q         fp16 [B][Hq][128]; query head hq reads KV head hq / (Hq/Hkv).
+ *   mode, R_k, R_v, perm   the rotations used at append time.
+ *   seq_lens  int32 [B] device: context length of each sequence (>= 1).
+ *   sink_fp16 must equal cache->sink_fp16.
+ *   max_ctx   host upper bound of seq_lens (sizes the work split).
+ *   workspace >= kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, SMs) bytes,
+ *             256-B aligned; contents need not be initialised.
+ *   out       fp16 [B][Hq][128].
+ * Computes q_rot = q . R_k, s_t = q_rot . k_t / sqrt(128) over the dequantised
+ * rotated keys (sinks in fp16), softmax, o_rot = sum p_t v_t and
+ * out = o_rot . R_v^T: the rotation is removed after attention (OptR page,
+ * "Key Details"); the attention itself is the standard one ("Why It Matters").
+ */
+KVQ_API kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                const int32_t *perm, const int32_t *seq_lens,
+                                int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                size_t ws_bytes, uint16_t *out, void *stream);
+
+/* Read (and leave set) the device status word: synchronises `stream`.
+ * host_out is a host pointer. */
+KVQ_API kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out);
+
+/* Clear the device status word (asynchronous on `stream`). */
+KVQ_API kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream);
+
+/*
+ * Test exports: the same device code as the hot path, with fp32 outputs.
+ * kvq_debug_rotate_f32: X fp16 [N][128] rows, all rotated by one head's
+ *   rotation (R fp32 [128][128] in dense mode, perm int32 [128] in FWHT mode)
+ *   -> Xrot fp32 [N][128].  `variant` selects the append kernel whose
+ *   rotation is exercised: 0 = the small-batch kernel, 1 = the bulk kernel.
+ * kvq_debug_quantize_f32: Xrot fp32 [N][128] -> codes [N][32] in the logical
+ *   packing, meta [N][4] as {s, z} fp16 pairs (uint16 [N][4][2]).
+ */
+KVQ_API kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mode mode,
+                                const float *R, const int32_t *perm, int32_t variant,
+                                float *Xrot, void *stream);
+KVQ_API kvq_status kvq_debug_quantize_f32(const float *Xrot, int32_t N, uint8_t *codes,
+                                  uint16_t *meta, void *stream);
+
+/* Short text for a status code (static storage). */
+KVQ_API const char *kvq_status_string(kvq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,179 @@
+// libkvq C ABI: argument validation, launch selection, workspace sizing and
+// the status word.  No allocation happens here or in any kernel; the only
+// state kept is a per-device cache of the SM count.
+#include <limits.h>
+
+#include "kvq_internal.cuh"
+
+
+using namespace kvq;
+
+namespace {
+
+constexpr int SPLIT_CTAS_PER_SM = 3;     // resident split CTAs per SM (launch bounds)
+constexpr int MIN_BLOCKS_PER_CTA = 16;   // 256 tokens: below this, fewer CTAs
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
+}
+
+kvq_status check_cache(const kvq_cache_desc *c) {
+    if (!c) return KVQ_ERR_INVALID_ARG;
+    if (c->head_dim != D || c->group != GS) return KVQ_ERR_UNSUPPORTED;
+    if (c->B < 1 || c->Hkv < 1 || c->capacity < BLK_TOK || c->capacity % BLK_TOK != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (c->sink_fp16 < 0 || c->sink_fp16 > MAX_SINK || c->sink_fp16 > c->capacity)
+        return KVQ_ERR_INVALID_ARG;
+    if (!c->blocks || !c->status) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(c->blocks, 16) || !aligned(c->status, 4)) return KVQ_ERR_UNSUPPORTED;
+    if (c->sink_fp16 > 0) {
+        if (!c->k_sink || !c->v_sink) return KVQ_ERR_INVALID_ARG;
+        if (!aligned(c->k_sink, 16) || !aligned(c->v_sink, 16)) return KVQ_ERR_UNSUPPORTED;
+    }
+    if ((long long)c->B * c->Hkv * (c->capacity / BLK_TOK) > INT_MAX) return KVQ_ERR_INVALID_ARG;
+    if (c->B > 32767) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+kvq_status check_rot(kvq_rot_mode mode, const float *R_k, const float *R_v, const int32_t *perm) {
+    if (mode == KVQ_ROT_DENSE) {
+        if (!R_k || !R_v) return KVQ_ERR_INVALID_ARG;
+        if (!aligned(R_k, 16) || !aligned(R_v, 16)) return KVQ_ERR_UNSUPPORTED;
+    } else if (mode == KVQ_ROT_PERM_FWHT) {
+        if (!perm) return KVQ_ERR_INVALID_ARG;
+        if (!aligned(perm, 16)) return KVQ_ERR_UNSUPPORTED;
+    } else {
+        return KVQ_ERR_INVALID_ARG;
+    }
+    return KVQ_OK;
+}
+
+int split_ctas(int B, int Hkv, int max_ctx, int sms) {
+    const long long blocks = (long long)B * Hkv * ((max_ctx + BLK_TOK - 1) / BLK_TOK);
+    long long want = (blocks + MIN_BLOCKS_PER_CTA - 1) / MIN_BLOCKS_PER_CTA;
+    const long long cap = (long long)sms * SPLIT_CTAS_PER_SM;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return (int)want;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_cache_bytes(int32_t B, int32_t Hkv, int32_t capacity) {
+    if (B < 1 || Hkv < 1 || capacity < BLK_TOK || capacity % BLK_TOK) return 0;
+    return (size_t)B * Hkv * (capacity / BLK_TOK) * BLK_BYTES;
+}
+
+kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int32_t T,
+                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                      const int32_t *perm, const kvq_cache_desc *cache,
+                                      int32_t *seq_lens, void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
+    if (T < 0 || !seq_lens || !aligned(seq_lens, 4)) return KVQ_ERR_INVALID_ARG;
+    if (T == 0) return KVQ_OK;
+    if (!K || !V) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16)) return KVQ_ERR_UNSUPPORTED;
+    if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
+    if (e == cudaSuccess) e = launch_seq_bump(seq_lens, cache->B, T, cache->capacity, st);
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max_ctx,
+                                 int32_t sm_count) {
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_ctx < 1 || sm_count < 1) return 0;
+    const int C = split_ctas(B, Hkv, max_ctx, sm_count);
+    return ws_layout(B, Hq, Hkv, C).total;
+}
+
+kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                const int32_t *perm, const int32_t *seq_lens,
+                                int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                size_t ws_bytes, uint16_t *out, void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
+    if (!Q || !out || !seq_lens || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(out, 16) || !aligned(workspace, 256) || !aligned(seq_lens, 4))
+        return KVQ_ERR_UNSUPPORTED;
+    if (Hq < cache->Hkv || Hq % cache->Hkv != 0 || Hq > 65535) return KVQ_ERR_INVALID_ARG;
+    const int G = Hq / cache->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return KVQ_ERR_UNSUPPORTED;
+    if (sink_fp16 != cache->sink_fp16) return KVQ_ERR_INVALID_ARG;
+    if (max_ctx < 1 || max_ctx > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    const int sms = device_sm_count();
+    if (sms < 1) return KVQ_ERR_CUDA;
+    const int C = split_ctas(cache->B, cache->Hkv, max_ctx, sms);
+    if (ws_bytes < ws_layout(cache->B, Hq, cache->Hkv, C).total) return KVQ_ERR_WORKSPACE;
+    cudaError_t e = launch_decode(Q, Hq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out,
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out) {
+    if (!cache || !cache->status || !host_out) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(host_out, cache->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+        return KVQ_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream) {
+    if (!cache || !cache->status) return KVQ_ERR_INVALID_ARG;
+    return cudaMemsetAsync(cache->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? KVQ_OK
+               : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mode mode, const float *R,
+                                const int32_t *perm, int32_t variant, float *Xrot, void *stream) {
+    if (!X || !Xrot || N < 0) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Xrot, 16)) return KVQ_ERR_UNSUPPORTED;
+    kvq_status s = check_rot(mode, R, R, perm);
+    if (s != KVQ_OK) return s;
+    if (variant != 0) return KVQ_ERR_UNSUPPORTED;
+    if (N == 0) return KVQ_OK;
+    cudaError_t e = launch_debug_rotate_small(X, N, mode, R, perm, Xrot,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_debug_quantize_f32(const float *Xrot, int32_t N, uint8_t *codes, uint16_t *meta,
+                                  void *stream) {
+    if (!Xrot || !codes || !meta || N < 0) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(Xrot, 16) || !aligned(codes, 4) || !aligned(meta, 4)) return KVQ_ERR_UNSUPPORTED;
+    if (N == 0) return KVQ_OK;
+    cudaError_t e = launch_debug_quantize(Xrot, N, codes, meta, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+const char *kvq_status_string(kvq_status s) {
+    switch (s) {
+        case KVQ_OK: return "ok";
+        case KVQ_ERR_INVALID_ARG: return "invalid argument";
+        case KVQ_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+        case KVQ_ERR_CUDA: return "CUDA error";
+        case KVQ_ERR_CAPACITY: return "capacity exceeded";
+        case KVQ_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,339 @@
+// Rotate -> quantize -> append kernels (CUDA cores).
+//
+// Method: each KV head owns an orthogonal rotation applied to keys and values
+// before INT2 quantization ("Output-Aware Rotation for INT2 KV-Cache
+// Quantization", section "Key Details"), either a dense 128x128 matrix or a
+// channel reordering followed by a fast Walsh-Hadamard transform ("RotateKV",
+// abstract item (i); "KVLinC", abstract).  The first positions of every
+// sequence are attention sinks kept in fp16 ("RotateKV", item (iii)).
+//
+// Kernels here:
+//   append_dense_kernel  dense rotation on CUDA cores; R is held in registers
+//                        and reused across the tokens of a CTA (small and
+//                        medium T; large T goes to the tensor-core kernel).
+//   append_fwht_kernel   one warp per row: permutation gather, 128-point FWHT
+//                        in registers and shuffles, quantize, pack.
+//   seq_bump_kernel      seq_lens[b] += T once every CTA has read it.
+//   debug kernels        the same rotation / quantizer code with fp32 outputs.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+// Where a rotated row goes: into the packed cache, or out as fp32 (tests).
+struct CacheDst {
+    uint8_t *blocks;
+    uint16_t *k_sink, *v_sink;
+    const int32_t *seq_lens;
+    int32_t *status;
+    int B, T, Hkv, capacity, S, nblk;
+};
+
+// Epilogue shared by both append kernels: row (b, t, h, kind) with rotated
+// values v (lane layout of quantize_row_warp).
+__device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, int h, int kind,
+                                               int L0, const float v[4]) {
+    const int lane = threadIdx.x & 31;
+    const int p = L0 + t;
+    uint8_t *block = c.blocks + ((size_t)(b * c.Hkv + h) * c.nblk + p / BLK_TOK) * BLK_BYTES;
+    const int tau = p % BLK_TOK;
+    if (p < c.S) {
+        uint16_t *sink = (kind == 0 ? c.k_sink : c.v_sink) +
+                         (((size_t)b * c.Hkv + h) * c.S + p) * D + 4 * lane;
+        uint2 pk;
+        pk.x = pack_half2(v[0], v[1]);
+        pk.y = pack_half2(v[2], v[3]);
+        *reinterpret_cast<uint2 *>(sink) = pk;
+        zero_token_warp(block, tau, kind);
+    } else {
+        const QuantWord q = quantize_row_warp(v);
+        store_token_warp(block, tau, kind, q);
+    }
+}
+
+// Reads seq_lens[b] and checks capacity; returns -1 (and flags) if the
+// sequence must be skipped.
+__device__ __forceinline__ int start_len(const CacheDst &c, int b) {
+    const int L0 = c.seq_lens[b];
+    if (L0 < 0) {
+        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_BAD_LEN);
+        return -1;
+    }
+    if ((long long)L0 + c.T > c.capacity) {
+        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_CAPACITY);
+        return -1;
+    }
+    return L0;
+}
+
+// ---- dense rotation on CUDA cores ---------------------------------------------------------
+// 256 threads.  Warp w owns rows 16w..16w+15 of R, lane l columns 4l..4l+3:
+// a 16x4 register tile, reused for every token of the CTA.  Tokens go in
+// batches of 8: every warp forms its partial dot products for all 8, the
+// partials are summed in a fixed order through shared memory, and warp k
+// finishes token k of the batch (quantize + store, or fp32 store).
+constexpr int DENSE_THREADS = 256;
+constexpr int DENSE_BATCH = 8;
+
+struct DenseRows {
+    // cache mode: grid (tchunks, Hkv, 2*B); debug mode: grid (chunks, 1, 1)
+    const uint16_t *X0, *X1;   // K, V (cache) or X (debug)
+    const float *R0, *R1;      // R_k, R_v [Hkv][128][128] (cache) or R (debug)
+    float *out_f32;            // debug output or nullptr
+    int n_rows;                // debug: N
+    int tchunk;                // tokens (rows) per CTA
+};
+
+template <bool TO_CACHE>
+__global__ void __launch_bounds__(DENSE_THREADS)
+    append_dense_kernel(DenseRows a, CacheDst c) {
+    __shared__ __align__(16) uint16_t xs[DENSE_BATCH][D];
+    __shared__ __align__(16) float red[DENSE_BATCH][8][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    int b = 0, h = 0, kind = 0, L0 = 0, row0, nrows;
+    const uint16_t *X;
+    const float *R;
+    if (TO_CACHE) {
+        h = blockIdx.y;
+        kind = blockIdx.z & 1;
+        b = blockIdx.z >> 1;
+        L0 = start_len(c, b);
+        if (L0 < 0) return;
+        row0 = blockIdx.x * a.tchunk;
+        nrows = min(a.tchunk, c.T - row0);
+        X = (kind == 0 ? a.X0 : a.X1);
+        R = (kind == 0 ? a.R0 : a.R1) + (size_t)h * D * D;
+    } else {
+        row0 = blockIdx.x * a.tchunk;
+        nrows = min(a.tchunk, a.n_rows - row0);
+        X = a.X0;
+        R = a.R0;
+    }
+    if (nrows <= 0) return;
+
+    float Rr[16][4];
+#pragma unroll
+    for (int ii = 0; ii < 16; ii++) {
+        const float4 r4 = *reinterpret_cast<const float4 *>(R + (16 * warp + ii) * D + 4 * lane);
+        Rr[ii][0] = r4.x;
+        Rr[ii][1] = r4.y;
+        Rr[ii][2] = r4.z;
+        Rr[ii][3] = r4.w;
+    }
+
+    for (int base = 0; base < nrows; base += DENSE_BATCH) {
+        const int nb = min(DENSE_BATCH, nrows - base);
+        // stage the batch's fp16 rows: 8 rows x 256 B, 16 B per thread
+        if (threadIdx.x < nb * 16) {
+            const int rr = threadIdx.x >> 4, piece = threadIdx.x & 15;
+            const int row = row0 + base + rr;
+            const uint16_t *src;
+            if (TO_CACHE)
+                src = X + (((size_t)b * c.T + row) * c.Hkv + h) * D;
+            else
+                src = X + (size_t)row * D;
+            *reinterpret_cast<uint4 *>(&xs[rr][piece * 8]) =
+                *reinterpret_cast<const uint4 *>(src + piece * 8);
+        }
+        __syncthreads();
+        for (int k = 0; k < nb; k++) {
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(&xs[k][16 * warp]);
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(&xs[k][16 * warp + 8]);
+            const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ii = 0; ii < 8; ii++) {
+                const float2 x2 = unpack_half2(w8[ii]);
+#pragma unroll
+                for (int cc = 0; cc < 4; cc++) {
+                    acc[cc] = fmaf(x2.x, Rr[2 * ii][cc], acc[cc]);
+                    acc[cc] = fmaf(x2.y, Rr[2 * ii + 1][cc], acc[cc]);
+                }
+            }
+            *reinterpret_cast<float4 *>(&red[k][warp][4 * lane]) =
+                make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+        __syncthreads();
+        if (warp < nb) {
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int w2 = 0; w2 < 8; w2++) {
+                const float4 p4 = *reinterpret_cast<const float4 *>(&red[warp][w2][4 * lane]);
+                v[0] += p4.x;
+                v[1] += p4.y;
+                v[2] += p4.z;
+                v[3] += p4.w;
+            }
+            const int row = row0 + base + warp;
+            if (TO_CACHE)
+                cache_epilogue(c, b, row, h, kind, L0, v);
+            else
+                *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+        }
+        __syncthreads();
+    }
+}
+
+// ---- permutation + FWHT ---------------------------------------------------------------------
+// One warp per row: y[i] = x[perm[i]], y <- FWHT(y) / sqrt(128).
+constexpr int FWHT_THREADS = 256;
+
+struct FwhtRows {
+    const uint16_t *X0, *X1;   // K, V (cache) or X (debug)
+    const int32_t *perm;       // [2][Hkv][128] (cache) or [128] (debug)
+    float *out_f32;
+    long long n_rows;          // cache: B*T*Hkv*2 ; debug: N
+};
+
+template <bool TO_CACHE>
+__global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, CacheDst c) {
+    __shared__ __align__(16) uint16_t xs[FWHT_THREADS / 32][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
+    if (row >= a.n_rows) return;
+    int b = 0, t = 0, h = 0, kind = 0, L0 = 0;
+    const uint16_t *src;
+    const int32_t *perm;
+    if (TO_CACHE) {
+        // row order (b, t, h, kind) with kind fastest
+        kind = (int)(row & 1);
+        long long r2 = row >> 1;
+        h = (int)(r2 % c.Hkv);
+        r2 /= c.Hkv;
+        t = (int)(r2 % c.T);
+        b = (int)(r2 / c.T);
+        const int L = c.seq_lens[b];
+        if (L < 0 || (long long)L + c.T > c.capacity) {
+            if (lane == 0 && t == 0 && h == 0 && kind == 0)
+                set_status(c.status, L < 0 ? KVQ_DEV_BAD_LEN : KVQ_DEV_CAPACITY);
+            return;
+        }
+        L0 = L;
+        src = (kind == 0 ? a.X0 : a.X1) + (((size_t)b * c.T + t) * c.Hkv + h) * D;
+        perm = a.perm + ((size_t)kind * c.Hkv + h) * D;
+    } else {
+        src = a.X0 + (size_t)row * D;
+        perm = a.perm;
+    }
+    *reinterpret_cast<uint2 *>(&xs[warp][4 * lane]) =
+        *reinterpret_cast<const uint2 *>(src + 4 * lane);
+    const int4 pi = *reinterpret_cast<const int4 *>(perm + 4 * lane);
+    __syncwarp();
+    float v[4];
+    v[0] = __half2float(__ushort_as_half(xs[warp][pi.x & (D - 1)]));
+    v[1] = __half2float(__ushort_as_half(xs[warp][pi.y & (D - 1)]));
+    v[2] = __half2float(__ushort_as_half(xs[warp][pi.z & (D - 1)]));
+    v[3] = __half2float(__ushort_as_half(xs[warp][pi.w & (D - 1)]));
+    fwht128_warp(v);
+    const float inv_sqrt_d = 0.08838834764831845f;
+#pragma unroll
+    for (int k = 0; k < 4; k++) v[k] *= inv_sqrt_d;
+    if (TO_CACHE)
+        cache_epilogue(c, b, t, h, kind, L0, v);
+    else
+        *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
+            make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// ---- length update ---------------------------------------------------------------------------
+__global__ void seq_bump_kernel(int32_t *seq_lens, int B, int T, int capacity) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    const int L0 = seq_lens[b];
+    if (L0 >= 0 && (long long)L0 + T <= capacity) seq_lens[b] = L0 + T;
+}
+
+// ---- quantizer test export ---------------------------------------------------------------------
+__global__ void debug_quantize_kernel(const float *X, int N, uint8_t *codes, uint16_t *meta) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (row >= N) return;
+    const float4 x4 = *reinterpret_cast<const float4 *>(X + row * D + 4 * lane);
+    const float v[4] = {x4.x, x4.y, x4.z, x4.w};
+    const QuantWord q = quantize_row_warp(v);
+    if (lane < 8) *reinterpret_cast<uint32_t *>(codes + row * 32 + 4 * lane) = q.word;
+    if ((lane & 7) == 0) {
+        const int g = lane >> 3;
+        meta[(row * NG + g) * 2] = q.s;
+        meta[(row * NG + g) * 2 + 1] = q.z;
+    }
+}
+
+// ---- host launchers (called from kvq_api.cu) -----------------------------------------------------
+cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int mode,
+                                const float *R_k, const float *R_v, const int32_t *perm,
+                                const kvq_cache_desc &cd, const int32_t *seq_lens,
+                                cudaStream_t st) {
+    CacheDst c;
+    c.blocks = static_cast<uint8_t *>(cd.blocks);
+    c.k_sink = cd.k_sink;
+    c.v_sink = cd.v_sink;
+    c.seq_lens = seq_lens;
+    c.status = cd.status;
+    c.B = cd.B;
+    c.T = T;
+    c.Hkv = cd.Hkv;
+    c.capacity = cd.capacity;
+    c.S = cd.sink_fp16;
+    c.nblk = cd.capacity / BLK_TOK;
+    if (mode == KVQ_ROT_DENSE) {
+        DenseRows a;
+        a.X0 = K;
+        a.X1 = V;
+        a.R0 = R_k;
+        a.R1 = R_v;
+        a.out_f32 = nullptr;
+        a.n_rows = 0;
+        a.tchunk = T <= 64 ? T : 64;
+        dim3 grid((T + a.tchunk - 1) / a.tchunk, cd.Hkv, 2 * cd.B);
+        append_dense_kernel<true><<<grid, DENSE_THREADS, 0, st>>>(a, c);
+    } else {
+        FwhtRows a;
+        a.X0 = K;
+        a.X1 = V;
+        a.perm = perm;
+        a.out_f32 = nullptr;
+        a.n_rows = (long long)cd.B * T * cd.Hkv * 2;
+        const long long per = FWHT_THREADS / 32;
+        append_fwht_kernel<true><<<(unsigned)((a.n_rows + per - 1) / per), FWHT_THREADS, 0, st>>>(
+            a, c);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_seq_bump(int32_t *seq_lens, int B, int T, int capacity, cudaStream_t st) {
+    seq_bump_kernel<<<(B + 255) / 256, 256, 0, st>>>(seq_lens, B, T, capacity);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
+                                      const int32_t *perm, float *out, cudaStream_t st) {
+    CacheDst c{};
+    if (mode == KVQ_ROT_DENSE) {
+        DenseRows a;
+        a.X0 = a.X1 = X;
+        a.R0 = a.R1 = R;
+        a.out_f32 = out;
+        a.n_rows = N;
+        a.tchunk = 64;
+        append_dense_kernel<false><<<(N + 63) / 64, DENSE_THREADS, 0, st>>>(a, c);
+    } else {
+        FwhtRows a;
+        a.X0 = a.X1 = X;
+        a.perm = perm;
+        a.out_f32 = out;
+        a.n_rows = N;
+        const int per = FWHT_THREADS / 32;
+        append_fwht_kernel<false><<<(N + per - 1) / per, FWHT_THREADS, 0, st>>>(a, c);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
+                                  cudaStream_t st) {
+    debug_quantize_kernel<<<(N + 7) / 8, 256, 0, st>>>(X, N, codes, meta);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,247 @@
+// Device-side helpers shared by the libkvq kernels: cache-block offsets, the
+// exact INT2 group quantizer, fp16 helpers, and mbarrier / bulk-copy PTX.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int D = 128;          // head_dim
+constexpr int GS = 32;          // quantization group (elements of head_dim)
+constexpr int NG = D / GS;      // groups per row
+constexpr int BLK_TOK = 16;     // tokens per cache block
+constexpr int BLK_BYTES = 1536; // bytes per cache block (96 per token)
+constexpr int OFF_VC = 512, OFF_KM = 1024, OFF_VS = 1280, OFF_VZ = 1408;
+constexpr int MAX_SINK = 64;
+
+// ---- cache block offsets (format documented in include/kvq.h) ---------------------
+// tau = token in block.  K code word wi = logical bytes 4wi..4wi+3.
+__device__ __forceinline__ int off_kword(int tau, int wi) {
+    const int r = tau & 7, th = tau >> 3;
+    return 16 * (4 * r + (wi & 3)) + 4 * (2 * th + (wi >> 2));
+}
+// V code piece w = logical bytes 2w, 2w+1 of the token.
+__device__ __forceinline__ int off_vpiece(int tau, int w) {
+    const int q = tau >> 1, side = tau & 1;
+    return OFF_VC + 16 * (4 * (w & 7) + (q & 3)) + 4 * (2 * (q >> 2) + (w >> 3)) + 2 * side;
+}
+__device__ __forceinline__ int off_kmeta(int tau, int g) {
+    const int r = tau & 7, th = tau >> 3;
+    return OFF_KM + 8 * (4 * r + g) + 4 * th;
+}
+__device__ __forceinline__ int off_vscale(int tau, int g) {
+    const int q = tau >> 1, side = tau & 1;
+    return OFF_VS + 8 * (4 * (q & 3) + g) + 4 * (q >> 2) + 2 * side;
+}
+
+__device__ __forceinline__ void set_status(int32_t *status, int bits) {
+    if (status) atomicOr(reinterpret_cast<int *>(status), bits);
+}
+
+// ---- exact INT2 group quantizer -----------------------------------------------------
+// One warp holds one 128-element rotated fp32 row, lane l holding elements
+// 4l..4l+3 (so lanes 8g..8g+7 hold group g).  Arithmetic is the documented
+// IEEE fp32 sequence with explicit round-to-nearest intrinsics (no
+// contraction), so it matches the reference quantizer bit for bit:
+//   s = fp16((max-min)/3), z = fp16(min), inv = s ? 1/s : 0,
+//   c = clamp(rint((x - z) * inv), 0, 3).
+// Returns, in every lane, the logical code word for bytes 4*(l%8)..+3 (the
+// byte e carries element e of each group at bits 2g) and the lane's group
+// scale/zero as fp16 bits.
+struct QuantWord {
+    uint32_t word;
+    uint16_t s, z;
+};
+
+__device__ __forceinline__ QuantWord quantize_row_warp(const float v[4]) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 3;
+    float mn = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
+    float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    const float r = __fsub_rn(mx, mn);
+    const float sf = __fdiv_rn(r, 3.0f);
+    const __half s = __float2half_rn(__fadd_rn(sf, 0.0f));   // zero stored as +0
+    const __half z = __float2half_rn(__fadd_rn(mn, 0.0f));
+    const float sF = __half2float(s), zF = __half2float(z);
+    const float inv = (sF == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sF);
+    uint32_t bits = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const float t = __fmul_rn(__fsub_rn(v[k], zF), inv);
+        const float rt = rintf(t);
+        const uint32_t c = rt < 0.0f ? 0u : (rt > 3.0f ? 3u : (uint32_t)rt);
+        bits |= c << (8 * k + 2 * g);
+    }
+    bits |= __shfl_xor_sync(0xffffffffu, bits, 8);
+    bits |= __shfl_xor_sync(0xffffffffu, bits, 16);
+    QuantWord q;
+    q.word = bits;
+    q.s = __half_as_ushort(s);
+    q.z = __half_as_ushort(z);
+    return q;
+}
+
+// Store one token of one kind (0 = K, 1 = V) into its block, from the warp
+// layout of quantize_row_warp.  Lanes 0..7 write the code word l, lanes 8g
+// write group g's metadata.
+__device__ __forceinline__ void store_token_warp(uint8_t *block, int tau, int kind,
+                                                 const QuantWord &q) {
+    const int lane = threadIdx.x & 31;
+    if (lane < 8) {
+        if (kind == 0) {
+            *reinterpret_cast<uint32_t *>(block + off_kword(tau, lane)) = q.word;
+        } else {
+            *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 2 * lane)) =
+                (uint16_t)(q.word & 0xffffu);
+            *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 2 * lane + 1)) =
+                (uint16_t)(q.word >> 16);
+        }
+    }
+    if ((lane & 7) == 0) {
+        const int g = lane >> 3;
+        if (kind == 0) {
+            *reinterpret_cast<uint32_t *>(block + off_kmeta(tau, g)) =
+                (uint32_t)q.s | ((uint32_t)q.z << 16);
+        } else {
+            *reinterpret_cast<uint16_t *>(block + off_vscale(tau, g)) = q.s;
+            *reinterpret_cast<uint16_t *>(block + off_vscale(tau, g) + 128) = q.z;
+        }
+    }
+}
+
+// Zero one token's slots of one kind (sink positions).
+__device__ __forceinline__ void zero_token_warp(uint8_t *block, int tau, int kind) {
+    QuantWord q;
+    q.word = 0;
+    q.s = 0;
+    q.z = 0;
+    store_token_warp(block, tau, kind, q);
+}
+
+// ---- warp FWHT of a 128-vector held as 4 consecutive elements per lane -------------
+// Sylvester order; butterflies (a, b) -> (a + b, a - b) at every stride.
+__device__ __forceinline__ void fwht128_warp(float v[4]) {
+    const int lane = threadIdx.x & 31;
+    float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+    v[0] = a0 + a2;
+    v[2] = a0 - a2;
+    v[1] = a1 + a3;
+    v[3] = a1 - a3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+            v[k] = upper ? (o - v[k]) : (v[k] + o);
+        }
+    }
+}
+
+// ---- mbarrier and bulk-copy (TMA, non-tensor) PTX wrappers ---------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` polls (each try_wait may itself
+// suspend for a while) and reports false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint32_t limit = (1u << 22)) {
+    for (uint32_t i = 0; i < limit; i++)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// 1-D bulk copy global -> shared, completion reported on `bar` as tx bytes.
+// Both addresses 16-B aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---- tensor-core MMA (m16n8k16, fp16 in, fp32 accumulate) ------------------------------
+__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_half2(uint32_t u) {
+    const __half2 h = *reinterpret_cast<const __half2 *>(&u);
+    return __half22float2(h);
+}
+
+// ---- host launchers (defined in kvq_append.cu / kvq_decode.cu) ---------------------------
+cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int mode,
+                                const float *R_k, const float *R_v, const int32_t *perm,
+                                const kvq_cache_desc &cd, const int32_t *seq_lens,
+                                cudaStream_t st);
+cudaError_t launch_seq_bump(int32_t *seq_lens, int B, int T, int capacity, cudaStream_t st);
+cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
+                                      const int32_t *perm, float *out, cudaStream_t st);
+cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
+                                  cudaStream_t st);
+cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
+                          const float *R_k, const float *R_v, const int32_t *perm,
+                          const int32_t *seq_lens, int C, void *ws, uint16_t *out,
+                          cudaStream_t st);
+
+// Decode workspace: prefix sums, prepared queries, sink partials, split partials.
+struct WsLayout {
+    size_t prefix, qprep, sinkp, part, total;
+};
+WsLayout ws_layout(int B, int Hq, int Hkv, int C);
+
+}  // namespace kvq

@@ -1,0 +1,216 @@
+"""Thin Python binding of libkvq's C ABI (include/kvq.h).
+
+Argument marshalling only: torch tensors are checked for dtype, shape and
+contiguity and passed to the library as raw device pointers together with
+the current CUDA stream.  Every step of the computation runs in libkvq's
+CUDA kernels; there is no Python or CPU fallback.  If libkvq.so is missing
+the import fails with an error that says how to build it.
+"""
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+D = 128
+GROUP = 32
+BLOCK_TOKENS = 16
+BLOCK_BYTES = 1536
+
+KVQ_ROT_DENSE = 0
+KVQ_ROT_PERM_FWHT = 1
+
+KVQ_DEV_CAPACITY = 1
+KVQ_DEV_BAD_LEN = 2
+KVQ_DEV_TIMEOUT = 4
+
+_STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CUDA",
+           4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_WORKSPACE"}
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s failed: %s (%d)" % (fn, _STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class CacheDesc(C.Structure):
+    _fields_ = [("B", C.c_int32), ("Hkv", C.c_int32), ("head_dim", C.c_int32),
+                ("group", C.c_int32), ("capacity", C.c_int32), ("sink_fp16", C.c_int32),
+                ("blocks", C.c_void_p), ("k_sink", C.c_void_p), ("v_sink", C.c_void_p),
+                ("status", C.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libkvq.so (built in-tree by rotated_int2_kv_head_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libkvq.so is not built (%s); run `python -m "
+                          "rotated_int2_kv_head_b200.build`" % LIB_PATH)
+    L = C.CDLL(LIB_PATH)
+    p, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+    L.kvq_cache_bytes.restype = sz
+    L.kvq_cache_bytes.argtypes = [i32, i32, i32]
+    L.kvq_rotate_quantize_append.restype = C.c_int
+    L.kvq_rotate_quantize_append.argtypes = [p, p, i32, C.c_int, p, p, p, C.POINTER(CacheDesc), p, p]
+    L.kvq_decode_workspace_size.restype = sz
+    L.kvq_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    L.kvq_decode_attention.restype = C.c_int
+    L.kvq_decode_attention.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p, i32, i32,
+                                       p, sz, p, p]
+    L.kvq_get_status.restype = C.c_int
+    L.kvq_get_status.argtypes = [C.POINTER(CacheDesc), p, C.POINTER(C.c_int32)]
+    L.kvq_clear_status.restype = C.c_int
+    L.kvq_clear_status.argtypes = [C.POINTER(CacheDesc), p]
+    L.kvq_debug_rotate_f32.restype = C.c_int
+    L.kvq_debug_rotate_f32.argtypes = [p, i32, C.c_int, p, p, i32, p, p]
+    L.kvq_debug_quantize_f32.restype = C.c_int
+    L.kvq_debug_quantize_f32.argtypes = [p, i32, p, p, p]
+    L.kvq_status_string.restype = C.c_char_p
+    L.kvq_status_string.argtypes = [C.c_int]
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise KvqError(fn, code)
+
+
+def _need(t, dtype, name, shape=None):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+class KVCache:
+    """A packed INT2 cache for B sequences x Hkv heads (memory owned by torch)."""
+
+    def __init__(self, B, Hkv, capacity, sink_fp16=0, device="cuda"):
+        nbytes = lib().kvq_cache_bytes(B, Hkv, capacity)
+        if nbytes == 0:
+            raise ValueError("bad cache shape B=%d Hkv=%d capacity=%d" % (B, Hkv, capacity))
+        self.B, self.Hkv, self.capacity, self.sink_fp16 = B, Hkv, capacity, sink_fp16
+        self.blocks = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        if sink_fp16 > 0:
+            self.k_sink = torch.zeros((B, Hkv, sink_fp16, D), dtype=torch.float16, device=device)
+            self.v_sink = torch.zeros_like(self.k_sink)
+        else:
+            self.k_sink = self.v_sink = None
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.desc = CacheDesc(B, Hkv, D, GROUP, capacity, sink_fp16, self.blocks.data_ptr(),
+                              0 if self.k_sink is None else self.k_sink.data_ptr(),
+                              0 if self.v_sink is None else self.v_sink.data_ptr(),
+                              self.status.data_ptr())
+
+    def block_view(self):
+        """blocks as uint8 [B][Hkv][capacity/16][1536]."""
+        return self.blocks.view(self.B, self.Hkv, self.capacity // BLOCK_TOKENS, BLOCK_BYTES)
+
+
+def kvq_cache_bytes(B, Hkv, capacity):
+    return lib().kvq_cache_bytes(B, Hkv, capacity)
+
+
+def kvq_rotate_quantize_append(K, V, mode, R_k, R_v, perm, cache, seq_lens, stream=None):
+    """K, V fp16 [B][T][Hkv][128]; seq_lens int32 [B] (updated in place)."""
+    B, T, Hkv, d = K.shape
+    _need(K, torch.float16, "K", (cache.B, T, cache.Hkv, D))
+    _need(V, torch.float16, "V", K.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    if mode == KVQ_ROT_DENSE:
+        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
+    else:
+        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
+    _check("kvq_rotate_quantize_append",
+           lib().kvq_rotate_quantize_append(_ptr(K), _ptr(V), T, mode, _ptr(R_k), _ptr(R_v),
+                                            _ptr(perm), C.byref(cache.desc), _ptr(seq_lens),
+                                            _stream(stream)))
+
+
+def kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count=None):
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return lib().kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count)
+
+
+def decode_workspace(B, Hq, Hkv, max_ctx, device="cuda"):
+    n = kvq_decode_workspace_size(B, Hq, Hkv, max_ctx)
+    if n == 0:
+        raise ValueError("bad decode shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kvq_decode_attention(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
+                         workspace, out, stream=None):
+    """Q fp16 [B][Hq][128] -> out fp16 [B][Hq][128]; seq_lens int32 [B] on device."""
+    B, Hq, d = Q.shape
+    _need(Q, torch.float16, "Q", (cache.B, Hq, D))
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    if mode == KVQ_ROT_DENSE:
+        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
+    else:
+        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
+    _check("kvq_decode_attention",
+           lib().kvq_decode_attention(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k), _ptr(R_v),
+                                      _ptr(perm), _ptr(seq_lens), sink_fp16, max_ctx,
+                                      _ptr(workspace), workspace.numel(), _ptr(out),
+                                      _stream(stream)))
+
+
+def kvq_get_status(cache, stream=None):
+    v = C.c_int32(0)
+    _check("kvq_get_status", lib().kvq_get_status(C.byref(cache.desc), _stream(stream), C.byref(v)))
+    return v.value
+
+
+def kvq_clear_status(cache, stream=None):
+    _check("kvq_clear_status", lib().kvq_clear_status(C.byref(cache.desc), _stream(stream)))
+
+
+def kvq_debug_rotate_f32(X, mode, R=None, perm=None, variant=0, stream=None):
+    """X fp16 [N][128] -> fp32 [N][128] rotated by one head's rotation."""
+    _need(X, torch.float16, "X")
+    N = X.shape[0]
+    out = torch.empty((N, D), dtype=torch.float32, device=X.device)
+    _check("kvq_debug_rotate_f32",
+           lib().kvq_debug_rotate_f32(_ptr(X), N, mode, _ptr(R), _ptr(perm), variant, _ptr(out),
+                                      _stream(stream)))
+    return out
+
+
+def kvq_debug_quantize_f32(Xrot, stream=None):
+    """fp32 [N][128] -> (codes uint8 [N][32] logical packing, meta int16 [N][4][2] {s, z})."""
+    _need(Xrot, torch.float32, "Xrot")
+    N = Xrot.shape[0]
+    codes = torch.empty((N, 32), dtype=torch.uint8, device=Xrot.device)
+    meta = torch.empty((N, 4, 2), dtype=torch.int16, device=Xrot.device)
+    _check("kvq_debug_quantize_f32",
+           lib().kvq_debug_quantize_f32(_ptr(Xrot), N, _ptr(codes), _ptr(meta), _stream(stream)))
+    return codes, meta

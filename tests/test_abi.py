@@ -1,0 +1,107 @@
+"""The C-ABI library loads, exports every entry point include/kvq.h declares,
+and rejects bad arguments on the host before touching a GPU.  CPU only."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import rotated_int2_kv_head_b200 as kvq
+from rotated_int2_kv_head_b200 import build as kbuild
+from rotated_int2_kv_head_b200.kvq import CacheDesc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kvq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ["kvq_rotate_quantize_append", "kvq_decode_attention", "kvq_decode_workspace_size",
+              "kvq_get_status", "kvq_debug_rotate_f32", "kvq_debug_quantize_f32"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_only_api_symbols_are_exported():
+    out = os.popen("nm -D --defined-only %s" % kbuild.LIB).read()
+    ours = sorted({l.split()[-1] for l in out.splitlines() if " T " in l and "kvq" in l})
+    assert ours == declared_functions()
+
+
+def desc(**kw):
+    d = dict(B=2, Hkv=2, head_dim=128, group=32, capacity=64, sink_fp16=0, blocks=4096,
+             k_sink=0, v_sink=0, status=256)
+    d.update(kw)
+    return CacheDesc(d["B"], d["Hkv"], d["head_dim"], d["group"], d["capacity"], d["sink_fp16"],
+                     d["blocks"], d["k_sink"], d["v_sink"], d["status"])
+
+
+def append(L, cache, mode=0, rk=1024, rv=1024, perm=2048, K=8192, V=8192, T=3, seq=512):
+    return L.kvq_rotate_quantize_append(C.c_void_p(K), C.c_void_p(V), T, mode, C.c_void_p(rk),
+                                        C.c_void_p(rv), C.c_void_p(perm), C.byref(cache),
+                                        C.c_void_p(seq), None)
+
+
+def test_append_rejects_bad_arguments_on_host(L):
+    assert append(L, desc(head_dim=64)) == 2              # UNSUPPORTED
+    assert append(L, desc(group=16)) == 2
+    assert append(L, desc(capacity=40)) == 1              # not a multiple of 16
+    assert append(L, desc(blocks=0)) == 1
+    assert append(L, desc(blocks=4100)) == 2              # misaligned
+    assert append(L, desc(sink_fp16=4)) == 1              # sinks without buffers
+    assert append(L, desc(sink_fp16=65, k_sink=64, v_sink=64)) == 1
+    assert append(L, desc(), rk=0) == 1                   # dense needs R
+    assert append(L, desc(), mode=1, perm=0) == 1         # FWHT needs perm
+    assert append(L, desc(), mode=7) == 1
+    assert append(L, desc(), K=0) == 1
+    assert append(L, desc(), K=8200) == 2
+    assert append(L, desc(), T=-1) == 1
+    assert append(L, desc(), T=65) == 1                   # T > capacity
+    assert append(L, desc(), T=0) == 0                    # nothing to do
+    assert L.kvq_rotate_quantize_append(None, None, 1, 0, None, None, None, None, None, None) == 1
+
+
+def test_decode_rejects_bad_arguments_on_host(L):
+    def dec(cache, Hq=2, sink=0, max_ctx=64, ws=4096, wsb=1 << 20, Q=8192, out=8192, seq=512):
+        return L.kvq_decode_attention(C.c_void_p(Q), Hq, C.byref(cache), 0, C.c_void_p(1024),
+                                      C.c_void_p(1024), None, C.c_void_p(seq), sink, max_ctx,
+                                      C.c_void_p(ws), wsb, C.c_void_p(out), None)
+    assert dec(desc(), Hq=3) == 1          # Hq not a multiple of Hkv
+    assert dec(desc(), Hq=6) == 2          # G = 3 unsupported
+    assert dec(desc(), Hq=32) == 2         # G = 16 unsupported
+    assert dec(desc(), sink=2) == 1        # sink count mismatch
+    assert dec(desc(), max_ctx=0) == 1
+    assert dec(desc(), max_ctx=65) == 1
+    assert dec(desc(), ws=4100) == 2       # workspace alignment
+    assert dec(desc(), Q=0) == 1
+
+
+def test_workspace_size_is_monotone_and_validated(L):
+    f = L.kvq_decode_workspace_size
+    assert f(0, 1, 1, 10, 148) == 0
+    assert f(1, 3, 2, 10, 148) == 0
+    a = f(1, 32, 32, 32768, 148)
+    b = f(64, 32, 32, 65536, 148)
+    assert 0 < a < b
+    assert f(8, 32, 8, 131072, 148) % 256 == 0
+
+
+def test_cache_bytes(L):
+    assert L.kvq_cache_bytes(1, 32, 32768) == 32 * 2048 * 1536
+    assert L.kvq_cache_bytes(1, 1, 17) == 0

@@ -1,0 +1,269 @@
+"""CUDA path (libkvq through its C ABI) against the CPU oracle, element by
+element, on seeded inputs.  Tolerances:
+  - codes, scales, zeros: bit-exact when both sides quantize the same
+    rotated fp32 rows;
+  - rotation: <= 1e-3 relative;
+  - packed cache vs the oracle's own rotation: <= 1e-4 of code elements
+    differ, each at a near tie;
+  - decode output: max-abs error <= 2e-3 * ||o_ref||_2 per (sequence, head).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import rotated_int2_kv_head_b200 as kvq
+import workloads as W
+from oracle import oracle as orc
+
+from kvq_testlib import (D, download_cache, f16bits, gpu_append, gpu_decode, logical,
+                         near_tie_ok, rel_err, rot_tensors, upload_oracle_cache)
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quantizer_worked.json")
+DEC_TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from rotated_int2_kv_head_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+# --- quantizer and rotation stages -------------------------------------------------------------
+
+def edge_rows():
+    rows = []
+    g = json.load(open(GOLDEN))["groups"]
+    for case in g:
+        rows.append(np.tile(np.array(case["x"], np.float32), 4))
+    rng = np.random.default_rng(1)
+    r = rng.standard_normal(D).astype(np.float32)
+    r[:32] = 7.0                                       # constant group
+    r[32:64] = np.linspace(-1, 2, 32)                  # exact grid
+    r[64:96] = 1000.0 + rng.standard_normal(32) * 1e-3  # offset >> range
+    r[96:] = rng.standard_normal(32) * 1e-6            # subnormal fp16 scale
+    rows.append(r)
+    rows.append(np.zeros(D, np.float32))
+    rows.append(-np.ones(D, np.float32) * 0.0)
+    return np.stack(rows)
+
+
+def test_quantizer_bit_exact():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal((8192, D)) * rng.uniform(0.01, 100, (8192, 1))).astype(np.float32)
+    x = np.concatenate([x, edge_rows()])
+    codes, meta = kvq.kvq_debug_quantize_f32(torch.from_numpy(x).cuda())
+    codes = codes.cpu().numpy()
+    meta = meta.cpu().numpy().view(np.uint16)
+    oc, os_, oz = orc.quantize_rows(x)
+    packed = np.stack([orc.pack_row(c) for c in oc])
+    assert np.array_equal(codes, packed)
+    assert np.array_equal(meta[:, :, 0], os_)
+    assert np.array_equal(meta[:, :, 1], oz)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_rotation_stage(mode):
+    w = W.custom(seed=3, Hkv=1, mode=mode, k_outliers=8)
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((3000, D)) * 3).astype(np.float16)
+    x[:, :8] *= 20
+    rt, rn = rot_tensors(w)
+    X = torch.from_numpy(x).cuda()
+    if mode == 0:
+        got = kvq.kvq_debug_rotate_f32(X, 0, R=rt[0][0].contiguous())
+        ref = orc.rotate_rows_f32(x.view(np.uint16), 0, R=rn[0][0])
+    else:
+        got = kvq.kvq_debug_rotate_f32(X, 1, perm=rt[2][0, 0].contiguous())
+        ref = orc.rotate_rows_f32(x.view(np.uint16), 1, perm=rn[2][0, 0])
+    got = got.cpu().numpy()
+    err = np.abs(got - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert err.max() <= 1e-3
+    assert err.max() <= 1e-5        # fp32 arithmetic: far inside the bound
+
+
+# --- append ---------------------------------------------------------------------------------------
+
+def run_append(w, L0, T, device="cuda"):
+    """Append T tokens at lengths L0 on both sides; return everything."""
+    rt, rn = rot_tensors(w)
+    B = w.B
+    K = torch.stack([W.kv_rows(w, b, L0[b], L0[b] + T, "cpu")[0] for b in range(B)])
+    V = torch.stack([W.kv_rows(w, b, L0[b], L0[b] + T, "cpu")[1] for b in range(B)])
+    cap = ((max(L0) + T + 15) // 16) * 16 + 16
+    cache = kvq.KVCache(B, w.Hkv, cap, w.sink)
+    sl = torch.tensor(L0, dtype=torch.int32, device=device)
+    gpu_append(cache, K.cuda(), V.cuda(), w, rt, sl)
+    oc = orc.Cache(B, w.Hkv, cap, w.sink)
+    osl = np.array(L0, np.int32)
+    st = orc.append(oc, f16bits(K), f16bits(V), w.mode, rn[0], rn[1], rn[2], osl)
+    assert st == 0
+    assert list(sl.cpu().numpy()) == list(osl)
+    assert kvq.kvq_get_status(cache) == 0
+    return cache, oc, K, V, rt, rn
+
+
+@pytest.mark.parametrize("mode,S,T,L0", [
+    (0, 0, 1, [0, 5, 16]),
+    (0, 4, 37, [0, 3, 29]),
+    (1, 0, 37, [0, 5, 16]),
+    (1, 4, 1, [3, 0, 21]),
+    (0, 20, 70, [0, 2, 31]),
+])
+def test_append_matches_oracle(mode, S, T, L0):
+    w = W.custom(seed=10 + T, B=3, Hkv=2, mode=mode, sink=S, k_outliers=4,
+                 channel_scale=(0.5, 20.0) if mode == 1 else None)
+    cache, oc, K, V, rt, rn = run_append(w, L0, T)
+    gc = download_cache(cache)
+    # (a) exact: the GPU bytes equal the oracle quantizer applied to the GPU's
+    #     own rotated rows, stored in the oracle's layout
+    exp = orc.Cache(w.B, w.Hkv, oc.capacity, S)
+    n_codes = n_diff = 0
+    for kind, X in ((0, K), (1, V)):
+        for h in range(w.Hkv):
+            rows = X[:, :, h].reshape(-1, D).cuda()
+            if mode == 0:
+                R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
+                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R).cpu().numpy()
+                orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 0,
+                                      R=(rn[0] if kind == 0 else rn[1])[h])
+            else:
+                pm = rt[2][kind, h].contiguous()
+                grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=pm).cpu().numpy()
+                orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 1,
+                                      perm=rn[2][kind, h])
+            grot = grot.reshape(w.B, T, D)
+            orot = orot.reshape(w.B, T, D)
+            for b in range(w.B):
+                for t in range(T):
+                    p = L0[b] + t
+                    if p < S:
+                        sink = (gc.k_sink if kind == 0 else gc.v_sink)[b, h, p]
+                        assert np.array_equal(sink, orc.f32_to_f16_bits(grot[b, t]))
+                        continue
+                    c, s, z = orc.quantize_rows(grot[b, t])
+                    lg = logical(gc, b, h, p)
+                    assert np.array_equal(lg[kind], c[0])
+                    assert np.array_equal(lg[2 + 2 * kind], s[0])
+                    assert np.array_equal(lg[3 + 2 * kind], z[0])
+                    # (b) against the oracle's own rotation: near ties only
+                    lo = logical(oc, b, h, p)
+                    n_codes += D
+                    n_diff += int((lo[kind] != lg[kind]).sum())
+                    if np.array_equal(lo[2 + 2 * kind], lg[2 + 2 * kind]) and \
+                            np.array_equal(lo[3 + 2 * kind], lg[3 + 2 * kind]):
+                        assert near_tie_ok(orot[b, t], lo[kind], lg[kind], lo[2 + 2 * kind],
+                                           lo[3 + 2 * kind])
+    assert n_diff <= max(2, 1e-4 * n_codes), (n_diff, n_codes)
+    # blocks of positions never written stay untouched (zero)
+    for b in range(w.B):
+        last = (L0[b] + T + 15) // 16
+        assert not gc.blocks[b, :, last:].any()
+
+
+def test_append_capacity_and_status():
+    w = W.custom(seed=4, B=2, Hkv=1, mode=0)
+    rt, _ = rot_tensors(w)
+    cache = kvq.KVCache(2, 1, 32, 0)
+    K = torch.randn((2, 8, 1, D), device="cuda").half()
+    sl = torch.tensor([30, 2], dtype=torch.int32, device="cuda")
+    gpu_append(cache, K, K, w, rt, sl)
+    assert list(sl.cpu().numpy()) == [30, 10]
+    assert kvq.kvq_get_status(cache) == kvq.KVQ_DEV_CAPACITY
+    assert not cache.block_view()[0].any()
+    kvq.kvq_clear_status(cache)
+    assert kvq.kvq_get_status(cache) == 0
+
+
+# --- decode ----------------------------------------------------------------------------------------
+
+def build_oracle_cache(w, lens, cap):
+    """The oracle appends every sequence's tokens [0, lens[b]) (one call per
+    distinct chunk so sequences can differ in length)."""
+    _, rn = rot_tensors(w)
+    oc = orc.Cache(w.B, w.Hkv, cap, w.sink)
+    for b in range(w.B):
+        k, v = W.kv_rows(w, b, 0, lens[b], "cpu")
+        sub = orc.Cache(1, w.Hkv, cap, w.sink)
+        sl = np.zeros(1, np.int32)
+        orc.append(sub, f16bits(k[None]), f16bits(v[None]), w.mode, rn[0], rn[1], rn[2], sl)
+        oc.blocks[b] = sub.blocks[0]
+        if w.sink:
+            oc.k_sink[b] = sub.k_sink[0]
+            oc.v_sink[b] = sub.v_sink[0]
+    return oc
+
+
+DECODE_CASES = [
+    # G, mode, S, lengths
+    (1, 0, 0, [1, 15, 16, 17, 300, 1000]),
+    (1, 1, 0, [33, 512, 2047]),
+    (2, 0, 4, [1, 4, 5, 19, 800]),
+    (4, 0, 4, [4, 3, 20, 257, 1500]),
+    (8, 1, 17, [16, 17, 18, 600]),
+    (4, 1, 0, [2048, 1, 999]),
+]
+
+
+@pytest.mark.parametrize("G,mode,S,lens", DECODE_CASES)
+def test_decode_matches_oracle(G, mode, S, lens):
+    Hkv = 2
+    w = W.custom(seed=20 + G + S, B=len(lens), Hq=Hkv * G, Hkv=Hkv, mode=mode, sink=S,
+                 k_outliers=6, sink_key_scale=50.0 if S else 1.0)
+    cap = ((max(lens) + 15) // 16) * 16
+    oc = build_oracle_cache(w, lens, cap)
+    rt, rn = rot_tensors(w)
+    Q = W.queries(w, "cpu")
+    sl = np.array(lens, np.int32)
+    ref, st = orc.decode(oc, f16bits(Q), mode, rn[0], rn[1], rn[2], sl, n_threads=8)
+    assert st == 0
+    cache = upload_oracle_cache(oc)
+    out = gpu_decode(cache, Q.cuda(), w, rt, torch.from_numpy(sl).cuda(), max(lens))
+    err = rel_err(out.cpu().numpy(), ref)
+    assert err.max() <= DEC_TOL, err.max()
+    assert kvq.kvq_get_status(cache) == 0
+
+
+@pytest.mark.parametrize("G,mode,S,lens", DECODE_CASES[:3])
+def test_append_then_decode_end_to_end(G, mode, S, lens):
+    """GPU append + GPU decode against oracle append + oracle decode."""
+    Hkv = 2
+    w = W.custom(seed=40 + G, B=len(lens), Hq=Hkv * G, Hkv=Hkv, mode=mode, sink=S, k_outliers=6)
+    cap = ((max(lens) + 15) // 16) * 16
+    oc = build_oracle_cache(w, lens, cap)
+    rt, rn = rot_tensors(w)
+    cache = kvq.KVCache(w.B, Hkv, cap, S)
+    for b in range(w.B):     # one sequence at a time: lengths differ
+        k, v = W.kv_rows(w, b, 0, lens[b], "cuda")
+        sub = kvq.KVCache(1, Hkv, cap, S)
+        sl1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        gpu_append(sub, k[None], v[None], w, rt, sl1)
+        cache.block_view()[b].copy_(sub.block_view()[0])
+        if S:
+            cache.k_sink[b].copy_(sub.k_sink[0])
+            cache.v_sink[b].copy_(sub.v_sink[0])
+    Q = W.queries(w, "cpu")
+    sl = np.array(lens, np.int32)
+    ref, _ = orc.decode(oc, f16bits(Q), mode, rn[0], rn[1], rn[2], sl, n_threads=8)
+    out = gpu_decode(cache, Q.cuda(), w, rt, torch.from_numpy(sl).cuda(), max(lens))
+    err = rel_err(out.cpu().numpy(), ref)
+    assert err.max() <= DEC_TOL, err.max()
+
+
+def test_decode_bad_lengths_give_zero_rows_and_status():
+    w = W.custom(seed=7, B=3, Hq=2, Hkv=2, mode=0)
+    lens = [40, 40, 40]
+    oc = build_oracle_cache(w, lens, 48)
+    rt, rn = rot_tensors(w)
+    cache = upload_oracle_cache(oc)
+    Q = W.queries(w, "cpu")
+    sl = np.array([40, 0, 49], np.int32)
+    out = gpu_decode(cache, Q.cuda(), w, rt, torch.from_numpy(sl).cuda(), 48).cpu().numpy()
+    assert not out[1].any() and not out[2].any()
+    assert kvq.kvq_get_status(cache) == kvq.KVQ_DEV_BAD_LEN
+    ref, _ = orc.decode(oc, f16bits(Q), 0, rn[0], rn[1], rn[2], sl)
+    assert rel_err(out[0:1], ref[0:1]).max() <= DEC_TOL
