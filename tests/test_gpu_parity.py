@@ -238,7 +238,8 @@ def test_append_then_decode_end_to_end(G, mode, S, lens):
     rt, rn = rot_tensors(w)
     cache = kvq.KVCache(w.B, Hkv, cap, S)
     for b in range(w.B):     # one sequence at a time: lengths differ
-        k, v = W.kv_rows(w, b, 0, lens[b], "cuda")
+        k, v = W.kv_rows(w, b, 0, lens[b], "cpu")
+        k, v = k.cuda(), v.cuda()
         sub = kvq.KVCache(1, Hkv, cap, S)
         sl1 = torch.zeros(1, dtype=torch.int32, device="cuda")
         gpu_append(sub, k[None], v[None], w, rt, sl1)

@@ -19,8 +19,10 @@ The five workloads (head_dim 128, INT2 groups of 32 along head_dim):
               bulk append of 32768 prefill tokens x 32 heads for B=4.
 
 Every K/V row is drawn from a stream keyed by (workload, kind, sequence,
-1024-token chunk), so any token range can be regenerated on its own, on any
-device, without drawing the rest.
+1024-token chunk), so any token range can be regenerated on its own without
+drawing the rest.  The stream depends on the device it is drawn on (torch's
+CPU and CUDA generators differ): a comparison draws once, on one device, and
+hands the same tensor to both sides.
 """
 from dataclasses import dataclass, field
 from typing import List, Optional
@@ -129,7 +131,8 @@ def channel_scales(w: Workload):
 
 def _chunk_rows(w: Workload, kind: int, b: int, chunk: int, device) -> torch.Tensor:
     g = torch.Generator(device=device)
-    g.manual_seed(((w.seed * 1_000_003 + kind) * 1_000_033 + b) * 1_000_037 + chunk)
+    key = ((w.seed * 1_000_003 + kind) * 1_000_033 + b) * 1_000_037 + chunk
+    g.manual_seed(key % (1 << 62))
     return torch.randn((CHUNK, w.Hkv, D), generator=g, device=device, dtype=torch.float32)
 
 
