@@ -51,8 +51,7 @@
  *   V codes  [512,1024)  logical 16-bit piece w (bytes 2w, 2w+1) at
  *                        512 + 16*(4*(w%8) + q%4) + 4*(2*(q/4) + w/8) + 2*side
  *   K meta   [1024,1280) group g: fp16 s then fp16 z at 1024 + 8*(4r + g) + 4*th
- *   V scales [1280,1408) group g: fp16 s at 1280 + 8*(4*(q%4) + g) + 4*(q/4) + 2*side
- *   V zeros  [1408,1536) same offset + 128
+ *   V meta   [1280,1536) group g: fp16 s then fp16 z at 1280 + 8*(4r + g) + 4*th
  * This order is the operand order of the decode kernel's tensor-core
  * fragments, so one warp reads each 512-byte region as 32 x 16 contiguous
  * bytes.  The 96 bytes per token-head (3 bits per element) are the whole

@@ -251,9 +251,8 @@ void orc_unpack_row(const uint8_t *bytes, uint8_t *codes) {
 /*                        512 + 16*(4*(w%8) + p%4) + 4*(2*(p/4) + w/8) + 2*side*/
 /*   K meta   [1024,1280): group g {s, z} (two fp16, s first) at              */
 /*                        1024 + 8*(4r + g) + 4*th                            */
-/*   V scale  [1280,1408): group g scale at                                   */
-/*                        1280 + 8*(4*(p%4) + g) + 4*(p/4) + 2*side           */
-/*   V zero   [1408,1536): same offset + 128                                  */
+/*   V meta   [1280,1536): group g {s, z} (two fp16, s first) at              */
+/*                        1280 + 8*(4r + g) + 4*th                            */
 /* ------------------------------------------------------------------------ */
 
 static size_t off_kword(int tau, int wi) {
@@ -268,9 +267,9 @@ static size_t off_kmeta(int tau, int g) {
     int r = tau % 8, th = tau / 8;
     return (size_t)(1024 + 8 * (4 * r + g) + 4 * th);
 }
-static size_t off_vscale(int tau, int g) {
-    int p = tau / 2, side = tau % 2;
-    return (size_t)(1280 + 8 * (4 * (p % 4) + g) + 4 * (p / 4) + 2 * side);
+static size_t off_vmeta(int tau, int g) {
+    int r = tau % 8, th = tau / 8;
+    return (size_t)(1280 + 8 * (4 * r + g) + 4 * th);
 }
 
 static void put16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)(v & 0xff); p[1] = (uint8_t)(v >> 8); }
@@ -285,8 +284,8 @@ void orc_store_token(uint8_t *block, int tau, const uint8_t *kbytes, const uint8
     for (int g = 0; g < NG; g++) {
         put16(block + off_kmeta(tau, g), ks[g]);
         put16(block + off_kmeta(tau, g) + 2, kz[g]);
-        put16(block + off_vscale(tau, g), vs[g]);
-        put16(block + off_vscale(tau, g) + 128, vz[g]);
+        put16(block + off_vmeta(tau, g), vs[g]);
+        put16(block + off_vmeta(tau, g) + 2, vz[g]);
     }
 }
 
@@ -297,8 +296,8 @@ void orc_load_token(const uint8_t *block, int tau, uint8_t *kbytes, uint8_t *vby
     for (int g = 0; g < NG; g++) {
         ks[g] = get16(block + off_kmeta(tau, g));
         kz[g] = get16(block + off_kmeta(tau, g) + 2);
-        vs[g] = get16(block + off_vscale(tau, g));
-        vz[g] = get16(block + off_vscale(tau, g) + 128);
+        vs[g] = get16(block + off_vmeta(tau, g));
+        vz[g] = get16(block + off_vmeta(tau, g) + 2);
     }
 }
 

@@ -36,12 +36,16 @@
 
 namespace kvq {
 
-constexpr int DEC_CONSUMER_WARPS = 4;
-constexpr int DEC_THREADS = 32 * (DEC_CONSUMER_WARPS + 1);
-constexpr int STAGE_BLKS = 2 * DEC_CONSUMER_WARPS;        // 8 blocks = 128 tokens
+constexpr int DEC_WARPS = 4;                              // consumer warps; warp 0 lane 0 also issues copies
+constexpr int DEC_THREADS = 32 * DEC_WARPS;
+constexpr int SPLIT_MIN_CTAS = 4;                         // resident CTAs per SM
+constexpr int STAGE_BLKS = 2 * DEC_WARPS;                 // 8 blocks = 128 tokens
 constexpr int STAGE_BYTES = STAGE_BLKS * BLK_BYTES;       // 12 KB
 constexpr int NSTAGE = 4;
-constexpr int QP = 132;     // per (b, hq): q_s[128] then sum of q_s per group [4]
+// Prepared query per (b, query head), QP floats = 288 bytes:
+//   int8 hi[128], int8 lo[128]  with q_s ~= sq_g * (hi + lo/254) per group g
+//   float kap[4] = sq_g / 4^g,  float qsum[4] = sum of q_s over group g
+constexpr int QP = 72;
 constexpr int PART = 132;   // per partial: m, l, 0, 0, o[128]
 constexpr float LOG2E = 1.4426950408889634f;
 #define NEG_INF (__int_as_float(0xff800000))
@@ -72,92 +76,126 @@ __device__ __forceinline__ int unit_blocks(int L, int S, int capacity) {
 // ---------------------------------------------------------------------------------------------
 // Prologue.
 // ---------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) decode_prologue_kernel(DecodeArgs a) {
+constexpr int PRO_THREADS = 256;
+
+__global__ void __launch_bounds__(PRO_THREADS) decode_prologue_kernel(DecodeArgs a) {
     __shared__ __align__(16) float qs[D];
+    __shared__ __align__(16) float red[PRO_THREADS / 32][D];
     __shared__ float ssc[MAX_SINK];
+    __shared__ int scan[PRO_THREADS];
     const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int h = hq / a.G;
     const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
 
     if (blockIdx.x == 0 && blockIdx.y == 0) {
-        // prefix[b+1] = prefix[b] + Hkv * blocks(b): chunked scan, 128 threads
-        __shared__ int part[128];
-        const int per = (a.B + 127) / 128;
+        // prefix[b+1] = prefix[b] + Hkv * blocks(b): chunked scan
+        const int per = (a.B + PRO_THREADS - 1) / PRO_THREADS;
         int s = 0;
         for (int i = t * per; i < min(a.B, (t + 1) * per); i++)
             s += a.Hkv * unit_blocks(a.seq_lens[i], a.S, a.capacity);
-        part[t] = s;
+        scan[t] = s;
         __syncthreads();
         if (t == 0) {
             int acc = 0;
-            for (int i = 0; i < 128; i++) {
-                const int v = part[i];
-                part[i] = acc;
+            for (int i = 0; i < PRO_THREADS; i++) {
+                const int v = scan[i];
+                scan[i] = acc;
                 acc += v;
             }
         }
         __syncthreads();
-        int acc = part[t];
+        int acc = scan[t];
         for (int i = t * per; i < min(a.B, (t + 1) * per); i++) {
             a.prefix[i] = acc;
             const int L = a.seq_lens[i];
             if (L < 1 || L > a.capacity) set_status(a.status, KVQ_DEV_BAD_LEN);
             acc += a.Hkv * unit_blocks(L, a.S, a.capacity);
         }
-        if (t == 127) a.prefix[a.B] = acc;
-        __syncthreads();
+        if (t == PRO_THREADS - 1) a.prefix[a.B] = acc;
     }
 
     // q_rot in fp32, then scaled by log2(e)/sqrt(128) so scores are exp2 exponents
-    float qr;
     if (a.mode == KVQ_ROT_DENSE) {
-        __shared__ float qin[D];
-        qin[t] = __half2float(__ushort_as_half(q[t]));
-        __syncthreads();
-        const float *R = a.R_k + (size_t)h * D * D;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; i++) acc = fmaf(qin[i], R[i * D + t], acc);
-        qr = acc;
-        qs[t] = qr;
-    } else {
-        if (warp == 0) {
-            __shared__ uint16_t xq[D];
-            *reinterpret_cast<uint2 *>(&xq[4 * lane]) = *reinterpret_cast<const uint2 *>(q + 4 * lane);
-            const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
-            __syncwarp();
-            float v[4] = {__half2float(__ushort_as_half(xq[pi.x & (D - 1)])),
-                          __half2float(__ushort_as_half(xq[pi.y & (D - 1)])),
-                          __half2float(__ushort_as_half(xq[pi.z & (D - 1)])),
-                          __half2float(__ushort_as_half(xq[pi.w & (D - 1)]))};
-            fwht128_warp(v);
-            *reinterpret_cast<float4 *>(&qs[4 * lane]) =
-                make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
-                            v[2] * 0.08838834764831845f, v[3] * 0.08838834764831845f);
+        // warp w: rows 16w..16w+15 of R_k, lane l: columns 4l..4l+3; all 16
+        // row loads are issued before any is used
+        const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
+        float4 rr[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+        const uint4 u0 = *reinterpret_cast<const uint4 *>(q + 16 * warp);
+        const uint4 u1 = *reinterpret_cast<const uint4 *>(q + 16 * warp + 8);
+        const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int ii = 0; ii < 8; ii++) {
+            const float2 x2 = unpack_half2(w8[ii]);
+            const float4 ra = rr[2 * ii], rb = rr[2 * ii + 1];
+            acc.x = fmaf(x2.x, ra.x, acc.x); acc.y = fmaf(x2.x, ra.y, acc.y);
+            acc.z = fmaf(x2.x, ra.z, acc.z); acc.w = fmaf(x2.x, ra.w, acc.w);
+            acc.x = fmaf(x2.y, rb.x, acc.x); acc.y = fmaf(x2.y, rb.y, acc.y);
+            acc.z = fmaf(x2.y, rb.z, acc.z); acc.w = fmaf(x2.y, rb.w, acc.w);
         }
+        *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
+        __syncthreads();
+        if (t < D) {
+            float v = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < PRO_THREADS / 32; w2++) v += red[w2][t];
+            qs[t] = v;
+        }
+    } else if (warp == 0) {
+        __shared__ uint16_t xq[D];
+        *reinterpret_cast<uint2 *>(&xq[4 * lane]) = *reinterpret_cast<const uint2 *>(q + 4 * lane);
+        const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
+        __syncwarp();
+        float v[4] = {__half2float(__ushort_as_half(xq[pi.x & (D - 1)])),
+                      __half2float(__ushort_as_half(xq[pi.y & (D - 1)])),
+                      __half2float(__ushort_as_half(xq[pi.z & (D - 1)])),
+                      __half2float(__ushort_as_half(xq[pi.w & (D - 1)]))};
+        fwht128_warp(v);
+        *reinterpret_cast<float4 *>(&qs[4 * lane]) =
+            make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
+                        v[2] * 0.08838834764831845f, v[3] * 0.08838834764831845f);
     }
     __syncthreads();
     const float qscale = LOG2E * 0.08838834764831845f;
-    const float qv = qs[t] * qscale;
-    float *qp = a.qprep + ((size_t)b * a.Hq + hq) * QP;
-    qp[t] = qv;
-    float gs = qv;
+    float qv = 0.f;
+    if (t < D) {
+        // q_s = q_rot * log2(e)/sqrt(128); per group, an int8 hi/lo pair on
+        // the scale max|q_s|/127 (about 15 significant bits)
+        qv = qs[t] * qscale;
+        uint8_t *qp = reinterpret_cast<uint8_t *>(a.qprep + ((size_t)b * a.Hq + hq) * QP);
+        float gs = qv, amax = fabsf(qv);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, off);
-    if (lane == 0) qp[D + warp] = gs;
+        for (int off = 16; off > 0; off >>= 1) {
+            gs += __shfl_xor_sync(0xffffffffu, gs, off);
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        }
+        const float sq = amax > 0.f ? amax * (1.0f / 127.0f) : 1.0f;
+        const float u = qv / sq;
+        const float hi = fminf(fmaxf(rintf(u), -127.f), 127.f);
+        const float lo = fminf(fmaxf(rintf((u - hi) * 254.0f), -127.f), 127.f);
+        qp[t] = (uint8_t)(int8_t)hi;
+        qp[D + t] = (uint8_t)(int8_t)lo;
+        if (lane == 0) {
+            float *qf = reinterpret_cast<float *>(qp + 2 * D);
+            qf[warp] = sq * __int_as_float((127 - 2 * warp) << 23);   // sq / 4^g
+            qf[4 + warp] = gs;
+        }
+    }
 
     // sink partial (fp32, CUDA cores): at most MAX_SINK tokens
     if (a.S > 0) {
         __syncthreads();
-        qs[t] = qv;
+        if (t < D) qs[t] = qv;
         __syncthreads();
         const int L = a.seq_lens[b];
         const bool ok = (L >= 1 && L <= a.capacity);
         const int ns = ok ? min(a.S, L) : 0;
         const uint16_t *ks = a.k_sink + ((size_t)b * a.Hkv + h) * a.S * D;
         const uint16_t *vs = a.v_sink + ((size_t)b * a.Hkv + h) * a.S * D;
-        for (int tk = warp; tk < ns; tk += 4) {
+        for (int tk = warp; tk < ns; tk += PRO_THREADS / 32) {
             const uint2 u = *reinterpret_cast<const uint2 *>(ks + (size_t)tk * D + 4 * lane);
             const float2 k01 = unpack_half2(u.x), k23 = unpack_half2(u.y);
             float d = qs[4 * lane] * k01.x + qs[4 * lane + 1] * k01.y + qs[4 * lane + 2] * k23.x +
@@ -167,19 +205,21 @@ __global__ void __launch_bounds__(128) decode_prologue_kernel(DecodeArgs a) {
             if (lane == 0) ssc[tk] = d;
         }
         __syncthreads();
-        float m = NEG_INF;
-        for (int tk = 0; tk < ns; tk++) m = fmaxf(m, ssc[tk]);
-        float l = 0.f, o = 0.f;
-        for (int tk = 0; tk < ns; tk++) {
-            const float p = exp2f(ssc[tk] - m);
-            l += p;
-            o = fmaf(p, __half2float(__ushort_as_half(vs[(size_t)tk * D + t])), o);
-        }
-        float *sp = a.sinkp + ((size_t)b * a.Hq + hq) * PART;
-        sp[4 + t] = o;
-        if (t == 0) {
-            sp[0] = m;
-            sp[1] = l;
+        if (t < D) {
+            float m = NEG_INF;
+            for (int tk = 0; tk < ns; tk++) m = fmaxf(m, ssc[tk]);
+            float l = 0.f, o = 0.f;
+            for (int tk = 0; tk < ns; tk++) {
+                const float p = exp2f(ssc[tk] - m);
+                l += p;
+                o = fmaf(p, __half2float(__ushort_as_half(vs[(size_t)tk * D + t])), o);
+            }
+            float *sp = a.sinkp + ((size_t)b * a.Hq + hq) * PART;
+            sp[4 + t] = o;
+            if (t == 0) {
+                sp[0] = m;
+                sp[1] = l;
+            }
         }
     }
 }
@@ -268,24 +308,36 @@ __device__ __forceinline__ int kslot_elem(int kappa, int delta) {
     return 4 * ((kappa >> 1) & 3) + 16 * (kappa >> 3) + 2 * (kappa & 1) + delta;
 }
 
+// Which (group, head) the score-layout lane with quad index c turns into
+// P.V weights, for its k-th weight register (k < NW).
 template <int G>
-__global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs a) {
+__device__ __forceinline__ void wsrc(int c, int k, int &g, int &head) {
+    if (G == 1) { g = c; head = 0; }
+    else if (G == 2) { g = (c >> 1) + 2 * k; head = c & 1; }
+    else if (G == 4) { g = k; head = c; }
+    else { g = k & 3; head = c + 4 * (k >> 2); }
+}
+
+template <int G>
+__global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kernel(DecodeArgs a) {
     using C = Cfg<G>;
+    constexpr int NW = G;                              // weight registers per lane per block
+    constexpr int NGL = G == 1 ? 1 : (G == 2 ? 2 : 4); // V-meta groups a lane reads
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + NSTAGE * STAGE_BYTES);
-    uint64_t *empty = full + NSTAGE;
-    float *fo = reinterpret_cast<float *>(empty + NSTAGE);          // [4][G][128]
-    float *fm = fo + DEC_CONSUMER_WARPS * G * D;                     // [4][G]
-    float *fl = fm + DEC_CONSUMER_WARPS * G;                         // [4][G]
-    float *fz = fl + DEC_CONSUMER_WARPS * G;                         // [4][G][4]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(fz + DEC_CONSUMER_WARPS * G * 4);
+    int *cnt = reinterpret_cast<int *>(full + NSTAGE);               // [NSTAGE]
+    float *fo = reinterpret_cast<float *>(cnt + NSTAGE);              // [W][G][128]
+    float *fm = fo + DEC_WARPS * G * D;                              // [W][G]
+    float *fl = fm + DEC_WARPS * G;                                  // [W][G]
+    float *fz = fl + DEC_WARPS * G;                                  // [W][G][4]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(fz + DEC_WARPS * G * 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], DEC_CONSUMER_WARPS);
+            cnt[s] = 0;
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -294,41 +346,37 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
 
     Sched sc;
     if (!sched_init(sc, a)) return;
-
-    // ------------------------------------------------------------------ producer
-    if (warp == DEC_CONSUMER_WARPS) {
-        if (lane == 0) {
-            int it = 0;
-            const int fb = a.S / BLK_TOK;
-            while (sc.cur < sc.end) {
-                sched_fix_unit(sc, a);
-                const int n = min(min(STAGE_BLKS, sc.end - sc.cur), sc.ustart + sc.nb - sc.cur);
-                const int s = it % NSTAGE;
-                if (!mbar_wait_bounded(&empty[s], ((it / NSTAGE) & 1) ^ 1)) {
-                    set_status(a.status, KVQ_DEV_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                const size_t unit = (size_t)sc.b * a.Hkv + sc.h;
-                const uint8_t *src =
-                    a.blocks + (unit * a.nblk + fb + (sc.cur - sc.ustart)) * (size_t)BLK_BYTES;
-                mbar_arrive_expect_tx(&full[s], n * BLK_BYTES);
-                bulk_g2s(ring + s * STAGE_BYTES, src, n * BLK_BYTES, &full[s]);
-                sc.cur += n;
-                ++it;
-            }
-        }
-        return;
-    }
-
-    // ------------------------------------------------------------------ consumers
-    const int r = lane >> 2, c = lane & 3;
     const int fb = a.S / BLK_TOK;
+
+    // Copies: every warp's lane 0 runs the schedule NSTAGE stages ahead; the
+    // last warp to release a ring slot refills it.
+    Sched ps = sc;
+    int pit = 0;
+    auto next_copy = [&](bool do_issue) {
+        if (ps.cur >= ps.end) return;
+        sched_fix_unit(ps, a);
+        const int n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
+        if (do_issue) {
+            const int s = pit % NSTAGE;
+            const size_t unit = (size_t)ps.b * a.Hkv + ps.h;
+            const uint8_t *src =
+                a.blocks + (unit * a.nblk + fb + (ps.cur - ps.ustart)) * (size_t)BLK_BYTES;
+            mbar_arrive_expect_tx(&full[s], n * BLK_BYTES);
+            bulk_g2s(ring + s * STAGE_BYTES, src, n * BLK_BYTES, &full[s]);
+        }
+        ps.cur += n;
+        ++pit;
+    };
+    if (lane == 0)
+        for (int k = 0; k < NSTAGE; k++) next_copy(threadIdx.x == 0);
+
+    const int r = lane >> 2, c = lane & 3;
     // per-unit query operands
-    uint32_t qB[8][C::NTK_STEP][2];
-    float qsum[C::NTK], alpha[C::NTK];
+    uint32_t qB[4][C::NTK_STEP][2];
+    float qsum[C::NTK], kap[C::NTK], kap2[C::NTK];
+    int Lcur = 0;
     // online-softmax state
-    float m_run[G], l_run[C::HPL], O[8][4], Z[C::NTV];
+    float m_run[G], l_run[C::HPL], O[8][4], Z[NW];
     int cur_unit = -1;
 
     auto reset_state = [&]() {
@@ -341,50 +389,45 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
 #pragma unroll
             for (int k = 0; k < 4; k++) O[i][k] = 0.f;
 #pragma unroll
-        for (int i = 0; i < C::NTV; i++) Z[i] = 0.f;
+        for (int i = 0; i < NW; i++) Z[i] = 0.f;
     };
 
     auto load_unit = [&](int b, int h) {
-        const float *qbase = a.qprep + ((size_t)b * a.Hq + (size_t)h * G) * QP;
+        // B fragments of the K-side IMMA, one per group: column n of the N
+        // tile is (group, head, hi/lo); k = element e of the group
+        const uint8_t *qbase = reinterpret_cast<const uint8_t *>(
+            a.qprep + ((size_t)b * a.Hq + (size_t)h * G) * QP);
         const int n = lane >> 2;
 #pragma unroll
-        for (int s8 = 0; s8 < 8; s8++) {
-            const int g = s8 & 3, delta = s8 >> 2;
+        for (int g = 0; g < 4; g++) {
 #pragma unroll
             for (int j = 0; j < C::NTK_STEP; j++) {
                 const int nu = (g * 2 * G) / 8 + j;
                 const int col = 8 * nu + n;
                 const int gcol = col / (2 * G), head = (col % (2 * G)) / 2, hl = col & 1;
-                uint32_t bb[2] = {0u, 0u};
+                uint32_t b0 = 0u, b1 = 0u;
                 if (gcol == g) {
-                    const float *qh = qbase + (size_t)head * QP + 32 * g;
-#pragma unroll
-                    for (int part = 0; part < 2; part++) {
-                        float vv[2];
-#pragma unroll
-                        for (int e2 = 0; e2 < 2; e2++) {
-                            const float x = qh[kslot_elem(2 * c + 8 * part + e2, delta)];
-                            const __half hi = __float2half_rn(x);
-                            vv[e2] = hl == 0 ? __half2float(hi)
-                                             : __half2float(__float2half_rn(x - __half2float(hi)));
-                        }
-                        bb[part] = pack_half2(vv[0], vv[1]);
-                    }
+                    const uint8_t *qh = qbase + (size_t)head * QP * 4 + hl * D + 32 * g;
+                    b0 = *reinterpret_cast<const uint32_t *>(qh + 4 * c);
+                    b1 = *reinterpret_cast<const uint32_t *>(qh + 16 + 4 * c);
                 }
-                qB[s8][j][0] = bb[0];
-                qB[s8][j][1] = bb[1];
+                qB[g][j][0] = b0;
+                qB[g][j][1] = b1;
             }
         }
 #pragma unroll
         for (int nu = 0; nu < C::NTK; nu++) {
             const int g = ktile_group<G>(nu, c), head = ktile_head<G>(nu, c);
-            qsum[nu] = qbase[(size_t)head * QP + D + g];
-            alpha[nu] = __int_as_float((127 + 24 - 2 * g) << 23);   // 2^24 / 4^g
+            const float *qf = reinterpret_cast<const float *>(qbase + (size_t)head * QP * 4 + 2 * D);
+            kap[nu] = qf[g];
+            kap2[nu] = qf[g] * (1.0f / 254.0f);
+            qsum[nu] = qf[4 + g];
         }
+        Lcur = a.seq_lens[b];
     };
 
     auto flush = [&](int slot) {
-        // reduce l over the 8 row lanes, Z over the 4 column lanes
+        // reduce l and Z over the 8 row lanes
 #pragma unroll
         for (int i = 0; i < C::HPL; i++) {
             l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
@@ -392,9 +435,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
             l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
         }
 #pragma unroll
-        for (int i = 0; i < C::NTV; i++) {
-            Z[i] += __shfl_xor_sync(0xffffffffu, Z[i], 1);
-            Z[i] += __shfl_xor_sync(0xffffffffu, Z[i], 2);
+        for (int i = 0; i < NW; i++) {
+            Z[i] += __shfl_xor_sync(0xffffffffu, Z[i], 4);
+            Z[i] += __shfl_xor_sync(0xffffffffu, Z[i], 8);
+            Z[i] += __shfl_xor_sync(0xffffffffu, Z[i], 16);
         }
         float *wo = fo + warp * G * D;
         if (lane == 0)
@@ -406,12 +450,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
                 const int head = lane_head<G>(lane, hh);
                 if (G == 1 ? lane == 0 : (G == 2 ? lane < 2 : true)) fl[warp * G + head] = l_run[hh];
             }
-        }
-        if (c == 0) {
 #pragma unroll
-            for (int i = 0; i < C::NTV; i++) {
-                const int col = 8 * i + (lane >> 2);
-                if (col < 4 * G) fz[(warp * G + col % G) * 4 + col / G] = Z[i];
+            for (int k = 0; k < NW; k++) {
+                int g, head;
+                wsrc<G>(lane, k, g, head);
+                fz[(warp * G + head) * 4 + g] = Z[k];
             }
         }
 #pragma unroll
@@ -428,15 +471,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
                         wo[head * D + j] = O[g * 2 + h2][k] * __int_as_float((127 + 24 - 2 * g) << 23);
                     }
                 }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * DEC_CONSUMER_WARPS));
+        __syncthreads();
         const int tj = threadIdx.x;   // 0..127: element
         for (int head = 0; head < G; head++) {
             float ms = NEG_INF;
 #pragma unroll
-            for (int w = 0; w < DEC_CONSUMER_WARPS; w++) ms = fmaxf(ms, fm[w * G + head]);
+            for (int w = 0; w < DEC_WARPS; w++) ms = fmaxf(ms, fm[w * G + head]);
             float acc = 0.f, lsum = 0.f;
 #pragma unroll
-            for (int w = 0; w < DEC_CONSUMER_WARPS; w++) {
+            for (int w = 0; w < DEC_WARPS; w++) {
                 const float mw = fm[w * G + head];
                 const float f = (mw == NEG_INF) ? 0.f : exp2f(mw - ms);
                 acc = fmaf(f, fo[(w * G + head) * D + tj] + fz[(w * G + head) * 4 + (tj >> 5)], acc);
@@ -449,7 +492,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
                 dst[1] = lsum;
             }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * DEC_CONSUMER_WARPS));
+        __syncthreads();
     };
 
     reset_state();
@@ -462,7 +505,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
             cur_unit = unit;
         }
         const int n = min(min(STAGE_BLKS, sc.end - sc.cur), sc.ustart + sc.nb - sc.cur);
-        const int L = a.seq_lens[sc.b];
         const int s = it % NSTAGE;
         const bool ok = mbar_wait_bounded(&full[s], (it / NSTAGE) & 1);
         if (!ok || *abort_flag) {
@@ -471,41 +513,44 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
             break;
         }
         const int nmine = min(2, max(0, n - 2 * warp));
-        float P[2][2][C::HPL];
-        float sco[2][2][C::HPL];
-        // ---- scores for my (up to) two blocks
+        if (nmine > 0) {
+            const uint8_t *blk0 = ring + s * STAGE_BYTES + (2 * warp) * BLK_BYTES;
+            const int tok0 = (fb + (sc.cur - sc.ustart) + 2 * warp) * BLK_TOK;   // first position
+            // a block needs masking if it is a phantom or crosses [S, L)
+            bool edge[2];
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++) {
+            for (int bi = 0; bi < 2; bi++)
+                edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
+            // ---- scores for both blocks (the second may be a phantom)
+            uint4 kq[2];
 #pragma unroll
-            for (int st = 0; st < 2; st++)
+            for (int bi = 0; bi < 2; bi++)
+                kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
+            int dk[2][C::NTK][4];
 #pragma unroll
-                for (int hh = 0; hh < C::HPL; hh++) sco[bi][st][hh] = NEG_INF;
-            if (bi < nmine) {
-                const uint8_t *blk = ring + s * STAGE_BYTES + (2 * warp + bi) * BLK_BYTES;
-                const uint4 kq = *reinterpret_cast<const uint4 *>(blk + 16 * (4 * r + c));
-                float dk[C::NTK][4];
+            for (int bi = 0; bi < 2; bi++)
 #pragma unroll
                 for (int nu = 0; nu < C::NTK; nu++)
 #pragma unroll
-                    for (int k = 0; k < 4; k++) dk[nu][k] = 0.f;
+                    for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
+            // one IMMA per group: the masked bytes are u8 codes c * 4^g
 #pragma unroll
-                for (int s8 = 0; s8 < 8; s8++) {
-                    const int g = s8 & 3;
-                    const uint32_t msk = 0x00030003u << (2 * g);
-                    uint32_t a0, a1, a2, a3;
-                    if (s8 < 4) {
-                        a0 = kq.x & msk; a1 = kq.z & msk; a2 = kq.y & msk; a3 = kq.w & msk;
-                    } else {
-                        a0 = (kq.x >> 8) & msk; a1 = (kq.z >> 8) & msk;
-                        a2 = (kq.y >> 8) & msk; a3 = (kq.w >> 8) & msk;
-                    }
+            for (int g = 0; g < 4; g++) {
+                const uint32_t msk = 0x03030303u << (2 * g);
+#pragma unroll
+                for (int bi = 0; bi < 2; bi++) {
+                    const uint4 q4 = kq[bi];
 #pragma unroll
                     for (int j = 0; j < C::NTK_STEP; j++) {
                         const int nu = (g * 2 * G) / 8 + j;
-                        mma16816(dk[nu], a0, a1, a2, a3, qB[s8][j][0], qB[s8][j][1]);
+                        imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
+                                  qB[g][j][0], qB[g][j][1]);
                     }
                 }
-                // combine groups: s = sum_g sc*(hi+lo)*2^24/4^g + z*sum(q_g)
+            }
+            float sco[2][2][C::HPL];
+#pragma unroll
+            for (int bi = 0; bi < 2; bi++) {
                 float part_sc[2][C::HPL];
 #pragma unroll
                 for (int st = 0; st < 2; st++)
@@ -514,11 +559,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int nu = 0; nu < C::NTK; nu++) {
                     const int g = ktile_group<G>(nu, c);
-                    const uint2 mk = *reinterpret_cast<const uint2 *>(blk + OFF_KM + 8 * (4 * r + g));
+                    const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
+                                                                      8 * (4 * r + g));
                     const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
                     const int hh = ktile_slot<G>(nu);
-                    part_sc[0][hh] += sz0.x * ((dk[nu][0] + dk[nu][1]) * alpha[nu]) + sz0.y * qsum[nu];
-                    part_sc[1][hh] += sz1.x * ((dk[nu][2] + dk[nu][3]) * alpha[nu]) + sz1.y * qsum[nu];
+                    const float d0 = fmaf(__int2float_rn(dk[bi][nu][1]), kap2[nu],
+                                          __int2float_rn(dk[bi][nu][0]) * kap[nu]);
+                    const float d1 = fmaf(__int2float_rn(dk[bi][nu][3]), kap2[nu],
+                                          __int2float_rn(dk[bi][nu][2]) * kap[nu]);
+                    part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
+                    part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
                 }
 #pragma unroll
                 for (int st = 0; st < 2; st++)
@@ -531,13 +581,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
                         } else if (G == 2) {
                             v += __shfl_xor_sync(0xffffffffu, v, 2);
                         }
-                        const int pos = (fb + (sc.cur - sc.ustart) + 2 * warp + bi) * BLK_TOK + r + 8 * st;
-                        sco[bi][st][hh] = (pos >= a.S && pos < L) ? v : NEG_INF;
+                        if (edge[bi]) {
+                            const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
+                            v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
+                        }
+                        sco[bi][st][hh] = v;
                     }
             }
-        }
-        // ---- online softmax update (all lanes of the warp take the same branch)
-        if (nmine > 0) {
+            // ---- online softmax update (the branch is uniform over the warp)
             float mt[C::HPL];
 #pragma unroll
             for (int hh = 0; hh < C::HPL; hh++) {
@@ -551,7 +602,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
             bool grow = false;
 #pragma unroll
             for (int hd = 0; hd < G; hd++) {
-                // owner lane (quad index) of head hd in the score layout
                 const int owner = G == 1 ? 0 : (G == 2 ? (hd & 1) : (hd & 3));
                 const float tmx = __shfl_sync(0xffffffffu, mt[G >= 8 ? (hd >> 2) : 0], owner);
                 mnew[hd] = fmaxf(m_run[hd], tmx);
@@ -567,27 +617,22 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
 #pragma unroll
-                for (int i = 0; i < C::NTV; i++) {
-                    const int col = 8 * i + (lane >> 2);
-                    float f = 1.f;
-#pragma unroll
-                    for (int hd = 0; hd < G; hd++)
-                        if (col % G == hd) f = al[hd];
-                    Z[i] *= f;
+                for (int k = 0; k < NW; k++) {
+                    int g, head;
+                    wsrc<G>(c, k, g, head);
+                    Z[k] *= pick<G>(al, head);
                 }
 #pragma unroll
                 for (int g = 0; g < 4; g++)
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         const int col = 8 * ((g * G) / 8) + 2 * c + (k & 1);
-                        float f = 1.f;
-#pragma unroll
-                        for (int hd = 0; hd < G; hd++)
-                            if (col % G == hd) f = al[hd];
+                        const float f = pick<G>(al, col % G);
                         O[2 * g][k] *= f;
                         O[2 * g + 1][k] *= f;
                     }
             }
+            float P[2][2][C::HPL];
 #pragma unroll
             for (int bi = 0; bi < 2; bi++)
 #pragma unroll
@@ -596,62 +641,99 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
                     for (int hh = 0; hh < C::HPL; hh++) {
                         const float v = sco[bi][st][hh];
                         const float mm = pick<G>(m_run, lane_head<G>(c, hh));
-                        const float p = (v == NEG_INF) ? 0.f : exp2f(v - mm);
+                        const float p = (edge[bi] && v == NEG_INF) ? 0.f : exp2f(v - mm);
                         P[bi][st][hh] = p;
                         l_run[hh] += p;
                     }
-            // ---- P.V for my blocks
+            // ---- P.V
 #pragma unroll
             for (int bi = 0; bi < 2; bi++) {
-                if (bi < nmine) {
-                    const uint8_t *blk = ring + s * STAGE_BYTES + (2 * warp + bi) * BLK_BYTES;
-                    uint32_t Bv[C::NTV][2];
+                const uint8_t *blk = blk0 + bi * BLK_BYTES;
+                // weights w = p * s_v in the score layout, as half2 (token r, token r+8)
+                uint32_t H[NW];
+                {
+                    float2 sz[NGL][2];
 #pragma unroll
-                    for (int i = 0; i < C::NTV; i++) {
-                        const int col = 8 * i + (lane >> 2);
-                        const bool valid = col < 4 * G;
-                        const int gv = valid ? col / G : 0;
-                        const int hv = col % G;
-                        const int owner = G == 1 ? c : (G == 2 ? (hv & 1) : (hv & 3));
-                        const int src0 = 4 * (2 * c) + owner, src1 = 4 * (2 * c + 1) + owner;
-                        float pp[4];
-#pragma unroll
-                        for (int hh = 0; hh < C::HPL; hh++) {
-                            const float q0 = __shfl_sync(0xffffffffu, P[bi][0][hh], src0);
-                            const float q1 = __shfl_sync(0xffffffffu, P[bi][0][hh], src1);
-                            const float q2 = __shfl_sync(0xffffffffu, P[bi][1][hh], src0);
-                            const float q3 = __shfl_sync(0xffffffffu, P[bi][1][hh], src1);
-                            if (hh == 0 || (hv >> 2) == hh) {
-                                pp[0] = q0; pp[1] = q1; pp[2] = q2; pp[3] = q3;
-                            }
-                        }
-                        const uint2 vsc = *reinterpret_cast<const uint2 *>(blk + OFF_VS + 8 * (4 * c + gv));
-                        const uint2 vzr = *reinterpret_cast<const uint2 *>(blk + OFF_VZ + 8 * (4 * c + gv));
-                        const float2 s01 = unpack_half2(vsc.x), s23 = unpack_half2(vsc.y);
-                        const float2 z01 = unpack_half2(vzr.x), z23 = unpack_half2(vzr.y);
-                        Bv[i][0] = valid ? pack_half2(pp[0] * s01.x, pp[1] * s01.y) : 0u;
-                        Bv[i][1] = valid ? pack_half2(pp[2] * s23.x, pp[3] * s23.y) : 0u;
-                        if (valid)
-                            Z[i] += pp[0] * z01.x + pp[1] * z01.y + pp[2] * z23.x + pp[3] * z23.y;
+                    for (int gl = 0; gl < NGL; gl++) {
+                        const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
+                        const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
+                        sz[gl][0] = unpack_half2(mv.x);
+                        sz[gl][1] = unpack_half2(mv.y);
                     }
-                    const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
-                    const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
 #pragma unroll
-                    for (int g = 0; g < 4; g++) {
-                        const uint32_t msk = 0x00030003u << (2 * g);
-                        const int nv = (g * G) / 8;
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; h2++) {
-                            const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
-                            mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk,
-                                     (w2 >> 8) & msk, Bv[nv][0], Bv[nv][1]);
+                    for (int k = 0; k < NW; k++) {
+                        const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
+                        const int hh = G >= 8 ? (k >> 2) : 0;
+                        const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
+                        float w0 = p0 * sz[gl][0].x, w1 = p1 * sz[gl][1].x;
+                        float z0 = p0 * sz[gl][0].y, z1 = p1 * sz[gl][1].y;
+                        if (edge[bi]) {      // masked tokens: never touch their metadata
+                            w0 = p0 == 0.f ? 0.f : w0; z0 = p0 == 0.f ? 0.f : z0;
+                            w1 = p1 == 0.f ? 0.f : w1; z1 = p1 == 0.f ? 0.f : z1;
                         }
+                        H[k] = pack_half2(w0, w1);
+                        Z[k] += z0 + z1;
+                    }
+                }
+                // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
+                // its column (group, head)
+                uint32_t Bv[C::NTV][2];
+#pragma unroll
+                for (int i = 0; i < C::NTV; i++) {
+                    const int col = 8 * i + (lane >> 2);
+                    const bool valid = col < 4 * G;
+                    const int g = col / G, head = col % G;
+                    int csrc, ksel;
+                    if (G == 1) { csrc = g; ksel = 0; }
+                    else if (G == 2) { csrc = head + 2 * (g & 1); ksel = g >> 1; }
+                    else if (G == 4) { csrc = head; ksel = g & 1; }
+                    else { csrc = head & 3; ksel = head >> 2; }
+                    const int src0 = 4 * (2 * c) + csrc, src1 = src0 + 4;
+                    uint32_t X, Y;
+                    if (G == 1) {
+                        X = __shfl_sync(0xffffffffu, H[0], src0);
+                        Y = __shfl_sync(0xffffffffu, H[0], src1);
+                    } else {
+                        // two candidate registers; the lane keeps the one it needs
+                        const int k0 = G == 2 ? 0 : (G == 4 ? 2 * i : i);
+                        const int k1 = G == 2 ? 1 : (G == 4 ? 2 * i + 1 : 4 + i);
+                        const uint32_t X0 = __shfl_sync(0xffffffffu, H[k0], src0);
+                        const uint32_t Y0 = __shfl_sync(0xffffffffu, H[k0], src1);
+                        const uint32_t X1 = __shfl_sync(0xffffffffu, H[k1], src0);
+                        const uint32_t Y1 = __shfl_sync(0xffffffffu, H[k1], src1);
+                        X = ksel ? X1 : X0;
+                        Y = ksel ? Y1 : Y0;
+                    }
+                    Bv[i][0] = valid ? __byte_perm(X, Y, 0x5410) : 0u;
+                    Bv[i][1] = valid ? __byte_perm(X, Y, 0x7632) : 0u;
+                }
+                const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
+                const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+                for (int g = 0; g < 4; g++) {
+                    const uint32_t msk = 0x00030003u << (2 * g);
+                    const int nv = (g * G) / 8;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
+                        mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk, (w2 >> 8) & msk,
+                                 Bv[nv][0], Bv[nv][1]);
                     }
                 }
             }
         }
+        // release the slot; the last warp out refills it
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0) {
+            __threadfence_block();
+            const int old = atomicAdd(&cnt[s], 1);
+            const bool last = (old % DEC_WARPS) == DEC_WARPS - 1;
+            if (last) {
+                __threadfence_block();
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            next_copy(last);
+        }
         sc.cur += n;
         ++it;
         // end of this CTA's segment of the unit: write the partial
@@ -665,15 +747,20 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) decode_split_kernel(DecodeArgs
 // ---------------------------------------------------------------------------------------------
 // Merge + rotate-out.
 // ---------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
+constexpr int MRG_THREADS = 256;
+constexpr int MRG_MAXP = 512;     // partials merged per pass
+
+__global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a) {
     __shared__ __align__(16) float o_s[D];
+    __shared__ __align__(16) float red[MRG_THREADS / 32][D];
+    __shared__ float pm[MRG_MAXP + 1], pl[MRG_MAXP + 1], wred[MRG_THREADS / 32];
     const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int G = a.G, h = hq / G, head = hq % G;
     uint16_t *out = a.out + ((size_t)b * a.Hq + hq) * D;
     const int L = a.seq_lens[b];
     if (L < 1 || L > a.capacity) {
-        out[t] = 0;
+        if (t < D) out[t] = 0;
         return;
     }
     const int u = b * a.Hkv + h;
@@ -681,41 +768,77 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
     const int N = a.prefix[a.B];
     const int W = max(1, (N + a.C - 1) / a.C);
     const int ustart = a.prefix[b] + h * nb;
-    int c0 = 0, c1 = -1;
-    if (nb > 0) {
-        c0 = ustart / W;
-        c1 = (ustart + nb - 1) / W;
-    }
+    const int c0 = nb > 0 ? ustart / W : 0;
+    const int np = nb > 0 ? (ustart + nb - 1) / W - c0 + 1 : 0;
     const float *sp = a.sinkp + ((size_t)b * a.Hq + hq) * PART;
-    const bool has_sink = a.S > 0;
-    float ms = has_sink ? sp[0] : NEG_INF;
-    for (int cc = c0; cc <= c1; cc++)
-        ms = fmaxf(ms, a.part[((size_t)(cc + u) * G + head) * PART]);
-    float acc = 0.f, lsum = 0.f;
-    if (has_sink && sp[0] != NEG_INF) {
-        const float f = exp2f(sp[0] - ms);
-        acc = f * sp[4 + t];
-        lsum = f * sp[1];
+    auto pptr = [&](int i) -> const float * {   // partial i (i == np: the sink partial)
+        return i < np ? a.part + ((size_t)(c0 + i + u) * G + head) * PART : sp;
+    };
+    const int ntot = np + (a.S > 0 ? 1 : 0);
+
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f, mglob = NEG_INF;
+    for (int base = 0; base < ntot; base += MRG_MAXP) {
+        const int n = min(MRG_MAXP, ntot - base);
+        // (m, l) of every partial, then the running max
+        float mloc = NEG_INF;
+        for (int i = t; i < n; i += MRG_THREADS) {
+            const float *pp = pptr(base + i);
+            pm[i] = pp[0];
+            pl[i] = pp[1];
+            mloc = fmaxf(mloc, pp[0]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+        if (lane == 0) wred[warp] = mloc;
+        __syncthreads();
+        float mnew = mglob;
+#pragma unroll
+        for (int w2 = 0; w2 < MRG_THREADS / 32; w2++) mnew = fmaxf(mnew, wred[w2]);
+        const float fold = (mglob == NEG_INF) ? 0.f : exp2f(mglob - mnew);
+        acc.x *= fold; acc.y *= fold; acc.z *= fold; acc.w *= fold;
+        lsum *= fold;
+        mglob = mnew;
+        // o: warp w sums partials w, w+8, ...; lane l holds elements 4l..4l+3
+        for (int i = warp; i < n; i += MRG_THREADS / 32) {
+            const float mi = pm[i];
+            const float f = (mi == NEG_INF) ? 0.f : exp2f(mi - mglob);
+            const float4 o4 = *reinterpret_cast<const float4 *>(pptr(base + i) + 4 + 4 * lane);
+            acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
+            acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
+            lsum = fmaf(f, pl[i], lsum);
+        }
+        __syncthreads();
     }
-    for (int cc = c0; cc <= c1; cc++) {
-        const float *pp = a.part + ((size_t)(cc + u) * G + head) * PART;
-        const float f = exp2f(pp[0] - ms);
-        acc = fmaf(f, pp[4 + t], acc);
-        lsum = fmaf(f, pp[1], lsum);
+    *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
+    if (lane == 0) wred[warp] = lsum;
+    __syncthreads();
+    if (t < D) {
+        float v = 0.f, l = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < MRG_THREADS / 32; w2++) {
+            v += red[w2][t];
+            l += wred[w2];
+        }
+        o_s[t] = v / l;
     }
-    o_s[t] = acc / lsum;
     __syncthreads();
     if (a.mode == KVQ_ROT_DENSE) {
-        // out[i] = sum_j o[j] * R_v[h][i][j]: one warp per row, lanes over j
-        const float *R = a.R_v + (size_t)h * D * D;
+        // out[i] = sum_j o[j] R_v[h][i][j]: warp w rows 16w..16w+15, lanes over j
+        const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
+        float4 rr[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
         const float4 o4 = *reinterpret_cast<const float4 *>(&o_s[4 * lane]);
-        for (int i = warp; i < D; i += 4) {
-            const float4 r4 = *reinterpret_cast<const float4 *>(R + (size_t)i * D + 4 * lane);
-            float d = o4.x * r4.x + o4.y * r4.y + o4.z * r4.z + o4.w * r4.w;
+        float mine = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < 16; ii++) {
+            float d = o4.x * rr[ii].x + o4.y * rr[ii].y + o4.z * rr[ii].z + o4.w * rr[ii].w;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            if (lane == 0) out[i] = __half_as_ushort(__float2half_rn(d));
+            if (lane == ii) mine = d;
         }
+        if (lane < 16) out[16 * warp + lane] = __half_as_ushort(__float2half_rn(mine));
     } else if (warp == 0) {
         float v[4] = {o_s[4 * lane], o_s[4 * lane + 1], o_s[4 * lane + 2], o_s[4 * lane + 3]};
         fwht128_warp(v);
@@ -731,9 +854,8 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
 // Host side.
 // ---------------------------------------------------------------------------------------------
 size_t split_smem_bytes(int G) {
-    return (size_t)NSTAGE * STAGE_BYTES + 2 * NSTAGE * sizeof(uint64_t) +
-           sizeof(float) * (DEC_CONSUMER_WARPS * G * D + 2 * DEC_CONSUMER_WARPS * G +
-                            DEC_CONSUMER_WARPS * G * 4) +
+    return (size_t)NSTAGE * STAGE_BYTES + NSTAGE * (sizeof(uint64_t) + sizeof(int)) +
+           sizeof(float) * (DEC_WARPS * G * D + 2 * DEC_WARPS * G + DEC_WARPS * G * 4) +
            16;
 }
 
@@ -789,7 +911,7 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.nblk = cd.capacity / BLK_TOK;
     a.mode = mode;
     a.C = C;
-    decode_prologue_kernel<<<dim3(Hq, cd.B), 128, 0, st>>>(a);
+    decode_prologue_kernel<<<dim3(Hq, cd.B), PRO_THREADS, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     switch (a.G) {
@@ -800,7 +922,7 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<dim3(Hq, cd.B), 128, 0, st>>>(a);
+    decode_merge_kernel<<<dim3(Hq, cd.B), MRG_THREADS, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -15,7 +15,7 @@ constexpr int GS = 32;          // quantization group (elements of head_dim)
 constexpr int NG = D / GS;      // groups per row
 constexpr int BLK_TOK = 16;     // tokens per cache block
 constexpr int BLK_BYTES = 1536; // bytes per cache block (96 per token)
-constexpr int OFF_VC = 512, OFF_KM = 1024, OFF_VS = 1280, OFF_VZ = 1408;
+constexpr int OFF_VC = 512, OFF_KM = 1024, OFF_VM = 1280;
 constexpr int MAX_SINK = 64;
 
 // ---- cache block offsets (format documented in include/kvq.h) ---------------------
@@ -33,9 +33,9 @@ __device__ __forceinline__ int off_kmeta(int tau, int g) {
     const int r = tau & 7, th = tau >> 3;
     return OFF_KM + 8 * (4 * r + g) + 4 * th;
 }
-__device__ __forceinline__ int off_vscale(int tau, int g) {
-    const int q = tau >> 1, side = tau & 1;
-    return OFF_VS + 8 * (4 * (q & 3) + g) + 4 * (q >> 2) + 2 * side;
+__device__ __forceinline__ int off_vmeta(int tau, int g) {
+    const int r = tau & 7, th = tau >> 3;
+    return OFF_VM + 8 * (4 * r + g) + 4 * th;
 }
 
 __device__ __forceinline__ void set_status(int32_t *status, int bits) {
@@ -108,13 +108,8 @@ __device__ __forceinline__ void store_token_warp(uint8_t *block, int tau, int ki
     }
     if ((lane & 7) == 0) {
         const int g = lane >> 3;
-        if (kind == 0) {
-            *reinterpret_cast<uint32_t *>(block + off_kmeta(tau, g)) =
-                (uint32_t)q.s | ((uint32_t)q.z << 16);
-        } else {
-            *reinterpret_cast<uint16_t *>(block + off_vscale(tau, g)) = q.s;
-            *reinterpret_cast<uint16_t *>(block + off_vscale(tau, g) + 128) = q.z;
-        }
+        *reinterpret_cast<uint32_t *>(block + (kind == 0 ? off_kmeta(tau, g) : off_vmeta(tau, g))) =
+            (uint32_t)q.s | ((uint32_t)q.z << 16);
     }
 }
 
@@ -173,20 +168,23 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
+    // The suspend-time hint lets the waiting thread sleep in hardware until
+    // the phase completes (or ~20 us pass) instead of spinning on the issue
+    // slots its SM-subpartition shares with working warps.
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls (each try_wait may itself
-// suspend for a while) and reports false.
+// Bounded wait: gives up after `limit` polls (each may suspend up to the
+// hint above, so the bound is about two seconds) and reports false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  uint32_t limit = (1u << 22)) {
+                                                  uint32_t limit = (1u << 17)) {
     for (uint32_t i = 0; i < limit; i++)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
@@ -210,6 +208,16 @@ __device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, u
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// m16n8k32 integer MMA: u8 A (codes) x s8 B (quantised query), s32 accumulate.
+__device__ __forceinline__ void imma16832(int d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 

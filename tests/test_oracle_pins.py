@@ -270,8 +270,7 @@ def test_block_layout_worked_offsets():
         vs[c["g"]], vz[c["g"]] = 0x1111, 0x2222
         z32, z4 = np.zeros(32, np.uint8), np.zeros(4, np.uint16)
         orc.store_token(block, c["tau"], z32, z32, z4, z4, vs, vz)
-        assert list(block[c["offset"]:c["offset"] + 2]) == [0x11, 0x11]
-        assert list(block[c["offset"] + 128:c["offset"] + 130]) == [0x22, 0x22]
+        assert list(block[c["offset"]:c["offset"] + 4]) == [0x11, 0x11, 0x22, 0x22]
 
 
 # --- append / decode ----------------------------------------------------------------------------
