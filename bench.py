@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated INT2 KV-cache hot path on B200.
+
+One step = rotate-quantize-append of the step's new token(s) + decode
+attention of one query per head over the packed cache (the whole hot path),
+on the "llama7b" workload by default: B=1, 32 heads (MHA), head_dim 128,
+context 32768 (32767 prefilled + 1 appended per step), dense per-head
+rotations, INT2 group 32 with fp16 scale/zero.  Inputs are seeded synthetic
+tensors (workloads.py).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle as reference arm
+    torchrun --nproc-per-node N bench.py --gpus N ...
+
+Timing: every step is bracketed by CUDA events on the launching stream; an
+L2 flush (256 MB write) and the reset of the sequence length to its
+pre-append value happen between steps, outside the events, so each step
+starts cold and at the same context.  K steps run back to back between a
+barrier + synchronize on both sides; the device time is summed per rank and
+the max over ranks is reported.  With N GPUs every rank serves its own
+independent batch (weak scaling, no collective on the data path).
+
+Prints one JSON line (rank 0).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "INT2-KV decode attention tokens/s and packed-KV GB/s (% of HBM peak), 1 B200"
+KERNELS_PER_STEP = 5      # append, length bump, decode prologue, split, merge
+FLUSH_BYTES = 256 << 20
+
+
+# --- distributed plumbing (also exercised by tests/test_bench_dist.py on CPU) ----------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend, world):
+    if world <= 1:
+        return False
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return True
+
+
+def barrier(enabled, device=None):
+    if enabled:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x, enabled, device):
+    """Max of a float over all ranks (identity when not distributed)."""
+    if not enabled:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w, rank):
+    """Each rank serves its own batch: same shapes, its own seed."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+# --- clocks -------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+               0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
+               0x200: "display_clock_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self.stop_flag = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of numbers
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_flag.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --- helpers ------------------------------------------------------------------------------------
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("kvq_decode.cu", "kvq_internal.cuh"):
+        with open(os.path.join(ROOT, "rotated_int2_kv_head_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """dram bytes per launch of the split kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_split_%s.txt" % workload)
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256") != kernel_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def packed_kv_bytes(w, lens):
+    """Algorithmic cache bytes one decode reads: 96 per token-head (codes 64,
+    scale/zero 32), 512 per fp16 sink token-head."""
+    tot = 0
+    for L in lens:
+        s = min(w.sink, int(L))
+        tot += w.Hkv * ((int(L) - s) * 96 + s * 512)
+    return tot
+
+
+# --- the CUDA arm ---------------------------------------------------------------------------------
+
+class Step:
+    """One pass of the hot path: append the new tokens, decode."""
+
+    def __init__(self, w, device, seed_rank=0):
+        import rotated_int2_kv_head_b200 as kvq
+        self.kvq, self.w, self.dev = kvq, w, device
+        lens = w.seq_lens()
+        self.L = int(lens.max())
+        self.T = w.append_T
+        self.cap = ((self.L + 15) // 16) * 16
+        Rk, Rv, perm = W.rotations(w)
+        self.Rk = torch.from_numpy(Rk).to(device) if Rk is not None else None
+        self.Rv = torch.from_numpy(Rv).to(device) if Rv is not None else None
+        self.perm = torch.from_numpy(perm).to(device) if perm is not None else None
+        self.rot_np = (Rk, Rv, perm)
+        self.cache = kvq.KVCache(w.B, w.Hkv, self.cap, w.sink, device=device)
+        self.len_full = torch.from_numpy(lens.astype(np.int32)).to(device)
+        self.len_base = self.len_full - self.T           # before the step's append
+        self.seq_lens = self.len_base.clone()
+        # prefill [0, L - T) on the GPU, in chunks, all sequences together
+        pre = self.L - self.T
+        fill = torch.zeros(w.B, dtype=torch.int32, device=device)
+        ch = 2048
+        for t0 in range(0, pre, ch):
+            t1 = min(pre, t0 + ch)
+            K, V = W.kv_batch(w, t0, t1, device)
+            kvq.kvq_rotate_quantize_append(K, V, w.mode, self.Rk, self.Rv, self.perm, self.cache,
+                                           fill)
+        self.Knew, self.Vnew = W.kv_batch(w, pre, self.L, device)
+        self.Q = W.queries(w, device)
+        self.out = torch.empty_like(self.Q)
+        self.ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, self.L, device=device)
+        torch.cuda.synchronize(device)
+        st = kvq.kvq_get_status(self.cache)
+        if st != 0:
+            raise RuntimeError("cache fill flagged device status %d" % st)
+        self.ev_split = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        for e in self.ev_split:
+            e.record()
+
+    def reset(self):
+        self.seq_lens.copy_(self.len_base)
+
+    def run(self, timed_split=False):
+        kvq, w = self.kvq, self.w
+        kvq.kvq_rotate_quantize_append(self.Knew, self.Vnew, w.mode, self.Rk, self.Rv, self.perm,
+                                       self.cache, self.seq_lens)
+        if timed_split:
+            kvq.kvq_decode_attention_timed(self.Q, self.cache, w.mode, self.Rk, self.Rv, self.perm,
+                                           self.seq_lens, w.sink, self.L, self.ws, self.out,
+                                           self.ev_split[0], self.ev_split[1])
+        else:
+            kvq.kvq_decode_attention(self.Q, self.cache, w.mode, self.Rk, self.Rv, self.perm,
+                                     self.seq_lens, w.sink, self.L, self.ws, self.out)
+
+
+def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload:
+    the first `heads` KV heads of sequence 0 (their K/V rows are the very
+    tensors the GPU arm used), timed for append + decode, scaled to the
+    whole step."""
+    from oracle import oracle as orc
+    heads = min(heads, w.Hkv)
+    pre = step.L - step.T
+    Rk, Rv, perm = step.rot_np
+    rk = Rk[:heads] if Rk is not None else None
+    rv = Rv[:heads] if Rv is not None else None
+    pm = perm[:, :heads] if perm is not None else None
+    oc = orc.Cache(1, heads, step.cap, w.sink)
+    sl = np.zeros(1, np.int32)
+    for t0 in range(0, pre, 4096):
+        t1 = min(pre, t0 + 4096)
+        K, V = W.kv_batch(w, t0, t1, device, bs=[0])
+        orc.append(oc, W.f16_bits(K[:, :, :heads]), W.f16_bits(V[:, :, :heads]), w.mode, rk, rv,
+                   pm, sl)
+    Kn = W.f16_bits(step.Knew[:1, :, :heads])
+    Vn = W.f16_bits(step.Vnew[:1, :, :heads])
+    Qs = W.f16_bits(step.Q[:1, :heads * w.G])
+    cores = len(os.sched_getaffinity(0))
+    n, t_start = 0, time.perf_counter()
+    while True:
+        sl[0] = pre
+        orc.append(oc, Kn, Vn, w.mode, rk, rv, pm, sl)
+        orc.decode(oc, Qs, w.mode, rk, rv, pm, sl, n_threads=cores)
+        n += 1
+        el = time.perf_counter() - t_start
+        if el >= min_seconds or n >= 1000:
+            break
+    per_step = el / n * (w.Hkv / heads) * w.B
+    return {"value": w.B / per_step, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "sequence 0, KV heads 0..%d of %d (append %d token + decode over %d), "
+                      "%d steps in %.1f s, scaled by %d/%d heads and B=%d"
+                      % (heads - 1, w.Hkv, step.T, step.L, n, el, w.Hkv, heads, w.B)}
+
+
+def run_cuda(args):
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_on = init_dist("nccl", world)
+    from rotated_int2_kv_head_b200 import build as kbuild
+    kbuild.build()
+    w = rank_workload(W.WORKLOADS[args.workload], rank)
+    step = Step(w, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lens = w.seq_lens()
+
+    def one(k, timed_split, evs=None):
+        flush.fill_(k & 0xff)
+        step.reset()
+        if evs:
+            evs[0].record()
+        step.run(timed_split)
+        if evs:
+            evs[1].record()
+
+    for k in range(args.warmup):
+        one(k, True)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    with ClockSampler(local) as clk:
+        barrier(dist_on, dev)
+        torch.cuda.synchronize(dev)
+        for k in range(K):
+            flush.fill_(k & 0xff)
+            step.reset()
+            ev[k][0].record()
+            step.run(False)
+            ev[k][1].record()
+        torch.cuda.synchronize(dev)
+        barrier(dist_on, dev)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), dist_on, dev)
+
+    # the streaming kernel alone, timed live by events the library records
+    # around it (a separate loop: events between kernels stop the
+    # programmatic overlap of the timed steps above)
+    n_split = min(K, 300)
+    split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n_split)]
+    for pair in split_ev:          # create the underlying events before handing them to C
+        for e in pair:
+            e.record()
+    torch.cuda.synchronize(dev)
+    for k in range(n_split):
+        flush.fill_(k & 0xff)
+        step.reset()
+        step.ev_split = split_ev[k]
+        step.run(True)
+    torch.cuda.synchronize(dev)
+    split_ms = [a.elapsed_time(b) for a, b in split_ev]
+    st = step.kvq.kvq_get_status(step.cache)
+    if st != 0:
+        raise RuntimeError("device status %d after timed steps" % st)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # new K/V and queries from pinned memory, append + decode, D2H of the output
+    hK = step.Knew.cpu().pin_memory()
+    hV = step.Vnew.cpu().pin_memory()
+    hQ = step.Q.cpu().pin_memory()
+    hO = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    n_e2e = min(K, 200)
+    e2e_s = 0.0
+    for k in range(n_e2e + 3):
+        flush.fill_(k & 0xff)
+        step.reset()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        step.Knew.copy_(hK, non_blocking=True)
+        step.Vnew.copy_(hV, non_blocking=True)
+        step.Q.copy_(hQ, non_blocking=True)
+        step.run(False)
+        hO.copy_(step.out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        if k >= 3:
+            e2e_s += time.perf_counter() - t0
+    e2e_s = max_over_ranks(e2e_s, dist_on, dev)
+    h2d = hK.numel() * 2 + hV.numel() * 2 + hQ.numel() * 2
+    d2h = hO.numel() * 2
+
+    if rank != 0:
+        if dist_on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    peak, peak_src = measured_peak()
+    kv_bytes = packed_kv_bytes(w, lens)
+    split_mean_s = float(np.mean(split_ms)) * 1e-3
+    achieved = kv_bytes / split_mean_s / 1e9
+    ms_per_step = total_ms / K
+    tokens = w.B * world
+    line = {
+        "metric": METRIC,
+        "value": tokens * K / (total_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int2 codes + fp16 scale/zero, fp32 accumulate",
+        "data": "synthetic (seeded; workloads.py)",
+        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
+                   "context": int(lens.max()), "append_T": w.append_T,
+                   "rotation": "dense" if w.mode == 0 else "perm+fwht", "sink_fp16": w.sink,
+                   "group": 32, "l2": "flushed between steps (256 MB write)",
+                   "parallelism": "replicas: one independent batch per GPU"},
+        "packed_kv_gbs": kv_bytes / (ms_per_step * 1e-3) / 1e9,
+        "packed_kv_bytes_per_step": kv_bytes,
+        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (streams the packed cache)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                     "algorithmic_bytes_per_launch": kv_bytes,
+                     "kernel_ms_mean": split_mean_s * 1e3, "peak_source": peak_src},
+        "e2e": {"value": tokens * n_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "how": "wall clock per step incl. pinned H2D of new "
+                                                  "K/V/Q and D2H of the output, synchronised"},
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, step, dev)
+    print(json.dumps(line), flush=True)
+    if dist_on:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# --- the reference arm: the CPU oracle ----------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    w = W.WORKLOADS[args.workload]
+    heads = 1
+    lens = w.seq_lens()
+    L, T = int(lens.max()), w.append_T
+    pre = L - T
+    Rk, Rv, perm = W.rotations(w)
+    rk = Rk[:heads] if Rk is not None else None
+    rv = Rv[:heads] if Rv is not None else None
+    pm = perm[:, :heads] if perm is not None else None
+    cap = ((L + 15) // 16) * 16
+    oc = orc.Cache(1, heads, cap, w.sink)
+    sl = np.zeros(1, np.int32)
+    for t0 in range(0, pre, 4096):
+        t1 = min(pre, t0 + 4096)
+        K, V = W.kv_batch(w, t0, t1, "cpu", bs=[0])
+        orc.append(oc, W.f16_bits(K[:, :, :heads]), W.f16_bits(V[:, :, :heads]), w.mode, rk, rv,
+                   pm, sl)
+    Kn, Vn = W.kv_batch(w, pre, L, "cpu", bs=[0])
+    Kn, Vn = W.f16_bits(Kn[:, :, :heads]), W.f16_bits(Vn[:, :, :heads])
+    Q = W.f16_bits(W.queries(w, "cpu")[:1, :heads * w.G])
+    cores = len(os.sched_getaffinity(0))
+
+    def one():
+        sl[0] = pre
+        orc.append(oc, Kn, Vn, w.mode, rk, rv, pm, sl)
+        orc.decode(oc, Q, w.mode, rk, rv, pm, sl, n_threads=cores)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    scale = (w.Hkv / heads) * w.B
+    per_step = el / args.steps * scale
+    value = w.B / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (fp32 quantizer)", "data": "synthetic (seeded; workloads.py)",
+        "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
+                   "context": L, "append_T": T, "rotation": "dense" if w.mode == 0 else "perm+fwht",
+                   "sink_fp16": w.sink, "group": 32},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "sequence 0, KV head 0 of %d per step (append %d + decode over "
+                                   "%d), time scaled by %d heads x B=%d" % (w.Hkv, T, L, w.Hkv, w.B)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--workload", default="llama7b", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

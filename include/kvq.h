@@ -156,6 +156,18 @@ KVQ_API kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq
                                 int32_t sink_fp16, int32_t max_ctx, void *workspace,
                                 size_t ws_bytes, uint16_t *out, void *stream);
 
+/* Same as kvq_decode_attention; in addition records the caller's CUDA events
+ * ev_begin / ev_end (cudaEvent_t, either may be NULL) on `stream` immediately
+ * before and after the kernel that streams the packed cache, so a caller can
+ * time that kernel alone. */
+KVQ_API kvq_status kvq_decode_attention_timed(const uint16_t *Q, int32_t Hq,
+                                              const kvq_cache_desc *cache, kvq_rot_mode mode,
+                                              const float *R_k, const float *R_v,
+                                              const int32_t *perm, const int32_t *seq_lens,
+                                              int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                              size_t ws_bytes, uint16_t *out, void *stream,
+                                              void *ev_begin, void *ev_end);
+
 /* Read (and leave set) the device status word: synchronises `stream`.
  * host_out is a host pointer. */
 KVQ_API kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out);

@@ -100,11 +100,12 @@ size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max
     return ws_layout(B, Hq, Hkv, C).total;
 }
 
-kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
-                                kvq_rot_mode mode, const float *R_k, const float *R_v,
-                                const int32_t *perm, const int32_t *seq_lens,
-                                int32_t sink_fp16, int32_t max_ctx, void *workspace,
-                                size_t ws_bytes, uint16_t *out, void *stream) {
+kvq_status kvq_decode_attention_timed(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                      const int32_t *perm, const int32_t *seq_lens,
+                                      int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                      size_t ws_bytes, uint16_t *out, void *stream, void *ev_begin,
+                                      void *ev_end) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
     if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
@@ -121,8 +122,18 @@ kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_d
     const int C = split_ctas(cache->B, cache->Hkv, max_ctx, sms);
     if (ws_bytes < ws_layout(cache->B, Hq, cache->Hkv, C).total) return KVQ_ERR_WORKSPACE;
     cudaError_t e = launch_decode(Q, Hq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out,
-                                  static_cast<cudaStream_t>(stream));
+                                  static_cast<cudaStream_t>(stream),
+                                  static_cast<cudaEvent_t>(ev_begin), static_cast<cudaEvent_t>(ev_end));
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                const int32_t *perm, const int32_t *seq_lens,
+                                int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                size_t ws_bytes, uint16_t *out, void *stream) {
+    return kvq_decode_attention_timed(Q, Hq, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
+                                      max_ctx, workspace, ws_bytes, out, stream, nullptr, nullptr);
 }
 
 kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out) {

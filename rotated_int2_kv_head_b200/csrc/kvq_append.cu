@@ -89,6 +89,8 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     __shared__ __align__(16) uint16_t xs[DENSE_BATCH][D];
     __shared__ __align__(16) float red[DENSE_BATCH][8][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
 
     int b = 0, h = 0, kind = 0, L0 = 0, row0, nrows;
     const uint16_t *X;
@@ -190,6 +192,8 @@ template <bool TO_CACHE>
 __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, CacheDst c) {
     __shared__ __align__(16) uint16_t xs[FWHT_THREADS / 32][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const long long row = (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
     if (row >= a.n_rows) return;
     int b = 0, t = 0, h = 0, kind = 0, L0 = 0;
@@ -238,6 +242,8 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
 
 // ---- length update ---------------------------------------------------------------------------
 __global__ void seq_bump_kernel(int32_t *seq_lens, int B, int T, int capacity) {
+    pdl_wait();
+    pdl_trigger();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     const int L0 = seq_lens[b];
@@ -287,7 +293,7 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.n_rows = 0;
         a.tchunk = T <= 64 ? T : 64;
         dim3 grid((T + a.tchunk - 1) / a.tchunk, cd.Hkv, 2 * cd.B);
-        append_dense_kernel<true><<<grid, DENSE_THREADS, 0, st>>>(a, c);
+        return launch_pdl(append_dense_kernel<true>, grid, dim3(DENSE_THREADS), 0, st, a, c);
     } else {
         FwhtRows a;
         a.X0 = K;
@@ -296,15 +302,14 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.out_f32 = nullptr;
         a.n_rows = (long long)cd.B * T * cd.Hkv * 2;
         const long long per = FWHT_THREADS / 32;
-        append_fwht_kernel<true><<<(unsigned)((a.n_rows + per - 1) / per), FWHT_THREADS, 0, st>>>(
-            a, c);
+        return launch_pdl(append_fwht_kernel<true>, dim3((unsigned)((a.n_rows + per - 1) / per)),
+                          dim3(FWHT_THREADS), 0, st, a, c);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_seq_bump(int32_t *seq_lens, int B, int T, int capacity, cudaStream_t st) {
-    seq_bump_kernel<<<(B + 255) / 256, 256, 0, st>>>(seq_lens, B, T, capacity);
-    return cudaGetLastError();
+    return launch_pdl(seq_bump_kernel, dim3((B + 255) / 256), dim3(256), 0, st, seq_lens, B, T,
+                      capacity);
 }
 
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,

@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(PRO_THREADS) decode_prologue_kernel(DecodeArgs
     const int warp = t >> 5, lane = t & 31;
     const int h = hq / a.G;
     const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
+    pdl_wait();
+    pdl_trigger();
 
     if (blockIdx.x == 0 && blockIdx.y == 0) {
         // prefix[b+1] = prefix[b] + Hkv * blocks(b): chunked scan
@@ -343,13 +345,15 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
 
     Sched sc;
     if (!sched_init(sc, a)) return;
     const int fb = a.S / BLK_TOK;
 
-    // Copies: every warp's lane 0 runs the schedule NSTAGE stages ahead; the
-    // last warp to release a ring slot refills it.
+    // Copies: thread 0 runs the schedule NSTAGE stages ahead of the
+    // consumers and refills a ring slot as soon as all warps released it.
     Sched ps = sc;
     int pit = 0;
     auto next_copy = [&](bool do_issue) {
@@ -367,13 +371,13 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
         ps.cur += n;
         ++pit;
     };
-    if (lane == 0)
-        for (int k = 0; k < NSTAGE; k++) next_copy(threadIdx.x == 0);
+    if (threadIdx.x == 0)
+        for (int k = 0; k < NSTAGE; k++) next_copy(true);
 
     const int r = lane >> 2, c = lane & 3;
     // per-unit query operands
     uint32_t qB[4][C::NTK_STEP][2];
-    float qsum[C::NTK], kap[C::NTK], kap2[C::NTK];
+    float qsum[C::NTK], kap2[C::NTK];
     int Lcur = 0;
     // online-softmax state
     float m_run[G], l_run[C::HPL], O[8][4], Z[NW];
@@ -419,7 +423,6 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
         for (int nu = 0; nu < C::NTK; nu++) {
             const int g = ktile_group<G>(nu, c), head = ktile_head<G>(nu, c);
             const float *qf = reinterpret_cast<const float *>(qbase + (size_t)head * QP * 4 + 2 * D);
-            kap[nu] = qf[g];
             kap2[nu] = qf[g] * (1.0f / 254.0f);
             qsum[nu] = qf[4 + g];
         }
@@ -563,10 +566,9 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                                                                       8 * (4 * r + g));
                     const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
                     const int hh = ktile_slot<G>(nu);
-                    const float d0 = fmaf(__int2float_rn(dk[bi][nu][1]), kap2[nu],
-                                          __int2float_rn(dk[bi][nu][0]) * kap[nu]);
-                    const float d1 = fmaf(__int2float_rn(dk[bi][nu][3]), kap2[nu],
-                                          __int2float_rn(dk[bi][nu][2]) * kap[nu]);
+                    // hi*254 + lo is exact in int32 (|.| < 2^28)
+                    const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
+                    const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
                     part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
                     part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
                 }
@@ -611,7 +613,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                 float al[G];
 #pragma unroll
                 for (int hd = 0; hd < G; hd++) {
-                    al[hd] = (mnew[hd] == NEG_INF) ? 1.f : exp2f(m_run[hd] - mnew[hd]);
+                    al[hd] = (mnew[hd] == NEG_INF) ? 1.f : fast_exp2(m_run[hd] - mnew[hd]);
                     m_run[hd] = mnew[hd];
                 }
 #pragma unroll
@@ -641,7 +643,9 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                     for (int hh = 0; hh < C::HPL; hh++) {
                         const float v = sco[bi][st][hh];
                         const float mm = pick<G>(m_run, lane_head<G>(c, hh));
-                        const float p = (edge[bi] && v == NEG_INF) ? 0.f : exp2f(v - mm);
+                        // every block holds a valid token, so mm is finite and
+                        // a masked score (-inf) gives exactly 0
+                        const float p = fast_exp2(v - mm);
                         P[bi][st][hh] = p;
                         l_run[hh] += p;
                     }
@@ -722,17 +726,11 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                 }
             }
         }
-        // release the slot; the last warp out refills it
-        __syncwarp();
-        if (lane == 0) {
-            __threadfence_block();
-            const int old = atomicAdd(&cnt[s], 1);
-            const bool last = (old % DEC_WARPS) == DEC_WARPS - 1;
-            if (last) {
-                __threadfence_block();
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            }
-            next_copy(last);
+        // release the slot: once every warp is done with it, thread 0 refills it
+        asm volatile("bar.sync 1, %0;" ::"n"(DEC_THREADS) : "memory");
+        if (threadIdx.x == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            next_copy(true);
         }
         sc.cur += n;
         ++it;
@@ -758,6 +756,16 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     const int warp = t >> 5, lane = t & 31;
     const int G = a.G, h = hq / G, head = hq % G;
     uint16_t *out = a.out + ((size_t)b * a.Hq + hq) * D;
+    // R_v rows for the rotate-out: no kernel of this chain writes R_v, so they
+    // are fetched before waiting on the split kernel
+    float4 rr[16];
+    if (a.mode == KVQ_ROT_DENSE) {
+        const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
+#pragma unroll
+        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+    }
+    pdl_wait();
+    pdl_trigger();
     const int L = a.seq_lens[b];
     if (L < 1 || L > a.capacity) {
         if (t < D) out[t] = 0;
@@ -825,10 +833,6 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     __syncthreads();
     if (a.mode == KVQ_ROT_DENSE) {
         // out[i] = sum_j o[j] R_v[h][i][j]: warp w rows 16w..16w+15, lanes over j
-        const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
-        float4 rr[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
         const float4 o4 = *reinterpret_cast<const float4 *>(&o_s[4 * lane]);
         float mine = 0.f;
 #pragma unroll
@@ -877,14 +881,13 @@ static cudaError_t launch_split(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_split_kernel<G><<<a.C, DEC_THREADS, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(decode_split_kernel<G>, dim3(a.C), dim3(DEC_THREADS), smem, st, a);
 }
 
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
-                          cudaStream_t st) {
+                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
     const WsLayout w = ws_layout(cd.B, Hq, cd.Hkv, C);
     uint8_t *base = static_cast<uint8_t *>(ws);
     DecodeArgs a;
@@ -911,9 +914,9 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.nblk = cd.capacity / BLK_TOK;
     a.mode = mode;
     a.C = C;
-    decode_prologue_kernel<<<dim3(Hq, cd.B), PRO_THREADS, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(decode_prologue_kernel, dim3(Hq, cd.B), dim3(PRO_THREADS), 0, st, a);
     if (e != cudaSuccess) return e;
+    if (ev_begin && (e = cudaEventRecord(ev_begin, st)) != cudaSuccess) return e;
     switch (a.G) {
         case 1: e = launch_split<1>(a, st); break;
         case 2: e = launch_split<2>(a, st); break;
@@ -922,8 +925,8 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<dim3(Hq, cd.B), MRG_THREADS, 0, st>>>(a);
-    return cudaGetLastError();
+    if (ev_end && (e = cudaEventRecord(ev_end, st)) != cudaSuccess) return e;
+    return launch_pdl(decode_merge_kernel, dim3(Hq, cd.B), dim3(MRG_THREADS), 0, st, a);
 }
 
 }  // namespace kvq

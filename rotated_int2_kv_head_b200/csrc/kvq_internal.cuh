@@ -221,6 +221,14 @@ __device__ __forceinline__ void imma16832(int d[4], uint32_t a0, uint32_t a1, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// 2^x by the SFU's ex2.approx (max relative error about 2^-22; results
+// below 2^-126 flush to 0, which a softmax weight may do).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
@@ -229,6 +237,35 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_half2(uint32_t u) {
     const __half2 h = *reinterpret_cast<const __half2 *>(&u);
     return __half22float2(h);
+}
+
+// ---- programmatic dependent launch ---------------------------------------------------------
+// Every kernel is launched with programmatic stream serialisation, so it may
+// start while the previous kernel in the stream drains.  Each kernel calls
+// pdl_wait() (the previous grid has completed and its writes are visible)
+// before it reads anything the previous kernel may write, and only then
+// pdl_trigger() to let the next kernel launch.  Hence when a kernel starts,
+// every grid before its predecessor has completed; work placed before
+// pdl_wait() touches only data no earlier kernel of the chain writes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // ---- host launchers (defined in kvq_append.cu / kvq_decode.cu) ---------------------------
@@ -244,7 +281,7 @@ cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
-                          cudaStream_t st);
+                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
 
 // Decode workspace: prefix sums, prepared queries, sink partials, split partials.
 struct WsLayout {
