@@ -168,6 +168,36 @@ KVQ_API kvq_status kvq_decode_attention_timed(const uint16_t *Q, int32_t Hq,
                                               size_t ws_bytes, uint16_t *out, void *stream,
                                               void *ev_begin, void *ev_end);
 
+/* Size of the fixed device array that kvq_decode_attention_noalloc uses as
+ * its workspace (4 MiB).  Decode shapes whose workspace
+ * (kvq_decode_workspace_size) exceeds it are rejected. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * kvq_decode_attention without a workspace argument, for callers that cannot
+ * allocate device memory (a serving loop whose device memory is fixed at
+ * start-up, a plugin inside a framework that owns every allocation).  The
+ * pages describe no such entry point; it is a deployment convenience with no
+ * counterpart in the method.
+ *   Same arguments and results as kvq_decode_attention, minus workspace /
+ *   ws_bytes.  The workspace is a fixed KVQ_NOALLOC_SCRATCH_BYTES array in
+ *   the library's own device memory, held by every GPU that loads the
+ *   library until the process exits; nothing is allocated or freed.
+ *   Errors: KVQ_ERR_WORKSPACE if the shape needs more than the fixed array
+ *   (checked on the host before any launch), otherwise as
+ *   kvq_decode_attention.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the array: calls that may overlap on the GPU (other
+ *   streams, other host threads) race and must be serialised by the caller.
+ */
+KVQ_API kvq_status kvq_decode_attention_noalloc(const uint16_t *Q, int32_t Hq,
+                                                const kvq_cache_desc *cache, kvq_rot_mode mode,
+                                                const float *R_k, const float *R_v,
+                                                const int32_t *perm, const int32_t *seq_lens,
+                                                int32_t sink_fp16, int32_t max_ctx, uint16_t *out,
+                                                void *stream);
+
 /* Read (and leave set) the device status word: synchronises `stream`.
  * host_out is a host pointer. */
 KVQ_API kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out);

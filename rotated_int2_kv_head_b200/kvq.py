@@ -68,6 +68,9 @@ def lib():
     L.kvq_decode_attention_timed.restype = C.c_int
     L.kvq_decode_attention_timed.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p, i32,
                                              i32, p, sz, p, p, p, p]
+    L.kvq_decode_attention_noalloc.restype = C.c_int
+    L.kvq_decode_attention_noalloc.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p,
+                                               i32, i32, p, p]
     L.kvq_get_status.restype = C.c_int
     L.kvq_get_status.argtypes = [C.POINTER(CacheDesc), p, C.POINTER(C.c_int32)]
     L.kvq_clear_status.restype = C.c_int
@@ -203,6 +206,21 @@ def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp
                                             max_ctx, _ptr(workspace), workspace.numel(), _ptr(out),
                                             _stream(stream), C.c_void_p(ev_begin.cuda_event),
                                             C.c_void_p(ev_end.cuda_event)))
+
+
+def kvq_decode_attention_noalloc(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
+                                 out, stream=None):
+    """kvq_decode_attention for callers that cannot allocate device memory:
+    no workspace argument, the library's fixed device array serves instead
+    (see include/kvq.h for its size and the sharing rules)."""
+    B, Hq, d = Q.shape
+    _need(Q, torch.float16, "Q", (cache.B, Hq, D))
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _check("kvq_decode_attention_noalloc",
+           lib().kvq_decode_attention_noalloc(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k),
+                                              _ptr(R_v), _ptr(perm), _ptr(seq_lens), sink_fp16,
+                                              max_ctx, _ptr(out), _stream(stream)))
 
 
 def kvq_get_status(cache, stream=None):
