@@ -1,0 +1,159 @@
+"""The five workloads at full size, in the launch configuration bench.py
+uses, checked against the CPU oracle on sampled (sequence, KV head) units.
+
+The GPU fills the whole cache from inputs drawn on the GPU; the rows of the
+sampled units are copied to the host and the oracle builds its own cache
+for them from the same tensors (the oracle never reads anything the CUDA
+path produced), then decodes.  Properties that hold at any size are checked
+on every output (finite, zero status).
+"""
+import numpy as np
+import pytest
+import torch
+
+import rotated_int2_kv_head_b200 as kvq
+import workloads as W
+from oracle import oracle as orc
+
+from kvq_testlib import rel_err
+
+pytestmark = pytest.mark.gpu
+DEC_TOL = 2e-3
+CHUNK = 2048
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from rotated_int2_kv_head_b200 import build
+    build.build()
+
+
+def run_workload(w, samples, prefill_to=None):
+    """Fill the GPU cache to each sequence's length (all sequences are
+    appended together up to the longest; shorter ones simply decode fewer
+    tokens), append the step's tokens, decode.  Returns GPU outputs and the
+    oracle outputs of the sampled (b, h) units."""
+    dev = "cuda"
+    lens = w.seq_lens().astype(np.int64)
+    L = int(lens.max())
+    T = w.append_T
+    cap = ((L + 15) // 16) * 16
+    Rk, Rv, perm = W.rotations(w)
+    rk = torch.from_numpy(Rk).to(dev) if Rk is not None else None
+    rv = torch.from_numpy(Rv).to(dev) if Rv is not None else None
+    pm = torch.from_numpy(perm).to(dev) if perm is not None else None
+    cache = kvq.KVCache(w.B, w.Hkv, cap, w.sink)
+    sl = torch.zeros(w.B, dtype=torch.int32, device=dev)
+    # host copies of the sampled units' rows: {(b, h): (K rows, V rows)}
+    keep = {u: ([], []) for u in samples}
+    pre = L - T
+    for t0 in list(range(0, pre, CHUNK)) + [pre]:
+        t1 = min(pre, t0 + CHUNK) if t0 < pre else L
+        if t1 <= t0:
+            continue
+        K, V = W.kv_batch(w, t0, t1, dev)
+        kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, pm, cache, sl)
+        for (b, h), (kl, vl) in keep.items():
+            kl.append(W.f16_bits(K[b, :, h]))
+            vl.append(W.f16_bits(V[b, :, h]))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    assert (sl.cpu().numpy() == L).all()
+    lens_t = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    Q = W.queries(w, dev)
+    ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, L)
+    out = torch.empty_like(Q)
+    kvq.kvq_decode_attention(Q, cache, w.mode, rk, rv, pm, lens_t, w.sink, L, ws, out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    assert torch.isfinite(out).all()
+    out = out.float().cpu().numpy()
+    Qh = W.f16_bits(Q)
+    refs = {}
+    for (b, h), (kl, vl) in keep.items():
+        Lb = int(lens[b])
+        k = np.concatenate(kl)[:Lb].reshape(1, Lb, 1, 128)
+        v = np.concatenate(vl)[:Lb].reshape(1, Lb, 1, 128)
+        oc = orc.Cache(1, 1, cap, w.sink)
+        s1 = np.zeros(1, np.int32)
+        orc.append(oc, k, v, w.mode, Rk[h:h + 1] if Rk is not None else None,
+                   Rv[h:h + 1] if Rv is not None else None,
+                   perm[:, h:h + 1] if perm is not None else None, s1)
+        q = Qh[b:b + 1, h * w.G:(h + 1) * w.G]
+        ref, st = orc.decode(oc, q, w.mode, Rk[h:h + 1] if Rk is not None else None,
+                             Rv[h:h + 1] if Rv is not None else None,
+                             perm[:, h:h + 1] if perm is not None else None,
+                             np.array([Lb], np.int32), n_threads=8)
+        assert st == 0
+        refs[(b, h)] = ref[0]
+    return out, refs
+
+
+def check(w, samples):
+    out, refs = run_workload(w, samples)
+    for (b, h), ref in refs.items():
+        got = out[b, h * w.G:(h + 1) * w.G]
+        err = rel_err(got, ref)
+        assert err.max() <= DEC_TOL, ((b, h), err.max())
+
+
+def test_tiny_full():
+    check(W.WORKLOADS["tiny"], [(0, 0)])
+
+
+def test_llama7b_full():
+    check(W.WORKLOADS["llama7b"], [(0, 0), (0, 17), (0, 31)])
+
+
+def test_hadamard_full():
+    check(W.WORKLOADS["hadamard"], [(0, 0), (7, 13), (15, 31)])
+
+
+def test_gqa_sinks_full():
+    check(W.WORKLOADS["gqa_sinks"], [(0, 0), (7, 7)])
+
+
+def test_ragged_full():
+    w = W.WORKLOADS["ragged"]
+    lens = w.seq_lens()
+    bmin, bmax = int(np.argmin(lens)), int(np.argmax(lens))
+    check(w, [(bmin, 0), (bmax, 31), (5, 7)])
+
+
+def test_ragged_prefill_append_full():
+    """The bulk prefill append (B=4, 32768 tokens x 32 heads): sampled
+    (sequence, head, token) rows of the GPU cache equal the oracle quantizer
+    applied to the GPU's own rotation of the same rows, and agree with the
+    oracle's rotation except at near ties."""
+    w0 = W.WORKLOADS["ragged"]
+    B, T = w0.extra["prefill_B"], w0.extra["prefill_T"]
+    w = W.custom(name="ragged_prefill", seed=w0.seed + 1, B=B, Hq=32, Hkv=32, mode=0,
+                 k_outliers=8, context=T)
+    Rk, Rv, _ = W.rotations(w)
+    rk, rv = torch.from_numpy(Rk).cuda(), torch.from_numpy(Rv).cuda()
+    K, V = W.kv_batch(w, 0, T, "cuda")
+    cache = kvq.KVCache(B, 32, T, 0)
+    sl = torch.zeros(B, dtype=torch.int32, device="cuda")
+    kvq.kvq_rotate_quantize_append(K, V, 0, rk, rv, None, cache, sl)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0 and (sl.cpu().numpy() == T).all()
+    rng = np.random.default_rng(3)
+    picks = [(b, h, t) for b, h, t in zip(rng.integers(0, B, 64), rng.integers(0, 32, 64),
+                                          rng.integers(0, T, 64))] + [(0, 0, 0), (B - 1, 31, T - 1)]
+    blocks = cache.block_view()
+    n_diff = n_codes = 0
+    for b, h, t in picks:
+        for kind, X, R in ((0, K, Rk), (1, V, Rv)):
+            x = X[b, t, h][None].contiguous()
+            grot = kvq.kvq_debug_rotate_f32(x, 0, R=(rk if kind == 0 else rv)[h].contiguous())
+            c, s, z = orc.quantize_rows(grot.cpu().numpy())
+            blk = blocks[b, h, t // 16].cpu().numpy()
+            kb, vb, ks, kz, vs, vz = orc.load_token(blk, t % 16)
+            got_c = orc.unpack_row(kb if kind == 0 else vb)
+            assert np.array_equal(got_c, c[0])
+            assert np.array_equal(ks if kind == 0 else vs, s[0])
+            assert np.array_equal(kz if kind == 0 else vz, z[0])
+            oc, _, _ = orc.quantize_rows(orc.rotate_rows_f32(W.f16_bits(x), 0, R=R[h]))
+            n_diff += int((oc[0] != got_c).sum())
+            n_codes += 128
+    assert n_diff <= max(2, 1e-4 * n_codes), (n_diff, n_codes)
