@@ -13,9 +13,11 @@ tensors (workloads.py).
     torchrun --nproc-per-node N bench.py --gpus N ...
 
 Timing: every step is bracketed by CUDA events on the launching stream; an
-L2 flush (256 MB write) and the reset of the sequence length to its
-pre-append value happen between steps, outside the events, so each step
-starts cold and at the same context.  K steps run back to back between a
+L2 flush and the reset of the sequence length to its pre-append value happen
+between steps, outside the events, so each step starts cold and at the same
+context.  The flush writes a 256 MB buffer and then reads another 256 MB one:
+a write alone would leave L2 full of dirty lines whose write-back the next
+timed kernel would pay for.  K steps run back to back between a
 barrier + synchronize on both sides; the device time is summed per rank and
 the max over ranks is reported.  With N GPUs every rank serves its own
 independent batch (weak scaling, no collective on the data path).
@@ -40,8 +42,21 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "INT2-KV decode attention tokens/s and packed-KV GB/s (% of HBM peak), 1 B200"
-KERNELS_PER_STEP = 5      # append, length bump, decode prologue, split, merge
+KERNELS_PER_STEP = 4      # append (with the length update), query preparation, decode split, merge
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Evicts the cache's data from L2: write one buffer larger than L2,
+    then read another, so L2 ends up holding clean lines."""
+
+    def __init__(self, device):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    def __call__(self, k):
+        self.w.fill_(k & 0xff)
+        self.r.sum()
 
 
 # --- distributed plumbing (also exercised by tests/test_bench_dist.py on CPU) ----------------
@@ -294,11 +309,11 @@ def run_cuda(args):
     kbuild.build()
     w = rank_workload(W.WORKLOADS[args.workload], rank)
     step = Step(w, dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     lens = w.seq_lens()
 
     def one(k, timed_split, evs=None):
-        flush.fill_(k & 0xff)
+        flush(k)
         step.reset()
         if evs:
             evs[0].record()
@@ -316,7 +331,7 @@ def run_cuda(args):
         barrier(dist_on, dev)
         torch.cuda.synchronize(dev)
         for k in range(K):
-            flush.fill_(k & 0xff)
+            flush(k)
             step.reset()
             ev[k][0].record()
             step.run(False)
@@ -337,7 +352,7 @@ def run_cuda(args):
             e.record()
     torch.cuda.synchronize(dev)
     for k in range(n_split):
-        flush.fill_(k & 0xff)
+        flush(k)
         step.reset()
         step.ev_split = split_ev[k]
         step.run(True)
@@ -356,7 +371,7 @@ def run_cuda(args):
     n_e2e = min(K, 200)
     e2e_s = 0.0
     for k in range(n_e2e + 3):
-        flush.fill_(k & 0xff)
+        flush(k)
         step.reset()
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
@@ -399,7 +414,7 @@ def run_cuda(args):
         "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
                    "context": int(lens.max()), "append_T": w.append_T,
                    "rotation": "dense" if w.mode == 0 else "perm+fwht", "sink_fp16": w.sink,
-                   "group": 32, "l2": "flushed between steps (256 MB write)",
+                   "group": 32, "l2": "flushed between steps (256 MB write, then 256 MB read)",
                    "parallelism": "replicas: one independent batch per GPU"},
         "packed_kv_gbs": kv_bytes / (ms_per_step * 1e-3) / 1e9,
         "packed_kv_bytes_per_step": kv_bytes,

@@ -29,8 +29,13 @@
  *     per-device attributes only).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Compute
  *     calls are asynchronous on it; argument errors are reported before any
- *     launch and nothing is launched then.
- *   - Device-detected errors never trap: they OR a bit into *cache->status
+ *     launch and nothing is launched then.  The kernels use programmatic
+ *     dependent launch: the rotation inputs (R_k, R_v, perm) may be read
+ *     while the work enqueued just before the call is still finishing, so
+ *     they must not be written by that work (set them up once, or make the
+ *     writer complete - e.g. with an event - before the call).  Every other
+ *     input is read only after the preceding work in the stream completed.
+ *   - Device-detected errors never trap: they OR a bit into cache->status[0]
  *     (see KVQ_DEV_*) and the affected work is skipped.
  *
  * Quantizer (exact IEEE fp32, no contraction), per group of 32 values x:
@@ -105,7 +110,11 @@ typedef struct {
     void *blocks;             /* [B][Hkv][capacity/16][1536] bytes, 16-B aligned */
     uint16_t *k_sink;         /* [B][Hkv][sink_fp16][128] fp16, or NULL if 0     */
     uint16_t *v_sink;         /* same                                           */
-    int32_t *status;          /* one device word, sticky error bits (KVQ_DEV_*) */
+    int32_t *status;          /* two device words, 8-B aligned: [0] sticky error
+                                 bits (KVQ_DEV_*); [1] the library's append
+                                 completion counter.  Zero both once before
+                                 first use; [1] is zero again after every
+                                 append.                                        */
 } kvq_cache_desc;
 
 /* Bytes of the blocks array for a cache of this shape (0 on bad arguments). */
@@ -202,7 +211,8 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(const uint16_t *Q, int32_t Hq,
  * host_out is a host pointer. */
 KVQ_API kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *host_out);
 
-/* Clear the device status word (asynchronous on `stream`). */
+/* Clear both device status words (asynchronous on `stream`); do not call it
+ * while an append may be in flight. */
 KVQ_API kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream);
 
 /*

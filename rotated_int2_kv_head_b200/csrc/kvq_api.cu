@@ -34,7 +34,7 @@ kvq_status check_cache(const kvq_cache_desc *c) {
     if (c->sink_fp16 < 0 || c->sink_fp16 > MAX_SINK || c->sink_fp16 > c->capacity)
         return KVQ_ERR_INVALID_ARG;
     if (!c->blocks || !c->status) return KVQ_ERR_INVALID_ARG;
-    if (!aligned(c->blocks, 16) || !aligned(c->status, 4)) return KVQ_ERR_UNSUPPORTED;
+    if (!aligned(c->blocks, 16) || !aligned(c->status, 8)) return KVQ_ERR_UNSUPPORTED;
     if (c->sink_fp16 > 0) {
         if (!c->k_sink || !c->v_sink) return KVQ_ERR_INVALID_ARG;
         if (!aligned(c->k_sink, 16) || !aligned(c->v_sink, 16)) return KVQ_ERR_UNSUPPORTED;
@@ -89,7 +89,6 @@ kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int3
     if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
-    if (e == cudaSuccess) e = launch_seq_bump(seq_lens, cache->B, T, cache->capacity, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -147,7 +146,7 @@ kvq_status kvq_get_status(const kvq_cache_desc *cache, void *stream, int32_t *ho
 
 kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream) {
     if (!cache || !cache->status) return KVQ_ERR_INVALID_ARG;
-    return cudaMemsetAsync(cache->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) ==
+    return cudaMemsetAsync(cache->status, 0, 2 * sizeof(int32_t), static_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? KVQ_OK
                : KVQ_ERR_CUDA;

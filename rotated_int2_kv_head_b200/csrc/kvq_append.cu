@@ -13,7 +13,9 @@
 //                        medium T; large T goes to the tensor-core kernel).
 //   append_fwht_kernel   one warp per row: permutation gather, 128-point FWHT
 //                        in registers and shuffles, quantize, pack.
-//   seq_bump_kernel      seq_lens[b] += T once every CTA has read it.
+//   The last CTA of an append to finish adds T to every valid seq_lens[b]
+//   (a completion counter in the cache's second status word tells it that it
+//   is last), so no separate kernel is needed.
 //   debug kernels        the same rotation / quantizer code with fp32 outputs.
 #include "kvq_internal.cuh"
 
@@ -23,10 +25,33 @@ namespace kvq {
 struct CacheDst {
     uint8_t *blocks;
     uint16_t *k_sink, *v_sink;
-    const int32_t *seq_lens;
-    int32_t *status;
+    int32_t *seq_lens;
+    int32_t *status;          // [0] error bits, [1] CTA completion counter
     int B, T, Hkv, capacity, S, nblk;
 };
+
+// Called by every CTA of an append kernel after its last read of seq_lens
+// and its last write: the CTA that completes last bumps the lengths and
+// resets the counter for the next append.
+__device__ void append_done(const CacheDst &c) {
+    __shared__ int last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+        const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(c.status + 1), 1u);
+        last = (prev == total - 1);
+        if (last) __threadfence();
+    }
+    __syncthreads();
+    if (last) {
+        for (int b = threadIdx.x; b < c.B; b += blockDim.x) {
+            const int L0 = c.seq_lens[b];
+            if (L0 >= 0 && (long long)L0 + c.T <= c.capacity) c.seq_lens[b] = L0 + c.T;
+        }
+        if (threadIdx.x == 0) atomicExch(reinterpret_cast<unsigned *>(c.status + 1), 0u);
+    }
+}
 
 // Epilogue shared by both append kernels: row (b, t, h, kind) with rotated
 // values v (lane layout of quantize_row_warp).
@@ -100,9 +125,8 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         kind = blockIdx.z & 1;
         b = blockIdx.z >> 1;
         L0 = start_len(c, b);
-        if (L0 < 0) return;
         row0 = blockIdx.x * a.tchunk;
-        nrows = min(a.tchunk, c.T - row0);
+        nrows = L0 < 0 ? 0 : min(a.tchunk, c.T - row0);     // skipped sequence: no rows
         X = (kind == 0 ? a.X0 : a.X1);
         R = (kind == 0 ? a.R0 : a.R1) + (size_t)h * D * D;
     } else {
@@ -111,7 +135,10 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         X = a.X0;
         R = a.R0;
     }
-    if (nrows <= 0) return;
+    if (nrows <= 0) {
+        if (TO_CACHE) append_done(c);
+        return;
+    }
 
     float Rr[16][4];
 #pragma unroll
@@ -175,6 +202,7 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         }
         __syncthreads();
     }
+    if (TO_CACHE) append_done(c);
 }
 
 // ---- permutation + FWHT ---------------------------------------------------------------------
@@ -195,11 +223,11 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
     pdl_wait();
     pdl_trigger();
     const long long row = (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
-    if (row >= a.n_rows) return;
+    bool active = row < a.n_rows;
     int b = 0, t = 0, h = 0, kind = 0, L0 = 0;
-    const uint16_t *src;
-    const int32_t *perm;
-    if (TO_CACHE) {
+    const uint16_t *src = nullptr;
+    const int32_t *perm = nullptr;
+    if (active && TO_CACHE) {
         // row order (b, t, h, kind) with kind fastest
         kind = (int)(row & 1);
         long long r2 = row >> 1;
@@ -211,43 +239,36 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
         if (L < 0 || (long long)L + c.T > c.capacity) {
             if (lane == 0 && t == 0 && h == 0 && kind == 0)
                 set_status(c.status, L < 0 ? KVQ_DEV_BAD_LEN : KVQ_DEV_CAPACITY);
-            return;
+            active = false;
         }
         L0 = L;
         src = (kind == 0 ? a.X0 : a.X1) + (((size_t)b * c.T + t) * c.Hkv + h) * D;
         perm = a.perm + ((size_t)kind * c.Hkv + h) * D;
-    } else {
+    } else if (active) {
         src = a.X0 + (size_t)row * D;
         perm = a.perm;
     }
-    *reinterpret_cast<uint2 *>(&xs[warp][4 * lane]) =
-        *reinterpret_cast<const uint2 *>(src + 4 * lane);
-    const int4 pi = *reinterpret_cast<const int4 *>(perm + 4 * lane);
-    __syncwarp();
-    float v[4];
-    v[0] = __half2float(__ushort_as_half(xs[warp][pi.x & (D - 1)]));
-    v[1] = __half2float(__ushort_as_half(xs[warp][pi.y & (D - 1)]));
-    v[2] = __half2float(__ushort_as_half(xs[warp][pi.z & (D - 1)]));
-    v[3] = __half2float(__ushort_as_half(xs[warp][pi.w & (D - 1)]));
-    fwht128_warp(v);
-    const float inv_sqrt_d = 0.08838834764831845f;
+    if (active) {
+        *reinterpret_cast<uint2 *>(&xs[warp][4 * lane]) =
+            *reinterpret_cast<const uint2 *>(src + 4 * lane);
+        const int4 pi = *reinterpret_cast<const int4 *>(perm + 4 * lane);
+        __syncwarp();
+        float v[4];
+        v[0] = __half2float(__ushort_as_half(xs[warp][pi.x & (D - 1)]));
+        v[1] = __half2float(__ushort_as_half(xs[warp][pi.y & (D - 1)]));
+        v[2] = __half2float(__ushort_as_half(xs[warp][pi.z & (D - 1)]));
+        v[3] = __half2float(__ushort_as_half(xs[warp][pi.w & (D - 1)]));
+        fwht128_warp(v);
+        const float inv_sqrt_d = 0.08838834764831845f;
 #pragma unroll
-    for (int k = 0; k < 4; k++) v[k] *= inv_sqrt_d;
-    if (TO_CACHE)
-        cache_epilogue(c, b, t, h, kind, L0, v);
-    else
-        *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
-            make_float4(v[0], v[1], v[2], v[3]);
-}
-
-// ---- length update ---------------------------------------------------------------------------
-__global__ void seq_bump_kernel(int32_t *seq_lens, int B, int T, int capacity) {
-    pdl_wait();
-    pdl_trigger();
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= B) return;
-    const int L0 = seq_lens[b];
-    if (L0 >= 0 && (long long)L0 + T <= capacity) seq_lens[b] = L0 + T;
+        for (int k = 0; k < 4; k++) v[k] *= inv_sqrt_d;
+        if (TO_CACHE)
+            cache_epilogue(c, b, t, h, kind, L0, v);
+        else
+            *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
+                make_float4(v[0], v[1], v[2], v[3]);
+    }
+    if (TO_CACHE) append_done(c);
 }
 
 // ---- quantizer test export ---------------------------------------------------------------------
@@ -269,7 +290,7 @@ __global__ void debug_quantize_kernel(const float *X, int N, uint8_t *codes, uin
 // ---- host launchers (called from kvq_api.cu) -----------------------------------------------------
 cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int mode,
                                 const float *R_k, const float *R_v, const int32_t *perm,
-                                const kvq_cache_desc &cd, const int32_t *seq_lens,
+                                const kvq_cache_desc &cd, int32_t *seq_lens,
                                 cudaStream_t st) {
     CacheDst c;
     c.blocks = static_cast<uint8_t *>(cd.blocks);
@@ -305,11 +326,6 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         return launch_pdl(append_fwht_kernel<true>, dim3((unsigned)((a.n_rows + per - 1) / per)),
                           dim3(FWHT_THREADS), 0, st, a, c);
     }
-}
-
-cudaError_t launch_seq_bump(int32_t *seq_lens, int B, int T, int capacity, cudaStream_t st) {
-    return launch_pdl(seq_bump_kernel, dim3((B + 255) / 256), dim3(256), 0, st, seq_lens, B, T,
-                      capacity);
 }
 
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,

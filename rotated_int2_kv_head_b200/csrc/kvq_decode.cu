@@ -8,22 +8,22 @@
 // Sinks are the leading positions stored in fp16 ("RotateKV", abstract item
 // (iii)).
 //
-// Three kernels:
-//   decode_prologue_kernel  per (b, query head): q_rot = q.R_k (or perm+FWHT),
-//                           scaled into the exp2 domain; sink-token partial
-//                           softmax in fp32; block 0 also writes the prefix
-//                           sums that balance the split kernel.
+// Two kernels:
 //   decode_split_kernel<G>  stream-K over all cache blocks of all (b, h)
 //                           units: every CTA takes an equal share of 16-token
-//                           blocks.  A producer warp streams them into a
+//                           blocks (the schedule is derived from seq_lens by
+//                           every CTA).  Thread 0 streams them into a
 //                           shared-memory ring with 1-D bulk copies (TMA);
-//                           four consumer warps run the scores and P.V on
-//                           tensor cores straight from the packed codes and
-//                           keep an online softmax; each (CTA, unit) segment
-//                           leaves one partial (m, l, o_rot[128]) per head.
-//   decode_merge_kernel     per (b, query head): merge the partials, then
+//                           the CTA rotates and quantises the unit's queries
+//                           while the first copies land; four warps run the
+//                           scores and P.V on tensor cores straight from the
+//                           packed codes with an online softmax; each (CTA,
+//                           unit) segment leaves one partial (m, l, o_rot[128])
+//                           per head.
+//   decode_merge_kernel     per (b, query head): the sink partial (fp16 sinks,
+//                           fp32 CUDA cores), the merge of all partials, then
 //                           out = o_rot . R_v^T (or FWHT + inverse permutation).
-//
+
 // Tensor-core operand trick.  A 2-bit code c sitting in bits [2g, 2g+1] of a
 // 16-bit lane, with every other bit zero, IS the fp16 subnormal c*4^g*2^-24.
 // So one AND turns a packed word into an m16n8k16 fragment register (two
@@ -42,10 +42,10 @@ constexpr int SPLIT_MIN_CTAS = 4;                         // resident CTAs per S
 constexpr int STAGE_BLKS = 2 * DEC_WARPS;                 // 8 blocks = 128 tokens
 constexpr int STAGE_BYTES = STAGE_BLKS * BLK_BYTES;       // 12 KB
 constexpr int NSTAGE = 4;
-// Prepared query per (b, query head), QP floats = 288 bytes:
+// Prepared query per query head, QB bytes:
 //   int8 hi[128], int8 lo[128]  with q_s ~= sq_g * (hi + lo/254) per group g
 //   float kap[4] = sq_g / 4^g,  float qsum[4] = sum of q_s over group g
-constexpr int QP = 72;
+constexpr int QB = 288;
 constexpr int PART = 132;   // per partial: m, l, 0, 0, o[128]
 constexpr float LOG2E = 1.4426950408889634f;
 #define NEG_INF (__int_as_float(0xff800000))
@@ -58,9 +58,8 @@ struct DecodeArgs {
     const int32_t *perm;
     const int32_t *seq_lens;
     int32_t *status;
-    int32_t *prefix;   // [B+1] workspace
-    float *qprep;      // [B*Hq][QP]
-    float *sinkp;      // [B*Hq][PART]
+    int32_t *prefix;   // [B+1] workspace, written by split CTA 0
+    uint8_t *qprep;    // [B*Hq][QB] prepared queries
     float *part;       // [(C+U)*G][PART]
     uint16_t *out;
     int B, Hq, Hkv, G, S, capacity, nblk, mode, C;
@@ -74,199 +73,182 @@ __device__ __forceinline__ int unit_blocks(int L, int S, int capacity) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Prologue.
-// ---------------------------------------------------------------------------------------------
-constexpr int PRO_THREADS = 256;
-
-__global__ void __launch_bounds__(PRO_THREADS) decode_prologue_kernel(DecodeArgs a) {
-    __shared__ __align__(16) float qs[D];
-    __shared__ __align__(16) float red[PRO_THREADS / 32][D];
-    __shared__ float ssc[MAX_SINK];
-    __shared__ int scan[PRO_THREADS];
-    const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
-    const int warp = t >> 5, lane = t & 31;
-    const int h = hq / a.G;
-    const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
-    pdl_wait();
-    pdl_trigger();
-
-    if (blockIdx.x == 0 && blockIdx.y == 0) {
-        // prefix[b+1] = prefix[b] + Hkv * blocks(b): chunked scan
-        const int per = (a.B + PRO_THREADS - 1) / PRO_THREADS;
-        int s = 0;
-        for (int i = t * per; i < min(a.B, (t + 1) * per); i++)
-            s += a.Hkv * unit_blocks(a.seq_lens[i], a.S, a.capacity);
-        scan[t] = s;
-        __syncthreads();
-        if (t == 0) {
-            int acc = 0;
-            for (int i = 0; i < PRO_THREADS; i++) {
-                const int v = scan[i];
-                scan[i] = acc;
-                acc += v;
-            }
-        }
-        __syncthreads();
-        int acc = scan[t];
-        for (int i = t * per; i < min(a.B, (t + 1) * per); i++) {
-            a.prefix[i] = acc;
-            const int L = a.seq_lens[i];
-            if (L < 1 || L > a.capacity) set_status(a.status, KVQ_DEV_BAD_LEN);
-            acc += a.Hkv * unit_blocks(L, a.S, a.capacity);
-        }
-        if (t == PRO_THREADS - 1) a.prefix[a.B] = acc;
-    }
-
-    // q_rot in fp32, then scaled by log2(e)/sqrt(128) so scores are exp2 exponents
-    if (a.mode == KVQ_ROT_DENSE) {
-        // warp w: rows 16w..16w+15 of R_k, lane l: columns 4l..4l+3; all 16
-        // row loads are issued before any is used
-        const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
-        float4 rr[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
-        const uint4 u0 = *reinterpret_cast<const uint4 *>(q + 16 * warp);
-        const uint4 u1 = *reinterpret_cast<const uint4 *>(q + 16 * warp + 8);
-        const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int ii = 0; ii < 8; ii++) {
-            const float2 x2 = unpack_half2(w8[ii]);
-            const float4 ra = rr[2 * ii], rb = rr[2 * ii + 1];
-            acc.x = fmaf(x2.x, ra.x, acc.x); acc.y = fmaf(x2.x, ra.y, acc.y);
-            acc.z = fmaf(x2.x, ra.z, acc.z); acc.w = fmaf(x2.x, ra.w, acc.w);
-            acc.x = fmaf(x2.y, rb.x, acc.x); acc.y = fmaf(x2.y, rb.y, acc.y);
-            acc.z = fmaf(x2.y, rb.z, acc.z); acc.w = fmaf(x2.y, rb.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
-        __syncthreads();
-        if (t < D) {
-            float v = 0.f;
-#pragma unroll
-            for (int w2 = 0; w2 < PRO_THREADS / 32; w2++) v += red[w2][t];
-            qs[t] = v;
-        }
-    } else if (warp == 0) {
-        __shared__ uint16_t xq[D];
-        *reinterpret_cast<uint2 *>(&xq[4 * lane]) = *reinterpret_cast<const uint2 *>(q + 4 * lane);
-        const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
-        __syncwarp();
-        float v[4] = {__half2float(__ushort_as_half(xq[pi.x & (D - 1)])),
-                      __half2float(__ushort_as_half(xq[pi.y & (D - 1)])),
-                      __half2float(__ushort_as_half(xq[pi.z & (D - 1)])),
-                      __half2float(__ushort_as_half(xq[pi.w & (D - 1)]))};
-        fwht128_warp(v);
-        *reinterpret_cast<float4 *>(&qs[4 * lane]) =
-            make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
-                        v[2] * 0.08838834764831845f, v[3] * 0.08838834764831845f);
-    }
-    __syncthreads();
-    const float qscale = LOG2E * 0.08838834764831845f;
-    float qv = 0.f;
-    if (t < D) {
-        // q_s = q_rot * log2(e)/sqrt(128); per group, an int8 hi/lo pair on
-        // the scale max|q_s|/127 (about 15 significant bits)
-        qv = qs[t] * qscale;
-        uint8_t *qp = reinterpret_cast<uint8_t *>(a.qprep + ((size_t)b * a.Hq + hq) * QP);
-        float gs = qv, amax = fabsf(qv);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            gs += __shfl_xor_sync(0xffffffffu, gs, off);
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        }
-        const float sq = amax > 0.f ? amax * (1.0f / 127.0f) : 1.0f;
-        const float u = qv / sq;
-        const float hi = fminf(fmaxf(rintf(u), -127.f), 127.f);
-        const float lo = fminf(fmaxf(rintf((u - hi) * 254.0f), -127.f), 127.f);
-        qp[t] = (uint8_t)(int8_t)hi;
-        qp[D + t] = (uint8_t)(int8_t)lo;
-        if (lane == 0) {
-            float *qf = reinterpret_cast<float *>(qp + 2 * D);
-            qf[warp] = sq * __int_as_float((127 - 2 * warp) << 23);   // sq / 4^g
-            qf[4 + warp] = gs;
-        }
-    }
-
-    // sink partial (fp32, CUDA cores): at most MAX_SINK tokens
-    if (a.S > 0) {
-        __syncthreads();
-        if (t < D) qs[t] = qv;
-        __syncthreads();
-        const int L = a.seq_lens[b];
-        const bool ok = (L >= 1 && L <= a.capacity);
-        const int ns = ok ? min(a.S, L) : 0;
-        const uint16_t *ks = a.k_sink + ((size_t)b * a.Hkv + h) * a.S * D;
-        const uint16_t *vs = a.v_sink + ((size_t)b * a.Hkv + h) * a.S * D;
-        for (int tk = warp; tk < ns; tk += PRO_THREADS / 32) {
-            const uint2 u = *reinterpret_cast<const uint2 *>(ks + (size_t)tk * D + 4 * lane);
-            const float2 k01 = unpack_half2(u.x), k23 = unpack_half2(u.y);
-            float d = qs[4 * lane] * k01.x + qs[4 * lane + 1] * k01.y + qs[4 * lane + 2] * k23.x +
-                      qs[4 * lane + 3] * k23.y;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            if (lane == 0) ssc[tk] = d;
-        }
-        __syncthreads();
-        if (t < D) {
-            float m = NEG_INF;
-            for (int tk = 0; tk < ns; tk++) m = fmaxf(m, ssc[tk]);
-            float l = 0.f, o = 0.f;
-            for (int tk = 0; tk < ns; tk++) {
-                const float p = exp2f(ssc[tk] - m);
-                l += p;
-                o = fmaf(p, __half2float(__ushort_as_half(vs[(size_t)tk * D + t])), o);
-            }
-            float *sp = a.sinkp + ((size_t)b * a.Hq + hq) * PART;
-            sp[4 + t] = o;
-            if (t == 0) {
-                sp[0] = m;
-                sp[1] = l;
-            }
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
 // Split kernel.
 // ---------------------------------------------------------------------------------------------
 // Per-CTA schedule over the global block space: unit u = b*Hkv + h holds
-// nb(b) consecutive global blocks starting at prefix[b] + h*nb(b).
+// nb(b) consecutive global blocks starting at prefix[b] + h*nb(b), where
+// prefix[b] = Hkv * sum over b' < b of nb(b').  `pref` carries prefix[b].
 struct Sched {
-    int b, h, nb, ustart, cur, end;
+    int b, h, nb, ustart, cur, end, pref;
 };
+
+__device__ __forceinline__ int seq_blocks(const DecodeArgs &a, int b) {
+    return unit_blocks(a.seq_lens[b], a.S, a.capacity);
+}
 
 __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
     // move (b, h) forward until cur lies inside the unit
     while (s.cur >= s.ustart + s.nb && s.cur < s.end) {
         if (++s.h == a.Hkv) {
             s.h = 0;
+            s.pref += a.Hkv * s.nb;
             ++s.b;
+            s.nb = seq_blocks(a, s.b);
         }
-        if (s.h == 0) s.nb = (a.prefix[s.b + 1] - a.prefix[s.b]) / a.Hkv;
-        s.ustart = a.prefix[s.b] + s.h * s.nb;
+        s.ustart = s.pref + s.h * s.nb;
     }
 }
 
-__device__ __forceinline__ bool sched_init(Sched &s, const DecodeArgs &a) {
-    const int N = a.prefix[a.B];
+// CTA-wide (all DEC_THREADS threads): total block count N from seq_lens, this
+// CTA's range [c*W, min(N, (c+1)*W)) with W = ceil(N / C), and the unit that
+// holds its first block.  CTA 0 also writes prefix[0..B] for the merge.
+// scan: DEC_THREADS + 2 ints of shared scratch.  Returns false for an empty
+// range (uniformly over the CTA).
+__device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scan) {
+    const int t = threadIdx.x;
+    const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
+    const int lo = min(a.B, t * per), hi = min(a.B, lo + per);
+    int sum = 0;
+    for (int b = lo; b < hi; b++) sum += a.Hkv * seq_blocks(a, b);
+    scan[t] = sum;
+    __syncthreads();
+    if (t == 0) {
+        int acc = 0;
+        for (int i = 0; i < DEC_THREADS; i++) {
+            const int v = scan[i];
+            scan[i] = acc;
+            acc += v;
+        }
+        scan[DEC_THREADS] = acc;
+    }
+    __syncthreads();
+    const int N = scan[DEC_THREADS];
+    if (blockIdx.x == 0) {
+        int acc = scan[t];
+        for (int b = lo; b < hi; b++) {
+            a.prefix[b] = acc;
+            const int L = a.seq_lens[b];
+            if (L < 1 || L > a.capacity) set_status(a.status, KVQ_DEV_BAD_LEN);
+            acc += a.Hkv * seq_blocks(a, b);
+        }
+        if (t == DEC_THREADS - 1) a.prefix[a.B] = N;
+    }
     const int W = max(1, (N + a.C - 1) / a.C);
-    s.cur = blockIdx.x * W;
-    s.end = min(N, s.cur + W);
-    if (s.cur >= s.end) return false;
-    int lo = 0, hi = a.B;            // largest b with prefix[b] <= cur
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (a.prefix[mid] <= s.cur) lo = mid; else hi = mid;
+    const int beg = blockIdx.x * W, end = min(N, beg + W);
+    if (beg >= end) return false;
+    // the chunk holding block `beg` finds its sequence
+    const int cstart = scan[t], cend = (t == DEC_THREADS - 1) ? N : scan[t + 1];
+    __syncthreads();
+    if (cstart <= beg && beg < cend) {
+        int acc = cstart;
+        for (int b = lo; b < hi; b++) {
+            const int nbb = a.Hkv * seq_blocks(a, b);
+            if (beg < acc + nbb) {
+                scan[DEC_THREADS] = b;
+                scan[DEC_THREADS + 1] = acc;
+                break;
+            }
+            acc += nbb;
+        }
     }
-    s.b = lo;
-    s.nb = (a.prefix[s.b + 1] - a.prefix[s.b]) / a.Hkv;
-    while (s.nb == 0) {              // empty sequences have prefix[b] == prefix[b+1]
-        ++s.b;
-        s.nb = (a.prefix[s.b + 1] - a.prefix[s.b]) / a.Hkv;
-    }
-    s.h = (s.cur - a.prefix[s.b]) / s.nb;
-    s.ustart = a.prefix[s.b] + s.h * s.nb;
+    __syncthreads();
+    s.b = scan[DEC_THREADS];
+    s.pref = scan[DEC_THREADS + 1];
+    s.nb = seq_blocks(a, s.b);
+    s.h = (beg - s.pref) / s.nb;
+    s.ustart = s.pref + s.h * s.nb;
+    s.cur = beg;
+    s.end = end;
+    __syncthreads();
     return true;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Query preparation: per (b, KV head), the G queries rotated by R_k (or perm +
+// FWHT), scaled by log2(e)/sqrt(128) so scores are exp2 exponents, and per
+// group an int8 hi/lo pair on the scale max|q_s|/127 (about 15 significant
+// bits): qprep[(b*Hq + hq)*QB] = {hi[128], lo[128], kap[4] = sq_g/4^g,
+// qsum[4]}.  R_k (64 KB per head, the bulk of what it reads) is loaded before
+// the dependency wait, alongside a preceding append; Q after it.
+// ---------------------------------------------------------------------------------------------
+constexpr int QP_THREADS = 256;
+
+__global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) {
+    __shared__ __align__(16) float red[QP_THREADS / 32][D];
+    __shared__ __align__(16) float qr_s[D];
+    const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int G = a.G;
+    float4 rr[16];
+    if (a.mode == KVQ_ROT_DENSE) {
+        // warp w: rows 16w..16w+15 of R_k, lane l: columns 4l..4l+3, all loads in flight
+        const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
+#pragma unroll
+        for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+    }
+    pdl_wait();
+    pdl_trigger();
+    for (int hd = 0; hd < G; hd++) {
+        const int hq = h * G + hd;
+        const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
+        __syncthreads();
+        if (a.mode == KVQ_ROT_DENSE) {
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(q + 16 * warp);
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(q + 16 * warp + 8);
+            const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int ii = 0; ii < 8; ii++) {
+                const float2 x2 = unpack_half2(w8[ii]);
+                const float4 ra = rr[2 * ii], rb = rr[2 * ii + 1];
+                acc.x = fmaf(x2.x, ra.x, acc.x); acc.y = fmaf(x2.x, ra.y, acc.y);
+                acc.z = fmaf(x2.x, ra.z, acc.z); acc.w = fmaf(x2.x, ra.w, acc.w);
+                acc.x = fmaf(x2.y, rb.x, acc.x); acc.y = fmaf(x2.y, rb.y, acc.y);
+                acc.z = fmaf(x2.y, rb.z, acc.z); acc.w = fmaf(x2.y, rb.w, acc.w);
+            }
+            *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
+            __syncthreads();
+            if (t < D) {
+                float v = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < QP_THREADS / 32; w2++) v += red[w2][t];
+                qr_s[t] = v;
+            }
+        } else if (warp == 0) {
+            const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
+            float v[4] = {__half2float(__ushort_as_half(q[pi.x & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.y & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.z & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.w & (D - 1)]))};
+            fwht128_warp(v);
+            *reinterpret_cast<float4 *>(&qr_s[4 * lane]) =
+                make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
+                            v[2] * 0.08838834764831845f, v[3] * 0.08838834764831845f);
+        }
+        __syncthreads();
+        if (t < D) {
+            // thread t = element t; warp g = group g
+            const float qv = qr_s[t] * (LOG2E * 0.08838834764831845f);
+            float gs = qv, amax = fabsf(qv);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                gs += __shfl_xor_sync(0xffffffffu, gs, off);
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            }
+            const float sq = amax > 0.f ? amax * (1.0f / 127.0f) : 1.0f;
+            const float u = qv / sq;
+            const float hi = fminf(fmaxf(rintf(u), -127.f), 127.f);
+            const float lo = fminf(fmaxf(rintf((u - hi) * 254.0f), -127.f), 127.f);
+            uint8_t *qp = reinterpret_cast<uint8_t *>(a.qprep) + ((size_t)b * a.Hq + hq) * QB;
+            qp[t] = (uint8_t)(int8_t)hi;
+            qp[D + t] = (uint8_t)(int8_t)lo;
+            if (lane == 0) {
+                float *qf = reinterpret_cast<float *>(qp + 2 * D);
+                qf[warp] = sq * __int_as_float((127 - 2 * warp) << 23);   // sq / 4^g
+                qf[4 + warp] = gs;
+            }
+        }
+    }
 }
 
 template <int G>
@@ -320,20 +302,45 @@ __device__ __forceinline__ void wsrc(int c, int k, int &g, int &head) {
     else { g = k & 3; head = c + 4 * (k >> 2); }
 }
 
+// Shared-memory carve-out of the split kernel: every piece starts on a
+// 16-byte boundary (descriptors are read as int4).
+struct SplitSmem {
+    unsigned full, cnt, desc, psm, qsm, fo, fm, fl, fz, abort, total;
+};
+__host__ __device__ constexpr unsigned smem_up16(unsigned x) { return (x + 15u) & ~15u; }
+__host__ __device__ inline SplitSmem split_smem_layout(int G) {
+    SplitSmem L{};
+    L.full = NSTAGE * STAGE_BYTES;
+    L.cnt = smem_up16(L.full + NSTAGE * 8u);
+    L.desc = smem_up16(L.cnt + NSTAGE * 4u);
+    L.psm = smem_up16(L.desc + 2u * NSTAGE * 16u);
+    L.qsm = smem_up16(L.psm + 32u);
+    L.fo = L.qsm;
+    L.fm = smem_up16(L.fo + 4u * DEC_WARPS * G * D);
+    L.fl = smem_up16(L.fm + 4u * DEC_WARPS * G);
+    L.fz = smem_up16(L.fl + 4u * DEC_WARPS * G);
+    L.abort = smem_up16(L.fz + 4u * DEC_WARPS * G * 4);
+    L.total = smem_up16(L.abort + 4u);
+    return L;
+}
+
 template <int G>
 __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kernel(DecodeArgs a) {
     using C = Cfg<G>;
     constexpr int NW = G;                              // weight registers per lane per block
     constexpr int NGL = G == 1 ? 1 : (G == 2 ? 2 : 4); // V-meta groups a lane reads
     extern __shared__ __align__(128) uint8_t smem[];
+    SplitSmem L = split_smem_layout(G);
     uint8_t *ring = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NSTAGE * STAGE_BYTES);
-    int *cnt = reinterpret_cast<int *>(full + NSTAGE);               // [NSTAGE]
-    float *fo = reinterpret_cast<float *>(cnt + NSTAGE);              // [W][G][128]
-    float *fm = fo + DEC_WARPS * G * D;                              // [W][G]
-    float *fl = fm + DEC_WARPS * G;                                  // [W][G]
-    float *fz = fl + DEC_WARPS * G;                                  // [W][G][4]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(fz + DEC_WARPS * G * 4);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);     // [NSTAGE]
+    int *cnt = reinterpret_cast<int *>(smem + L.cnt);                 // [NSTAGE]
+    int4 *desc = reinterpret_cast<int4 *>(smem + L.desc);             // [2*NSTAGE] stage descriptors
+    Sched *psm = reinterpret_cast<Sched *>(smem + L.psm);             // producer schedule state
+    float *fo = reinterpret_cast<float *>(smem + L.fo);               // [W][G][128]; also scratch
+    float *fm = reinterpret_cast<float *>(smem + L.fm);               // [W][G]
+    float *fl = reinterpret_cast<float *>(smem + L.fl);               // [W][G]
+    float *fz = reinterpret_cast<float *>(smem + L.fz);               // [W][G][4]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -345,34 +352,49 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_wait();
-    pdl_trigger();
-
+    // The append before this decode has completed (the query-preparation
+    // kernel waited on it before letting this kernel launch), so seq_lens and
+    // the cache are read - and the first copies issued - before waiting on
+    // the prepared queries.
     Sched sc;
-    if (!sched_init(sc, a)) return;
+    if (!sched_init_cta(sc, a, reinterpret_cast<int *>(fo))) {
+        pdl_wait();
+        pdl_trigger();
+        return;
+    }
     const int fb = a.S / BLK_TOK;
 
-    // Copies: thread 0 runs the schedule NSTAGE stages ahead of the
-    // consumers and refills a ring slot as soon as all warps released it.
-    Sched ps = sc;
-    int pit = 0;
-    auto next_copy = [&](bool do_issue) {
+    // Copies.  Thread 0 keeps the producer state (the schedule NSTAGE stages
+    // ahead of the consumers) in shared memory; when all warps have released
+    // a ring slot it issues the next stage into it and writes that stage's
+    // descriptor:
+    //   {unit, b, h, first cache block}, n blocks | flags << 8
+    // flags: 1 = last stage of this CTA's segment of the unit, 2 = last stage
+    // of the CTA.  Consumers read descriptors instead of running the schedule.
+    auto issue_next = [&](int slot) {
+        Sched ps = *psm;
         if (ps.cur >= ps.end) return;
         sched_fix_unit(ps, a);
         const int n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
-        if (do_issue) {
-            const int s = pit % NSTAGE;
-            const size_t unit = (size_t)ps.b * a.Hkv + ps.h;
-            const uint8_t *src =
-                a.blocks + (unit * a.nblk + fb + (ps.cur - ps.ustart)) * (size_t)BLK_BYTES;
-            mbar_arrive_expect_tx(&full[s], n * BLK_BYTES);
-            bulk_g2s(ring + s * STAGE_BYTES, src, n * BLK_BYTES, &full[s]);
-        }
+        const int unit = ps.b * a.Hkv + ps.h;
+        const int kblk = fb + (ps.cur - ps.ustart);
         ps.cur += n;
-        ++pit;
+        const int flags = (ps.cur == ps.ustart + ps.nb || ps.cur == ps.end ? 1 : 0) |
+                          (ps.cur == ps.end ? 2 : 0);
+        desc[2 * slot] = make_int4(unit, ps.b, ps.h, kblk);
+        desc[2 * slot + 1] = make_int4(n | (flags << 8), 0, 0, 0);
+        *psm = ps;
+        mbar_arrive_expect_tx(&full[slot], n * BLK_BYTES);
+        bulk_g2s(ring + slot * STAGE_BYTES,
+                 a.blocks + ((size_t)unit * a.nblk + kblk) * (size_t)BLK_BYTES, n * BLK_BYTES,
+                 &full[slot]);
     };
-    if (threadIdx.x == 0)
-        for (int k = 0; k < NSTAGE; k++) next_copy(true);
+    if (threadIdx.x == 0) {
+        *psm = sc;
+        for (int k = 0; k < NSTAGE; k++) issue_next(k);
+    }
+    pdl_wait();
+    pdl_trigger();
 
     const int r = lane >> 2, c = lane & 3;
     // per-unit query operands
@@ -399,8 +421,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
     auto load_unit = [&](int b, int h) {
         // B fragments of the K-side IMMA, one per group: column n of the N
         // tile is (group, head, hi/lo); k = element e of the group
-        const uint8_t *qbase = reinterpret_cast<const uint8_t *>(
-            a.qprep + ((size_t)b * a.Hq + (size_t)h * G) * QP);
+        const uint8_t *qbase = a.qprep + ((size_t)b * a.Hq + (size_t)h * G) * QB;
         const int n = lane >> 2;
 #pragma unroll
         for (int g = 0; g < 4; g++) {
@@ -411,7 +432,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                 const int gcol = col / (2 * G), head = (col % (2 * G)) / 2, hl = col & 1;
                 uint32_t b0 = 0u, b1 = 0u;
                 if (gcol == g) {
-                    const uint8_t *qh = qbase + (size_t)head * QP * 4 + hl * D + 32 * g;
+                    const uint8_t *qh = qbase + head * QB + hl * D + 32 * g;
                     b0 = *reinterpret_cast<const uint32_t *>(qh + 4 * c);
                     b1 = *reinterpret_cast<const uint32_t *>(qh + 16 + 4 * c);
                 }
@@ -422,7 +443,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
 #pragma unroll
         for (int nu = 0; nu < C::NTK; nu++) {
             const int g = ktile_group<G>(nu, c), head = ktile_head<G>(nu, c);
-            const float *qf = reinterpret_cast<const float *>(qbase + (size_t)head * QP * 4 + 2 * D);
+            const float *qf = reinterpret_cast<const float *>(qbase + head * QB + 2 * D);
             kap2[nu] = qf[g] * (1.0f / 254.0f);
             qsum[nu] = qf[4 + g];
         }
@@ -499,15 +520,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
     };
 
     reset_state();
-    int it = 0;
-    while (sc.cur < sc.end) {
-        sched_fix_unit(sc, a);
-        const int unit = sc.b * a.Hkv + sc.h;
-        if (unit != cur_unit) {
-            load_unit(sc.b, sc.h);
-            cur_unit = unit;
-        }
-        const int n = min(min(STAGE_BLKS, sc.end - sc.cur), sc.ustart + sc.nb - sc.cur);
+    for (int it = 0;; ++it) {
         const int s = it % NSTAGE;
         const bool ok = mbar_wait_bounded(&full[s], (it / NSTAGE) & 1);
         if (!ok || *abort_flag) {
@@ -515,10 +528,17 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
             *abort_flag = 1;
             break;
         }
+        const int4 d0 = desc[2 * s];
+        const int d1 = desc[2 * s + 1].x;
+        const int unit = d0.x, n = d1 & 0xff, flags = d1 >> 8;
+        if (unit != cur_unit) {
+            load_unit(d0.y, d0.z);
+            cur_unit = unit;
+        }
         const int nmine = min(2, max(0, n - 2 * warp));
         if (nmine > 0) {
             const uint8_t *blk0 = ring + s * STAGE_BYTES + (2 * warp) * BLK_BYTES;
-            const int tok0 = (fb + (sc.cur - sc.ustart) + 2 * warp) * BLK_TOK;   // first position
+            const int tok0 = (d0.w + 2 * warp) * BLK_TOK;   // first position of my first block
             // a block needs masking if it is a phantom or crosses [S, L)
             bool edge[2];
 #pragma unroll
@@ -590,7 +610,18 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                         sco[bi][st][hh] = v;
                     }
             }
-            // ---- online softmax update (the branch is uniform over the warp)
+            // ---- online softmax.  The running max only moves when a score of
+            // this stage exceeds it (rare after the first stages), so the
+            // common path is one vote; the branch is uniform over the warp.
+            bool over = false;
+#pragma unroll
+            for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+                for (int st = 0; st < 2; st++)
+#pragma unroll
+                    for (int hh = 0; hh < C::HPL; hh++)
+                        over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
+            if (__any_sync(0xffffffffu, over)) {
             float mt[C::HPL];
 #pragma unroll
             for (int hh = 0; hh < C::HPL; hh++) {
@@ -634,6 +665,7 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                         O[2 * g + 1][k] *= f;
                     }
             }
+            }
             float P[2][2][C::HPL];
 #pragma unroll
             for (int bi = 0; bi < 2; bi++)
@@ -653,30 +685,38 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
 #pragma unroll
             for (int bi = 0; bi < 2; bi++) {
                 const uint8_t *blk = blk0 + bi * BLK_BYTES;
-                // weights w = p * s_v in the score layout, as half2 (token r, token r+8)
+                // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
+                // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
                 uint32_t H[NW];
                 {
-                    float2 sz[NGL][2];
+                    uint32_t spair[NGL];
+                    float zr[NGL][2];
 #pragma unroll
                     for (int gl = 0; gl < NGL; gl++) {
                         const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
                         const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
-                        sz[gl][0] = unpack_half2(mv.x);
-                        sz[gl][1] = unpack_half2(mv.y);
+                        spair[gl] = __byte_perm(mv.x, mv.y, 0x5410);      // (s_r, s_r+8)
+                        zr[gl][0] = __half2float(__ushort_as_half((unsigned short)(mv.x >> 16)));
+                        zr[gl][1] = __half2float(__ushort_as_half((unsigned short)(mv.y >> 16)));
                     }
 #pragma unroll
                     for (int k = 0; k < NW; k++) {
                         const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
                         const int hh = G >= 8 ? (k >> 2) : 0;
                         const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
-                        float w0 = p0 * sz[gl][0].x, w1 = p1 * sz[gl][1].x;
-                        float z0 = p0 * sz[gl][0].y, z1 = p1 * sz[gl][1].y;
-                        if (edge[bi]) {      // masked tokens: never touch their metadata
-                            w0 = p0 == 0.f ? 0.f : w0; z0 = p0 == 0.f ? 0.f : z0;
-                            w1 = p1 == 0.f ? 0.f : w1; z1 = p1 == 0.f ? 0.f : z1;
+                        const uint32_t ph = pack_half2(p0, p1);
+                        const __half2 w2 = __hmul2(*reinterpret_cast<const __half2 *>(&ph),
+                                                   *reinterpret_cast<const __half2 *>(&spair[gl]));
+                        uint32_t hw = *reinterpret_cast<const uint32_t *>(&w2);
+                        float z0 = zr[gl][0], z1 = zr[gl][1];
+                        if (edge[bi]) {      // masked tokens (p == 0): never use their metadata
+                            hw &= (p0 == 0.f ? 0xffff0000u : 0xffffffffu) &
+                                  (p1 == 0.f ? 0x0000ffffu : 0xffffffffu);
+                            z0 = p0 == 0.f ? 0.f : z0;
+                            z1 = p1 == 0.f ? 0.f : z1;
                         }
-                        H[k] = pack_half2(w0, w1);
-                        Z[k] += z0 + z1;
+                        H[k] = hw;
+                        Z[k] = fmaf(p0, z0, fmaf(p1, z1, Z[k]));
                     }
                 }
                 // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
@@ -730,15 +770,14 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
         asm volatile("bar.sync 1, %0;" ::"n"(DEC_THREADS) : "memory");
         if (threadIdx.x == 0) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            next_copy(true);
+            issue_next(s);
         }
-        sc.cur += n;
-        ++it;
         // end of this CTA's segment of the unit: write the partial
-        if (sc.cur == sc.ustart + sc.nb || sc.cur == sc.end) {
+        if (flags & 1) {
             flush(blockIdx.x + unit);
             reset_state();
         }
+        if (flags & 2) break;
     }
 }
 
@@ -752,12 +791,92 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     __shared__ __align__(16) float o_s[D];
     __shared__ __align__(16) float red[MRG_THREADS / 32][D];
     __shared__ float pm[MRG_MAXP + 1], pl[MRG_MAXP + 1], wred[MRG_THREADS / 32];
+    __shared__ __align__(16) float qs[D];
+    __shared__ float ssc[MAX_SINK];
+    __shared__ __align__(16) float sinkp[PART];          // the sink partial: m, l, 0, 0, o[128]
     const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int G = a.G, h = hq / G, head = hq % G;
     uint16_t *out = a.out + ((size_t)b * a.Hq + hq) * D;
-    // R_v rows for the rotate-out: no kernel of this chain writes R_v, so they
-    // are fetched before waiting on the split kernel
+    // Before waiting on the split kernel: only data that kernel does not write
+    // (its predecessor, the append, has completed by the time this kernel can
+    // start).  The sink partial, in fp32 on CUDA cores: q_rot, scores over the
+    // fp16 sink rows, softmax, weighted sum.
+    const int L = a.seq_lens[b];
+    const bool lok = (L >= 1 && L <= a.capacity);
+    const int ns = (a.S > 0 && lok) ? min(a.S, L) : 0;
+    if (ns > 0) {
+        const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
+        if (a.mode == KVQ_ROT_DENSE) {
+            const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
+            float4 rr[16];
+#pragma unroll
+            for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(q + 16 * warp);
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(q + 16 * warp + 8);
+            const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int ii = 0; ii < 8; ii++) {
+                const float2 x2 = unpack_half2(w8[ii]);
+                const float4 ra = rr[2 * ii], rb = rr[2 * ii + 1];
+                acc.x = fmaf(x2.x, ra.x, acc.x); acc.y = fmaf(x2.x, ra.y, acc.y);
+                acc.z = fmaf(x2.x, ra.z, acc.z); acc.w = fmaf(x2.x, ra.w, acc.w);
+                acc.x = fmaf(x2.y, rb.x, acc.x); acc.y = fmaf(x2.y, rb.y, acc.y);
+                acc.z = fmaf(x2.y, rb.z, acc.z); acc.w = fmaf(x2.y, rb.w, acc.w);
+            }
+            *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
+            __syncthreads();
+            if (t < D) {
+                float v = 0.f;
+#pragma unroll
+                for (int w2 = 0; w2 < MRG_THREADS / 32; w2++) v += red[w2][t];
+                qs[t] = v;
+            }
+        } else if (warp == 0) {
+            const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
+            float v[4] = {__half2float(__ushort_as_half(q[pi.x & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.y & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.z & (D - 1)])),
+                          __half2float(__ushort_as_half(q[pi.w & (D - 1)]))};
+            fwht128_warp(v);
+            *reinterpret_cast<float4 *>(&qs[4 * lane]) =
+                make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
+                            v[2] * 0.08838834764831845f, v[3] * 0.08838834764831845f);
+        }
+        __syncthreads();
+        if (t < D) qs[t] *= LOG2E * 0.08838834764831845f;      // exp2 domain, like the partials
+        __syncthreads();
+        const uint16_t *ks = a.k_sink + ((size_t)b * a.Hkv + h) * a.S * D;
+        const uint16_t *vs = a.v_sink + ((size_t)b * a.Hkv + h) * a.S * D;
+        for (int tk = warp; tk < ns; tk += MRG_THREADS / 32) {
+            const uint2 uu = *reinterpret_cast<const uint2 *>(ks + (size_t)tk * D + 4 * lane);
+            const float2 k01 = unpack_half2(uu.x), k23 = unpack_half2(uu.y);
+            float d = qs[4 * lane] * k01.x + qs[4 * lane + 1] * k01.y + qs[4 * lane + 2] * k23.x +
+                      qs[4 * lane + 3] * k23.y;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            if (lane == 0) ssc[tk] = d;
+        }
+        __syncthreads();
+        if (t < D) {
+            float m = NEG_INF;
+            for (int tk = 0; tk < ns; tk++) m = fmaxf(m, ssc[tk]);
+            float l = 0.f, o = 0.f;
+            for (int tk = 0; tk < ns; tk++) {
+                const float p = exp2f(ssc[tk] - m);
+                l += p;
+                o = fmaf(p, __half2float(__ushort_as_half(vs[(size_t)tk * D + t])), o);
+            }
+            sinkp[4 + t] = o;
+            if (t == 0) {
+                sinkp[0] = m;
+                sinkp[1] = l;
+            }
+        }
+        __syncthreads();
+    }
+    // R_v rows for the rotate-out (no kernel of this chain writes R_v)
     float4 rr[16];
     if (a.mode == KVQ_ROT_DENSE) {
         const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
@@ -766,8 +885,7 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     }
     pdl_wait();
     pdl_trigger();
-    const int L = a.seq_lens[b];
-    if (L < 1 || L > a.capacity) {
+    if (!lok) {
         if (t < D) out[t] = 0;
         return;
     }
@@ -778,11 +896,10 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     const int ustart = a.prefix[b] + h * nb;
     const int c0 = nb > 0 ? ustart / W : 0;
     const int np = nb > 0 ? (ustart + nb - 1) / W - c0 + 1 : 0;
-    const float *sp = a.sinkp + ((size_t)b * a.Hq + hq) * PART;
     auto pptr = [&](int i) -> const float * {   // partial i (i == np: the sink partial)
-        return i < np ? a.part + ((size_t)(c0 + i + u) * G + head) * PART : sp;
+        return i < np ? a.part + ((size_t)(c0 + i + u) * G + head) * PART : sinkp;
     };
-    const int ntot = np + (a.S > 0 ? 1 : 0);
+    const int ntot = np + (ns > 0 ? 1 : 0);
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f, mglob = NEG_INF;
@@ -858,9 +975,8 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
 // Host side.
 // ---------------------------------------------------------------------------------------------
 size_t split_smem_bytes(int G) {
-    return (size_t)NSTAGE * STAGE_BYTES + NSTAGE * (sizeof(uint64_t) + sizeof(int)) +
-           sizeof(float) * (DEC_WARPS * G * D + 2 * DEC_WARPS * G + DEC_WARPS * G * 4) +
-           16;
+    static_assert(sizeof(Sched) <= 32, "producer state slot");
+    return split_smem_layout(G).total;
 }
 
 WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
@@ -869,8 +985,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
     const int G = Hq / Hkv;
     w.prefix = 0;
     w.qprep = up(w.prefix + sizeof(int32_t) * (B + 1));
-    w.sinkp = up(w.qprep + sizeof(float) * (size_t)B * Hq * QP);
-    w.part = up(w.sinkp + sizeof(float) * (size_t)B * Hq * PART);
+    w.part = up(w.qprep + (size_t)B * Hq * QB);
     w.total = up(w.part + sizeof(float) * ((size_t)C + (size_t)B * Hkv) * G * PART);
     return w;
 }
@@ -901,8 +1016,7 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.seq_lens = seq_lens;
     a.status = cd.status;
     a.prefix = reinterpret_cast<int32_t *>(base + w.prefix);
-    a.qprep = reinterpret_cast<float *>(base + w.qprep);
-    a.sinkp = reinterpret_cast<float *>(base + w.sinkp);
+    a.qprep = base + w.qprep;
     a.part = reinterpret_cast<float *>(base + w.part);
     a.out = out;
     a.B = cd.B;
@@ -914,7 +1028,7 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.nblk = cd.capacity / BLK_TOK;
     a.mode = mode;
     a.C = C;
-    cudaError_t e = launch_pdl(decode_prologue_kernel, dim3(Hq, cd.B), dim3(PRO_THREADS), 0, st, a);
+    cudaError_t e = launch_pdl(decode_qprep_kernel, dim3(cd.Hkv, cd.B), dim3(QP_THREADS), 0, st, a);
     if (e != cudaSuccess) return e;
     if (ev_begin && (e = cudaEventRecord(ev_begin, st)) != cudaSuccess) return e;
     switch (a.G) {

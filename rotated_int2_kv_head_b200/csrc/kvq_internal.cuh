@@ -271,9 +271,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---- host launchers (defined in kvq_append.cu / kvq_decode.cu) ---------------------------
 cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int mode,
                                 const float *R_k, const float *R_v, const int32_t *perm,
-                                const kvq_cache_desc &cd, const int32_t *seq_lens,
+                                const kvq_cache_desc &cd, int32_t *seq_lens,
                                 cudaStream_t st);
-cudaError_t launch_seq_bump(int32_t *seq_lens, int B, int T, int capacity, cudaStream_t st);
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
                                       const int32_t *perm, float *out, cudaStream_t st);
 cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
@@ -283,9 +282,9 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
                           cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
 
-// Decode workspace: prefix sums, prepared queries, sink partials, split partials.
+// Decode workspace: per-sequence block prefix sums, prepared queries, split partials.
 struct WsLayout {
-    size_t prefix, qprep, sinkp, part, total;
+    size_t prefix, qprep, part, total;
 };
 WsLayout ws_layout(int B, int Hq, int Hkv, int C);
 

@@ -125,7 +125,7 @@ class KVCache:
             self.v_sink = torch.zeros_like(self.k_sink)
         else:
             self.k_sink = self.v_sink = None
-        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.status = torch.zeros(2, dtype=torch.int32, device=device)   # errors, append counter
         self.desc = CacheDesc(B, Hkv, D, GROUP, capacity, sink_fp16, self.blocks.data_ptr(),
                               0 if self.k_sink is None else self.k_sink.data_ptr(),
                               0 if self.v_sink is None else self.v_sink.data_ptr(),
