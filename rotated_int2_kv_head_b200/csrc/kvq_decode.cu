@@ -8,29 +8,32 @@
 // Sinks are the leading positions stored in fp16 ("RotateKV", abstract item
 // (iii)).
 //
-// Two kernels:
+// Three kernels per call:
+//   decode_qprep_kernel     per (b, KV head): the G queries rotated by R_k
+//                           (or perm + FWHT) and split into int8 hi/lo per
+//                           group for the integer tensor cores.
 //   decode_split_kernel<G>  stream-K over all cache blocks of all (b, h)
 //                           units: every CTA takes an equal share of 16-token
 //                           blocks (the schedule is derived from seq_lens by
 //                           every CTA).  Thread 0 streams them into a
 //                           shared-memory ring with 1-D bulk copies (TMA);
-//                           the CTA rotates and quantises the unit's queries
-//                           while the first copies land; four warps run the
-//                           scores and P.V on tensor cores straight from the
-//                           packed codes with an online softmax; each (CTA,
-//                           unit) segment leaves one partial (m, l, o_rot[128])
-//                           per head.
+//                           four warps run the scores and P.V on tensor cores
+//                           straight from the packed codes with an online
+//                           softmax; each (CTA, unit) segment leaves one
+//                           partial (m, l, o_rot[128]) per head.
 //   decode_merge_kernel     per (b, query head): the sink partial (fp16 sinks,
 //                           fp32 CUDA cores), the merge of all partials, then
 //                           out = o_rot . R_v^T (or FWHT + inverse permutation).
 
-// Tensor-core operand trick.  A 2-bit code c sitting in bits [2g, 2g+1] of a
-// 16-bit lane, with every other bit zero, IS the fp16 subnormal c*4^g*2^-24.
-// So one AND turns a packed word into an m16n8k16 fragment register (two
-// codes); the 4^g*2^-24 factor is folded into a per-group fp32 scale
-// afterwards.  Products and sums stay exact or fp32: the query enters as an
-// fp16 hi/lo pair (two N columns), the softmax weights times V scales as fp16.
-// The dequantisation c*s + z is factored: sum_j q_j (c_j s + z) =
+// Tensor-core operand tricks.  Scores: a code byte masked with 0x03 << 2g is
+// the u8 value c*4^g, so one AND turns 4 packed bytes into an m16n8k32 IMMA
+// operand register; the query enters as an int8 hi/lo pair per group (about
+// 15 bits) and the products accumulate exactly in int32.  P.V: a 2-bit code
+// in bits [2g, 2g+1] of a 16-bit lane, every other bit zero, IS the fp16
+// subnormal c*4^g*2^-24, so one AND gives an m16n8k16 HMMA operand register
+// (two codes); the softmax weights times the fp16 V scales are the other
+// operand.  The 4^g factors are folded into per-group fp32 scales.  The
+// dequantisation c*s + z is factored: sum_j q_j (c_j s + z) =
 // s*sum_j q_j c_j + z*sum_j q_j, so only the integer codes go through the MMA.
 #include "kvq_internal.cuh"
 
@@ -58,7 +61,6 @@ struct DecodeArgs {
     const int32_t *perm;
     const int32_t *seq_lens;
     int32_t *status;
-    int32_t *prefix;   // [B+1] workspace, written by split CTA 0
     uint8_t *qprep;    // [B*Hq][QB] prepared queries
     float *part;       // [(C+U)*G][PART]
     uint16_t *out;
@@ -101,44 +103,41 @@ __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
 
 // CTA-wide (all DEC_THREADS threads): total block count N from seq_lens, this
 // CTA's range [c*W, min(N, (c+1)*W)) with W = ceil(N / C), and the unit that
-// holds its first block.  CTA 0 also writes prefix[0..B] for the merge.
-// scan: DEC_THREADS + 2 ints of shared scratch.  Returns false for an empty
-// range (uniformly over the CTA).
+// holds its first block.  Thread t covers a contiguous run of sequences; an
+// exclusive shuffle scan of the runs' block counts gives every run's offset.
+// scan: DEC_THREADS + 6 ints of shared scratch.  Returns false for an empty
+// range (uniformly over the CTA).  CTA 0 flags invalid lengths.
 __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scan) {
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
     const int lo = min(a.B, t * per), hi = min(a.B, lo + per);
     int sum = 0;
-    for (int b = lo; b < hi; b++) sum += a.Hkv * seq_blocks(a, b);
-    scan[t] = sum;
-    __syncthreads();
-    if (t == 0) {
-        int acc = 0;
-        for (int i = 0; i < DEC_THREADS; i++) {
-            const int v = scan[i];
-            scan[i] = acc;
-            acc += v;
-        }
-        scan[DEC_THREADS] = acc;
+    for (int b = lo; b < hi; b++) {
+        const int L = a.seq_lens[b];
+        if (blockIdx.x == 0 && (L < 1 || L > a.capacity)) set_status(a.status, KVQ_DEV_BAD_LEN);
+        sum += a.Hkv * unit_blocks(L, a.S, a.capacity);
     }
-    __syncthreads();
-    const int N = scan[DEC_THREADS];
-    if (blockIdx.x == 0) {
-        int acc = scan[t];
-        for (int b = lo; b < hi; b++) {
-            a.prefix[b] = acc;
-            const int L = a.seq_lens[b];
-            if (L < 1 || L > a.capacity) set_status(a.status, KVQ_DEV_BAD_LEN);
-            acc += a.Hkv * seq_blocks(a, b);
-        }
-        if (t == DEC_THREADS - 1) a.prefix[a.B] = N;
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
     }
+    int *wsum = scan + DEC_THREADS + 2;           // [DEC_WARPS]
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int woff = 0, N = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < DEC_WARPS; w2++) {
+        const int v = wsum[w2];
+        woff += (w2 < warp) ? v : 0;
+        N += v;
+    }
+    const int cstart = woff + incl - sum, cend = woff + incl;   // this thread's run
     const int W = max(1, (N + a.C - 1) / a.C);
     const int beg = blockIdx.x * W, end = min(N, beg + W);
     if (beg >= end) return false;
-    // the chunk holding block `beg` finds its sequence
-    const int cstart = scan[t], cend = (t == DEC_THREADS - 1) ? N : scan[t + 1];
-    __syncthreads();
+    // the run holding block `beg` finds its sequence
     if (cstart <= beg && beg < cend) {
         int acc = cstart;
         for (int b = lo; b < hi; b++) {
@@ -785,12 +784,13 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
 // Merge + rotate-out.
 // ---------------------------------------------------------------------------------------------
 constexpr int MRG_THREADS = 256;
-constexpr int MRG_MAXP = 512;     // partials merged per pass
+constexpr int MRG_BATCH = 32;     // partials loaded together
 
 __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a) {
     __shared__ __align__(16) float o_s[D];
     __shared__ __align__(16) float red[MRG_THREADS / 32][D];
-    __shared__ float pm[MRG_MAXP + 1], pl[MRG_MAXP + 1], wred[MRG_THREADS / 32];
+    __shared__ float wred[MRG_THREADS / 32];
+    __shared__ int ired[2 * (MRG_THREADS / 32)];
     __shared__ __align__(16) float qs[D];
     __shared__ float ssc[MAX_SINK];
     __shared__ __align__(16) float sinkp[PART];          // the sink partial: m, l, 0, 0, o[128]
@@ -876,12 +876,39 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         }
         __syncthreads();
     }
+    // This unit's place in the split kernel's block list, from seq_lens (the
+    // same arithmetic the split CTAs use): blocks of sequences before b, and
+    // in total.
+    {
+        int sb = 0, sn = 0;
+        for (int i = t; i < a.B; i += MRG_THREADS) {
+            const int nbi = a.Hkv * unit_blocks(a.seq_lens[i], a.S, a.capacity);
+            sn += nbi;
+            sb += i < b ? nbi : 0;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sb += __shfl_xor_sync(0xffffffffu, sb, off);
+            sn += __shfl_xor_sync(0xffffffffu, sn, off);
+        }
+        if (lane == 0) {
+            ired[warp] = sb;
+            ired[MRG_THREADS / 32 + warp] = sn;
+        }
+    }
     // R_v rows for the rotate-out (no kernel of this chain writes R_v)
     float4 rr[16];
     if (a.mode == KVQ_ROT_DENSE) {
         const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
 #pragma unroll
         for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+    }
+    __syncthreads();
+    int pre = 0, N = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < MRG_THREADS / 32; w2++) {
+        pre += ired[w2];
+        N += ired[MRG_THREADS / 32 + w2];
     }
     pdl_wait();
     pdl_trigger();
@@ -890,10 +917,9 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         return;
     }
     const int u = b * a.Hkv + h;
-    const int nb = (a.prefix[b + 1] - a.prefix[b]) / a.Hkv;
-    const int N = a.prefix[a.B];
+    const int nb = unit_blocks(L, a.S, a.capacity);
     const int W = max(1, (N + a.C - 1) / a.C);
-    const int ustart = a.prefix[b] + h * nb;
+    const int ustart = pre + h * nb;
     const int c0 = nb > 0 ? ustart / W : 0;
     const int np = nb > 0 ? (ustart + nb - 1) / W - c0 + 1 : 0;
     auto pptr = [&](int i) -> const float * {   // partial i (i == np: the sink partial)
@@ -901,39 +927,46 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     };
     const int ntot = np + (ns > 0 ? 1 : 0);
 
+    // Partials in batches of MRG_BATCH: warp w takes partials w, w+8, w+16,
+    // w+24 of the batch and issues all their loads before using any.
+    constexpr int PW = MRG_BATCH / (MRG_THREADS / 32);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f, mglob = NEG_INF;
-    for (int base = 0; base < ntot; base += MRG_MAXP) {
-        const int n = min(MRG_MAXP, ntot - base);
-        // (m, l) of every partial, then the running max
-        float mloc = NEG_INF;
-        for (int i = t; i < n; i += MRG_THREADS) {
-            const float *pp = pptr(base + i);
-            pm[i] = pp[0];
-            pl[i] = pp[1];
-            mloc = fmaxf(mloc, pp[0]);
-        }
+    for (int base = 0; base < ntot; base += MRG_BATCH) {
+        float2 ml[PW];
+        float4 o4[PW];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+        for (int j = 0; j < PW; j++) {
+            const int i = base + warp + j * (MRG_THREADS / 32);
+            if (i < ntot) {
+                const float *pp = pptr(i);
+                ml[j] = make_float2(pp[0], pp[1]);
+                o4[j] = *reinterpret_cast<const float4 *>(pp + 4 + 4 * lane);
+            } else {
+                ml[j] = make_float2(NEG_INF, 0.f);
+                o4[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        float mloc = NEG_INF;
+#pragma unroll
+        for (int j = 0; j < PW; j++) mloc = fmaxf(mloc, ml[j].x);
         if (lane == 0) wred[warp] = mloc;
         __syncthreads();
         float mnew = mglob;
 #pragma unroll
         for (int w2 = 0; w2 < MRG_THREADS / 32; w2++) mnew = fmaxf(mnew, wred[w2]);
+        __syncthreads();
         const float fold = (mglob == NEG_INF) ? 0.f : exp2f(mglob - mnew);
         acc.x *= fold; acc.y *= fold; acc.z *= fold; acc.w *= fold;
         lsum *= fold;
         mglob = mnew;
-        // o: warp w sums partials w, w+8, ...; lane l holds elements 4l..4l+3
-        for (int i = warp; i < n; i += MRG_THREADS / 32) {
-            const float mi = pm[i];
-            const float f = (mi == NEG_INF) ? 0.f : exp2f(mi - mglob);
-            const float4 o4 = *reinterpret_cast<const float4 *>(pptr(base + i) + 4 + 4 * lane);
-            acc.x = fmaf(f, o4.x, acc.x); acc.y = fmaf(f, o4.y, acc.y);
-            acc.z = fmaf(f, o4.z, acc.z); acc.w = fmaf(f, o4.w, acc.w);
-            lsum = fmaf(f, pl[i], lsum);
+#pragma unroll
+        for (int j = 0; j < PW; j++) {
+            const float f = (ml[j].x == NEG_INF) ? 0.f : exp2f(ml[j].x - mglob);
+            acc.x = fmaf(f, o4[j].x, acc.x); acc.y = fmaf(f, o4[j].y, acc.y);
+            acc.z = fmaf(f, o4[j].z, acc.z); acc.w = fmaf(f, o4[j].w, acc.w);
+            lsum = fmaf(f, ml[j].y, lsum);
         }
-        __syncthreads();
     }
     *reinterpret_cast<float4 *>(&red[warp][4 * lane]) = acc;
     if (lane == 0) wred[warp] = lsum;
@@ -983,8 +1016,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     WsLayout w;
     const int G = Hq / Hkv;
-    w.prefix = 0;
-    w.qprep = up(w.prefix + sizeof(int32_t) * (B + 1));
+    w.qprep = 0;
     w.part = up(w.qprep + (size_t)B * Hq * QB);
     w.total = up(w.part + sizeof(float) * ((size_t)C + (size_t)B * Hkv) * G * PART);
     return w;
@@ -1015,7 +1047,6 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.perm = perm;
     a.seq_lens = seq_lens;
     a.status = cd.status;
-    a.prefix = reinterpret_cast<int32_t *>(base + w.prefix);
     a.qprep = base + w.qprep;
     a.part = reinterpret_cast<float *>(base + w.part);
     a.out = out;

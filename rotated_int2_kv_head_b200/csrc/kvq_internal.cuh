@@ -282,9 +282,9 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
                           cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
 
-// Decode workspace: per-sequence block prefix sums, prepared queries, split partials.
+// Decode workspace: prepared queries and split partials.
 struct WsLayout {
-    size_t prefix, qprep, part, total;
+    size_t qprep, part, total;
 };
 WsLayout ws_layout(int B, int Hq, int Hkv, int C);
 
