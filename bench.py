@@ -12,14 +12,19 @@ tensors (workloads.py).
     python bench.py --impl reference ...      # the CPU oracle as reference arm
     torchrun --nproc-per-node N bench.py --gpus N ...
 
-Timing: every step is bracketed by CUDA events on the launching stream; an
-L2 flush and the reset of the sequence length to its pre-append value happen
-between steps, outside the events, so each step starts cold and at the same
-context.  The flush writes a 256 MB buffer and then reads another 256 MB one:
-a write alone would leave L2 full of dirty lines whose write-back the next
-timed kernel would pay for.  K steps run back to back between a
-barrier + synchronize on both sides; the device time is summed per rank and
-the max over ranks is reported.  With N GPUs every rank serves its own
+Timing: K steps run back to back on the launching stream between one pair
+of CUDA events, with a barrier + synchronize on both sides; the max over
+ranks is reported.  L2 (126 MB) must not serve the cache across steps: a
+cache smaller than 3x L2 is replicated into independent layers (distinct
+memory, same contents, like the layers of a model) that the steps cycle
+through, so every step reads a cache that at least 3x L2 of other cache
+traffic has passed through L2 since its last use.  Each step appends at the
+same position (its own row of pre-append lengths), so the context is the
+same for every step.  A cache too small for 64 layers to cover that falls
+back to flushing L2 between steps (256 MB written, then 256 MB read, so L2
+holds clean lines) with each step bracketed by its own events.  The
+isolated-step latency (flush, then one step between its own events) is
+reported beside the throughput.  With N GPUs every rank serves its own
 independent batch (weak scaling, no collective on the data path).
 
 Prints one JSON line (rank 0).
@@ -44,6 +49,8 @@ import workloads as W  # noqa: E402
 METRIC = "INT2-KV decode attention tokens/s and packed-KV GB/s (% of HBM peak), 1 B200"
 KERNELS_PER_STEP = 4      # append (with the length update), query preparation, decode split, merge
 FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20      # B200 L2
+MAX_LAYERS = 64
 
 
 class L2Flush:
@@ -205,10 +212,27 @@ def packed_kv_bytes(w, lens):
 
 # --- the CUDA arm ---------------------------------------------------------------------------------
 
-class Step:
-    """One pass of the hot path: append the new tokens, decode."""
+def layers_for(cache_bytes):
+    """How many independent layers to cycle so that, with no flush, each step
+    reads a cache that the steps since its last use have pushed out of L2
+    (at least 3x L2 of other cache traffic in between); 0 = too small for
+    that, flush L2 between steps instead."""
+    if cache_bytes >= 3 * L2_BYTES:
+        return 1
+    n = -(-3 * L2_BYTES // cache_bytes) + 1
+    return n if n <= MAX_LAYERS else 0
 
-    def __init__(self, w, device, seed_rank=0):
+
+class Step:
+    """One pass of the hot path: append the step's new tokens to one layer's
+    cache, then decode over it.  With n_layers > 1 the layers are
+    independent copies (cache, rotations: same contents, distinct memory)
+    used round robin, like the layers of a model; the new K/V rows and the
+    queries are shared.  Sequence lengths come from a caller-provided row
+    holding the pre-append lengths, so every step runs at the same context
+    without a reset kernel."""
+
+    def __init__(self, w, device, n_layers=1):
         import rotated_int2_kv_head_b200 as kvq
         self.kvq, self.w, self.dev = kvq, w, device
         lens = w.seq_lens()
@@ -216,49 +240,54 @@ class Step:
         self.T = w.append_T
         self.cap = ((self.L + 15) // 16) * 16
         Rk, Rv, perm = W.rotations(w)
-        self.Rk = torch.from_numpy(Rk).to(device) if Rk is not None else None
-        self.Rv = torch.from_numpy(Rv).to(device) if Rv is not None else None
-        self.perm = torch.from_numpy(perm).to(device) if perm is not None else None
         self.rot_np = (Rk, Rv, perm)
-        self.cache = kvq.KVCache(w.B, w.Hkv, self.cap, w.sink, device=device)
-        self.len_full = torch.from_numpy(lens.astype(np.int32)).to(device)
-        self.len_base = self.len_full - self.T           # before the step's append
-        self.seq_lens = self.len_base.clone()
+        Rk = torch.from_numpy(Rk).to(device) if Rk is not None else None
+        Rv = torch.from_numpy(Rv).to(device) if Rv is not None else None
+        perm = torch.from_numpy(perm).to(device) if perm is not None else None
+        cache = kvq.KVCache(w.B, w.Hkv, self.cap, w.sink, device=device)
+        self.len_base = torch.from_numpy(lens.astype(np.int32)).to(device) - self.T
         # prefill [0, L - T) on the GPU, in chunks, all sequences together
         pre = self.L - self.T
         fill = torch.zeros(w.B, dtype=torch.int32, device=device)
-        ch = 2048
-        for t0 in range(0, pre, ch):
-            t1 = min(pre, t0 + ch)
+        for t0 in range(0, pre, 2048):
+            t1 = min(pre, t0 + 2048)
             K, V = W.kv_batch(w, t0, t1, device)
-            kvq.kvq_rotate_quantize_append(K, V, w.mode, self.Rk, self.Rv, self.perm, self.cache,
-                                           fill)
+            kvq.kvq_rotate_quantize_append(K, V, w.mode, Rk, Rv, perm, cache, fill)
+        torch.cuda.synchronize(device)
+        if kvq.kvq_get_status(cache) != 0:
+            raise RuntimeError("cache fill flagged device status %d" % kvq.kvq_get_status(cache))
+        self.layers = [(cache, Rk, Rv, perm)]
+        for _ in range(1, n_layers):
+            c2 = kvq.KVCache(w.B, w.Hkv, self.cap, w.sink, device=device)
+            c2.blocks.copy_(cache.blocks)
+            if cache.k_sink is not None:
+                c2.k_sink.copy_(cache.k_sink)
+                c2.v_sink.copy_(cache.v_sink)
+            self.layers.append((c2, *(None if x is None else x.clone() for x in (Rk, Rv, perm))))
         self.Knew, self.Vnew = W.kv_batch(w, pre, self.L, device)
         self.Q = W.queries(w, device)
         self.out = torch.empty_like(self.Q)
         self.ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, self.L, device=device)
         torch.cuda.synchronize(device)
-        st = kvq.kvq_get_status(self.cache)
-        if st != 0:
-            raise RuntimeError("cache fill flagged device status %d" % st)
-        self.ev_split = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        for e in self.ev_split:
-            e.record()
+        self.cache_bytes = cache.blocks.numel()
 
-    def reset(self):
-        self.seq_lens.copy_(self.len_base)
+    def lengths(self, n):
+        """n rows of pre-append sequence lengths, one per step."""
+        return self.len_base.repeat(n, 1).contiguous()
 
-    def run(self, timed_split=False):
+    def run(self, k, seq_lens, split_events=None):
         kvq, w = self.kvq, self.w
-        kvq.kvq_rotate_quantize_append(self.Knew, self.Vnew, w.mode, self.Rk, self.Rv, self.perm,
-                                       self.cache, self.seq_lens)
-        if timed_split:
-            kvq.kvq_decode_attention_timed(self.Q, self.cache, w.mode, self.Rk, self.Rv, self.perm,
-                                           self.seq_lens, w.sink, self.L, self.ws, self.out,
-                                           self.ev_split[0], self.ev_split[1])
+        cache, Rk, Rv, perm = self.layers[k % len(self.layers)]
+        kvq.kvq_rotate_quantize_append(self.Knew, self.Vnew, w.mode, Rk, Rv, perm, cache, seq_lens)
+        if split_events is not None:
+            kvq.kvq_decode_attention_timed(self.Q, cache, w.mode, Rk, Rv, perm, seq_lens, w.sink,
+                                           self.L, self.ws, self.out, *split_events)
         else:
-            kvq.kvq_decode_attention(self.Q, self.cache, w.mode, self.Rk, self.Rv, self.perm,
-                                     self.seq_lens, w.sink, self.L, self.ws, self.out)
+            kvq.kvq_decode_attention(self.Q, cache, w.mode, Rk, Rv, perm, seq_lens, w.sink, self.L,
+                                     self.ws, self.out)
+
+    def status(self):
+        return max(self.kvq.kvq_get_status(c[0]) for c in self.layers)
 
 
 def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
@@ -308,42 +337,50 @@ def run_cuda(args):
     from rotated_int2_kv_head_b200 import build as kbuild
     kbuild.build()
     w = rank_workload(W.WORKLOADS[args.workload], rank)
-    step = Step(w, dev)
-    flush = L2Flush(dev)
     lens = w.seq_lens()
-
-    def one(k, timed_split, evs=None):
-        flush(k)
-        step.reset()
-        if evs:
-            evs[0].record()
-        step.run(timed_split)
-        if evs:
-            evs[1].record()
-
-    for k in range(args.warmup):
-        one(k, True)
-    torch.cuda.synchronize(dev)
+    cap = ((int(lens.max()) + 15) // 16) * 16
+    n_layers = layers_for(w.B * w.Hkv * (cap // 16) * 1536)
+    step = Step(w, dev, max(1, n_layers))
+    flush = L2Flush(dev) if n_layers == 0 else None
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+
+    def steps(n, sl, timed=None, split_events=None):
+        """n steps; with `timed`, one event pair around all of them (layers
+        mode) or around each (flush mode, the flush outside the events)."""
+        ms = 0.0
+        if flush is None and timed is not None:
+            timed[0].record()
+        for k in range(n):
+            if flush is not None:
+                flush(k)
+                if timed is not None:
+                    timed[0].record()
+            step.run(k, sl[k], None if split_events is None else split_events[k])
+            if flush is not None and timed is not None:
+                timed[1].record()
+                torch.cuda.synchronize(dev)
+                ms += timed[0].elapsed_time(timed[1])
+        if flush is None and timed is not None:
+            timed[1].record()
+            torch.cuda.synchronize(dev)
+            ms = timed[0].elapsed_time(timed[1])
+        return ms
+
+    steps(args.warmup, step.lengths(args.warmup))
+    torch.cuda.synchronize(dev)
+    sl = step.lengths(K)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     with ClockSampler(local) as clk:
         barrier(dist_on, dev)
         torch.cuda.synchronize(dev)
-        for k in range(K):
-            flush(k)
-            step.reset()
-            ev[k][0].record()
-            step.run(False)
-            ev[k][1].record()
+        total_ms = steps(K, sl, ev)
         torch.cuda.synchronize(dev)
         barrier(dist_on, dev)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), dist_on, dev)
+    total_ms = max_over_ranks(total_ms, dist_on, dev)
 
     # the streaming kernel alone, timed live by events the library records
     # around it (a separate loop: events between kernels stop the
-    # programmatic overlap of the timed steps above)
+    # programmatic overlap of the steps above)
     n_split = min(K, 300)
     split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(n_split)]
@@ -351,16 +388,26 @@ def run_cuda(args):
         for e in pair:
             e.record()
     torch.cuda.synchronize(dev)
-    for k in range(n_split):
-        flush(k)
-        step.reset()
-        step.ev_split = split_ev[k]
-        step.run(True)
+    steps(n_split, step.lengths(n_split), None, split_ev)
     torch.cuda.synchronize(dev)
-    split_ms = [a.elapsed_time(b) for a, b in split_ev]
-    st = step.kvq.kvq_get_status(step.cache)
-    if st != 0:
-        raise RuntimeError("device status %d after timed steps" % st)
+    split_ms = [x.elapsed_time(y) for x, y in split_ev]
+
+    # one step at a time after an L2 flush, each bracketed by its own events
+    # (the latency of an isolated step, for reference)
+    n_iso = min(K, 200)
+    iso_flush = flush or L2Flush(dev)
+    sl_iso = step.lengths(n_iso)
+    iso_ms = []
+    for k in range(n_iso):
+        iso_flush(k)
+        ev[0].record()
+        step.run(k, sl_iso[k])
+        ev[1].record()
+        torch.cuda.synchronize(dev)
+        iso_ms.append(ev[0].elapsed_time(ev[1]))
+    del iso_flush
+    if step.status() != 0:
+        raise RuntimeError("device status %d after timed steps" % step.status())
 
     # end to end through the public API with host buffers: H2D of the step's
     # new K/V and queries from pinned memory, append + decode, D2H of the output
@@ -369,16 +416,17 @@ def run_cuda(args):
     hQ = step.Q.cpu().pin_memory()
     hO = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     n_e2e = min(K, 200)
+    sl_e2e = step.lengths(n_e2e + 3)
     e2e_s = 0.0
     for k in range(n_e2e + 3):
-        flush(k)
-        step.reset()
+        if flush is not None:
+            flush(k)
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
         step.Knew.copy_(hK, non_blocking=True)
         step.Vnew.copy_(hV, non_blocking=True)
         step.Q.copy_(hQ, non_blocking=True)
-        step.run(False)
+        step.run(k, sl_e2e[k])
         hO.copy_(step.out, non_blocking=True)
         torch.cuda.synchronize(dev)
         if k >= 3:
@@ -398,6 +446,15 @@ def run_cuda(args):
     achieved = kv_bytes / split_mean_s / 1e9
     ms_per_step = total_ms / K
     tokens = w.B * world
+    if n_layers == 0:
+        l2_note = "flushed between steps (256 MB write, then 256 MB read); steps timed one by one"
+    else:
+        l2_note = ("inputs larger than L2: %d independent layers (%.1f MB of cache each) cycled, "
+                   "so each step reads a cache %d other steps (%.0f MB) after its last use; "
+                   "steps back to back" % (n_layers, step.cache_bytes / 1e6, n_layers - 1,
+                                           (n_layers - 1) * step.cache_bytes / 1e6)
+                   if n_layers > 1 else "inputs larger than L2 (one %.0f MB cache); steps back "
+                   "to back" % (step.cache_bytes / 1e6))
     line = {
         "metric": METRIC,
         "value": tokens * K / (total_ms * 1e-3),
@@ -414,7 +471,7 @@ def run_cuda(args):
         "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
                    "context": int(lens.max()), "append_T": w.append_T,
                    "rotation": "dense" if w.mode == 0 else "perm+fwht", "sink_fp16": w.sink,
-                   "group": 32, "l2": "flushed between steps (256 MB write, then 256 MB read)",
+                   "group": 32, "l2": l2_note, "layers": max(1, n_layers),
                    "parallelism": "replicas: one independent batch per GPU"},
         "packed_kv_gbs": kv_bytes / (ms_per_step * 1e-3) / 1e9,
         "packed_kv_bytes_per_step": kv_bytes,
@@ -426,6 +483,8 @@ def run_cuda(args):
         "e2e": {"value": tokens * n_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "how": "wall clock per step incl. pinned H2D of new "
                                                   "K/V/Q and D2H of the output, synchronised"},
+        "isolated_step": {"ms": float(np.median(iso_ms)), "how": "median of %d steps, each after "
+                          "an L2 flush and bracketed by its own events" % n_iso},
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clk.summary(),
     }
