@@ -10,8 +10,8 @@ using namespace kvq;
 
 namespace {
 
-constexpr int SPLIT_CTAS_PER_SM = 4;     // resident split CTAs per SM (launch bounds)
-constexpr int MIN_BLOCKS_PER_CTA = 16;   // 256 tokens: below this, fewer CTAs
+constexpr int SPLIT_CTAS_PER_SM = 1;     // one split CTA (four groups) per SM
+constexpr int MIN_BLOCKS_PER_CTA = 64;   // 1024 tokens: below this, fewer CTAs
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 

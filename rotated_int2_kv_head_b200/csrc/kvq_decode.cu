@@ -39,12 +39,17 @@
 
 namespace kvq {
 
-constexpr int DEC_WARPS = 4;                              // consumer warps; warp 0 lane 0 also issues copies
-constexpr int DEC_THREADS = 32 * DEC_WARPS;
-constexpr int SPLIT_MIN_CTAS = 4;                         // resident CTAs per SM
-constexpr int STAGE_BLKS = 2 * DEC_WARPS;                 // 8 blocks = 128 tokens
+// Split kernel: one CTA per SM made of DEC_GROUPS independent groups of
+// GROUP_WARPS warps; each group streams its own ring of stages.
+constexpr int DEC_GROUPS = 4;
+constexpr int GROUP_WARPS = 4;
+constexpr int GROUP_THREADS = 32 * GROUP_WARPS;           // 128
+constexpr int DEC_THREADS = DEC_GROUPS * GROUP_THREADS;   // 512
+constexpr int DEC_WARPS = DEC_GROUPS * GROUP_WARPS;       // 16
+constexpr int STAGE_BLKS = 2 * GROUP_WARPS;               // 8 blocks = 128 tokens
 constexpr int STAGE_BYTES = STAGE_BLKS * BLK_BYTES;       // 12 KB
-constexpr int NSTAGE = 4;
+// ring slots per group (the flush scratch grows with G)
+__host__ __device__ constexpr int nstage_for(int G) { return G >= 4 ? 3 : 4; }
 // Prepared query per query head, QB bytes:
 //   int8 hi[128], int8 lo[128]  with q_s ~= sq_g * (hi + lo/254) per group g
 //   float kap[4] = sq_g / 4^g,  float qsum[4] = sum of q_s over group g
@@ -102,12 +107,15 @@ __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
 }
 
 // CTA-wide (all DEC_THREADS threads): total block count N from seq_lens, this
-// CTA's range [c*W, min(N, (c+1)*W)) with W = ceil(N / C), and the unit that
-// holds its first block.  Thread t covers a contiguous run of sequences; an
-// exclusive shuffle scan of the runs' block counts gives every run's offset.
-// scan: DEC_THREADS + 6 ints of shared scratch.  Returns false for an empty
-// range (uniformly over the CTA).  CTA 0 flags invalid lengths.
-__device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scan) {
+// CTA's range [c*W, min(N, (c+1)*W)) with W = ceil(N / C), split into
+// DEC_GROUPS contiguous parts, and for each part the unit holding its first
+// block: group g gets s (an empty range when the CTA's range is short).
+// Thread t covers a contiguous run of sequences; an exclusive shuffle scan
+// of the runs' block counts gives every run's offset.  scratch:
+// 2*DEC_GROUPS + DEC_WARPS ints of shared memory.  Returns false when the
+// CTA's range is empty (uniformly over the CTA).  CTA 0 flags invalid
+// lengths.
+__device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
     const int lo = min(a.B, t * per), hi = min(a.B, lo + per);
@@ -123,7 +131,7 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scan) {
         const int v = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += v;
     }
-    int *wsum = scan + DEC_THREADS + 2;           // [DEC_WARPS]
+    int *wsum = scratch + 2 * DEC_GROUPS;         // [DEC_WARPS]
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     int woff = 0, N = 0;
@@ -137,28 +145,55 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scan) {
     const int W = max(1, (N + a.C - 1) / a.C);
     const int beg = blockIdx.x * W, end = min(N, beg + W);
     if (beg >= end) return false;
-    // the run holding block `beg` finds its sequence
-    if (cstart <= beg && beg < cend) {
-        int acc = cstart;
-        for (int b = lo; b < hi; b++) {
-            const int nbb = a.Hkv * seq_blocks(a, b);
-            if (beg < acc + nbb) {
-                scan[DEC_THREADS] = b;
-                scan[DEC_THREADS + 1] = acc;
-                break;
+    const int Wg = (end - beg + DEC_GROUPS - 1) / DEC_GROUPS;
+    // the run holding each part's first block finds its sequence
+#pragma unroll
+    for (int g = 0; g < DEC_GROUPS; g++) {
+        const int p = beg + g * Wg;
+        if (p < end && cstart <= p && p < cend) {
+            int acc = cstart;
+            for (int b = lo; b < hi; b++) {
+                const int nbb = a.Hkv * seq_blocks(a, b);
+                if (p < acc + nbb) {
+                    scratch[2 * g] = b;
+                    scratch[2 * g + 1] = acc;
+                    break;
+                }
+                acc += nbb;
             }
-            acc += nbb;
         }
     }
     __syncthreads();
-    s.b = scan[DEC_THREADS];
-    s.pref = scan[DEC_THREADS + 1];
-    s.nb = seq_blocks(a, s.b);
-    s.h = (beg - s.pref) / s.nb;
-    s.ustart = s.pref + s.h * s.nb;
-    s.cur = beg;
-    s.end = end;
+    const int g = threadIdx.x / GROUP_THREADS;
+    const int p = beg + g * Wg;
+    if (p < end) {
+        s.b = scratch[2 * g];
+        s.pref = scratch[2 * g + 1];
+        s.nb = seq_blocks(a, s.b);
+        s.h = (p - s.pref) / s.nb;
+        s.ustart = s.pref + s.h * s.nb;
+        s.cur = p;
+        s.end = min(end, p + Wg);
+    } else {
+        s.b = s.h = s.nb = s.ustart = s.pref = 0;
+        s.cur = s.end = 0;
+    }
     __syncthreads();
+    return true;
+}
+
+// Next stage of a group's own range (up to STAGE_BLKS blocks, never crossing
+// a unit); false when the range is exhausted.  Leader thread only.
+__device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &unit, int &b,
+                                           int &h, int &kblk, int &n) {
+    if (ps.cur >= ps.end) return false;
+    sched_fix_unit(ps, a);
+    n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
+    unit = ps.b * a.Hkv + ps.h;
+    b = ps.b;
+    h = ps.h;
+    kblk = ps.cur - ps.ustart;
+    ps.cur += n;
     return true;
 }
 
@@ -187,6 +222,15 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
     }
     pdl_wait();
     pdl_trigger();
+    // mark every split partial empty (m = -inf, l = 0): a group of the split
+    // kernel writes only the units it took stages of
+    {
+        const size_t nslots = (size_t)DEC_GROUPS * ((size_t)a.C + (size_t)a.B * a.Hkv) * G;
+        const size_t stride = (size_t)gridDim.x * gridDim.y * QP_THREADS;
+        for (size_t i = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * QP_THREADS + t; i < nslots;
+             i += stride)
+            *reinterpret_cast<float2 *>(a.part + i * PART) = make_float2(NEG_INF, 0.f);
+    }
     for (int hd = 0; hd < G; hd++) {
         const int hq = h * G + hd;
         const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
@@ -301,53 +345,61 @@ __device__ __forceinline__ void wsrc(int c, int k, int &g, int &head) {
     else { g = k & 3; head = c + 4 * (k >> 2); }
 }
 
-// Shared-memory carve-out of the split kernel: every piece starts on a
-// 16-byte boundary (descriptors are read as int4).
+// Shared-memory carve-out of the split kernel: DEC_GROUPS group regions of
+// `gstride` bytes (ring, stage barriers, descriptors, flush scratch), then
+// the schedule scratch.  Every piece starts on a
+// 16-byte boundary (descriptors are read as int4, copies land 16-B aligned).
 struct SplitSmem {
-    unsigned full, cnt, desc, psm, qsm, fo, fm, fl, fz, abort, total;
+    unsigned full, desc, fo, fm, fl, fz, gstride, scratch, total;
 };
 __host__ __device__ constexpr unsigned smem_up16(unsigned x) { return (x + 15u) & ~15u; }
 __host__ __device__ inline SplitSmem split_smem_layout(int G) {
+    const unsigned ns = nstage_for(G);
     SplitSmem L{};
-    L.full = NSTAGE * STAGE_BYTES;
-    L.cnt = smem_up16(L.full + NSTAGE * 8u);
-    L.desc = smem_up16(L.cnt + NSTAGE * 4u);
-    L.psm = smem_up16(L.desc + 2u * NSTAGE * 16u);
-    L.qsm = smem_up16(L.psm + 32u);
-    L.fo = L.qsm;
-    L.fm = smem_up16(L.fo + 4u * DEC_WARPS * G * D);
-    L.fl = smem_up16(L.fm + 4u * DEC_WARPS * G);
-    L.fz = smem_up16(L.fl + 4u * DEC_WARPS * G);
-    L.abort = smem_up16(L.fz + 4u * DEC_WARPS * G * 4);
-    L.total = smem_up16(L.abort + 4u);
+    L.full = ns * STAGE_BYTES;                                   // ring at offset 0
+    L.desc = smem_up16(L.full + ns * 8u);
+    L.fo = smem_up16(L.desc + 2u * ns * 16u);
+    L.fm = smem_up16(L.fo + 4u * GROUP_WARPS * G * D);
+    L.fl = smem_up16(L.fm + 4u * GROUP_WARPS * G);
+    L.fz = smem_up16(L.fl + 4u * GROUP_WARPS * G);
+    L.gstride = (L.fz + 4u * GROUP_WARPS * G * 4 + 127u) & ~127u;
+    L.scratch = DEC_GROUPS * L.gstride;
+    L.total = smem_up16(L.scratch + 4u * (2 * DEC_GROUPS + DEC_WARPS));
     return L;
 }
 
+// Index of the partial a group writes for a unit: (CTA, unit) pairs of a
+// static contiguous split never collide under c + u, and each has one slot
+// per group.
+__host__ __device__ inline size_t part_slot(int cta, int unit, int grp) {
+    return (size_t)DEC_GROUPS * ((size_t)cta + unit) + grp;
+}
+
 template <int G>
-__global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs a) {
     using C = Cfg<G>;
+    constexpr int NS = nstage_for(G);
     constexpr int NW = G;                              // weight registers per lane per block
     constexpr int NGL = G == 1 ? 1 : (G == 2 ? 2 : 4); // V-meta groups a lane reads
     extern __shared__ __align__(128) uint8_t smem[];
-    SplitSmem L = split_smem_layout(G);
-    uint8_t *ring = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full);     // [NSTAGE]
-    int *cnt = reinterpret_cast<int *>(smem + L.cnt);                 // [NSTAGE]
-    int4 *desc = reinterpret_cast<int4 *>(smem + L.desc);             // [2*NSTAGE] stage descriptors
-    Sched *psm = reinterpret_cast<Sched *>(smem + L.psm);             // producer schedule state
-    float *fo = reinterpret_cast<float *>(smem + L.fo);               // [W][G][128]; also scratch
-    float *fm = reinterpret_cast<float *>(smem + L.fm);               // [W][G]
-    float *fl = reinterpret_cast<float *>(smem + L.fl);               // [W][G]
-    float *fz = reinterpret_cast<float *>(smem + L.fz);               // [W][G][4]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
+    const SplitSmem L = split_smem_layout(G);
+    const int grp = threadIdx.x / GROUP_THREADS, gt = threadIdx.x % GROUP_THREADS;
+    const int warp = gt >> 5, lane = threadIdx.x & 31;        // warp within the group
+    const bool leader = gt == 0;
+    uint8_t *gbase = smem + grp * L.gstride;
+    uint8_t *ring = gbase;                                            // [NS][STAGE_BYTES]
+    uint64_t *full = reinterpret_cast<uint64_t *>(gbase + L.full);    // [NS]
+    int4 *desc = reinterpret_cast<int4 *>(gbase + L.desc);            // [2*NS] stage descriptors
+    float *fo = reinterpret_cast<float *>(gbase + L.fo);              // [W][G][128]
+    float *fm = reinterpret_cast<float *>(gbase + L.fm);              // [W][G]
+    float *fl = reinterpret_cast<float *>(gbase + L.fl);              // [W][G]
+    float *fz = reinterpret_cast<float *>(gbase + L.fz);              // [W][G][4]
+    int *scratch = reinterpret_cast<int *>(smem + L.scratch);
+    // named barrier of this group (id 0 is __syncthreads)
+    auto bar_group = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(GROUP_THREADS) : "memory"); };
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NSTAGE; s++) {
-            mbar_init(&full[s], 1);
-            cnt[s] = 0;
-        }
-        *abort_flag = 0;
+    if (leader) {
+        for (int k = 0; k < NS; k++) mbar_init(&full[k], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -355,43 +407,41 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
     // kernel waited on it before letting this kernel launch), so seq_lens and
     // the cache are read - and the first copies issued - before waiting on
     // the prepared queries.
-    Sched sc;
-    if (!sched_init_cta(sc, a, reinterpret_cast<int *>(fo))) {
+    Sched sc;   // this group's part of the CTA's range (leader's copy is the producer state)
+    if (!sched_init_cta(sc, a, scratch)) {
         pdl_wait();
         pdl_trigger();
         return;
     }
     const int fb = a.S / BLK_TOK;
 
-    // Copies.  Thread 0 keeps the producer state (the schedule NSTAGE stages
-    // ahead of the consumers) in shared memory; when all warps have released
-    // a ring slot it issues the next stage into it and writes that stage's
-    // descriptor:
-    //   {unit, b, h, first cache block}, n blocks | flags << 8
-    // flags: 1 = last stage of this CTA's segment of the unit, 2 = last stage
-    // of the CTA.  Consumers read descriptors instead of running the schedule.
+    // Copies.  The group leader fills ring slot `slot` with the next stage of
+    // the group's range and writes its descriptor {unit, b, h, first cache
+    // block}, {n}; unit -1 marks the end (the slot's phase is completed by a
+    // plain arrive).  Descriptors are written NS-1 group barriers before
+    // anyone reads them, so they are read without waiting on the copy.
+    int issued = 0;      // leader: stages issued (= the iteration they belong to)
+    bool ended = false;  // leader: the end marker is written
     auto issue_next = [&](int slot) {
-        Sched ps = *psm;
-        if (ps.cur >= ps.end) return;
-        sched_fix_unit(ps, a);
-        const int n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
-        const int unit = ps.b * a.Hkv + ps.h;
-        const int kblk = fb + (ps.cur - ps.ustart);
-        ps.cur += n;
-        const int flags = (ps.cur == ps.ustart + ps.nb || ps.cur == ps.end ? 1 : 0) |
-                          (ps.cur == ps.end ? 2 : 0);
-        desc[2 * slot] = make_int4(unit, ps.b, ps.h, kblk);
-        desc[2 * slot + 1] = make_int4(n | (flags << 8), 0, 0, 0);
-        *psm = ps;
-        mbar_arrive_expect_tx(&full[slot], n * BLK_BYTES);
-        bulk_g2s(ring + slot * STAGE_BYTES,
-                 a.blocks + ((size_t)unit * a.nblk + kblk) * (size_t)BLK_BYTES, n * BLK_BYTES,
-                 &full[slot]);
+        if (ended) return;
+        int unit = 0, b = 0, h = 0, kblk = 0, n = 0;
+        if (sched_take(sc, a, unit, b, h, kblk, n)) {
+            desc[2 * slot] = make_int4(unit, b, h, fb + kblk);
+            desc[2 * slot + 1] = make_int4(n, 0, 0, 0);
+            mbar_arrive_expect_tx(&full[slot], n * BLK_BYTES);
+            bulk_g2s(ring + slot * STAGE_BYTES,
+                     a.blocks + ((size_t)unit * a.nblk + fb + kblk) * (size_t)BLK_BYTES,
+                     n * BLK_BYTES, &full[slot]);
+        } else {
+            desc[2 * slot] = make_int4(-1, 0, 0, 0);
+            mbar_arrive(&full[slot]);
+            ended = true;
+        }
+        ++issued;
     };
-    if (threadIdx.x == 0) {
-        *psm = sc;
-        for (int k = 0; k < NSTAGE; k++) issue_next(k);
-    }
+    if (leader)
+        for (int k = 0; k < NS; k++) issue_next(k);
+    bar_group();
     pdl_wait();
     pdl_trigger();
 
@@ -494,15 +544,15 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                         wo[head * D + j] = O[g * 2 + h2][k] * __int_as_float((127 + 24 - 2 * g) << 23);
                     }
                 }
-        __syncthreads();
-        const int tj = threadIdx.x;   // 0..127: element
+        bar_group();
+        const int tj = gt;            // 0..127: element
         for (int head = 0; head < G; head++) {
             float ms = NEG_INF;
 #pragma unroll
-            for (int w = 0; w < DEC_WARPS; w++) ms = fmaxf(ms, fm[w * G + head]);
+            for (int w = 0; w < GROUP_WARPS; w++) ms = fmaxf(ms, fm[w * G + head]);
             float acc = 0.f, lsum = 0.f;
 #pragma unroll
-            for (int w = 0; w < DEC_WARPS; w++) {
+            for (int w = 0; w < GROUP_WARPS; w++) {
                 const float mw = fm[w * G + head];
                 const float f = (mw == NEG_INF) ? 0.f : exp2f(mw - ms);
                 acc = fmaf(f, fo[(w * G + head) * D + tj] + fz[(w * G + head) * 4 + (tj >> 5)], acc);
@@ -515,269 +565,288 @@ __global__ void __launch_bounds__(DEC_THREADS, SPLIT_MIN_CTAS) decode_split_kern
                 dst[1] = lsum;
             }
         }
-        __syncthreads();
+        bar_group();
     };
 
     reset_state();
-    for (int it = 0;; ++it) {
-        const int s = it % NSTAGE;
-        const bool ok = mbar_wait_bounded(&full[s], (it / NSTAGE) & 1);
-        if (!ok || *abort_flag) {
-            if (lane == 0) set_status(a.status, KVQ_DEV_TIMEOUT);
-            *abort_flag = 1;
-            break;
-        }
+    bool aborted = false;
+    int it = 0;
+    for (;; ++it) {
+        const int s = it % NS;
         const int4 d0 = desc[2 * s];
-        const int d1 = desc[2 * s + 1].x;
-        const int unit = d0.x, n = d1 & 0xff, flags = d1 >> 8;
-        if (unit != cur_unit) {
+        const int n = desc[2 * s + 1].x;
+        const int unit = d0.x;
+        if (unit < 0) break;                                   // end of the schedule
+        if (unit != cur_unit) {                                // uniform over the group
+            if (cur_unit >= 0) {
+                flush(part_slot(blockIdx.x, cur_unit, grp));
+                reset_state();
+            }
             load_unit(d0.y, d0.z);
             cur_unit = unit;
         }
-        const int nmine = min(2, max(0, n - 2 * warp));
-        if (nmine > 0) {
-            const uint8_t *blk0 = ring + s * STAGE_BYTES + (2 * warp) * BLK_BYTES;
-            const int tok0 = (d0.w + 2 * warp) * BLK_TOK;   // first position of my first block
-            // a block needs masking if it is a phantom or crosses [S, L)
-            bool edge[2];
+        const bool ok = mbar_wait_bounded(&full[s], (it / NS) & 1);
+        if (ok) {
+            const int nmine = min(2, max(0, n - 2 * warp));
+            if (nmine > 0) {
+                const uint8_t *blk0 = ring + s * STAGE_BYTES + (2 * warp) * BLK_BYTES;
+                const int tok0 = (d0.w + 2 * warp) * BLK_TOK;   // first position of my first block
+                // a block needs masking if it is a phantom or crosses [S, L)
+                bool edge[2];
 #pragma unroll
-            for (int bi = 0; bi < 2; bi++)
-                edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
-            // ---- scores for both blocks (the second may be a phantom)
-            uint4 kq[2];
+                for (int bi = 0; bi < 2; bi++)
+                    edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
+                // ---- scores for both blocks (the second may be a phantom)
+                uint4 kq[2];
 #pragma unroll
-            for (int bi = 0; bi < 2; bi++)
-                kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
-            int dk[2][C::NTK][4];
+                for (int bi = 0; bi < 2; bi++)
+                    kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
+                int dk[2][C::NTK][4];
 #pragma unroll
-            for (int bi = 0; bi < 2; bi++)
+                for (int bi = 0; bi < 2; bi++)
 #pragma unroll
-                for (int nu = 0; nu < C::NTK; nu++)
+                    for (int nu = 0; nu < C::NTK; nu++)
 #pragma unroll
-                    for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
-            // one IMMA per group: the masked bytes are u8 codes c * 4^g
-#pragma unroll
-            for (int g = 0; g < 4; g++) {
-                const uint32_t msk = 0x03030303u << (2 * g);
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++) {
-                    const uint4 q4 = kq[bi];
-#pragma unroll
-                    for (int j = 0; j < C::NTK_STEP; j++) {
-                        const int nu = (g * 2 * G) / 8 + j;
-                        imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
-                                  qB[g][j][0], qB[g][j][1]);
-                    }
-                }
-            }
-            float sco[2][2][C::HPL];
-#pragma unroll
-            for (int bi = 0; bi < 2; bi++) {
-                float part_sc[2][C::HPL];
-#pragma unroll
-                for (int st = 0; st < 2; st++)
-#pragma unroll
-                    for (int hh = 0; hh < C::HPL; hh++) part_sc[st][hh] = 0.f;
-#pragma unroll
-                for (int nu = 0; nu < C::NTK; nu++) {
-                    const int g = ktile_group<G>(nu, c);
-                    const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
-                                                                      8 * (4 * r + g));
-                    const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
-                    const int hh = ktile_slot<G>(nu);
-                    // hi*254 + lo is exact in int32 (|.| < 2^28)
-                    const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
-                    const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
-                    part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
-                    part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
-                }
-#pragma unroll
-                for (int st = 0; st < 2; st++)
-#pragma unroll
-                    for (int hh = 0; hh < C::HPL; hh++) {
-                        float v = part_sc[st][hh];
-                        if (G == 1) {
-                            v += __shfl_xor_sync(0xffffffffu, v, 1);
-                            v += __shfl_xor_sync(0xffffffffu, v, 2);
-                        } else if (G == 2) {
-                            v += __shfl_xor_sync(0xffffffffu, v, 2);
-                        }
-                        if (edge[bi]) {
-                            const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
-                            v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
-                        }
-                        sco[bi][st][hh] = v;
-                    }
-            }
-            // ---- online softmax.  The running max only moves when a score of
-            // this stage exceeds it (rare after the first stages), so the
-            // common path is one vote; the branch is uniform over the warp.
-            bool over = false;
-#pragma unroll
-            for (int bi = 0; bi < 2; bi++)
-#pragma unroll
-                for (int st = 0; st < 2; st++)
-#pragma unroll
-                    for (int hh = 0; hh < C::HPL; hh++)
-                        over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
-            if (__any_sync(0xffffffffu, over)) {
-            float mt[C::HPL];
-#pragma unroll
-            for (int hh = 0; hh < C::HPL; hh++) {
-                float v = fmaxf(fmaxf(sco[0][0][hh], sco[0][1][hh]), fmaxf(sco[1][0][hh], sco[1][1][hh]));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                mt[hh] = v;
-            }
-            float mnew[G];
-            bool grow = false;
-#pragma unroll
-            for (int hd = 0; hd < G; hd++) {
-                const int owner = G == 1 ? 0 : (G == 2 ? (hd & 1) : (hd & 3));
-                const float tmx = __shfl_sync(0xffffffffu, mt[G >= 8 ? (hd >> 2) : 0], owner);
-                mnew[hd] = fmaxf(m_run[hd], tmx);
-                grow |= mnew[hd] > m_run[hd];
-            }
-            if (grow) {
-                float al[G];
-#pragma unroll
-                for (int hd = 0; hd < G; hd++) {
-                    al[hd] = (mnew[hd] == NEG_INF) ? 1.f : fast_exp2(m_run[hd] - mnew[hd]);
-                    m_run[hd] = mnew[hd];
-                }
-#pragma unroll
-                for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
-#pragma unroll
-                for (int k = 0; k < NW; k++) {
-                    int g, head;
-                    wsrc<G>(c, k, g, head);
-                    Z[k] *= pick<G>(al, head);
-                }
-#pragma unroll
-                for (int g = 0; g < 4; g++)
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        const int col = 8 * ((g * G) / 8) + 2 * c + (k & 1);
-                        const float f = pick<G>(al, col % G);
-                        O[2 * g][k] *= f;
-                        O[2 * g + 1][k] *= f;
-                    }
-            }
-            }
-            float P[2][2][C::HPL];
-#pragma unroll
-            for (int bi = 0; bi < 2; bi++)
-#pragma unroll
-                for (int st = 0; st < 2; st++)
-#pragma unroll
-                    for (int hh = 0; hh < C::HPL; hh++) {
-                        const float v = sco[bi][st][hh];
-                        const float mm = pick<G>(m_run, lane_head<G>(c, hh));
-                        // every block holds a valid token, so mm is finite and
-                        // a masked score (-inf) gives exactly 0
-                        const float p = fast_exp2(v - mm);
-                        P[bi][st][hh] = p;
-                        l_run[hh] += p;
-                    }
-            // ---- P.V
-#pragma unroll
-            for (int bi = 0; bi < 2; bi++) {
-                const uint8_t *blk = blk0 + bi * BLK_BYTES;
-                // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
-                // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
-                uint32_t H[NW];
-                {
-                    uint32_t spair[NGL];
-                    float zr[NGL][2];
-#pragma unroll
-                    for (int gl = 0; gl < NGL; gl++) {
-                        const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
-                        const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
-                        spair[gl] = __byte_perm(mv.x, mv.y, 0x5410);      // (s_r, s_r+8)
-                        zr[gl][0] = __half2float(__ushort_as_half((unsigned short)(mv.x >> 16)));
-                        zr[gl][1] = __half2float(__ushort_as_half((unsigned short)(mv.y >> 16)));
-                    }
-#pragma unroll
-                    for (int k = 0; k < NW; k++) {
-                        const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
-                        const int hh = G >= 8 ? (k >> 2) : 0;
-                        const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
-                        const uint32_t ph = pack_half2(p0, p1);
-                        const __half2 w2 = __hmul2(*reinterpret_cast<const __half2 *>(&ph),
-                                                   *reinterpret_cast<const __half2 *>(&spair[gl]));
-                        uint32_t hw = *reinterpret_cast<const uint32_t *>(&w2);
-                        float z0 = zr[gl][0], z1 = zr[gl][1];
-                        if (edge[bi]) {      // masked tokens (p == 0): never use their metadata
-                            hw &= (p0 == 0.f ? 0xffff0000u : 0xffffffffu) &
-                                  (p1 == 0.f ? 0x0000ffffu : 0xffffffffu);
-                            z0 = p0 == 0.f ? 0.f : z0;
-                            z1 = p1 == 0.f ? 0.f : z1;
-                        }
-                        H[k] = hw;
-                        Z[k] = fmaf(p0, z0, fmaf(p1, z1, Z[k]));
-                    }
-                }
-                // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
-                // its column (group, head)
-                uint32_t Bv[C::NTV][2];
-#pragma unroll
-                for (int i = 0; i < C::NTV; i++) {
-                    const int col = 8 * i + (lane >> 2);
-                    const bool valid = col < 4 * G;
-                    const int g = col / G, head = col % G;
-                    int csrc, ksel;
-                    if (G == 1) { csrc = g; ksel = 0; }
-                    else if (G == 2) { csrc = head + 2 * (g & 1); ksel = g >> 1; }
-                    else if (G == 4) { csrc = head; ksel = g & 1; }
-                    else { csrc = head & 3; ksel = head >> 2; }
-                    const int src0 = 4 * (2 * c) + csrc, src1 = src0 + 4;
-                    uint32_t X, Y;
-                    if (G == 1) {
-                        X = __shfl_sync(0xffffffffu, H[0], src0);
-                        Y = __shfl_sync(0xffffffffu, H[0], src1);
-                    } else {
-                        // two candidate registers; the lane keeps the one it needs
-                        const int k0 = G == 2 ? 0 : (G == 4 ? 2 * i : i);
-                        const int k1 = G == 2 ? 1 : (G == 4 ? 2 * i + 1 : 4 + i);
-                        const uint32_t X0 = __shfl_sync(0xffffffffu, H[k0], src0);
-                        const uint32_t Y0 = __shfl_sync(0xffffffffu, H[k0], src1);
-                        const uint32_t X1 = __shfl_sync(0xffffffffu, H[k1], src0);
-                        const uint32_t Y1 = __shfl_sync(0xffffffffu, H[k1], src1);
-                        X = ksel ? X1 : X0;
-                        Y = ksel ? Y1 : Y0;
-                    }
-                    Bv[i][0] = valid ? __byte_perm(X, Y, 0x5410) : 0u;
-                    Bv[i][1] = valid ? __byte_perm(X, Y, 0x7632) : 0u;
-                }
-                const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
-                const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
+                        for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
+                // one IMMA per group: the masked bytes are u8 codes c * 4^g
 #pragma unroll
                 for (int g = 0; g < 4; g++) {
-                    const uint32_t msk = 0x00030003u << (2 * g);
-                    const int nv = (g * G) / 8;
+                    const uint32_t msk = 0x03030303u << (2 * g);
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; h2++) {
-                        const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
-                        mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk, (w2 >> 8) & msk,
-                                 Bv[nv][0], Bv[nv][1]);
+                    for (int bi = 0; bi < 2; bi++) {
+                        const uint4 q4 = kq[bi];
+#pragma unroll
+                        for (int j = 0; j < C::NTK_STEP; j++) {
+                            const int nu = (g * 2 * G) / 8 + j;
+                            imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
+                                      qB[g][j][0], qB[g][j][1]);
+                        }
+                    }
+                }
+                float sco[2][2][C::HPL];
+#pragma unroll
+                for (int bi = 0; bi < 2; bi++) {
+                    float part_sc[2][C::HPL];
+#pragma unroll
+                    for (int st = 0; st < 2; st++)
+#pragma unroll
+                        for (int hh = 0; hh < C::HPL; hh++) part_sc[st][hh] = 0.f;
+#pragma unroll
+                    for (int nu = 0; nu < C::NTK; nu++) {
+                        const int g = ktile_group<G>(nu, c);
+                        const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
+                                                                          8 * (4 * r + g));
+                        const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
+                        const int hh = ktile_slot<G>(nu);
+                        // hi*254 + lo is exact in int32 (|.| < 2^28)
+                        const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
+                        const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
+                        part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
+                        part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
+                    }
+#pragma unroll
+                    for (int st = 0; st < 2; st++)
+#pragma unroll
+                        for (int hh = 0; hh < C::HPL; hh++) {
+                            float v = part_sc[st][hh];
+                            if (G == 1) {
+                                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                            } else if (G == 2) {
+                                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                            }
+                            if (edge[bi]) {
+                                const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
+                                v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
+                            }
+                            sco[bi][st][hh] = v;
+                        }
+                }
+                // ---- online softmax.  The running max only moves when a score of
+                // this stage exceeds it (rare after the first stages), so the
+                // common path is one vote; the branch is uniform over the warp.
+                bool over = false;
+#pragma unroll
+                for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+                    for (int st = 0; st < 2; st++)
+#pragma unroll
+                        for (int hh = 0; hh < C::HPL; hh++)
+                            over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
+                if (__any_sync(0xffffffffu, over)) {
+                float mt[C::HPL];
+#pragma unroll
+                for (int hh = 0; hh < C::HPL; hh++) {
+                    float v = fmaxf(fmaxf(sco[0][0][hh], sco[0][1][hh]), fmaxf(sco[1][0][hh], sco[1][1][hh]));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                    mt[hh] = v;
+                }
+                float mnew[G];
+                bool grow = false;
+#pragma unroll
+                for (int hd = 0; hd < G; hd++) {
+                    const int owner = G == 1 ? 0 : (G == 2 ? (hd & 1) : (hd & 3));
+                    const float tmx = __shfl_sync(0xffffffffu, mt[G >= 8 ? (hd >> 2) : 0], owner);
+                    mnew[hd] = fmaxf(m_run[hd], tmx);
+                    grow |= mnew[hd] > m_run[hd];
+                }
+                if (grow) {
+                    float al[G];
+#pragma unroll
+                    for (int hd = 0; hd < G; hd++) {
+                        al[hd] = (mnew[hd] == NEG_INF) ? 1.f : fast_exp2(m_run[hd] - mnew[hd]);
+                        m_run[hd] = mnew[hd];
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
+#pragma unroll
+                    for (int k = 0; k < NW; k++) {
+                        int g, head;
+                        wsrc<G>(c, k, g, head);
+                        Z[k] *= pick<G>(al, head);
+                    }
+#pragma unroll
+                    for (int g = 0; g < 4; g++)
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const int col = 8 * ((g * G) / 8) + 2 * c + (k & 1);
+                            const float f = pick<G>(al, col % G);
+                            O[2 * g][k] *= f;
+                            O[2 * g + 1][k] *= f;
+                        }
+                }
+                }
+                float P[2][2][C::HPL];
+#pragma unroll
+                for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+                    for (int st = 0; st < 2; st++)
+#pragma unroll
+                        for (int hh = 0; hh < C::HPL; hh++) {
+                            const float v = sco[bi][st][hh];
+                            const float mm = pick<G>(m_run, lane_head<G>(c, hh));
+                            // every block holds a valid token, so mm is finite and
+                            // a masked score (-inf) gives exactly 0
+                            const float p = fast_exp2(v - mm);
+                            P[bi][st][hh] = p;
+                            l_run[hh] += p;
+                        }
+                // ---- P.V
+#pragma unroll
+                for (int bi = 0; bi < 2; bi++) {
+                    const uint8_t *blk = blk0 + bi * BLK_BYTES;
+                    // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
+                    // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
+                    uint32_t H[NW];
+                    {
+                        uint32_t spair[NGL];
+                        float zr[NGL][2];
+#pragma unroll
+                        for (int gl = 0; gl < NGL; gl++) {
+                            const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
+                            const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
+                            spair[gl] = __byte_perm(mv.x, mv.y, 0x5410);      // (s_r, s_r+8)
+                            zr[gl][0] = __half2float(__ushort_as_half((unsigned short)(mv.x >> 16)));
+                            zr[gl][1] = __half2float(__ushort_as_half((unsigned short)(mv.y >> 16)));
+                        }
+#pragma unroll
+                        for (int k = 0; k < NW; k++) {
+                            const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
+                            const int hh = G >= 8 ? (k >> 2) : 0;
+                            const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
+                            const uint32_t ph = pack_half2(p0, p1);
+                            const __half2 w2 = __hmul2(*reinterpret_cast<const __half2 *>(&ph),
+                                                       *reinterpret_cast<const __half2 *>(&spair[gl]));
+                            uint32_t hw = *reinterpret_cast<const uint32_t *>(&w2);
+                            float z0 = zr[gl][0], z1 = zr[gl][1];
+                            if (edge[bi]) {      // masked tokens (p == 0): never use their metadata
+                                hw &= (p0 == 0.f ? 0xffff0000u : 0xffffffffu) &
+                                      (p1 == 0.f ? 0x0000ffffu : 0xffffffffu);
+                                z0 = p0 == 0.f ? 0.f : z0;
+                                z1 = p1 == 0.f ? 0.f : z1;
+                            }
+                            H[k] = hw;
+                            Z[k] = fmaf(p0, z0, fmaf(p1, z1, Z[k]));
+                        }
+                    }
+                    // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
+                    // its column (group, head)
+                    uint32_t Bv[C::NTV][2];
+#pragma unroll
+                    for (int i = 0; i < C::NTV; i++) {
+                        const int col = 8 * i + (lane >> 2);
+                        const bool valid = col < 4 * G;
+                        const int g = col / G, head = col % G;
+                        int csrc, ksel;
+                        if (G == 1) { csrc = g; ksel = 0; }
+                        else if (G == 2) { csrc = head + 2 * (g & 1); ksel = g >> 1; }
+                        else if (G == 4) { csrc = head; ksel = g & 1; }
+                        else { csrc = head & 3; ksel = head >> 2; }
+                        const int src0 = 4 * (2 * c) + csrc, src1 = src0 + 4;
+                        uint32_t X, Y;
+                        if (G == 1) {
+                            X = __shfl_sync(0xffffffffu, H[0], src0);
+                            Y = __shfl_sync(0xffffffffu, H[0], src1);
+                        } else {
+                            // two candidate registers; the lane keeps the one it needs
+                            const int k0 = G == 2 ? 0 : (G == 4 ? 2 * i : i);
+                            const int k1 = G == 2 ? 1 : (G == 4 ? 2 * i + 1 : 4 + i);
+                            const uint32_t X0 = __shfl_sync(0xffffffffu, H[k0], src0);
+                            const uint32_t Y0 = __shfl_sync(0xffffffffu, H[k0], src1);
+                            const uint32_t X1 = __shfl_sync(0xffffffffu, H[k1], src0);
+                            const uint32_t Y1 = __shfl_sync(0xffffffffu, H[k1], src1);
+                            X = ksel ? X1 : X0;
+                            Y = ksel ? Y1 : Y0;
+                        }
+                        Bv[i][0] = valid ? __byte_perm(X, Y, 0x5410) : 0u;
+                        Bv[i][1] = valid ? __byte_perm(X, Y, 0x7632) : 0u;
+                    }
+                    const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
+                    const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+                    for (int g = 0; g < 4; g++) {
+                        const uint32_t msk = 0x00030003u << (2 * g);
+                        const int nv = (g * G) / 8;
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; h2++) {
+                            const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
+                            mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk, (w2 >> 8) & msk,
+                                     Bv[nv][0], Bv[nv][1]);
+                        }
                     }
                 }
             }
+        } else {
+            set_status(a.status, KVQ_DEV_TIMEOUT);
         }
-        // release the slot: once every warp is done with it, thread 0 refills it
-        asm volatile("bar.sync 1, %0;" ::"n"(DEC_THREADS) : "memory");
-        if (threadIdx.x == 0) {
+        // release the slot (a failed wait anywhere in the group ends it);
+        // the leader refills it
+        int any_bad;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.or.pred p, %2, %3, p;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(any_bad)
+            : "r"((unsigned)!ok), "r"(1 + grp), "n"(GROUP_THREADS)
+            : "memory");
+        if (any_bad) {
+            aborted = true;
+            break;
+        }
+        if (leader) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             issue_next(s);
         }
-        // end of this CTA's segment of the unit: write the partial
-        if (flags & 1) {
-            flush(blockIdx.x + unit);
-            reset_state();
-        }
-        if (flags & 2) break;
     }
+    if (aborted) {
+        // leave no copy in flight into this CTA's shared memory: wait (briefly,
+        // bounded) for every stage issued from this iteration on
+        if (leader)
+            for (int j = it; j < issued; j++) mbar_wait_bounded(&full[j % NS], (j / NS) & 1, 1u << 8);
+        return;
+    }
+    if (cur_unit >= 0) flush(part_slot(blockIdx.x, cur_unit, grp));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -922,10 +991,14 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     const int ustart = pre + h * nb;
     const int c0 = nb > 0 ? ustart / W : 0;
     const int np = nb > 0 ? (ustart + nb - 1) / W - c0 + 1 : 0;
-    auto pptr = [&](int i) -> const float * {   // partial i (i == np: the sink partial)
-        return i < np ? a.part + ((size_t)(c0 + i + u) * G + head) * PART : sinkp;
+    // partial i < DEC_GROUPS*np: group i % DEC_GROUPS of CTA c0 + i / DEC_GROUPS
+    // (m = -inf if that group took no stage of the unit); then the sink partial
+    auto pptr = [&](int i) -> const float * {
+        return i < DEC_GROUPS * np
+                   ? a.part + (part_slot(c0 + i / DEC_GROUPS, u, i % DEC_GROUPS) * G + head) * PART
+                   : sinkp;
     };
-    const int ntot = np + (ns > 0 ? 1 : 0);
+    const int ntot = DEC_GROUPS * np + (ns > 0 ? 1 : 0);
 
     // Partials in batches of MRG_BATCH: warp w takes partials w, w+8, w+16,
     // w+24 of the batch and issues all their loads before using any.
@@ -962,7 +1035,10 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         mglob = mnew;
 #pragma unroll
         for (int j = 0; j < PW; j++) {
-            const float f = (ml[j].x == NEG_INF) ? 0.f : exp2f(ml[j].x - mglob);
+            // an empty partial (m = -inf) has only its header written: its
+            // o and l are skipped, never multiplied by 0
+            if (ml[j].x == NEG_INF) continue;
+            const float f = exp2f(ml[j].x - mglob);
             acc.x = fmaf(f, o4[j].x, acc.x); acc.y = fmaf(f, o4[j].y, acc.y);
             acc.z = fmaf(f, o4[j].z, acc.z); acc.w = fmaf(f, o4[j].w, acc.w);
             lsum = fmaf(f, ml[j].y, lsum);
@@ -1018,7 +1094,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
     const int G = Hq / Hkv;
     w.qprep = 0;
     w.part = up(w.qprep + (size_t)B * Hq * QB);
-    w.total = up(w.part + sizeof(float) * ((size_t)C + (size_t)B * Hkv) * G * PART);
+    w.total = up(w.part + sizeof(float) * DEC_GROUPS * ((size_t)C + (size_t)B * Hkv) * G * PART);
     return w;
 }
 

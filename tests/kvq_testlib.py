@@ -27,7 +27,10 @@ def gpu_append(cache, K, V, w, rt, seq_lens):
 
 
 def gpu_decode(cache, Q, w, rt, seq_lens, max_ctx):
+    # The workspace need not be initialised: poison it (all bytes 0xFF, NaN
+    # as fp32) so that a read of anything the call did not write shows up.
     ws = kvq.decode_workspace(cache.B, Q.shape[1], cache.Hkv, max_ctx)
+    ws.fill_(0xFF)
     out = torch.empty_like(Q)
     kvq.kvq_decode_attention(Q.contiguous(), cache, w.mode, rt[0], rt[1], rt[2], seq_lens,
                              cache.sink_fp16, max_ctx, ws, out)

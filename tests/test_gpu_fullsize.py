@@ -62,6 +62,7 @@ def run_workload(w, samples, prefill_to=None):
     lens_t = torch.from_numpy(lens.astype(np.int32)).to(dev)
     Q = W.queries(w, dev)
     ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, L)
+    ws.fill_(0xFF)                           # uninitialised by contract: poison it
     out = torch.empty_like(Q)
     kvq.kvq_decode_attention(Q, cache, w.mode, rk, rv, pm, lens_t, w.sink, L, ws, out)
     torch.cuda.synchronize()
