@@ -568,6 +568,262 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         bar_group();
     };
 
+    // Scores, part 1: the K codes of a warp's two blocks of a stage through
+    // the integer tensor cores (one IMMA per group and block; the second
+    // block may be a phantom).
+    auto k_mma = [&](const uint8_t *blk0, int (&dk)[2][C::NTK][4]) {
+        uint4 kq[2];
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++)
+            kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+            for (int nu = 0; nu < C::NTK; nu++)
+#pragma unroll
+                for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
+        // one IMMA per group: the masked bytes are u8 codes c * 4^g
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+            const uint32_t msk = 0x03030303u << (2 * g);
+#pragma unroll
+            for (int bi = 0; bi < 2; bi++) {
+                const uint4 q4 = kq[bi];
+#pragma unroll
+                for (int j = 0; j < C::NTK_STEP; j++) {
+                    const int nu = (g * 2 * G) / 8 + j;
+                    imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
+                              qB[g][j][0], qB[g][j][1]);
+                }
+            }
+        }
+    };
+    // Scores, part 2: integer dots -> fp32 scores (group scale and zero,
+    // query scale), summed over the groups; positions outside [S, L) and
+    // phantom blocks are masked to -inf.
+    auto k_combine = [&](const uint8_t *blk0, const int (&dk)[2][C::NTK][4], int tok0, int nmine,
+                         float (&sco)[2][2][C::HPL], bool (&edge)[2]) {
+        // a block needs masking if it is a phantom or crosses [S, L)
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++)
+            edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++) {
+            float part_sc[2][C::HPL];
+#pragma unroll
+            for (int st = 0; st < 2; st++)
+#pragma unroll
+                for (int hh = 0; hh < C::HPL; hh++) part_sc[st][hh] = 0.f;
+#pragma unroll
+            for (int nu = 0; nu < C::NTK; nu++) {
+                const int g = ktile_group<G>(nu, c);
+                const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
+                                                                  8 * (4 * r + g));
+                const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
+                const int hh = ktile_slot<G>(nu);
+                // hi*254 + lo is exact in int32 (|.| < 2^28)
+                const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
+                const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
+                part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
+                part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
+            }
+#pragma unroll
+            for (int st = 0; st < 2; st++)
+#pragma unroll
+                for (int hh = 0; hh < C::HPL; hh++) {
+                    float v = part_sc[st][hh];
+                    if (G == 1) {
+                        v += __shfl_xor_sync(0xffffffffu, v, 1);
+                        v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    } else if (G == 2) {
+                        v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    }
+                    if (edge[bi]) {
+                        const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
+                        v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
+                    }
+                    sco[bi][st][hh] = v;
+                }
+        }
+    };
+    // Online softmax and P.V of one stage.
+    auto v_side = [&](const uint8_t *blk0, const float (&sco)[2][2][C::HPL], const bool (&edge)[2]) {
+        // ---- online softmax.  The running max only moves when a score of
+        // this stage exceeds it (rare after the first stages), so the
+        // common path is one vote; the branch is uniform over the warp.
+        bool over = false;
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+            for (int st = 0; st < 2; st++)
+#pragma unroll
+                for (int hh = 0; hh < C::HPL; hh++)
+                    over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
+        if (__any_sync(0xffffffffu, over)) {
+        float mt[C::HPL];
+#pragma unroll
+        for (int hh = 0; hh < C::HPL; hh++) {
+            float v = fmaxf(fmaxf(sco[0][0][hh], sco[0][1][hh]), fmaxf(sco[1][0][hh], sco[1][1][hh]));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+            mt[hh] = v;
+        }
+        float mnew[G];
+        bool grow = false;
+#pragma unroll
+        for (int hd = 0; hd < G; hd++) {
+            const int owner = G == 1 ? 0 : (G == 2 ? (hd & 1) : (hd & 3));
+            const float tmx = __shfl_sync(0xffffffffu, mt[G >= 8 ? (hd >> 2) : 0], owner);
+            mnew[hd] = fmaxf(m_run[hd], tmx);
+            grow |= mnew[hd] > m_run[hd];
+        }
+        if (grow) {
+            float al[G];
+#pragma unroll
+            for (int hd = 0; hd < G; hd++) {
+                al[hd] = (mnew[hd] == NEG_INF) ? 1.f : fast_exp2(m_run[hd] - mnew[hd]);
+                m_run[hd] = mnew[hd];
+            }
+#pragma unroll
+            for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
+#pragma unroll
+            for (int k = 0; k < NW; k++) {
+                int g, head;
+                wsrc<G>(c, k, g, head);
+                Z[k] *= pick<G>(al, head);
+            }
+#pragma unroll
+            for (int g = 0; g < 4; g++)
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const int col = 8 * ((g * G) / 8) + 2 * c + (k & 1);
+                    const float f = pick<G>(al, col % G);
+                    O[2 * g][k] *= f;
+                    O[2 * g + 1][k] *= f;
+                }
+        }
+        }
+        float P[2][2][C::HPL];
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++)
+#pragma unroll
+            for (int st = 0; st < 2; st++)
+#pragma unroll
+                for (int hh = 0; hh < C::HPL; hh++) {
+                    const float v = sco[bi][st][hh];
+                    const float mm = pick<G>(m_run, lane_head<G>(c, hh));
+                    // every block holds a valid token, so mm is finite and
+                    // a masked score (-inf) gives exactly 0
+                    const float p = fast_exp2(v - mm);
+                    P[bi][st][hh] = p;
+                    l_run[hh] += p;
+                }
+        // ---- P.V
+#pragma unroll
+        for (int bi = 0; bi < 2; bi++) {
+            const uint8_t *blk = blk0 + bi * BLK_BYTES;
+            // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
+            // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
+            uint32_t H[NW];
+            {
+                uint32_t spair[NGL];
+                float zr[NGL][2];
+#pragma unroll
+                for (int gl = 0; gl < NGL; gl++) {
+                    const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
+                    const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
+                    spair[gl] = __byte_perm(mv.x, mv.y, 0x5410);      // (s_r, s_r+8)
+                    zr[gl][0] = __half2float(__ushort_as_half((unsigned short)(mv.x >> 16)));
+                    zr[gl][1] = __half2float(__ushort_as_half((unsigned short)(mv.y >> 16)));
+                }
+#pragma unroll
+                for (int k = 0; k < NW; k++) {
+                    const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
+                    const int hh = G >= 8 ? (k >> 2) : 0;
+                    const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
+                    const uint32_t ph = pack_half2(p0, p1);
+                    const __half2 w2 = __hmul2(*reinterpret_cast<const __half2 *>(&ph),
+                                               *reinterpret_cast<const __half2 *>(&spair[gl]));
+                    uint32_t hw = *reinterpret_cast<const uint32_t *>(&w2);
+                    float z0 = zr[gl][0], z1 = zr[gl][1];
+                    if (edge[bi]) {      // masked tokens (p == 0): never use their metadata
+                        hw &= (p0 == 0.f ? 0xffff0000u : 0xffffffffu) &
+                              (p1 == 0.f ? 0x0000ffffu : 0xffffffffu);
+                        z0 = p0 == 0.f ? 0.f : z0;
+                        z1 = p1 == 0.f ? 0.f : z1;
+                    }
+                    H[k] = hw;
+                    Z[k] = fmaf(p0, z0, fmaf(p1, z1, Z[k]));
+                }
+            }
+            // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
+            // its column (group, head)
+            uint32_t Bv[C::NTV][2];
+#pragma unroll
+            for (int i = 0; i < C::NTV; i++) {
+                const int col = 8 * i + (lane >> 2);
+                const bool valid = col < 4 * G;
+                const int g = col / G, head = col % G;
+                int csrc, ksel;
+                if (G == 1) { csrc = g; ksel = 0; }
+                else if (G == 2) { csrc = head + 2 * (g & 1); ksel = g >> 1; }
+                else if (G == 4) { csrc = head; ksel = g & 1; }
+                else { csrc = head & 3; ksel = head >> 2; }
+                const int src0 = 4 * (2 * c) + csrc, src1 = src0 + 4;
+                uint32_t X, Y;
+                if (G == 1) {
+                    X = __shfl_sync(0xffffffffu, H[0], src0);
+                    Y = __shfl_sync(0xffffffffu, H[0], src1);
+                } else {
+                    // two candidate registers; the lane keeps the one it needs
+                    const int k0 = G == 2 ? 0 : (G == 4 ? 2 * i : i);
+                    const int k1 = G == 2 ? 1 : (G == 4 ? 2 * i + 1 : 4 + i);
+                    const uint32_t X0 = __shfl_sync(0xffffffffu, H[k0], src0);
+                    const uint32_t Y0 = __shfl_sync(0xffffffffu, H[k0], src1);
+                    const uint32_t X1 = __shfl_sync(0xffffffffu, H[k1], src0);
+                    const uint32_t Y1 = __shfl_sync(0xffffffffu, H[k1], src1);
+                    X = ksel ? X1 : X0;
+                    Y = ksel ? Y1 : Y0;
+                }
+                Bv[i][0] = valid ? __byte_perm(X, Y, 0x5410) : 0u;
+                Bv[i][1] = valid ? __byte_perm(X, Y, 0x7632) : 0u;
+            }
+            const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
+            const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+            for (int g = 0; g < 4; g++) {
+                const uint32_t msk = 0x00030003u << (2 * g);
+                const int nv = (g * G) / 8;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; h2++) {
+                    const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
+                    mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk, (w2 >> 8) & msk,
+                             Bv[nv][0], Bv[nv][1]);
+                }
+            }
+        }
+    };
+    // Release ring slot `slot` once the whole group is done with it; the
+    // leader refills it.  Returns true (uniformly over the group) when a wait
+    // failed anywhere in the group: the group then stops.
+    auto release = [&](int slot, bool ok) -> bool {
+        int any_bad;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.or.pred p, %2, %3, p;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(any_bad)
+            : "r"((unsigned)!ok), "r"(1 + grp), "n"(GROUP_THREADS)
+            : "memory");
+        if (any_bad) return true;
+        if (leader) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue_next(slot);
+        }
+        return false;
+    };
+    auto wblk = [&](int slot) { return ring + slot * STAGE_BYTES + (2 * warp) * BLK_BYTES; };
+
     reset_state();
     bool aborted = false;
     int it = 0;
@@ -576,8 +832,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         const int4 d0 = desc[2 * s];
         const int n = desc[2 * s + 1].x;
         const int unit = d0.x;
-        if (unit < 0) break;                                   // end of the schedule
-        if (unit != cur_unit) {                                // uniform over the group
+        if (unit < 0) break;                               // end of the schedule
+        if (unit != cur_unit) {                            // uniform over the group
             if (cur_unit >= 0) {
                 flush(part_slot(blockIdx.x, cur_unit, grp));
                 reset_state();
@@ -586,257 +842,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             cur_unit = unit;
         }
         const bool ok = mbar_wait_bounded(&full[s], (it / NS) & 1);
-        if (ok) {
-            const int nmine = min(2, max(0, n - 2 * warp));
-            if (nmine > 0) {
-                const uint8_t *blk0 = ring + s * STAGE_BYTES + (2 * warp) * BLK_BYTES;
-                const int tok0 = (d0.w + 2 * warp) * BLK_TOK;   // first position of my first block
-                // a block needs masking if it is a phantom or crosses [S, L)
-                bool edge[2];
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++)
-                    edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
-                // ---- scores for both blocks (the second may be a phantom)
-                uint4 kq[2];
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++)
-                    kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
-                int dk[2][C::NTK][4];
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++)
-#pragma unroll
-                    for (int nu = 0; nu < C::NTK; nu++)
-#pragma unroll
-                        for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
-                // one IMMA per group: the masked bytes are u8 codes c * 4^g
-#pragma unroll
-                for (int g = 0; g < 4; g++) {
-                    const uint32_t msk = 0x03030303u << (2 * g);
-#pragma unroll
-                    for (int bi = 0; bi < 2; bi++) {
-                        const uint4 q4 = kq[bi];
-#pragma unroll
-                        for (int j = 0; j < C::NTK_STEP; j++) {
-                            const int nu = (g * 2 * G) / 8 + j;
-                            imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
-                                      qB[g][j][0], qB[g][j][1]);
-                        }
-                    }
-                }
-                float sco[2][2][C::HPL];
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++) {
-                    float part_sc[2][C::HPL];
-#pragma unroll
-                    for (int st = 0; st < 2; st++)
-#pragma unroll
-                        for (int hh = 0; hh < C::HPL; hh++) part_sc[st][hh] = 0.f;
-#pragma unroll
-                    for (int nu = 0; nu < C::NTK; nu++) {
-                        const int g = ktile_group<G>(nu, c);
-                        const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
-                                                                          8 * (4 * r + g));
-                        const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
-                        const int hh = ktile_slot<G>(nu);
-                        // hi*254 + lo is exact in int32 (|.| < 2^28)
-                        const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
-                        const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
-                        part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
-                        part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
-                    }
-#pragma unroll
-                    for (int st = 0; st < 2; st++)
-#pragma unroll
-                        for (int hh = 0; hh < C::HPL; hh++) {
-                            float v = part_sc[st][hh];
-                            if (G == 1) {
-                                v += __shfl_xor_sync(0xffffffffu, v, 1);
-                                v += __shfl_xor_sync(0xffffffffu, v, 2);
-                            } else if (G == 2) {
-                                v += __shfl_xor_sync(0xffffffffu, v, 2);
-                            }
-                            if (edge[bi]) {
-                                const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
-                                v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
-                            }
-                            sco[bi][st][hh] = v;
-                        }
-                }
-                // ---- online softmax.  The running max only moves when a score of
-                // this stage exceeds it (rare after the first stages), so the
-                // common path is one vote; the branch is uniform over the warp.
-                bool over = false;
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++)
-#pragma unroll
-                    for (int st = 0; st < 2; st++)
-#pragma unroll
-                        for (int hh = 0; hh < C::HPL; hh++)
-                            over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
-                if (__any_sync(0xffffffffu, over)) {
-                float mt[C::HPL];
-#pragma unroll
-                for (int hh = 0; hh < C::HPL; hh++) {
-                    float v = fmaxf(fmaxf(sco[0][0][hh], sco[0][1][hh]), fmaxf(sco[1][0][hh], sco[1][1][hh]));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                    mt[hh] = v;
-                }
-                float mnew[G];
-                bool grow = false;
-#pragma unroll
-                for (int hd = 0; hd < G; hd++) {
-                    const int owner = G == 1 ? 0 : (G == 2 ? (hd & 1) : (hd & 3));
-                    const float tmx = __shfl_sync(0xffffffffu, mt[G >= 8 ? (hd >> 2) : 0], owner);
-                    mnew[hd] = fmaxf(m_run[hd], tmx);
-                    grow |= mnew[hd] > m_run[hd];
-                }
-                if (grow) {
-                    float al[G];
-#pragma unroll
-                    for (int hd = 0; hd < G; hd++) {
-                        al[hd] = (mnew[hd] == NEG_INF) ? 1.f : fast_exp2(m_run[hd] - mnew[hd]);
-                        m_run[hd] = mnew[hd];
-                    }
-#pragma unroll
-                    for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
-#pragma unroll
-                    for (int k = 0; k < NW; k++) {
-                        int g, head;
-                        wsrc<G>(c, k, g, head);
-                        Z[k] *= pick<G>(al, head);
-                    }
-#pragma unroll
-                    for (int g = 0; g < 4; g++)
-#pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            const int col = 8 * ((g * G) / 8) + 2 * c + (k & 1);
-                            const float f = pick<G>(al, col % G);
-                            O[2 * g][k] *= f;
-                            O[2 * g + 1][k] *= f;
-                        }
-                }
-                }
-                float P[2][2][C::HPL];
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++)
-#pragma unroll
-                    for (int st = 0; st < 2; st++)
-#pragma unroll
-                        for (int hh = 0; hh < C::HPL; hh++) {
-                            const float v = sco[bi][st][hh];
-                            const float mm = pick<G>(m_run, lane_head<G>(c, hh));
-                            // every block holds a valid token, so mm is finite and
-                            // a masked score (-inf) gives exactly 0
-                            const float p = fast_exp2(v - mm);
-                            P[bi][st][hh] = p;
-                            l_run[hh] += p;
-                        }
-                // ---- P.V
-#pragma unroll
-                for (int bi = 0; bi < 2; bi++) {
-                    const uint8_t *blk = blk0 + bi * BLK_BYTES;
-                    // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
-                    // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
-                    uint32_t H[NW];
-                    {
-                        uint32_t spair[NGL];
-                        float zr[NGL][2];
-#pragma unroll
-                        for (int gl = 0; gl < NGL; gl++) {
-                            const int g = G == 1 ? c : (G == 2 ? (c >> 1) + 2 * gl : gl);
-                            const uint2 mv = *reinterpret_cast<const uint2 *>(blk + OFF_VM + 8 * (4 * r + g));
-                            spair[gl] = __byte_perm(mv.x, mv.y, 0x5410);      // (s_r, s_r+8)
-                            zr[gl][0] = __half2float(__ushort_as_half((unsigned short)(mv.x >> 16)));
-                            zr[gl][1] = __half2float(__ushort_as_half((unsigned short)(mv.y >> 16)));
-                        }
-#pragma unroll
-                        for (int k = 0; k < NW; k++) {
-                            const int gl = G == 1 ? 0 : (G == 2 ? k : (k & 3));
-                            const int hh = G >= 8 ? (k >> 2) : 0;
-                            const float p0 = P[bi][0][hh], p1 = P[bi][1][hh];
-                            const uint32_t ph = pack_half2(p0, p1);
-                            const __half2 w2 = __hmul2(*reinterpret_cast<const __half2 *>(&ph),
-                                                       *reinterpret_cast<const __half2 *>(&spair[gl]));
-                            uint32_t hw = *reinterpret_cast<const uint32_t *>(&w2);
-                            float z0 = zr[gl][0], z1 = zr[gl][1];
-                            if (edge[bi]) {      // masked tokens (p == 0): never use their metadata
-                                hw &= (p0 == 0.f ? 0xffff0000u : 0xffffffffu) &
-                                      (p1 == 0.f ? 0x0000ffffu : 0xffffffffu);
-                                z0 = p0 == 0.f ? 0.f : z0;
-                                z1 = p1 == 0.f ? 0.f : z1;
-                            }
-                            H[k] = hw;
-                            Z[k] = fmaf(p0, z0, fmaf(p1, z1, Z[k]));
-                        }
-                    }
-                    // B fragments: lane (n, c') needs tokens 2c', 2c'+1, 2c'+8, 2c'+9 of
-                    // its column (group, head)
-                    uint32_t Bv[C::NTV][2];
-#pragma unroll
-                    for (int i = 0; i < C::NTV; i++) {
-                        const int col = 8 * i + (lane >> 2);
-                        const bool valid = col < 4 * G;
-                        const int g = col / G, head = col % G;
-                        int csrc, ksel;
-                        if (G == 1) { csrc = g; ksel = 0; }
-                        else if (G == 2) { csrc = head + 2 * (g & 1); ksel = g >> 1; }
-                        else if (G == 4) { csrc = head; ksel = g & 1; }
-                        else { csrc = head & 3; ksel = head >> 2; }
-                        const int src0 = 4 * (2 * c) + csrc, src1 = src0 + 4;
-                        uint32_t X, Y;
-                        if (G == 1) {
-                            X = __shfl_sync(0xffffffffu, H[0], src0);
-                            Y = __shfl_sync(0xffffffffu, H[0], src1);
-                        } else {
-                            // two candidate registers; the lane keeps the one it needs
-                            const int k0 = G == 2 ? 0 : (G == 4 ? 2 * i : i);
-                            const int k1 = G == 2 ? 1 : (G == 4 ? 2 * i + 1 : 4 + i);
-                            const uint32_t X0 = __shfl_sync(0xffffffffu, H[k0], src0);
-                            const uint32_t Y0 = __shfl_sync(0xffffffffu, H[k0], src1);
-                            const uint32_t X1 = __shfl_sync(0xffffffffu, H[k1], src0);
-                            const uint32_t Y1 = __shfl_sync(0xffffffffu, H[k1], src1);
-                            X = ksel ? X1 : X0;
-                            Y = ksel ? Y1 : Y0;
-                        }
-                        Bv[i][0] = valid ? __byte_perm(X, Y, 0x5410) : 0u;
-                        Bv[i][1] = valid ? __byte_perm(X, Y, 0x7632) : 0u;
-                    }
-                    const uint4 vq = *reinterpret_cast<const uint4 *>(blk + OFF_VC + 16 * (4 * r + c));
-                    const uint32_t Wv[4] = {vq.x, vq.y, vq.z, vq.w};
-#pragma unroll
-                    for (int g = 0; g < 4; g++) {
-                        const uint32_t msk = 0x00030003u << (2 * g);
-                        const int nv = (g * G) / 8;
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; h2++) {
-                            const uint32_t w0 = Wv[h2], w2 = Wv[2 + h2];
-                            mma16816(O[2 * g + h2], w0 & msk, (w0 >> 8) & msk, w2 & msk, (w2 >> 8) & msk,
-                                     Bv[nv][0], Bv[nv][1]);
-                        }
-                    }
-                }
-            }
-        } else {
-            set_status(a.status, KVQ_DEV_TIMEOUT);
+        const int nmine = min(2, max(0, n - 2 * warp));
+        if (ok && nmine > 0) {
+            int dk[2][C::NTK][4];
+            float sco[2][2][C::HPL];
+            bool edge[2];
+            k_mma(wblk(s), dk);
+            k_combine(wblk(s), dk, (d0.w + 2 * warp) * BLK_TOK, nmine, sco, edge);
+            v_side(wblk(s), sco, edge);
         }
-        // release the slot (a failed wait anywhere in the group ends it);
-        // the leader refills it
-        int any_bad;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-            "bar.red.or.pred p, %2, %3, p;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(any_bad)
-            : "r"((unsigned)!ok), "r"(1 + grp), "n"(GROUP_THREADS)
-            : "memory");
-        if (any_bad) {
+        if (!ok) set_status(a.status, KVQ_DEV_TIMEOUT);
+        if (release(s, ok)) {
             aborted = true;
             break;
-        }
-        if (leader) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue_next(s);
         }
     }
     if (aborted) {
