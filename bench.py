@@ -290,6 +290,51 @@ class Step:
         return max(self.kvq.kvq_get_status(c[0]) for c in self.layers)
 
 
+def append_rates(device, peak, reps=5):
+    """Throughput of the append alone (rotate + quantize + pack + store) on the
+    two bulk appends of the workload set: the ragged workload's prefill (B=4,
+    32768 tokens, 32 heads, dense rotation) and the hadamard workload's step
+    append (B=16, 128 tokens, 32 heads, permutation + FWHT).  Bytes = fp16 K
+    and V read (512 B per token-head) + packed codes and metadata written
+    (96 B) + the rotations read once; L2 flushed before each timed call."""
+    import rotated_int2_kv_head_b200 as kvq
+    flush = L2Flush(device)
+    out = {}
+    w0 = W.WORKLOADS["ragged"]
+    cases = [("ragged prefill", W.custom(name="ragged_prefill", seed=w0.seed + 1, B=w0.extra["prefill_B"],
+                                         Hq=32, Hkv=32, mode=0, k_outliers=8,
+                                         context=w0.extra["prefill_T"]), w0.extra["prefill_T"]),
+             ("hadamard step append", W.WORKLOADS["hadamard"], W.WORKLOADS["hadamard"].append_T)]
+    for name, w, T in cases:
+        Rk, Rv, perm = W.rotations(w)
+        rk = torch.from_numpy(Rk).to(device) if Rk is not None else None
+        rv = torch.from_numpy(Rv).to(device) if Rv is not None else None
+        pm = torch.from_numpy(perm).to(device) if perm is not None else None
+        K, V = W.kv_batch(w, 0, T, device)
+        cache = kvq.KVCache(w.B, w.Hkv, ((T + 15) // 16) * 16, w.sink, device=device)
+        sl = torch.zeros(w.B, dtype=torch.int32, device=device)
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        ms = []
+        for k in range(reps + 2):
+            sl.zero_()
+            flush(k)
+            ev[0].record()
+            kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, pm, cache, sl)
+            ev[1].record()
+            torch.cuda.synchronize(device)
+            if k >= 2:
+                ms.append(ev[0].elapsed_time(ev[1]))
+        if kvq.kvq_get_status(cache) != 0:
+            raise RuntimeError("append status %d" % kvq.kvq_get_status(cache))
+        nbytes = T * w.B * w.Hkv * (512 + 96) + (2 * w.Hkv * 128 * 128 * 4 if w.mode == 0 else 0)
+        t = float(np.median(ms)) * 1e-3
+        out[name] = {"B": w.B, "T": T, "Hkv": w.Hkv, "rotation": "dense" if w.mode == 0 else "perm+fwht",
+                     "ms": t * 1e3, "GB_per_s": nbytes / t / 1e9, "frac_of_hbm_peak": nbytes / t / 1e9 / peak,
+                     "bytes": nbytes}
+        del K, V, cache
+    return out
+
+
 def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
     the first `heads` KV heads of sequence 0 (their K/V rows are the very
@@ -488,6 +533,8 @@ def run_cuda(args):
         "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clk.summary(),
     }
+    if world == 1 and not args.no_append:
+        line["append"] = append_rates(dev, peak)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, step, dev)
     print(json.dumps(line), flush=True)
@@ -563,6 +610,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--workload", default="llama7b", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
