@@ -88,7 +88,9 @@ kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int3
     if (!aligned(K, 16) || !aligned(V, 16)) return KVQ_ERR_UNSUPPORTED;
     if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
+    cudaError_t e = (mode == KVQ_ROT_DENSE && append_tc_eligible(K, V, T))
+                        ? launch_append_tc(K, V, T, R_k, R_v, *cache, seq_lens, st)
+                        : launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -158,10 +160,12 @@ kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mode mode,
     if (!aligned(X, 16) || !aligned(Xrot, 16)) return KVQ_ERR_UNSUPPORTED;
     kvq_status s = check_rot(mode, R, R, perm);
     if (s != KVQ_OK) return s;
-    if (variant != 0) return KVQ_ERR_UNSUPPORTED;
+    if (variant != 0 && variant != 1) return KVQ_ERR_INVALID_ARG;
     if (N == 0) return KVQ_OK;
-    cudaError_t e = launch_debug_rotate_small(X, N, mode, R, perm, Xrot,
-                                              static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = (variant == 1 && mode == KVQ_ROT_DENSE)
+                        ? launch_debug_rotate_tc(X, N, R, Xrot, st)
+                        : launch_debug_rotate_small(X, N, mode, R, perm, Xrot, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

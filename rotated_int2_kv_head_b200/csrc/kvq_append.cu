@@ -21,38 +21,6 @@
 
 namespace kvq {
 
-// Where a rotated row goes: into the packed cache, or out as fp32 (tests).
-struct CacheDst {
-    uint8_t *blocks;
-    uint16_t *k_sink, *v_sink;
-    int32_t *seq_lens;
-    int32_t *status;          // [0] error bits, [1] CTA completion counter
-    int B, T, Hkv, capacity, S, nblk;
-};
-
-// Called by every CTA of an append kernel after its last read of seq_lens
-// and its last write: the CTA that completes last bumps the lengths and
-// resets the counter for the next append.
-__device__ void append_done(const CacheDst &c) {
-    __shared__ int last;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned total = gridDim.x * gridDim.y * gridDim.z;
-        const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(c.status + 1), 1u);
-        last = (prev == total - 1);
-        if (last) __threadfence();
-    }
-    __syncthreads();
-    if (last) {
-        for (int b = threadIdx.x; b < c.B; b += blockDim.x) {
-            const int L0 = c.seq_lens[b];
-            if (L0 >= 0 && (long long)L0 + c.T <= c.capacity) c.seq_lens[b] = L0 + c.T;
-        }
-        if (threadIdx.x == 0) atomicExch(reinterpret_cast<unsigned *>(c.status + 1), 0u);
-    }
-}
-
 // Epilogue shared by both append kernels: row (b, t, h, kind) with rotated
 // values v (lane layout of quantize_row_warp).
 __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, int h, int kind,
@@ -73,21 +41,6 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
         const QuantWord q = quantize_row_warp(v);
         store_token_warp(block, tau, kind, q);
     }
-}
-
-// Reads seq_lens[b] and checks capacity; returns -1 (and flags) if the
-// sequence must be skipped.
-__device__ __forceinline__ int start_len(const CacheDst &c, int b) {
-    const int L0 = c.seq_lens[b];
-    if (L0 < 0) {
-        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_BAD_LEN);
-        return -1;
-    }
-    if ((long long)L0 + c.T > c.capacity) {
-        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_CAPACITY);
-        return -1;
-    }
-    return L0;
 }
 
 // ---- dense rotation on CUDA cores ---------------------------------------------------------

@@ -275,6 +275,15 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
                                 cudaStream_t st);
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
                                       const int32_t *perm, float *out, cudaStream_t st);
+// Bulk dense appends (T >= TC_MIN_T, 16-byte aligned K and V) run the
+// rotation on the tensor cores.
+constexpr int TC_MIN_T = 256;
+bool append_tc_eligible(const uint16_t *K, const uint16_t *V, int T);
+cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const float *R_k,
+                             const float *R_v, const kvq_cache_desc &cd, int32_t *seq_lens,
+                             cudaStream_t st);
+cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, const float *R, float *out,
+                                   cudaStream_t st);
 cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
                                   cudaStream_t st);
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
@@ -287,5 +296,69 @@ struct WsLayout {
     size_t qprep, part, total;
 };
 WsLayout ws_layout(int B, int Hq, int Hkv, int C);
+
+
+// ---- append destination and completion (shared by the append kernels) ---------------
+// Where a rotated row goes: into the packed cache, or out as fp32 (tests).
+struct CacheDst {
+    uint8_t *blocks;
+    uint16_t *k_sink, *v_sink;
+    int32_t *seq_lens;
+    int32_t *status;          // [0] error bits, [1] CTA completion counter
+    int B, T, Hkv, capacity, S, nblk;
+};
+
+// Called by every CTA of an append kernel after its last read of seq_lens
+// and its last write: the CTA that completes last bumps the lengths and
+// resets the counter for the next append.
+static __device__ void append_done(const CacheDst &c) {
+    __shared__ int last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+        const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(c.status + 1), 1u);
+        last = (prev == total - 1);
+        if (last) __threadfence();
+    }
+    __syncthreads();
+    if (last) {
+        for (int b = threadIdx.x; b < c.B; b += blockDim.x) {
+            const int L0 = c.seq_lens[b];
+            if (L0 >= 0 && (long long)L0 + c.T <= c.capacity) c.seq_lens[b] = L0 + c.T;
+        }
+        if (threadIdx.x == 0) atomicExch(reinterpret_cast<unsigned *>(c.status + 1), 0u);
+    }
+}
+
+// Reads seq_lens[b] and checks capacity; returns -1 (and flags) if the
+// sequence must be skipped.
+__device__ __forceinline__ int start_len(const CacheDst &c, int b) {
+    const int L0 = c.seq_lens[b];
+    if (L0 < 0) {
+        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_BAD_LEN);
+        return -1;
+    }
+    if ((long long)L0 + c.T > c.capacity) {
+        if (threadIdx.x == 0) set_status(c.status, KVQ_DEV_CAPACITY);
+        return -1;
+    }
+    return L0;
+}
+
+// Per-thread variant: every caller gets L0 (or -1); only callers with
+// `report` set flag the status.
+__device__ __forceinline__ int start_len_thread(const CacheDst &c, int b, bool report) {
+    const int L0 = c.seq_lens[b];
+    if (L0 < 0) {
+        if (report) set_status(c.status, KVQ_DEV_BAD_LEN);
+        return -1;
+    }
+    if ((long long)L0 + c.T > c.capacity) {
+        if (report) set_status(c.status, KVQ_DEV_CAPACITY);
+        return -1;
+    }
+    return L0;
+}
 
 }  // namespace kvq

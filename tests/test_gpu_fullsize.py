@@ -146,7 +146,9 @@ def test_ragged_prefill_append_full():
     for b, h, t in picks:
         for kind, X, R in ((0, K, Rk), (1, V, Rv)):
             x = X[b, t, h][None].contiguous()
-            grot = kvq.kvq_debug_rotate_f32(x, 0, R=(rk if kind == 0 else rv)[h].contiguous())
+            # the bulk append ran the tensor-core kernel: same rotation here
+            grot = kvq.kvq_debug_rotate_f32(x, 0, R=(rk if kind == 0 else rv)[h].contiguous(),
+                                            variant=1)
             c, s, z = orc.quantize_rows(grot.cpu().numpy())
             blk = blocks[b, h, t // 16].cpu().numpy()
             kb, vb, ks, kz, vs, vz = orc.load_token(blk, t % 16)

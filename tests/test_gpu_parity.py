@@ -66,8 +66,11 @@ def test_quantizer_bit_exact():
     assert np.array_equal(meta[:, :, 1], oz)
 
 
-@pytest.mark.parametrize("mode", [0, 1])
-def test_rotation_stage(mode):
+@pytest.mark.parametrize("mode,variant", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_rotation_stage(mode, variant):
+    """variant 0: the small-batch append kernel's rotation; 1: the bulk
+    kernel's (dense: tcgen05 with R as fp16 hi + lo), over 3000 rows =
+    23 full 128-row tiles and a ragged one."""
     w = W.custom(seed=3, Hkv=1, mode=mode, k_outliers=8)
     rng = np.random.default_rng(2)
     x = (rng.standard_normal((3000, D)) * 3).astype(np.float16)
@@ -75,7 +78,7 @@ def test_rotation_stage(mode):
     rt, rn = rot_tensors(w)
     X = torch.from_numpy(x).cuda()
     if mode == 0:
-        got = kvq.kvq_debug_rotate_f32(X, 0, R=rt[0][0].contiguous())
+        got = kvq.kvq_debug_rotate_f32(X, 0, R=rt[0][0].contiguous(), variant=variant)
         ref = orc.rotate_rows_f32(x.view(np.uint16), 0, R=rn[0][0])
     else:
         got = kvq.kvq_debug_rotate_f32(X, 1, perm=rt[2][0, 0].contiguous())
@@ -113,6 +116,10 @@ def run_append(w, L0, T, device="cuda"):
     (1, 0, 37, [0, 5, 16]),
     (1, 4, 1, [3, 0, 21]),
     (0, 20, 70, [0, 2, 31]),
+    # bulk dense appends (T >= 256): tensor-core kernel; T=2400 gives 228
+    # tiles, so CTAs cross (sequence, head, K|V) boundaries mid-range
+    (0, 20, 520, [0, 2, 31]),
+    (0, 0, 2400, [0, 7, 16]),
 ])
 def test_append_matches_oracle(mode, S, T, L0):
     w = W.custom(seed=10 + T, B=3, Hkv=2, mode=mode, sink=S, k_outliers=4,
@@ -128,7 +135,8 @@ def test_append_matches_oracle(mode, S, T, L0):
             rows = X[:, :, h].reshape(-1, D).cuda()
             if mode == 0:
                 R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
-                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R).cpu().numpy()
+                variant = 1 if T >= 256 else 0     # the kernel the append used
+                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=variant).cpu().numpy()
                 orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 0,
                                       R=(rn[0] if kind == 0 else rn[1])[h])
             else:
