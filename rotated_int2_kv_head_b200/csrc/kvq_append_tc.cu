@@ -12,9 +12,9 @@
 //     x . R_hi + x . R_lo carries about 22 bits of R and accumulates in fp32.
 //   * warp 0 streams 128-row tiles of x with 3-D TMA copies (128-byte
 //     swizzle, the layout the MMA reads) into a 3-stage ring;
-//   * warp 1 owns 256 TMEM columns (two 128x128 fp32 accumulators) and
+//   * warp 1 owns all 512 TMEM columns (four 128x128 fp32 accumulators) and
 //     issues, per tile, 16 tcgen05.mma (hi and lo, K = 128 in steps of 16);
-//   * warps 2..9 form two epilogue groups that take alternate tiles: each
+//   * warps 2..17 form four epilogue groups that take every fourth tile: each
 //     thread reads one accumulator row with tcgen05.ld and quantizes it
 //     group by group in registers (min/max, fp16 scale and zero, codes
 //     packed four per byte) and writes the row into the packed cache (or
@@ -43,18 +43,20 @@ constexpr int A_HALF = TILE_M * 128;           // one 64-column half of an x til
 constexpr int A_BYTES = 2 * A_HALF;            // 32 KB
 constexpr int B_HALF = D * 128;                // one 64-column (K) half of R^T (16 KB)
 constexpr int B_PART = 2 * B_HALF;             // R_hi or R_lo (32 KB)
-constexpr int EPI_GROUPS = 2;
+constexpr int EPI_GROUPS = 4;                  // epilogue groups = accumulators in flight
 constexpr int EPI_WARPS = 4 * EPI_GROUPS;
-constexpr int THREADS = 32 * (2 + EPI_WARPS);  // 320
-constexpr uint32_t TMEM_COLS = 256;            // two 128-column fp32 accumulators
+constexpr int THREADS = 32 * (2 + EPI_WARPS);  // 576
+constexpr uint32_t TMEM_COLS = 128 * EPI_GROUPS;   // one 128-column fp32 accumulator per group
 
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + A_STAGES * A_BYTES;
 constexpr int OFF_BAR = OFF_B + 2 * B_PART;
-// barriers: full_a[A_STAGES], empty_a[A_STAGES], acc_full[2], acc_empty[2], b_ready
+// barriers: full_a[A_STAGES], empty_a[A_STAGES], acc_full[EPI_GROUPS],
+// acc_empty[EPI_GROUPS], b_ready
 constexpr int BAR_FULL = 0, BAR_EMPTY = A_STAGES, BAR_ACCF = 2 * A_STAGES,
-              BAR_ACCE = 2 * A_STAGES + 2, BAR_BREADY = 2 * A_STAGES + 4, NBAR = 2 * A_STAGES + 5;
+              BAR_ACCE = 2 * A_STAGES + EPI_GROUPS, BAR_BREADY = 2 * A_STAGES + 2 * EPI_GROUPS,
+              NBAR = 2 * A_STAGES + 2 * EPI_GROUPS + 1;
 constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
 constexpr int SMEM_USED = OFF_ABORT + 16;
@@ -182,21 +184,34 @@ __device__ __forceinline__ void convert_r(const float *R, uint8_t *bhi, uint8_t 
 // pattern is 0x4B400000 + c.  That pattern, shifted to the code's place, is
 // added into the word (one integer multiply-add; the codes' bits never
 // overlap), and the constant 0x4B400000-terms are taken out once per word.
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t quantize_group_thread(const float (&v)[32], int g,
                                                           uint32_t (&words)[8]) {
-    float mn[16], mx[16];
+    // min and max of the 32 values with three-input min/max: 32 -> 12 -> 4 -> 1
+    float mn[12], mx[12];
 #pragma unroll
-    for (int e = 0; e < 16; e++) {
-        mn[e] = fminf(v[e], v[e + 16]);
-        mx[e] = fmaxf(v[e], v[e + 16]);
+    for (int e = 0; e < 10; e++) {
+        mn[e] = fmin3(v[3 * e], v[3 * e + 1], v[3 * e + 2]);
+        mx[e] = fmax3(v[3 * e], v[3 * e + 1], v[3 * e + 2]);
     }
+    mn[10] = v[30], mn[11] = v[31], mx[10] = v[30], mx[11] = v[31];
 #pragma unroll
-    for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-        for (int e = 0; e < w; e++) {
-            mn[e] = fminf(mn[e], mn[e + w]);
-            mx[e] = fmaxf(mx[e], mx[e + w]);
-        }
+    for (int e = 0; e < 4; e++) {
+        mn[e] = fmin3(mn[3 * e], mn[3 * e + 1], mn[3 * e + 2]);
+        mx[e] = fmax3(mx[3 * e], mx[3 * e + 1], mx[3 * e + 2]);
+    }
+    mn[0] = fminf(fmin3(mn[0], mn[1], mn[2]), mn[3]);
+    mx[0] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
     const float r = __fsub_rn(mx[0], mn[0]);
     const float sf = __fdiv_rn(r, 3.0f);
     const __half s = __float2half_rn(__fadd_rn(sf, 0.0f));   // zero stored as +0
@@ -251,7 +266,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_init(&bar[BAR_FULL + i], 1);
             mbar_init(&bar[BAR_EMPTY + i], 1);
         }
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < EPI_GROUPS; i++) {
             mbar_init(&bar[BAR_ACCF + i], 1);
             mbar_init(&bar[BAR_ACCE + i], 4);       // the four warps of an epilogue group
         }
@@ -307,12 +322,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             int nb = 0;   // B-operand versions consumed
             int i = 0;
             for (; i < nmy && !*abort_flag; i++) {
-                const int k = k0 + i, s = i % A_STAGES, buf = i & 1;
+                const int k = k0 + i, s = i % A_STAGES, buf = i % EPI_GROUPS;
                 if (i == 0 || job_of(k) != job_of(k - 1)) {
                     if (!mbar_wait_bounded(&bar[BAR_BREADY], nb & 1)) { fail(); break; }
                     ++nb;
                 }
-                if (i >= 2 && !mbar_wait_bounded(&bar[BAR_ACCE + buf], ((i >> 1) - 1) & 1)) {
+                if (i >= EPI_GROUPS &&
+                    !mbar_wait_bounded(&bar[BAR_ACCE + buf], ((i / EPI_GROUPS) - 1) & 1)) {
                     fail();
                     break;
                 }
@@ -337,11 +353,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 mma_commit(&bar[BAR_ACCF + buf]);     // accumulator ready
             }
             // the accumulators are freed below: the last MMAs must have completed
-            if (i > 0) mbar_wait_bounded(&bar[BAR_ACCF + ((i - 1) & 1)], ((i - 1) >> 1) & 1, 1u << 10);
+            if (i > 0)
+                mbar_wait_bounded(&bar[BAR_ACCF + (i - 1) % EPI_GROUPS], ((i - 1) / EPI_GROUPS) & 1,
+                                  1u << 10);
         }
     } else {
         // ---- epilogue groups
-        const int eg = (warp - 2) >> 2;                 // group 0: warps 2-5, group 1: warps 6-9
+        const int eg = (warp - 2) >> 2;                 // group g: warps 2+4g .. 5+4g
         const int gt = threadIdx.x - 64 - 128 * eg;     // 0..127 within the group
         const int q = warp & 3;                         // TMEM lane quarter this warp may read
         const int row = 32 * q + lane;                  // accumulator row = tile row
@@ -358,8 +376,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         for (int i = eg; i < nmy; i += EPI_GROUPS) {
             // decisions stay warp-uniform: tcgen05.ld below is .sync.aligned
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            const int k = k0 + i, j = job_of(k), buf = i & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bar[BAR_ACCF + buf], (i >> 1) & 1))) {
+            const int k = k0 + i, j = job_of(k), buf = i % EPI_GROUPS;     // = eg
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(&bar[BAR_ACCF + buf], (i / EPI_GROUPS) & 1))) {
                 fail();
                 break;
             }
