@@ -30,11 +30,13 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Compute
  *     calls are asynchronous on it; argument errors are reported before any
  *     launch and nothing is launched then.  The kernels use programmatic
- *     dependent launch: the rotation inputs (R_k, R_v, perm) may be read
- *     while the work enqueued just before the call is still finishing, so
- *     they must not be written by that work (set them up once, or make the
- *     writer complete - e.g. with an event - before the call).  Every other
- *     input is read only after the preceding work in the stream completed.
+ *     dependent launch: the rotation inputs (R_k, R_v, perm) and the decode
+ *     queries Q may be read while the kernel enqueued just before the call
+ *     is still finishing, so they must not be written by that kernel when it
+ *     is itself launched with programmatic dependent launch (a kernel
+ *     launched the ordinary way has completed by then; a libkvq append
+ *     before a decode writes neither).  Every other input is read only after
+ *     the preceding work in the stream completed.
  *   - Device-detected errors never trap: they OR a bit into cache->status[0]
  *     (see KVQ_DEV_*) and the affected work is skipped.
  *

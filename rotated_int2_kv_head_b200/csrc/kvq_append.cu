@@ -67,9 +67,6 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     __shared__ __align__(16) uint16_t xs[DENSE_BATCH][D];
     __shared__ __align__(16) float red[DENSE_BATCH][8][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    pdl_wait();
-    pdl_trigger();
-
     int b = 0, h = 0, kind = 0, L0 = 0, row0, nrows;
     const uint16_t *X;
     const float *R;
@@ -77,22 +74,14 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         h = blockIdx.y;
         kind = blockIdx.z & 1;
         b = blockIdx.z >> 1;
-        L0 = start_len(c, b);
-        row0 = blockIdx.x * a.tchunk;
-        nrows = L0 < 0 ? 0 : min(a.tchunk, c.T - row0);     // skipped sequence: no rows
         X = (kind == 0 ? a.X0 : a.X1);
         R = (kind == 0 ? a.R0 : a.R1) + (size_t)h * D * D;
     } else {
-        row0 = blockIdx.x * a.tchunk;
-        nrows = min(a.tchunk, a.n_rows - row0);
         X = a.X0;
         R = a.R0;
     }
-    if (nrows <= 0) {
-        if (TO_CACHE) append_done(c);
-        return;
-    }
-
+    // R (a rotation input, never written by the work this kernel waits on) is
+    // fetched before the dependency wait, overlapping the preceding kernel
     float Rr[16][4];
 #pragma unroll
     for (int ii = 0; ii < 16; ii++) {
@@ -101,6 +90,20 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         Rr[ii][1] = r4.y;
         Rr[ii][2] = r4.z;
         Rr[ii][3] = r4.w;
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (TO_CACHE) {
+        L0 = start_len(c, b);
+        row0 = blockIdx.x * a.tchunk;
+        nrows = L0 < 0 ? 0 : min(a.tchunk, c.T - row0);     // skipped sequence: no rows
+    } else {
+        row0 = blockIdx.x * a.tchunk;
+        nrows = min(a.tchunk, a.n_rows - row0);
+    }
+    if (nrows <= 0) {
+        if (TO_CACHE) append_done(c);
+        return;
     }
 
     for (int base = 0; base < nrows; base += DENSE_BATCH) {

@@ -112,18 +112,20 @@ __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
 // block: group g gets s (an empty range when the CTA's range is short).
 // Thread t covers a contiguous run of sequences; an exclusive shuffle scan
 // of the runs' block counts gives every run's offset.  scratch:
-// 2*DEC_GROUPS + DEC_WARPS ints of shared memory.  Returns false when the
+// 3*DEC_GROUPS + DEC_WARPS ints of shared memory.  Returns false when the
 // CTA's range is empty (uniformly over the CTA).  CTA 0 flags invalid
 // lengths.
 __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
     const int lo = min(a.B, t * per), hi = min(a.B, lo + per);
-    int sum = 0;
+    int sum = 0, nb_lo = 0;          // nb_lo: blocks per unit of sequence lo (kept in a register)
     for (int b = lo; b < hi; b++) {
         const int L = a.seq_lens[b];
         if (blockIdx.x == 0 && (L < 1 || L > a.capacity)) set_status(a.status, KVQ_DEV_BAD_LEN);
-        sum += a.Hkv * unit_blocks(L, a.S, a.capacity);
+        const int nb = unit_blocks(L, a.S, a.capacity);
+        if (b == lo) nb_lo = nb;
+        sum += a.Hkv * nb;
     }
     int incl = sum;
 #pragma unroll
@@ -131,7 +133,7 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
         const int v = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += v;
     }
-    int *wsum = scratch + 2 * DEC_GROUPS;         // [DEC_WARPS]
+    int *wsum = scratch + 3 * DEC_GROUPS;         // [DEC_WARPS]
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     int woff = 0, N = 0;
@@ -146,20 +148,22 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     const int beg = blockIdx.x * W, end = min(N, beg + W);
     if (beg >= end) return false;
     const int Wg = (end - beg + DEC_GROUPS - 1) / DEC_GROUPS;
-    // the run holding each part's first block finds its sequence
+    // the run holding each part's first block publishes (sequence, its first
+    // global block, blocks per unit)
 #pragma unroll
     for (int g = 0; g < DEC_GROUPS; g++) {
         const int p = beg + g * Wg;
         if (p < end && cstart <= p && p < cend) {
             int acc = cstart;
             for (int b = lo; b < hi; b++) {
-                const int nbb = a.Hkv * seq_blocks(a, b);
-                if (p < acc + nbb) {
-                    scratch[2 * g] = b;
-                    scratch[2 * g + 1] = acc;
+                const int nbu = b == lo ? nb_lo : seq_blocks(a, b);
+                if (p < acc + a.Hkv * nbu) {
+                    scratch[3 * g] = b;
+                    scratch[3 * g + 1] = acc;
+                    scratch[3 * g + 2] = nbu;
                     break;
                 }
-                acc += nbb;
+                acc += a.Hkv * nbu;
             }
         }
     }
@@ -167,9 +171,9 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     const int g = threadIdx.x / GROUP_THREADS;
     const int p = beg + g * Wg;
     if (p < end) {
-        s.b = scratch[2 * g];
-        s.pref = scratch[2 * g + 1];
-        s.nb = seq_blocks(a, s.b);
+        s.b = scratch[3 * g];
+        s.pref = scratch[3 * g + 1];
+        s.nb = scratch[3 * g + 2];
         s.h = (p - s.pref) / s.nb;
         s.ustart = s.pref + s.h * s.nb;
         s.cur = p;
@@ -178,7 +182,6 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
         s.b = s.h = s.nb = s.ustart = s.pref = 0;
         s.cur = s.end = 0;
     }
-    __syncthreads();
     return true;
 }
 
@@ -202,8 +205,8 @@ __device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &
 // FWHT), scaled by log2(e)/sqrt(128) so scores are exp2 exponents, and per
 // group an int8 hi/lo pair on the scale max|q_s|/127 (about 15 significant
 // bits): qprep[(b*Hq + hq)*QB] = {hi[128], lo[128], kap[4] = sq_g/4^g,
-// qsum[4]}.  R_k (64 KB per head, the bulk of what it reads) is loaded before
-// the dependency wait, alongside a preceding append; Q after it.
+// qsum[4]}.  The whole preparation (R_k, 64 KB per head, and Q) runs before
+// the dependency wait, alongside a preceding append.
 // ---------------------------------------------------------------------------------------------
 constexpr int QP_THREADS = 256;
 
@@ -219,17 +222,6 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
         const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
 #pragma unroll
         for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
-    }
-    pdl_wait();
-    pdl_trigger();
-    // mark every split partial empty (m = -inf, l = 0): a group of the split
-    // kernel writes only the units it took stages of
-    {
-        const size_t nslots = (size_t)DEC_GROUPS * ((size_t)a.C + (size_t)a.B * a.Hkv) * G;
-        const size_t stride = (size_t)gridDim.x * gridDim.y * QP_THREADS;
-        for (size_t i = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * QP_THREADS + t; i < nslots;
-             i += stride)
-            *reinterpret_cast<float2 *>(a.part + i * PART) = make_float2(NEG_INF, 0.f);
     }
     for (int hd = 0; hd < G; hd++) {
         const int hq = h * G + hd;
@@ -291,6 +283,22 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
                 qf[4 + warp] = gs;
             }
         }
+    }
+    // Everything above reads only inputs of the call and writes only the
+    // prepared queries (whose last reader, the previous call's split kernel,
+    // finished before this kernel could start), so it runs before the
+    // dependency wait, alongside a preceding append.  The partial slots may
+    // still be read by a preceding call's merge: they are reset after it.
+    pdl_wait();
+    pdl_trigger();
+    // mark every split partial empty (m = -inf, l = 0): a group of the split
+    // kernel writes only the units it took stages of
+    {
+        const size_t nslots = (size_t)DEC_GROUPS * ((size_t)a.C + (size_t)a.B * a.Hkv) * G;
+        const size_t stride = (size_t)gridDim.x * gridDim.y * QP_THREADS;
+        for (size_t i = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * QP_THREADS + t; i < nslots;
+             i += stride)
+            *reinterpret_cast<float2 *>(a.part + i * PART) = make_float2(NEG_INF, 0.f);
     }
 }
 
@@ -364,7 +372,7 @@ __host__ __device__ inline SplitSmem split_smem_layout(int G) {
     L.fz = smem_up16(L.fl + 4u * GROUP_WARPS * G);
     L.gstride = (L.fz + 4u * GROUP_WARPS * G * 4 + 127u) & ~127u;
     L.scratch = DEC_GROUPS * L.gstride;
-    L.total = smem_up16(L.scratch + 4u * (2 * DEC_GROUPS + DEC_WARPS));
+    L.total = smem_up16(L.scratch + 4u * (3 * DEC_GROUPS + DEC_WARPS));
     return L;
 }
 

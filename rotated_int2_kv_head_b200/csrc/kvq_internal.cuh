@@ -313,13 +313,15 @@ struct CacheDst {
 // resets the counter for the next append.
 static __device__ void append_done(const CacheDst &c) {
     __shared__ int last;
+    // Ordering: every thread of this CTA has read seq_lens (and used the
+    // value) before the barrier, nothing writes seq_lens during the kernel,
+    // and the next kernel sees the bump once this one completes, so no
+    // memory fence is needed around the counter.
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
         const unsigned total = gridDim.x * gridDim.y * gridDim.z;
         const unsigned prev = atomicAdd(reinterpret_cast<unsigned *>(c.status + 1), 1u);
         last = (prev == total - 1);
-        if (last) __threadfence();
     }
     __syncthreads();
     if (last) {
