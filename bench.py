@@ -295,16 +295,21 @@ class Step:
 
 def append_rates(device, peak, reps=5):
     """Throughput of the append alone (rotate + quantize + pack + store) on the
-    two bulk appends of the workload set: the ragged workload's prefill (B=4,
-    32768 tokens, 32 heads, dense rotation) and the hadamard workload's step
-    append (B=16, 128 tokens, 32 heads, permutation + FWHT).  Bytes = fp16 K
+    bulk appends of the workload set: the llama7b prefill (B=1, 32768 tokens,
+    32 heads, dense), the ragged workload's prefill (B=4, 32768 tokens, 32
+    heads, dense) and the hadamard workload's step append (B=16, 128 tokens,
+    32 heads, permutation + FWHT).  Bytes = fp16 K
     and V read (512 B per token-head) + packed codes and metadata written
     (96 B) + the rotations read once; L2 flushed before each timed call."""
     import rotated_int2_kv_head_b200 as kvq
     flush = L2Flush(device)
     out = {}
     w0 = W.WORKLOADS["ragged"]
-    cases = [("ragged prefill", W.custom(name="ragged_prefill", seed=w0.seed + 1, B=w0.extra["prefill_B"],
+    wl = W.WORKLOADS["llama7b"]
+    cases = [("llama7b prefill", W.custom(name="llama7b_prefill", seed=wl.seed + 1, B=1, Hq=32,
+                                          Hkv=32, mode=0, k_outliers=8, context=wl.context),
+              wl.context),
+             ("ragged prefill", W.custom(name="ragged_prefill", seed=w0.seed + 1, B=w0.extra["prefill_B"],
                                          Hq=32, Hkv=32, mode=0, k_outliers=8,
                                          context=w0.extra["prefill_T"]), w0.extra["prefill_T"]),
              ("hadamard step append", W.WORKLOADS["hadamard"], W.WORKLOADS["hadamard"].append_T)]
@@ -650,11 +655,20 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama7b", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
+    ap.add_argument("--append-only", action="store_true",
+                    help="only the bulk-append rates (one GPU), as one JSON line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.append_only:
+        torch.cuda.set_device(0)
+        from rotated_int2_kv_head_b200 import build as kbuild
+        kbuild.build()
+        peak, src = measured_peak()
+        print(json.dumps({"append": append_rates(torch.device("cuda", 0), peak), "peak_gbs": peak,
+                          "peak_source": src}), flush=True)
     else:
         run_cuda(args)
 
