@@ -30,13 +30,13 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Compute
  *     calls are asynchronous on it; argument errors are reported before any
  *     launch and nothing is launched then.  The kernels use programmatic
- *     dependent launch: the rotation inputs (R_k, R_v, perm) and the decode
- *     queries Q may be read while the kernel enqueued just before the call
- *     is still finishing, so they must not be written by that kernel when it
- *     is itself launched with programmatic dependent launch (a kernel
- *     launched the ordinary way has completed by then; a libkvq append
- *     before a decode writes neither).  Every other input is read only after
- *     the preceding work in the stream completed.
+ *     dependent launch: the rotation inputs (R_k, R_v, perm) may be read
+ *     while the kernel enqueued just before the call is still finishing, so
+ *     they must not be written by that kernel when it is itself launched
+ *     with programmatic dependent launch (a kernel launched the ordinary way
+ *     has completed by then; a libkvq append writes none of them).  Every
+ *     other input is read only after the preceding work in the stream
+ *     completed.
  *   - Device-detected errors never trap: they OR a bit into cache->status[0]
  *     (see KVQ_DEV_*) and the affected work is skipped.
  *
@@ -234,6 +234,34 @@ KVQ_API kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mo
                                 float *Xrot, void *stream);
 KVQ_API kvq_status kvq_debug_quantize_f32(const float *Xrot, int32_t N, uint8_t *codes,
                                   uint16_t *meta, void *stream);
+
+/* Options of kvq_decode_attention_ex. */
+#define KVQ_DECODE_OUT_ROTATED 1u  /* out = o_rot: the caller applies R_v^T (or the inverse
+                                      permutation + FWHT) itself, e.g. folded into W_O */
+
+/*
+ * Decode with q_len new tokens per sequence (multi-query / speculative
+ * decode) and options.  The q_len tokens are the last ones already appended:
+ * query i (0 <= i < q_len) of a sequence of length L is the token at
+ * position L - q_len + i and attends to positions [0, L - q_len + i], i.e.
+ * causally among the new tokens; each is the standard attention of
+ * kvq_decode_attention (OptR page, "Why It Matters") over its own prefix.
+ *   Q        fp16 [B][Hq][q_len][128]; out fp16 [B][Hq][q_len][128].
+ *   q_len    1..8 with (Hq / Hkv) * q_len in {1, 2, 4, 8}.
+ *   flags    0 or KVQ_DECODE_OUT_ROTATED.
+ *   workspace >= kvq_decode_workspace_size(B, Hq * q_len, Hkv, max_ctx, SMs).
+ *   max_ctx  >= q_len.
+ * Other arguments and errors as kvq_decode_attention.  A sequence with
+ * seq_lens[b] < q_len gets zero rows for the queries that would start
+ * before position 0 and sets KVQ_DEV_BAD_LEN.  q_len = 1 with flags = 0 is
+ * exactly kvq_decode_attention.
+ */
+KVQ_API kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_t q_len,
+                                   uint32_t flags, const kvq_cache_desc *cache,
+                                   kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                   const int32_t *perm, const int32_t *seq_lens,
+                                   int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                   size_t ws_bytes, uint16_t *out, void *stream);
 
 /* Short text for a status code (static storage). */
 KVQ_API const char *kvq_status_string(kvq_status s);

@@ -101,31 +101,63 @@ size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max
     return ws_layout(B, Hq, Hkv, C).total;
 }
 
-kvq_status kvq_decode_attention_timed(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
-                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
-                                      const int32_t *perm, const int32_t *seq_lens,
-                                      int32_t sink_fp16, int32_t max_ctx, void *workspace,
-                                      size_t ws_bytes, uint16_t *out, void *stream, void *ev_begin,
-                                      void *ev_end) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of the decode entry points: q_len queries per sequence (Hq
+// heads each), options in flags, optional events around the split kernel.
+kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t flags,
+                       const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
+                       const float *R_v, const int32_t *perm, const int32_t *seq_lens,
+                       int32_t sink_fp16, int32_t max_ctx, void *workspace, size_t ws_bytes,
+                       uint16_t *out, void *stream, void *ev_begin, void *ev_end) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
     if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
     if (!Q || !out || !seq_lens || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(Q, 16) || !aligned(out, 16) || !aligned(workspace, 256) || !aligned(seq_lens, 4))
         return KVQ_ERR_UNSUPPORTED;
-    if (Hq < cache->Hkv || Hq % cache->Hkv != 0 || Hq > 65535) return KVQ_ERR_INVALID_ARG;
-    const int G = Hq / cache->Hkv;
+    if (q_len < 1 || q_len > 8 || (flags & ~KVQ_DECODE_OUT_ROTATED) != 0) return KVQ_ERR_INVALID_ARG;
+    if (Hq < cache->Hkv || Hq % cache->Hkv != 0 || (long long)Hq * q_len > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    const int Hqq = Hq * q_len;                     // query rows per sequence
+    const int G = Hqq / cache->Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8) return KVQ_ERR_UNSUPPORTED;
     if (sink_fp16 != cache->sink_fp16) return KVQ_ERR_INVALID_ARG;
-    if (max_ctx < 1 || max_ctx > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    if (max_ctx < q_len || max_ctx > cache->capacity) return KVQ_ERR_INVALID_ARG;
     const int sms = device_sm_count();
     if (sms < 1) return KVQ_ERR_CUDA;
     const int C = split_ctas(cache->B, cache->Hkv, max_ctx, sms);
-    if (ws_bytes < ws_layout(cache->B, Hq, cache->Hkv, C).total) return KVQ_ERR_WORKSPACE;
-    cudaError_t e = launch_decode(Q, Hq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out,
+    if (ws_bytes < ws_layout(cache->B, Hqq, cache->Hkv, C).total) return KVQ_ERR_WORKSPACE;
+    cudaError_t e = launch_decode(Q, Hqq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out,
                                   static_cast<cudaStream_t>(stream),
-                                  static_cast<cudaEvent_t>(ev_begin), static_cast<cudaEvent_t>(ev_end));
+                                  static_cast<cudaEvent_t>(ev_begin), static_cast<cudaEvent_t>(ev_end),
+                                  q_len, (flags & KVQ_DECODE_OUT_ROTATED) ? 1 : 0);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention_timed(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                      const int32_t *perm, const int32_t *seq_lens,
+                                      int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                      size_t ws_bytes, uint16_t *out, void *stream, void *ev_begin,
+                                      void *ev_end) {
+    return decode_impl(Q, Hq, 1, 0u, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
+                       workspace, ws_bytes, out, stream, ev_begin, ev_end);
+}
+
+kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t flags,
+                                   const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
+                                   const float *R_v, const int32_t *perm, const int32_t *seq_lens,
+                                   int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                   size_t ws_bytes, uint16_t *out, void *stream) {
+    return decode_impl(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
+                       max_ctx, workspace, ws_bytes, out, stream, nullptr, nullptr);
 }
 
 kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,

@@ -70,6 +70,10 @@ struct DecodeArgs {
     float *part;       // [(C+U)*G][PART]
     uint16_t *out;
     int B, Hq, Hkv, G, S, capacity, nblk, mode, C;
+    // qlen queries per sequence: query "head" hq (of Hq = heads x qlen) is
+    // query i = hq % qlen of its head and sees positions < L - (qlen-1-i)
+    int qlen;
+    int out_rotated;   // 1: out = o_rot (the caller folds R_v^T into its projection)
 };
 
 // Blocks of 16 tokens that hold codes for a sequence of length L: positions
@@ -205,8 +209,8 @@ __device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &
 // FWHT), scaled by log2(e)/sqrt(128) so scores are exp2 exponents, and per
 // group an int8 hi/lo pair on the scale max|q_s|/127 (about 15 significant
 // bits): qprep[(b*Hq + hq)*QB] = {hi[128], lo[128], kap[4] = sq_g/4^g,
-// qsum[4]}.  The whole preparation (R_k, 64 KB per head, and Q) runs before
-// the dependency wait, alongside a preceding append.
+// qsum[4]}.  R_k (64 KB per head, the bulk of what it reads) is fetched
+// before the dependency wait, alongside a preceding append; Q after it.
 // ---------------------------------------------------------------------------------------------
 constexpr int QP_THREADS = 256;
 
@@ -222,6 +226,19 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
         const float *R = a.R_k + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
 #pragma unroll
         for (int ii = 0; ii < 16; ii++) rr[ii] = *reinterpret_cast<const float4 *>(R + ii * D);
+    }
+    // Waiting here (R_k is already on its way) and letting the split kernel
+    // launch right away lets the query work below overlap its start-up.
+    pdl_wait();
+    pdl_trigger();
+    // mark every split partial empty (m = -inf, l = 0): a group of the split
+    // kernel writes only the units it took stages of
+    {
+        const size_t nslots = (size_t)DEC_GROUPS * ((size_t)a.C + (size_t)a.B * a.Hkv) * G;
+        const size_t stride = (size_t)gridDim.x * gridDim.y * QP_THREADS;
+        for (size_t i = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * QP_THREADS + t; i < nslots;
+             i += stride)
+            *reinterpret_cast<float2 *>(a.part + i * PART) = make_float2(NEG_INF, 0.f);
     }
     for (int hd = 0; hd < G; hd++) {
         const int hq = h * G + hd;
@@ -283,22 +300,6 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
                 qf[4 + warp] = gs;
             }
         }
-    }
-    // Everything above reads only inputs of the call and writes only the
-    // prepared queries (whose last reader, the previous call's split kernel,
-    // finished before this kernel could start), so it runs before the
-    // dependency wait, alongside a preceding append.  The partial slots may
-    // still be read by a preceding call's merge: they are reset after it.
-    pdl_wait();
-    pdl_trigger();
-    // mark every split partial empty (m = -inf, l = 0): a group of the split
-    // kernel writes only the units it took stages of
-    {
-        const size_t nslots = (size_t)DEC_GROUPS * ((size_t)a.C + (size_t)a.B * a.Hkv) * G;
-        const size_t stride = (size_t)gridDim.x * gridDim.y * QP_THREADS;
-        for (size_t i = ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * QP_THREADS + t; i < nslots;
-             i += stride)
-            *reinterpret_cast<float2 *>(a.part + i * PART) = make_float2(NEG_INF, 0.f);
     }
 }
 
@@ -614,7 +615,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         // a block needs masking if it is a phantom or crosses [S, L)
 #pragma unroll
         for (int bi = 0; bi < 2; bi++)
-            edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S || tok0 + (bi + 1) * BLK_TOK > Lcur;
+            edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S ||
+                       tok0 + (bi + 1) * BLK_TOK > Lcur - (a.qlen - 1);
 #pragma unroll
         for (int bi = 0; bi < 2; bi++) {
             float part_sc[2][C::HPL];
@@ -648,7 +650,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                     }
                     if (edge[bi]) {
                         const int pos = tok0 + bi * BLK_TOK + r + 8 * st;
-                        v = (bi < nmine && pos >= a.S && pos < Lcur) ? v : NEG_INF;
+                        const int lim = Lcur - (a.qlen - 1 - lane_head<G>(c, hh) % a.qlen);
+                        v = (bi < nmine && pos >= a.S && pos < lim) ? v : NEG_INF;
                     }
                     sco[bi][st][hh] = v;
                 }
@@ -720,9 +723,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int hh = 0; hh < C::HPL; hh++) {
                     const float v = sco[bi][st][hh];
-                    const float mm = pick<G>(m_run, lane_head<G>(c, hh));
-                    // every block holds a valid token, so mm is finite and
-                    // a masked score (-inf) gives exactly 0
+                    const float mr = pick<G>(m_run, lane_head<G>(c, hh));
+                    // a masked score (-inf) must give exactly 0: with several
+                    // queries per sequence a head can have seen no valid
+                    // position yet (mr = -inf), so subtract 0 then
+                    const float mm = mr == NEG_INF ? 0.f : mr;
                     const float p = fast_exp2(v - mm);
                     P[bi][st][hh] = p;
                     l_run[hh] += p;
@@ -898,8 +903,9 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     // start).  The sink partial, in fp32 on CUDA cores: q_rot, scores over the
     // fp16 sink rows, softmax, weighted sum.
     const int L = a.seq_lens[b];
-    const bool lok = (L >= 1 && L <= a.capacity);
-    const int ns = (a.S > 0 && lok) ? min(a.S, L) : 0;
+    const int Li = L - (a.qlen - 1 - hq % a.qlen);           // this query's context
+    const bool lok = (L >= 1 && L <= a.capacity && Li >= 1);
+    const int ns = (a.S > 0 && lok) ? min(a.S, Li) : 0;
     if (ns > 0) {
         const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
         if (a.mode == KVQ_ROT_DENSE) {
@@ -1009,6 +1015,7 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     pdl_trigger();
     if (!lok) {
         if (t < D) out[t] = 0;
+        if (t == 0 && L >= 1 && L <= a.capacity) set_status(a.status, KVQ_DEV_BAD_LEN);   // L < qlen
         return;
     }
     const int u = b * a.Hkv + h;
@@ -1083,7 +1090,10 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         o_s[t] = v / l;
     }
     __syncthreads();
-    if (a.mode == KVQ_ROT_DENSE) {
+    if (a.out_rotated) {
+        // the caller folds R_v^T into its own projection: o_rot as it is
+        if (t < D) out[t] = __half_as_ushort(__float2half_rn(o_s[t]));
+    } else if (a.mode == KVQ_ROT_DENSE) {
         // out[i] = sum_j o[j] R_v[h][i][j]: warp w rows 16w..16w+15, lanes over j
         const float4 o4 = *reinterpret_cast<const float4 *>(&o_s[4 * lane]);
         float mine = 0.f;
@@ -1136,7 +1146,8 @@ static cudaError_t launch_split(const DecodeArgs &a, cudaStream_t st) {
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
-                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end, int qlen,
+                          int out_rotated) {
     const WsLayout w = ws_layout(cd.B, Hq, cd.Hkv, C);
     uint8_t *base = static_cast<uint8_t *>(ws);
     DecodeArgs a;
@@ -1161,6 +1172,8 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.nblk = cd.capacity / BLK_TOK;
     a.mode = mode;
     a.C = C;
+    a.qlen = qlen;
+    a.out_rotated = out_rotated;
     cudaError_t e = launch_pdl(decode_qprep_kernel, dim3(cd.Hkv, cd.B), dim3(QP_THREADS), 0, st, a);
     if (e != cudaSuccess) return e;
     if (ev_begin && (e = cudaEventRecord(ev_begin, st)) != cudaSuccess) return e;

@@ -289,7 +289,8 @@ cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
-                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
+                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end, int qlen,
+                          int out_rotated);
 
 // Decode workspace: prepared queries and split partials.
 struct WsLayout {

@@ -68,6 +68,9 @@ def lib():
     L.kvq_decode_attention_timed.restype = C.c_int
     L.kvq_decode_attention_timed.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p, i32,
                                              i32, p, sz, p, p, p, p]
+    L.kvq_decode_attention_ex.restype = C.c_int
+    L.kvq_decode_attention_ex.argtypes = [p, i32, i32, C.c_uint32, C.POINTER(CacheDesc), C.c_int, p,
+                                          p, p, p, i32, i32, p, sz, p, p]
     L.kvq_decode_attention_noalloc.restype = C.c_int
     L.kvq_decode_attention_noalloc.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p,
                                                i32, i32, p, p]
@@ -188,6 +191,30 @@ def kvq_decode_attention(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, ma
                                       _ptr(perm), _ptr(seq_lens), sink_fp16, max_ctx,
                                       _ptr(workspace), workspace.numel(), _ptr(out),
                                       _stream(stream)))
+
+
+KVQ_DECODE_OUT_ROTATED = 1
+
+
+def kvq_decode_attention_ex(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
+                            workspace, out, flags=0, stream=None):
+    """Q fp16 [B][Hq][q_len][128] -> out fp16 [B][Hq][q_len][128]: q_len new tokens
+    per sequence, each attending causally; flags: KVQ_DECODE_OUT_ROTATED."""
+    B, Hq, q_len, d = Q.shape
+    _need(Q, torch.float16, "Q", (cache.B, Hq, q_len, D))
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    if mode == KVQ_ROT_DENSE:
+        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
+    else:
+        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
+    _check("kvq_decode_attention_ex",
+           lib().kvq_decode_attention_ex(_ptr(Q), Hq, q_len, flags, C.byref(cache.desc), mode,
+                                         _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
+                                         sink_fp16, max_ctx, _ptr(workspace), workspace.numel(),
+                                         _ptr(out), _stream(stream)))
 
 
 def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,

@@ -276,3 +276,106 @@ def test_decode_bad_lengths_give_zero_rows_and_status():
     assert kvq.kvq_get_status(cache) == kvq.KVQ_DEV_BAD_LEN
     ref, _ = orc.decode(oc, f16bits(Q), 0, rn[0], rn[1], rn[2], sl)
     assert rel_err(out[0:1], ref[0:1]).max() <= DEC_TOL
+
+
+# --- decode with several new tokens per sequence, and output in the rotated basis -----------------
+
+MQ_CASES = [
+    # G, q_len, mode, S, lengths
+    (1, 2, 0, 0, [2, 17, 300, 1000]),
+    (1, 4, 1, 0, [4, 33, 512]),
+    (1, 8, 0, 4, [8, 9, 700]),
+    (2, 2, 0, 4, [3, 40, 257]),
+    (4, 2, 1, 0, [2, 1500]),
+]
+
+
+@pytest.mark.parametrize("G,q_len,mode,S,lens", MQ_CASES)
+def test_multi_query_decode_matches_oracle(G, q_len, mode, S, lens):
+    """q_len new tokens per sequence: query i sees positions [0, L - q_len + i];
+    each is checked against the oracle's ordinary decode over that prefix."""
+    Hkv = 2
+    w = W.custom(seed=60 + 10 * G + q_len, B=len(lens), Hq=Hkv * G, Hkv=Hkv, mode=mode, sink=S,
+                 k_outliers=4, sink_key_scale=50.0 if S else 1.0)
+    cap = ((max(lens) + 15) // 16) * 16
+    oc = build_oracle_cache(w, lens, cap)
+    rt, rn = rot_tensors(w)
+    g = torch.Generator().manual_seed(900 + q_len)
+    Q = torch.randn((w.B, w.Hq, q_len, D), generator=g).to(torch.float16)
+    cache = upload_oracle_cache(oc)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = kvq.decode_workspace(w.B, w.Hq * q_len, Hkv, max(lens))
+    ws.fill_(0xFF)
+    out = torch.empty_like(Q).cuda()
+    kvq.kvq_decode_attention_ex(Q.cuda(), cache, mode, rt[0], rt[1], rt[2], sl, S, max(lens), ws,
+                                out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    got = out.cpu().numpy()
+    for i in range(q_len):
+        li = np.array(lens, np.int32) - (q_len - 1 - i)
+        ref, st = orc.decode(oc, f16bits(Q[:, :, i].contiguous()), mode, rn[0], rn[1], rn[2], li,
+                             n_threads=8)
+        assert st == 0
+        err = rel_err(got[:, :, i], ref)
+        assert err.max() <= DEC_TOL, (i, err.max())
+
+
+def test_multi_query_short_sequence_gives_zero_rows_and_status():
+    """A sequence shorter than q_len: the queries that would start before
+    position 0 get zero rows and KVQ_DEV_BAD_LEN; the others are normal."""
+    w = W.custom(seed=71, B=2, Hq=2, Hkv=2, mode=0, k_outliers=4)
+    lens = [2, 50]
+    q_len = 4
+    cap = 64
+    oc = build_oracle_cache(w, lens, cap)
+    rt, rn = rot_tensors(w)
+    Q = torch.randn((2, 2, q_len, D), generator=torch.Generator().manual_seed(5)).to(torch.float16)
+    cache = upload_oracle_cache(oc)
+    ws = kvq.decode_workspace(2, 2 * q_len, 2, 50)
+    out = torch.full_like(Q, float("nan")).cuda()
+    kvq.kvq_decode_attention_ex(Q.cuda(), cache, 0, rt[0], rt[1], None,
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), 0, 50, ws, out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) & kvq.KVQ_DEV_BAD_LEN
+    got = out.cpu().float().numpy()
+    assert (got[0, :, :2] == 0).all()                    # positions -2 and -1: no context
+    for i in range(2, q_len):                            # sequence 0, queries at positions 0, 1
+        ref, _ = orc.decode(oc, f16bits(Q[:, :, i].contiguous()), 0, rn[0], rn[1], None,
+                            np.array([i - 1, 50 - (q_len - 1 - i)], np.int32), n_threads=4)
+        assert rel_err(got[0, :, i], ref[0]).max() <= DEC_TOL
+    assert np.isfinite(got[1]).all()
+
+
+@pytest.mark.parametrize("mode,G,S", [(0, 1, 0), (1, 2, 4), (0, 4, 4)])
+def test_decode_out_rotated(mode, G, S):
+    """KVQ_DECODE_OUT_ROTATED returns o_rot: the oracle's output carried back
+    into the rotated basis (out . R_v, or perm + FWHT) must match."""
+    Hkv = 2
+    lens = [5, 300, 1025]
+    w = W.custom(seed=80 + G, B=len(lens), Hq=Hkv * G, Hkv=Hkv, mode=mode, sink=S, k_outliers=4)
+    cap = ((max(lens) + 15) // 16) * 16
+    oc = build_oracle_cache(w, lens, cap)
+    rt, rn = rot_tensors(w)
+    Q = W.queries(w, "cpu")
+    sl = np.array(lens, np.int32)
+    ref, st = orc.decode(oc, f16bits(Q), mode, rn[0], rn[1], rn[2], sl, n_threads=8)
+    assert st == 0
+    ref_rot = np.empty_like(ref)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            h = hq // G
+            if mode == 0:
+                ref_rot[b, hq] = orc.rotate_f64(ref[b, hq][None], 0, R=rn[1][h])[0]
+            else:
+                ref_rot[b, hq] = orc.rotate_f64(ref[b, hq][None], 1, perm=rn[2][1, h])[0]
+    cache = upload_oracle_cache(oc)
+    ws = kvq.decode_workspace(w.B, w.Hq, Hkv, max(lens))
+    out = torch.empty((w.B, w.Hq, 1, D), dtype=torch.float16, device="cuda")
+    kvq.kvq_decode_attention_ex(Q.cuda()[:, :, None].contiguous(), cache, mode, rt[0], rt[1], rt[2],
+                                torch.from_numpy(sl).cuda(), S, max(lens), ws, out,
+                                flags=kvq.KVQ_DECODE_OUT_ROTATED)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    err = rel_err(out[:, :, 0].cpu().numpy(), ref_rot)
+    assert err.max() <= DEC_TOL, err.max()
