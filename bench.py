@@ -343,6 +343,66 @@ def append_rates(device, peak, reps=5):
     return out
 
 
+def extension_rates(step, device, reps=50):
+    """Decode-only timings (L2 flushed before each call, events around it) of
+    the serving extensions on the workload's cache (layer 0): the plain
+    decode, the same cache paged through a random block table (one pool
+    block per 16 tokens x all heads), and q_len = 4 new tokens per sequence
+    (each attending causally)."""
+    import rotated_int2_kv_head_b200 as kvq
+    w = step.w
+    cache, Rk, Rv, perm = step.layers[0]
+    L = step.L
+    lens = step.len_base + step.T
+    nblk = step.cap // 16
+    flush = L2Flush(device)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def timed(fn):
+        ms = []
+        for k in range(reps + 3):
+            flush(k)
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize(device)
+            if k >= 3:
+                ms.append(ev[0].elapsed_time(ev[1]))
+        return float(np.median(ms))
+
+    out = torch.empty_like(step.Q)
+    plain = timed(lambda: kvq.kvq_decode_attention(step.Q, cache, w.mode, Rk, Rv, perm, lens, w.sink,
+                                                   L, step.ws, out))
+    num_blocks = w.B * nblk + 64
+    g = torch.Generator().manual_seed(11)
+    table = torch.randperm(num_blocks, generator=g)[:w.B * nblk].view(w.B, nblk).to(torch.int32)
+    table = table.to(device)
+    paged = kvq.PagedKVCache(w.B, w.Hkv, step.cap, num_blocks, table, w.sink, device=device)
+    paged.block_view()[table.long()] = cache.block_view().permute(0, 2, 1, 3)
+    if w.sink:
+        paged.k_sink.copy_(cache.k_sink)
+        paged.v_sink.copy_(cache.v_sink)
+    out_p = torch.empty_like(step.Q)
+    paged_ms = timed(lambda: kvq.kvq_decode_attention(step.Q, paged, w.mode, Rk, Rv, perm, lens,
+                                                      w.sink, L, step.ws, out_p))
+    same = bool(torch.equal(out, out_p))
+    res = {"how": "decode only, L2 flushed before each call, median of %d" % reps,
+           "plain_decode_ms": plain,
+           "paged_decode_ms": paged_ms, "paged_output_bit_identical": same}
+    q_len = 4
+    if (w.Hq // w.Hkv) * q_len <= 8:
+        Qm = torch.randn((w.B, w.Hq, q_len, 128), generator=torch.Generator().manual_seed(12)
+                         ).to(torch.float16).to(device)
+        wsm = kvq.decode_workspace(w.B, w.Hq * q_len, w.Hkv, L, device=device)
+        outm = torch.empty_like(Qm)
+        res["multi_query_q_len"] = q_len
+        res["multi_query_decode_ms"] = timed(lambda: kvq.kvq_decode_attention_ex(
+            Qm, cache, w.mode, Rk, Rv, perm, lens, w.sink, L, wsm, outm))
+    if max(kvq.kvq_get_status(cache), kvq.kvq_get_status(paged)) != 0:
+        raise RuntimeError("device status after the extension timings")
+    return res
+
+
 def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
     the first `heads` KV heads of sequence 0 (their K/V rows are the very
@@ -579,6 +639,8 @@ def run_cuda(args):
     }
     if world == 1 and not args.no_append:
         line["append"] = append_rates(dev, peak)
+    if world == 1 and not args.no_extensions:
+        line["extensions"] = extension_rates(step, dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, step, dev)
     print(json.dumps(line), flush=True)
@@ -655,6 +717,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama7b", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
+    ap.add_argument("--no-extensions", action="store_true",
+                    help="skip the paged / multi-query decode timings")
     ap.add_argument("--append-only", action="store_true",
                     help="only the bulk-append rates (one GPU), as one JSON line")
     args = ap.parse_args(argv)

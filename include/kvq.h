@@ -51,6 +51,10 @@
  * Cache layout.  One cache holds B sequences x Hkv KV heads; each (b, h)
  * "unit" owns capacity/16 blocks of 16 tokens, 1536 bytes each:
  *   blocks + ((b*Hkv + h) * (capacity/16) + p/16) * 1536   for position p.
+ * A paged cache (kvq_cache_desc.block_table set) keeps the same 1536-byte
+ * blocks in a pool of num_blocks x Hkv blocks and finds position p of
+ * sequence b through the table:
+ *   blocks + (block_table[b*(capacity/16) + p/16] * Hkv + h) * 1536.
  * Inside a block, with tau = p % 16, r = tau % 8, th = tau / 8,
  * pair q = tau / 2, side = tau % 2 (all offsets in bytes):
  *   K codes  [0,512)     logical 32-bit word wi (bytes 4wi..4wi+3 of the
@@ -101,6 +105,10 @@ typedef enum {
 #define KVQ_DEV_BAD_LEN 2     /* seq_lens[b] < 0 (append) or not in [1, capacity]
                                  (decode): skipped, decode output row is 0      */
 #define KVQ_DEV_TIMEOUT 4     /* a bounded pipeline wait gave up: output invalid */
+#define KVQ_DEV_BAD_TABLE 8   /* paged cache: a block-table entry outside
+                                 [0, num_blocks): the append skips that store,
+                                 the decode reads pool block 0 instead (output
+                                 invalid)                                       */
 
 typedef struct {
     int32_t B;                /* sequences                                      */
@@ -109,7 +117,8 @@ typedef struct {
     int32_t group;            /* must be 32                                     */
     int32_t capacity;         /* tokens per sequence, multiple of 16            */
     int32_t sink_fp16;        /* leading positions kept in fp16 (0..64)         */
-    void *blocks;             /* [B][Hkv][capacity/16][1536] bytes, 16-B aligned */
+    void *blocks;             /* [B][Hkv][capacity/16][1536] bytes (paged:
+                                 [num_blocks][Hkv][1536]), 16-B aligned          */
     uint16_t *k_sink;         /* [B][Hkv][sink_fp16][128] fp16, or NULL if 0     */
     uint16_t *v_sink;         /* same                                           */
     int32_t *status;          /* two device words, 8-B aligned: [0] sticky error
@@ -117,6 +126,17 @@ typedef struct {
                                  completion counter.  Zero both once before
                                  first use; [1] is zero again after every
                                  append.                                        */
+    const int32_t *block_table; /* NULL: the contiguous layout above.  Otherwise
+                                 a paged cache: int32 [B][capacity/16] device
+                                 array, 4-B aligned; logical block lb of
+                                 sequence b (positions 16lb..16lb+15) lives in
+                                 pool block n = block_table[b*(capacity/16) + lb],
+                                 whose KV head h is the 1536-byte block at
+                                 blocks + (n*Hkv + h)*1536.  Entries of blocks a
+                                 call touches must be in [0, num_blocks);
+                                 several sequences may not share a block.      */
+    int32_t num_blocks;       /* paged: pool blocks (blocks holds
+                                 num_blocks*Hkv*1536 bytes); ignored otherwise */
 } kvq_cache_desc;
 
 /* Bytes of the blocks array for a cache of this shape (0 on bad arguments). */

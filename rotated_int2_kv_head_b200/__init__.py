@@ -6,7 +6,8 @@ the CUDA sources (csrc/), the in-tree build (build.py) and a thin ctypes
 binding (kvq.py) with the same function names as the C ABI.
 """
 from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ_DEV_TIMEOUT,
-                  KVQ_ROT_DENSE, KVQ_ROT_PERM_FWHT, KVCache, KvqError, decode_workspace,
+                  KVQ_DEV_BAD_TABLE, KVQ_ROT_DENSE, KVQ_ROT_PERM_FWHT, KVCache, KvqError, PagedKVCache,
+                  decode_workspace,
                   kvq_cache_bytes, kvq_clear_status, kvq_debug_quantize_f32, kvq_debug_rotate_f32,
                   kvq_decode_attention, kvq_decode_attention_ex, kvq_decode_attention_noalloc,
                   kvq_decode_attention_timed,
@@ -14,7 +15,7 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_rotate_quantize_append, lib)
 
 __all__ = [
-    "KVCache", "KvqError", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
+    "KVCache", "PagedKVCache", "KvqError", "KVQ_DEV_BAD_TABLE", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
     "KVQ_DEV_CAPACITY",
     "KVQ_DEV_BAD_LEN", "KVQ_DEV_TIMEOUT", "decode_workspace", "kvq_cache_bytes",
     "kvq_clear_status", "kvq_debug_quantize_f32", "kvq_debug_rotate_f32",

@@ -41,6 +41,10 @@ kvq_status check_cache(const kvq_cache_desc *c) {
     }
     if ((long long)c->B * c->Hkv * (c->capacity / BLK_TOK) > INT_MAX) return KVQ_ERR_INVALID_ARG;
     if (c->B > 32767) return KVQ_ERR_INVALID_ARG;
+    if (c->block_table) {
+        if (!aligned(c->block_table, 4)) return KVQ_ERR_UNSUPPORTED;
+        if (c->num_blocks < 1 || (long long)c->num_blocks * c->Hkv > INT_MAX) return KVQ_ERR_INVALID_ARG;
+    }
     return KVQ_OK;
 }
 

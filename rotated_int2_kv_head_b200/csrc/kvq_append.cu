@@ -27,7 +27,9 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
                                                int L0, const float v[4]) {
     const int lane = threadIdx.x & 31;
     const int p = L0 + t;
-    uint8_t *block = c.blocks + ((size_t)(b * c.Hkv + h) * c.nblk + p / BLK_TOK) * BLK_BYTES;
+    const long long bi = cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, p / BLK_TOK);
+    if (bi < 0 && lane == 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+    uint8_t *block = c.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
     const int tau = p % BLK_TOK;
     if (p < c.S) {
         uint16_t *sink = (kind == 0 ? c.k_sink : c.v_sink) +
@@ -36,10 +38,10 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
         pk.x = pack_half2(v[0], v[1]);
         pk.y = pack_half2(v[2], v[3]);
         *reinterpret_cast<uint2 *>(sink) = pk;
-        zero_token_warp(block, tau, kind);
+        if (bi >= 0) zero_token_warp(block, tau, kind);
     } else {
-        const QuantWord q = quantize_row_warp(v);
-        store_token_warp(block, tau, kind, q);
+        const QuantWord q = quantize_row_warp(v);      // warp-collective: every lane runs it
+        if (bi >= 0) store_token_warp(block, tau, kind, q);
     }
 }
 
@@ -250,6 +252,8 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
                                 cudaStream_t st) {
     CacheDst c;
     c.blocks = static_cast<uint8_t *>(cd.blocks);
+    c.table = cd.block_table;
+    c.num_blocks = cd.num_blocks;
     c.k_sink = cd.k_sink;
     c.v_sink = cd.v_sink;
     c.seq_lens = seq_lens;

@@ -439,9 +439,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     meta[g] = quantize_group_thread(v, g, words);
                 }
             }
-            if (TO_CACHE && valid) {
+            const long long bix =
+                TO_CACHE && valid
+                    ? cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, p / BLK_TOK)
+                    : 0;
+            if (bix < 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+            if (TO_CACHE && valid && bix >= 0) {
                 // sink rows leave zero codes and metadata in their cache slots
-                uint8_t *block = c.blocks + ((size_t)(b * c.Hkv + h) * c.nblk + p / BLK_TOK) * BLK_BYTES;
+                uint8_t *block = c.blocks + (size_t)bix * BLK_BYTES;
                 const int tau = p % BLK_TOK;
                 if (kind == 0) {
 #pragma unroll
@@ -536,6 +541,8 @@ cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const 
     if (!make_map(&mk, K, cd.Hkv, rows) || !make_map(&mv, V, cd.Hkv, rows)) return cudaErrorInvalidValue;
     CacheDst c;
     c.blocks = static_cast<uint8_t *>(cd.blocks);
+    c.table = cd.block_table;
+    c.num_blocks = cd.num_blocks;
     c.k_sink = cd.k_sink;
     c.v_sink = cd.v_sink;
     c.seq_lens = seq_lens;

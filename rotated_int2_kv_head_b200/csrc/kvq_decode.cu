@@ -61,6 +61,8 @@ constexpr float LOG2E = 1.4426950408889634f;
 struct DecodeArgs {
     const uint16_t *Q;
     const uint8_t *blocks;
+    const int32_t *table;   // paged cache: [B][nblk] pool block per logical block, else null
+    int num_blocks;         // paged: pool blocks
     const uint16_t *k_sink, *v_sink;
     const float *R_k, *R_v;
     const int32_t *perm;
@@ -384,7 +386,7 @@ __host__ __device__ inline size_t part_slot(int cta, int unit, int grp) {
     return (size_t)DEC_GROUPS * ((size_t)cta + unit) + grp;
 }
 
-template <int G>
+template <int G, bool PAGED>
 __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs a) {
     using C = Cfg<G>;
     constexpr int NS = nstage_for(G);
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     // kernel waited on it before letting this kernel launch), so seq_lens and
     // the cache are read - and the first copies issued - before waiting on
     // the prepared queries.
-    Sched sc;   // this group's part of the CTA's range (leader's copy is the producer state)
+    Sched sc;   // this group's part of the CTA's range (warp 0's copy is the producer state)
     if (!sched_init_cta(sc, a, scratch)) {
         pdl_wait();
         pdl_trigger();
@@ -424,31 +426,51 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     }
     const int fb = a.S / BLK_TOK;
 
-    // Copies.  The group leader fills ring slot `slot` with the next stage of
-    // the group's range and writes its descriptor {unit, b, h, first cache
-    // block}, {n}; unit -1 marks the end (the slot's phase is completed by a
-    // plain arrive).  Descriptors are written NS-1 group barriers before
-    // anyone reads them, so they are read without waiting on the copy.
-    int issued = 0;      // leader: stages issued (= the iteration they belong to)
-    bool ended = false;  // leader: the end marker is written
+    // Copies.  Ring slot `slot` is filled with the next stage of the group's
+    // range, with its descriptor {unit, b, h, first cache block}, {n}; unit -1
+    // marks the end (the slot's phase is completed by a plain arrive).
+    // Descriptors are written NS-1 group barriers before anyone reads them,
+    // so they are read without waiting on the copy.
+    // Producer: the group leader for a contiguous cache (a stage is one bulk
+    // copy); the group's whole first warp for a paged one, all lanes in step
+    // (the schedule state sc evolves identically in every lane), lane j
+    // copying block j of the stage so that the table entries load in
+    // parallel.  Lane 0 writes the descriptor and the expected byte count.
+    int issued = 0;      // stages issued (= the iteration they belong to)
+    bool ended = false;  // the end marker is written
     auto issue_next = [&](int slot) {
         if (ended) return;
         int unit = 0, b = 0, h = 0, kblk = 0, n = 0;
         if (sched_take(sc, a, unit, b, h, kblk, n)) {
-            desc[2 * slot] = make_int4(unit, b, h, fb + kblk);
-            desc[2 * slot + 1] = make_int4(n, 0, 0, 0);
-            mbar_arrive_expect_tx(&full[slot], n * BLK_BYTES);
-            bulk_g2s(ring + slot * STAGE_BYTES,
-                     a.blocks + ((size_t)unit * a.nblk + fb + kblk) * (size_t)BLK_BYTES,
-                     n * BLK_BYTES, &full[slot]);
+            if (lane == 0) {
+                desc[2 * slot] = make_int4(unit, b, h, fb + kblk);
+                desc[2 * slot + 1] = make_int4(n, 0, 0, 0);
+                mbar_arrive_expect_tx(&full[slot], n * BLK_BYTES);
+            }
+            if (!PAGED) {          // contiguous: the stage's blocks are adjacent
+                if (lane == 0)
+                    bulk_g2s(ring + slot * STAGE_BYTES,
+                             a.blocks + ((size_t)unit * a.nblk + fb + kblk) * (size_t)BLK_BYTES,
+                             n * BLK_BYTES, &full[slot]);
+            } else if (lane < n) { // paged: block `lane` of the stage
+                const int ph = a.table[(size_t)b * a.nblk + fb + kblk + lane];
+                const bool okb = ph >= 0 && ph < a.num_blocks;
+                if (!okb) set_status(a.status, KVQ_DEV_BAD_TABLE);
+                const size_t bi = okb ? (size_t)ph * a.Hkv + h : 0;   // bad entry: block 0
+                bulk_g2s(ring + slot * STAGE_BYTES + lane * BLK_BYTES, a.blocks + bi * BLK_BYTES,
+                         BLK_BYTES, &full[slot]);
+            }
         } else {
-            desc[2 * slot] = make_int4(-1, 0, 0, 0);
-            mbar_arrive(&full[slot]);
+            if (lane == 0) {
+                desc[2 * slot] = make_int4(-1, 0, 0, 0);
+                mbar_arrive(&full[slot]);
+            }
             ended = true;
         }
         ++issued;
     };
-    if (leader)
+    const bool producer = PAGED ? warp == 0 : leader;   // contiguous: lane 0 alone suffices
+    if (producer)
         for (int k = 0; k < NS; k++) issue_next(k);
     bar_group();
     pdl_wait();
@@ -818,7 +840,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         }
     };
     // Release ring slot `slot` once the whole group is done with it; the
-    // leader refills it.  Returns true (uniformly over the group) when a wait
+    // group's first warp refills it.  Returns true (uniformly over the group) when a wait
     // failed anywhere in the group: the group then stops.
     auto release = [&](int slot, bool ok) -> bool {
         int any_bad;
@@ -829,7 +851,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             : "r"((unsigned)!ok), "r"(1 + grp), "n"(GROUP_THREADS)
             : "memory");
         if (any_bad) return true;
-        if (leader) {
+        if (producer) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             issue_next(slot);
         }
@@ -1134,13 +1156,18 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
     return w;
 }
 
-template <int G>
-static cudaError_t launch_split(const DecodeArgs &a, cudaStream_t st) {
+template <int G, bool PAGED>
+static cudaError_t launch_split_t(const DecodeArgs &a, cudaStream_t st) {
     const size_t smem = split_smem_bytes(G);
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G>,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G, PAGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_split_kernel<G>, dim3(a.C), dim3(DEC_THREADS), smem, st, a);
+    return launch_pdl(decode_split_kernel<G, PAGED>, dim3(a.C), dim3(DEC_THREADS), smem, st, a);
+}
+
+template <int G>
+static cudaError_t launch_split(const DecodeArgs &a, cudaStream_t st) {
+    return a.table ? launch_split_t<G, true>(a, st) : launch_split_t<G, false>(a, st);
 }
 
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
@@ -1153,6 +1180,8 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     DecodeArgs a;
     a.Q = Q;
     a.blocks = static_cast<const uint8_t *>(cd.blocks);
+    a.table = cd.block_table;
+    a.num_blocks = cd.num_blocks;
     a.k_sink = cd.k_sink;
     a.v_sink = cd.v_sink;
     a.R_k = R_k;

@@ -307,7 +307,19 @@ struct CacheDst {
     int32_t *seq_lens;
     int32_t *status;          // [0] error bits, [1] CTA completion counter
     int B, T, Hkv, capacity, S, nblk;
+    const int32_t *table;     // paged cache: [B][nblk] pool block per logical block, else null
+    int num_blocks;           // paged: pool blocks
 };
+
+// Index (in 1536-byte blocks from `blocks`) of KV head h of logical block lb
+// of sequence b; -1 for a paged entry outside the pool.
+__device__ __forceinline__ long long cache_block_index(const int32_t *table, int num_blocks, int nblk,
+                                                       int Hkv, int b, int h, int lb) {
+    if (!table) return ((long long)b * Hkv + h) * nblk + lb;
+    const int n = table[(size_t)b * nblk + lb];
+    if (n < 0 || n >= num_blocks) return -1;
+    return (long long)n * Hkv + h;
+}
 
 // Called by every CTA of an append kernel after its last read of seq_lens
 // and its last write: the CTA that completes last bumps the lengths and

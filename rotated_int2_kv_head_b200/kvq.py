@@ -25,6 +25,7 @@ KVQ_ROT_PERM_FWHT = 1
 KVQ_DEV_CAPACITY = 1
 KVQ_DEV_BAD_LEN = 2
 KVQ_DEV_TIMEOUT = 4
+KVQ_DEV_BAD_TABLE = 8
 
 _STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CUDA",
            4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_WORKSPACE"}
@@ -40,7 +41,7 @@ class CacheDesc(C.Structure):
     _fields_ = [("B", C.c_int32), ("Hkv", C.c_int32), ("head_dim", C.c_int32),
                 ("group", C.c_int32), ("capacity", C.c_int32), ("sink_fp16", C.c_int32),
                 ("blocks", C.c_void_p), ("k_sink", C.c_void_p), ("v_sink", C.c_void_p),
-                ("status", C.c_void_p)]
+                ("status", C.c_void_p), ("block_table", C.c_void_p), ("num_blocks", C.c_int32)]
 
 
 _lib = None
@@ -137,6 +138,40 @@ class KVCache:
     def block_view(self):
         """blocks as uint8 [B][Hkv][capacity/16][1536]."""
         return self.blocks.view(self.B, self.Hkv, self.capacity // BLOCK_TOKENS, BLOCK_BYTES)
+
+
+class PagedKVCache(KVCache):
+    """A paged cache: a pool of num_blocks blocks (each 16 tokens x Hkv heads x
+    1536 bytes) and an int32 block table [B][capacity/16] mapping every
+    sequence's logical blocks to pool blocks (memory owned by torch)."""
+
+    def __init__(self, B, Hkv, capacity, num_blocks, block_table, sink_fp16=0, device="cuda"):
+        if capacity % BLOCK_TOKENS or num_blocks < 1:
+            raise ValueError("bad paged cache shape")
+        _need(block_table, torch.int32, "block_table", (B, capacity // BLOCK_TOKENS))
+        self.B, self.Hkv, self.capacity, self.sink_fp16 = B, Hkv, capacity, sink_fp16
+        self.num_blocks, self.block_table = num_blocks, block_table
+        self.blocks = torch.zeros(num_blocks * Hkv * BLOCK_BYTES, dtype=torch.uint8, device=device)
+        if sink_fp16 > 0:
+            self.k_sink = torch.zeros((B, Hkv, sink_fp16, D), dtype=torch.float16, device=device)
+            self.v_sink = torch.zeros_like(self.k_sink)
+        else:
+            self.k_sink = self.v_sink = None
+        self.status = torch.zeros(2, dtype=torch.int32, device=device)
+        self.desc = CacheDesc(B, Hkv, D, GROUP, capacity, sink_fp16, self.blocks.data_ptr(),
+                              0 if self.k_sink is None else self.k_sink.data_ptr(),
+                              0 if self.v_sink is None else self.v_sink.data_ptr(),
+                              self.status.data_ptr(), block_table.data_ptr(), num_blocks)
+
+    def block_view(self):
+        """The pool as uint8 [num_blocks][Hkv][1536]."""
+        return self.blocks.view(self.num_blocks, self.Hkv, BLOCK_BYTES)
+
+    def logical_view(self):
+        """The blocks gathered into the contiguous layout [B][Hkv][capacity/16][1536]
+        (a copy; entries outside the pool must not occur)."""
+        t = self.block_table.long()
+        return self.block_view()[t].permute(0, 2, 1, 3).contiguous()
 
 
 def kvq_cache_bytes(B, Hkv, capacity):

@@ -379,3 +379,66 @@ def test_decode_out_rotated(mode, G, S):
     assert kvq.kvq_get_status(cache) == 0
     err = rel_err(out[:, :, 0].cpu().numpy(), ref_rot)
     assert err.max() <= DEC_TOL, err.max()
+
+
+# --- paged caches ------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode,S", [(0, 0), (0, 20), (1, 4)])
+def test_paged_cache_matches_contiguous(mode, S):
+    """The same appends into a contiguous cache and into a paged one (a random
+    block table over a larger pool) give byte-identical blocks once the pool is
+    gathered through the table, and bit-identical decodes.  The appends cover
+    the small-batch kernel (T=37), the bulk kernel (T=300) and single tokens."""
+    B, Hkv, cap = 3, 2, 1024
+    nblk = cap // 16
+    w = W.custom(seed=90 + mode + S, B=B, Hq=2 * Hkv, Hkv=Hkv, mode=mode, sink=S, k_outliers=4)
+    rt, _ = rot_tensors(w)
+    num_blocks = B * nblk + 7
+    perm = torch.randperm(num_blocks, generator=torch.Generator().manual_seed(3))[:B * nblk]
+    table = perm.view(B, nblk).to(torch.int32).cuda()
+    flat = kvq.KVCache(B, Hkv, cap, S)
+    paged = kvq.PagedKVCache(B, Hkv, cap, num_blocks, table, S)
+    L0 = [0, 5, 16]
+    sl_f = torch.tensor(L0, dtype=torch.int32, device="cuda")
+    sl_p = sl_f.clone()
+    pos = list(L0)
+    for T in (37, 300, 1, 1):
+        K = torch.stack([W.kv_rows(w, b, pos[b], pos[b] + T, "cpu")[0] for b in range(B)]).cuda()
+        V = torch.stack([W.kv_rows(w, b, pos[b], pos[b] + T, "cpu")[1] for b in range(B)]).cuda()
+        gpu_append(flat, K, V, w, rt, sl_f)
+        gpu_append(paged, K, V, w, rt, sl_p)
+        pos = [p + T for p in pos]
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(flat) == 0 and kvq.kvq_get_status(paged) == 0
+    assert torch.equal(sl_f, sl_p)
+    assert torch.equal(paged.logical_view(), flat.block_view())
+    if S:
+        assert torch.equal(paged.k_sink, flat.k_sink) and torch.equal(paged.v_sink, flat.v_sink)
+    Q = W.queries(w, "cuda")
+    out_f = gpu_decode(flat, Q, w, rt, sl_f, max(pos))
+    out_p = gpu_decode(paged, Q, w, rt, sl_p, max(pos))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(paged) == 0
+    assert torch.equal(out_f, out_p)
+
+
+def test_paged_bad_table_entry_sets_status():
+    """A table entry outside the pool: the append skips that block and the
+    decode reads pool block 0 instead; both report KVQ_DEV_BAD_TABLE."""
+    B, Hkv, cap = 2, 2, 64
+    w = W.custom(seed=97, B=B, Hq=Hkv, Hkv=Hkv, mode=0, k_outliers=4)
+    rt, _ = rot_tensors(w)
+    num_blocks = 8
+    table = torch.arange(8, dtype=torch.int32).view(2, 4)
+    table[1, 1] = 99                                    # logical block 1 of sequence 1
+    paged = kvq.PagedKVCache(B, Hkv, cap, num_blocks, table.cuda())
+    K, V = W.kv_batch(w, 0, 40, "cuda")
+    sl = torch.zeros(B, dtype=torch.int32, device="cuda")
+    gpu_append(paged, K, V, w, rt, sl)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(paged) & kvq.KVQ_DEV_BAD_TABLE
+    kvq.kvq_clear_status(paged)
+    out = gpu_decode(paged, W.queries(w, "cuda"), w, rt, sl, 40)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(paged) & kvq.KVQ_DEV_BAD_TABLE
+    assert torch.isfinite(out[0]).all()
