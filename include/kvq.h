@@ -67,8 +67,18 @@
  * fragments, so one warp reads each 512-byte region as 32 x 16 contiguous
  * bytes.  The 96 bytes per token-head (3 bits per element) are the whole
  * cache read of a decode step.
- * Sinks: positions p < sink_fp16 are kept as fp16 rotated rows in
- *   k_sink / v_sink [B][Hkv][sink_fp16][128]; their block slots are zeroed.
+ * Sinks (RotateKV abstract, item (iii): attention sinks are protected from
+ *   2-bit quantization) are kept as fp16 rotated rows in
+ *   k_sink / v_sink [B][Hkv][sink_fp16][128], in one of two ways:
+ *   - leading sinks (sink_pos == NULL): positions p < sink_fp16 of every
+ *     sequence, row p; their block slots are zeroed;
+ *   - identified sinks (sink_pos != NULL): the positions that
+ *     kvq_identify_sinks picked because their activations are massive
+ *     (same item: massive activations single out the sinks), listed in
+ *     ascending order in sink_pos[b][0 .. sink_count[b]); the one at list
+ *     index j is row j.  Its block slot holds zero codes, V meta
+ *     {0, 0} and K meta {s, z} = {0x7E00 (a quiet NaN), 0} in every group:
+ *     the marker that keeps the INT2 path from scoring the position.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -137,6 +147,14 @@ typedef struct {
                                  several sequences may not share a block.      */
     int32_t num_blocks;       /* paged: pool blocks (blocks holds
                                  num_blocks*Hkv*1536 bytes); ignored otherwise */
+    int32_t *sink_pos;        /* NULL: leading sinks.  Otherwise identified
+                                 sinks: int32 [B][sink_fp16], ascending
+                                 positions (sink_fp16 >= 1); written by
+                                 kvq_identify_sinks, read by the append and the
+                                 decode.  4-B aligned.                         */
+    int32_t *sink_count;      /* identified sinks: int32 [B], entries of
+                                 sink_pos in use (0..sink_fp16); zero it with
+                                 the cache.  Ignored when sink_pos is NULL.    */
 } kvq_cache_desc;
 
 /* Bytes of the blocks array for a cache of this shape (0 on bad arguments). */
@@ -160,6 +178,30 @@ KVQ_API kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t 
                                       kvq_rot_mode mode, const float *R_k, const float *R_v,
                                       const int32_t *perm, const kvq_cache_desc *cache,
                                       int32_t *seq_lens, void *stream);
+
+/*
+ * Pick the attention sinks among the next T positions of every sequence by
+ * their activation magnitude (RotateKV abstract, item (iii)); call it just
+ * before the kvq_rotate_quantize_append of the same T tokens, with the same
+ * seq_lens (it does not change them).
+ *   act       fp32 [B][T]: the caller's activation magnitude of each new token
+ *             (for instance the largest |hidden-state| entry of the token at
+ *             this layer's input; the library only compares it).
+ *   tau       threshold: token t of sequence b is a sink when
+ *             act[b*T + t] >= tau (NaN compares false) and the sequence has a
+ *             free sink row; rows are taken in position order, so the first
+ *             sink_fp16 such positions of a sequence are kept.
+ *   cache     needs sink_pos / sink_count (identified sinks).
+ *   seq_lens  int32 [B] device, the lengths before the append.  A sequence
+ *             the append would skip (seq_lens[b] < 0 or seq_lens[b] + T >
+ *             capacity) is skipped here too.
+ * Appends the picked positions to sink_pos[b] and raises sink_count[b].
+ * Errors: KVQ_ERR_INVALID_ARG for null pointers, T < 1, or a cache without
+ * sink_pos; nothing is launched then.
+ */
+KVQ_API kvq_status kvq_identify_sinks(const float *act, int32_t T, float tau,
+                                      const kvq_cache_desc *cache, const int32_t *seq_lens,
+                                      void *stream);
 
 /* Workspace bytes needed by kvq_decode_attention for these sizes on a GPU
  * with sm_count SMs (0 on bad arguments). */

@@ -302,20 +302,59 @@ void orc_load_token(const uint8_t *block, int tau, uint8_t *kbytes, uint8_t *vby
 }
 
 /* ------------------------------------------------------------------------ */
+/* Attention sinks (RotateKV abstract, item (iii)).                           */
+/* ------------------------------------------------------------------------ */
+
+/* Identified sinks: the sinks are the tokens whose activations are massive.
+ * act: fp32 [B][T], the activation magnitude of each of the T tokens about to
+ * be appended.  Position seq_lens[b] + t becomes a sink when
+ * act[b][t] >= tau while sequence b still has a free fp16 row (S rows per
+ * sequence); rows are handed out in position order and recorded in
+ * sink_pos[b][row], sink_count[b] = rows in use.  A sequence that the
+ * append will skip (negative length, or no room for T more tokens) is
+ * skipped here too. */
+void orc_identify_sinks(const float *act, int B, int T, float tau, int S, int capacity,
+                        const int32_t *seq_lens, int32_t *sink_pos, int32_t *sink_count) {
+    for (int b = 0; b < B; b++) {
+        int L0 = seq_lens[b];
+        if (L0 < 0 || (int64_t)L0 + T > capacity) continue;
+        for (int t = 0; t < T; t++) {
+            if (act[(size_t)b * T + t] >= tau && sink_count[b] < S) {
+                sink_pos[(size_t)b * S + sink_count[b]] = L0 + t;
+                sink_count[b] += 1;
+            }
+        }
+    }
+}
+
+/* The fp16 row that holds position p of sequence b, or -1 if p is stored
+ * in INT2.  sink_pos == NULL: leading sinks, positions 0..S-1 are rows
+ * 0..S-1.  Otherwise the identified sinks of sequence b. */
+static int sink_row(int S, const int32_t *sink_pos, const int32_t *sink_count, int b, int p) {
+    if (sink_pos == NULL) return p < S ? p : -1;
+    for (int j = 0; j < sink_count[b] && j < S; j++)
+        if (sink_pos[(size_t)b * S + j] == p) return j;
+    return -1;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Rotate -> quantize -> append.                                              */
 /* ------------------------------------------------------------------------ */
 
 /* K, V: fp16 [B][T][Hkv][128].  R_k, R_v: fp32 [Hkv][128][128] (dense mode).
  * perm: int32 [2][Hkv][128] (FWHT mode; plane 0 keys, plane 1 values).
  * blocks: [B][Hkv][capacity/16][1536].  k_sink, v_sink: fp16 [B][Hkv][S][128].
- * seq_lens[b] (in: old length, out: old + T).  Position p = seq_lens[b] + t
- * with p < S is an attention sink (RotateKV item (iii)): stored as the fp16
- * rounding of its rotated fp32 row; its code and meta slots are zeroed.
+ * seq_lens[b] (in: old length, out: old + T).  A position that is an
+ * attention sink (RotateKV item (iii); sink_row above) is stored as the fp16
+ * rounding of its rotated fp32 row in its sink row.  Its code slots are
+ * zeroed; its meta slots too for leading sinks, while an identified sink's
+ * K meta is the marker {s, z} = {0x7E00, 0} in every group (V meta zero).
  * A sequence whose new length would exceed capacity is skipped whole and
  * flags ST_CAPACITY.  Returns the status bits. */
 int orc_append(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int mode,
                const float *R_k, const float *R_v, const int32_t *perm, int capacity, int S,
-               uint8_t *blocks, uint16_t *k_sink, uint16_t *v_sink, int32_t *seq_lens) {
+               uint8_t *blocks, uint16_t *k_sink, uint16_t *v_sink, int32_t *seq_lens,
+               const int32_t *sink_pos, const int32_t *sink_count) {
     int status = 0;
     const int nblk = capacity / BLK_TOK;
     for (int b = 0; b < B; b++) {
@@ -336,9 +375,10 @@ int orc_append(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int 
                 uint8_t *block = blocks + (((size_t)b * Hkv + h) * nblk + p / BLK_TOK) * BLK_BYTES;
                 uint8_t kc[D], vc[D], kb[32], vb[32];
                 uint16_t ks[NG], kz[NG], vs[NG], vz[NG];
-                if (p < S) {
-                    uint16_t *ksr = k_sink + (((size_t)b * Hkv + h) * S + p) * D;
-                    uint16_t *vsr = v_sink + (((size_t)b * Hkv + h) * S + p) * D;
+                const int row = sink_row(S, sink_pos, sink_count, b, p);
+                if (row >= 0) {
+                    uint16_t *ksr = k_sink + (((size_t)b * Hkv + h) * S + row) * D;
+                    uint16_t *vsr = v_sink + (((size_t)b * Hkv + h) * S + row) * D;
                     for (int i = 0; i < D; i++) {
                         ksr[i] = orc_f32_to_f16(kr[i]);
                         vsr[i] = orc_f32_to_f16(vr[i]);
@@ -349,6 +389,8 @@ int orc_append(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int 
                     memset(kz, 0, sizeof kz);
                     memset(vs, 0, sizeof vs);
                     memset(vz, 0, sizeof vz);
+                    if (sink_pos != NULL)
+                        for (int g = 0; g < NG; g++) ks[g] = 0x7E00;
                 } else {
                     orc_quantize_row(kr, kc, ks, kz);
                     orc_quantize_row(vr, vc, vs, vz);
@@ -367,13 +409,14 @@ int orc_append(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int 
 /* Decode attention over the packed cache (fp64).                            */
 /* ------------------------------------------------------------------------ */
 
-/* Dequantise token t of unit (b, h) into fp64 rotated K and V rows. */
+/* Dequantise token t of unit (b, h) into fp64 rotated K and V rows; row is
+ * its fp16 sink row (sink_row), or -1 for an INT2 token. */
 static void dequant_token(const uint8_t *unit_blocks, const uint16_t *ksink_u,
-                          const uint16_t *vsink_u, int S, int t, double *k, double *v) {
-    if (t < S) {
+                          const uint16_t *vsink_u, int row, int t, double *k, double *v) {
+    if (row >= 0) {
         for (int i = 0; i < D; i++) {
-            k[i] = (double)orc_f16_to_f32(ksink_u[(size_t)t * D + i]);
-            v[i] = (double)orc_f16_to_f32(vsink_u[(size_t)t * D + i]);
+            k[i] = (double)orc_f16_to_f32(ksink_u[(size_t)row * D + i]);
+            v[i] = (double)orc_f16_to_f32(vsink_u[(size_t)row * D + i]);
         }
         return;
     }
@@ -395,7 +438,8 @@ static void dequant_token(const uint8_t *unit_blocks, const uint16_t *ksink_u,
  * Query head h uses KV head h / G (contiguous GQA grouping). */
 static void decode_one(const uint16_t *q, int mode, const float *Rk, const float *Rv,
                        const int32_t *pk, const int32_t *pv, const uint8_t *unit_blocks,
-                       const uint16_t *ksink_u, const uint16_t *vsink_u, int S, int L,
+                       const uint16_t *ksink_u, const uint16_t *vsink_u, int S,
+                       const int32_t *sink_pos, const int32_t *sink_count, int b, int L,
                        double *out) {
     double qin[D], qr[D], k[D], v[D], o[D];
     for (int i = 0; i < D; i++) qin[i] = (double)orc_f16_to_f32(q[i]);
@@ -404,7 +448,7 @@ static void decode_one(const uint16_t *q, int mode, const float *Rk, const float
     const double scale = 1.0 / sqrt((double)D);
     double m = -INFINITY;
     for (int t = 0; t < L; t++) {
-        dequant_token(unit_blocks, ksink_u, vsink_u, S, t, k, v);
+        dequant_token(unit_blocks, ksink_u, vsink_u, sink_row(S, sink_pos, sink_count, b, t), t, k, v);
         double acc = 0.0;
         for (int i = 0; i < D; i++) acc += qr[i] * k[i];
         s[t] = acc * scale;
@@ -415,7 +459,7 @@ static void decode_one(const uint16_t *q, int mode, const float *Rk, const float
     for (int t = 0; t < L; t++) {
         double p = exp(s[t] - m);
         l += p;
-        dequant_token(unit_blocks, ksink_u, vsink_u, S, t, k, v);
+        dequant_token(unit_blocks, ksink_u, vsink_u, sink_row(S, sink_pos, sink_count, b, t), t, k, v);
         for (int i = 0; i < D; i++) o[i] += p * v[i];
     }
     for (int i = 0; i < D; i++) o[i] /= l;
@@ -423,7 +467,9 @@ static void decode_one(const uint16_t *q, int mode, const float *Rk, const float
     free(s);
 }
 
-/* Q: fp16 [B][Hq][128].  out: fp64 [B][Hq][128].  Units with an invalid
+/* Q: fp16 [B][Hq][128].  out: fp64 [B][Hq][128].  sink_pos / sink_count:
+ * identified sinks of each sequence, or NULL for leading sinks (the
+ * position-to-row map is sink_row's).  Units with an invalid
  * length (L < 1 or L > capacity) get out = 0 and flag ST_BAD_LEN.
  * only_b / only_h >= 0 restrict the work to one sequence / KV head (used to
  * sample large workloads); other outputs are left untouched.
@@ -431,7 +477,8 @@ static void decode_one(const uint16_t *q, int mode, const float *Rk, const float
 int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
                const float *R_v, const int32_t *perm, int capacity, int S,
                const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
-               const int32_t *seq_lens, int only_b, int only_h, int n_threads, double *out) {
+               const int32_t *seq_lens, const int32_t *sink_pos, const int32_t *sink_count,
+               int only_b, int only_h, int n_threads, double *out) {
     int status = 0;
     const int G = Hq / Hkv;
     const int nblk = capacity / BLK_TOK;
@@ -458,7 +505,7 @@ int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float 
                    mode == 1 ? perm + ((size_t)Hkv + h) * D : NULL,
                    blocks + u * (size_t)nblk * BLK_BYTES,
                    S > 0 ? k_sink + u * (size_t)S * D : NULL,
-                   S > 0 ? v_sink + u * (size_t)S * D : NULL, S, L, o);
+                   S > 0 ? v_sink + u * (size_t)S * D : NULL, S, sink_pos, sink_count, b, L, o);
     }
     return status;
 }

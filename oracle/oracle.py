@@ -45,10 +45,12 @@ def lib():
         L.orc_unpack_row.argtypes = [p, p]
         L.orc_store_token.argtypes = [p, ci, p, p, p, p, p, p]
         L.orc_load_token.argtypes = [p, ci, p, p, p, p, p, p]
+        L.orc_identify_sinks.argtypes = [p, ci, ci, C.c_float, ci, ci, p, p, p]
         L.orc_append.restype = ci
-        L.orc_append.argtypes = [p, p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p]
+        L.orc_append.argtypes = [p, p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, p, p]
         L.orc_decode.restype = ci
-        L.orc_decode.argtypes = [p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, ci, ci, ci, p]
+        L.orc_decode.argtypes = [p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, p, p, ci, ci,
+                                 ci, p]
         L.orc_attention_f64.argtypes = [p, p, p, ci, p]
         _lib = L
     return _lib
@@ -164,14 +166,30 @@ def load_token(block, tau):
 # --- cache ---------------------------------------------------------------------------
 
 class Cache:
-    """Host copy of a packed cache in the library's byte format."""
+    """Host copy of a packed cache in the library's byte format.
+    identified=True: sinks are the positions identify_sinks picks (listed in
+    sink_pos [B][S], sink_count [B]); otherwise the leading S positions."""
 
-    def __init__(self, B, Hkv, capacity, S):
+    def __init__(self, B, Hkv, capacity, S, identified=False):
         assert capacity % BLK_TOK == 0
+        assert not identified or S >= 1
         self.B, self.Hkv, self.capacity, self.S = B, Hkv, capacity, S
         self.blocks = np.zeros((B, Hkv, capacity // BLK_TOK, BLK_BYTES), np.uint8)
         self.k_sink = np.zeros((B, Hkv, max(S, 0), D), np.uint16)
         self.v_sink = np.zeros((B, Hkv, max(S, 0), D), np.uint16)
+        self.sink_pos = np.zeros((B, S), np.int32) if identified else None
+        self.sink_count = np.zeros(B, np.int32) if identified else None
+
+
+def identify_sinks(cache, act, tau, seq_lens):
+    """act: fp32 [B][T] activation magnitudes of the next T tokens.  Adds
+    the picked positions to cache.sink_pos / sink_count (in place)."""
+    assert cache.sink_pos is not None
+    act = _c(act, np.float32)
+    B, T = act.shape
+    sl = _c(seq_lens, np.int32)
+    lib().orc_identify_sinks(_p(act), B, T, float(tau), cache.S, cache.capacity, _p(sl),
+                             _p(cache.sink_pos), _p(cache.sink_count))
 
 
 def append(cache, K, V, mode, R_k=None, R_v=None, perm=None, seq_lens=None):
@@ -187,7 +205,8 @@ def append(cache, K, V, mode, R_k=None, R_v=None, perm=None, seq_lens=None):
     pc = _c(perm, np.int32) if mode == 1 else None
     return lib().orc_append(_p(K), _p(V), B, T, Hkv, mode, _p(Rk), _p(Rv), _p(pc),
                             cache.capacity, cache.S, _p(cache.blocks), _p(cache.k_sink),
-                            _p(cache.v_sink), _p(seq_lens))
+                            _p(cache.v_sink), _p(seq_lens), _p(cache.sink_pos),
+                            _p(cache.sink_count))
 
 
 def decode(cache, Q, mode, R_k=None, R_v=None, perm=None, seq_lens=None,
@@ -204,7 +223,8 @@ def decode(cache, Q, mode, R_k=None, R_v=None, perm=None, seq_lens=None,
     out = np.zeros((B, Hq, D), np.float64)
     st = lib().orc_decode(_p(Q), B, Hq, cache.Hkv, mode, _p(Rk), _p(Rv), _p(pc),
                           cache.capacity, cache.S, _p(cache.blocks), _p(cache.k_sink),
-                          _p(cache.v_sink), _p(sl), only_b, only_h, n_threads, _p(out))
+                          _p(cache.v_sink), _p(sl), _p(cache.sink_pos), _p(cache.sink_count),
+                          only_b, only_h, n_threads, _p(out))
     return out, st
 
 

@@ -433,3 +433,137 @@ def test_decode_bad_length_gives_zero_and_status():
     Q = np.ones((2, 1, D), np.float16).view(np.uint16)
     out, st = orc.decode(cache, Q, 0, R, R, None, np.array([0, 17], np.int32))
     assert st == orc.ST_BAD_LEN and not out.any()
+
+
+# --- identified sinks (RotateKV abstract, item (iii)) -----------------------------------------
+
+def _rot_inputs(rng, mode, Hkv):
+    if mode == 0:
+        Rk = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        Rv = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        return Rk, Rv, None
+    perm = np.stack([np.stack([rng.permutation(D) for _ in range(Hkv)])
+                     for _ in range(2)]).astype(np.int32)
+    return None, None, perm
+
+
+@pytest.mark.parametrize("mode,G", [(0, 2), (1, 1)])
+def test_identified_sinks_equal_leading_sinks_of_the_reordered_sequence(mode, G):
+    """Attention does not depend on the order of the positions and the
+    quantizer works token by token, so a sequence whose identified sinks sit
+    anywhere must give what the leading-sink layout gives for the same
+    tokens reordered with the sinks first: the same fp16 rows, the same
+    bytes for every INT2 token, and the same output up to the order of the
+    fp64 sums.  Appended in three calls, so the position bookkeeping across
+    calls is exercised; sequence 0 has more massive tokens than rows."""
+    rng = np.random.default_rng(41 + mode)
+    B, Hkv, S, cap = 3, 2, 3, 64
+    Hq = Hkv * G
+    chunks = [17, 1, 22]
+    Ttot = sum(chunks)
+    massive = [[2, 18, 30, 35], [0, 39], []]
+    picks = [[2, 18, 30], [0, 39], []]
+    K = (rng.standard_normal((B, Ttot, Hkv, D)) * 3).astype(np.float32)
+    V = rng.standard_normal((B, Ttot, Hkv, D)).astype(np.float32)
+    act = np.abs(rng.standard_normal((B, Ttot))).astype(np.float32)
+    for b, ts in enumerate(massive):
+        K[b, ts] *= 50
+        act[b, ts] = 1000.0
+    K = K.astype(np.float16)
+    V = V.astype(np.float16)
+    Rk, Rv, perm = _rot_inputs(rng, mode, Hkv)
+    ic = orc.Cache(B, Hkv, cap, S, identified=True)
+    sl = np.zeros(B, np.int32)
+    t0 = 0
+    for T in chunks:
+        orc.identify_sinks(ic, act[:, t0:t0 + T], 100.0, sl)
+        assert orc.append(ic, K[:, t0:t0 + T].view(np.uint16), V[:, t0:t0 + T].view(np.uint16),
+                          mode, Rk, Rv, perm, sl) == 0
+        t0 += T
+    assert list(sl) == [Ttot] * B
+    assert list(ic.sink_count) == [len(p) for p in picks]
+    for b in range(B):
+        assert list(ic.sink_pos[b, :len(picks[b])]) == picks[b]
+    Q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    out, st = orc.decode(ic, Q.view(np.uint16), mode, Rk, Rv, perm, sl)
+    assert st == 0
+    for b in range(B):
+        order = picks[b] + [t for t in range(Ttot) if t not in picks[b]]
+        n = len(picks[b])
+        lc = orc.Cache(1, Hkv, cap, n)
+        sl1 = np.zeros(1, np.int32)
+        assert orc.append(lc, K[b:b + 1, order].view(np.uint16), V[b:b + 1, order].view(np.uint16),
+                          mode, Rk, Rv, perm, sl1) == 0
+        assert np.array_equal(ic.k_sink[b, :, :n], lc.k_sink[0])
+        assert np.array_equal(ic.v_sink[b, :, :n], lc.v_sink[0])
+        assert not ic.k_sink[b, :, n:].any() and not ic.v_sink[b, :, n:].any()
+        for h in range(Hkv):
+            for pnew, p in enumerate(order):
+                got = orc.load_token(ic.blocks[b, h, p // 16], p % 16)
+                if pnew < n:
+                    kb, vb, ks, kz, vs, vz = got
+                    assert not kb.any() and not vb.any() and not kz.any()
+                    assert not vs.any() and not vz.any()
+                    assert list(ks) == [0x7E00] * 4          # the INT2 path's marker
+                else:
+                    exp = orc.load_token(lc.blocks[0, h, pnew // 16], pnew % 16)
+                    assert all(np.array_equal(x, y) for x, y in zip(got, exp))
+        ref, st1 = orc.decode(lc, Q[b:b + 1].view(np.uint16), mode, Rk, Rv, perm, sl1)
+        assert st1 == 0
+        assert np.allclose(out[b], ref[0], rtol=0, atol=1e-12)
+
+
+def test_identified_sinks_with_threshold_minus_inf_are_the_leading_sinks():
+    """tau = -inf marks every token: the first S positions get the rows, which
+    is the leading-sink layout exactly (same rows, same INT2 bytes, same
+    decode bit for bit); only the marker in the sinks' K meta differs."""
+    rng = np.random.default_rng(43)
+    B, Hkv, S, cap, T = 2, 1, 4, 48, 37
+    K = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    Rk, Rv, _ = _rot_inputs(rng, 0, Hkv)
+    ic = orc.Cache(B, Hkv, cap, S, identified=True)
+    lc = orc.Cache(B, Hkv, cap, S)
+    sl_i = np.zeros(B, np.int32)
+    sl_l = np.zeros(B, np.int32)
+    orc.identify_sinks(ic, np.zeros((B, T), np.float32), -np.inf, sl_i)
+    orc.append(ic, K.view(np.uint16), V.view(np.uint16), 0, Rk, Rv, None, sl_i)
+    orc.append(lc, K.view(np.uint16), V.view(np.uint16), 0, Rk, Rv, None, sl_l)
+    assert list(ic.sink_count) == [S] * B
+    assert np.array_equal(ic.sink_pos, np.tile(np.arange(S, dtype=np.int32), (B, 1)))
+    assert np.array_equal(ic.k_sink, lc.k_sink) and np.array_equal(ic.v_sink, lc.v_sink)
+    diff = ic.blocks != lc.blocks
+    # the differing bytes are exactly the K-meta scale fields of the S sink slots
+    exp = np.zeros_like(diff)
+    for tau in range(S):
+        r, th = tau % 8, tau // 8
+        for g in range(4):
+            off = 1024 + 8 * (4 * r + g) + 4 * th
+            exp[:, :, 0, off + 1] = True                  # 0x7E00: high byte 0x7E, low byte 0
+    assert np.array_equal(diff, exp)
+    Q = rng.standard_normal((B, Hkv, D)).astype(np.float16).view(np.uint16)
+    o_i, _ = orc.decode(ic, Q, 0, Rk, Rv, None, sl_i)
+    o_l, _ = orc.decode(lc, Q, 0, Rk, Rv, None, sl_l)
+    assert np.array_equal(o_i, o_l)
+
+
+def test_identify_sinks_threshold_order_and_skips():
+    """Ties count (act == tau), NaN never does, rows go to the earliest
+    positions, the list continues across calls, and a sequence that the
+    append would skip (no room for T tokens, or a negative length) gets no
+    sink."""
+    cache = orc.Cache(4, 1, 32, 2, identified=True)
+    act = np.array([[1, 5, 5, 9],                   # tie at 5 counts: rows -> 1, 2
+                    [np.nan, 4.99, 5, 7],           # NaN and 4.99 do not: rows -> 2, 3
+                    [9, 9, 9, 9],                   # no room: 30 + 4 > 32
+                    [9, 9, 9, 9]], np.float32)      # negative length
+    sl = np.array([0, 0, 30, -1], np.int32)
+    orc.identify_sinks(cache, act, 5.0, sl)
+    assert list(cache.sink_count) == [2, 2, 0, 0]
+    assert list(cache.sink_pos[0]) == [1, 2] and list(cache.sink_pos[1]) == [2, 3]
+    assert list(sl) == [0, 0, 30, -1]                # lengths are the append's business
+    # a later call continues at the current length and stops at S rows
+    cache2 = orc.Cache(1, 1, 32, 3, identified=True)
+    orc.identify_sinks(cache2, np.array([[0, 7, 0]], np.float32), 5.0, np.array([0], np.int32))
+    orc.identify_sinks(cache2, np.array([[7, 7, 7]], np.float32), 5.0, np.array([3], np.int32))
+    assert cache2.sink_count[0] == 3 and list(cache2.sink_pos[0]) == [1, 3, 4]
