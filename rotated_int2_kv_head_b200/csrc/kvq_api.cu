@@ -45,6 +45,10 @@ kvq_status check_cache(const kvq_cache_desc *c) {
         if (!aligned(c->block_table, 4)) return KVQ_ERR_UNSUPPORTED;
         if (c->num_blocks < 1 || (long long)c->num_blocks * c->Hkv > INT_MAX) return KVQ_ERR_INVALID_ARG;
     }
+    if (c->sink_pos) {                       // identified sinks
+        if (c->sink_fp16 < 1 || !c->sink_count) return KVQ_ERR_INVALID_ARG;
+        if (!aligned(c->sink_pos, 4) || !aligned(c->sink_count, 4)) return KVQ_ERR_UNSUPPORTED;
+    }
     return KVQ_OK;
 }
 
@@ -95,6 +99,18 @@ kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int3
     cudaError_t e = (mode == KVQ_ROT_DENSE && append_tc_eligible(K, V, T))
                         ? launch_append_tc(K, V, T, R_k, R_v, *cache, seq_lens, st)
                         : launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_identify_sinks(const float *act, int32_t T, float tau, const kvq_cache_desc *cache,
+                              const int32_t *seq_lens, void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if (!cache->sink_pos || !act || !seq_lens || T < 1) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(act, 4) || !aligned(seq_lens, 4)) return KVQ_ERR_UNSUPPORTED;
+    if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    const cudaError_t e =
+        launch_identify_sinks(act, T, tau, *cache, seq_lens, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

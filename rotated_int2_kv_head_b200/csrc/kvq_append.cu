@@ -31,14 +31,22 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
     if (bi < 0 && lane == 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
     uint8_t *block = c.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
     const int tau = p % BLK_TOK;
-    if (p < c.S) {
+    const int row = sink_row(c, b, p);                 // uniform over the warp
+    if (row >= 0) {
         uint16_t *sink = (kind == 0 ? c.k_sink : c.v_sink) +
-                         (((size_t)b * c.Hkv + h) * c.S + p) * D + 4 * lane;
+                         (((size_t)b * c.Hkv + h) * c.S + (size_t)row) * D + 4 * lane;
         uint2 pk;
         pk.x = pack_half2(v[0], v[1]);
         pk.y = pack_half2(v[2], v[3]);
         *reinterpret_cast<uint2 *>(sink) = pk;
-        if (bi >= 0) zero_token_warp(block, tau, kind);
+        if (bi >= 0) {
+            // zero codes and meta; an identified sink's K meta carries the marker
+            QuantWord q;
+            q.word = 0;
+            q.s = (c.sink_pos && kind == 0) ? (uint16_t)SINK_KMETA_MARK : (uint16_t)0;
+            q.z = 0;
+            store_token_warp(block, tau, kind, q);
+        }
     } else {
         const QuantWord q = quantize_row_warp(v);      // warp-collective: every lane runs it
         if (bi >= 0) store_token_warp(block, tau, kind, q);
@@ -245,25 +253,78 @@ __global__ void debug_quantize_kernel(const float *X, int N, uint8_t *codes, uin
     }
 }
 
+// ---- sink identification ------------------------------------------------------------------
+// One CTA per sequence.  The sinks are the tokens whose activations are
+// massive ("RotateKV", abstract item (iii)): token t of the T about to be
+// appended is one when act[b][t] >= tau, and the sequence's free fp16 rows
+// go to such tokens in position order.  Tokens go in passes of up to
+// ID_THREADS * 32: thread i flags a contiguous run of at most 32 tokens in a
+// bit mask, an exclusive scan of the flag counts over the CTA ranks the
+// flagged tokens, and each thread writes the positions whose rank is below
+// the number of rows.
+constexpr int ID_THREADS = 1024;
+constexpr int ID_RUN = 32;
+
+__global__ void __launch_bounds__(ID_THREADS)
+    identify_sinks_kernel(const float *act, int T, float tau, CacheDst c) {
+    __shared__ int wsum[ID_THREADS / 32];
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_wait();
+    pdl_trigger();
+    const int L0 = c.seq_lens[b];
+    // a sequence the append skips (and flags) gets no sinks
+    if (L0 < 0 || (long long)L0 + T > c.capacity) return;
+    int cnt = min(max(c.sink_count[b], 0), c.S);
+    const float *ab = act + (size_t)b * T;
+    for (int pass0 = 0; pass0 < T && cnt < c.S; pass0 += ID_THREADS * ID_RUN) {
+        const int n = min(T - pass0, ID_THREADS * ID_RUN);
+        const int run = (n + ID_THREADS - 1) / ID_THREADS;        // <= ID_RUN
+        const int lo = pass0 + threadIdx.x * run;
+        const int hi = min(lo + run, pass0 + n);
+        uint32_t mask = 0;
+        for (int t = lo; t < hi; t++)
+            if (ab[t] >= tau) mask |= 1u << (t - lo);
+        const int k = __popc(mask);
+        int incl = k;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll 4
+        for (int w = 0; w < ID_THREADS / 32; w++) {
+            const int x = wsum[w];
+            before += w < warp ? x : 0;
+            total += x;
+        }
+        int rank = cnt + before + incl - k;
+        while (mask != 0u && rank < c.S) {
+            const int i = __ffs(mask) - 1;
+            mask &= mask - 1u;
+            c.sink_pos[(size_t)b * c.S + rank] = L0 + lo + i;
+            ++rank;
+        }
+        cnt = min(c.S, cnt + total);
+        __syncthreads();                                   // wsum is rewritten next pass
+    }
+    if (threadIdx.x == 0) c.sink_count[b] = cnt;
+}
+
+cudaError_t launch_identify_sinks(const float *act, int T, float tau, const kvq_cache_desc &cd,
+                                  const int32_t *seq_lens, cudaStream_t st) {
+    const CacheDst c = cache_dst(cd, const_cast<int32_t *>(seq_lens), T);   // seq_lens only read
+    return launch_pdl(identify_sinks_kernel, dim3(cd.B), dim3(ID_THREADS), 0, st, act, T, tau, c);
+}
+
 // ---- host launchers (called from kvq_api.cu) -----------------------------------------------------
 cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int mode,
                                 const float *R_k, const float *R_v, const int32_t *perm,
                                 const kvq_cache_desc &cd, int32_t *seq_lens,
                                 cudaStream_t st) {
-    CacheDst c;
-    c.blocks = static_cast<uint8_t *>(cd.blocks);
-    c.table = cd.block_table;
-    c.num_blocks = cd.num_blocks;
-    c.k_sink = cd.k_sink;
-    c.v_sink = cd.v_sink;
-    c.seq_lens = seq_lens;
-    c.status = cd.status;
-    c.B = cd.B;
-    c.T = T;
-    c.Hkv = cd.Hkv;
-    c.capacity = cd.capacity;
-    c.S = cd.sink_fp16;
-    c.nblk = cd.capacity / BLK_TOK;
+    const CacheDst c = cache_dst(cd, seq_lens, T);
     if (mode == KVQ_ROT_DENSE) {
         DenseRows a;
         a.X0 = K;

@@ -373,6 +373,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
         }
         int cur_job = -1, L0 = -1;
+        int s_n = 0, s_last = -1;                       // identified sinks of the job's sequence
         for (int i = eg; i < nmy; i += EPI_GROUPS) {
             // decisions stay warp-uniform: tcgen05.ld below is .sync.aligned
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
@@ -402,6 +403,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 b = (j >> 1) / c.Hkv;
                 if (j != cur_job) {
                     L0 = start_len_thread(c, b, kind == 0 && h == 0 && gt == 0);
+                    sink_list_end(c, b, s_n, s_last);
                     cur_job = j;
                 }
             }
@@ -409,7 +411,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             const bool valid = t < a.T && (!TO_CACHE || L0 >= 0);
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * 128);
             const int p = L0 + t;
-            const bool sink = TO_CACHE && valid && p < c.S;
+            const int srow = TO_CACHE && valid ? sink_row_after(c, b, p, s_n, s_last) : -1;
+            const bool sink = srow >= 0;
             uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0}, meta[4] = {0, 0, 0, 0};
 #pragma unroll 1
             for (int g = 0; g < NG; g++) {
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                         *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                 } else if (sink) {
                     uint16_t *dst = (kind == 0 ? c.k_sink : c.v_sink) +
-                                    (((size_t)b * c.Hkv + h) * c.S + p) * D + 32 * g;
+                                    (((size_t)b * c.Hkv + h) * c.S + (size_t)srow) * D + 32 * g;
 #pragma unroll
                     for (int e = 0; e < 32; e += 8)
                         *reinterpret_cast<uint4 *>(dst + e) =
@@ -444,8 +447,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     ? cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, p / BLK_TOK)
                     : 0;
             if (bix < 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+            if (sink && c.sink_pos && kind == 0) {
+#pragma unroll
+                for (int g = 0; g < NG; g++) meta[g] = SINK_KMETA_MARK;
+            }
             if (TO_CACHE && valid && bix >= 0) {
                 // sink rows leave zero codes and metadata in their cache slots
+                // (an identified sink: the marker in its K meta)
                 uint8_t *block = c.blocks + (size_t)bix * BLK_BYTES;
                 const int tau = p % BLK_TOK;
                 if (kind == 0) {
@@ -539,20 +547,7 @@ cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const 
     CUtensorMap mk, mv;
     const long long rows = (long long)cd.B * T;
     if (!make_map(&mk, K, cd.Hkv, rows) || !make_map(&mv, V, cd.Hkv, rows)) return cudaErrorInvalidValue;
-    CacheDst c;
-    c.blocks = static_cast<uint8_t *>(cd.blocks);
-    c.table = cd.block_table;
-    c.num_blocks = cd.num_blocks;
-    c.k_sink = cd.k_sink;
-    c.v_sink = cd.v_sink;
-    c.seq_lens = seq_lens;
-    c.status = cd.status;
-    c.B = cd.B;
-    c.T = T;
-    c.Hkv = cd.Hkv;
-    c.capacity = cd.capacity;
-    c.S = cd.sink_fp16;
-    c.nblk = cd.capacity / BLK_TOK;
+    const CacheDst c = cache_dst(cd, seq_lens, T);
     TcArgs a;
     a.R0 = R_k;
     a.R1 = R_v;

@@ -71,6 +71,13 @@ struct DecodeArgs {
     uint8_t *qprep;    // [B*Hq][QB] prepared queries
     float *part;       // [(C+U)*G][PART]
     uint16_t *out;
+    // S: leading fp16 sinks (positions 0..S-1; 0 with identified sinks).
+    // Srows: fp16 sink rows per (b, h).  sink_pos / sink_count: identified
+    // sinks ([B][Srows] ascending positions, rows in use), else null; their
+    // INT2 slots carry a NaN K scale, so their scores come out NaN and are
+    // turned into -inf.
+    const int32_t *sink_pos, *sink_count;
+    int Srows;
     int B, Hq, Hkv, G, S, capacity, nblk, mode, C;
     // qlen queries per sequence: query "head" hq (of Hq = heads x qlen) is
     // query i = hq % qlen of its head and sees positions < L - (qlen-1-i)
@@ -675,7 +682,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                         const int lim = Lcur - (a.qlen - 1 - lane_head<G>(c, hh) % a.qlen);
                         v = (bi < nmine && pos >= a.S && pos < lim) ? v : NEG_INF;
                     }
-                    sco[bi][st][hh] = v;
+                    // an identified sink's slot scores NaN (its K scale is the
+                    // marker): fmax with -inf returns -inf for NaN, v otherwise
+                    sco[bi][st][hh] = fmaxf(v, NEG_INF);
                 }
         }
     };
@@ -927,7 +936,16 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     const int L = a.seq_lens[b];
     const int Li = L - (a.qlen - 1 - hq % a.qlen);           // this query's context
     const bool lok = (L >= 1 && L <= a.capacity && Li >= 1);
-    const int ns = (a.S > 0 && lok) ? min(a.S, Li) : 0;
+    // fp16 rows this query sees: rows 0..ns-1.  Leading sinks: positions
+    // < min(S, Li).  Identified sinks: the listed positions below Li (a
+    // prefix of the ascending list).
+    int ns;
+    if (!a.sink_pos) {
+        ns = (a.S > 0 && lok) ? min(a.S, Li) : 0;
+    } else {
+        const int n = min(max(a.sink_count[b], 0), a.Srows);
+        ns = __syncthreads_count(lok && t < n && a.sink_pos[(size_t)b * a.Srows + t] < Li);
+    }
     if (ns > 0) {
         const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
         if (a.mode == KVQ_ROT_DENSE) {
@@ -970,8 +988,8 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         __syncthreads();
         if (t < D) qs[t] *= LOG2E * 0.08838834764831845f;      // exp2 domain, like the partials
         __syncthreads();
-        const uint16_t *ks = a.k_sink + ((size_t)b * a.Hkv + h) * a.S * D;
-        const uint16_t *vs = a.v_sink + ((size_t)b * a.Hkv + h) * a.S * D;
+        const uint16_t *ks = a.k_sink + ((size_t)b * a.Hkv + h) * a.Srows * D;
+        const uint16_t *vs = a.v_sink + ((size_t)b * a.Hkv + h) * a.Srows * D;
         for (int tk = warp; tk < ns; tk += MRG_THREADS / 32) {
             const uint2 uu = *reinterpret_cast<const uint2 *>(ks + (size_t)tk * D + 4 * lane);
             const float2 k01 = unpack_half2(uu.x), k23 = unpack_half2(uu.y);
@@ -1196,7 +1214,10 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.Hq = Hq;
     a.Hkv = cd.Hkv;
     a.G = Hq / cd.Hkv;
-    a.S = cd.sink_fp16;
+    a.sink_pos = cd.sink_pos;
+    a.sink_count = cd.sink_count;
+    a.Srows = cd.sink_fp16;
+    a.S = cd.sink_pos ? 0 : cd.sink_fp16;
     a.capacity = cd.capacity;
     a.nblk = cd.capacity / BLK_TOK;
     a.mode = mode;

@@ -286,6 +286,8 @@ cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, const float *R, flo
                                    cudaStream_t st);
 cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
                                   cudaStream_t st);
+cudaError_t launch_identify_sinks(const float *act, int T, float tau, const kvq_cache_desc &cd,
+                                  const int32_t *seq_lens, cudaStream_t st);
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
@@ -309,7 +311,64 @@ struct CacheDst {
     int B, T, Hkv, capacity, S, nblk;
     const int32_t *table;     // paged cache: [B][nblk] pool block per logical block, else null
     int num_blocks;           // paged: pool blocks
+    int32_t *sink_pos;        // identified sinks: [B][S] ascending positions, else null
+    int32_t *sink_count;      // identified sinks: [B] rows in use
 };
+
+// The append destination of cache `cd`.
+inline CacheDst cache_dst(const kvq_cache_desc &cd, int32_t *seq_lens, int T) {
+    CacheDst c;
+    c.blocks = static_cast<uint8_t *>(cd.blocks);
+    c.table = cd.block_table;
+    c.num_blocks = cd.num_blocks;
+    c.k_sink = cd.k_sink;
+    c.v_sink = cd.v_sink;
+    c.seq_lens = seq_lens;
+    c.status = cd.status;
+    c.B = cd.B;
+    c.T = T;
+    c.Hkv = cd.Hkv;
+    c.capacity = cd.capacity;
+    c.S = cd.sink_fp16;
+    c.nblk = cd.capacity / BLK_TOK;
+    c.sink_pos = cd.sink_pos;
+    c.sink_count = cd.sink_count;
+    return c;
+}
+
+// K meta word {s, z} of an identified sink's INT2 slot in every group: s is
+// the fp16 quiet NaN 0x7E00, z = 0.  Any score computed from it is NaN,
+// which the decode turns into -inf.
+constexpr uint32_t SINK_KMETA_MARK = 0x7E00u;
+
+// fp16 sink row of position p of sequence b, or -1 if p is stored in INT2.
+// Leading sinks: positions 0..S-1 are rows 0..S-1.  Identified sinks: the
+// index of p in the sequence's ascending list; `last` is the list's last
+// entry (or -1 for an empty list), which almost every position lies past.
+__device__ __forceinline__ int sink_row_after(const CacheDst &c, int b, int p, int n, int last) {
+    if (!c.sink_pos) return p < c.S ? p : -1;
+    if (p > last) return -1;
+    const int32_t *sp = c.sink_pos + (size_t)b * c.S;
+    int lo = 0, hi = n - 1;                      // first entry >= p (one exists: p <= last)
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (sp[mid] < p) lo = mid + 1; else hi = mid;
+    }
+    return sp[lo] == p ? lo : -1;
+}
+// Rows in use and last listed position of sequence b (identified sinks).
+__device__ __forceinline__ void sink_list_end(const CacheDst &c, int b, int &n, int &last) {
+    n = 0;
+    last = -1;
+    if (!c.sink_pos) return;
+    n = min(max(c.sink_count[b], 0), c.S);
+    if (n > 0) last = c.sink_pos[(size_t)b * c.S + n - 1];
+}
+__device__ __forceinline__ int sink_row(const CacheDst &c, int b, int p) {
+    int n, last;
+    sink_list_end(c, b, n, last);
+    return sink_row_after(c, b, p, n, last);
+}
 
 // Index (in 1536-byte blocks from `blocks`) of KV head h of logical block lb
 // of sequence b; -1 for a paged entry outside the pool.

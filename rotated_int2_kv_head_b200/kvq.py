@@ -41,7 +41,8 @@ class CacheDesc(C.Structure):
     _fields_ = [("B", C.c_int32), ("Hkv", C.c_int32), ("head_dim", C.c_int32),
                 ("group", C.c_int32), ("capacity", C.c_int32), ("sink_fp16", C.c_int32),
                 ("blocks", C.c_void_p), ("k_sink", C.c_void_p), ("v_sink", C.c_void_p),
-                ("status", C.c_void_p), ("block_table", C.c_void_p), ("num_blocks", C.c_int32)]
+                ("status", C.c_void_p), ("block_table", C.c_void_p), ("num_blocks", C.c_int32),
+                ("sink_pos", C.c_void_p), ("sink_count", C.c_void_p)]
 
 
 _lib = None
@@ -61,6 +62,8 @@ def lib():
     L.kvq_cache_bytes.argtypes = [i32, i32, i32]
     L.kvq_rotate_quantize_append.restype = C.c_int
     L.kvq_rotate_quantize_append.argtypes = [p, p, i32, C.c_int, p, p, p, C.POINTER(CacheDesc), p, p]
+    L.kvq_identify_sinks.restype = C.c_int
+    L.kvq_identify_sinks.argtypes = [p, i32, C.c_float, C.POINTER(CacheDesc), p, p]
     L.kvq_decode_workspace_size.restype = sz
     L.kvq_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     L.kvq_decode_attention.restype = C.c_int
@@ -115,25 +118,45 @@ def _need(t, dtype, name, shape=None):
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
 
 
-class KVCache:
-    """A packed INT2 cache for B sequences x Hkv heads (memory owned by torch)."""
+def _sink_arrays(cache, B, Hkv, sink_fp16, identified_sinks, device):
+    """fp16 sink rows, and for identified sinks the position list and counts."""
+    if identified_sinks and sink_fp16 < 1:
+        raise ValueError("identified sinks need sink_fp16 >= 1")
+    if sink_fp16 > 0:
+        cache.k_sink = torch.zeros((B, Hkv, sink_fp16, D), dtype=torch.float16, device=device)
+        cache.v_sink = torch.zeros_like(cache.k_sink)
+    else:
+        cache.k_sink = cache.v_sink = None
+    if identified_sinks:
+        cache.sink_pos = torch.zeros((B, sink_fp16), dtype=torch.int32, device=device)
+        cache.sink_count = torch.zeros(B, dtype=torch.int32, device=device)
+    else:
+        cache.sink_pos = cache.sink_count = None
 
-    def __init__(self, B, Hkv, capacity, sink_fp16=0, device="cuda"):
+
+def _desc(cache, table=0, num_blocks=0):
+    p = lambda t: 0 if t is None else t.data_ptr()
+    return CacheDesc(cache.B, cache.Hkv, D, GROUP, cache.capacity, cache.sink_fp16,
+                     cache.blocks.data_ptr(), p(cache.k_sink), p(cache.v_sink),
+                     cache.status.data_ptr(), table, num_blocks, p(cache.sink_pos),
+                     p(cache.sink_count))
+
+
+class KVCache:
+    """A packed INT2 cache for B sequences x Hkv heads (memory owned by torch).
+    sink_fp16 rows of fp16 sinks per (sequence, head): the leading positions,
+    or with identified_sinks=True the positions kvq_identify_sinks picks
+    (listed in sink_pos [B][sink_fp16], sink_count [B])."""
+
+    def __init__(self, B, Hkv, capacity, sink_fp16=0, device="cuda", identified_sinks=False):
         nbytes = lib().kvq_cache_bytes(B, Hkv, capacity)
         if nbytes == 0:
             raise ValueError("bad cache shape B=%d Hkv=%d capacity=%d" % (B, Hkv, capacity))
         self.B, self.Hkv, self.capacity, self.sink_fp16 = B, Hkv, capacity, sink_fp16
         self.blocks = torch.zeros(nbytes, dtype=torch.uint8, device=device)
-        if sink_fp16 > 0:
-            self.k_sink = torch.zeros((B, Hkv, sink_fp16, D), dtype=torch.float16, device=device)
-            self.v_sink = torch.zeros_like(self.k_sink)
-        else:
-            self.k_sink = self.v_sink = None
+        _sink_arrays(self, B, Hkv, sink_fp16, identified_sinks, device)
         self.status = torch.zeros(2, dtype=torch.int32, device=device)   # errors, append counter
-        self.desc = CacheDesc(B, Hkv, D, GROUP, capacity, sink_fp16, self.blocks.data_ptr(),
-                              0 if self.k_sink is None else self.k_sink.data_ptr(),
-                              0 if self.v_sink is None else self.v_sink.data_ptr(),
-                              self.status.data_ptr())
+        self.desc = _desc(self)
 
     def block_view(self):
         """blocks as uint8 [B][Hkv][capacity/16][1536]."""
@@ -145,23 +168,17 @@ class PagedKVCache(KVCache):
     1536 bytes) and an int32 block table [B][capacity/16] mapping every
     sequence's logical blocks to pool blocks (memory owned by torch)."""
 
-    def __init__(self, B, Hkv, capacity, num_blocks, block_table, sink_fp16=0, device="cuda"):
+    def __init__(self, B, Hkv, capacity, num_blocks, block_table, sink_fp16=0, device="cuda",
+                 identified_sinks=False):
         if capacity % BLOCK_TOKENS or num_blocks < 1:
             raise ValueError("bad paged cache shape")
         _need(block_table, torch.int32, "block_table", (B, capacity // BLOCK_TOKENS))
         self.B, self.Hkv, self.capacity, self.sink_fp16 = B, Hkv, capacity, sink_fp16
         self.num_blocks, self.block_table = num_blocks, block_table
         self.blocks = torch.zeros(num_blocks * Hkv * BLOCK_BYTES, dtype=torch.uint8, device=device)
-        if sink_fp16 > 0:
-            self.k_sink = torch.zeros((B, Hkv, sink_fp16, D), dtype=torch.float16, device=device)
-            self.v_sink = torch.zeros_like(self.k_sink)
-        else:
-            self.k_sink = self.v_sink = None
+        _sink_arrays(self, B, Hkv, sink_fp16, identified_sinks, device)
         self.status = torch.zeros(2, dtype=torch.int32, device=device)
-        self.desc = CacheDesc(B, Hkv, D, GROUP, capacity, sink_fp16, self.blocks.data_ptr(),
-                              0 if self.k_sink is None else self.k_sink.data_ptr(),
-                              0 if self.v_sink is None else self.v_sink.data_ptr(),
-                              self.status.data_ptr(), block_table.data_ptr(), num_blocks)
+        self.desc = _desc(self, block_table.data_ptr(), num_blocks)
 
     def block_view(self):
         """The pool as uint8 [num_blocks][Hkv][1536]."""
@@ -193,6 +210,19 @@ def kvq_rotate_quantize_append(K, V, mode, R_k, R_v, perm, cache, seq_lens, stre
            lib().kvq_rotate_quantize_append(_ptr(K), _ptr(V), T, mode, _ptr(R_k), _ptr(R_v),
                                             _ptr(perm), C.byref(cache.desc), _ptr(seq_lens),
                                             _stream(stream)))
+
+
+def kvq_identify_sinks(act, tau, cache, seq_lens, stream=None):
+    """act fp32 [B][T]: activation magnitudes of the next T tokens (call just
+    before appending them); seq_lens int32 [B], the lengths before that
+    append.  Tokens with act >= tau take the free fp16 sink rows."""
+    _need(act, torch.float32, "act")
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    if act.dim() != 2 or act.shape[0] != cache.B:
+        raise ValueError("act must have shape (B, T)")
+    _check("kvq_identify_sinks",
+           lib().kvq_identify_sinks(_ptr(act), act.shape[1], float(tau), C.byref(cache.desc),
+                                    _ptr(seq_lens), _stream(stream)))
 
 
 def kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count=None):

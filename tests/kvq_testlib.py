@@ -38,21 +38,29 @@ def gpu_decode(cache, Q, w, rt, seq_lens, max_ctx):
 
 
 def upload_oracle_cache(oc, device="cuda"):
-    """A libkvq cache holding the oracle's bytes."""
-    c = kvq.KVCache(oc.B, oc.Hkv, oc.capacity, oc.S, device=device)
+    """A libkvq cache holding the oracle's bytes (and its sink list)."""
+    identified = oc.sink_pos is not None
+    c = kvq.KVCache(oc.B, oc.Hkv, oc.capacity, oc.S, device=device, identified_sinks=identified)
     c.blocks.copy_(torch.from_numpy(oc.blocks.reshape(-1)))
     if oc.S > 0:
         c.k_sink.copy_(torch.from_numpy(oc.k_sink.view(np.float16)))
         c.v_sink.copy_(torch.from_numpy(oc.v_sink.view(np.float16)))
+    if identified:
+        c.sink_pos.copy_(torch.from_numpy(oc.sink_pos))
+        c.sink_count.copy_(torch.from_numpy(oc.sink_count))
     return c
 
 
 def download_cache(c):
-    oc = orc.Cache(c.B, c.Hkv, c.capacity, c.sink_fp16)
+    identified = getattr(c, "sink_pos", None) is not None
+    oc = orc.Cache(c.B, c.Hkv, c.capacity, c.sink_fp16, identified=identified)
     oc.blocks[:] = c.block_view().cpu().numpy()
     if c.sink_fp16 > 0:
         oc.k_sink[:] = f16bits(c.k_sink)
         oc.v_sink[:] = f16bits(c.v_sink)
+    if identified:
+        oc.sink_pos[:] = c.sink_pos.cpu().numpy()
+        oc.sink_count[:] = c.sink_count.cpu().numpy()
     return oc
 
 

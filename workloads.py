@@ -17,6 +17,10 @@ The five workloads (head_dim 128, INT2 groups of 32 along head_dim):
   ragged      B=64, 32 heads, context lengths uniform in [1024, 65536],
               dense rotation, 8 key outlier channels x20; plus a separate
               bulk append of 32768 prefill tokens x 32 heads for B=4.
+  gqa_sinks_identified
+              gqa_sinks, but the 4 fp16 rows go to the tokens picked by their
+              activation magnitude: position 0 and each other token with
+              probability 4e-5 are massive (magnitude >= 1000, keys x50).
 
 Every K/V row is drawn from a stream keyed by (workload, kind, sequence,
 1024-token chunk), so any token range can be regenerated on its own without
@@ -50,6 +54,10 @@ class Workload:
     channel_scale: Optional[tuple] = None   # (lo, hi) log-uniform per channel
     sink_key_scale: float = 1.0
     ragged: Optional[tuple] = None          # (lo, hi) uniform context lengths
+    # identified sinks: each token is "massive" with this probability (and
+    # position 0 always is); its activation magnitude is >= 1000 against
+    # |N(0,1)| for the rest, and its key row is scaled by sink_key_scale
+    massive_rate: float = 0.0
     extra: dict = field(default_factory=dict)
 
     @property
@@ -78,16 +86,25 @@ WORKLOADS = {
                           context=131072, sink_key_scale=50.0),
     "ragged": Workload("ragged", 1005, B=64, Hq=32, Hkv=32, mode=0, ragged=(1024, 65536),
                        k_outliers=8, extra={"prefill_B": 4, "prefill_T": 32768}),
+    # gqa_sinks with its 4 fp16 rows given to the massive tokens instead of
+    # the leading ones (position 0 plus about 5 more per sequence)
+    "gqa_sinks_identified": Workload("gqa_sinks_identified", 1006, B=8, Hq=32, Hkv=8, mode=0,
+                                     sink=4, context=131072, sink_key_scale=50.0,
+                                     massive_rate=4e-5),
 }
+
+# activation magnitude at and above which a token counts as massive (the
+# drawn magnitudes are |N(0,1)| or >= 1000)
+MASSIVE_TAU = 100.0
 
 
 def custom(name="custom", seed=1, B=1, Hq=1, Hkv=1, mode=0, sink=0, context=64,
-           append_T=1, k_outliers=0, channel_scale=None, sink_key_scale=1.0,
+           append_T=1, k_outliers=0, channel_scale=None, sink_key_scale=1.0, massive_rate=0.0,
            ragged=None) -> Workload:
     """A small workload of the same families, for edge-case tests."""
     return Workload(name, seed, B=B, Hq=Hq, Hkv=Hkv, mode=mode, sink=sink, context=context,
                     append_T=append_T, k_outliers=k_outliers, channel_scale=channel_scale,
-                    sink_key_scale=sink_key_scale, ragged=ragged)
+                    sink_key_scale=sink_key_scale, ragged=ragged, massive_rate=massive_rate)
 
 
 # --- rotations and per-channel structure (numpy, seeded) -------------------------------
@@ -136,6 +153,29 @@ def _chunk_rows(w: Workload, kind: int, b: int, chunk: int, device) -> torch.Ten
     return torch.randn((CHUNK, w.Hkv, D), generator=g, device=device, dtype=torch.float32)
 
 
+def _chunk_act(w: Workload, b: int, chunk: int) -> np.ndarray:
+    rng = np.random.default_rng([w.seed, 77, b, chunk])
+    a = np.abs(rng.standard_normal(CHUNK)).astype(np.float32)
+    massive = rng.random(CHUNK) < w.massive_rate
+    if chunk == 0:
+        massive[0] = True
+    a[massive] = (1000.0 * (1.0 + rng.random(int(massive.sum())))).astype(np.float32)
+    return a
+
+
+def activations(w: Workload, b: int, t0: int, t1: int) -> np.ndarray:
+    """Activation magnitude of the tokens [t0, t1) of sequence b, fp32 (numpy):
+    |N(0,1)|, or >= 1000 for massive tokens (none unless massive_rate > 0)."""
+    if t1 <= t0:
+        return np.zeros(0, np.float32)
+    if w.massive_rate <= 0.0:
+        return np.abs(np.random.default_rng([w.seed, 78, b, t0]).standard_normal(t1 - t0)
+                      ).astype(np.float32)
+    parts = [_chunk_act(w, b, c) for c in range(t0 // CHUNK, (t1 - 1) // CHUNK + 1)]
+    a = np.concatenate(parts)
+    return a[t0 - (t0 // CHUNK) * CHUNK:][:t1 - t0]
+
+
 def kv_rows(w: Workload, b: int, t0: int, t1: int, device="cpu"):
     """K and V rows of sequence b for positions [t0, t1): fp16 [t1-t0][Hkv][128]."""
     ks, vs = channel_scales(w)
@@ -151,7 +191,11 @@ def kv_rows(w: Workload, b: int, t0: int, t1: int, device="cpu"):
             parts.append(rows[lo:hi])
         x = torch.cat(parts) if parts else torch.empty((0, w.Hkv, D), device=device)
         x = x * sc[None]
-        if kind == 0 and w.sink and w.sink_key_scale != 1.0 and t0 < w.sink:
+        if w.massive_rate > 0.0:
+            if kind == 0 and w.sink_key_scale != 1.0 and t1 > t0:
+                m = torch.from_numpy(activations(w, b, t0, t1) >= MASSIVE_TAU).to(device)
+                x[m] *= w.sink_key_scale
+        elif kind == 0 and w.sink and w.sink_key_scale != 1.0 and t0 < w.sink:
             n = min(w.sink, t1) - t0
             x[:n] *= w.sink_key_scale
         outs.append(x.to(torch.float16))
