@@ -403,6 +403,86 @@ def extension_rates(step, device, reps=50):
     return res
 
 
+def sink_rates(device, reps=30):
+    """Identified sinks on their full-size workload (gqa_sinks_identified:
+    B=8, 32 query heads over 8 KV heads, context 131072, 4 fp16 rows per
+    sequence): the same tokens appended into a cache with identified sinks
+    (kvq_identify_sinks before each append) and into one with the 4 leading
+    positions as sinks; decode-only times of both (L2 flushed before each
+    call) and the time of the identification kernel for one decode step
+    (T=1) and for a 32768-token prefill chunk."""
+    import rotated_int2_kv_head_b200 as kvq
+    w = W.WORKLOADS["gqa_sinks_identified"]
+    L = int(w.context)
+    cap = L
+    Rk, Rv, _ = W.rotations(w)
+    rk = torch.from_numpy(Rk).to(device)
+    rv = torch.from_numpy(Rv).to(device)
+    ident = kvq.KVCache(w.B, w.Hkv, cap, w.sink, device=device, identified_sinks=True)
+    lead = kvq.KVCache(w.B, w.Hkv, cap, w.sink, device=device)
+    sl_i = torch.zeros(w.B, dtype=torch.int32, device=device)
+    sl_l = torch.zeros_like(sl_i)
+    chunk = 8192
+    for t0 in range(0, L, chunk):
+        t1 = min(L, t0 + chunk)
+        K, V = W.kv_batch(w, t0, t1, device)
+        act = torch.from_numpy(np.stack([W.activations(w, b, t0, t1) for b in range(w.B)])).to(device)
+        kvq.kvq_identify_sinks(act, W.MASSIVE_TAU, ident, sl_i)
+        kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, None, ident, sl_i)
+        kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, None, lead, sl_l)
+    torch.cuda.synchronize(device)
+    Q = W.queries(w, device)
+    ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, L, device=device)
+    flush = L2Flush(device)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def timed(fn, n=reps):
+        ms = []
+        for k in range(n + 3):
+            flush(k)
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize(device)
+            if k >= 3:
+                ms.append(ev[0].elapsed_time(ev[1]))
+        return float(np.median(ms))
+
+    out_i = torch.empty_like(Q)
+    out_l = torch.empty_like(Q)
+    dec_i = timed(lambda: kvq.kvq_decode_attention(Q, ident, w.mode, rk, rv, None, sl_i, w.sink, L,
+                                                   ws, out_i))
+    dec_l = timed(lambda: kvq.kvq_decode_attention(Q, lead, w.mode, rk, rv, None, sl_l, w.sink, L,
+                                                   ws, out_l))
+    # identification alone, on a scratch copy of the sink list (the
+    # lengths are set so that every sequence has room for the tokens)
+    probe = kvq.KVCache(w.B, w.Hkv, 32768 + 16, w.sink, device=device, identified_sinks=True)
+    sl0 = torch.zeros(w.B, dtype=torch.int32, device=device)
+    a1 = torch.from_numpy(np.stack([W.activations(w, b, 5, 6) for b in range(w.B)])).to(device)
+    aP = torch.from_numpy(np.stack([W.activations(w, b, 0, 32768) for b in range(w.B)])).to(device)
+
+    def ident_once(a):
+        probe.sink_count.zero_()
+        kvq.kvq_identify_sinks(a, W.MASSIVE_TAU, probe, sl0)
+
+    id_step = timed(lambda: ident_once(a1))
+    id_pre = timed(lambda: ident_once(aP))
+    counts = ident.sink_count.cpu().tolist()
+    if max(kvq.kvq_get_status(ident), kvq.kvq_get_status(lead)) != 0:
+        raise RuntimeError("device status after the identified-sink timings")
+    if not bool(torch.isfinite(out_i.float()).all()):
+        raise RuntimeError("non-finite decode output with identified sinks")
+    kv_bytes = w.B * w.Hkv * L * 96
+    return {"workload": "gqa_sinks_identified", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+            "context": L, "sink_rows": w.sink, "sinks_per_sequence": counts,
+            "how": "decode only / identification only, L2 flushed before each call, "
+                   "median of %d; includes a sink-count reset memset in the identification "
+                   "timings" % reps,
+            "decode_identified_ms": dec_i, "decode_leading_ms": dec_l,
+            "decode_identified_packed_kv_gbs": kv_bytes / (dec_i * 1e-3) / 1e9,
+            "identify_step_ms": id_step, "identify_prefill_32768_ms": id_pre}
+
+
 def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
     the first `heads` KV heads of sequence 0 (their K/V rows are the very
@@ -641,6 +721,7 @@ def run_cuda(args):
         line["append"] = append_rates(dev, peak)
     if world == 1 and not args.no_extensions:
         line["extensions"] = extension_rates(step, dev)
+        line["extensions"]["identified_sinks"] = sink_rates(dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, step, dev)
     print(json.dumps(line), flush=True)
