@@ -1,6 +1,7 @@
 // libkvq C ABI: argument validation, launch selection, workspace sizing and
 // the status word.  No allocation happens here or in any kernel; the only
 // state kept is a per-device cache of the SM count.
+#include <atomic>
 #include <limits.h>
 
 #include "kvq_internal.cuh"
@@ -16,13 +17,16 @@ constexpr int MIN_BLOCKS_PER_CTA = 64;   // 1024 tokens: below this, fewer CTAs
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 int device_sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    if (dev >= 0 && dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) cached[dev] = n;
+    if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 

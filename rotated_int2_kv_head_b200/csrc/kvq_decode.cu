@@ -35,6 +35,8 @@
 // operand.  The 4^g factors are folded into per-group fp32 scales.  The
 // dequantisation c*s + z is factored: sum_j q_j (c_j s + z) =
 // s*sum_j q_j c_j + z*sum_j q_j, so only the integer codes go through the MMA.
+#include <atomic>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -1177,9 +1179,18 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int C) {
 template <int G, bool PAGED>
 static cudaError_t launch_split_t(const DecodeArgs &a, cudaStream_t st) {
     const size_t smem = split_smem_bytes(G);
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<G, PAGED>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // the dynamic shared-memory opt-in holds per device: set it once on each
+    static std::atomic<unsigned long long> opted{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+    if (bit == 0ull || (opted.load(std::memory_order_acquire) & bit) == 0ull) {
+        e = cudaFuncSetAttribute(decode_split_kernel<G, PAGED>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        opted.fetch_or(bit, std::memory_order_acq_rel);
+    }
     return launch_pdl(decode_split_kernel<G, PAGED>, dim3(a.C), dim3(DEC_THREADS), smem, st, a);
 }
 

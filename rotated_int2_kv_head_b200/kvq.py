@@ -93,13 +93,24 @@ def lib():
 
 
 def _ptr(t):
-    return None if t is None else C.c_void_p(t.data_ptr())
+    # ctypes turns the int into the c_void_p argument
+    return None if t is None else t.data_ptr()
 
 
-def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return C.c_void_p(stream.cuda_stream)
+# torch's raw current-stream query (an int, no Stream object); the public
+# torch.cuda.current_stream() builds a Python object per call, which costs
+# more than a kernel launch on the host.  Fall back to it if absent.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, t=None):
+    """cudaStream_t (as an int) for a call on tensor t's device: `stream` if
+    given, else torch's current stream of that device."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and t is not None:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _check(fn, code):
@@ -112,9 +123,9 @@ def _need(t, dtype, name, shape=None):
         return
     if t.dtype != dtype:
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
-    if not t.is_cuda or not t.is_contiguous():
+    if not (t.is_cuda and t.is_contiguous()):
         raise ValueError("%s must be a contiguous CUDA tensor" % name)
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
 
 
@@ -209,7 +220,7 @@ def kvq_rotate_quantize_append(K, V, mode, R_k, R_v, perm, cache, seq_lens, stre
     _check("kvq_rotate_quantize_append",
            lib().kvq_rotate_quantize_append(_ptr(K), _ptr(V), T, mode, _ptr(R_k), _ptr(R_v),
                                             _ptr(perm), C.byref(cache.desc), _ptr(seq_lens),
-                                            _stream(stream)))
+                                            _stream(stream, K)))
 
 
 def kvq_identify_sinks(act, tau, cache, seq_lens, stream=None):
@@ -222,7 +233,7 @@ def kvq_identify_sinks(act, tau, cache, seq_lens, stream=None):
         raise ValueError("act must have shape (B, T)")
     _check("kvq_identify_sinks",
            lib().kvq_identify_sinks(_ptr(act), act.shape[1], float(tau), C.byref(cache.desc),
-                                    _ptr(seq_lens), _stream(stream)))
+                                    _ptr(seq_lens), _stream(stream, act)))
 
 
 def kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count=None):
@@ -255,7 +266,7 @@ def kvq_decode_attention(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, ma
            lib().kvq_decode_attention(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k), _ptr(R_v),
                                       _ptr(perm), _ptr(seq_lens), sink_fp16, max_ctx,
                                       _ptr(workspace), workspace.numel(), _ptr(out),
-                                      _stream(stream)))
+                                      _stream(stream, Q)))
 
 
 KVQ_DECODE_OUT_ROTATED = 1
@@ -279,7 +290,7 @@ def kvq_decode_attention_ex(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
            lib().kvq_decode_attention_ex(_ptr(Q), Hq, q_len, flags, C.byref(cache.desc), mode,
                                          _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
                                          sink_fp16, max_ctx, _ptr(workspace), workspace.numel(),
-                                         _ptr(out), _stream(stream)))
+                                         _ptr(out), _stream(stream, Q)))
 
 
 def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
@@ -296,7 +307,7 @@ def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp
            lib().kvq_decode_attention_timed(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k),
                                             _ptr(R_v), _ptr(perm), _ptr(seq_lens), sink_fp16,
                                             max_ctx, _ptr(workspace), workspace.numel(), _ptr(out),
-                                            _stream(stream), C.c_void_p(ev_begin.cuda_event),
+                                            _stream(stream, Q), C.c_void_p(ev_begin.cuda_event),
                                             C.c_void_p(ev_end.cuda_event)))
 
 
@@ -312,17 +323,19 @@ def kvq_decode_attention_noalloc(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_
     _check("kvq_decode_attention_noalloc",
            lib().kvq_decode_attention_noalloc(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k),
                                               _ptr(R_v), _ptr(perm), _ptr(seq_lens), sink_fp16,
-                                              max_ctx, _ptr(out), _stream(stream)))
+                                              max_ctx, _ptr(out), _stream(stream, Q)))
 
 
 def kvq_get_status(cache, stream=None):
     v = C.c_int32(0)
-    _check("kvq_get_status", lib().kvq_get_status(C.byref(cache.desc), _stream(stream), C.byref(v)))
+    _check("kvq_get_status", lib().kvq_get_status(C.byref(cache.desc), _stream(stream, cache.status),
+                                                  C.byref(v)))
     return v.value
 
 
 def kvq_clear_status(cache, stream=None):
-    _check("kvq_clear_status", lib().kvq_clear_status(C.byref(cache.desc), _stream(stream)))
+    _check("kvq_clear_status", lib().kvq_clear_status(C.byref(cache.desc),
+                                                      _stream(stream, cache.status)))
 
 
 def kvq_debug_rotate_f32(X, mode, R=None, perm=None, variant=0, stream=None):
@@ -332,7 +345,7 @@ def kvq_debug_rotate_f32(X, mode, R=None, perm=None, variant=0, stream=None):
     out = torch.empty((N, D), dtype=torch.float32, device=X.device)
     _check("kvq_debug_rotate_f32",
            lib().kvq_debug_rotate_f32(_ptr(X), N, mode, _ptr(R), _ptr(perm), variant, _ptr(out),
-                                      _stream(stream)))
+                                      _stream(stream, X)))
     return out
 
 
@@ -343,5 +356,6 @@ def kvq_debug_quantize_f32(Xrot, stream=None):
     codes = torch.empty((N, 32), dtype=torch.uint8, device=Xrot.device)
     meta = torch.empty((N, 4, 2), dtype=torch.int16, device=Xrot.device)
     _check("kvq_debug_quantize_f32",
-           lib().kvq_debug_quantize_f32(_ptr(Xrot), N, _ptr(codes), _ptr(meta), _stream(stream)))
+           lib().kvq_debug_quantize_f32(_ptr(Xrot), N, _ptr(codes), _ptr(meta),
+                                        _stream(stream, Xrot)))
     return codes, meta
