@@ -17,8 +17,10 @@
  *     kernel itself is unchanged.
  *   - "RotateKV: Accurate and Robust 2-Bit KV Cache Quantization ..."
  *     abstract, item (i): the rotation is a channel reordering followed by a
- *     fast Walsh-Hadamard transform; item (iii): attention sinks are
- *     protected from 2-bit quantization.
+ *     fast Walsh-Hadamard transform; item (ii): that rotation applied to the
+ *     keys before RoPE and across a group of heads; item (iii): attention
+ *     sinks, singled out by massive activations, are protected from 2-bit
+ *     quantization.
  *   - "KVLinC : KV Cache Quantization with Hadamard Rotation and Linear
  *     Correction", abstract: a Hadamard rotation of the values.
  * The pages fix the 2-bit width only.  The group of 32 along head_dim, the
@@ -539,4 +541,171 @@ void orc_f32_to_f16_array(const float *x, int64_t n, uint16_t *out) {
 
 void orc_f16_to_f32_array(const uint16_t *x, int64_t n, float *out) {
     for (int64_t i = 0; i < n; i++) out[i] = orc_f16_to_f32(x[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Pre-RoPE grouped-head rotation (RotateKV abstract, item (ii)).             */
+/* ------------------------------------------------------------------------ */
+/* Keys are rotated before RoPE, and one rotation spans the keys of a group
+ * of gh consecutive KV heads: the concatenation x (n = 128*gh channels) is
+ * reordered, y[i] = x[perm[i]] (perm a permutation of 0..n-1), and
+ * x_rot = FWHT_n(y)/sqrt(n).  Each head's 128-channel slice of x_rot is
+ * quantized and stored in that head's cache unit.  At decode time the key
+ * of position t is the inverse rotation of the dequantised group row, then
+ * RoPE at position t.  Values are rotated per head, as in FWHT mode.
+ *
+ * RoPE (rotate-half pairing): channel c < 64 pairs with c + 64, with
+ * frequency theta_c = base^(-2c/128) and angle t * theta_c:
+ *   out[c]      = x[c] cos(a) - x[c+64] sin(a)
+ *   out[c + 64] = x[c+64] cos(a) + x[c] sin(a). */
+
+void orc_rope_f64(double *x, int64_t t, double base) {
+    for (int c = 0; c < D / 2; c++) {
+        const double th = pow(base, -2.0 * (double)c / (double)D);
+        const double a = (double)t * th;
+        const double cs = cos(a), sn = sin(a);
+        const double x0 = x[c], x1 = x[c + D / 2];
+        x[c] = x0 * cs - x1 * sn;
+        x[c + D / 2] = x1 * cs + x0 * sn;
+    }
+}
+
+/* x (n channels) -> FWHT_n(x[perm]) / sqrt(n). */
+void orc_rotate_group_f64(const double *x, int n, const int32_t *perm, double *out) {
+    for (int i = 0; i < n; i++) out[i] = x[perm[i]];
+    orc_fwht_f64(out, n);
+    const double sc = 1.0 / sqrt((double)n);
+    for (int i = 0; i < n; i++) out[i] *= sc;
+}
+
+/* The inverse: y = FWHT_n(o) / sqrt(n), out[perm[i]] = y[i]. */
+void orc_unrotate_group_f64(const double *o, int n, const int32_t *perm, double *out) {
+    double *y = (double *)malloc(sizeof(double) * (size_t)n);
+    for (int i = 0; i < n; i++) y[i] = o[i];
+    orc_fwht_f64(y, n);
+    const double sc = 1.0 / sqrt((double)n);
+    for (int i = 0; i < n; i++) out[perm[i]] = y[i] * sc;
+    free(y);
+}
+
+/* Pre-RoPE append.  K (pre-RoPE), V: fp16 [B][T][Hkv][128]; gh divides Hkv;
+ * perm int32 [2][Hkv*128]: plane 0 holds Hkv/gh key permutations of n =
+ * 128*gh entries each (group q at perm + q*n), plane 1 one value permutation
+ * of 128 entries per head.  No sinks.  Returns the status bits; seq_lens
+ * advance by T for every sequence that fits. */
+int orc_append_prerope(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int gh,
+                       const int32_t *perm, int capacity, uint8_t *blocks, int32_t *seq_lens) {
+    int status = 0;
+    const int nblk = capacity / BLK_TOK;
+    const int n = D * gh;
+    double *xg = (double *)malloc(sizeof(double) * (size_t)n);
+    double *xr = (double *)malloc(sizeof(double) * (size_t)n);
+    for (int b = 0; b < B; b++) {
+        const int L0 = seq_lens[b];
+        if (L0 < 0 || (int64_t)L0 + T > capacity) {
+            status |= (L0 < 0) ? ST_BAD_LEN : ST_CAPACITY;
+            continue;
+        }
+        for (int t = 0; t < T; t++) {
+            const int p = L0 + t;
+            for (int q = 0; q < Hkv / gh; q++) {
+                for (int j = 0; j < gh; j++)
+                    for (int i = 0; i < D; i++)
+                        xg[j * D + i] = (double)orc_f16_to_f32(
+                            K[(((size_t)b * T + t) * Hkv + q * gh + j) * D + i]);
+                orc_rotate_group_f64(xg, n, perm + (size_t)q * n, xr);
+                for (int j = 0; j < gh; j++) {
+                    const int h = q * gh + j;
+                    float kr[D], vr[D];
+                    for (int i = 0; i < D; i++) kr[i] = (float)xr[j * D + i];
+                    orc_rotate_rows_f32(V + (((size_t)b * T + t) * Hkv + h) * D, 1, 1, NULL,
+                                        perm + ((size_t)Hkv + h) * D, vr);
+                    uint8_t kc[D], vc[D], kb[32], vb[32];
+                    uint16_t ks[NG], kz[NG], vs[NG], vz[NG];
+                    orc_quantize_row(kr, kc, ks, kz);
+                    orc_quantize_row(vr, vc, vs, vz);
+                    orc_pack_row(kc, kb);
+                    orc_pack_row(vc, vb);
+                    uint8_t *block =
+                        blocks + (((size_t)b * Hkv + h) * nblk + p / BLK_TOK) * BLK_BYTES;
+                    orc_store_token(block, p % BLK_TOK, kb, vb, ks, kz, vs, vz);
+                }
+            }
+        }
+        seq_lens[b] = L0 + T;
+    }
+    free(xg);
+    free(xr);
+    return status;
+}
+
+/* Pre-RoPE decode.  Q: fp16 [B][Hq][128] post-RoPE queries (query head hq
+ * reads KV head hq / G).  For every position t < L: the dequantised rotated
+ * key rows of the gh heads of the group, inversely rotated, the head's slice
+ * taken and RoPE'd at position t; s_t = q . k_t / sqrt(128); softmax; the
+ * values as in FWHT mode: o_rot = sum p_t v_t, out = FWHT(o_rot)/sqrt(128)
+ * scattered through the head's value permutation.  Output fp64 [B][Hq][128];
+ * invalid lengths give zeros and ST_BAD_LEN. */
+int orc_decode_prerope(const uint16_t *Q, int B, int Hq, int Hkv, int gh, const int32_t *perm,
+                       double rope_base, int capacity, const uint8_t *blocks,
+                       const int32_t *seq_lens, int only_b, int only_h, int n_threads,
+                       double *out) {
+    int status = 0;
+    const int G = Hq / Hkv;
+    const int nblk = capacity / BLK_TOK;
+    const int n = D * gh;
+    for (int b = 0; b < B; b++) {
+        const int L = seq_lens[b];
+        if ((only_b < 0 || b == only_b) && (L < 1 || L > capacity)) status |= ST_BAD_LEN;
+    }
+    const int64_t npairs = (int64_t)B * Hq;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int64_t bh = 0; bh < npairs; bh++) {
+        const int b = (int)(bh / Hq), hq = (int)(bh % Hq), h = hq / G;
+        const int q = h / gh, j = h % gh;
+        if (only_b >= 0 && b != only_b) continue;
+        if (only_h >= 0 && h != only_h) continue;
+        double *o = out + (size_t)bh * D;
+        const int L = seq_lens[b];
+        if (L < 1 || L > capacity) {
+            for (int i = 0; i < D; i++) o[i] = 0.0;
+            continue;
+        }
+        double qv[D], k[D], v[D], orot[D];
+        for (int i = 0; i < D; i++) qv[i] = (double)orc_f16_to_f32(Q[(size_t)bh * D + i]);
+        double *kg = (double *)malloc(sizeof(double) * (size_t)n);
+        double *ku = (double *)malloc(sizeof(double) * (size_t)n);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L);
+        const double scale = 1.0 / sqrt((double)D);
+        double m = -INFINITY;
+        for (int t = 0; t < L; t++) {
+            for (int jj = 0; jj < gh; jj++) {
+                const size_t u = (size_t)b * Hkv + q * gh + jj;
+                dequant_token(blocks + u * (size_t)nblk * BLK_BYTES, NULL, NULL, -1, t, k, v);
+                for (int i = 0; i < D; i++) kg[jj * D + i] = k[i];
+            }
+            orc_unrotate_group_f64(kg, n, perm + (size_t)q * n, ku);
+            for (int i = 0; i < D; i++) k[i] = ku[j * D + i];
+            orc_rope_f64(k, t, rope_base);
+            double acc = 0.0;
+            for (int i = 0; i < D; i++) acc += qv[i] * k[i];
+            s[t] = acc * scale;
+            if (s[t] > m) m = s[t];
+        }
+        double l = 0.0;
+        for (int i = 0; i < D; i++) orot[i] = 0.0;
+        const size_t uh = (size_t)b * Hkv + h;
+        for (int t = 0; t < L; t++) {
+            const double p = exp(s[t] - m);
+            l += p;
+            dequant_token(blocks + uh * (size_t)nblk * BLK_BYTES, NULL, NULL, -1, t, k, v);
+            for (int i = 0; i < D; i++) orot[i] += p * v[i];
+        }
+        for (int i = 0; i < D; i++) orot[i] /= l;
+        unrotate_f64(orot, 1, NULL, perm + ((size_t)Hkv + h) * D, o);
+        free(kg);
+        free(ku);
+        free(s);
+    }
+    return status;
 }

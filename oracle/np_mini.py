@@ -81,3 +81,40 @@ def decode_one(q_f16, khat, vhat, mode, Rk=None, Rv=None, pk=None, pv=None):
     p = np.exp(s - s.max())
     o = (p / p.sum()) @ vhat
     return o @ Mv.T
+
+
+# --- pre-RoPE grouped-head rotation ------------------------------------------------------
+
+def group_rotation_matrix(perm):
+    """x_rot = x @ M for a group row of n = len(perm) channels:
+    y[i] = x[perm[i]], x_rot = y @ H_n / sqrt(n)."""
+    n = len(perm)
+    M = np.zeros((n, n))
+    M[np.asarray(perm), :] = hadamard(n) / np.sqrt(n)
+    return M
+
+
+def rope_complex(x, t, base):
+    """RoPE with rotate-half pairing as a complex rotation: channel c < 64
+    and c + 64 are the real and imaginary parts of z_c, turned by t*theta_c,
+    theta_c = base^(-2c/128)."""
+    x = np.asarray(x, np.float64)
+    z = x[:D // 2] + 1j * x[D // 2:]
+    theta = np.power(float(base), -2.0 * np.arange(D // 2) / D)
+    z = z * np.exp(1j * t * theta)
+    return np.concatenate([z.real, z.imag])
+
+
+def decode_prerope_one(q_f16, kgroup_hat, j, perm_group, base, vhat, pv):
+    """q fp16 [128] post-RoPE; kgroup_hat fp64 [L, n] rotated group key rows
+    (dequantised); j the head's slot in its group; vhat fp64 [L,128] rotated
+    value rows; pv the head's value permutation."""
+    q = np.asarray(q_f16, np.float16).astype(np.float64)
+    M = group_rotation_matrix(perm_group)
+    kpre = kgroup_hat @ M.T                        # inverse of an orthogonal map
+    k = np.stack([rope_complex(kpre[t, j * D:(j + 1) * D], t, base)
+                  for t in range(kpre.shape[0])])
+    s = k @ q / np.sqrt(D)
+    p = np.exp(s - s.max())
+    o = (p / p.sum()) @ vhat
+    return o @ rotation_matrix(1, perm=pv).T

@@ -52,6 +52,13 @@ def lib():
         L.orc_decode.argtypes = [p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, p, p, ci, ci,
                                  ci, p]
         L.orc_attention_f64.argtypes = [p, p, p, ci, p]
+        L.orc_rope_f64.argtypes = [p, i64, C.c_double]
+        L.orc_rotate_group_f64.argtypes = [p, ci, p, p]
+        L.orc_unrotate_group_f64.argtypes = [p, ci, p, p]
+        L.orc_append_prerope.restype = ci
+        L.orc_append_prerope.argtypes = [p, p, ci, ci, ci, ci, p, ci, p, p]
+        L.orc_decode_prerope.restype = ci
+        L.orc_decode_prerope.argtypes = [p, ci, ci, ci, ci, p, C.c_double, ci, p, p, ci, ci, ci, p]
         _lib = L
     return _lib
 
@@ -235,3 +242,58 @@ def attention_f64(q, K, V):
     out = np.empty(D, np.float64)
     lib().orc_attention_f64(_p(q), _p(K), _p(V), K.shape[0], _p(out))
     return out
+
+
+# --- pre-RoPE grouped-head rotation (keys rotated before RoPE, across gh heads) ----------
+
+def rope_f64(x, t, base):
+    """RoPE (rotate-half pairing) of one fp64 row x [128] at position t."""
+    x = _c(x, np.float64).copy()
+    lib().orc_rope_f64(_p(x), int(t), float(base))
+    return x
+
+
+def rotate_group_f64(x, perm):
+    """x [n] -> FWHT_n(x[perm]) / sqrt(n)."""
+    x = _c(x, np.float64)
+    pc = _c(perm, np.int32)
+    out = np.empty_like(x)
+    lib().orc_rotate_group_f64(_p(x), x.size, _p(pc), _p(out))
+    return out
+
+
+def unrotate_group_f64(o, perm):
+    o = _c(o, np.float64)
+    pc = _c(perm, np.int32)
+    out = np.empty_like(o)
+    lib().orc_unrotate_group_f64(_p(o), o.size, _p(pc), _p(out))
+    return out
+
+
+def append_prerope(cache, K, V, gh, perm, seq_lens):
+    """K (pre-RoPE), V: fp16 bit patterns [B][T][Hkv][128]; perm int32
+    [2][Hkv*128] (plane 0: Hkv/gh key permutations of 128*gh entries; plane 1:
+    one value permutation of 128 per head).  Needs a cache without sinks."""
+    assert cache.S == 0
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    B, T, Hkv, d = K.shape
+    assert d == D and B == cache.B and Hkv == cache.Hkv and V.shape == K.shape and Hkv % gh == 0
+    assert seq_lens.dtype == np.int32 and seq_lens.flags.c_contiguous
+    pc = _c(perm, np.int32).reshape(2, Hkv * D)
+    return lib().orc_append_prerope(_p(K), _p(V), B, T, Hkv, gh, _p(pc), cache.capacity,
+                                    _p(cache.blocks), _p(seq_lens))
+
+
+def decode_prerope(cache, Q, gh, perm, rope_base, seq_lens, only_b=-1, only_h=-1, n_threads=1):
+    """Q: fp16 bit patterns [B][Hq][128] (post-RoPE).  Returns (out fp64, status)."""
+    Q = _c(Q, np.uint16)
+    B, Hq, d = Q.shape
+    assert d == D and B == cache.B and Hq % cache.Hkv == 0 and cache.S == 0
+    pc = _c(perm, np.int32).reshape(2, cache.Hkv * D)
+    sl = _c(seq_lens, np.int32)
+    out = np.zeros((B, Hq, D), np.float64)
+    st = lib().orc_decode_prerope(_p(Q), B, Hq, cache.Hkv, gh, _p(pc), float(rope_base),
+                                  cache.capacity, _p(cache.blocks), _p(sl), only_b, only_h,
+                                  n_threads, _p(out))
+    return out, st

@@ -567,3 +567,99 @@ def test_identify_sinks_threshold_order_and_skips():
     orc.identify_sinks(cache2, np.array([[0, 7, 0]], np.float32), 5.0, np.array([0], np.int32))
     orc.identify_sinks(cache2, np.array([[7, 7, 7]], np.float32), 5.0, np.array([3], np.int32))
     assert cache2.sink_count[0] == 3 and list(cache2.sink_pos[0]) == [1, 3, 4]
+
+
+# --- pre-RoPE grouped-head rotation (RotateKV abstract, item (ii)) ----------------------------
+
+@pytest.mark.parametrize("base", [10000.0, 500000.0])
+def test_rope_is_the_complex_rotation(base):
+    """RoPE against an independent complex-exponential formulation, plus two
+    facts of any rotary embedding: it keeps norms, and q.k after RoPE at
+    positions p and t depends on p - t only."""
+    rng = np.random.default_rng(50)
+    for t in (0, 1, 7, 4095, 131071):
+        x = rng.standard_normal(D)
+        got = orc.rope_f64(x, t, base)
+        # theta_c from two pow() implementations may differ in the last bit,
+        # which the angle t*theta_c scales by t
+        assert np.allclose(got, np_mini.rope_complex(x, t, base), rtol=0, atol=1e-13 * (1 + t))
+        assert abs(np.linalg.norm(got) - np.linalg.norm(x)) < 1e-12
+    q, k = rng.standard_normal(D), rng.standard_normal(D)
+    for p, t in ((10, 3), (5000, 4990), (70000, 12)):
+        lhs = orc.rope_f64(q, p, base) @ orc.rope_f64(k, t, base)
+        assert abs(lhs - orc.rope_f64(q, p - t, base) @ k) < 1e-9
+    # a pair is turned by exactly t*theta_c: channel 0 pairs with channel 64 at theta_0 = 1
+    e0 = np.zeros(D)
+    e0[0] = 1.0
+    r = orc.rope_f64(e0, 3, base)
+    assert abs(r[0] - np.cos(3.0)) < 1e-15 and abs(r[64] - np.sin(3.0)) < 1e-15
+    assert np.count_nonzero(r) == 2
+
+
+@pytest.mark.parametrize("gh", [1, 2, 4, 8])
+def test_group_rotation_is_the_permuted_hadamard_matrix(gh):
+    n = D * gh
+    rng = np.random.default_rng(51 + gh)
+    perm = rng.permutation(n).astype(np.int32)
+    x = rng.standard_normal(n)
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    exp = H @ x[perm] / np.sqrt(n)
+    got = orc.rotate_group_f64(x, perm)
+    assert np.allclose(got, exp, rtol=0, atol=1e-12)
+    assert np.allclose(orc.unrotate_group_f64(got, perm), x, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("gh,G", [(1, 1), (2, 2), (4, 1)])
+def test_prerope_c_oracle_matches_numpy_mini_oracle(gh, G):
+    """Append (pre-RoPE keys rotated per group of gh heads, values per head)
+    and decode against the independent numpy oracle: codes and metadata
+    bit-exact on the same rotated fp32 rows, outputs within 1e-12."""
+    rng = np.random.default_rng(60 + gh + G)
+    B, T, Hkv, base = 2, 41, 4, 10000.0
+    Hq = Hkv * G
+    n = D * gh
+    K = (rng.standard_normal((B, T, Hkv, D)) * 3).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    perm = np.concatenate([np.concatenate([rng.permutation(n) for _ in range(Hkv // gh)]),
+                           np.concatenate([rng.permutation(D) for _ in range(Hkv)])]
+                          ).astype(np.int32).reshape(2, Hkv * D)
+    cache = orc.Cache(B, Hkv, 48, 0)
+    L0 = [0, 5]
+    sl = np.array(L0, np.int32)
+    assert orc.append_prerope(cache, K.view(np.uint16), V.view(np.uint16), gh, perm, sl) == 0
+    assert list(sl) == [T, 5 + T]
+    Q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    out, st = orc.decode_prerope(cache, Q.view(np.uint16), gh, perm, base, sl)
+    assert st == 0
+    for b in range(B):
+        for q in range(Hkv // gh):
+            pg = perm[0, q * n:(q + 1) * n]
+            # rotated fp32 group rows of every appended token, numpy and C
+            xg = K[b, :, q * gh:(q + 1) * gh].astype(np.float64).reshape(T, n)
+            rot_n = (xg @ np_mini.group_rotation_matrix(pg)).astype(np.float32)
+            rot_c = np.stack([orc.rotate_group_f64(xg[t], pg) for t in range(T)]).astype(np.float32)
+            assert np.max(np.abs(rot_c - rot_n) / (np.abs(rot_n) + 1e-3)) < 1e-6
+            khat = np.zeros((L0[b] + T, n))        # never-written positions decode to 0
+            for jj in range(gh):
+                h = q * gh + jj
+                codes, s, z = np_mini.quantize_rows(rot_c[:, jj * D:(jj + 1) * D])
+                vr = np_mini.rotate_rows_f32(V[b, :, h], 1, perm=perm[1, h * D:(h + 1) * D])
+                vcodes = np_mini.quantize_rows(vr)[0]
+                for t in range(T):
+                    p = L0[b] + t
+                    kb, vb, ks, kz, _, _ = orc.load_token(cache.blocks[b, h, p // 16], p % 16)
+                    assert np.array_equal(orc.unpack_row(kb), codes[t])
+                    assert np.array_equal(ks, s[t]) and np.array_equal(kz, z[t])
+                    assert np.array_equal(orc.unpack_row(vb), vcodes[t])
+                    khat[p, jj * D:(jj + 1) * D] = np_mini.dequant(codes[t], s[t], z[t])
+            for jj in range(gh):
+                h = q * gh + jj
+                vhat = np.zeros((L0[b] + T, D))
+                vr = np_mini.rotate_rows_f32(V[b, :, h], 1, perm=perm[1, h * D:(h + 1) * D])
+                vcodes, vs, vz = np_mini.quantize_rows(vr)
+                for t in range(T):
+                    vhat[L0[b] + t] = np_mini.dequant(vcodes[t], vs[t], vz[t])
+                for hq in range(h * G, (h + 1) * G):
+                    ref = np_mini.decode_prerope_one(Q[b, hq], khat, jj, pg, base, vhat,
+                                                     perm[1, h * D:(h + 1) * D])
+                    assert np.allclose(out[b, hq], ref, rtol=0, atol=1e-12)
