@@ -325,6 +325,52 @@ KVQ_API kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_
                                    int32_t sink_fp16, int32_t max_ctx, void *workspace,
                                    size_t ws_bytes, uint16_t *out, void *stream);
 
+/*
+ * Pre-RoPE grouped-head key rotation (RotateKV abstract, item (ii): the
+ * outlier-aware rotation applied to the keys before RoPE and across heads).
+ * The keys of group_heads (gh) consecutive KV heads form one row of
+ * n = 128*gh channels, which is reordered and Hadamard-transformed:
+ *   x_rot = FWHT_n(x[perm_group]) / sqrt(n),
+ * and head j of the group stores channels 128j .. 128j+127 of x_rot in its
+ * cache unit (the same block format).  Values are rotated per head as in
+ * KVQ_ROT_PERM_FWHT.  RoPE is the rotate-half form: channel c < 64 pairs with
+ * c + 64 and turns by t * base^(-2c/128) at position t (0-based).
+ *   perm   int32 [2][Hkv*128]: plane 0 holds the Hkv/gh key permutations of n
+ *          entries (group q at perm + q*n, each a permutation of 0..n-1),
+ *          plane 1 one value permutation of 0..127 per head (at
+ *          perm + Hkv*128 + h*128).  16-B aligned.
+ *   gh     1, 2, 4 or 8, dividing Hkv.
+ * The cache must have no fp16 sinks (sink_fp16 == 0); paged caches are fine.
+ */
+/* Append T tokens: K fp16 [B][T][Hkv][128] PRE-RoPE keys, V fp16 values
+ * (same layout), 16-B aligned; seq_lens as in kvq_rotate_quantize_append. */
+KVQ_API kvq_status kvq_prerope_append(const uint16_t *K, const uint16_t *V, int32_t T,
+                                      int32_t group_heads, const int32_t *perm,
+                                      const kvq_cache_desc *cache, int32_t *seq_lens,
+                                      void *stream);
+/* Workspace bytes of kvq_prerope_decode for these sizes (0 on bad arguments). */
+KVQ_API size_t kvq_prerope_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
+                                          int32_t group_heads, int32_t max_ctx,
+                                          int32_t sm_count);
+/* Decode one query per query head over a pre-RoPE cache.
+ *   Q     fp16 [B][Hq][128] POST-RoPE queries (the model's own q at the new
+ *         position); query head hq reads KV head hq / (Hq/Hkv).
+ *   (Hq/Hkv) * group_heads <= 8.
+ * For every position t < seq_lens[b]: k_t = RoPE_t(head slice of the inverse
+ * group rotation of the dequantised keys), s_t = q . k_t / sqrt(128),
+ * softmax, o_rot = sum p_t v_t over the rotated values, out = o_rot rotated
+ * back (FWHT + value permutation).  Other arguments and errors as
+ * kvq_decode_attention; KVQ_ERR_UNSUPPORTED for a cache with sinks or a
+ * shape outside the limits above. */
+KVQ_API kvq_status kvq_prerope_decode(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                      int32_t group_heads, const int32_t *perm, float rope_base,
+                                      const int32_t *seq_lens, int32_t max_ctx, void *workspace,
+                                      size_t ws_bytes, uint16_t *out, void *stream);
+/* Test export: the pre-RoPE append's key rotation with fp32 output.
+ * X fp16 [N][128*gh] group rows, perm int32 [128*gh] -> Xrot fp32 [N][128*gh]. */
+KVQ_API kvq_status kvq_debug_rotate_group_f32(const uint16_t *X, int32_t N, int32_t group_heads,
+                                              const int32_t *perm, float *Xrot, void *stream);
+
 /* Short text for a status code (static storage). */
 KVQ_API const char *kvq_status_string(kvq_status s);
 

@@ -12,7 +12,8 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_decode_attention, kvq_decode_attention_ex, kvq_decode_attention_noalloc,
                   kvq_decode_attention_timed,
                   kvq_decode_workspace_size, kvq_get_status, kvq_identify_sinks,
-                  kvq_rotate_quantize_append, lib)
+                  kvq_rotate_quantize_append, lib, kvq_prerope_append, kvq_prerope_decode,
+                  kvq_prerope_workspace_size, prerope_workspace, kvq_debug_rotate_group_f32)
 
 __all__ = [
     "KVCache", "PagedKVCache", "KvqError", "KVQ_DEV_BAD_TABLE", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
@@ -22,5 +23,6 @@ __all__ = [
     "kvq_decode_attention", "kvq_decode_attention_ex", "kvq_decode_attention_noalloc",
     "kvq_decode_attention_timed",
     "kvq_decode_workspace_size", "kvq_get_status", "kvq_identify_sinks",
-    "kvq_rotate_quantize_append", "lib",
+    "kvq_rotate_quantize_append", "lib", "kvq_prerope_append", "kvq_prerope_decode",
+    "kvq_prerope_workspace_size", "prerope_workspace", "kvq_debug_rotate_group_f32",
 ]

@@ -118,6 +118,74 @@ kvq_status kvq_identify_sinks(const float *act, int32_t T, float tau, const kvq_
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+static bool gh_ok(int gh, int Hkv) {
+    return (gh == 1 || gh == 2 || gh == 4 || gh == 8) && Hkv % gh == 0;
+}
+
+kvq_status kvq_prerope_append(const uint16_t *K, const uint16_t *V, int32_t T, int32_t group_heads,
+                              const int32_t *perm, const kvq_cache_desc *cache, int32_t *seq_lens,
+                              void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if (cache->sink_fp16 != 0 || cache->sink_pos) return KVQ_ERR_UNSUPPORTED;
+    if (!gh_ok(group_heads, cache->Hkv)) return KVQ_ERR_UNSUPPORTED;
+    if (!perm || T < 0 || !seq_lens || !aligned(seq_lens, 4)) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(perm, 16)) return KVQ_ERR_UNSUPPORTED;
+    if (T == 0) return KVQ_OK;
+    if (!K || !V) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16)) return KVQ_ERR_UNSUPPORTED;
+    if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    const cudaError_t e = launch_append_prerope(K, V, T, group_heads, perm, *cache, seq_lens,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+size_t kvq_prerope_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t group_heads,
+                                  int32_t max_ctx, int32_t sm_count) {
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_ctx < 1 || sm_count < 1) return 0;
+    if (!gh_ok(group_heads, Hkv)) return 0;
+    return prerope_ws_bytes(B, Hq, Hkv, group_heads, max_ctx, sm_count);
+}
+
+kvq_status kvq_prerope_decode(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                              int32_t group_heads, const int32_t *perm, float rope_base,
+                              const int32_t *seq_lens, int32_t max_ctx, void *workspace,
+                              size_t ws_bytes, uint16_t *out, void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if (cache->sink_fp16 != 0 || cache->sink_pos) return KVQ_ERR_UNSUPPORTED;
+    if (!gh_ok(group_heads, cache->Hkv)) return KVQ_ERR_UNSUPPORTED;
+    if (!Q || !out || !seq_lens || !workspace || !perm) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        !aligned(seq_lens, 4) || !aligned(perm, 16))
+        return KVQ_ERR_UNSUPPORTED;
+    if (Hq < cache->Hkv || Hq % cache->Hkv != 0 || Hq > 65535) return KVQ_ERR_INVALID_ARG;
+    const int G = Hq / cache->Hkv;
+    if ((G != 1 && G != 2 && G != 4 && G != 8) || G * group_heads > 8) return KVQ_ERR_UNSUPPORTED;
+    if (!(rope_base > 1.0f) || !(rope_base < 3.0e38f)) return KVQ_ERR_INVALID_ARG;
+    if (max_ctx < 1 || max_ctx > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    const int sms = device_sm_count();
+    if (sms < 1) return KVQ_ERR_CUDA;
+    if (ws_bytes < prerope_ws_bytes(cache->B, Hq, cache->Hkv, group_heads, max_ctx, sms))
+        return KVQ_ERR_WORKSPACE;
+    const cudaError_t e = launch_decode_prerope(Q, Hq, *cache, group_heads, perm, rope_base,
+                                                seq_lens, max_ctx, sms, workspace, out,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_debug_rotate_group_f32(const uint16_t *X, int32_t N, int32_t group_heads,
+                                      const int32_t *perm, float *Xrot, void *stream) {
+    if (!X || !Xrot || !perm || N < 0) return KVQ_ERR_INVALID_ARG;
+    if (group_heads != 1 && group_heads != 2 && group_heads != 4 && group_heads != 8)
+        return KVQ_ERR_UNSUPPORTED;
+    if (!aligned(X, 16) || !aligned(Xrot, 16) || !aligned(perm, 16)) return KVQ_ERR_UNSUPPORTED;
+    if (N == 0) return KVQ_OK;
+    const cudaError_t e = launch_debug_rotate_group(X, N, group_heads, perm, Xrot,
+                                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max_ctx,
                                  int32_t sm_count) {
     if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || max_ctx < 1 || sm_count < 1) return 0;

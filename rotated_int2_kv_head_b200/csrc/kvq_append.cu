@@ -237,6 +237,165 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
     if (TO_CACHE) append_done(c);
 }
 
+// ---- pre-RoPE grouped-head key rotation ----------------------------------------------------------
+// "RotateKV", abstract item (ii): the keys are rotated before RoPE, by one
+// rotation across a group of GH consecutive KV heads.  The group's pre-RoPE
+// keys (n = 128*GH channels, contiguous in K) are reordered by the group's
+// permutation and transformed by an n-point FWHT / sqrt(n); each head's
+// 128-channel slice is quantized into its own cache unit.  Values are
+// rotated per head as in FWHT mode.  One warp per row: rows [0, nk) are key
+// groups (b, t, group), rows [nk, nk + nv) value rows (b, t, h).  Lane l
+// holds the group elements j*128 + 4l + k (j < GH, k < 4): the FWHT stages
+// over k and l are fwht128_warp's, the ones over j run in registers (the
+// Sylvester transform is a product of commuting butterfly stages, one per
+// index bit, so their order does not matter).
+struct PreRopeRows {
+    const uint16_t *K, *V;     // cache: [B][T][Hkv][128]; debug: K = X [N][128*GH]
+    const int32_t *perm;       // cache: [2][Hkv*128] (plane 0 key groups, plane 1 value
+                               // heads); debug: one group permutation [128*GH]
+    float *out_f32;            // debug output [N][128*GH] or nullptr
+    long long nk, nv;          // cache: B*T*(Hkv/GH) key-group rows, B*T*Hkv value rows
+};
+
+template <int GH>
+__device__ __forceinline__ float inv_sqrt_group() {
+    return GH == 1 ? 0.08838834764831845f
+                   : (GH == 2 ? 0.0625f : (GH == 4 ? 0.04419417382415922f : 0.03125f));
+}
+
+template <int GH, bool TO_CACHE>
+__global__ void __launch_bounds__(FWHT_THREADS) append_prerope_kernel(PreRopeRows a, CacheDst c) {
+    constexpr int n = GH * D;
+    __shared__ __align__(16) uint16_t xs[FWHT_THREADS / 32][n];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
+    const long long row = (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
+    if (row < a.nk + a.nv) {
+        const bool key = row < a.nk;
+        int b = 0, t = 0, hh = 0, L0 = 0;
+        if (TO_CACHE) {
+            const int nper = key ? c.Hkv / GH : c.Hkv;     // groups (keys) or heads (values)
+            long long r2 = key ? row : row - a.nk;
+            hh = (int)(r2 % nper);
+            r2 /= nper;
+            t = (int)(r2 % c.T);
+            b = (int)(r2 / c.T);
+            L0 = start_len_thread(c, b, key && lane == 0 && t == 0 && hh == 0);
+        }
+        if (L0 >= 0 && key) {
+            const uint16_t *src = TO_CACHE
+                                      ? a.K + (((size_t)b * c.T + t) * c.Hkv + (size_t)hh * GH) * D
+                                      : a.K + (size_t)row * n;
+            const int32_t *pg = TO_CACHE ? a.perm + (size_t)hh * n : a.perm;
+#pragma unroll
+            for (int j = 0; j < GH; j++)
+                *reinterpret_cast<uint2 *>(&xs[warp][j * D + 4 * lane]) =
+                    *reinterpret_cast<const uint2 *>(src + j * D + 4 * lane);
+            __syncwarp();
+            float v[GH][4];
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                const int4 pi = *reinterpret_cast<const int4 *>(pg + j * D + 4 * lane);
+                v[j][0] = __half2float(__ushort_as_half(xs[warp][pi.x & (n - 1)]));
+                v[j][1] = __half2float(__ushort_as_half(xs[warp][pi.y & (n - 1)]));
+                v[j][2] = __half2float(__ushort_as_half(xs[warp][pi.z & (n - 1)]));
+                v[j][3] = __half2float(__ushort_as_half(xs[warp][pi.w & (n - 1)]));
+                fwht128_warp(v[j]);
+            }
+#pragma unroll
+            for (int st = 1; st < GH; st <<= 1)
+#pragma unroll
+                for (int j = 0; j < GH; j++)
+                    if ((j & st) == 0)
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const float x0 = v[j][k], x1 = v[j + st][k];
+                            v[j][k] = x0 + x1;
+                            v[j + st][k] = x0 - x1;
+                        }
+            const float sc = inv_sqrt_group<GH>();
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+#pragma unroll
+                for (int k = 0; k < 4; k++) v[j][k] *= sc;
+                if (TO_CACHE)
+                    cache_epilogue(c, b, t, hh * GH + j, 0, L0, v[j]);
+                else
+                    *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * n + j * D + 4 * lane) =
+                        make_float4(v[j][0], v[j][1], v[j][2], v[j][3]);
+            }
+        } else if (L0 >= 0 && TO_CACHE) {
+            // a value row: per-head permutation + 128-point FWHT
+            const uint16_t *src = a.V + (((size_t)b * c.T + t) * c.Hkv + hh) * D;
+            const int32_t *pv = a.perm + ((size_t)c.Hkv + hh) * D;
+            *reinterpret_cast<uint2 *>(&xs[warp][4 * lane]) =
+                *reinterpret_cast<const uint2 *>(src + 4 * lane);
+            const int4 pi = *reinterpret_cast<const int4 *>(pv + 4 * lane);
+            __syncwarp();
+            float v[4];
+            v[0] = __half2float(__ushort_as_half(xs[warp][pi.x & (D - 1)]));
+            v[1] = __half2float(__ushort_as_half(xs[warp][pi.y & (D - 1)]));
+            v[2] = __half2float(__ushort_as_half(xs[warp][pi.z & (D - 1)]));
+            v[3] = __half2float(__ushort_as_half(xs[warp][pi.w & (D - 1)]));
+            fwht128_warp(v);
+#pragma unroll
+            for (int k = 0; k < 4; k++) v[k] *= 0.08838834764831845f;
+            cache_epilogue(c, b, t, hh, 1, L0, v);
+        }
+    }
+    if (TO_CACHE) append_done(c);
+}
+
+template <int GH>
+static cudaError_t launch_prerope_t(const PreRopeRows &a, const CacheDst &c, bool to_cache,
+                                    cudaStream_t st) {
+    const long long rows = a.nk + a.nv;
+    const unsigned grid = (unsigned)((rows + FWHT_THREADS / 32 - 1) / (FWHT_THREADS / 32));
+    if (to_cache)
+        return launch_pdl(append_prerope_kernel<GH, true>, dim3(grid), dim3(FWHT_THREADS), 0, st,
+                          a, c);
+    append_prerope_kernel<GH, false><<<grid, FWHT_THREADS, 0, st>>>(a, c);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_prerope(int gh, const PreRopeRows &a, const CacheDst &c, bool to_cache,
+                                  cudaStream_t st) {
+    switch (gh) {
+        case 1: return launch_prerope_t<1>(a, c, to_cache, st);
+        case 2: return launch_prerope_t<2>(a, c, to_cache, st);
+        case 4: return launch_prerope_t<4>(a, c, to_cache, st);
+        case 8: return launch_prerope_t<8>(a, c, to_cache, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_append_prerope(const uint16_t *K, const uint16_t *V, int T, int gh,
+                                  const int32_t *perm, const kvq_cache_desc &cd,
+                                  int32_t *seq_lens, cudaStream_t st) {
+    const CacheDst c = cache_dst(cd, seq_lens, T);
+    PreRopeRows a;
+    a.K = K;
+    a.V = V;
+    a.perm = perm;
+    a.out_f32 = nullptr;
+    a.nk = (long long)cd.B * T * (cd.Hkv / gh);
+    a.nv = (long long)cd.B * T * cd.Hkv;
+    return launch_prerope(gh, a, c, true, st);
+}
+
+cudaError_t launch_debug_rotate_group(const uint16_t *X, int N, int gh, const int32_t *perm,
+                                     float *out, cudaStream_t st) {
+    CacheDst c{};
+    PreRopeRows a;
+    a.K = a.V = X;
+    a.perm = perm;
+    a.out_f32 = out;
+    a.nk = N;
+    a.nv = 0;
+    return launch_prerope(gh, a, c, false, st);
+}
+
 // ---- quantizer test export ---------------------------------------------------------------------
 __global__ void debug_quantize_kernel(const float *X, int N, uint8_t *codes, uint16_t *meta) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -288,6 +288,16 @@ cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_
                                   cudaStream_t st);
 cudaError_t launch_identify_sinks(const float *act, int T, float tau, const kvq_cache_desc &cd,
                                   const int32_t *seq_lens, cudaStream_t st);
+// pre-RoPE grouped-head key rotation (kvq_append.cu / kvq_prerope.cu)
+cudaError_t launch_append_prerope(const uint16_t *K, const uint16_t *V, int T, int gh,
+                                  const int32_t *perm, const kvq_cache_desc &cd,
+                                  int32_t *seq_lens, cudaStream_t st);
+cudaError_t launch_debug_rotate_group(const uint16_t *X, int N, int gh, const int32_t *perm,
+                                     float *out, cudaStream_t st);
+size_t prerope_ws_bytes(int B, int Hq, int Hkv, int gh, int max_ctx, int sms);
+cudaError_t launch_decode_prerope(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int gh,
+                                  const int32_t *perm, float rope_base, const int32_t *seq_lens,
+                                  int max_ctx, int sms, void *ws, uint16_t *out, cudaStream_t st);
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,

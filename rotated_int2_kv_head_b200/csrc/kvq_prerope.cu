@@ -1,0 +1,373 @@
+// Decode attention over a cache whose keys were rotated before RoPE, across
+// groups of GH consecutive KV heads ("RotateKV: Accurate and Robust 2-Bit KV
+// Cache Quantization for LLMs via Outlier-Aware Adaptive Rotations", abstract
+// item (ii)).  The cached key of position t is the quantized slice of
+// FWHT_n(k_group[perm]) / sqrt(n), n = 128*GH, so the attention key is
+//   k_t = RoPE_t( (FWHT_n(k_hat_group) / sqrt(n)) scattered through perm )
+// for the head's slice: every position needs its own inverse rotation and
+// its own RoPE angle, which no single query-side transform can absorb.  The
+// values are rotated per head as in FWHT mode and the rotation is removed
+// once, after the attention.
+//
+// Two kernels:
+//   prerope_split_kernel<GH, G>  grid (splits, B * Hkv/GH).  A CTA of 8 warps
+//       takes a contiguous range of 16-token cache blocks of one (b, group);
+//       warp w takes the range's blocks w, w+8, ... and their tokens in
+//       order.  Per token: the GH heads' K codes are dequantised (4 elements
+//       per lane), un-rotated by a warp FWHT (stages over the lane's 4
+//       elements and the 32 lanes by shuffles, stages across the GH heads in
+//       registers), scattered back through the permutation in shared memory,
+//       RoPE'd (the pair partner of channel c < 64 is c + 64, 16 lanes away)
+//       and dotted with each query head; online softmax and P.V on the
+//       dequantised rotated values.  Each CTA leaves one partial
+//       (m, l, o_rot[128]) per query head.
+//   prerope_merge_kernel  per (b, query head): merges the partials and
+//       removes the value rotation (FWHT + inverse permutation).
+// The RoPE angle t * theta_f is taken as 2 pi * frac(t * theta_f / (2 pi))
+// in fp64 at the start of every 16-token block (theta_f / (2 pi) comes from
+// the host in fp64), then advanced token by token with the rotation by
+// theta_f, so fp32 never holds an angle larger than 2 pi.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+constexpr int PR_WARPS = 8;
+constexpr int PR_THREADS = 32 * PR_WARPS;
+constexpr int PR_PART = 132;           // m, l, 0, 0, o[128]
+constexpr int PR_MIN_BLOCKS = 8;       // cache blocks per split at least
+constexpr float PR_LOG2E = 1.4426950408889634f;
+#define PR_NEG_INF (__int_as_float(0xff800000))
+
+struct PreRopeArgs {
+    const uint16_t *Q;          // [B][Hq][128] post-RoPE queries
+    const uint8_t *blocks;
+    const int32_t *table;       // paged cache, else null
+    int num_blocks;
+    const int32_t *perm;        // [2][Hkv*128]: key groups, then value heads
+    const int32_t *seq_lens;
+    int32_t *status;
+    float *part;                // [B*Hq][nsplit][PR_PART]
+    uint16_t *out;              // [B][Hq][128]
+    int B, Hq, Hkv, capacity, nblk, nsplit, bps;
+    double phi[D / 2];          // theta_f / (2 pi), theta_f = base^(-2f/128)
+};
+
+__host__ __device__ inline int pr_nsplit(int B, int ngroups, int max_ctx, int sms) {
+    const int nb = (max_ctx + BLK_TOK - 1) / BLK_TOK;
+    const int units = B * ngroups;
+    int want = (4 * sms + units - 1) / units;                 // about 4 CTAs per SM
+    const int most = (nb + PR_MIN_BLOCKS - 1) / PR_MIN_BLOCKS;
+    if (want > most) want = most;
+    return want < 1 ? 1 : want;
+}
+
+template <int GH, int G>
+__global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a) {
+    constexpr int n = GH * D;
+    constexpr int NQ = GH * G;                        // query heads of the group
+    __shared__ __align__(16) int32_t pg_s[n];         // the group's key permutation
+    // per warp: the un-rotation scatter (n floats), then the warp's o (NQ x 128)
+    __shared__ __align__(16) float kb_s[PR_WARPS][NQ * D];
+    __shared__ float m_s[PR_WARPS][NQ], l_s[PR_WARPS][NQ];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x;
+    const int ng = a.Hkv / GH;
+    const int b = blockIdx.y / ng, grp = blockIdx.y % ng;
+    const float isq = GH == 1 ? 0.08838834764831845f
+                              : (GH == 2 ? 0.0625f : (GH == 4 ? 0.04419417382415922f : 0.03125f));
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < n; i += PR_THREADS)
+        pg_s[i] = a.perm[(size_t)grp * n + i] & (n - 1);
+    const int L = a.seq_lens[b];
+    const bool lok = L >= 1 && L <= a.capacity;
+    const int nb = lok ? (L + BLK_TOK - 1) / BLK_TOK : 0;
+    const int blk0 = split * a.bps, blk1 = min(nb, blk0 + a.bps);
+
+    // queries of the group, in the exp2 domain with the 1/sqrt(128) scale
+    float qr[NQ][4];
+#pragma unroll
+    for (int i = 0; i < NQ; i++) {
+        const int hq = grp * NQ + i;       // = (grp*GH + j)*G + g
+        const uint2 u = *reinterpret_cast<const uint2 *>(a.Q + ((size_t)b * a.Hq + hq) * D + 4 * lane);
+        const float2 x01 = unpack_half2(u.x), x23 = unpack_half2(u.y);
+        const float sc = PR_LOG2E * 0.08838834764831845f;
+        qr[i][0] = x01.x * sc;
+        qr[i][1] = x01.y * sc;
+        qr[i][2] = x23.x * sc;
+        qr[i][3] = x23.y * sc;
+    }
+    // RoPE frequencies of the lane's 4 channels (f = (4 lane + k) mod 64):
+    // the per-token step rotation
+    float cst[4], snt[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const int f = 4 * (lane & 15) + k;
+        sincospif((float)(2.0 * a.phi[f]), &snt[k], &cst[k]);
+    }
+    const float psign = lane < 16 ? -1.f : 1.f;       // c < 64: x cos - x' sin
+
+    float m_run[NQ], l_run[NQ], o[NQ][4];
+#pragma unroll
+    for (int i = 0; i < NQ; i++) {
+        m_run[i] = PR_NEG_INF;
+        l_run[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; k++) o[i][k] = 0.f;
+    }
+    __syncthreads();                                  // pg_s
+
+    const int wi = lane & 7, g4 = lane >> 3;          // logical code word, quant group
+    for (int blk = blk0 + warp; blk < blk1; blk += PR_WARPS) {
+        // block addresses of the group's GH heads (and the V block of each)
+        const uint8_t *bp[GH];
+#pragma unroll
+        for (int j = 0; j < GH; j++) {
+            const long long bi = cache_block_index(a.table, a.num_blocks, a.nblk, a.Hkv, b,
+                                                   grp * GH + j, blk);
+            if (bi < 0 && lane == 0) set_status(a.status, KVQ_DEV_BAD_TABLE);
+            bp[j] = a.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
+        }
+        // RoPE angle of the block's first token, reduced in fp64
+        float cs[4], sn[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const double u = (double)(blk * BLK_TOK) * a.phi[4 * (lane & 15) + k];
+            const double fr = u - floor(u);
+            sincospif((float)(2.0 * fr), &sn[k], &cs[k]);
+        }
+        const int ntok = min(BLK_TOK, L - blk * BLK_TOK);
+        for (int tau = 0; tau < ntok; tau++) {
+            const int r = tau & 7, th = tau >> 3;
+            float v[GH][4];
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                    bp[j] + 16 * (4 * r + (wi & 3)) + 4 * (2 * th + (wi >> 2)));
+                const uint32_t mk =
+                    *reinterpret_cast<const uint32_t *>(bp[j] + 1024 + 8 * (4 * r + g4) + 4 * th);
+                const float2 sz = unpack_half2(mk);
+                const float s = sz.x * isq, z = sz.y * isq;
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    v[j][k] = fmaf((float)((w >> (8 * k + 2 * g4)) & 3u), s, z);
+                fwht128_warp(v[j]);
+            }
+#pragma unroll
+            for (int st = 1; st < GH; st <<= 1)
+#pragma unroll
+                for (int j = 0; j < GH; j++)
+                    if ((j & st) == 0)
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const float x0 = v[j][k], x1 = v[j + st][k];
+                            v[j][k] = x0 + x1;
+                            v[j + st][k] = x0 - x1;
+                        }
+            // k_pre[perm[i]] = y[i]: scatter, then read back in channel order
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                const int4 pi = *reinterpret_cast<const int4 *>(&pg_s[j * D + 4 * lane]);
+                kb_s[warp][pi.x] = v[j][0];
+                kb_s[warp][pi.y] = v[j][1];
+                kb_s[warp][pi.z] = v[j][2];
+                kb_s[warp][pi.w] = v[j][3];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                const float4 x = *reinterpret_cast<const float4 *>(&kb_s[warp][j * D + 4 * lane]);
+                v[j][0] = x.x;
+                v[j][1] = x.y;
+                v[j][2] = x.z;
+                v[j][3] = x.w;
+            }
+            __syncwarp();
+            // RoPE at position t: channel c < 64 with its partner c + 64
+#pragma unroll
+            for (int j = 0; j < GH; j++)
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const float px = __shfl_xor_sync(0xffffffffu, v[j][k], 16);
+                    v[j][k] = fmaf(psign * px, sn[k], v[j][k] * cs[k]);
+                }
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                // rotated values of head j at this token: pieces 2wi, 2wi+1
+                const int q2 = tau >> 1, side = tau & 1;
+                const uint8_t *vb = bp[j] + 512;
+                const int w0 = 2 * wi, w1 = 2 * wi + 1;
+                const uint32_t c0 = *reinterpret_cast<const uint16_t *>(
+                    vb + 16 * (4 * (w0 & 7) + (q2 & 3)) + 4 * (2 * (q2 >> 2) + (w0 >> 3)) + 2 * side);
+                const uint32_t c1 = *reinterpret_cast<const uint16_t *>(
+                    vb + 16 * (4 * (w1 & 7) + (q2 & 3)) + 4 * (2 * (q2 >> 2) + (w1 >> 3)) + 2 * side);
+                const uint32_t vw = c0 | (c1 << 16);
+                const uint32_t vmk =
+                    *reinterpret_cast<const uint32_t *>(bp[j] + 1280 + 8 * (4 * r + g4) + 4 * th);
+                const float2 vsz = unpack_half2(vmk);
+                float vv[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    vv[k] = fmaf((float)((vw >> (8 * k + 2 * g4)) & 3u), vsz.x, vsz.y);
+#pragma unroll
+                for (int g = 0; g < G; g++) {
+                    const int i = j * G + g;
+                    float d = qr[i][0] * v[j][0] + qr[i][1] * v[j][1] + qr[i][2] * v[j][2] +
+                              qr[i][3] * v[j][3];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                    if (d > m_run[i]) {
+                        const float al = exp2f(m_run[i] - d);   // 0 for the first token
+                        l_run[i] *= al;
+#pragma unroll
+                        for (int k = 0; k < 4; k++) o[i][k] *= al;
+                        m_run[i] = d;
+                    }
+                    const float p = exp2f(d - m_run[i]);
+                    l_run[i] += p;
+#pragma unroll
+                    for (int k = 0; k < 4; k++) o[i][k] = fmaf(p, vv[k], o[i][k]);
+                }
+            }
+            // next token: turn the RoPE angle by theta_f
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const float c2 = cs[k] * cst[k] - sn[k] * snt[k];
+                sn[k] = fmaf(sn[k], cst[k], cs[k] * snt[k]);
+                cs[k] = c2;
+            }
+        }
+    }
+
+    // combine the warps through kb_s, reused as [PR_WARPS][NQ][128]
+    __syncthreads();
+    float *ob = &kb_s[0][0];
+#pragma unroll
+    for (int i = 0; i < NQ; i++) {
+        *reinterpret_cast<float4 *>(&ob[((size_t)warp * NQ + i) * D + 4 * lane]) =
+            make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+        if (lane == 0) {
+            m_s[warp][i] = m_run[i];
+            l_s[warp][i] = l_run[i];
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < NQ * D; e += PR_THREADS) {
+        const int i = e / D, c = e % D;
+        float mx = PR_NEG_INF;
+#pragma unroll
+        for (int w = 0; w < PR_WARPS; w++) mx = fmaxf(mx, m_s[w][i]);
+        float lt = 0.f, ot = 0.f;
+        if (mx != PR_NEG_INF) {
+#pragma unroll
+            for (int w = 0; w < PR_WARPS; w++) {
+                if (m_s[w][i] == PR_NEG_INF) continue;        // a warp without tokens
+                const float f = exp2f(m_s[w][i] - mx);
+                lt = fmaf(f, l_s[w][i], lt);
+                ot = fmaf(f, ob[((size_t)w * NQ + i) * D + c], ot);
+            }
+        }
+        const int hq = grp * NQ + i;
+        float *pp = a.part + (((size_t)b * a.Hq + hq) * a.nsplit + split) * PR_PART;
+        pp[4 + c] = ot;
+        if (c == 0) {
+            pp[0] = mx;
+            pp[1] = lt;
+        }
+    }
+}
+
+// Merge of the splits and the inverse value rotation, one CTA of 128
+// threads per (b, query head).
+__global__ void __launch_bounds__(D) prerope_merge_kernel(PreRopeArgs a) {
+    __shared__ __align__(16) float os[D];
+    const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+    const int h = hq / (a.Hq / a.Hkv);
+    pdl_wait();
+    pdl_trigger();
+    const int L = a.seq_lens[b];
+    uint16_t *out = a.out + ((size_t)b * a.Hq + hq) * D;
+    if (L < 1 || L > a.capacity) {
+        out[t] = 0;
+        if (t == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
+        return;
+    }
+    const float *pp = a.part + ((size_t)b * a.Hq + hq) * a.nsplit * PR_PART;
+    float mx = PR_NEG_INF;
+    for (int s = 0; s < a.nsplit; s++) mx = fmaxf(mx, pp[(size_t)s * PR_PART]);
+    float lt = 0.f, ot = 0.f;
+    for (int s = 0; s < a.nsplit; s++) {
+        const float ms = pp[(size_t)s * PR_PART];
+        if (ms == PR_NEG_INF) continue;                     // a split without tokens
+        const float f = exp2f(ms - mx);
+        lt = fmaf(f, pp[(size_t)s * PR_PART + 1], lt);
+        ot = fmaf(f, pp[(size_t)s * PR_PART + 4 + t], ot);
+    }
+    os[t] = lt > 0.f ? ot / lt : 0.f;
+    __syncthreads();
+    if (t < 32) {
+        float v[4] = {os[4 * t], os[4 * t + 1], os[4 * t + 2], os[4 * t + 3]};
+        fwht128_warp(v);
+        const int4 pi = *reinterpret_cast<const int4 *>(a.perm + ((size_t)a.Hkv + h) * D + 4 * t);
+        out[pi.x & (D - 1)] = __half_as_ushort(__float2half_rn(v[0] * 0.08838834764831845f));
+        out[pi.y & (D - 1)] = __half_as_ushort(__float2half_rn(v[1] * 0.08838834764831845f));
+        out[pi.z & (D - 1)] = __half_as_ushort(__float2half_rn(v[2] * 0.08838834764831845f));
+        out[pi.w & (D - 1)] = __half_as_ushort(__float2half_rn(v[3] * 0.08838834764831845f));
+    }
+}
+
+size_t prerope_ws_bytes(int B, int Hq, int Hkv, int gh, int max_ctx, int sms) {
+    const int ns = pr_nsplit(B, Hkv / gh, max_ctx, sms);
+    return sizeof(float) * (size_t)B * Hq * ns * PR_PART;
+}
+
+template <int GH, int G>
+static cudaError_t launch_split_pr(const PreRopeArgs &a, cudaStream_t st) {
+    return launch_pdl(prerope_split_kernel<GH, G>, dim3(a.nsplit, a.B * (a.Hkv / GH)),
+                      dim3(PR_THREADS), 0, st, a);
+}
+
+cudaError_t launch_decode_prerope(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int gh,
+                                  const int32_t *perm, float rope_base, const int32_t *seq_lens,
+                                  int max_ctx, int sms, void *ws, uint16_t *out, cudaStream_t st) {
+    PreRopeArgs a;
+    a.Q = Q;
+    a.blocks = static_cast<const uint8_t *>(cd.blocks);
+    a.table = cd.block_table;
+    a.num_blocks = cd.num_blocks;
+    a.perm = perm;
+    a.seq_lens = seq_lens;
+    a.status = cd.status;
+    a.part = static_cast<float *>(ws);
+    a.out = out;
+    a.B = cd.B;
+    a.Hq = Hq;
+    a.Hkv = cd.Hkv;
+    a.capacity = cd.capacity;
+    a.nblk = cd.capacity / BLK_TOK;
+    a.nsplit = pr_nsplit(cd.B, cd.Hkv / gh, max_ctx, sms);
+    const int nb = (max_ctx + BLK_TOK - 1) / BLK_TOK;
+    a.bps = (nb + a.nsplit - 1) / a.nsplit;
+    // theta_f / (2 pi) in fp64: the kernel reduces t * theta_f modulo 2 pi
+    for (int f = 0; f < D / 2; f++)
+        a.phi[f] = pow((double)rope_base, -2.0 * f / D) / (2.0 * 3.14159265358979323846);
+    const int G = Hq / cd.Hkv;
+    cudaError_t e;
+    switch (gh * 16 + G) {
+        case 1 * 16 + 1: e = launch_split_pr<1, 1>(a, st); break;
+        case 1 * 16 + 2: e = launch_split_pr<1, 2>(a, st); break;
+        case 1 * 16 + 4: e = launch_split_pr<1, 4>(a, st); break;
+        case 1 * 16 + 8: e = launch_split_pr<1, 8>(a, st); break;
+        case 2 * 16 + 1: e = launch_split_pr<2, 1>(a, st); break;
+        case 2 * 16 + 2: e = launch_split_pr<2, 2>(a, st); break;
+        case 2 * 16 + 4: e = launch_split_pr<2, 4>(a, st); break;
+        case 4 * 16 + 1: e = launch_split_pr<4, 1>(a, st); break;
+        case 4 * 16 + 2: e = launch_split_pr<4, 2>(a, st); break;
+        case 8 * 16 + 1: e = launch_split_pr<8, 1>(a, st); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
+    return launch_pdl(prerope_merge_kernel, dim3(Hq, cd.B), dim3(D), 0, st, a);
+}
+
+}  // namespace kvq

@@ -64,6 +64,15 @@ def lib():
     L.kvq_rotate_quantize_append.argtypes = [p, p, i32, C.c_int, p, p, p, C.POINTER(CacheDesc), p, p]
     L.kvq_identify_sinks.restype = C.c_int
     L.kvq_identify_sinks.argtypes = [p, i32, C.c_float, C.POINTER(CacheDesc), p, p]
+    L.kvq_prerope_append.restype = C.c_int
+    L.kvq_prerope_append.argtypes = [p, p, i32, i32, p, C.POINTER(CacheDesc), p, p]
+    L.kvq_prerope_workspace_size.restype = sz
+    L.kvq_prerope_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.kvq_prerope_decode.restype = C.c_int
+    L.kvq_prerope_decode.argtypes = [p, i32, C.POINTER(CacheDesc), i32, p, C.c_float, p, i32, p,
+                                     sz, p, p]
+    L.kvq_debug_rotate_group_f32.restype = C.c_int
+    L.kvq_debug_rotate_group_f32.argtypes = [p, i32, i32, p, p, p]
     L.kvq_decode_workspace_size.restype = sz
     L.kvq_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     L.kvq_decode_attention.restype = C.c_int
@@ -359,3 +368,59 @@ def kvq_debug_quantize_f32(Xrot, stream=None):
            lib().kvq_debug_quantize_f32(_ptr(Xrot), N, _ptr(codes), _ptr(meta),
                                         _stream(stream, Xrot)))
     return codes, meta
+
+
+# --- pre-RoPE grouped-head key rotation ---------------------------------------------------
+
+def kvq_prerope_append(K, V, group_heads, perm, cache, seq_lens, stream=None):
+    """K (pre-RoPE), V fp16 [B][T][Hkv][128]; perm int32 [2][Hkv*128] (plane 0:
+    Hkv/group_heads key permutations of 128*group_heads entries; plane 1: one
+    value permutation of 128 per head); seq_lens int32 [B], updated."""
+    B, T, Hkv, d = K.shape
+    _need(K, torch.float16, "K", (cache.B, T, cache.Hkv, D))
+    _need(V, torch.float16, "V", K.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(perm, torch.int32, "perm", (2, cache.Hkv * D))
+    _check("kvq_prerope_append",
+           lib().kvq_prerope_append(_ptr(K), _ptr(V), T, group_heads, _ptr(perm),
+                                    C.byref(cache.desc), _ptr(seq_lens), _stream(stream, K)))
+
+
+def kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx, sm_count=None):
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return lib().kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx, sm_count)
+
+
+def prerope_workspace(B, Hq, Hkv, group_heads, max_ctx, device="cuda"):
+    n = kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx)
+    if n == 0:
+        raise ValueError("bad pre-RoPE decode shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kvq_prerope_decode(Q, cache, group_heads, perm, rope_base, seq_lens, max_ctx, workspace, out,
+                       stream=None):
+    """Q fp16 [B][Hq][128] post-RoPE queries -> out fp16 [B][Hq][128]."""
+    B, Hq, d = Q.shape
+    _need(Q, torch.float16, "Q", (cache.B, Hq, D))
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    _need(perm, torch.int32, "perm", (2, cache.Hkv * D))
+    _check("kvq_prerope_decode",
+           lib().kvq_prerope_decode(_ptr(Q), Hq, C.byref(cache.desc), group_heads, _ptr(perm),
+                                    float(rope_base), _ptr(seq_lens), max_ctx, _ptr(workspace),
+                                    workspace.numel(), _ptr(out), _stream(stream, Q)))
+
+
+def kvq_debug_rotate_group_f32(X, group_heads, perm, stream=None):
+    """X fp16 [N][128*group_heads] -> fp32 rows rotated by one group permutation + FWHT."""
+    _need(X, torch.float16, "X")
+    _need(perm, torch.int32, "perm", (D * group_heads,))
+    N = X.shape[0]
+    out = torch.empty((N, D * group_heads), dtype=torch.float32, device=X.device)
+    _check("kvq_debug_rotate_group_f32",
+           lib().kvq_debug_rotate_group_f32(_ptr(X), N, group_heads, _ptr(perm), _ptr(out),
+                                            _stream(stream, X)))
+    return out

@@ -219,3 +219,14 @@ def queries(w: Workload, device="cpu", step: int = 0) -> torch.Tensor:
 def f16_bits(t: torch.Tensor) -> np.ndarray:
     """fp16 tensor -> numpy uint16 bit patterns (host)."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# --- pre-RoPE grouped-head rotation -------------------------------------------------------
+
+def prerope_perm(w: Workload, gh: int) -> np.ndarray:
+    """int32 [2][Hkv*128]: plane 0 the Hkv/gh key-group permutations of
+    128*gh channels, plane 1 one value permutation of 128 per head (seeded)."""
+    rng = np.random.default_rng([w.seed, 91, gh])
+    keys = np.concatenate([rng.permutation(D * gh) for _ in range(w.Hkv // gh)])
+    vals = np.concatenate([rng.permutation(D) for _ in range(w.Hkv)])
+    return np.stack([keys, vals]).astype(np.int32)
