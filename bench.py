@@ -493,6 +493,68 @@ def sink_rates(device, reps=30):
             "identify_step_ms": id_step, "identify_prefill_32768_ms": id_pre}
 
 
+def prerope_rates(device, reps=20):
+    """Pre-RoPE grouped-head key rotation on the llama7b shape (B=1, 32
+    heads, context 32768): the 32768-token prefill appended through
+    kvq_prerope_append, then decode-only timings (L2 flushed before each
+    call) for group sizes 1 and 4, beside the post-RoPE FWHT decode of the
+    same tokens.  The decode is bound by its instruction stream (a 128*gh
+    point FWHT, the permutation scatter and RoPE per cached token), so its
+    roofline is reported as packed-KV bytes / time for comparison only."""
+    import rotated_int2_kv_head_b200 as kvq
+    w = W.custom(name="llama7b_prerope", seed=1002, B=1, Hq=32, Hkv=32, mode=1, context=32768,
+                 k_outliers=8)
+    L = 32768
+    flush = L2Flush(device)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def timed(fn, n=reps):
+        ms = []
+        for k in range(n + 3):
+            flush(k)
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize(device)
+            if k >= 3:
+                ms.append(ev[0].elapsed_time(ev[1]))
+        return float(np.median(ms))
+
+    K, V = W.kv_batch(w, 0, L, device)
+    Q = W.queries(w, device)
+    lens = torch.full((1,), L, dtype=torch.int32, device=device)
+    res = {"workload": "llama7b shape, pre-RoPE keys", "B": 1, "Hq": 32, "Hkv": 32, "context": L,
+           "how": "L2 flushed before each call, median of %d" % reps}
+    for gh in (1, 4):
+        perm = torch.from_numpy(W.prerope_perm(w, gh)).to(device)
+        cache = kvq.KVCache(1, 32, L, device=device)
+        sl = torch.zeros(1, dtype=torch.int32, device=device)
+
+        def app():
+            sl.zero_()
+            kvq.kvq_prerope_append(K, V, gh, perm, cache, sl)
+
+        app_ms = timed(app, 5)
+        ws = kvq.prerope_workspace(1, 32, 32, gh, L, device=device)
+        out = torch.empty_like(Q)
+        dec_ms = timed(lambda: kvq.kvq_prerope_decode(Q, cache, gh, perm, 10000.0, lens, L, ws, out))
+        if kvq.kvq_get_status(cache) != 0 or not bool(torch.isfinite(out.float()).all()):
+            raise RuntimeError("pre-RoPE timings: bad status or output")
+        res["gh%d" % gh] = {"prefill_append_ms": app_ms, "decode_ms": dec_ms,
+                            "decode_packed_kv_gbs": 32 * L * 96 / (dec_ms * 1e-3) / 1e9}
+    # the post-RoPE FWHT decode over the same tokens, for comparison
+    Rk = Rv = None
+    perm1 = torch.from_numpy(W.rotations(w)[2]).to(device)
+    cache = kvq.KVCache(1, 32, L, device=device)
+    sl = torch.zeros(1, dtype=torch.int32, device=device)
+    kvq.kvq_rotate_quantize_append(K, V, 1, Rk, Rv, perm1, cache, sl)
+    ws = kvq.decode_workspace(1, 32, 32, L, device=device)
+    out = torch.empty_like(Q)
+    res["post_rope_fwht_decode_ms"] = timed(lambda: kvq.kvq_decode_attention(
+        Q, cache, 1, Rk, Rv, perm1, lens, 0, L, ws, out))
+    return res
+
+
 def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
     the first `heads` KV heads of sequence 0 (their K/V rows are the very
@@ -729,6 +791,7 @@ def run_cuda(args):
     if world == 1 and not args.no_extensions:
         line["extensions"] = extension_rates(step, dev)
         line["extensions"]["identified_sinks"] = sink_rates(dev)
+        line["extensions"]["pre_rope"] = prerope_rates(dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, step, dev)
     print(json.dumps(line), flush=True)
@@ -806,7 +869,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
     ap.add_argument("--no-extensions", action="store_true",
-                    help="skip the paged / multi-query decode timings")
+                    help="skip the extension timings (paged, multi-query, identified sinks, pre-RoPE)")
+    ap.add_argument("--extension", choices=["pre_rope", "identified_sinks"], default=None,
+                    help="time one extension alone and print its JSON")
     ap.add_argument("--append-only", action="store_true",
                     help="only the bulk-append rates (one GPU), as one JSON line")
     args = ap.parse_args(argv)
@@ -821,6 +886,15 @@ def main(argv=None):
         peak, src = measured_peak()
         print(json.dumps({"append": append_rates(torch.device("cuda", 0), peak), "peak_gbs": peak,
                           "peak_source": src}), flush=True)
+    elif args.extension:
+        # one extension's timings alone (the same functions the full run
+        # reports under "extensions")
+        torch.cuda.set_device(0)
+        from rotated_int2_kv_head_b200 import build as kbuild
+        kbuild.build()
+        dev = torch.device("cuda", 0)
+        fn = {"pre_rope": prerope_rates, "identified_sinks": sink_rates}[args.extension]
+        print(json.dumps({args.extension: fn(dev)}), flush=True)
     else:
         run_cuda(args)
 

@@ -11,9 +11,9 @@
 //
 // Two kernels:
 //   prerope_split_kernel<GH, G>  grid (splits, B * Hkv/GH).  A CTA of 8 warps
-//       takes a contiguous range of 16-token cache blocks of one (b, group);
-//       warp w takes the range's blocks w, w+8, ... and their tokens in
-//       order.  Per token: the GH heads' K codes are dequantised (4 elements
+//       takes a contiguous range of 16-token cache blocks of one (b, group),
+//       split into 8 equal token runs, one per warp, taken in order.  Per
+//       token: the GH heads' K codes are dequantised (4 elements
 //       per lane), un-rotated by a warp FWHT (stages over the lane's 4
 //       elements and the 32 lanes by shuffles, stages across the GH heads in
 //       registers), scattered back through the permutation in shared memory,
@@ -24,7 +24,7 @@
 //   prerope_merge_kernel  per (b, query head): merges the partials and
 //       removes the value rotation (FWHT + inverse permutation).
 // The RoPE angle t * theta_f is taken as 2 pi * frac(t * theta_f / (2 pi))
-// in fp64 at the start of every 16-token block (theta_f / (2 pi) comes from
+// in fp64 at a warp's first token in every 16-token block (theta_f / (2 pi) comes from
 // the host in fp64), then advanced token by token with the rotation by
 // theta_f, so fp32 never holds an angle larger than 2 pi.
 #include "kvq_internal.cuh"
@@ -37,6 +37,37 @@ constexpr int PR_PART = 132;           // m, l, 0, 0, o[128]
 constexpr int PR_MIN_BLOCKS = 8;       // cache blocks per split at least
 constexpr float PR_LOG2E = 1.4426950408889634f;
 #define PR_NEG_INF (__int_as_float(0xff800000))
+
+// 128-point FWHT of a vector held as 4 consecutive elements per lane (the
+// layout of fwht128_warp): the cross-lane butterflies as one fma with a
+// per-lane sign, o + sgn*v (sgn = -1 in the upper lane of a pair), which
+// rounds exactly like o - v or v + o.
+__device__ __forceinline__ void fwht128_warp_fma(float v[4]) {
+    const int lane = threadIdx.x & 31;
+    float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+    v[0] = a0 + a2;
+    v[2] = a0 - a2;
+    v[1] = a1 + a3;
+    v[3] = a1 - a3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+            v[k] = fmaf(sgn, v[k], o);
+        }
+    }
+}
+
+// The four 2-bit codes of a lane (bits 2*g4 of the bytes of w) as exact
+// floats: each byte is put under the exponent of 2^23 and 2^23 subtracted.
+__device__ __forceinline__ void unpack4(uint32_t w, int g4, float c[4]) {
+    const uint32_t m = (w >> (2 * g4)) & 0x03030303u;
+#pragma unroll
+    for (int k = 0; k < 4; k++)
+        c[k] = __uint_as_float(__byte_perm(m, 0x4B000000u, 0x7540u + k)) - 8388608.0f;
+}
 
 struct PreRopeArgs {
     const uint16_t *Q;          // [B][Hq][128] post-RoPE queries
@@ -52,10 +83,13 @@ struct PreRopeArgs {
     double phi[D / 2];          // theta_f / (2 pi), theta_f = base^(-2f/128)
 };
 
+// Splits per (b, group): 12 CTAs per SM in all, i.e. whole waves at 1, 2, 3,
+// 4 or 6 resident CTAs per SM (equal ranges, so waves end together), and
+// at least PR_MIN_BLOCKS cache blocks per split.
 __host__ __device__ inline int pr_nsplit(int B, int ngroups, int max_ctx, int sms) {
     const int nb = (max_ctx + BLK_TOK - 1) / BLK_TOK;
     const int units = B * ngroups;
-    int want = (4 * sms + units - 1) / units;                 // about 4 CTAs per SM
+    int want = (12 * sms) / units;
     const int most = (nb + PR_MIN_BLOCKS - 1) / PR_MIN_BLOCKS;
     if (want > most) want = most;
     return want < 1 ? 1 : want;
@@ -116,9 +150,17 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
         for (int k = 0; k < 4; k++) o[i][k] = 0.f;
     }
     __syncthreads();                                  // pg_s
+    int4 preg[GH <= 2 ? GH : 1];                      // small groups: the lane's indices in registers
+#pragma unroll
+    for (int j = 0; j < (GH <= 2 ? GH : 1); j++)
+        preg[j] = *reinterpret_cast<const int4 *>(&pg_s[j * D + 4 * lane]);
 
     const int wi = lane & 7, g4 = lane >> 3;          // logical code word, quant group
-    for (int blk = blk0 + warp; blk < blk1; blk += PR_WARPS) {
+    // the CTA's tokens in PR_WARPS contiguous, equal runs, one per warp
+    const int t_beg = min(L, blk0 * BLK_TOK), t_end = min(L, blk1 * BLK_TOK);
+    const int per = (t_end - t_beg + PR_WARPS - 1) / PR_WARPS;
+    const int w0 = min(t_end, t_beg + warp * per), w1 = min(t_end, w0 + per);
+    for (int blk = w0 / BLK_TOK; w0 < w1 && blk <= (w1 - 1) / BLK_TOK; blk++) {
         // block addresses of the group's GH heads (and the V block of each)
         const uint8_t *bp[GH];
 #pragma unroll
@@ -128,16 +170,29 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
             if (bi < 0 && lane == 0) set_status(a.status, KVQ_DEV_BAD_TABLE);
             bp[j] = a.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
         }
-        // RoPE angle of the block's first token, reduced in fp64
+        // the warp's next block into L2 while this one is worked on (its
+        // 1536-byte blocks are 12 lines per head)
+        if ((blk + 1) * BLK_TOK < w1 && lane < 12) {
+#pragma unroll
+            for (int j = 0; j < GH; j++) {
+                const long long bn = cache_block_index(a.table, a.num_blocks, a.nblk, a.Hkv, b,
+                                                       grp * GH + j, blk + 1);
+                if (bn >= 0)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.blocks + (size_t)bn * BLK_BYTES +
+                                                                  128 * lane));
+            }
+        }
+        const int tau0 = max(w0, blk * BLK_TOK) - blk * BLK_TOK;
+        const int tau1 = min(w1, (blk + 1) * BLK_TOK) - blk * BLK_TOK;
+        // RoPE angle of the first token taken here, reduced in fp64
         float cs[4], sn[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-            const double u = (double)(blk * BLK_TOK) * a.phi[4 * (lane & 15) + k];
+            const double u = (double)(blk * BLK_TOK + tau0) * a.phi[4 * (lane & 15) + k];
             const double fr = u - floor(u);
             sincospif((float)(2.0 * fr), &sn[k], &cs[k]);
         }
-        const int ntok = min(BLK_TOK, L - blk * BLK_TOK);
-        for (int tau = 0; tau < ntok; tau++) {
+        for (int tau = tau0; tau < tau1; tau++) {
             const int r = tau & 7, th = tau >> 3;
             float v[GH][4];
 #pragma unroll
@@ -148,10 +203,11 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
                     *reinterpret_cast<const uint32_t *>(bp[j] + 1024 + 8 * (4 * r + g4) + 4 * th);
                 const float2 sz = unpack_half2(mk);
                 const float s = sz.x * isq, z = sz.y * isq;
+                float cf[4];
+                unpack4(w, g4, cf);
 #pragma unroll
-                for (int k = 0; k < 4; k++)
-                    v[j][k] = fmaf((float)((w >> (8 * k + 2 * g4)) & 3u), s, z);
-                fwht128_warp(v[j]);
+                for (int k = 0; k < 4; k++) v[j][k] = fmaf(cf[k], s, z);
+                fwht128_warp_fma(v[j]);
             }
 #pragma unroll
             for (int st = 1; st < GH; st <<= 1)
@@ -167,7 +223,7 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
             // k_pre[perm[i]] = y[i]: scatter, then read back in channel order
 #pragma unroll
             for (int j = 0; j < GH; j++) {
-                const int4 pi = *reinterpret_cast<const int4 *>(&pg_s[j * D + 4 * lane]);
+                const int4 pi = GH <= 2 ? preg[j] : *reinterpret_cast<const int4 *>(&pg_s[j * D + 4 * lane]);
                 kb_s[warp][pi.x] = v[j][0];
                 kb_s[warp][pi.y] = v[j][1];
                 kb_s[warp][pi.z] = v[j][2];
@@ -206,9 +262,9 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
                     *reinterpret_cast<const uint32_t *>(bp[j] + 1280 + 8 * (4 * r + g4) + 4 * th);
                 const float2 vsz = unpack_half2(vmk);
                 float vv[4];
+                unpack4(vw, g4, vv);
 #pragma unroll
-                for (int k = 0; k < 4; k++)
-                    vv[k] = fmaf((float)((vw >> (8 * k + 2 * g4)) & 3u), vsz.x, vsz.y);
+                for (int k = 0; k < 4; k++) vv[k] = fmaf(vv[k], vsz.x, vsz.y);
 #pragma unroll
                 for (int g = 0; g < G; g++) {
                     const int i = j * G + g;
