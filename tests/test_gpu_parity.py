@@ -442,3 +442,37 @@ def test_paged_bad_table_entry_sets_status():
     torch.cuda.synchronize()
     assert kvq.kvq_get_status(paged) & kvq.KVQ_DEV_BAD_TABLE
     assert torch.isfinite(out[0]).all()
+
+
+# --- values-only Hadamard rotation (the rotation split of "KVLinC", abstract) -------------------
+
+@pytest.mark.parametrize("T", [37, 300])
+def test_values_only_hadamard_rotation(T):
+    """KVLinC rotates the values by a Hadamard matrix and leaves the keys
+    unrotated (its key-error adapters are trained and not part of this
+    library): the dense mode with R_k = I and R_v = H/sqrt(128) serves that
+    split, through the CUDA-core (T=37) and tensor-core (T=300) appends."""
+    import scipy.linalg
+    B, Hkv, G = 2, 2, 2
+    w = W.custom(seed=300 + T, B=B, Hq=Hkv * G, Hkv=Hkv, mode=0, k_outliers=6)
+    Rk = np.stack([np.eye(D, dtype=np.float32)] * Hkv)
+    Rv = np.stack([(scipy.linalg.hadamard(D) / np.sqrt(D)).astype(np.float32)] * Hkv)
+    rt = (torch.from_numpy(Rk).cuda(), torch.from_numpy(Rv).cuda(), None)
+    L0 = [0, 9]
+    K = torch.stack([W.kv_rows(w, b, L0[b], L0[b] + T, "cpu")[0] for b in range(B)])
+    V = torch.stack([W.kv_rows(w, b, L0[b], L0[b] + T, "cpu")[1] for b in range(B)])
+    cap = ((max(L0) + T + 15) // 16) * 16
+    cache = kvq.KVCache(B, Hkv, cap)
+    sl = torch.tensor(L0, dtype=torch.int32, device="cuda")
+    gpu_append(cache, K.cuda(), V.cuda(), w, rt, sl)
+    oc = orc.Cache(B, Hkv, cap, 0)
+    osl = np.array(L0, np.int32)
+    assert orc.append(oc, f16bits(K), f16bits(V), 0, Rk, Rv, None, osl) == 0
+    Q = W.queries(w, "cpu")
+    ref, st = orc.decode(oc, f16bits(Q), 0, Rk, Rv, None, osl, n_threads=8)
+    assert st == 0
+    out = gpu_decode(cache, Q.cuda(), w, rt, sl, max(L0) + T)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    err = rel_err(out.cpu().numpy(), ref)
+    assert err.max() <= DEC_TOL, err.max()
