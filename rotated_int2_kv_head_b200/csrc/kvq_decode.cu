@@ -94,18 +94,32 @@ __device__ __forceinline__ int unit_blocks(int L, int S, int capacity) {
     return (L - 1) / BLK_TOK - S / BLK_TOK + 1;
 }
 
+// Schedule slots of a unit: its blocks plus UNIT_PHANTOM leading phantom
+// slots that stand for the cost of starting the unit (loading its queries,
+// and the flush of the partial when a group leaves it; measured at about
+// 8 blocks' streaming time).  Work is split evenly over slots, so a group
+// whose range takes in the start of a unit streams that many fewer blocks
+// and the groups finish together.  Phantom slots are skipped, never
+// processed.
+constexpr int UNIT_PHANTOM = 8;
+__device__ __forceinline__ int unit_slots(int L, int S, int capacity) {
+    const int nb = unit_blocks(L, S, capacity);
+    return nb > 0 ? nb + UNIT_PHANTOM : 0;
+}
+
 // ---------------------------------------------------------------------------------------------
 // Split kernel.
 // ---------------------------------------------------------------------------------------------
-// Per-CTA schedule over the global block space: unit u = b*Hkv + h holds
-// nb(b) consecutive global blocks starting at prefix[b] + h*nb(b), where
-// prefix[b] = Hkv * sum over b' < b of nb(b').  `pref` carries prefix[b].
+// Per-CTA schedule over the global slot space: unit u = b*Hkv + h holds
+// nb(b) = unit_slots consecutive slots (UNIT_PHANTOM phantom slots, then one
+// per cache block) starting at prefix[b] + h*nb(b), where prefix[b] = Hkv *
+// sum over b' < b of nb(b').  `pref` carries prefix[b].
 struct Sched {
     int b, h, nb, ustart, cur, end, pref;
 };
 
 __device__ __forceinline__ int seq_blocks(const DecodeArgs &a, int b) {
-    return unit_blocks(a.seq_lens[b], a.S, a.capacity);
+    return unit_slots(a.seq_lens[b], a.S, a.capacity);
 }
 
 __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
@@ -138,7 +152,7 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     for (int b = lo; b < hi; b++) {
         const int L = a.seq_lens[b];
         if (blockIdx.x == 0 && (L < 1 || L > a.capacity)) set_status(a.status, KVQ_DEV_BAD_LEN);
-        const int nb = unit_blocks(L, a.S, a.capacity);
+        const int nb = unit_slots(L, a.S, a.capacity);
         if (b == lo) nb_lo = nb;
         sum += a.Hkv * nb;
     }
@@ -206,11 +220,16 @@ __device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &
                                            int &h, int &kblk, int &n) {
     if (ps.cur >= ps.end) return false;
     sched_fix_unit(ps, a);
+    const int first = ps.ustart + UNIT_PHANTOM;       // slot of the unit's block 0
+    if (ps.cur < first) {                             // skip the phantom slots
+        ps.cur = first;
+        if (ps.cur >= ps.end) return false;
+    }
     n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
     unit = ps.b * a.Hkv + ps.h;
     b = ps.b;
     h = ps.h;
-    kblk = ps.cur - ps.ustart;
+    kblk = ps.cur - first;
     ps.cur += n;
     return true;
 }
@@ -1025,7 +1044,7 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
     {
         int sb = 0, sn = 0;
         for (int i = t; i < a.B; i += MRG_THREADS) {
-            const int nbi = a.Hkv * unit_blocks(a.seq_lens[i], a.S, a.capacity);
+            const int nbi = a.Hkv * unit_slots(a.seq_lens[i], a.S, a.capacity);
             sn += nbi;
             sb += i < b ? nbi : 0;
         }
@@ -1061,7 +1080,7 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         return;
     }
     const int u = b * a.Hkv + h;
-    const int nb = unit_blocks(L, a.S, a.capacity);
+    const int nb = unit_slots(L, a.S, a.capacity);
     const int W = max(1, (N + a.C - 1) / a.C);
     const int ustart = pre + h * nb;
     const int c0 = nb > 0 ? ustart / W : 0;
