@@ -493,6 +493,64 @@ def sink_rates(device, reps=30):
             "identify_step_ms": id_step, "identify_prefill_32768_ms": id_pre}
 
 
+def decode_rates(device, peak, reps=20):
+    """Decode alone on every workload of workloads.py at its full size (the
+    cache filled through the library's append, L2 flushed before each timed
+    call, median of `reps`): tokens/s = B / t, context tokens/s = sum of
+    L_b * Hkv / t, packed-KV GB/s (96 B per cached token-head, 512 B per fp16
+    sink token-head) and its fraction of the HBM peak, and a total-bytes rate
+    that adds the rotations (dense: 2 * Hkv * 64 KB; FWHT: the permutations),
+    Q and the output."""
+    import rotated_int2_kv_head_b200 as kvq
+    flush = L2Flush(device)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    res = {"how": "decode only, cache filled first, L2 flushed before each call, median of %d"
+                  % reps}
+    for name in ("tiny", "llama7b", "hadamard", "gqa_sinks", "ragged"):
+        w = W.WORKLOADS[name]
+        lens_np = w.seq_lens().astype(np.int32)
+        L = int(lens_np.max())
+        cap = ((L + 15) // 16) * 16
+        Rk, Rv, perm = W.rotations(w)
+        rk = torch.from_numpy(Rk).to(device) if Rk is not None else None
+        rv = torch.from_numpy(Rv).to(device) if Rv is not None else None
+        pm = torch.from_numpy(perm).to(device) if perm is not None else None
+        cache = kvq.KVCache(w.B, w.Hkv, cap, w.sink, device=device)
+        fill = torch.zeros(w.B, dtype=torch.int32, device=device)
+        for t0 in range(0, L, 4096):
+            K, V = W.kv_batch(w, t0, min(L, t0 + 4096), device)
+            kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, pm, cache, fill)
+            del K, V
+        lens = torch.from_numpy(lens_np).to(device)
+        Q = W.queries(w, device)
+        ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, L, device=device)
+        out = torch.empty_like(Q)
+        ms = []
+        for k in range(reps + 3):
+            flush(k)
+            ev[0].record()
+            kvq.kvq_decode_attention(Q, cache, w.mode, rk, rv, pm, lens, w.sink, L, ws, out)
+            ev[1].record()
+            torch.cuda.synchronize(device)
+            if k >= 3:
+                ms.append(ev[0].elapsed_time(ev[1]))
+        if kvq.kvq_get_status(cache) != 0 or not bool(torch.isfinite(out.float()).all()):
+            raise RuntimeError("decode timings on %s: bad status or output" % name)
+        t = float(np.median(ms)) * 1e-3
+        kv = packed_kv_bytes(w, lens_np)
+        rot = 2 * w.Hkv * 128 * 128 * 4 if w.mode == 0 else 2 * w.Hkv * 128 * 4
+        total = kv + rot + 2 * Q.numel() * 2
+        res[name] = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "context_max": L,
+                     "rotation": "dense" if w.mode == 0 else "perm+fwht", "sink_fp16": w.sink,
+                     "decode_us": t * 1e6, "tokens_per_s": w.B / t,
+                     "context_tokens_per_s": float(lens_np.astype(np.int64).sum()) * w.Hkv / t,
+                     "packed_kv_bytes": kv, "packed_kv_gbs": kv / t / 1e9,
+                     "frac_of_hbm_peak": kv / t / 1e9 / peak, "total_bytes_gbs": total / t / 1e9}
+        del cache, ws
+        torch.cuda.empty_cache()
+    return res
+
+
 def prerope_rates(device, reps=20):
     """Pre-RoPE grouped-head key rotation on the llama7b shape (B=1, 32
     heads, context 32768): the 32768-token prefill appended through
@@ -792,6 +850,8 @@ def run_cuda(args):
         line["extensions"] = extension_rates(step, dev)
         line["extensions"]["identified_sinks"] = sink_rates(dev)
         line["extensions"]["pre_rope"] = prerope_rates(dev)
+    if world == 1 and not args.no_workloads:
+        line["workloads"] = decode_rates(dev, peak)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, step, dev)
     print(json.dumps(line), flush=True)
@@ -870,7 +930,10 @@ def main(argv=None):
     ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the extension timings (paged, multi-query, identified sinks, pre-RoPE)")
-    ap.add_argument("--extension", choices=["pre_rope", "identified_sinks"], default=None,
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the decode timings of every workload at full size")
+    ap.add_argument("--extension", choices=["pre_rope", "identified_sinks", "workloads"],
+                    default=None,
                     help="time one extension alone and print its JSON")
     ap.add_argument("--append-only", action="store_true",
                     help="only the bulk-append rates (one GPU), as one JSON line")
@@ -893,8 +956,11 @@ def main(argv=None):
         from rotated_int2_kv_head_b200 import build as kbuild
         kbuild.build()
         dev = torch.device("cuda", 0)
-        fn = {"pre_rope": prerope_rates, "identified_sinks": sink_rates}[args.extension]
-        print(json.dumps({args.extension: fn(dev)}), flush=True)
+        if args.extension == "workloads":
+            print(json.dumps({"workloads": decode_rates(dev, measured_peak()[0])}), flush=True)
+        else:
+            fn = {"pre_rope": prerope_rates, "identified_sinks": sink_rates}[args.extension]
+            print(json.dumps({args.extension: fn(dev)}), flush=True)
     else:
         run_cuda(args)
 
