@@ -188,19 +188,19 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
     pdl_trigger();
-    const long long row = (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
-    bool active = row < a.n_rows;
+    // cache: CTA (bt, y) takes token bt = b*T + t, warp w the (head, kind)
+    // pair 8y + w (kind fastest); debug: one row per warp
+    const long long row = TO_CACHE ? 0 : (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
+    const int hk = TO_CACHE ? (int)blockIdx.y * (FWHT_THREADS / 32) + warp : 0;
+    bool active = TO_CACHE ? hk < 2 * c.Hkv : row < a.n_rows;
     int b = 0, t = 0, h = 0, kind = 0, L0 = 0;
     const uint16_t *src = nullptr;
     const int32_t *perm = nullptr;
     if (active && TO_CACHE) {
-        // row order (b, t, h, kind) with kind fastest
-        kind = (int)(row & 1);
-        long long r2 = row >> 1;
-        h = (int)(r2 % c.Hkv);
-        r2 /= c.Hkv;
-        t = (int)(r2 % c.T);
-        b = (int)(r2 / c.T);
+        kind = hk & 1;
+        h = hk >> 1;
+        b = (int)(blockIdx.x / (unsigned)c.T);
+        t = (int)(blockIdx.x - (unsigned)b * (unsigned)c.T);
         const int L = c.seq_lens[b];
         if (L < 0 || (long long)L + c.T > c.capacity) {
             if (lane == 0 && t == 0 && h == 0 && kind == 0)
@@ -502,8 +502,9 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.perm = perm;
         a.out_f32 = nullptr;
         a.n_rows = (long long)cd.B * T * cd.Hkv * 2;
-        const long long per = FWHT_THREADS / 32;
-        return launch_pdl(append_fwht_kernel<true>, dim3((unsigned)((a.n_rows + per - 1) / per)),
+        const int per = FWHT_THREADS / 32;
+        return launch_pdl(append_fwht_kernel<true>,
+                          dim3((unsigned)((long long)cd.B * T), (2 * cd.Hkv + per - 1) / per),
                           dim3(FWHT_THREADS), 0, st, a, c);
     }
 }

@@ -184,17 +184,6 @@ __device__ __forceinline__ void convert_r(const float *R, uint8_t *bhi, uint8_t 
 // pattern is 0x4B400000 + c.  That pattern, shifted to the code's place, is
 // added into the word (one integer multiply-add; the codes' bits never
 // overlap), and the constant 0x4B400000-terms are taken out once per word.
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
-    float r;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
 __device__ __forceinline__ uint32_t quantize_group_thread(const float (&v)[32], int g,
                                                           uint32_t (&words)[8]) {
     // min and max of the 32 values with three-input min/max: 32 -> 12 -> 4 -> 1
@@ -217,7 +206,7 @@ __device__ __forceinline__ uint32_t quantize_group_thread(const float (&v)[32], 
     const __half s = __float2half_rn(__fadd_rn(sf, 0.0f));   // zero stored as +0
     const __half z = __float2half_rn(__fadd_rn(mn[0], 0.0f));
     const float sF = __half2float(s), zF = __half2float(z);
-    const float inv = (sF == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sF);
+    const float inv = (sF == 0.0f) ? 0.0f : __frcp_rn(sF);   // = the IEEE quotient 1/s
     constexpr float MAGIC = 12582912.0f;                     // 1.5 * 2^23
     constexpr uint32_t MAGIC_BITS = 0x4B400000u;
 #pragma unroll

@@ -57,11 +57,30 @@ struct QuantWord {
     uint16_t s, z;
 };
 
+// Three-input fp32 min / max (one instruction each).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Per element the code is formed without a float-to-int conversion: clamp t
+// to [0, 3] first (clamping then rounding equals rounding then clamping on
+// that interval), then add 1.5 * 2^23, after which fp32 round-to-nearest-
+// even leaves rint(t) in the low mantissa bits (bit pattern 0x4B400000 + c).
+// The four patterns are added into the word at their codes' places and the
+// constant terms taken out once.  1/s is the correctly rounded reciprocal
+// (__frcp_rn), the same value as the IEEE division 1/s.
 __device__ __forceinline__ QuantWord quantize_row_warp(const float v[4]) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 3;
-    float mn = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
-    float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+    float mn = fminf(fmin3(v[0], v[1], v[2]), v[3]);
+    float mx = fmaxf(fmax3(v[0], v[1], v[2]), v[3]);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -72,15 +91,18 @@ __device__ __forceinline__ QuantWord quantize_row_warp(const float v[4]) {
     const __half s = __float2half_rn(__fadd_rn(sf, 0.0f));   // zero stored as +0
     const __half z = __float2half_rn(__fadd_rn(mn, 0.0f));
     const float sF = __half2float(s), zF = __half2float(z);
-    const float inv = (sF == 0.0f) ? 0.0f : __fdiv_rn(1.0f, sF);
+    const float inv = (sF == 0.0f) ? 0.0f : __frcp_rn(sF);
+    constexpr float MAGIC = 12582912.0f;                     // 1.5 * 2^23
+    constexpr uint32_t MAGIC_BITS = 0x4B400000u;
     uint32_t bits = 0;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
-        const float t = __fmul_rn(__fsub_rn(v[k], zF), inv);
-        const float rt = rintf(t);
-        const uint32_t c = rt < 0.0f ? 0u : (rt > 3.0f ? 3u : (uint32_t)rt);
-        bits |= c << (8 * k + 2 * g);
+        float t = __fmul_rn(__fsub_rn(v[k], zF), inv);
+        t = fminf(fmaxf(t, 0.0f), 3.0f);
+        bits += __float_as_uint(__fadd_rn(t, MAGIC)) << (8 * k + 2 * g);
     }
+    bits -= (MAGIC_BITS << (2 * g)) + (MAGIC_BITS << (8 + 2 * g)) + (MAGIC_BITS << (16 + 2 * g)) +
+            (MAGIC_BITS << (24 + 2 * g));
     bits |= __shfl_xor_sync(0xffffffffu, bits, 8);
     bits |= __shfl_xor_sync(0xffffffffu, bits, 16);
     QuantWord q;
@@ -124,6 +146,9 @@ __device__ __forceinline__ void zero_token_warp(uint8_t *block, int tau, int kin
 
 // ---- warp FWHT of a 128-vector held as 4 consecutive elements per lane -------------
 // Sylvester order; butterflies (a, b) -> (a + b, a - b) at every stride.
+// The cross-lane butterflies are one fma with a per-lane sign, o + sgn*v
+// (sgn = -1 in the upper lane of a pair): it rounds exactly like o - v or
+// v + o.
 __device__ __forceinline__ void fwht128_warp(float v[4]) {
     const int lane = threadIdx.x & 31;
     float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
@@ -133,11 +158,11 @@ __device__ __forceinline__ void fwht128_warp(float v[4]) {
     v[3] = a1 - a3;
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
+        const float sgn = (lane & m) ? -1.f : 1.f;
 #pragma unroll
         for (int k = 0; k < 4; k++) {
             const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
-            v[k] = upper ? (o - v[k]) : (v[k] + o);
+            v[k] = fmaf(sgn, v[k], o);
         }
     }
 }

@@ -38,28 +38,6 @@ constexpr int PR_MIN_BLOCKS = 8;       // cache blocks per split at least
 constexpr float PR_LOG2E = 1.4426950408889634f;
 #define PR_NEG_INF (__int_as_float(0xff800000))
 
-// 128-point FWHT of a vector held as 4 consecutive elements per lane (the
-// layout of fwht128_warp): the cross-lane butterflies as one fma with a
-// per-lane sign, o + sgn*v (sgn = -1 in the upper lane of a pair), which
-// rounds exactly like o - v or v + o.
-__device__ __forceinline__ void fwht128_warp_fma(float v[4]) {
-    const int lane = threadIdx.x & 31;
-    float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
-    v[0] = a0 + a2;
-    v[2] = a0 - a2;
-    v[1] = a1 + a3;
-    v[3] = a1 - a3;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const float sgn = (lane & m) ? -1.f : 1.f;
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
-            v[k] = fmaf(sgn, v[k], o);
-        }
-    }
-}
-
 // The four 2-bit codes of a lane (bits 2*g4 of the bytes of w) as exact
 // floats: each byte is put under the exponent of 2^23 and 2^23 subtracted.
 __device__ __forceinline__ void unpack4(uint32_t w, int g4, float c[4]) {
@@ -207,7 +185,7 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
                 unpack4(w, g4, cf);
 #pragma unroll
                 for (int k = 0; k < 4; k++) v[j][k] = fmaf(cf[k], s, z);
-                fwht128_warp_fma(v[j]);
+                fwht128_warp(v[j]);
             }
 #pragma unroll
             for (int st = 1; st < GH; st <<= 1)
