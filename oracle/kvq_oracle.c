@@ -591,10 +591,16 @@ void orc_unrotate_group_f64(const double *o, int n, const int32_t *perm, double 
 /* Pre-RoPE append.  K (pre-RoPE), V: fp16 [B][T][Hkv][128]; gh divides Hkv;
  * perm int32 [2][Hkv*128]: plane 0 holds Hkv/gh key permutations of n =
  * 128*gh entries each (group q at perm + q*n), plane 1 one value permutation
- * of 128 entries per head.  No sinks.  Returns the status bits; seq_lens
- * advance by T for every sequence that fits. */
+ * of 128 entries per head.  Sinks (RotateKV item (iii); sink_row above): the
+ * sink row keeps the key as given (pre-RoPE, not rotated: it is never
+ * quantized, and RoPE is applied at decode time) and the rotated value in
+ * fp16; the INT2 slot is zeroed, with the K-meta marker for identified
+ * sinks.  Returns the status bits; seq_lens advance by T for every sequence
+ * that fits. */
 int orc_append_prerope(const uint16_t *K, const uint16_t *V, int B, int T, int Hkv, int gh,
-                       const int32_t *perm, int capacity, uint8_t *blocks, int32_t *seq_lens) {
+                       const int32_t *perm, int capacity, int S, uint8_t *blocks,
+                       uint16_t *k_sink, uint16_t *v_sink, int32_t *seq_lens,
+                       const int32_t *sink_pos, const int32_t *sink_count) {
     int status = 0;
     const int nblk = capacity / BLK_TOK;
     const int n = D * gh;
@@ -614,6 +620,7 @@ int orc_append_prerope(const uint16_t *K, const uint16_t *V, int B, int T, int H
                         xg[j * D + i] = (double)orc_f16_to_f32(
                             K[(((size_t)b * T + t) * Hkv + q * gh + j) * D + i]);
                 orc_rotate_group_f64(xg, n, perm + (size_t)q * n, xr);
+                const int row = sink_row(S, sink_pos, sink_count, b, p);
                 for (int j = 0; j < gh; j++) {
                     const int h = q * gh + j;
                     float kr[D], vr[D];
@@ -622,10 +629,28 @@ int orc_append_prerope(const uint16_t *K, const uint16_t *V, int B, int T, int H
                                         perm + ((size_t)Hkv + h) * D, vr);
                     uint8_t kc[D], vc[D], kb[32], vb[32];
                     uint16_t ks[NG], kz[NG], vs[NG], vz[NG];
-                    orc_quantize_row(kr, kc, ks, kz);
-                    orc_quantize_row(vr, vc, vs, vz);
-                    orc_pack_row(kc, kb);
-                    orc_pack_row(vc, vb);
+                    if (row >= 0) {
+                        const uint16_t *kin = K + (((size_t)b * T + t) * Hkv + h) * D;
+                        uint16_t *ksr = k_sink + (((size_t)b * Hkv + h) * S + row) * D;
+                        uint16_t *vsr = v_sink + (((size_t)b * Hkv + h) * S + row) * D;
+                        for (int i = 0; i < D; i++) {
+                            ksr[i] = kin[i];
+                            vsr[i] = orc_f32_to_f16(vr[i]);
+                        }
+                        memset(kb, 0, 32);
+                        memset(vb, 0, 32);
+                        memset(ks, 0, sizeof ks);
+                        memset(kz, 0, sizeof kz);
+                        memset(vs, 0, sizeof vs);
+                        memset(vz, 0, sizeof vz);
+                        if (sink_pos != NULL)
+                            for (int g = 0; g < NG; g++) ks[g] = 0x7E00;
+                    } else {
+                        orc_quantize_row(kr, kc, ks, kz);
+                        orc_quantize_row(vr, vc, vs, vz);
+                        orc_pack_row(kc, kb);
+                        orc_pack_row(vc, vb);
+                    }
                     uint8_t *block =
                         blocks + (((size_t)b * Hkv + h) * nblk + p / BLK_TOK) * BLK_BYTES;
                     orc_store_token(block, p % BLK_TOK, kb, vb, ks, kz, vs, vz);
@@ -642,14 +667,16 @@ int orc_append_prerope(const uint16_t *K, const uint16_t *V, int B, int T, int H
 /* Pre-RoPE decode.  Q: fp16 [B][Hq][128] post-RoPE queries (query head hq
  * reads KV head hq / G).  For every position t < L: the dequantised rotated
  * key rows of the gh heads of the group, inversely rotated, the head's slice
- * taken and RoPE'd at position t; s_t = q . k_t / sqrt(128); softmax; the
- * values as in FWHT mode: o_rot = sum p_t v_t, out = FWHT(o_rot)/sqrt(128)
- * scattered through the head's value permutation.  Output fp64 [B][Hq][128];
- * invalid lengths give zeros and ST_BAD_LEN. */
+ * taken and RoPE'd at position t (a sink: its stored pre-RoPE key RoPE'd);
+ * s_t = q . k_t / sqrt(128); softmax; the values as in FWHT mode:
+ * o_rot = sum p_t v_t, out = FWHT(o_rot)/sqrt(128) scattered through the
+ * head's value permutation.  Output fp64 [B][Hq][128]; invalid lengths give
+ * zeros and ST_BAD_LEN. */
 int orc_decode_prerope(const uint16_t *Q, int B, int Hq, int Hkv, int gh, const int32_t *perm,
-                       double rope_base, int capacity, const uint8_t *blocks,
-                       const int32_t *seq_lens, int only_b, int only_h, int n_threads,
-                       double *out) {
+                       double rope_base, int capacity, int S, const uint8_t *blocks,
+                       const uint16_t *k_sink, const uint16_t *v_sink, const int32_t *seq_lens,
+                       const int32_t *sink_pos, const int32_t *sink_count, int only_b,
+                       int only_h, int n_threads, double *out) {
     int status = 0;
     const int G = Hq / Hkv;
     const int nblk = capacity / BLK_TOK;
@@ -678,14 +705,21 @@ int orc_decode_prerope(const uint16_t *Q, int B, int Hq, int Hkv, int gh, const 
         double *s = (double *)malloc(sizeof(double) * (size_t)L);
         const double scale = 1.0 / sqrt((double)D);
         double m = -INFINITY;
+        const size_t uh = (size_t)b * Hkv + h;
         for (int t = 0; t < L; t++) {
-            for (int jj = 0; jj < gh; jj++) {
-                const size_t u = (size_t)b * Hkv + q * gh + jj;
-                dequant_token(blocks + u * (size_t)nblk * BLK_BYTES, NULL, NULL, -1, t, k, v);
-                for (int i = 0; i < D; i++) kg[jj * D + i] = k[i];
+            const int row = sink_row(S, sink_pos, sink_count, b, t);
+            if (row >= 0) {
+                for (int i = 0; i < D; i++)
+                    k[i] = (double)orc_f16_to_f32(k_sink[(uh * S + row) * D + i]);
+            } else {
+                for (int jj = 0; jj < gh; jj++) {
+                    const size_t u = (size_t)b * Hkv + q * gh + jj;
+                    dequant_token(blocks + u * (size_t)nblk * BLK_BYTES, NULL, NULL, -1, t, k, v);
+                    for (int i = 0; i < D; i++) kg[jj * D + i] = k[i];
+                }
+                orc_unrotate_group_f64(kg, n, perm + (size_t)q * n, ku);
+                for (int i = 0; i < D; i++) k[i] = ku[j * D + i];
             }
-            orc_unrotate_group_f64(kg, n, perm + (size_t)q * n, ku);
-            for (int i = 0; i < D; i++) k[i] = ku[j * D + i];
             orc_rope_f64(k, t, rope_base);
             double acc = 0.0;
             for (int i = 0; i < D; i++) acc += qv[i] * k[i];
@@ -694,11 +728,13 @@ int orc_decode_prerope(const uint16_t *Q, int B, int Hq, int Hkv, int gh, const 
         }
         double l = 0.0;
         for (int i = 0; i < D; i++) orot[i] = 0.0;
-        const size_t uh = (size_t)b * Hkv + h;
         for (int t = 0; t < L; t++) {
             const double p = exp(s[t] - m);
             l += p;
-            dequant_token(blocks + uh * (size_t)nblk * BLK_BYTES, NULL, NULL, -1, t, k, v);
+            dequant_token(blocks + uh * (size_t)nblk * BLK_BYTES,
+                          S > 0 ? k_sink + uh * (size_t)S * D : NULL,
+                          S > 0 ? v_sink + uh * (size_t)S * D : NULL,
+                          sink_row(S, sink_pos, sink_count, b, t), t, k, v);
             for (int i = 0; i < D; i++) orot[i] += p * v[i];
         }
         for (int i = 0; i < D; i++) orot[i] /= l;

@@ -105,15 +105,17 @@ def rope_complex(x, t, base):
     return np.concatenate([z.real, z.imag])
 
 
-def decode_prerope_one(q_f16, kgroup_hat, j, perm_group, base, vhat, pv):
+def decode_prerope_one(q_f16, kgroup_hat, j, perm_group, base, vhat, pv, sink_keys=None):
     """q fp16 [128] post-RoPE; kgroup_hat fp64 [L, n] rotated group key rows
     (dequantised); j the head's slot in its group; vhat fp64 [L,128] rotated
-    value rows; pv the head's value permutation."""
+    value rows; pv the head's value permutation; sink_keys {t: pre-RoPE key
+    row} for positions kept in fp16 (their kgroup_hat rows are ignored)."""
     q = np.asarray(q_f16, np.float16).astype(np.float64)
     M = group_rotation_matrix(perm_group)
     kpre = kgroup_hat @ M.T                        # inverse of an orthogonal map
-    k = np.stack([rope_complex(kpre[t, j * D:(j + 1) * D], t, base)
-                  for t in range(kpre.shape[0])])
+    sink_keys = sink_keys or {}
+    k = np.stack([rope_complex(sink_keys[t] if t in sink_keys else kpre[t, j * D:(j + 1) * D],
+                               t, base) for t in range(kpre.shape[0])])
     s = k @ q / np.sqrt(D)
     p = np.exp(s - s.max())
     o = (p / p.sum()) @ vhat

@@ -56,9 +56,10 @@ def lib():
         L.orc_rotate_group_f64.argtypes = [p, ci, p, p]
         L.orc_unrotate_group_f64.argtypes = [p, ci, p, p]
         L.orc_append_prerope.restype = ci
-        L.orc_append_prerope.argtypes = [p, p, ci, ci, ci, ci, p, ci, p, p]
+        L.orc_append_prerope.argtypes = [p, p, ci, ci, ci, ci, p, ci, ci, p, p, p, p, p, p]
         L.orc_decode_prerope.restype = ci
-        L.orc_decode_prerope.argtypes = [p, ci, ci, ci, ci, p, C.c_double, ci, p, p, ci, ci, ci, p]
+        L.orc_decode_prerope.argtypes = [p, ci, ci, ci, ci, p, C.c_double, ci, ci, p, p, p, p, p, p,
+                                         ci, ci, ci, p]
         _lib = L
     return _lib
 
@@ -273,27 +274,29 @@ def unrotate_group_f64(o, perm):
 def append_prerope(cache, K, V, gh, perm, seq_lens):
     """K (pre-RoPE), V: fp16 bit patterns [B][T][Hkv][128]; perm int32
     [2][Hkv*128] (plane 0: Hkv/gh key permutations of 128*gh entries; plane 1:
-    one value permutation of 128 per head).  Needs a cache without sinks."""
-    assert cache.S == 0
+    one value permutation of 128 per head).  Sinks (leading or identified) keep
+    the pre-RoPE key as given and the rotated value, in fp16."""
     K = _c(K, np.uint16)
     V = _c(V, np.uint16)
     B, T, Hkv, d = K.shape
     assert d == D and B == cache.B and Hkv == cache.Hkv and V.shape == K.shape and Hkv % gh == 0
     assert seq_lens.dtype == np.int32 and seq_lens.flags.c_contiguous
     pc = _c(perm, np.int32).reshape(2, Hkv * D)
-    return lib().orc_append_prerope(_p(K), _p(V), B, T, Hkv, gh, _p(pc), cache.capacity,
-                                    _p(cache.blocks), _p(seq_lens))
+    return lib().orc_append_prerope(_p(K), _p(V), B, T, Hkv, gh, _p(pc), cache.capacity, cache.S,
+                                    _p(cache.blocks), _p(cache.k_sink), _p(cache.v_sink),
+                                    _p(seq_lens), _p(cache.sink_pos), _p(cache.sink_count))
 
 
 def decode_prerope(cache, Q, gh, perm, rope_base, seq_lens, only_b=-1, only_h=-1, n_threads=1):
     """Q: fp16 bit patterns [B][Hq][128] (post-RoPE).  Returns (out fp64, status)."""
     Q = _c(Q, np.uint16)
     B, Hq, d = Q.shape
-    assert d == D and B == cache.B and Hq % cache.Hkv == 0 and cache.S == 0
+    assert d == D and B == cache.B and Hq % cache.Hkv == 0
     pc = _c(perm, np.int32).reshape(2, cache.Hkv * D)
     sl = _c(seq_lens, np.int32)
     out = np.zeros((B, Hq, D), np.float64)
     st = lib().orc_decode_prerope(_p(Q), B, Hq, cache.Hkv, gh, _p(pc), float(rope_base),
-                                  cache.capacity, _p(cache.blocks), _p(sl), only_b, only_h,
-                                  n_threads, _p(out))
+                                  cache.capacity, cache.S, _p(cache.blocks), _p(cache.k_sink),
+                                  _p(cache.v_sink), _p(sl), _p(cache.sink_pos),
+                                  _p(cache.sink_count), only_b, only_h, n_threads, _p(out))
     return out, st

@@ -663,3 +663,109 @@ def test_prerope_c_oracle_matches_numpy_mini_oracle(gh, G):
                     ref = np_mini.decode_prerope_one(Q[b, hq], khat, jj, pg, base, vhat,
                                                      perm[1, h * D:(h + 1) * D])
                     assert np.allclose(out[b, hq], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("gh", [1, 2])
+def test_prerope_all_sinks_is_fp16_attention_with_rope(gh):
+    """With every position a sink nothing is quantized: the decode must be
+    the attention over the stored fp16 rows, keys RoPE'd at their positions
+    (complex-exponential formulation), softmax from scipy, values rotated
+    back through the explicit permuted Hadamard matrix.  The sink rows must
+    hold the pre-RoPE keys exactly as given."""
+    rng = np.random.default_rng(70 + gh)
+    B, T, Hkv, G, base = 2, 13, 2 * gh, 2, 10000.0
+    n = D * gh
+    K = (rng.standard_normal((B, T, Hkv, D)) * 2).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    perm = np.concatenate([np.concatenate([rng.permutation(n) for _ in range(Hkv // gh)]),
+                           np.concatenate([rng.permutation(D) for _ in range(Hkv)])]
+                          ).astype(np.int32).reshape(2, Hkv * D)
+    cache = orc.Cache(B, Hkv, 32, 16)
+    sl = np.zeros(B, np.int32)
+    assert orc.append_prerope(cache, K.view(np.uint16), V.view(np.uint16), gh, perm, sl) == 0
+    assert np.array_equal(cache.k_sink[:, :, :T], K.transpose(0, 2, 1, 3).view(np.uint16))
+    assert not cache.blocks.any()                         # no INT2 token, nothing written there
+    Q = rng.standard_normal((B, Hkv * G, D)).astype(np.float16)
+    out, st = orc.decode_prerope(cache, Q.view(np.uint16), gh, perm, base, sl)
+    assert st == 0
+    for b in range(B):
+        for h in range(Hkv):
+            pv = perm[1, h * D:(h + 1) * D]
+            vr = np_mini.rotate_rows_f32(V[b, :, h], 1, perm=pv)
+            # the stored value rows are the fp16 rounding of the rotated rows
+            vs = cache.v_sink[b, h, :T].view(np.float16).astype(np.float64)
+            assert np.max(np.abs(vs - vr.astype(np.float16).astype(np.float64))) <= \
+                np.max(np.abs(vs)) * 2.0 ** -10
+            k = np.stack([np_mini.rope_complex(K[b, t, h].astype(np.float64), t, base)
+                          for t in range(T)])
+            for hq in range(h * G, (h + 1) * G):
+                sc = k @ Q[b, hq].astype(np.float64) / np.sqrt(D)
+                p = scipy.special.softmax(sc)
+                ref = (p @ vs) @ np_mini.rotation_matrix(1, perm=pv).T
+                assert np.allclose(out[b, hq], ref, rtol=0, atol=1e-12)
+
+
+def test_prerope_identified_sinks_threshold_minus_inf_are_the_leading_sinks():
+    rng = np.random.default_rng(75)
+    B, T, Hkv, gh, S = 2, 40, 2, 2, 4
+    K = (rng.standard_normal((B, T, Hkv, D)) * 2).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    perm = np.concatenate([rng.permutation(D * gh), np.concatenate(
+        [rng.permutation(D) for _ in range(Hkv)])]).astype(np.int32).reshape(2, Hkv * D)
+    ic = orc.Cache(B, Hkv, 48, S, identified=True)
+    lc = orc.Cache(B, Hkv, 48, S)
+    sl_i = np.zeros(B, np.int32)
+    sl_l = np.zeros(B, np.int32)
+    orc.identify_sinks(ic, np.zeros((B, T), np.float32), -np.inf, sl_i)
+    orc.append_prerope(ic, K.view(np.uint16), V.view(np.uint16), gh, perm, sl_i)
+    orc.append_prerope(lc, K.view(np.uint16), V.view(np.uint16), gh, perm, sl_l)
+    assert np.array_equal(ic.k_sink, lc.k_sink) and np.array_equal(ic.v_sink, lc.v_sink)
+    Q = rng.standard_normal((B, Hkv, D)).astype(np.float16).view(np.uint16)
+    o_i, _ = orc.decode_prerope(ic, Q, gh, perm, 10000.0, sl_i)
+    o_l, _ = orc.decode_prerope(lc, Q, gh, perm, 10000.0, sl_l)
+    assert np.array_equal(o_i, o_l)
+
+
+def test_prerope_identified_sinks_match_numpy_mini_oracle():
+    """Identified sinks at positions that are not their row numbers, in a
+    pre-RoPE cache: every sink is RoPE'd at its own position from its stored
+    pre-RoPE key, every other position from its dequantised, un-rotated
+    group row (independent numpy oracle), to 1e-12."""
+    rng = np.random.default_rng(77)
+    B, T, Hkv, gh, G, S, base = 1, 30, 2, 2, 1, 3, 10000.0
+    n = D * gh
+    K = (rng.standard_normal((B, T, Hkv, D)) * 2).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    perm = np.concatenate([rng.permutation(n), np.concatenate(
+        [rng.permutation(D) for _ in range(Hkv)])]).astype(np.int32).reshape(2, Hkv * D)
+    cache = orc.Cache(B, Hkv, 32, S, identified=True)
+    act = np.zeros((B, T), np.float32)
+    act[0, [4, 17, 23, 29]] = 1.0                   # four massive tokens, three rows
+    sl = np.zeros(B, np.int32)
+    orc.identify_sinks(cache, act, 0.5, sl)
+    assert list(cache.sink_pos[0]) == [4, 17, 23]
+    assert orc.append_prerope(cache, K.view(np.uint16), V.view(np.uint16), gh, perm, sl) == 0
+    Q = rng.standard_normal((B, Hkv * G, D)).astype(np.float16)
+    out, st = orc.decode_prerope(cache, Q.view(np.uint16), gh, perm, base, sl)
+    assert st == 0
+    sinks = [4, 17, 23]
+    khat = np.zeros((T, n))
+    for t in range(T):
+        if t in sinks:
+            continue
+        for jj in range(gh):
+            kb, vb, ks, kz, vs, vz = orc.load_token(cache.blocks[0, jj, t // 16], t % 16)
+            khat[t, jj * D:(jj + 1) * D] = np_mini.dequant(orc.unpack_row(kb), ks, kz)
+    for h in range(Hkv):
+        pv = perm[1, h * D:(h + 1) * D]
+        vhat = np.zeros((T, D))
+        for t in range(T):
+            kb, vb, ks, kz, vs, vz = orc.load_token(cache.blocks[0, h, t // 16], t % 16)
+            if t in sinks:
+                vhat[t] = cache.v_sink[0, h, sinks.index(t)].view(np.float16).astype(np.float64)
+                assert list(ks) == [0x7E00] * 4 and not kb.any()
+            else:
+                vhat[t] = np_mini.dequant(orc.unpack_row(vb), vs, vz)
+        keys = {t: K[0, t, h].astype(np.float64) for t in sinks}
+        ref = np_mini.decode_prerope_one(Q[0, h], khat, h, perm[0], base, vhat, pv, keys)
+        assert np.allclose(out[0, h], ref, rtol=0, atol=1e-12)
