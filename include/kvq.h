@@ -340,7 +340,10 @@ KVQ_API kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_
  *          plane 1 one value permutation of 0..127 per head (at
  *          perm + Hkv*128 + h*128).  16-B aligned.
  *   gh     1, 2, 4 or 8, dividing Hkv.
- * The cache must have no fp16 sinks (sink_fp16 == 0); paged caches are fine.
+ * Sinks, leading or identified (kvq_identify_sinks before the append), keep
+ * the key as given (fp16, pre-RoPE, unrotated) and the rotated value in their
+ * fp16 rows; the decode turns a sink key by RoPE at the sink's position.
+ * Paged caches are fine.
  */
 /* Append T tokens: K fp16 [B][T][Hkv][128] PRE-RoPE keys, V fp16 values
  * (same layout), 16-B aligned; seq_lens as in kvq_rotate_quantize_append. */
@@ -360,8 +363,8 @@ KVQ_API size_t kvq_prerope_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
  * group rotation of the dequantised keys), s_t = q . k_t / sqrt(128),
  * softmax, o_rot = sum p_t v_t over the rotated values, out = o_rot rotated
  * back (FWHT + value permutation).  Other arguments and errors as
- * kvq_decode_attention; KVQ_ERR_UNSUPPORTED for a cache with sinks or a
- * shape outside the limits above. */
+ * kvq_decode_attention; KVQ_ERR_UNSUPPORTED for a shape outside the limits
+ * above. */
 KVQ_API kvq_status kvq_prerope_decode(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
                                       int32_t group_heads, const int32_t *perm, float rope_base,
                                       const int32_t *seq_lens, int32_t max_ctx, void *workspace,

@@ -127,7 +127,6 @@ kvq_status kvq_prerope_append(const uint16_t *K, const uint16_t *V, int32_t T, i
                               void *stream) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
-    if (cache->sink_fp16 != 0 || cache->sink_pos) return KVQ_ERR_UNSUPPORTED;
     if (!gh_ok(group_heads, cache->Hkv)) return KVQ_ERR_UNSUPPORTED;
     if (!perm || T < 0 || !seq_lens || !aligned(seq_lens, 4)) return KVQ_ERR_INVALID_ARG;
     if (!aligned(perm, 16)) return KVQ_ERR_UNSUPPORTED;
@@ -153,7 +152,6 @@ kvq_status kvq_prerope_decode(const uint16_t *Q, int32_t Hq, const kvq_cache_des
                               size_t ws_bytes, uint16_t *out, void *stream) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
-    if (cache->sink_fp16 != 0 || cache->sink_pos) return KVQ_ERR_UNSUPPORTED;
     if (!gh_ok(group_heads, cache->Hkv)) return KVQ_ERR_UNSUPPORTED;
     if (!Q || !out || !seq_lens || !workspace || !perm) return KVQ_ERR_INVALID_ARG;
     if (!aligned(Q, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||

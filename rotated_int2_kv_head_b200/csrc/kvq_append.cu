@@ -21,10 +21,13 @@
 
 namespace kvq {
 
-// Epilogue shared by both append kernels: row (b, t, h, kind) with rotated
-// values v (lane layout of quantize_row_warp).
+// Epilogue shared by the append kernels: row (b, t, h, kind) with rotated
+// values v (lane layout of quantize_row_warp).  A sink stores v in fp16, or,
+// when raw is given, the lane's 4 halves of the row as it came in (the
+// pre-RoPE mode keeps sink keys unrotated).
 __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, int h, int kind,
-                                               int L0, const float v[4]) {
+                                               int L0, const float v[4],
+                                               const uint16_t *raw = nullptr) {
     const int lane = threadIdx.x & 31;
     const int p = L0 + t;
     const long long bi = cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, p / BLK_TOK);
@@ -36,8 +39,12 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
         uint16_t *sink = (kind == 0 ? c.k_sink : c.v_sink) +
                          (((size_t)b * c.Hkv + h) * c.S + (size_t)row) * D + 4 * lane;
         uint2 pk;
-        pk.x = pack_half2(v[0], v[1]);
-        pk.y = pack_half2(v[2], v[3]);
+        if (raw) {          // the row as given (pre-RoPE keys), the lane's 4 halves
+            pk = *reinterpret_cast<const uint2 *>(raw);
+        } else {
+            pk.x = pack_half2(v[0], v[1]);
+            pk.y = pack_half2(v[2], v[3]);
+        }
         *reinterpret_cast<uint2 *>(sink) = pk;
         if (bi >= 0) {
             // zero codes and meta; an identified sink's K meta carries the marker
@@ -243,7 +250,9 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
 // keys (n = 128*GH channels, contiguous in K) are reordered by the group's
 // permutation and transformed by an n-point FWHT / sqrt(n); each head's
 // 128-channel slice is quantized into its own cache unit.  Values are
-// rotated per head as in FWHT mode.  One warp per row: rows [0, nk) are key
+// rotated per head as in FWHT mode.  A sink keeps its key as given (fp16,
+// pre-RoPE: the decode turns it by RoPE at its position) and its rotated
+// value.  One warp per row: rows [0, nk) are key
 // groups (b, t, group), rows [nk, nk + nv) value rows (b, t, h).  Lane l
 // holds the group elements j*128 + 4l + k (j < GH, k < 4): the FWHT stages
 // over k and l are fwht128_warp's, the ones over j run in registers (the
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_prerope_kernel(PreRopeRow
 #pragma unroll
                 for (int k = 0; k < 4; k++) v[j][k] *= sc;
                 if (TO_CACHE)
-                    cache_epilogue(c, b, t, hh * GH + j, 0, L0, v[j]);
+                    cache_epilogue(c, b, t, hh * GH + j, 0, L0, v[j], &xs[warp][j * D + 4 * lane]);
                 else
                     *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * n + j * D + 4 * lane) =
                         make_float4(v[j][0], v[j][1], v[j][2], v[j][3]);

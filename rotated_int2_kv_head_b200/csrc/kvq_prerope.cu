@@ -21,8 +21,10 @@
 //       and dotted with each query head; online softmax and P.V on the
 //       dequantised rotated values.  Each CTA leaves one partial
 //       (m, l, o_rot[128]) per query head.
-//   prerope_merge_kernel  per (b, query head): merges the partials and
-//       removes the value rotation (FWHT + inverse permutation).
+//   prerope_merge_kernel  per (b, query head): the partial over the fp16
+//       sinks ("RotateKV", item (iii); keys kept pre-RoPE and turned at their
+//       positions), the merge of all partials, and the removal of the value
+//       rotation (FWHT + inverse permutation).
 // The RoPE angle t * theta_f is taken as 2 pi * frac(t * theta_f / (2 pi))
 // in fp64 at a warp's first token in every 16-token block (theta_f / (2 pi) comes from
 // the host in fp64), then advanced token by token with the rotation by
@@ -37,6 +39,10 @@ constexpr int PR_PART = 132;           // m, l, 0, 0, o[128]
 constexpr int PR_MIN_BLOCKS = 8;       // cache blocks per split at least
 constexpr float PR_LOG2E = 1.4426950408889634f;
 #define PR_NEG_INF (__int_as_float(0xff800000))
+// Start of a running max: finite, below any score, so exp2(score - max) is
+// never exp2(-inf - -inf); a run without tokens keeps it with l = 0, o = 0,
+// which every merge weights by exp2(PR_M0 - max) = 0 (or carries as zeros).
+constexpr float PR_M0 = -1.0e30f;
 
 // The four 2-bit codes of a lane (bits 2*g4 of the bytes of w) as exact
 // floats: each byte is put under the exponent of 2^23 and 2^23 subtracted.
@@ -57,6 +63,12 @@ struct PreRopeArgs {
     int32_t *status;
     float *part;                // [B*Hq][nsplit][PR_PART]
     uint16_t *out;              // [B][Hq][128]
+    // fp16 sinks: rows [B][Hkv][Srows][128] (keys pre-RoPE as given, values
+    // rotated); leading sinks are positions < S, identified ones listed in
+    // sink_pos [B][Srows] (sink_count rows in use) with a NaN-marked INT2 slot
+    const uint16_t *k_sink, *v_sink;
+    const int32_t *sink_pos, *sink_count;
+    int S, Srows;
     int B, Hq, Hkv, capacity, nblk, nsplit, bps;
     double phi[D / 2];          // theta_f / (2 pi), theta_f = base^(-2f/128)
 };
@@ -122,7 +134,7 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
     float m_run[NQ], l_run[NQ], o[NQ][4];
 #pragma unroll
     for (int i = 0; i < NQ; i++) {
-        m_run[i] = PR_NEG_INF;
+        m_run[i] = PR_M0;
         l_run[i] = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; k++) o[i][k] = 0.f;
@@ -135,7 +147,8 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
 
     const int wi = lane & 7, g4 = lane >> 3;          // logical code word, quant group
     // the CTA's tokens in PR_WARPS contiguous, equal runs, one per warp
-    const int t_beg = min(L, blk0 * BLK_TOK), t_end = min(L, blk1 * BLK_TOK);
+    // (leading sinks are not INT2 tokens: they start at S)
+    const int t_beg = min(L, max(a.S, blk0 * BLK_TOK)), t_end = max(t_beg, min(L, blk1 * BLK_TOK));
     const int per = (t_end - t_beg + PR_WARPS - 1) / PR_WARPS;
     const int w0 = min(t_end, t_beg + warp * per), w1 = min(t_end, w0 + per);
     for (int blk = w0 / BLK_TOK; w0 < w1 && blk <= (w1 - 1) / BLK_TOK; blk++) {
@@ -250,6 +263,10 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
                               qr[i][3] * v[j][3];
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                    // an identified sink's slot (NaN scale) scores NaN: fmax with
+                    // -inf makes it -inf, whose weight below is exp2(-inf) = 0
+                    // (m_run starts at PR_M0, finite)
+                    d = fmaxf(d, PR_NEG_INF);
                     if (d > m_run[i]) {
                         const float al = exp2f(m_run[i] - d);   // 0 for the first token
                         l_run[i] *= al;
@@ -315,6 +332,7 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
 // threads per (b, query head).
 __global__ void __launch_bounds__(D) prerope_merge_kernel(PreRopeArgs a) {
     __shared__ __align__(16) float os[D];
+    __shared__ float red4[D / 32];
     const int hq = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
     const int h = hq / (a.Hq / a.Hkv);
     pdl_wait();
@@ -326,10 +344,59 @@ __global__ void __launch_bounds__(D) prerope_merge_kernel(PreRopeArgs a) {
         if (t == 0) set_status(a.status, KVQ_DEV_BAD_LEN);
         return;
     }
+    // ---- the fp16 sinks this query sees, scored on CUDA cores: the stored
+    // pre-RoPE key turned by RoPE at the sink's position (thread t = channel
+    // t, its pair partner t ^ 64), dotted with q; softmax partial over them
+    int ns = 0;
+    if (a.Srows > 0) {
+        if (!a.sink_pos) {
+            ns = min(a.S, L);
+        } else {
+            const int n = min(max(a.sink_count[b], 0), a.Srows);
+            for (int r = 0; r < n; r++) ns += a.sink_pos[(size_t)b * a.Srows + r] < L ? 1 : 0;
+        }
+    }
+    float sm = PR_NEG_INF, sl = 0.f, so = 0.f;
+    if (ns > 0) {
+        const size_t uh = (size_t)b * a.Hkv + h;
+        const uint16_t *ks = a.k_sink + uh * a.Srows * D;
+        const uint16_t *vs = a.v_sink + uh * a.Srows * D;
+        const float qv = __half2float(__ushort_as_half(a.Q[((size_t)b * a.Hq + hq) * D + t])) *
+                         (PR_LOG2E * 0.08838834764831845f);
+        const double ph = a.phi[t & (D / 2 - 1)];
+        const float sgn = t < D / 2 ? -1.f : 1.f;
+        const int lane = t & 31, warp = t >> 5;
+        for (int r = 0; r < ns; r++) {
+            const int pos = a.sink_pos ? a.sink_pos[(size_t)b * a.Srows + r] : r;
+            const double u = (double)pos * ph;
+            float sn, cs;
+            sincospif((float)(2.0 * (u - floor(u))), &sn, &cs);
+            const float x = __half2float(__ushort_as_half(ks[(size_t)r * D + t]));
+            const float xp = __half2float(__ushort_as_half(ks[(size_t)r * D + (t ^ (D / 2))]));
+            float d = qv * fmaf(sgn * xp, sn, x * cs);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            if (lane == 0) red4[warp] = d;
+            __syncthreads();
+            const float sc = red4[0] + red4[1] + red4[2] + red4[3];
+            __syncthreads();
+            const float mnew = fmaxf(sm, sc);
+            const float al = sm == PR_NEG_INF ? 0.f : exp2f(sm - mnew);
+            const float p = exp2f(sc - mnew);
+            sl = fmaf(sl, al, p);
+            so = fmaf(so, al, p * __half2float(__ushort_as_half(vs[(size_t)r * D + t])));
+            sm = mnew;
+        }
+    }
     const float *pp = a.part + ((size_t)b * a.Hq + hq) * a.nsplit * PR_PART;
-    float mx = PR_NEG_INF;
+    float mx = sm;
     for (int s = 0; s < a.nsplit; s++) mx = fmaxf(mx, pp[(size_t)s * PR_PART]);
     float lt = 0.f, ot = 0.f;
+    if (sm != PR_NEG_INF) {
+        const float f = exp2f(sm - mx);
+        lt = f * sl;
+        ot = f * so;
+    }
     for (int s = 0; s < a.nsplit; s++) {
         const float ms = pp[(size_t)s * PR_PART];
         if (ms == PR_NEG_INF) continue;                     // a split without tokens
@@ -374,6 +441,12 @@ cudaError_t launch_decode_prerope(const uint16_t *Q, int Hq, const kvq_cache_des
     a.status = cd.status;
     a.part = static_cast<float *>(ws);
     a.out = out;
+    a.k_sink = cd.k_sink;
+    a.v_sink = cd.v_sink;
+    a.sink_pos = cd.sink_pos;
+    a.sink_count = cd.sink_count;
+    a.Srows = cd.sink_fp16;
+    a.S = cd.sink_pos ? 0 : cd.sink_fp16;
     a.B = cd.B;
     a.Hq = Hq;
     a.Hkv = cd.Hkv;

@@ -236,13 +236,81 @@ def test_prerope_bad_length_and_unsupported():
     torch.cuda.synchronize()
     assert not out.float().abs().sum().item()
     assert kvq.kvq_get_status(cache) == kvq.KVQ_DEV_BAD_LEN
-    sinks = kvq.KVCache(2, 2, 64, 4)
-    ws = kvq.prerope_workspace(2, 2, 2, 1, 64)
-    with pytest.raises(kvq.KvqError) as e:
-        kvq.kvq_prerope_decode(Q, sinks, 1, perm, BASE, sl, 64, ws, out)
-    assert e.value.code == 2
     with pytest.raises(kvq.KvqError) as e:                       # G * gh > 8
         Q8 = torch.randn((2, 16, D), device="cuda").half()
         kvq.kvq_prerope_decode(Q8, cache, 2, perm, BASE, sl, 64,
                                kvq.prerope_workspace(2, 16, 2, 2, 64), torch.empty_like(Q8))
     assert e.value.code == 2
+
+
+# --- with fp16 sinks (RotateKV items ii and iii together) -----------------------------------------
+
+@pytest.mark.parametrize("identified", [False, True])
+def test_prerope_sinks_append_and_decode(identified):
+    """Leading sinks (the first 4 positions) or identified ones (massive
+    tokens): sink rows hold the pre-RoPE key exactly as given and the fp16
+    of the kernel's rotated value; INT2 slots zero (identified: the K-scale
+    marker); the decode against the oracle over appends of 37, 300 and 1
+    tokens."""
+    gh, G, Hkv, B, S = 2, 2, 4, 3, 4
+    w = W.custom(seed=280 + identified, B=B, Hq=Hkv * G, Hkv=Hkv, mode=1, sink=S, k_outliers=4,
+                 sink_key_scale=50.0, massive_rate=0.01 if identified else 0.0)
+    perm = W.prerope_perm(w, gh)
+    pt = torch.from_numpy(perm).cuda()
+    L0 = [0, 2, 16]
+    chunks = [37, 300, 1]
+    cap = ((max(L0) + sum(chunks) + 15) // 16) * 16
+    cache = kvq.KVCache(B, Hkv, cap, S, identified_sinks=identified)
+    oc = orc.Cache(B, Hkv, cap, S, identified=identified)
+    sl = torch.tensor(L0, dtype=torch.int32, device="cuda")
+    osl = np.array(L0, np.int32)
+    pos = list(L0)
+    Ks, Vs = [], []
+    for T in chunks:
+        K = torch.stack([W.kv_rows(w, b, pos[b], pos[b] + T, "cpu")[0] for b in range(B)])
+        V = torch.stack([W.kv_rows(w, b, pos[b], pos[b] + T, "cpu")[1] for b in range(B)])
+        if identified:
+            act = np.stack([W.activations(w, b, pos[b], pos[b] + T) for b in range(B)])
+            kvq.kvq_identify_sinks(torch.from_numpy(act).cuda(), W.MASSIVE_TAU, cache, sl)
+            orc.identify_sinks(oc, act, W.MASSIVE_TAU, osl)
+        kvq.kvq_prerope_append(K.cuda(), V.cuda(), gh, pt, cache, sl)
+        assert orc.append_prerope(oc, f16bits(K), f16bits(V), gh, perm, osl) == 0
+        Ks.append((list(pos), K, V))
+        pos = [p + T for p in pos]
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    if identified:
+        assert np.array_equal(cache.sink_count.cpu().numpy(), oc.sink_count)
+        assert np.array_equal(cache.sink_pos.cpu().numpy(), oc.sink_pos)
+        assert (oc.sink_count >= 1).all()
+    gks, gvs = f16bits(cache.k_sink), f16bits(cache.v_sink)
+    gb = cache.block_view().cpu().numpy()
+    n_sink = 0
+    for starts, K, V in Ks:
+        T = K.shape[1]
+        for h in range(Hkv):
+            vrot = kvq.kvq_debug_rotate_f32(V[:, :, h].reshape(-1, D).cuda(), 1, perm=torch.from_numpy(
+                np.ascontiguousarray(perm[1, h * D:(h + 1) * D])).cuda()).cpu().numpy().reshape(B, T, D)
+            for b in range(B):
+                plist = (list(oc.sink_pos[b, :oc.sink_count[b]]) if identified
+                         else list(range(S)))
+                for t in range(T):
+                    p = starts[b] + t
+                    if p not in plist:
+                        continue
+                    j = plist.index(p)
+                    assert np.array_equal(gks[b, h, j], f16bits(K[b, t, h]))
+                    assert np.array_equal(gvs[b, h, j], orc.f32_to_f16_bits(vrot[b, t]))
+                    kb, vb, ks, kz, vs, vz = orc.load_token(gb[b, h, p // 16], p % 16)
+                    assert not kb.any() and not vb.any() and not kz.any() and not vs.any()
+                    assert list(ks) == ([0x7E00] * 4 if identified else [0] * 4)
+                    n_sink += 1
+    assert n_sink > 0
+    Q = W.queries(w, "cpu")
+    ref, st = orc.decode_prerope(oc, f16bits(Q), gh, perm, BASE, osl, n_threads=8)
+    assert st == 0
+    out = gpu_prerope_decode(cache, Q.cuda(), gh, pt, sl, max(pos))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    err = rel_err(out.cpu().numpy(), ref)
+    assert err.max() <= DEC_TOL, err.max()
