@@ -122,8 +122,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
-// 3-D tiled TMA load (no multicast) of box {64, 1, 128} at coordinates
-// (c0, c1, c2) into 1024-byte aligned shared memory, completion on `bar`.
+// 3-D tiled TMA load of box {64, 1, 128} at coordinates (c0, c1, c2) into
+// this CTA's own 1024-byte aligned shared memory, completion on `bar`.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
                                             uint64_t *bar) {
     asm volatile(
