@@ -160,3 +160,101 @@ def test_ragged_prefill_append_full():
             n_diff += int((oc[0] != got_c).sum())
             n_codes += 128
     assert n_diff <= max(2, 1e-4 * n_codes), (n_diff, n_codes)
+
+
+def test_gqa_sinks_identified_full():
+    """gqa_sinks with its fp16 rows given to the massive tokens (identified
+    before each chunk is appended), at full size; the oracle identifies and
+    appends the sampled units' tokens from the same activations and rows."""
+    w = W.WORKLOADS["gqa_sinks_identified"]
+    dev = "cuda"
+    L = int(w.context)
+    Rk, Rv, _ = W.rotations(w)
+    rk, rv = torch.from_numpy(Rk).to(dev), torch.from_numpy(Rv).to(dev)
+    cache = kvq.KVCache(w.B, w.Hkv, L, w.sink, identified_sinks=True)
+    sl = torch.zeros(w.B, dtype=torch.int32, device=dev)
+    samples = [(0, 0), (5, 7)]
+    keep = {u: ([], []) for u in samples}
+    for t0 in range(0, L, 8192):
+        t1 = min(L, t0 + 8192)
+        K, V = W.kv_batch(w, t0, t1, dev)
+        act = np.stack([W.activations(w, b, t0, t1) for b in range(w.B)])
+        kvq.kvq_identify_sinks(torch.from_numpy(act).to(dev), W.MASSIVE_TAU, cache, sl)
+        kvq.kvq_rotate_quantize_append(K, V, 0, rk, rv, None, cache, sl)
+        for (b, h), (kl, vl) in keep.items():
+            kl.append(W.f16_bits(K[b, :, h]))
+            vl.append(W.f16_bits(V[b, :, h]))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    lens = torch.full((w.B,), L, dtype=torch.int32, device=dev)
+    Q = W.queries(w, dev)
+    ws = kvq.decode_workspace(w.B, w.Hq, w.Hkv, L)
+    ws.fill_(0xFF)
+    out = torch.empty_like(Q)
+    kvq.kvq_decode_attention(Q, cache, 0, rk, rv, None, lens, w.sink, L, ws, out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0 and torch.isfinite(out).all()
+    out = out.float().cpu().numpy()
+    Qh = W.f16_bits(Q)
+    counts = cache.sink_count.cpu().numpy()
+    for (b, h), (kl, vl) in keep.items():
+        oc = orc.Cache(1, 1, L, w.sink, identified=True)
+        s1 = np.zeros(1, np.int32)
+        orc.identify_sinks(oc, W.activations(w, b, 0, L)[None], W.MASSIVE_TAU, s1)
+        assert oc.sink_count[0] == counts[b]
+        assert np.array_equal(oc.sink_pos[0], cache.sink_pos[b].cpu().numpy())
+        orc.append(oc, np.concatenate(kl).reshape(1, L, 1, 128),
+                   np.concatenate(vl).reshape(1, L, 1, 128), 0, Rk[h:h + 1], Rv[h:h + 1], None, s1)
+        ref, st = orc.decode(oc, Qh[b:b + 1, h * w.G:(h + 1) * w.G], 0, Rk[h:h + 1], Rv[h:h + 1],
+                             None, np.array([L], np.int32), n_threads=8)
+        assert st == 0
+        err = rel_err(out[b, h * w.G:(h + 1) * w.G], ref[0])
+        assert err.max() <= DEC_TOL, ((b, h), err.max())
+
+
+@pytest.mark.parametrize("gh", [1, 4])
+def test_prerope_llama7b_full(gh):
+    """Pre-RoPE keys on the llama7b shape (B=1, 32 heads, context 32768),
+    appended in 4096-token chunks; sampled head groups against the oracle's
+    append + decode of the same rows (the oracle cache holds the group's gh
+    heads)."""
+    w = W.custom(name="llama7b_prerope", seed=1002, B=1, Hq=32, Hkv=32, mode=1, context=32768,
+                 k_outliers=8)
+    dev = "cuda"
+    L, base = 32768, 10000.0
+    perm = W.prerope_perm(w, gh)
+    pt = torch.from_numpy(perm).to(dev)
+    cache = kvq.KVCache(1, 32, L)
+    sl = torch.zeros(1, dtype=torch.int32, device=dev)
+    groups = [0, 32 // gh - 1]
+    keep = {q: ([], []) for q in groups}
+    for t0 in range(0, L, 4096):
+        K, V = W.kv_batch(w, t0, t0 + 4096, dev)
+        kvq.kvq_prerope_append(K, V, gh, pt, cache, sl)
+        for q, (kl, vl) in keep.items():
+            kl.append(W.f16_bits(K[0, :, q * gh:(q + 1) * gh]))
+            vl.append(W.f16_bits(V[0, :, q * gh:(q + 1) * gh]))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0
+    Q = W.queries(w, dev)
+    ws = kvq.prerope_workspace(1, 32, 32, gh, L)
+    ws.fill_(0xFF)
+    out = torch.empty_like(Q)
+    kvq.kvq_prerope_decode(Q, cache, gh, pt, base, sl, L, ws, out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0 and torch.isfinite(out).all()
+    out = out.float().cpu().numpy()
+    Qh = W.f16_bits(Q)
+    for q, (kl, vl) in keep.items():
+        n = 128 * gh
+        psub = np.stack([perm[0, q * n:(q + 1) * n],
+                         perm[1, q * n:(q + 1) * n]]).astype(np.int32)   # Hkv=gh: n entries each
+        oc = orc.Cache(1, gh, L, 0)
+        s1 = np.zeros(1, np.int32)
+        orc.append_prerope(oc, np.concatenate(kl).reshape(1, L, gh, 128),
+                           np.concatenate(vl).reshape(1, L, gh, 128), gh, psub, s1)
+        ref, st = orc.decode_prerope(oc, Qh[:, q * gh:(q + 1) * gh], gh, psub, base, s1,
+                                     n_threads=8)
+        assert st == 0
+        err = rel_err(out[0, q * gh:(q + 1) * gh], ref[0])
+        assert err.max() <= DEC_TOL, (q, err.max())
