@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(DENSE_THREADS)
 // ---- permutation + FWHT ---------------------------------------------------------------------
 // One warp per row: y[i] = x[perm[i]], y <- FWHT(y) / sqrt(128).
 constexpr int FWHT_THREADS = 256;
+constexpr int FWHT_ROWS = FWHT_THREADS / 4;   // rows per CTA: four threads per row
 
 struct FwhtRows {
     const uint16_t *X0, *X1;   // K, V (cache) or X (debug)
@@ -189,16 +190,24 @@ struct FwhtRows {
     long long n_rows;          // cache: B*T*Hkv*2 ; debug: N
 };
 
+// Four threads per row.  Thread q (0..3) owns elements 32q..32q+31 of the
+// rotated row, which is exactly quantization group q: the FWHT's five
+// stages over index bits 0..4 run in its registers, the two over bits 5 and
+// 6 across the row's four threads (consecutive lanes: shuffles xor 1 and 2,
+// each butterfly one fma with a per-thread sign), and then the thread
+// quantizes its group alone (quantize_group_thread); the row's code words
+// are OR-ed together over its four threads.  The row is gathered through
+// the permutation from shared memory.  Cache: CTA (bt, y) takes token
+// bt = b*T + t and the (head, kind) pairs 64y .. 64y+63 (kind fastest);
+// debug: rows 64x .. 64x+63.
 template <bool TO_CACHE>
 __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, CacheDst c) {
-    __shared__ __align__(16) uint16_t xs[FWHT_THREADS / 32][D];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ __align__(16) uint16_t xs[FWHT_ROWS][D];
+    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
     pdl_wait();
     pdl_trigger();
-    // cache: CTA (bt, y) takes token bt = b*T + t, warp w the (head, kind)
-    // pair 8y + w (kind fastest); debug: one row per warp
-    const long long row = TO_CACHE ? 0 : (long long)blockIdx.x * (FWHT_THREADS / 32) + warp;
-    const int hk = TO_CACHE ? (int)blockIdx.y * (FWHT_THREADS / 32) + warp : 0;
+    const long long row = TO_CACHE ? 0 : (long long)blockIdx.x * FWHT_ROWS + r;
+    const int hk = TO_CACHE ? (int)blockIdx.y * FWHT_ROWS + r : 0;
     bool active = TO_CACHE ? hk < 2 * c.Hkv : row < a.n_rows;
     int b = 0, t = 0, h = 0, kind = 0, L0 = 0;
     const uint16_t *src = nullptr;
@@ -208,40 +217,114 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
         h = hk >> 1;
         b = (int)(blockIdx.x / (unsigned)c.T);
         t = (int)(blockIdx.x - (unsigned)b * (unsigned)c.T);
-        const int L = c.seq_lens[b];
-        if (L < 0 || (long long)L + c.T > c.capacity) {
-            if (lane == 0 && t == 0 && h == 0 && kind == 0)
-                set_status(c.status, L < 0 ? KVQ_DEV_BAD_LEN : KVQ_DEV_CAPACITY);
-            active = false;
-        }
-        L0 = L;
+        L0 = start_len_thread(c, b, q == 0 && t == 0 && h == 0 && kind == 0);
+        if (L0 < 0) active = false;
         src = (kind == 0 ? a.X0 : a.X1) + (((size_t)b * c.T + t) * c.Hkv + h) * D;
         perm = a.perm + ((size_t)kind * c.Hkv + h) * D;
     } else if (active) {
         src = a.X0 + (size_t)row * D;
         perm = a.perm;
     }
+    // stage the row (thread q copies 64 of its 256 bytes)
     if (active) {
-        *reinterpret_cast<uint2 *>(&xs[warp][4 * lane]) =
-            *reinterpret_cast<const uint2 *>(src + 4 * lane);
-        const int4 pi = *reinterpret_cast<const int4 *>(perm + 4 * lane);
-        __syncwarp();
-        float v[4];
-        v[0] = __half2float(__ushort_as_half(xs[warp][pi.x & (D - 1)]));
-        v[1] = __half2float(__ushort_as_half(xs[warp][pi.y & (D - 1)]));
-        v[2] = __half2float(__ushort_as_half(xs[warp][pi.z & (D - 1)]));
-        v[3] = __half2float(__ushort_as_half(xs[warp][pi.w & (D - 1)]));
-        fwht128_warp(v);
-        const float inv_sqrt_d = 0.08838834764831845f;
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src) + 4 * q;
+        uint4 *d4 = reinterpret_cast<uint4 *>(&xs[r][0]) + 4 * q;
 #pragma unroll
-        for (int k = 0; k < 4; k++) v[k] *= inv_sqrt_d;
-        if (TO_CACHE)
-            cache_epilogue(c, b, t, h, kind, L0, v);
-        else
-            *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
-                make_float4(v[0], v[1], v[2], v[3]);
+        for (int i = 0; i < 4; i++) d4[i] = s4[i];
     }
-    if (TO_CACHE) append_done(c);
+    __syncwarp();
+    // every lane takes part in the shuffles; a row out of range computes zeros
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        int4 pi = make_int4(0, 0, 0, 0);
+        if (active) pi = *reinterpret_cast<const int4 *>(perm + 32 * q + 4 * i);
+        v[4 * i] = active ? __half2float(__ushort_as_half(xs[r][pi.x & (D - 1)])) : 0.f;
+        v[4 * i + 1] = active ? __half2float(__ushort_as_half(xs[r][pi.y & (D - 1)])) : 0.f;
+        v[4 * i + 2] = active ? __half2float(__ushort_as_half(xs[r][pi.z & (D - 1)])) : 0.f;
+        v[4 * i + 3] = active ? __half2float(__ushort_as_half(xs[r][pi.w & (D - 1)])) : 0.f;
+    }
+#pragma unroll
+    for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+        for (int e = 0; e < 32; e++)
+            if ((e & st) == 0) {
+                const float x0 = v[e], x1 = v[e + st];
+                v[e] = x0 + x1;
+                v[e + st] = x0 - x1;
+            }
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1) {
+        const float sgn = (q & m) ? -1.f : 1.f;
+#pragma unroll
+        for (int e = 0; e < 32; e++) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+            v[e] = fmaf(sgn, v[e], o);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
+
+    if (!TO_CACHE) {
+        if (active) {
+            float *dst = a.out_f32 + (size_t)row * D + 32 * q;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+        return;
+    }
+    uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint32_t meta = quantize_group_thread(v, q, words);
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        words[w] |= __shfl_xor_sync(0xffffffffu, words[w], 1);
+        words[w] |= __shfl_xor_sync(0xffffffffu, words[w], 2);
+    }
+    if (active) {
+        const int p = L0 + t;
+        const long long bi = cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, p / BLK_TOK);
+        if (bi < 0 && q == 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+        uint8_t *block = c.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
+        const int tau = p % BLK_TOK;
+        const int srow = sink_row(c, b, p);
+        if (srow >= 0) {
+            // a sink: the rotated row in fp16; its slot zero (identified: K marker)
+            uint16_t *dst = (kind == 0 ? c.k_sink : c.v_sink) +
+                            (((size_t)b * c.Hkv + h) * c.S + (size_t)srow) * D + 32 * q;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+                *reinterpret_cast<uint4 *>(dst + e) =
+                    make_uint4(pack_half2(v[e], v[e + 1]), pack_half2(v[e + 2], v[e + 3]),
+                               pack_half2(v[e + 4], v[e + 5]), pack_half2(v[e + 6], v[e + 7]));
+#pragma unroll
+            for (int w = 0; w < 8; w++) words[w] = 0u;
+            meta = (c.sink_pos && kind == 0) ? SINK_KMETA_MARK : 0u;
+        }
+        // thread q stores code words 2q and 2q+1 (selected without indexing
+        // the array by a runtime value, which would put it in local memory)
+        uint32_t wa = words[0], wb = words[1];
+#pragma unroll
+        for (int k = 1; k < 4; k++)
+            if (q == k) {
+                wa = words[2 * k];
+                wb = words[2 * k + 1];
+            }
+        if (bi >= 0) {
+            if (kind == 0) {
+                *reinterpret_cast<uint32_t *>(block + off_kword(tau, 2 * q)) = wa;
+                *reinterpret_cast<uint32_t *>(block + off_kword(tau, 2 * q + 1)) = wb;
+                *reinterpret_cast<uint32_t *>(block + off_kmeta(tau, q)) = meta;
+            } else {                                    // 16-bit pieces 4q .. 4q+3
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q)) = (uint16_t)wa;
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 1)) = (uint16_t)(wa >> 16);
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 2)) = (uint16_t)wb;
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 3)) = (uint16_t)(wb >> 16);
+                *reinterpret_cast<uint32_t *>(block + off_vmeta(tau, q)) = meta;
+            }
+        }
+    }
+    append_done(c);
 }
 
 // ---- pre-RoPE grouped-head key rotation ----------------------------------------------------------
@@ -511,9 +594,8 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.perm = perm;
         a.out_f32 = nullptr;
         a.n_rows = (long long)cd.B * T * cd.Hkv * 2;
-        const int per = FWHT_THREADS / 32;
         return launch_pdl(append_fwht_kernel<true>,
-                          dim3((unsigned)((long long)cd.B * T), (2 * cd.Hkv + per - 1) / per),
+                          dim3((unsigned)((long long)cd.B * T), (2 * cd.Hkv + FWHT_ROWS - 1) / FWHT_ROWS),
                           dim3(FWHT_THREADS), 0, st, a, c);
     }
 }
@@ -535,8 +617,7 @@ cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const 
         a.perm = perm;
         a.out_f32 = out;
         a.n_rows = N;
-        const int per = FWHT_THREADS / 32;
-        append_fwht_kernel<false><<<(N + per - 1) / per, FWHT_THREADS, 0, st>>>(a, c);
+        append_fwht_kernel<false><<<(N + FWHT_ROWS - 1) / FWHT_ROWS, FWHT_THREADS, 0, st>>>(a, c);
     }
     return cudaGetLastError();
 }

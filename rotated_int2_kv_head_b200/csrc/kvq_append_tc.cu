@@ -173,60 +173,8 @@ __device__ __forceinline__ void convert_r(const float *R, uint8_t *bhi, uint8_t 
     }
 }
 
-// The exact group quantizer on one thread's 32 values of group g: codes go
-// into byte e of words (bits 2g, 2g+1), scale and zero are returned as fp16
-// bits.  Same results as quantize_row_warp: s = fp16((max - min) / 3),
-// z = fp16(min), c = clamp(rint(fp32(fp32(x - z) * inv)), 0, 3).
-//
-// Per element: clamp to [0, 3] first (clamping then rounding equals rounding
-// then clamping on that interval), then add 1.5 * 2^23: fp32 round-to-
-// nearest-even leaves rint(t) in the low mantissa bits, so the sum's bit
-// pattern is 0x4B400000 + c.  That pattern, shifted to the code's place, is
-// added into the word (one integer multiply-add; the codes' bits never
-// overlap), and the constant 0x4B400000-terms are taken out once per word.
-__device__ __forceinline__ uint32_t quantize_group_thread(const float (&v)[32], int g,
-                                                          uint32_t (&words)[8]) {
-    // min and max of the 32 values with three-input min/max: 32 -> 12 -> 4 -> 1
-    float mn[12], mx[12];
-#pragma unroll
-    for (int e = 0; e < 10; e++) {
-        mn[e] = fmin3(v[3 * e], v[3 * e + 1], v[3 * e + 2]);
-        mx[e] = fmax3(v[3 * e], v[3 * e + 1], v[3 * e + 2]);
-    }
-    mn[10] = v[30], mn[11] = v[31], mx[10] = v[30], mx[11] = v[31];
-#pragma unroll
-    for (int e = 0; e < 4; e++) {
-        mn[e] = fmin3(mn[3 * e], mn[3 * e + 1], mn[3 * e + 2]);
-        mx[e] = fmax3(mx[3 * e], mx[3 * e + 1], mx[3 * e + 2]);
-    }
-    mn[0] = fminf(fmin3(mn[0], mn[1], mn[2]), mn[3]);
-    mx[0] = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-    const float r = __fsub_rn(mx[0], mn[0]);
-    const float sf = __fdiv_rn(r, 3.0f);
-    const __half s = __float2half_rn(__fadd_rn(sf, 0.0f));   // zero stored as +0
-    const __half z = __float2half_rn(__fadd_rn(mn[0], 0.0f));
-    const float sF = __half2float(s), zF = __half2float(z);
-    const float inv = (sF == 0.0f) ? 0.0f : __frcp_rn(sF);   // = the IEEE quotient 1/s
-    constexpr float MAGIC = 12582912.0f;                     // 1.5 * 2^23
-    constexpr uint32_t MAGIC_BITS = 0x4B400000u;
-#pragma unroll
-    for (int w = 0; w < 8; w++) {
-        uint32_t acc = words[w];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int e = 4 * w + j;
-            float t = __fmul_rn(__fsub_rn(v[e], zF), inv);
-            t = fminf(fmaxf(t, 0.0f), 3.0f);
-            const uint32_t bits = __float_as_uint(__fadd_rn(t, MAGIC));
-            acc += bits << (8 * j + 2 * g);
-        }
-        // remove sum_j (MAGIC_BITS << (8j + 2g)) (mod 2^32)
-        acc -= (MAGIC_BITS << (2 * g)) + (MAGIC_BITS << (8 + 2 * g)) + (MAGIC_BITS << (16 + 2 * g)) +
-               (MAGIC_BITS << (24 + 2 * g));
-        words[w] = acc;
-    }
-    return (uint32_t)__half_as_ushort(s) | ((uint32_t)__half_as_ushort(z) << 16);
-}
+// The epilogue quantizes one row per thread with quantize_group_thread
+// (kvq_internal.cuh), group by group.
 
 template <bool TO_CACHE>
 __global__ void __launch_bounds__(tc::THREADS, 1)
