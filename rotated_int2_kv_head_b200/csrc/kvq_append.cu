@@ -182,6 +182,10 @@ __global__ void __launch_bounds__(DENSE_THREADS)
 // One warp per row: y[i] = x[perm[i]], y <- FWHT(y) / sqrt(128).
 constexpr int FWHT_THREADS = 256;
 constexpr int FWHT_ROWS = FWHT_THREADS / 4;   // rows per CTA: four threads per row
+// Staged rows are 272 bytes apart: the 8 rows of a warp that gather the same
+// permuted index then fall in 8 different shared-memory banks (at 256 bytes
+// they would all share one).
+constexpr int XS_STRIDE = D + 8;
 
 struct FwhtRows {
     const uint16_t *X0, *X1;   // K, V (cache) or X (debug)
@@ -189,6 +193,44 @@ struct FwhtRows {
     float *out_f32;
     long long n_rows;          // cache: B*T*Hkv*2 ; debug: N
 };
+
+// Thread q (0..3) of a row staged in shared memory: its 32 elements of
+// FWHT(x[perm]) / sqrt(128), elements 32q .. 32q+31 (quantization group q).
+// Five butterfly stages run in registers, the two over index bits 5 and 6
+// across the row's four consecutive lanes.  Every lane of the warp calls it
+// (shuffles); a row that is not active computes zeros.
+__device__ __forceinline__ void fwht_row_quarter(const uint16_t *xrow, const int32_t *perm,
+                                                 bool active, int q, float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        int4 pi = make_int4(0, 0, 0, 0);
+        if (active) pi = *reinterpret_cast<const int4 *>(perm + 32 * q + 4 * i);
+        v[4 * i] = active ? __half2float(__ushort_as_half(xrow[pi.x & (D - 1)])) : 0.f;
+        v[4 * i + 1] = active ? __half2float(__ushort_as_half(xrow[pi.y & (D - 1)])) : 0.f;
+        v[4 * i + 2] = active ? __half2float(__ushort_as_half(xrow[pi.z & (D - 1)])) : 0.f;
+        v[4 * i + 3] = active ? __half2float(__ushort_as_half(xrow[pi.w & (D - 1)])) : 0.f;
+    }
+#pragma unroll
+    for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+        for (int e = 0; e < 32; e++)
+            if ((e & st) == 0) {
+                const float x0 = v[e], x1 = v[e + st];
+                v[e] = x0 + x1;
+                v[e + st] = x0 - x1;
+            }
+#pragma unroll
+    for (int m = 1; m < 4; m <<= 1) {
+        const float sgn = (q & m) ? -1.f : 1.f;
+#pragma unroll
+        for (int e = 0; e < 32; e++) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+            v[e] = fmaf(sgn, v[e], o);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
+}
 
 // Four threads per row.  Thread q (0..3) owns elements 32q..32q+31 of the
 // rotated row, which is exactly quantization group q: the FWHT's five
@@ -202,7 +244,7 @@ struct FwhtRows {
 // debug: rows 64x .. 64x+63.
 template <bool TO_CACHE>
 __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, CacheDst c) {
-    __shared__ __align__(16) uint16_t xs[FWHT_ROWS][D];
+    __shared__ __align__(16) uint16_t xs[FWHT_ROWS][XS_STRIDE];
     const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
     pdl_wait();
     pdl_trigger();
@@ -233,37 +275,8 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
         for (int i = 0; i < 4; i++) d4[i] = s4[i];
     }
     __syncwarp();
-    // every lane takes part in the shuffles; a row out of range computes zeros
     float v[32];
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        int4 pi = make_int4(0, 0, 0, 0);
-        if (active) pi = *reinterpret_cast<const int4 *>(perm + 32 * q + 4 * i);
-        v[4 * i] = active ? __half2float(__ushort_as_half(xs[r][pi.x & (D - 1)])) : 0.f;
-        v[4 * i + 1] = active ? __half2float(__ushort_as_half(xs[r][pi.y & (D - 1)])) : 0.f;
-        v[4 * i + 2] = active ? __half2float(__ushort_as_half(xs[r][pi.z & (D - 1)])) : 0.f;
-        v[4 * i + 3] = active ? __half2float(__ushort_as_half(xs[r][pi.w & (D - 1)])) : 0.f;
-    }
-#pragma unroll
-    for (int st = 1; st < 32; st <<= 1)
-#pragma unroll
-        for (int e = 0; e < 32; e++)
-            if ((e & st) == 0) {
-                const float x0 = v[e], x1 = v[e + st];
-                v[e] = x0 + x1;
-                v[e + st] = x0 - x1;
-            }
-#pragma unroll
-    for (int m = 1; m < 4; m <<= 1) {
-        const float sgn = (q & m) ? -1.f : 1.f;
-#pragma unroll
-        for (int e = 0; e < 32; e++) {
-            const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
-            v[e] = fmaf(sgn, v[e], o);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
+    fwht_row_quarter(xs[r], perm, active, q, v);
 
     if (!TO_CACHE) {
         if (active) {
@@ -321,6 +334,111 @@ __global__ void __launch_bounds__(FWHT_THREADS) append_fwht_kernel(FwhtRows a, C
                 *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 2)) = (uint16_t)wb;
                 *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 3)) = (uint16_t)(wb >> 16);
                 *reinterpret_cast<uint32_t *>(block + off_vmeta(tau, q)) = meta;
+            }
+        }
+    }
+    append_done(c);
+}
+
+// Bulk FWHT appends (T >= FWHT_CHUNK_MIN_T): CTA (chunk, 2h + kind, b)
+// takes FWHT_ROWS consecutive new tokens of one (sequence, head, kind), four
+// threads per row as above.  A cache block the chunk covers whole (16
+// tokens) is assembled in shared memory and written out as the kind's
+// 512-byte code region and 256-byte metadata region in 16-byte stores; the
+// tokens of a block the chunk covers only in part are stored one by one.
+constexpr int FWHT_CHUNK_MIN_T = 16;
+constexpr int FWHT_TILE_BLKS = FWHT_ROWS / BLK_TOK + 1;   // blocks a chunk can touch
+
+__global__ void __launch_bounds__(FWHT_THREADS) append_fwht_chunk_kernel(FwhtRows a, CacheDst c) {
+    __shared__ __align__(16) uint16_t xs[FWHT_ROWS][XS_STRIDE];
+    __shared__ __align__(16) uint8_t tile[FWHT_TILE_BLKS][BLK_BYTES];
+    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
+    const int kind = blockIdx.y & 1, h = blockIdx.y >> 1, b = blockIdx.z;
+    const int t0 = blockIdx.x * FWHT_ROWS;
+    pdl_wait();
+    pdl_trigger();
+    const int L0 = start_len_thread(c, b, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0);
+    const int nrows = min(FWHT_ROWS, c.T - t0);
+    const bool active = L0 >= 0 && r < nrows;                 // L0 is uniform over the CTA
+    const int32_t *perm = a.perm + ((size_t)kind * c.Hkv + h) * D;
+    if (active) {
+        const uint16_t *src = (kind == 0 ? a.X0 : a.X1) + (((size_t)b * c.T + t0 + r) * c.Hkv + h) * D;
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src) + 4 * q;
+        uint4 *d4 = reinterpret_cast<uint4 *>(&xs[r][0]) + 4 * q;
+#pragma unroll
+        for (int i = 0; i < 4; i++) d4[i] = s4[i];
+    }
+    __syncwarp();
+    float v[32];
+    fwht_row_quarter(xs[r], perm, active, q, v);
+    uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint32_t meta = quantize_group_thread(v, q, words);
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        words[w] |= __shfl_xor_sync(0xffffffffu, words[w], 1);
+        words[w] |= __shfl_xor_sync(0xffffffffu, words[w], 2);
+    }
+    uint32_t wa = words[0], wb = words[1];                     // thread q's words 2q, 2q+1
+#pragma unroll
+    for (int k = 1; k < 4; k++)
+        if (q == k) {
+            wa = words[2 * k];
+            wb = words[2 * k + 1];
+        }
+    const int P0 = L0 + t0, P1 = P0 + nrows;                  // positions of the chunk
+    const int lb0 = P0 / BLK_TOK;
+    if (active) {
+        const int p = P0 + r, lb = p / BLK_TOK, tau = p % BLK_TOK;
+        const int srow = sink_row(c, b, p);
+        if (srow >= 0) {
+            uint16_t *dst = (kind == 0 ? c.k_sink : c.v_sink) +
+                            (((size_t)b * c.Hkv + h) * c.S + (size_t)srow) * D + 32 * q;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+                *reinterpret_cast<uint4 *>(dst + e) =
+                    make_uint4(pack_half2(v[e], v[e + 1]), pack_half2(v[e + 2], v[e + 3]),
+                               pack_half2(v[e + 4], v[e + 5]), pack_half2(v[e + 6], v[e + 7]));
+            wa = wb = 0u;
+            meta = (c.sink_pos && kind == 0) ? SINK_KMETA_MARK : 0u;
+        }
+        const bool whole = lb * BLK_TOK >= P0 && (lb + 1) * BLK_TOK <= P1;
+        uint8_t *block;
+        if (whole) {
+            block = tile[lb - lb0];
+        } else {
+            const long long bi = cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, lb);
+            if (bi < 0 && q == 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+            block = bi < 0 ? nullptr : c.blocks + (size_t)bi * BLK_BYTES;
+        }
+        if (block) {
+            if (kind == 0) {
+                *reinterpret_cast<uint32_t *>(block + off_kword(tau, 2 * q)) = wa;
+                *reinterpret_cast<uint32_t *>(block + off_kword(tau, 2 * q + 1)) = wb;
+                *reinterpret_cast<uint32_t *>(block + off_kmeta(tau, q)) = meta;
+            } else {
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q)) = (uint16_t)wa;
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 1)) = (uint16_t)(wa >> 16);
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 2)) = (uint16_t)wb;
+                *reinterpret_cast<uint16_t *>(block + off_vpiece(tau, 4 * q + 3)) = (uint16_t)(wb >> 16);
+                *reinterpret_cast<uint32_t *>(block + off_vmeta(tau, q)) = meta;
+            }
+        }
+    }
+    __syncthreads();
+    // the whole blocks, 48 x 16 bytes each (32 of codes, 16 of metadata)
+    if (L0 >= 0) {
+        const int first = (P0 + BLK_TOK - 1) / BLK_TOK, last = P1 / BLK_TOK;   // [first, last)
+        const int i = threadIdx.x, k = i / 48, j = i % 48;
+        if (first + k < last) {
+            const int lb = first + k;
+            const long long bi = cache_block_index(c.table, c.num_blocks, c.nblk, c.Hkv, b, h, lb);
+            if (bi < 0) {
+                if (j == 0) set_status(c.status, KVQ_DEV_BAD_TABLE);
+            } else {
+                const int off = j < 32 ? (kind == 0 ? 0 : OFF_VC) + 16 * j
+                                       : (kind == 0 ? OFF_KM : OFF_VM) + 16 * (j - 32);
+                *reinterpret_cast<uint4 *>(c.blocks + (size_t)bi * BLK_BYTES + off) =
+                    *reinterpret_cast<const uint4 *>(&tile[lb - lb0][off]);
             }
         }
     }
@@ -594,6 +712,10 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.perm = perm;
         a.out_f32 = nullptr;
         a.n_rows = (long long)cd.B * T * cd.Hkv * 2;
+        if (T >= FWHT_CHUNK_MIN_T)
+            return launch_pdl(append_fwht_chunk_kernel,
+                              dim3((T + FWHT_ROWS - 1) / FWHT_ROWS, 2 * cd.Hkv, cd.B),
+                              dim3(FWHT_THREADS), 0, st, a, c);
         return launch_pdl(append_fwht_kernel<true>,
                           dim3((unsigned)((long long)cd.B * T), (2 * cd.Hkv + FWHT_ROWS - 1) / FWHT_ROWS),
                           dim3(FWHT_THREADS), 0, st, a, c);
