@@ -291,13 +291,14 @@ class Step:
     def run(self, k, seq_lens, split_events=None):
         kvq, w = self.kvq, self.w
         cache, Rk, Rv, perm = self.layers[k % len(self.layers)]
-        kvq.kvq_rotate_quantize_append(self.Knew, self.Vnew, w.mode, Rk, Rv, perm, cache, seq_lens)
         if split_events is not None:
+            kvq.kvq_rotate_quantize_append(self.Knew, self.Vnew, w.mode, Rk, Rv, perm, cache,
+                                           seq_lens)
             kvq.kvq_decode_attention_timed(self.Q, cache, w.mode, Rk, Rv, perm, seq_lens, w.sink,
                                            self.L, self.ws, self.out, *split_events)
-        else:
-            kvq.kvq_decode_attention(self.Q, cache, w.mode, Rk, Rv, perm, seq_lens, w.sink, self.L,
-                                     self.ws, self.out)
+        else:          # the serving step's one call: append, then decode
+            kvq.kvq_append_decode(self.Knew, self.Vnew, self.Q, cache, w.mode, Rk, Rv, perm,
+                                  seq_lens, self.L, self.ws, self.out)
 
     def status(self):
         return max(self.kvq.kvq_get_status(c[0]) for c in self.layers)

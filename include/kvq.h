@@ -374,6 +374,20 @@ KVQ_API kvq_status kvq_prerope_decode(const uint16_t *Q, int32_t Hq, const kvq_c
 KVQ_API kvq_status kvq_debug_rotate_group_f32(const uint16_t *X, int32_t N, int32_t group_heads,
                                               const int32_t *perm, float *Xrot, void *stream);
 
+/*
+ * One serving step in one call: kvq_rotate_quantize_append of the step's T
+ * new tokens, then kvq_decode_attention of one query per query head over the
+ * updated cache (seq_lens, updated by the append on the device, are the
+ * decode's lengths).  Arguments as in those two calls; all argument checks
+ * run before anything is launched; an error leaves nothing enqueued.
+ */
+KVQ_API kvq_status kvq_append_decode(const uint16_t *K, const uint16_t *V, int32_t T,
+                                     const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
+                                     kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                     const int32_t *perm, int32_t *seq_lens, int32_t max_ctx,
+                                     void *workspace, size_t ws_bytes, uint16_t *out,
+                                     void *stream);
+
 /* Short text for a status code (static storage). */
 KVQ_API const char *kvq_status_string(kvq_status s);
 

@@ -13,6 +13,7 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_decode_attention_timed,
                   kvq_decode_workspace_size, kvq_get_status, kvq_identify_sinks,
                   kvq_rotate_quantize_append, lib, kvq_prerope_append, kvq_prerope_decode,
+                  kvq_append_decode,
                   kvq_prerope_workspace_size, prerope_workspace, kvq_debug_rotate_group_f32)
 
 __all__ = [
@@ -24,5 +25,6 @@ __all__ = [
     "kvq_decode_attention_timed",
     "kvq_decode_workspace_size", "kvq_get_status", "kvq_identify_sinks",
     "kvq_rotate_quantize_append", "lib", "kvq_prerope_append", "kvq_prerope_decode",
+    "kvq_append_decode",
     "kvq_prerope_workspace_size", "prerope_workspace", "kvq_debug_rotate_group_f32",
 ]

@@ -87,10 +87,14 @@ size_t kvq_cache_bytes(int32_t B, int32_t Hkv, int32_t capacity) {
     return (size_t)B * Hkv * (capacity / BLK_TOK) * BLK_BYTES;
 }
 
-kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int32_t T,
-                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
-                                      const int32_t *perm, const kvq_cache_desc *cache,
-                                      int32_t *seq_lens, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks of an append (nothing is launched).
+kvq_status append_check(const uint16_t *K, const uint16_t *V, int32_t T, kvq_rot_mode mode,
+                        const float *R_k, const float *R_v, const int32_t *perm,
+                        const kvq_cache_desc *cache, const int32_t *seq_lens) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
     if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
@@ -99,11 +103,32 @@ kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int3
     if (!K || !V) return KVQ_ERR_INVALID_ARG;
     if (!aligned(K, 16) || !aligned(V, 16)) return KVQ_ERR_UNSUPPORTED;
     if (T > cache->capacity) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+// The append's kernel, arguments already checked.
+kvq_status append_launch(const uint16_t *K, const uint16_t *V, int32_t T, kvq_rot_mode mode,
+                         const float *R_k, const float *R_v, const int32_t *perm,
+                         const kvq_cache_desc *cache, int32_t *seq_lens, void *stream) {
+    if (T == 0) return KVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = (mode == KVQ_ROT_DENSE && append_tc_eligible(K, V, T))
                         ? launch_append_tc(K, V, T, R_k, R_v, *cache, seq_lens, st)
                         : launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_rotate_quantize_append(const uint16_t *K, const uint16_t *V, int32_t T,
+                                      kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                      const int32_t *perm, const kvq_cache_desc *cache,
+                                      int32_t *seq_lens, void *stream) {
+    const kvq_status s = append_check(K, V, T, mode, R_k, R_v, perm, cache, seq_lens);
+    if (s != KVQ_OK) return s;
+    return append_launch(K, V, T, mode, R_k, R_v, perm, cache, seq_lens, stream);
 }
 
 kvq_status kvq_identify_sinks(const float *act, int32_t T, float tau, const kvq_cache_desc *cache,
@@ -195,13 +220,12 @@ size_t kvq_decode_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t max
 
 namespace {
 
-// Shared body of the decode entry points: q_len queries per sequence (Hq
-// heads each), options in flags, optional events around the split kernel.
-kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t flags,
-                       const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
-                       const float *R_v, const int32_t *perm, const int32_t *seq_lens,
-                       int32_t sink_fp16, int32_t max_ctx, void *workspace, size_t ws_bytes,
-                       uint16_t *out, void *stream, void *ev_begin, void *ev_end) {
+// Argument checks of a decode (nothing is launched); C = split CTAs.
+kvq_status decode_check(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t flags,
+                        const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
+                        const float *R_v, const int32_t *perm, const int32_t *seq_lens,
+                        int32_t sink_fp16, int32_t max_ctx, const void *workspace,
+                        size_t ws_bytes, const uint16_t *out, int &C) {
     kvq_status s = check_cache(cache);
     if (s != KVQ_OK) return s;
     if ((s = check_rot(mode, R_k, R_v, perm)) != KVQ_OK) return s;
@@ -218,10 +242,24 @@ kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t fl
     if (max_ctx < q_len || max_ctx > cache->capacity) return KVQ_ERR_INVALID_ARG;
     const int sms = device_sm_count();
     if (sms < 1) return KVQ_ERR_CUDA;
-    const int C = split_ctas(cache->B, cache->Hkv, max_ctx, sms);
+    C = split_ctas(cache->B, cache->Hkv, max_ctx, sms);
     if (ws_bytes < ws_layout(cache->B, Hqq, cache->Hkv, C).total) return KVQ_ERR_WORKSPACE;
-    cudaError_t e = launch_decode(Q, Hqq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out,
-                                  static_cast<cudaStream_t>(stream),
+    return KVQ_OK;
+}
+
+// Shared body of the decode entry points: q_len queries per sequence (Hq
+// heads each), options in flags, optional events around the split kernel.
+kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t flags,
+                       const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
+                       const float *R_v, const int32_t *perm, const int32_t *seq_lens,
+                       int32_t sink_fp16, int32_t max_ctx, void *workspace, size_t ws_bytes,
+                       uint16_t *out, void *stream, void *ev_begin, void *ev_end) {
+    int C = 0;
+    const kvq_status s = decode_check(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens,
+                                      sink_fp16, max_ctx, workspace, ws_bytes, out, C);
+    if (s != KVQ_OK) return s;
+    cudaError_t e = launch_decode(Q, Hq * q_len, *cache, mode, R_k, R_v, perm, seq_lens, C,
+                                  workspace, out, static_cast<cudaStream_t>(stream),
                                   static_cast<cudaEvent_t>(ev_begin), static_cast<cudaEvent_t>(ev_end),
                                   q_len, (flags & KVQ_DECODE_OUT_ROTATED) ? 1 : 0);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -248,6 +286,24 @@ kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_t q_len,
                                    size_t ws_bytes, uint16_t *out, void *stream) {
     return decode_impl(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
                        max_ctx, workspace, ws_bytes, out, stream, nullptr, nullptr);
+}
+
+kvq_status kvq_append_decode(const uint16_t *K, const uint16_t *V, int32_t T, const uint16_t *Q,
+                             int32_t Hq, const kvq_cache_desc *cache, kvq_rot_mode mode,
+                             const float *R_k, const float *R_v, const int32_t *perm,
+                             int32_t *seq_lens, int32_t max_ctx, void *workspace, size_t ws_bytes,
+                             uint16_t *out, void *stream) {
+    kvq_status s = append_check(K, V, T, mode, R_k, R_v, perm, cache, seq_lens);
+    if (s != KVQ_OK) return s;
+    int C = 0;
+    s = decode_check(Q, Hq, 1, 0u, cache, mode, R_k, R_v, perm, seq_lens, cache->sink_fp16,
+                     max_ctx, workspace, ws_bytes, out, C);
+    if (s != KVQ_OK) return s;
+    if ((s = append_launch(K, V, T, mode, R_k, R_v, perm, cache, seq_lens, stream)) != KVQ_OK)
+        return s;
+    const cudaError_t e = launch_decode(Q, Hq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace,
+                                        out, static_cast<cudaStream_t>(stream), nullptr, nullptr, 1, 0);
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,

@@ -64,6 +64,9 @@ def lib():
     L.kvq_rotate_quantize_append.argtypes = [p, p, i32, C.c_int, p, p, p, C.POINTER(CacheDesc), p, p]
     L.kvq_identify_sinks.restype = C.c_int
     L.kvq_identify_sinks.argtypes = [p, i32, C.c_float, C.POINTER(CacheDesc), p, p]
+    L.kvq_append_decode.restype = C.c_int
+    L.kvq_append_decode.argtypes = [p, p, i32, p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p,
+                                    i32, p, sz, p, p]
     L.kvq_prerope_append.restype = C.c_int
     L.kvq_prerope_append.argtypes = [p, p, i32, i32, p, C.POINTER(CacheDesc), p, p]
     L.kvq_prerope_workspace_size.restype = sz
@@ -276,6 +279,32 @@ def kvq_decode_attention(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, ma
                                       _ptr(perm), _ptr(seq_lens), sink_fp16, max_ctx,
                                       _ptr(workspace), workspace.numel(), _ptr(out),
                                       _stream(stream, Q)))
+
+
+def kvq_append_decode(K, V, Q, cache, mode, R_k, R_v, perm, seq_lens, max_ctx, workspace, out,
+                      stream=None):
+    """One serving step: append K, V fp16 [B][T][Hkv][128] (seq_lens int32 [B]
+    advance by T on the device), then decode Q fp16 [B][Hq][128] into out over
+    the updated cache."""
+    B, T, Hkv, d = K.shape
+    _need(K, torch.float16, "K", (cache.B, T, cache.Hkv, D))
+    _need(V, torch.float16, "V", K.shape)
+    _need(Q, torch.float16, "Q")
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    if Q.dim() != 3 or Q.shape[0] != cache.B or Q.shape[2] != D:
+        raise ValueError("Q must have shape (B, Hq, 128)")
+    if mode == KVQ_ROT_DENSE:
+        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
+    else:
+        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
+    _check("kvq_append_decode",
+           lib().kvq_append_decode(_ptr(K), _ptr(V), T, _ptr(Q), Q.shape[1], C.byref(cache.desc),
+                                   mode, _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
+                                   max_ctx, _ptr(workspace), workspace.numel(), _ptr(out),
+                                   _stream(stream, Q)))
 
 
 KVQ_DECODE_OUT_ROTATED = 1

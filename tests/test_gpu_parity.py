@@ -476,3 +476,44 @@ def test_values_only_hadamard_rotation(T):
     assert kvq.kvq_get_status(cache) == 0
     err = rel_err(out.cpu().numpy(), ref)
     assert err.max() <= DEC_TOL, err.max()
+
+
+def test_append_decode_step_equals_the_two_calls():
+    """kvq_append_decode is the append followed by the decode: the same cache
+    bytes, lengths and output bits; a call that fails its checks (workspace
+    too small) enqueues nothing, the append included."""
+    w = W.custom(seed=310, B=2, Hq=4, Hkv=2, mode=0, k_outliers=4)
+    rt, _ = rot_tensors(w)
+    cap, L0, T = 256, [100, 37], 1
+    K = torch.stack([W.kv_rows(w, b, 0, 130, "cpu")[0] for b in range(2)]).cuda()
+    V = torch.stack([W.kv_rows(w, b, 0, 130, "cpu")[1] for b in range(2)]).cuda()
+    caches, outs, lens = [], [], []
+    for fused in (False, True):
+        cache = kvq.KVCache(2, 2, cap)
+        sl = torch.zeros(2, dtype=torch.int32, device="cuda")
+        gpu_append(cache, K[:, :100].contiguous(), V[:, :100].contiguous(), w, rt, sl)
+        sl.copy_(torch.tensor(L0, dtype=torch.int32))
+        Kn = K[:, 100:101].contiguous()
+        Vn = V[:, 100:101].contiguous()
+        Q = W.queries(w, "cuda")
+        ws = kvq.decode_workspace(2, 4, 2, cap)
+        out = torch.empty_like(Q)
+        if fused:
+            kvq.kvq_append_decode(Kn, Vn, Q, cache, 0, rt[0], rt[1], None, sl, cap, ws, out)
+        else:
+            gpu_append(cache, Kn, Vn, w, rt, sl)
+            kvq.kvq_decode_attention(Q, cache, 0, rt[0], rt[1], None, sl, 0, cap, ws, out)
+        torch.cuda.synchronize()
+        assert kvq.kvq_get_status(cache) == 0
+        caches.append(cache.blocks.clone())
+        outs.append(out.clone())
+        lens.append(sl.clone())
+    assert torch.equal(caches[0], caches[1]) and torch.equal(outs[0], outs[1])
+    assert torch.equal(lens[0], lens[1]) and list(lens[1].cpu().numpy()) == [101, 38]
+    before = caches[1].clone()
+    small = torch.empty(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_append_decode(Kn, Vn, Q, cache, 0, rt[0], rt[1], None, sl, cap, small, out)
+    assert e.value.code == 5                               # KVQ_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.equal(cache.blocks, before) and list(sl.cpu().numpy()) == [101, 38]
