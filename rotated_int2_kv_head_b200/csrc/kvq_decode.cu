@@ -401,7 +401,7 @@ __host__ __device__ inline SplitSmem split_smem_layout(int G) {
     L.fm = smem_up16(L.fo + 4u * GROUP_WARPS * G * D);
     L.fl = smem_up16(L.fm + 4u * GROUP_WARPS * G);
     L.fz = smem_up16(L.fl + 4u * GROUP_WARPS * G);
-    L.gstride = (L.fz + 4u * GROUP_WARPS * G * 4 + 127u) & ~127u;
+    L.gstride = (L.fz + 4u * GROUP_WARPS * G * 4 + 4u + 127u) & ~127u;   // + one dump float
     L.scratch = DEC_GROUPS * L.gstride;
     L.total = smem_up16(L.scratch + 4u * (3 * DEC_GROUPS + DEC_WARPS));
     return L;
@@ -433,6 +433,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     float *fm = reinterpret_cast<float *>(gbase + L.fm);              // [W][G]
     float *fl = reinterpret_cast<float *>(gbase + L.fl);              // [W][G]
     float *fz = reinterpret_cast<float *>(gbase + L.fz);              // [W][G][4]
+    float *dump = fz + GROUP_WARPS * G * 4;                           // write-only
     int *scratch = reinterpret_cast<int *>(smem + L.scratch);
     // named barrier of this group (id 0 is __syncthreads)
     auto bar_group = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(GROUP_THREADS) : "memory"); };
@@ -597,10 +598,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                 for (int k = 0; k < 4; k++) {
                     const int nv = (g * G) / 8;
                     const int col = 8 * nv + 2 * c + (k & 1);
-                    if (col / G == g) {
-                        const int head = col % G;
-                        const int j = 32 * g + 16 * h2 + 2 * r + (k >> 1);
-                        wo[head * D + j] = O[g * 2 + h2][k] * __int_as_float((127 + 24 - 2 * g) << 23);
+                    const int head = col % G;
+                    const int j = 32 * g + 16 * h2 + 2 * r + (k >> 1);
+                    const float val = O[g * 2 + h2][k] * __int_as_float((127 + 24 - 2 * g) << 23);
+                    if constexpr (G >= 4) {
+                        // an accumulator of another group's column goes to the
+                        // dump float: with a branch on the lane here the compiler
+                        // kept O in local memory (a 16-byte store per stage)
+                        float *dst = col / G == g ? &wo[head * D + j] : dump;
+                        *dst = val;
+                    } else if (col / G == g) {
+                        wo[head * D + j] = val;
                     }
                 }
         bar_group();
