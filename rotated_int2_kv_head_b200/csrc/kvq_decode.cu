@@ -638,13 +638,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     // Scores, part 1: the K codes of a warp's two blocks of a stage through
     // the integer tensor cores (one IMMA per group and block; the second
     // block may be a phantom).
-    auto k_mma = [&](const uint8_t *blk0, int (&dk)[2][C::NTK][4]) {
+    // Blocks b_lo .. b_hi-1 of the pair (G = 8 takes them one at a time: the
+    // accumulators of both would not fit the 128 registers).
+    auto k_mma = [&](const uint8_t *blk0, int (&dk)[2][C::NTK][4], int b_lo, int b_hi) {
         uint4 kq[2];
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++)
+        for (int bi = b_lo; bi < b_hi; bi++)
             kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++)
+        for (int bi = b_lo; bi < b_hi; bi++)
 #pragma unroll
             for (int nu = 0; nu < C::NTK; nu++)
 #pragma unroll
@@ -654,7 +656,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         for (int g = 0; g < 4; g++) {
             const uint32_t msk = 0x03030303u << (2 * g);
 #pragma unroll
-            for (int bi = 0; bi < 2; bi++) {
+            for (int bi = b_lo; bi < b_hi; bi++) {
                 const uint4 q4 = kq[bi];
 #pragma unroll
                 for (int j = 0; j < C::NTK_STEP; j++) {
@@ -669,14 +671,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     // query scale), summed over the groups; positions outside [S, L) and
     // phantom blocks are masked to -inf.
     auto k_combine = [&](const uint8_t *blk0, const int (&dk)[2][C::NTK][4], int tok0, int nmine,
-                         float (&sco)[2][2][C::HPL], bool (&edge)[2]) {
+                         float (&sco)[2][2][C::HPL], bool (&edge)[2], int b_lo, int b_hi) {
         // a block needs masking if it is a phantom or crosses [S, L)
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++)
+        for (int bi = b_lo; bi < b_hi; bi++)
             edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S ||
                        tok0 + (bi + 1) * BLK_TOK > Lcur - (a.qlen - 1);
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++) {
+        for (int bi = b_lo; bi < b_hi; bi++) {
             float part_sc[2][C::HPL];
 #pragma unroll
             for (int st = 0; st < 2; st++)
@@ -920,8 +922,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             int dk[2][C::NTK][4];
             float sco[2][2][C::HPL];
             bool edge[2];
-            k_mma(wblk(s), dk);
-            k_combine(wblk(s), dk, (d0.w + 2 * warp) * BLK_TOK, nmine, sco, edge);
+            const int tok0 = (d0.w + 2 * warp) * BLK_TOK;
+            if constexpr (G >= 8) {
+                k_mma(wblk(s), dk, 0, 1);
+                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 0, 1);
+                k_mma(wblk(s), dk, 1, 2);
+                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 1, 2);
+            } else {
+                k_mma(wblk(s), dk, 0, 2);
+                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 0, 2);
+            }
             v_side(wblk(s), sco, edge);
         }
         if (!ok) set_status(a.status, KVQ_DEV_TIMEOUT);
