@@ -768,11 +768,20 @@ def run_cuda(args):
     if step.status() != 0:
         raise RuntimeError("device status %d after timed steps" % step.status())
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # new K/V and queries from pinned memory (one copy: they sit in one
-    # buffer), append + decode, D2H of the output
+    # end to end through the C-ABI call with host buffers: one
+    # kvq_append_decode_host per step copies the step's new K/V rows and
+    # queries in from pinned memory, appends, decodes and copies the output
+    # back; the host then waits for the stream
+    import rotated_int2_kv_head_b200 as kvq
+    # the inputs are views of one pinned buffer, back to back, so the call
+    # moves them with a single copy
     hIn = step.inbuf.cpu().pin_memory()
+    nk = step.Knew.numel()
+    hK = hIn[:nk].view(step.Knew.shape)
+    hV = hIn[nk:2 * nk].view(step.Vnew.shape)
+    hQ = hIn[2 * nk:].view(step.Q.shape)
     hO = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    wsh = kvq.step_workspace(w.B, step.T, w.Hq, w.Hkv, step.L, device=dev)
     n_e2e = min(K, 200)
     sl_e2e = step.lengths(n_e2e + 3)
     e2e_s = 0.0
@@ -780,16 +789,18 @@ def run_cuda(args):
         if flush is not None:
             flush(k)
         torch.cuda.synchronize(dev)
+        cache, Rk, Rv, perm = step.layers[k % len(step.layers)]
         t0 = time.perf_counter()
-        step.inbuf.copy_(hIn, non_blocking=True)
-        step.run(k, sl_e2e[k])
-        hO.copy_(step.out, non_blocking=True)
+        kvq.kvq_append_decode_host(hK, hV, hQ, cache, w.mode, Rk, Rv, perm, sl_e2e[k], step.L, wsh,
+                                   hO)
         torch.cuda.synchronize(dev)
         if k >= 3:
             e2e_s += time.perf_counter() - t0
     e2e_s = max_over_ranks(e2e_s, dist_on, dev)
-    h2d = hIn.numel() * 2
+    h2d = (hK.numel() + hV.numel() + hQ.numel()) * 2
     d2h = hO.numel() * 2
+    if not torch.equal(hO.to(dev), step.out):      # the same step as the device-timed one
+        raise RuntimeError("host-buffer step output differs from the device step")
 
     if rank != 0:
         if dist_on:
@@ -838,8 +849,9 @@ def run_cuda(args):
                      "algorithmic_bytes_per_launch": kv_bytes,
                      "kernel_ms_mean": split_mean_s * 1e3, "peak_source": peak_src},
         "e2e": {"value": tokens * n_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "how": "wall clock per step incl. pinned H2D of new "
-                                                  "K/V/Q and D2H of the output, synchronised"},
+                "d2h_bytes_per_step": d2h, "how": "wall clock per step: one kvq_append_decode_host "
+                                                  "call (pinned H2D of the new K/V/Q, append, decode, "
+                                                  "D2H of the output), then a stream synchronise"},
         "isolated_step": {"ms": float(np.median(iso_ms)), "how": "median of %d steps, each after "
                           "an L2 flush and bracketed by its own events" % n_iso},
         "gpu_launches": KERNELS_PER_STEP * K,

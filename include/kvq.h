@@ -388,6 +388,31 @@ KVQ_API kvq_status kvq_append_decode(const uint16_t *K, const uint16_t *V, int32
                                      void *workspace, size_t ws_bytes, uint16_t *out,
                                      void *stream);
 
+/*
+ * The serving step with host buffers: the step's new K, V rows and queries
+ * are in host memory, and so is the output.  Inside one call: the
+ * host-to-device copies of K, V and Q into the staging part of the
+ * workspace (one copy when V_host starts where K_host ends and Q_host where
+ * V_host ends, else three), kvq_append_decode on them, and one
+ * device-to-host copy of the output,
+ * all asynchronous on `stream` (host memory should be pinned for the copies
+ * to overlap; pageable memory works, synchronously).  Synchronise the
+ * stream before reading out_host.
+ *   K_host, V_host  fp16 [B][T][Hkv][128];  Q_host, out_host fp16 [B][Hq][128].
+ *   workspace       device, >= kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx,
+ *                   SMs) bytes, 256-B aligned.
+ * Other arguments and errors as kvq_append_decode.
+ */
+KVQ_API size_t kvq_step_workspace_size(int32_t B, int32_t T, int32_t Hq, int32_t Hkv,
+                                       int32_t max_ctx, int32_t sm_count);
+KVQ_API kvq_status kvq_append_decode_host(const uint16_t *K_host, const uint16_t *V_host,
+                                          int32_t T, const uint16_t *Q_host, int32_t Hq,
+                                          const kvq_cache_desc *cache, kvq_rot_mode mode,
+                                          const float *R_k, const float *R_v,
+                                          const int32_t *perm, int32_t *seq_lens,
+                                          int32_t max_ctx, void *workspace, size_t ws_bytes,
+                                          uint16_t *out_host, void *stream);
+
 /* Short text for a status code (static storage). */
 KVQ_API const char *kvq_status_string(kvq_status s);
 

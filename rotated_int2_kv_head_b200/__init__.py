@@ -13,7 +13,8 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_decode_attention_timed,
                   kvq_decode_workspace_size, kvq_get_status, kvq_identify_sinks,
                   kvq_rotate_quantize_append, lib, kvq_prerope_append, kvq_prerope_decode,
-                  kvq_append_decode,
+                  kvq_append_decode, kvq_append_decode_host, kvq_step_workspace_size,
+                  step_workspace,
                   kvq_prerope_workspace_size, prerope_workspace, kvq_debug_rotate_group_f32)
 
 __all__ = [
@@ -25,6 +26,6 @@ __all__ = [
     "kvq_decode_attention_timed",
     "kvq_decode_workspace_size", "kvq_get_status", "kvq_identify_sinks",
     "kvq_rotate_quantize_append", "lib", "kvq_prerope_append", "kvq_prerope_decode",
-    "kvq_append_decode",
+    "kvq_append_decode", "kvq_append_decode_host", "kvq_step_workspace_size", "step_workspace",
     "kvq_prerope_workspace_size", "prerope_workspace", "kvq_debug_rotate_group_f32",
 ]

@@ -306,6 +306,90 @@ kvq_status kvq_append_decode(const uint16_t *K, const uint16_t *V, int32_t T, co
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Staging layout of the host-buffer step, after the decode workspace:
+// K, V [B][T][Hkv][128], Q and out [B][Hq][128], each 256-B aligned.
+struct StepLayout {
+    size_t k, v, q, out, total;
+};
+StepLayout step_layout(int B, int T, int Hq, int Hkv, size_t dec_ws) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    StepLayout l;
+    const size_t kv = (size_t)B * T * Hkv * D * 2, qb = (size_t)B * Hq * D * 2;
+    l.k = up(dec_ws);
+    l.v = up(l.k + kv);
+    l.q = up(l.v + kv);
+    l.out = up(l.q + qb);
+    l.total = up(l.out + qb);
+    return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_step_workspace_size(int32_t B, int32_t T, int32_t Hq, int32_t Hkv, int32_t max_ctx,
+                               int32_t sm_count) {
+    if (T < 1) return 0;
+    const size_t dec = kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count);
+    if (dec == 0) return 0;
+    return step_layout(B, T, Hq, Hkv, dec).total;
+}
+
+kvq_status kvq_append_decode_host(const uint16_t *K_host, const uint16_t *V_host, int32_t T,
+                                  const uint16_t *Q_host, int32_t Hq, const kvq_cache_desc *cache,
+                                  kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                  const int32_t *perm, int32_t *seq_lens, int32_t max_ctx,
+                                  void *workspace, size_t ws_bytes, uint16_t *out_host,
+                                  void *stream) {
+    kvq_status s = check_cache(cache);
+    if (s != KVQ_OK) return s;
+    if (!K_host || !V_host || !Q_host || !out_host || !workspace || T < 1) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return KVQ_ERR_UNSUPPORTED;
+    if (Hq < cache->Hkv || Hq % cache->Hkv != 0) return KVQ_ERR_INVALID_ARG;
+    const int sms = device_sm_count();
+    if (sms < 1) return KVQ_ERR_CUDA;
+    const size_t dec = kvq_decode_workspace_size(cache->B, Hq, cache->Hkv, max_ctx, sms);
+    if (dec == 0) return KVQ_ERR_INVALID_ARG;
+    const StepLayout l = step_layout(cache->B, T, Hq, cache->Hkv, dec);
+    if (ws_bytes < l.total) return KVQ_ERR_WORKSPACE;
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    uint16_t *K = reinterpret_cast<uint16_t *>(w + l.k), *V = reinterpret_cast<uint16_t *>(w + l.v);
+    uint16_t *Q = reinterpret_cast<uint16_t *>(w + l.q), *out = reinterpret_cast<uint16_t *>(w + l.out);
+    // every check of the two device calls before the first copy
+    if ((s = append_check(K, V, T, mode, R_k, R_v, perm, cache, seq_lens)) != KVQ_OK) return s;
+    int C = 0;
+    if ((s = decode_check(Q, Hq, 1, 0u, cache, mode, R_k, R_v, perm, seq_lens, cache->sink_fp16,
+                          max_ctx, workspace, dec, out, C)) != KVQ_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t kv = (size_t)cache->B * T * cache->Hkv * D * 2, qb = (size_t)cache->B * Hq * D * 2;
+    // kv and qb are multiples of 256 B, so the K, V and Q regions of the
+    // workspace are back to back: host inputs that are back to back as well
+    // (views of one pinned buffer) go in with a single copy
+    const uint8_t *hk = reinterpret_cast<const uint8_t *>(K_host);
+    const bool one = reinterpret_cast<const uint8_t *>(V_host) == hk + kv &&
+                     reinterpret_cast<const uint8_t *>(Q_host) == hk + 2 * kv && l.v == l.k + kv &&
+                     l.q == l.v + kv;
+    if (one) {
+        if (cudaMemcpyAsync(K, K_host, 2 * kv + qb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+    } else if (cudaMemcpyAsync(K, K_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+               cudaMemcpyAsync(V, V_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+               cudaMemcpyAsync(Q, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+        return KVQ_ERR_CUDA;
+    }
+    if ((s = append_launch(K, V, T, mode, R_k, R_v, perm, cache, seq_lens, stream)) != KVQ_OK) return s;
+    if (launch_decode(Q, Hq, *cache, mode, R_k, R_v, perm, seq_lens, C, workspace, out, st, nullptr,
+                      nullptr, 1, 0) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    return cudaMemcpyAsync(out_host, out, qb, cudaMemcpyDeviceToHost, st) == cudaSuccess ? KVQ_OK
+                                                                                      : KVQ_ERR_CUDA;
+}
+
 kvq_status kvq_decode_attention(const uint16_t *Q, int32_t Hq, const kvq_cache_desc *cache,
                                 kvq_rot_mode mode, const float *R_k, const float *R_v,
                                 const int32_t *perm, const int32_t *seq_lens,

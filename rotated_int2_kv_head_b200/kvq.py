@@ -67,6 +67,11 @@ def lib():
     L.kvq_append_decode.restype = C.c_int
     L.kvq_append_decode.argtypes = [p, p, i32, p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p,
                                     i32, p, sz, p, p]
+    L.kvq_step_workspace_size.restype = sz
+    L.kvq_step_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.kvq_append_decode_host.restype = C.c_int
+    L.kvq_append_decode_host.argtypes = [p, p, i32, p, i32, C.POINTER(CacheDesc), C.c_int, p, p,
+                                         p, p, i32, p, sz, p, p]
     L.kvq_prerope_append.restype = C.c_int
     L.kvq_prerope_append.argtypes = [p, p, i32, i32, p, C.POINTER(CacheDesc), p, p]
     L.kvq_prerope_workspace_size.restype = sz
@@ -305,6 +310,56 @@ def kvq_append_decode(K, V, Q, cache, mode, R_k, R_v, perm, seq_lens, max_ctx, w
                                    mode, _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
                                    max_ctx, _ptr(workspace), workspace.numel(), _ptr(out),
                                    _stream(stream, Q)))
+
+
+def _need_host(t, dtype, name, shape=None):
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous host tensor (pinned for overlap)" % name)
+    if shape is not None and t.shape != shape:
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx, sm_count=None):
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return lib().kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx, sm_count)
+
+
+def step_workspace(B, T, Hq, Hkv, max_ctx, device="cuda"):
+    n = kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx)
+    if n == 0:
+        raise ValueError("bad step shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kvq_append_decode_host(K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, seq_lens, max_ctx,
+                           workspace, out_host, stream=None):
+    """The serving step with host tensors (pin them): K, V fp16 [B][T][Hkv][128]
+    and Q fp16 [B][Hq][128] are copied in, appended and decoded, and the output
+    copied back into out_host, all queued on the stream (synchronise before
+    reading out_host).  workspace: step_workspace(...) on the device."""
+    B, T, Hkv, d = K_host.shape
+    _need_host(K_host, torch.float16, "K_host", (cache.B, T, cache.Hkv, D))
+    _need_host(V_host, torch.float16, "V_host", K_host.shape)
+    _need_host(Q_host, torch.float16, "Q_host")
+    _need_host(out_host, torch.float16, "out_host", Q_host.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    if Q_host.dim() != 3 or Q_host.shape[0] != cache.B or Q_host.shape[2] != D:
+        raise ValueError("Q_host must have shape (B, Hq, 128)")
+    if mode == KVQ_ROT_DENSE:
+        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
+    else:
+        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
+    _check("kvq_append_decode_host",
+           lib().kvq_append_decode_host(_ptr(K_host), _ptr(V_host), T, _ptr(Q_host),
+                                        Q_host.shape[1], C.byref(cache.desc), mode, _ptr(R_k),
+                                        _ptr(R_v), _ptr(perm), _ptr(seq_lens), max_ctx,
+                                        _ptr(workspace), workspace.numel(), _ptr(out_host),
+                                        _stream(stream, workspace)))
 
 
 KVQ_DECODE_OUT_ROTATED = 1

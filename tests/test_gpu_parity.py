@@ -517,3 +517,60 @@ def test_append_decode_step_equals_the_two_calls():
     assert e.value.code == 5                               # KVQ_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert torch.equal(cache.blocks, before) and list(sl.cpu().numpy()) == [101, 38]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_append_decode_host_equals_the_device_step(mode):
+    """kvq_append_decode_host is kvq_append_decode with its inputs and output
+    in host memory: the same cache bytes, lengths and output bits; a call
+    that fails its checks (workspace too small) touches neither the cache,
+    the lengths nor the host output."""
+    w = W.custom(seed=311 + mode, B=2, Hq=8, Hkv=2, mode=mode, k_outliers=4)
+    rt, _ = rot_tensors(w)
+    cap, L0, T = 256, [120, 53], 3
+    K = torch.stack([W.kv_rows(w, b, 0, 140, "cpu")[0] for b in range(2)]).cuda()
+    V = torch.stack([W.kv_rows(w, b, 0, 140, "cpu")[1] for b in range(2)]).cuda()
+    Q = W.queries(w, "cuda")
+    res = []
+    for host in (False, True, "one buffer"):
+        cache = kvq.KVCache(2, 2, cap, 4)
+        sl = torch.zeros(2, dtype=torch.int32, device="cuda")
+        gpu_append(cache, K[:, :120].contiguous(), V[:, :120].contiguous(), w, rt, sl)
+        sl.copy_(torch.tensor(L0, dtype=torch.int32))
+        Kn = K[:, 120:120 + T].contiguous()
+        Vn = V[:, 120:120 + T].contiguous()
+        if host:
+            ws = kvq.step_workspace(2, T, 8, 2, cap)
+            ws.fill_(0xFF)
+            hO = torch.full(Q.shape, float("nan"), dtype=torch.float16).pin_memory()
+            if host == "one buffer":          # back to back: a single H2D copy
+                buf = torch.cat([Kn.reshape(-1), Vn.reshape(-1), Q.reshape(-1)]).cpu().pin_memory()
+                n = Kn.numel()
+                hk, hv = buf[:n].view(Kn.shape), buf[n:2 * n].view(Vn.shape)
+                hq = buf[2 * n:].view(Q.shape)
+            else:
+                hk, hv, hq = Kn.cpu().pin_memory(), Vn.cpu().pin_memory(), Q.cpu().pin_memory()
+            kvq.kvq_append_decode_host(hk, hv, hq, cache, mode, *rt, sl, cap, ws, hO)
+            torch.cuda.synchronize()
+            out = hO.cuda()
+        else:
+            ws = kvq.decode_workspace(2, 8, 2, cap)
+            out = torch.empty_like(Q)
+            kvq.kvq_append_decode(Kn, Vn, Q, cache, mode, *rt, sl, cap, ws, out)
+            torch.cuda.synchronize()
+        assert kvq.kvq_get_status(cache) == 0
+        res.append((cache.blocks.clone(), cache.k_sink.clone(), out, sl.clone()))
+    for r in res[1:]:
+        for a, b in zip(res[0], r):
+            assert torch.equal(a, b)
+    assert list(res[1][3].cpu().numpy()) == [120 + T, 53 + T]
+    before = cache.blocks.clone()
+    small = torch.empty(64, dtype=torch.uint8, device="cuda")
+    hO = torch.zeros(Q.shape, dtype=torch.float16).pin_memory()
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_append_decode_host(Kn.cpu().pin_memory(), Vn.cpu().pin_memory(),
+                                   Q.cpu().pin_memory(), cache, mode, *rt, sl, cap, small, hO)
+    assert e.value.code == 5                               # KVQ_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.equal(cache.blocks, before) and not hO.any()
+    assert list(sl.cpu().numpy()) == [120 + T, 53 + T]
