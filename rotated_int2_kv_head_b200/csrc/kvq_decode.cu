@@ -144,8 +144,47 @@ __device__ __forceinline__ void sched_fix_unit(Sched &s, const DecodeArgs &a) {
 // 3*DEC_GROUPS + DEC_WARPS ints of shared memory.  Returns false when the
 // CTA's range is empty (uniformly over the CTA).  CTA 0 flags invalid
 // lengths.
+constexpr int SCHED_SMALL_B = 32;
 __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    if (a.B <= SCHED_SMALL_B) {
+        // Few sequences: every thread reads all lengths (the same addresses
+        // in every thread) and finds its group's first unit alone, with no
+        // scan and no barrier.
+        int N = 0;
+#pragma unroll 4
+        for (int b = 0; b < a.B; b++) {
+            const int L = a.seq_lens[b];
+            if (blockIdx.x == 0 && t == 0 && (L < 1 || L > a.capacity))
+                set_status(a.status, KVQ_DEV_BAD_LEN);
+            N += a.Hkv * unit_slots(L, a.S, a.capacity);
+        }
+        const int W = max(1, (N + a.C - 1) / a.C);
+        const int beg = blockIdx.x * W, end = min(N, beg + W);
+        if (beg >= end) return false;
+        const int Wg = (end - beg + DEC_GROUPS - 1) / DEC_GROUPS;
+        const int p = beg + (t / GROUP_THREADS) * Wg;
+        s.b = s.h = s.nb = s.ustart = s.pref = 0;
+        s.cur = s.end = 0;
+        if (p < end) {
+            int acc = 0;
+            for (int b = 0; b < a.B; b++) {
+                const int nbu = seq_blocks(a, b);
+                if (p < acc + a.Hkv * nbu) {
+                    s.b = b;
+                    s.pref = acc;
+                    s.nb = nbu;
+                    break;
+                }
+                acc += a.Hkv * nbu;
+            }
+            s.h = (p - s.pref) / s.nb;
+            s.ustart = s.pref + s.h * s.nb;
+            s.cur = p;
+            s.end = min(end, p + Wg);
+        }
+        return true;
+    }
     const int per = (a.B + DEC_THREADS - 1) / DEC_THREADS;
     const int lo = min(a.B, t * per), hi = min(a.B, lo + per);
     int sum = 0, nb_lo = 0;          // nb_lo: blocks per unit of sequence lo (kept in a register)
