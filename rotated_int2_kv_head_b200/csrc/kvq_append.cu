@@ -110,33 +110,37 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     }
     pdl_wait();
     pdl_trigger();
+    row0 = blockIdx.x * a.tchunk;
+    const int avail = min(a.tchunk, (TO_CACHE ? c.T : a.n_rows) - row0);   // >= 1 by the grid
+    // thread t stages 16 B of row (base + t/16) of a batch: 8 rows x 256 B
+    const int rr = threadIdx.x >> 4, piece = threadIdx.x & 15;
+    auto piece_ptr = [&](int row) -> const uint4 * {
+        const uint16_t *src = TO_CACHE ? X + (((size_t)b * c.T + row) * c.Hkv + h) * D
+                                       : X + (size_t)row * D;
+        return reinterpret_cast<const uint4 *>(src + piece * 8);
+    };
+    // the first batch's input is loaded before seq_lens is examined: the two
+    // loads are independent and overlap
+    uint4 first = make_uint4(0u, 0u, 0u, 0u);
+    if (rr < min(DENSE_BATCH, avail)) first = *piece_ptr(row0 + rr);
+    unsigned claim = 0u;
     if (TO_CACHE) {
         L0 = start_len(c, b);
-        row0 = blockIdx.x * a.tchunk;
-        nrows = L0 < 0 ? 0 : min(a.tchunk, c.T - row0);     // skipped sequence: no rows
+        nrows = L0 < 0 ? 0 : avail;                          // skipped sequence: no rows
+        claim = append_claim(c);                             // seq_lens is not read again
     } else {
-        row0 = blockIdx.x * a.tchunk;
-        nrows = min(a.tchunk, a.n_rows - row0);
+        nrows = avail;
     }
     if (nrows <= 0) {
-        if (TO_CACHE) append_done(c);
+        if (TO_CACHE) append_finish(c, claim);
         return;
     }
 
     for (int base = 0; base < nrows; base += DENSE_BATCH) {
         const int nb = min(DENSE_BATCH, nrows - base);
-        // stage the batch's fp16 rows: 8 rows x 256 B, 16 B per thread
-        if (threadIdx.x < nb * 16) {
-            const int rr = threadIdx.x >> 4, piece = threadIdx.x & 15;
-            const int row = row0 + base + rr;
-            const uint16_t *src;
-            if (TO_CACHE)
-                src = X + (((size_t)b * c.T + row) * c.Hkv + h) * D;
-            else
-                src = X + (size_t)row * D;
+        if (rr < nb)
             *reinterpret_cast<uint4 *>(&xs[rr][piece * 8]) =
-                *reinterpret_cast<const uint4 *>(src + piece * 8);
-        }
+                base == 0 ? first : *piece_ptr(row0 + base + rr);
         __syncthreads();
         for (int k = 0; k < nb; k++) {
             const uint4 u0 = *reinterpret_cast<const uint4 *>(&xs[k][16 * warp]);
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(DENSE_THREADS)
         }
         __syncthreads();
     }
-    if (TO_CACHE) append_done(c);
+    if (TO_CACHE) append_finish(c, claim);
 }
 
 // ---- permutation + FWHT ---------------------------------------------------------------------

@@ -1115,7 +1115,8 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
             ired[MRG_THREADS / 32 + warp] = sn;
         }
     }
-    // R_v rows for the rotate-out (no kernel of this chain writes R_v)
+    // R_v rows for the rotate-out (no kernel of this chain writes R_v): warp w
+    // rows 16w..16w+15, lane l columns 4l..4l+3, each load one whole row
     float4 rr[16];
     if (a.mode == KVQ_ROT_DENSE) {
         const float *R = a.R_v + (size_t)h * D * D + (size_t)(16 * warp) * D + 4 * lane;
@@ -1212,17 +1213,30 @@ __global__ void __launch_bounds__(MRG_THREADS) decode_merge_kernel(DecodeArgs a)
         // the caller folds R_v^T into its own projection: o_rot as it is
         if (t < D) out[t] = __half_as_ushort(__float2half_rn(o_s[t]));
     } else if (a.mode == KVQ_ROT_DENSE) {
-        // out[i] = sum_j o[j] R_v[h][i][j]: warp w rows 16w..16w+15, lanes over j
+        // out[i] = sum_j o[j] R_v[h][i][j] for the warp's 16 rows: each lane
+        // dots its 4 columns, then a reduce-scatter over the lanes (at the
+        // exchange over lane bit m a lane keeps the half of its rows that bit
+        // selects) leaves row 8b4 + 4b3 + 2b2 + b1 of lane bits b4..b1 in
+        // lanes 2k and 2k+1: 16 shuffles instead of 5 per row
         const float4 o4 = *reinterpret_cast<const float4 *>(&o_s[4 * lane]);
-        float mine = 0.f;
+        float v[16];
 #pragma unroll
-        for (int ii = 0; ii < 16; ii++) {
-            float d = o4.x * rr[ii].x + o4.y * rr[ii].y + o4.z * rr[ii].z + o4.w * rr[ii].w;
+        for (int ii = 0; ii < 16; ii++)
+            v[ii] = o4.x * rr[ii].x + o4.y * rr[ii].y + o4.z * rr[ii].z + o4.w * rr[ii].w;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            if (lane == ii) mine = d;
+        for (int m = 16, n = 8; m >= 2; m >>= 1, n >>= 1) {
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < n; i++) {
+                const float send = up ? v[i] : v[i + n];
+                const float keep = up ? v[i + n] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
         }
-        if (lane < 16) out[16 * warp + lane] = __half_as_ushort(__float2half_rn(mine));
+        const float d = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int row = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1) +
+                        ((lane >> 1) & 1);
+        if ((lane & 1) == 0) out[16 * warp + row] = __half_as_ushort(__float2half_rn(d));
     } else if (warp == 0) {
         float v[4] = {o_s[4 * lane], o_s[4 * lane + 1], o_s[4 * lane + 2], o_s[4 * lane + 3]};
         fwht128_warp(v);

@@ -492,6 +492,30 @@ static __device__ void append_done(const CacheDst &c) {
     }
 }
 
+// The same completion count in two halves, for kernels whose threads read
+// seq_lens only at their start: append_claim right after the last read (the
+// atomic's round trip then overlaps the CTA's work), append_finish at the
+// end.  The last CTA to claim bumps the lengths when it finishes: every
+// other CTA has read them by then.
+__device__ __forceinline__ unsigned append_claim(const CacheDst &c) {
+    __syncthreads();
+    unsigned prev = 0u;
+    if (threadIdx.x == 0) prev = atomicAdd(reinterpret_cast<unsigned *>(c.status + 1), 1u);
+    return prev;   // meaningful in thread 0
+}
+static __device__ void append_finish(const CacheDst &c, unsigned prev) {
+    __shared__ int last;
+    if (threadIdx.x == 0) last = (prev == gridDim.x * gridDim.y * gridDim.z - 1);
+    __syncthreads();
+    if (last) {
+        for (int b = threadIdx.x; b < c.B; b += blockDim.x) {
+            const int L0 = c.seq_lens[b];
+            if (L0 >= 0 && (long long)L0 + c.T <= c.capacity) c.seq_lens[b] = L0 + c.T;
+        }
+        if (threadIdx.x == 0) atomicExch(reinterpret_cast<unsigned *>(c.status + 1), 0u);
+    }
+}
+
 // Reads seq_lens[b] and checks capacity; returns -1 (and flags) if the
 // sequence must be skipped.
 __device__ __forceinline__ int start_len(const CacheDst &c, int b) {
