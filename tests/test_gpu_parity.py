@@ -214,6 +214,11 @@ DECODE_CASES = [
     (4, 0, 4, [4, 3, 20, 257, 1500]),
     (8, 1, 17, [16, 17, 18, 600]),
     (4, 1, 0, [2048, 1, 999]),
+    # many sequences: up to 32 the split kernel sets its schedule up per
+    # thread, above 32 through a scan over the CTA (both sides of the switch)
+    (1, 0, 0, [1 + (37 * i) % 200 for i in range(32)]),
+    (2, 1, 4, [1 + (53 * i) % 260 for i in range(33)]),
+    (4, 0, 0, [16 * (1 + i % 7) + i % 3 for i in range(40)]),
 ]
 
 

@@ -125,6 +125,32 @@ def test_rotation_invariance_of_attention(mode):
     assert np.max(np.abs(back - ref)) <= (1e-6 if mode == 0 else 1e-12)
 
 
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_rotation_lowers_int2_error_on_outlier_channels(seed):
+    """The pages' reason for rotating (KVLinC abstract: the Hadamard rotation
+    reduces quantization error; RotateKV abstract item (i): outlier-aware
+    rotation; OptR introduction): keys with a few channels 20x larger than
+    the rest, quantized to INT2 in groups of 32, come back closer to the
+    input when they are rotated first (dense orthogonal R or perm + FWHT)
+    and the rotation is removed after dequantisation than when they are
+    quantized as they are."""
+    rng = np.random.default_rng(100 + seed)
+    K = rng.standard_normal((256, D))
+    K[:, rng.choice(D, 8, replace=False)] *= 20
+    kb = orc.f32_to_f16_bits(K.astype(np.float32))
+    Kh = orc.f16_bits_to_f32(kb).astype(np.float64)
+
+    def rel_error(mode, **kw):
+        c, s, z = orc.quantize_rows(orc.rotate_rows_f32(kb, mode, **kw))
+        back = orc.unrotate_f64(np_mini.dequant(c, s, z), mode, **kw)
+        return np.linalg.norm(back - Kh) / np.linalg.norm(Kh)
+
+    plain = rel_error(0, R=np.eye(D, dtype=np.float32))
+    dense = rel_error(0, R=rand_orth(rng).astype(np.float32))
+    fwht = rel_error(1, perm=rng.permutation(D).astype(np.int32))
+    assert dense < 0.85 * plain and fwht < 0.85 * plain, (plain, dense, fwht)
+
+
 def test_attention_f64_against_scipy_softmax():
     rng = np.random.default_rng(5)
     L = 9
