@@ -253,14 +253,22 @@ def kvq_identify_sinks(act, tau, cache, seq_lens, stream=None):
                                     _ptr(seq_lens), _stream(stream, act)))
 
 
+def _sm_count(device=None):
+    """SM count of `device` (default: the current CUDA device); the library
+    sizes its split from the SM count of the device the call runs on."""
+    d = torch.device("cuda" if device is None else device)
+    idx = d.index if d.index is not None else torch.cuda.current_device()
+    return torch.cuda.get_device_properties(idx).multi_processor_count
+
+
 def kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count=None):
     if sm_count is None:
-        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        sm_count = _sm_count()
     return lib().kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, sm_count)
 
 
 def decode_workspace(B, Hq, Hkv, max_ctx, device="cuda"):
-    n = kvq_decode_workspace_size(B, Hq, Hkv, max_ctx)
+    n = kvq_decode_workspace_size(B, Hq, Hkv, max_ctx, _sm_count(device))
     if n == 0:
         raise ValueError("bad decode shape")
     return torch.empty(n, dtype=torch.uint8, device=device)
@@ -323,12 +331,12 @@ def _need_host(t, dtype, name, shape=None):
 
 def kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx, sm_count=None):
     if sm_count is None:
-        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        sm_count = _sm_count()
     return lib().kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx, sm_count)
 
 
 def step_workspace(B, T, Hq, Hkv, max_ctx, device="cuda"):
-    n = kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx)
+    n = kvq_step_workspace_size(B, T, Hq, Hkv, max_ctx, _sm_count(device))
     if n == 0:
         raise ValueError("bad step shape")
     return torch.empty(n, dtype=torch.uint8, device=device)
@@ -472,12 +480,12 @@ def kvq_prerope_append(K, V, group_heads, perm, cache, seq_lens, stream=None):
 
 def kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx, sm_count=None):
     if sm_count is None:
-        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        sm_count = _sm_count()
     return lib().kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx, sm_count)
 
 
 def prerope_workspace(B, Hq, Hkv, group_heads, max_ctx, device="cuda"):
-    n = kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx)
+    n = kvq_prerope_workspace_size(B, Hq, Hkv, group_heads, max_ctx, _sm_count(device))
     if n == 0:
         raise ValueError("bad pre-RoPE decode shape")
     return torch.empty(n, dtype=torch.uint8, device=device)
