@@ -622,6 +622,35 @@ def test_rope_is_the_complex_rotation(base):
     assert np.count_nonzero(r) == 2
 
 
+@pytest.mark.parametrize("gh", [1, 4])
+def test_prerope_score_has_a_query_side_form(gh):
+    """The pre-RoPE score needs no per-position un-rotation of the key: with
+    k_hat the cached (group-rotated) key row, M the group rotation and x the
+    head's slice of k_hat M^T, the RoPE'd score q . RoPE_t(x) equals
+    sum_c cos(t theta_c) (k_hat . a_c) + sin(t theta_c) (k_hat . b_c), where
+    a_c = q_c M[c] + q_{c+64} M[c+64] and b_c = q_{c+64} M[c] - q_c M[c+64]
+    (rows of M at the head's offset) are fixed per query: RoPE's pairs
+    (c, c+64) turn by t theta_c, and M is orthogonal."""
+    rng = np.random.default_rng(31 + gh)
+    n = D * gh
+    M = np_mini.group_rotation_matrix(rng.permutation(n))
+    j, base = gh - 1, 10000.0
+    q = rng.standard_normal(D)
+    khat = rng.standard_normal((6, n))
+    ts = np.array([0, 1, 2, 17, 4096, 131071])
+    direct = np.array([q @ np_mini.rope_complex((khat[i] @ M.T)[j * D:(j + 1) * D], t, base)
+                       for i, t in enumerate(ts)])
+    Mj = M[j * D:(j + 1) * D]                   # rows of the head's channels
+    h = D // 2
+    a = q[:h, None] * Mj[:h] + q[h:, None] * Mj[h:]
+    b = q[h:, None] * Mj[:h] - q[:h, None] * Mj[h:]
+    theta = np.power(base, -2.0 * np.arange(h) / D)
+    query_side = np.array([np.cos(t * theta) @ (a @ khat[i]) + np.sin(t * theta) @ (b @ khat[i])
+                           for i, t in enumerate(ts)])
+    assert np.allclose(query_side, direct, rtol=1e-10, atol=1e-10)
+
+
+
 @pytest.mark.parametrize("gh", [1, 2, 4, 8])
 def test_group_rotation_is_the_permuted_hadamard_matrix(gh):
     n = D * gh
