@@ -579,3 +579,30 @@ def test_append_decode_host_equals_the_device_step(mode):
     torch.cuda.synchronize()
     assert torch.equal(cache.blocks, before) and not hO.any()
     assert list(sl.cpu().numpy()) == [120 + T, 53 + T]
+
+
+def test_append_decode_host_rejects_bad_calls():
+    """Bad host-step calls fail before anything is enqueued: no rows (null
+    input), a workspace off its 256-byte alignment, an output of the wrong
+    shape, a device tensor where a host one belongs."""
+    w = W.custom(seed=320, B=1, Hq=2, Hkv=2, mode=0)
+    rt, _ = rot_tensors(w)
+    cache = kvq.KVCache(1, 2, 64)
+    sl = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Q = torch.zeros((1, 2, 128), dtype=torch.float16).pin_memory()
+    hO = torch.zeros((1, 2, 128), dtype=torch.float16).pin_memory()
+    ws = kvq.step_workspace(1, 1, 2, 2, 64)
+    K0 = torch.zeros((1, 0, 2, 128), dtype=torch.float16)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_append_decode_host(K0, K0, Q, cache, 0, *rt, sl, 64, ws, hO)
+    assert e.value.code == 1                               # KVQ_ERR_INVALID_ARG
+    K1 = torch.zeros((1, 1, 2, 128), dtype=torch.float16).pin_memory()
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_append_decode_host(K1, K1, Q, cache, 0, *rt, sl, 64, ws[16:], hO)
+    assert e.value.code == 2                               # KVQ_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        kvq.kvq_append_decode_host(K1, K1, Q, cache, 0, *rt, sl, 64, ws, hO[:, :1])
+    with pytest.raises(ValueError):
+        kvq.kvq_append_decode_host(K1.cuda(), K1, Q, cache, 0, *rt, sl, 64, ws, hO)
+    torch.cuda.synchronize()
+    assert list(sl.cpu().numpy()) == [0] and kvq.kvq_get_status(cache) == 0
