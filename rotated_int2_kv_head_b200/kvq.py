@@ -347,7 +347,9 @@ def kvq_append_decode_host(K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, 
     """The serving step with host tensors (pin them): K, V fp16 [B][T][Hkv][128]
     and Q fp16 [B][Hq][128] are copied in, appended and decoded, and the output
     copied back into out_host, all queued on the stream (synchronise before
-    reading out_host).  workspace: step_workspace(...) on the device."""
+    reading out_host).  K, V and Q that are consecutive views of one buffer
+    (V right after K, Q right after V) go in with a single copy.
+    workspace: step_workspace(...) on the device."""
     B, T, Hkv, d = K_host.shape
     _need_host(K_host, torch.float16, "K_host", (cache.B, T, cache.Hkv, D))
     _need_host(V_host, torch.float16, "V_host", K_host.shape)
