@@ -105,3 +105,42 @@ def test_workspace_size_is_monotone_and_validated(L):
 def test_cache_bytes(L):
     assert L.kvq_cache_bytes(1, 32, 32768) == 32 * 2048 * 1536
     assert L.kvq_cache_bytes(1, 1, 17) == 0
+
+
+def test_step_calls_reject_bad_arguments_on_host(L):
+    """kvq_append_decode and kvq_append_decode_host check every argument of
+    both halves before anything reaches the GPU."""
+    def dev(cache, T=1, Hq=2, K=8192, Q=8192, ws=4096, max_ctx=64, out=8192):
+        return L.kvq_append_decode(K, K, T, Q, Hq, C.byref(cache), 0, 1024, 1024, None, 512,
+                                   max_ctx, ws, 1 << 24, out, None)
+
+    def host(cache, T=1, Hq=2, K=8192, Q=8192, ws=4096, out=8192):
+        return L.kvq_append_decode_host(K, K, T, Q, Hq, C.byref(cache), 0, 1024, 1024, None, 512,
+                                        64, ws, 1 << 24, out, None)
+
+    assert dev(desc(head_dim=64)) == 2         # UNSUPPORTED
+    assert dev(desc(), K=0) == 1               # append half: no rows
+    assert dev(desc(), T=65) == 1              # T > capacity
+    assert dev(desc(), Q=0) == 1               # decode half: no queries
+    assert dev(desc(), ws=4100) == 2           # workspace alignment
+    assert dev(desc(), Hq=3) == 1              # Hq not a multiple of Hkv
+    assert dev(desc(), Hq=6) == 2              # G = 3
+    assert dev(desc(), max_ctx=0) == 1
+    assert dev(desc(), max_ctx=65) == 1
+    assert host(desc(head_dim=64)) == 2
+    assert host(desc(), K=0) == 1
+    assert host(desc(), out=0) == 1
+    assert host(desc(), T=0) == 1              # the host step always carries rows
+    assert host(desc(), ws=4100) == 2
+    assert host(desc(), Hq=3) == 1
+
+
+def test_step_workspace_size(L):
+    f, g = L.kvq_step_workspace_size, L.kvq_decode_workspace_size
+    assert f(1, 0, 32, 32, 32768, 148) == 0
+    assert f(0, 1, 32, 32, 32768, 148) == 0
+    for B, T, Hq, Hkv in [(1, 1, 32, 32), (8, 3, 32, 8), (64, 128, 32, 32)]:
+        n, d = f(B, T, Hq, Hkv, 32768, 148), g(B, Hq, Hkv, 32768, 148)
+        assert n % 256 == 0
+        # the decode workspace, then K, V [B][T][Hkv][128] and Q, out [B][Hq][128] in fp16
+        assert n >= d + 2 * B * T * Hkv * 256 + 2 * B * Hq * 256
