@@ -144,3 +144,54 @@ def test_step_workspace_size(L):
         assert n % 256 == 0
         # the decode workspace, then K, V [B][T][Hkv][128] and Q, out [B][Hq][128] in fp16
         assert n >= d + 2 * B * T * Hkv * 256 + 2 * B * Hq * 256
+
+
+def test_prerope_and_sink_calls_reject_bad_arguments_on_host(L):
+    """The pre-RoPE pair, its workspace size and sink identification check
+    their arguments on the host before any launch."""
+    def papp(cache, T=3, gh=1, K=8192, perm=2048):
+        return L.kvq_prerope_append(K, K, T, gh, perm, C.byref(cache), 512, None)
+
+    assert papp(desc(head_dim=64)) == 2
+    assert papp(desc(), gh=3) == 2               # group of 3 heads
+    assert papp(desc(), gh=4) == 2               # 4 does not divide Hkv = 2
+    assert papp(desc(), perm=0) == 1
+    assert papp(desc(), perm=2052) == 2          # perm off its 16-byte alignment
+    assert papp(desc(), T=-1) == 1
+    assert papp(desc(), T=0) == 0                # nothing to do
+    assert papp(desc(), K=0) == 1
+    assert papp(desc(), K=8200) == 2
+    assert papp(desc(), T=65) == 1               # T > capacity
+
+    def pdec(cache, Hq=2, gh=1, Q=8192, ws=4096, base=10000.0, max_ctx=64):
+        return L.kvq_prerope_decode(Q, Hq, C.byref(cache), gh, 2048, base, 512, max_ctx, ws,
+                                    1 << 24, 8192, None)
+
+    assert pdec(desc(), gh=3) == 2
+    assert pdec(desc(), Q=0) == 1
+    assert pdec(desc(), ws=4100) == 2
+    assert pdec(desc(), Hq=3) == 1
+    assert pdec(desc(), Hq=16, gh=2) == 2        # G * group_heads = 16 > 8
+    assert pdec(desc(), base=1.0) == 1           # RoPE base must exceed 1
+    assert pdec(desc(), base=float("nan")) == 1
+    assert pdec(desc(), max_ctx=0) == 1
+    assert pdec(desc(), max_ctx=65) == 1
+
+    f = L.kvq_prerope_workspace_size
+    assert f(1, 32, 32, 3, 32768, 148) == 0      # group of 3 heads
+    assert f(1, 32, 32, 1, 0, 148) == 0
+    assert f(1, 32, 32, 1, 32768, 148) > 0
+
+    def ident(cache, act=8192, T=4, tau=100.0):
+        return L.kvq_identify_sinks(act, T, tau, C.byref(cache), 512, None)
+
+    with_sinks = dict(sink_fp16=4, k_sink=8192, v_sink=8192)
+    assert ident(desc(**with_sinks)) == 1        # no sink list in the descriptor
+    d = desc(**with_sinks)
+    d.sink_pos, d.sink_count = 1024, 1536
+    assert ident(d, act=0) == 1
+    assert ident(d, T=0) == 1
+    assert ident(d, act=8194) == 2               # act off its 4-byte alignment
+    assert ident(d, T=65) == 1                   # T > capacity
+    d.sink_count = None
+    assert ident(d) == 1                         # a sink list without its counts
