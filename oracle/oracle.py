@@ -6,7 +6,6 @@ exact dtype the C side expects.  Cache buffers use the library's byte format
 (blocks of 16 tokens, 1536 bytes), so results can be compared byte for byte.
 """
 import ctypes as C
-import os
 
 import numpy as np
 

@@ -3,7 +3,6 @@ ranks, per-rank batches) on 2 CPU ranks with the gloo backend."""
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))

@@ -1,7 +1,6 @@
 """Host-side arithmetic of bench.py: the algorithmic bytes a decode reads,
 the number of layers cycled to keep the cache out of L2, and the source hash
 that ties a committed ncu summary to the kernel it measured.  CPU only."""
-import os
 
 import bench
 import workloads as W

@@ -29,7 +29,7 @@ CPU and CUDA generators differ): a comparison draws once, on one device, and
 hands the same tensor to both sides.
 """
 from dataclasses import dataclass, field
-from typing import List, Optional
+from typing import Optional
 
 import numpy as np
 import torch
