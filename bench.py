@@ -2,30 +2,37 @@
 """Benchmark of the rotated INT2 KV-cache hot path on B200.
 
 One step = rotate-quantize-append of the step's new token(s) + decode
-attention of one query per head over the packed cache (the whole hot path),
-on the "llama7b" workload by default: B=1, 32 heads (MHA), head_dim 128,
-context 32768 (32767 prefilled + 1 appended per step), dense per-head
-rotations, INT2 group 32 with fp16 scale/zero.  Inputs are seeded synthetic
-tensors (workloads.py).
+attention of one query per head over the packed cache (the whole hot path).
+The default workload is the largest single-GPU one, "ragged": a serving
+batch of B=64 sequences with context lengths drawn uniformly from [1024,
+65536] (seeded; 6.5 GB of packed cache read per step), 32 heads (MHA),
+head_dim 128, dense per-head rotations, INT2 group 32 with fp16 scale/zero;
+each step appends one token per sequence, then decodes one query per head.
+Beside it: the single-layer llama7b step (B=1, 32 heads, context 32768),
+the bulk appends (the ragged workload's 4 x 32768-token prefill among
+them), the decode of every workload, the extensions, and the CPU oracle on a
+bounded sample.  Inputs are seeded synthetic tensors (workloads.py).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the CPU oracle as reference arm
     torchrun --nproc-per-node N bench.py --gpus N ...
 
-Timing: K steps run back to back on the launching stream between one pair
-of CUDA events, with a barrier + synchronize on both sides; the max over
-ranks is reported.  The steps are replayed from a CUDA graph (whole rounds
-over the layers, with their programmatic dependent launches), as a serving
-loop would run them, so the host's launch cost stays out of the device
-time; `e2e` still drives every step through the public API.  L2 (126 MB) must not serve the cache across steps: a
-cache smaller than 3x L2 is replicated into independent layers (distinct
-memory, same contents, like the layers of a model) that the steps cycle
-through, so every step reads a cache that at least 3x L2 of other cache
-traffic has passed through L2 since its last use.  Each step appends at the
-same position (its own row of pre-append lengths), so the context is the
-same for every step.  A cache too small for 64 layers to cover that falls
-back to flushing L2 between steps (256 MB written, then 256 MB read, so L2
-holds clean lines) with each step bracketed by its own events.  The
+Timing: exactly K steps run back to back on the launching stream between
+one pair of CUDA events, with a barrier + synchronize on both sides; the
+max over ranks is reported.  The steps are replayed from CUDA graphs (whole
+rounds over the layers plus one graph of the remainder, with their
+programmatic dependent launches), as a serving loop would run them, so the
+host's launch cost stays out of the device time; `e2e` still drives every
+step through the public API.  L2 (126 MB) must not serve the cache across
+steps: a cache larger than 3x L2 (ragged: 12.9 GB allocated) is read
+afresh by every step; a smaller one is replicated into independent layers
+(distinct memory, same contents, like the layers of a model) that the steps
+cycle through, so every step reads a cache that at least 3x L2 of other
+cache traffic has passed through L2 since its last use.  Each step appends
+at the same position (its own row of pre-append lengths), so the context is
+the same for every step.  A cache too small for 64 layers to cover that
+falls back to flushing L2 between steps (256 MB written, then 256 MB read,
+so L2 holds clean lines) with each step bracketed by its own events.  The
 isolated-step latency (flush, then one step between its own events) is
 reported beside the throughput.  With N GPUs every rank serves its own
 independent batch (weak scaling, no collective on the data path).
@@ -119,7 +126,7 @@ class ClockSampler:
                0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
                0x200: "display_clock_setting"}
 
-    def __init__(self, index, period=0.005):
+    def __init__(self, index, period=0.002):
         self.samples, self.reasons, self.ok = [], set(), False
         self.period, self.stop_flag = period, threading.Event()
         try:
@@ -184,9 +191,12 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """dram bytes per launch of the split kernel from the committed ncu summary,
-    if it was taken on the current kernel source; else None."""
+def profiled_traffic(workload, kv_bytes=None):
+    """dram bytes per launch of the split kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None.  A
+    summary taken on a smaller case of the workload (its
+    algorithmic_bytes_per_launch below kv_bytes) is scaled to a full launch
+    by the ratio of algorithmic bytes (the units processed)."""
     p = os.path.join(ROOT, "profiles", "decode_split_%s.txt" % workload)
     if not os.path.exists(p):
         return None
@@ -194,13 +204,20 @@ def profiled_traffic(workload):
     for line in open(p):
         if ":" in line:
             k, v = line.split(":", 1)
-            vals[k.strip()] = v.strip()
+            vals[k.strip()] = v.strip().split()[0] if v.strip() else ""
     if vals.get("source_sha256") != kernel_source_sha():
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        dram = float(vals["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
+    try:
+        alg = float(vals["algorithmic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        alg = None
+    if kv_bytes is not None and alg:
+        dram *= kv_bytes / alg
+    return dram
 
 
 def packed_kv_bytes(w, lens):
@@ -362,13 +379,14 @@ def append_rates(device, peak, reps=5):
     return out
 
 
-def extension_rates(step, device, reps=50):
+def extension_rates(device, reps=50):
     """Decode-only timings (L2 flushed before each call, events around it) of
-    the serving extensions on the workload's cache (layer 0): the plain
-    decode, the same cache paged through a random block table (one pool
-    block per 16 tokens x all heads), and q_len = 4 new tokens per sequence
-    (each attending causally)."""
+    the serving extensions on the llama7b cache (B=1, 32 heads, context
+    32768): the plain decode, the same cache paged through a random block
+    table (one pool block per 16 tokens x all heads), and q_len = 4 new
+    tokens per sequence (each attending causally)."""
     import rotated_int2_kv_head_b200 as kvq
+    step = Step(W.WORKLOADS["llama7b"], device, 1)
     w = step.w
     cache, Rk, Rv, perm = step.layers[0]
     L = step.L
@@ -626,59 +644,115 @@ def prerope_rates(device, reps=20):
     return res
 
 
-def cpu_baseline(w, step, device, heads=4, min_seconds=5.0):
-    """The CPU oracle, as it stands, on a bounded sample of the same workload:
-    the first `heads` KV heads of sequence 0 (their K/V rows are the very
-    tensors the GPU arm used), timed for append + decode, scaled to the
-    whole step."""
-    from oracle import oracle as orc
+def sample_sequence(lens):
+    """The sequence whose length is the batch median (the lower middle one
+    for an even batch; the first of equal lengths): the CPU oracle's sample
+    of a ragged batch."""
+    order = np.argsort(np.asarray(lens), kind="stable")
+    return int(order[(len(order) - 1) // 2])
+
+
+def sample_scale(w, lens, b, heads):
+    """Factor from the oracle's sample (KV heads 0..heads-1 of sequence b) to
+    the whole step: decode work grows with the context, so the factor is the
+    batch's context token-heads over the sample's, sum_b' L_b' * Hkv /
+    (L_b * heads); for a uniform batch it is B * Hkv / heads."""
+    lens = np.asarray(lens, np.int64)
+    return float(lens.sum()) * w.Hkv / (float(lens[b]) * heads)
+
+
+class OracleSample:
+    """The CPU oracle holding one sequence's cache for the first `heads` KV
+    heads, filled to the step's pre-append length, ready to run the step's
+    append of T tokens and its decode; rows drawn on `device` (the very
+    tensors the GPU arm used, when given that arm's Step)."""
+
+    def __init__(self, w, b, heads, device, step=None):
+        from oracle import oracle as orc
+        self.orc, self.w, self.b, self.heads = orc, w, b, heads
+        lens = w.seq_lens()
+        self.L, T = int(lens[b]), w.append_T
+        self.pre = self.L - T
+        Rk, Rv, perm = W.rotations(w)
+        self.rk = Rk[:heads] if Rk is not None else None
+        self.rv = Rv[:heads] if Rv is not None else None
+        self.pm = perm[:, :heads] if perm is not None else None
+        self.oc = orc.Cache(1, heads, ((self.L + 15) // 16) * 16, w.sink)
+        self.sl = np.zeros(1, np.int32)
+        for t0 in range(0, self.pre, 4096):
+            t1 = min(self.pre, t0 + 4096)
+            K, V = W.kv_batch(w, t0, t1, device, bs=[b])
+            orc.append(self.oc, W.f16_bits(K[:, :, :heads]), W.f16_bits(V[:, :, :heads]), w.mode,
+                       self.rk, self.rv, self.pm, self.sl)
+        if step is not None:
+            Kn, Vn, Q = step.Knew[b:b + 1], step.Vnew[b:b + 1], step.Q[b:b + 1]
+        else:
+            Kn, Vn = W.kv_batch(w, self.pre, self.L, device, bs=[b])
+            Q = W.queries(w, device)[b:b + 1]
+        self.Kn = W.f16_bits(Kn[:, :, :heads])
+        self.Vn = W.f16_bits(Vn[:, :, :heads])
+        self.Q = W.f16_bits(Q[:, :heads * w.G])
+        self.cores = len(os.sched_getaffinity(0))
+
+    def step(self):
+        """The step's append of T tokens at the pre-append length, then the
+        decode over the sample's context (OpenMP over the cores)."""
+        self.sl[0] = self.pre
+        self.orc.append(self.oc, self.Kn, self.Vn, self.w.mode, self.rk, self.rv, self.pm, self.sl)
+        self.orc.decode(self.oc, self.Q, self.w.mode, self.rk, self.rv, self.pm, self.sl,
+                        n_threads=self.cores)
+
+    def describe(self, n, el, scale):
+        return ("sequence %d (context %d, the batch median), KV heads 0..%d of %d: append %d "
+                "token(s) + decode, %d sample steps in %.2f s; per-step time scaled by %.1f "
+                "(the batch's context token-heads over the sample's)"
+                % (self.b, self.L, self.heads - 1, self.w.Hkv, self.w.append_T, n, el, scale))
+
+
+def cpu_baseline(w, step, device, heads=2, min_seconds=5.0):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload
+    (the first `heads` KV heads of the batch's median-length sequence; its
+    rows drawn on `device`, or the GPU arm's own step inputs when `step` is
+    given), timed for append + decode and scaled to the whole step by
+    sample_scale."""
+    lens = w.seq_lens()
+    b = sample_sequence(lens)
     heads = min(heads, w.Hkv)
-    pre = step.L - step.T
-    Rk, Rv, perm = step.rot_np
-    rk = Rk[:heads] if Rk is not None else None
-    rv = Rv[:heads] if Rv is not None else None
-    pm = perm[:, :heads] if perm is not None else None
-    oc = orc.Cache(1, heads, step.cap, w.sink)
-    sl = np.zeros(1, np.int32)
-    for t0 in range(0, pre, 4096):
-        t1 = min(pre, t0 + 4096)
-        K, V = W.kv_batch(w, t0, t1, device, bs=[0])
-        orc.append(oc, W.f16_bits(K[:, :, :heads]), W.f16_bits(V[:, :, :heads]), w.mode, rk, rv,
-                   pm, sl)
-    Kn = W.f16_bits(step.Knew[:1, :, :heads])
-    Vn = W.f16_bits(step.Vnew[:1, :, :heads])
-    Qs = W.f16_bits(step.Q[:1, :heads * w.G])
-    cores = len(os.sched_getaffinity(0))
+    smp = OracleSample(w, b, heads, device, step)
     n, t_start = 0, time.perf_counter()
     while True:
-        sl[0] = pre
-        orc.append(oc, Kn, Vn, w.mode, rk, rv, pm, sl)
-        orc.decode(oc, Qs, w.mode, rk, rv, pm, sl, n_threads=cores)
+        smp.step()
         n += 1
         el = time.perf_counter() - t_start
         if el >= min_seconds or n >= 1000:
             break
-    per_step = el / n * (w.Hkv / heads) * w.B
-    return {"value": w.B / per_step, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "sequence 0, KV heads 0..%d of %d (append %d token + decode over %d), "
-                      "%d steps in %.1f s, scaled by %d/%d heads and B=%d"
-                      % (heads - 1, w.Hkv, step.T, step.L, n, el, w.Hkv, heads, w.B)}
+    scale = sample_scale(w, lens, b, heads)
+    per_step = el / n * scale
+    return {"value": w.B / per_step, "unit": "tokens/s", "cores": smp.cores, "kind": "oracle",
+            "sample": smp.describe(n, el, scale)}
 
 
-def run_cuda(args):
-    rank, world, local = dist_env()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    dist_on = init_dist("nccl", world)
-    from rotated_int2_kv_head_b200 import build as kbuild
-    kbuild.build()
-    w = rank_workload(W.WORKLOADS[args.workload], rank)
+def graph_plan(K, n_layers, per_graph_target=40):
+    """Exactly K steps as CUDA-graph replays: (per_graph, full, remainder) =
+    `full` replays of a graph of per_graph steps (whole rounds over the
+    layers) and, if remainder > 0, one replay of a graph of the remaining
+    steps."""
+    per_graph = n_layers * max(1, per_graph_target // n_layers)
+    return per_graph, K // per_graph, K % per_graph
+
+
+def measure_step(w, dev, K, warmup, dist_on, local, e2e=True):
+    """Times K steps (append + decode) of workload w on device dev: the
+    throughput loop (graph replay over independent layers, or flushed
+    single steps for caches too small for layers), the split kernel alone by
+    library events, the isolated flushed step, and (e2e) the host-buffer
+    step through kvq_append_decode_host.  Returns a dict of raw timings."""
+    import rotated_int2_kv_head_b200 as kvq
     lens = w.seq_lens()
     cap = ((int(lens.max()) + 15) // 16) * 16
     n_layers = layers_for(w.B * w.Hkv * (cap // 16) * 1536)
     step = Step(w, dev, max(1, n_layers))
     flush = L2Flush(dev) if n_layers == 0 else None
-    K = args.steps
 
     def steps(n, sl, timed=None, split_events=None):
         """n steps; with `timed`, one event pair around all of them (layers
@@ -702,52 +776,60 @@ def run_cuda(args):
             ms = timed[0].elapsed_time(timed[1])
         return ms
 
-    steps(args.warmup, step.lengths(args.warmup))
+    steps(warmup, step.lengths(warmup))
     torch.cuda.synchronize(dev)
     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    graph = None
+    graphs = []
+    per_graph = 0
     if flush is None:
-        # Layers mode: the steps are replayed from a CUDA graph, as a serving
+        # Layers mode: the steps are replayed from CUDA graphs, as a serving
         # loop would, so the host's per-call launch cost (about 33 us per
         # step through the Python binding) stays out of the device timing.
-        # One graph = `per_graph` consecutive steps (whole rounds over the
-        # layers): a copy that resets its rows of pre-append lengths, then
-        # the steps' kernels with their programmatic dependent launches.
-        per_graph = len(step.layers) * max(1, 40 // len(step.layers))
-        sl_g = step.lengths(per_graph)
-        sl_init = sl_g.clone()
+        # A graph = a copy that resets its rows of pre-append lengths, then
+        # its steps' kernels with their programmatic dependent launches;
+        # exactly K steps run: `full` graphs of per_graph steps, then one of
+        # the remainder.
+        per_graph, full, rem = graph_plan(K, len(step.layers))
         side = torch.cuda.Stream(dev)
-        side.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(side):
-            for k in range(per_graph):
-                step.run(k, sl_g[k])
-        torch.cuda.current_stream(dev).wait_stream(side)
+        for n_g, reps in ((per_graph, full), (rem, 1)):
+            if n_g == 0 or reps == 0:
+                continue
+            sl_g = step.lengths(n_g)
+            sl_init = sl_g.clone()
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                for k in range(n_g):
+                    step.run(k, sl_g[k])
+            torch.cuda.current_stream(dev).wait_stream(side)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                sl_g.copy_(sl_init)
+                for k in range(n_g):
+                    step.run(k, sl_g[k])
+            graphs.append((g, reps, sl_g, sl_init))
+        for _ in range(max(1, -(-warmup // max(1, per_graph)))):
+            graphs[0][0].replay()
         torch.cuda.synchronize(dev)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            sl_g.copy_(sl_init)
-            for k in range(per_graph):
-                step.run(k, sl_g[k])
-        for _ in range(max(1, -(-args.warmup // per_graph))):
-            graph.replay()
-        torch.cuda.synchronize(dev)
-        K = per_graph * max(1, round(K / per_graph))
-    sl = step.lengths(K) if graph is None else None
+    sl = step.lengths(K) if not graphs else None
     with ClockSampler(local) as clk:
         barrier(dist_on, dev)
         torch.cuda.synchronize(dev)
-        if graph is None:
+        if not graphs:
             total_ms = steps(K, sl, ev)
         else:
             ev[0].record()
-            for _ in range(K // per_graph):
-                graph.replay()
+            for g, reps, _, _ in graphs:
+                for _ in range(reps):
+                    g.replay()
             ev[1].record()
             torch.cuda.synchronize(dev)
             total_ms = ev[0].elapsed_time(ev[1])
         torch.cuda.synchronize(dev)
         barrier(dist_on, dev)
+    steps_run = K
     total_ms = max_over_ranks(total_ms, dist_on, dev)
+    del graphs
 
     # the streaming kernel alone, timed live by events the library records
     # around it (a separate loop: events between kernels stop the
@@ -761,9 +843,9 @@ def run_cuda(args):
     sl_split = step.lengths(n_split)
     torch.cuda.synchronize(dev)
     # The host takes about as long to submit a step as the device takes to
-    # run it, so a kernel could wait on its own submission between the
-    # events.  torch's spin kernel (a fixed cycle count) at the head of the
-    # stream lets the host queue every step before the first one runs.
+    # run a small one, so a kernel could wait on its own submission between
+    # the events.  torch's spin kernel (a fixed cycle count) at the head of
+    # the stream lets the host queue every step before the first one runs.
     host_ahead(n_split * 80e-6 + 2e-3)
     steps(n_split, sl_split, None, split_ev)
     torch.cuda.synchronize(dev)
@@ -771,7 +853,7 @@ def run_cuda(args):
 
     # one step at a time after an L2 flush, each bracketed by its own events
     # (the latency of an isolated step, for reference)
-    n_iso = min(K, 200)
+    n_iso = min(K, 50)
     iso_flush = flush or L2Flush(dev)
     sl_iso = step.lengths(n_iso)
     iso_ms = []
@@ -786,14 +868,17 @@ def run_cuda(args):
     del iso_flush
     if step.status() != 0:
         raise RuntimeError("device status %d after timed steps" % step.status())
+    res = {"step": step, "n_layers": n_layers, "total_ms": total_ms, "steps": steps_run,
+           "per_graph": per_graph, "split_ms": split_ms, "iso_ms": iso_ms,
+           "clocks": clk.summary()}
+    if not e2e:
+        return res
 
     # end to end through the C-ABI call with host buffers: one
     # kvq_append_decode_host per step copies the step's new K/V rows and
     # queries in from pinned memory, appends, decodes and copies the output
-    # back; the host then waits for the stream
-    import rotated_int2_kv_head_b200 as kvq
-    # the inputs are views of one pinned buffer, back to back, so the call
-    # moves them with a single copy
+    # back; the host then waits for the stream.  The inputs are views of one
+    # pinned buffer, back to back, so the call moves them with a single copy.
     hIn = step.inbuf.cpu().pin_memory()
     nk = step.Knew.numel()
     hK = hIn[:nk].view(step.Knew.shape)
@@ -816,10 +901,56 @@ def run_cuda(args):
         if k >= 3:
             e2e_s += time.perf_counter() - t0
     e2e_s = max_over_ranks(e2e_s, dist_on, dev)
-    h2d = (hK.numel() + hV.numel() + hQ.numel()) * 2
-    d2h = hO.numel() * 2
     if not torch.equal(hO.to(dev), step.out):      # the same step as the device-timed one
         raise RuntimeError("host-buffer step output differs from the device step")
+    res.update(e2e_s=e2e_s, n_e2e=n_e2e, h2d=(hK.numel() + hV.numel() + hQ.numel()) * 2,
+               d2h=hO.numel() * 2)
+    return res
+
+
+def l2_note(m):
+    step, n_layers = m["step"], m["n_layers"]
+    if n_layers == 0:
+        return "flushed between steps (256 MB write, then 256 MB read); steps timed one by one"
+    if n_layers > 1:
+        note = ("inputs larger than L2: %d independent layers (%.1f MB of cache each) cycled, so "
+                "each step reads a cache %d other steps (%.0f MB) after its last use; steps back "
+                "to back" % (n_layers, step.cache_bytes / 1e6, n_layers - 1,
+                             (n_layers - 1) * step.cache_bytes / 1e6))
+    else:
+        note = ("inputs larger than L2 (one %.0f MB cache, %.0f MB of it read per step); steps "
+                "back to back" % (step.cache_bytes / 1e6, packed_kv_bytes(step.w, step.w.seq_lens())
+                                  / 1e6))
+    return note + "; timed steps replayed from CUDA graphs of %d steps (+ one of the remainder)" \
+        % m["per_graph"]
+
+
+def split_roofline(w, m, peak, peak_src, workload):
+    kv_bytes = packed_kv_bytes(w, w.seq_lens())
+    split_mean_s = float(np.mean(m["split_ms"])) * 1e-3
+    achieved = kv_bytes / split_mean_s / 1e9
+    return {"bound": "hbm", "kernel": "decode_split_kernel (streams the packed cache)",
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": profiled_traffic(workload, kv_bytes),
+            "algorithmic_bytes_per_launch": kv_bytes, "kernel_ms_mean": split_mean_s * 1e3,
+            "peak_source": peak_src,
+            "timing": "CUDA events the library records around the kernel, %d eager steps "
+                      "queued behind a spin kernel (no host gap inside the events)"
+                      % len(m["split_ms"])}
+
+
+def run_cuda(args):
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_on = init_dist("nccl", world)
+    from rotated_int2_kv_head_b200 import build as kbuild
+    kbuild.build()
+    w = rank_workload(W.WORKLOADS[args.workload], rank)
+    lens = w.seq_lens()
+    K = args.steps
+    m = measure_step(w, dev, K, args.warmup, dist_on, local)
+    step = m["step"]
 
     if rank != 0:
         if dist_on:
@@ -828,26 +959,14 @@ def run_cuda(args):
         return
     peak, peak_src = measured_peak()
     kv_bytes = packed_kv_bytes(w, lens)
-    split_mean_s = float(np.mean(split_ms)) * 1e-3
-    achieved = kv_bytes / split_mean_s / 1e9
-    ms_per_step = total_ms / K
+    ms_per_step = m["total_ms"] / K
     tokens = w.B * world
-    if n_layers == 0:
-        l2_note = "flushed between steps (256 MB write, then 256 MB read); steps timed one by one"
-    else:
-        l2_note = ("inputs larger than L2: %d independent layers (%.1f MB of cache each) cycled, "
-                   "so each step reads a cache %d other steps (%.0f MB) after its last use; "
-                   "steps back to back" % (n_layers, step.cache_bytes / 1e6, n_layers - 1,
-                                           (n_layers - 1) * step.cache_bytes / 1e6)
-                   if n_layers > 1 else "inputs larger than L2 (one %.0f MB cache); steps back "
-                   "to back" % (step.cache_bytes / 1e6))
-        l2_note += "; timed steps replayed from a CUDA graph of %d steps" % per_graph
     line = {
         "metric": METRIC,
-        "value": tokens * K / (total_ms * 1e-3),
+        "value": tokens * K / (m["total_ms"] * 1e-3),
         "unit": "tokens/s",
         "n_gpus": world,
-        "steps": K,
+        "steps": m["steps"],
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
@@ -856,39 +975,53 @@ def run_cuda(args):
         "dtype": "int2 codes + fp16 scale/zero, fp32 accumulate",
         "data": "synthetic (seeded; workloads.py)",
         "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
-                   "context": int(lens.max()), "append_T": w.append_T,
+                   "context": int(lens.max()) if w.ragged is None else
+                   "ragged U[%d, %d] (sum %d)" % (w.ragged[0], w.ragged[1], int(lens.sum())),
+                   "append_T": w.append_T,
                    "rotation": "dense" if w.mode == 0 else "perm+fwht", "sink_fp16": w.sink,
-                   "group": 32, "l2": l2_note, "layers": max(1, n_layers),
+                   "group": 32, "l2": l2_note(m), "layers": max(1, m["n_layers"]),
                    "parallelism": "replicas: one independent batch per GPU"},
         "packed_kv_gbs": kv_bytes / (ms_per_step * 1e-3) / 1e9,
         "packed_kv_bytes_per_step": kv_bytes,
-        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel (streams the packed cache)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                     "algorithmic_bytes_per_launch": kv_bytes,
-                     "kernel_ms_mean": split_mean_s * 1e3, "peak_source": peak_src,
-                     "timing": "CUDA events the library records around the kernel, %d eager steps "
-                               "queued behind a spin kernel (no host gap inside the events)"
-                               % n_split},
-        "e2e": {"value": tokens * n_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "how": "wall clock per step: one kvq_append_decode_host "
-                                                  "call (pinned H2D of the new K/V/Q, append, decode, "
-                                                  "D2H of the output), then a stream synchronise"},
-        "isolated_step": {"ms": float(np.median(iso_ms)), "how": "median of %d steps, each after "
-                          "an L2 flush and bracketed by its own events, queued behind a spin kernel" % n_iso},
+        "context_tokens_per_s": float(lens.astype(np.int64).sum()) * w.Hkv * world
+        / (ms_per_step * 1e-3),
+        "roofline": split_roofline(w, m, peak, peak_src, args.workload),
+        "e2e": {"value": tokens * m["n_e2e"] / m["e2e_s"], "unit": "tokens/s",
+                "h2d_bytes_per_step": m["h2d"], "d2h_bytes_per_step": m["d2h"],
+                "how": "wall clock per step: one kvq_append_decode_host call (pinned H2D of the new "
+                       "K/V/Q, append, decode, D2H of the output), then a stream synchronise"},
+        "isolated_step": {"ms": float(np.median(m["iso_ms"])), "how": "median of %d steps, each "
+                          "after an L2 flush and bracketed by its own events, queued behind a "
+                          "spin kernel" % len(m["iso_ms"])},
         "gpu_launches": KERNELS_PER_STEP * K,
-        "clocks": clk.summary(),
+        "clocks": m["clocks"],
     }
+    del m, step
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras and args.workload != "llama7b":
+        # the single-layer 32-head decode step (B=1, context 32768) as an extra
+        wl = W.WORKLOADS["llama7b"]
+        ml = measure_step(wl, dev, min(K, 400), args.warmup, False, local, e2e=True)
+        msl = ml["total_ms"] / ml["steps"]
+        line["llama7b_step"] = {
+            "tokens_per_s": wl.B * ml["steps"] / (ml["total_ms"] * 1e-3), "ms_per_step": msl,
+            "steps": ml["steps"], "l2": l2_note(ml),
+            "roofline": split_roofline(wl, ml, peak, peak_src, "llama7b"),
+            "e2e_tokens_per_s": wl.B * ml["n_e2e"] / ml["e2e_s"],
+            "isolated_step_ms": float(np.median(ml["iso_ms"]))}
+        del ml
+        torch.cuda.empty_cache()
     if world == 1 and not args.no_append:
         line["append"] = append_rates(dev, peak)
     if world == 1 and not args.no_extensions:
-        line["extensions"] = extension_rates(step, dev)
+        line["extensions"] = extension_rates(dev)
         line["extensions"]["identified_sinks"] = sink_rates(dev)
         line["extensions"]["pre_rope"] = prerope_rates(dev)
     if world == 1 and not args.no_workloads:
         line["workloads"] = decode_rates(dev, peak)
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, step, dev)
+        sw = rank_workload(W.WORKLOADS[args.workload], rank)
+        line["cpu_baseline"] = cpu_baseline(sw, None, "cpu")
     print(json.dumps(line), flush=True)
     if dist_on:
         import torch.distributed as dist
@@ -901,54 +1034,37 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    from oracle import oracle as orc
     w = W.WORKLOADS[args.workload]
-    heads = 1
     lens = w.seq_lens()
-    L, T = int(lens.max()), w.append_T
-    pre = L - T
-    Rk, Rv, perm = W.rotations(w)
-    rk = Rk[:heads] if Rk is not None else None
-    rv = Rv[:heads] if Rv is not None else None
-    pm = perm[:, :heads] if perm is not None else None
-    cap = ((L + 15) // 16) * 16
-    oc = orc.Cache(1, heads, cap, w.sink)
-    sl = np.zeros(1, np.int32)
-    for t0 in range(0, pre, 4096):
-        t1 = min(pre, t0 + 4096)
-        K, V = W.kv_batch(w, t0, t1, "cpu", bs=[0])
-        orc.append(oc, W.f16_bits(K[:, :, :heads]), W.f16_bits(V[:, :, :heads]), w.mode, rk, rv,
-                   pm, sl)
-    Kn, Vn = W.kv_batch(w, pre, L, "cpu", bs=[0])
-    Kn, Vn = W.f16_bits(Kn[:, :, :heads]), W.f16_bits(Vn[:, :, :heads])
-    Q = W.f16_bits(W.queries(w, "cpu")[:1, :heads * w.G])
-    cores = len(os.sched_getaffinity(0))
-
-    def one():
-        sl[0] = pre
-        orc.append(oc, Kn, Vn, w.mode, rk, rv, pm, sl)
-        orc.decode(oc, Q, w.mode, rk, rv, pm, sl, n_threads=cores)
-
+    b = sample_sequence(lens)
+    heads = 1
+    smp = OracleSample(w, b, heads, "cpu")
     for _ in range(args.warmup):
-        one()
+        smp.step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        one()
+        smp.step()
     el = time.perf_counter() - t0
-    scale = (w.Hkv / heads) * w.B
-    per_step = el / args.steps * scale
-    value = w.B / per_step
+    scale = sample_scale(w, lens, b, heads)
+    ms_sample = el / args.steps * 1e3
+    value = w.B / (ms_sample * 1e-3 * scale)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "steps": args.steps, "warmup": args.warmup,
+        # the time each sample step actually took; the whole-batch step would
+        # take sample_scale times as long (the value is computed from that)
+        "ms_per_step": ms_sample, "sample_scale": scale,
+        "ms_per_step_scaled_estimate": ms_sample * scale,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (fp32 quantizer)", "data": "synthetic (seeded; workloads.py)",
         "config": {"workload": args.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": 128,
-                   "context": L, "append_T": T, "rotation": "dense" if w.mode == 0 else "perm+fwht",
+                   "context": int(lens.max()) if w.ragged is None else
+                   "ragged U[%d, %d] (sum %d)" % (w.ragged[0], w.ragged[1], int(lens.sum())),
+                   "append_T": w.append_T,
+                   "rotation": "dense" if w.mode == 0 else "perm+fwht",
                    "sink_fp16": w.sink, "group": 32},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": "sequence 0, KV head 0 of %d per step (append %d + decode over "
-                                   "%d), time scaled by %d heads x B=%d" % (w.Hkv, T, L, w.Hkv, w.B)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.cores, "kind": "oracle",
+                         "sample": smp.describe(args.steps, el, scale)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -957,16 +1073,18 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
-    ap.add_argument("--workload", default="llama7b", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="ragged", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append", action="store_true", help="skip the bulk-append rates")
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the extension timings (paged, multi-query, identified sinks, pre-RoPE)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the decode timings of every workload at full size")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the llama7b step measured beside a ragged headline")
     ap.add_argument("--extension", choices=["pre_rope", "identified_sinks", "workloads"],
                     default=None,
                     help="time one extension alone and print its JSON")
@@ -975,6 +1093,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
     if args.impl == "reference":
         run_reference(args)
     elif args.append_only:

@@ -39,3 +39,31 @@ def test_profile_traffic_is_tied_to_the_kernel_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("x") == 123.0
     assert bench.profiled_traffic("y") is None           # taken on another kernel source
     assert bench.profiled_traffic("z") is None           # no summary
+    # a summary taken on a smaller case scales to the full launch by the
+    # ratio of algorithmic bytes (units processed)
+    (prof / "decode_split_s.txt").write_text("source_sha256: %s\ndram_bytes_per_launch: 150\n"
+                                             "algorithmic_bytes_per_launch: 100\n" % sha)
+    assert bench.profiled_traffic("s", 400) == 600.0
+    assert bench.profiled_traffic("s") == 150.0
+
+
+def test_graph_plan_runs_exactly_the_requested_steps():
+    for K in (1, 3, 20, 39, 40, 41, 100, 2000):
+        for layers in (1, 5, 7):
+            per, full, rem = bench.graph_plan(K, layers)
+            assert per % layers == 0 and per >= layers
+            assert per * full + rem == K and 0 <= rem < per
+
+
+def test_oracle_sample_scale():
+    # the median sequence of a ragged batch, and the factor from its
+    # (sequence, heads) sample to the whole step's context token-heads
+    assert bench.sample_sequence([5, 1, 9, 3]) == 3        # sorted 1, 3, 5, 9: lower middle
+    assert bench.sample_sequence([7, 7, 7]) == 1
+    w = W.WORKLOADS["ragged"]
+    lens = w.seq_lens()
+    b = bench.sample_sequence(lens)
+    s = bench.sample_scale(w, lens, b, 2)
+    assert abs(s * lens[b] * 2 - lens.sum() * 32) < 1e-6 * s
+    u = W.WORKLOADS["llama7b"]
+    assert bench.sample_scale(u, u.seq_lens(), 0, 4) == 32 / 4
