@@ -156,10 +156,22 @@ def test_ragged_prefill_append_full():
             assert np.array_equal(got_c, c[0])
             assert np.array_equal(ks if kind == 0 else vs, s[0])
             assert np.array_equal(kz if kind == 0 else vz, z[0])
-            oc, _, _ = orc.quantize_rows(orc.rotate_rows_f32(W.f16_bits(x), 0, R=R[h]))
-            n_diff += int((oc[0] != got_c).sum())
-            n_codes += 128
-    assert n_diff <= max(2, 1e-4 * n_codes), (n_diff, n_codes)
+    # near ties against the oracle's own (fp64) rotation: the oracle appends
+    # 4096 consecutive tokens of two (sequence, head) units, 2,097,152 codes,
+    # and at most 1e-4 of them may differ from the GPU's
+    for b, h, t0 in ((0, 0, 0), (B - 1, 31, T - 4096)):
+        oc = orc.Cache(1, 1, 4096, 0)
+        osl = np.zeros(1, np.int32)
+        assert orc.append(oc, W.f16_bits(K[b:b + 1, t0:t0 + 4096, h:h + 1]),
+                          W.f16_bits(V[b:b + 1, t0:t0 + 4096, h:h + 1]), 0, Rk[h:h + 1],
+                          Rv[h:h + 1], None, osl) == 0
+        g = blocks[b, h, t0 // 16:(t0 + 4096) // 16].cpu().numpy()
+        x = np.bitwise_xor(g[:, :1024], oc.blocks[0, 0, :, :1024])
+        n_diff += int(sum(bin((v | (v >> 1)) & 0x55).count("1") * int(c)
+                          for v, c in enumerate(np.bincount(x.reshape(-1), minlength=256))))
+        n_codes += 4096 * 2 * 128
+    assert n_codes >= 1_000_000
+    assert n_diff <= 1e-4 * n_codes, (n_diff, n_codes)
 
 
 def test_gqa_sinks_identified_full():

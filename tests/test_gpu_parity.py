@@ -166,11 +166,66 @@ def test_append_matches_oracle(mode, S, T, L0):
                             np.array_equal(lo[3 + 2 * kind], lg[3 + 2 * kind]):
                         assert near_tie_ok(orot[b, t], lo[kind], lg[kind], lo[2 + 2 * kind],
                                            lo[3 + 2 * kind])
-    assert n_diff <= max(2, 1e-4 * n_codes), (n_diff, n_codes)
+    # every differing code above is a near tie; the rate of such codes is
+    # measured over more than a million codes per append kernel in
+    # test_near_tie_rate_over_a_million_codes
+    assert n_diff < n_codes
     # blocks of positions never written stay untouched (zero)
     for b in range(w.B):
         last = (L0[b] + T + 15) // 16
         assert not gc.blocks[b, :, last:].any()
+
+
+# number of set 2-bit fields in each byte value: (x | x >> 1) & 0x55 keeps one
+# bit per nonzero code
+_NONZERO_CODES = np.array([bin((x | (x >> 1)) & 0x55).count("1") for x in range(256)], np.int64)
+
+
+def code_mismatches(blocks_a, blocks_b):
+    """Differing 2-bit codes between two arrays of cache blocks [..., 1536]
+    (K codes in bytes [0, 512), V codes in [512, 1024) of every block)."""
+    x = np.bitwise_xor(blocks_a[..., :1024], blocks_b[..., :1024])
+    return int(_NONZERO_CODES[x].sum())
+
+
+@pytest.mark.parametrize("path", ["dense_cuda_cores", "dense_tensor_cores", "fwht_step",
+                                  "fwht_chunk", "prerope_gh4"])
+def test_near_tie_rate_over_a_million_codes(path):
+    """Codes that differ between the packed cache and the oracle's append of
+    the same rows (its fp64 rotation) come only from near ties: at most 1e-4
+    of the codes, counted over 2,097,152 codes (2048 tokens x 4 heads x K and
+    V) for every append kernel - the CUDA-core dense append (T < 256), the
+    tensor-core bulk append, the FWHT append one token at a time and in
+    chunks, and the pre-RoPE group rotation."""
+    Hkv, T = 4, 2048
+    mode = 0 if path.startswith("dense") else 1
+    chunk = {"dense_cuda_cores": 128, "dense_tensor_cores": T, "fwht_step": 8,
+             "fwht_chunk": 128, "prerope_gh4": 256}[path]
+    w = W.custom(seed=540 + len(path), B=1, Hq=Hkv, Hkv=Hkv, mode=mode, context=T,
+                 k_outliers=8, channel_scale=(0.5, 20.0) if mode == 1 else None)
+    rt, rn = rot_tensors(w)
+    K, V = W.kv_batch(w, 0, T, "cuda")
+    cache = kvq.KVCache(1, Hkv, T)
+    sl = torch.zeros(1, dtype=torch.int32, device="cuda")
+    oc = orc.Cache(1, Hkv, T, 0)
+    osl = np.zeros(1, np.int32)
+    if path == "prerope_gh4":
+        perm = W.prerope_perm(w, 4)
+        pt = torch.from_numpy(perm).cuda()
+        for t0 in range(0, T, chunk):
+            kvq.kvq_prerope_append(K[:, t0:t0 + chunk].contiguous(), V[:, t0:t0 + chunk].contiguous(),
+                                   4, pt, cache, sl)
+        assert orc.append_prerope(oc, f16bits(K), f16bits(V), 4, perm, osl) == 0
+    else:
+        for t0 in range(0, T, chunk):
+            gpu_append(cache, K[:, t0:t0 + chunk], V[:, t0:t0 + chunk], w, rt, sl)
+        assert orc.append(oc, f16bits(K), f16bits(V), mode, *rn, osl) == 0
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0 and int(sl.item()) == T
+    n_codes = Hkv * T * 2 * D
+    n_diff = code_mismatches(cache.block_view().cpu().numpy(), oc.blocks)
+    assert n_codes >= 1_000_000
+    assert n_diff <= 1e-4 * n_codes, (n_diff, n_codes)
 
 
 def test_append_capacity_and_status():
