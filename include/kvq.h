@@ -297,6 +297,26 @@ KVQ_API kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mo
 KVQ_API kvq_status kvq_debug_quantize_f32(const float *Xrot, int32_t N, uint8_t *codes,
                                   uint16_t *meta, void *stream);
 
+/*
+ * Test export for the failure path of the kernels' bounded waits (device
+ * errors are reported in a status word, never by a trap).  One thread runs
+ * the decode ring protocol on two slots: a real 1536-byte bulk copy of `src`
+ * into slot 0, and a wait on slot 1, which nothing ever fills, that gives up
+ * after poll_limit polls (each poll may sleep up to about 20 us).  It then
+ * ORs KVQ_DEV_TIMEOUT into *status and drains the ring with the same routine
+ * an aborted decode CTA runs before it returns, so that no copy still
+ * targets its shared memory.
+ *   src     device, 1536 bytes, 16-byte aligned.
+ *   status  device int32 word (e.g. a cache's status).
+ *   result  device int32 [3]: [0] = 1 if the wait gave up, [1] = stages the
+ *           drain could not see land (0 expected), [2] = sum of the 1536
+ *           bytes as copied into shared memory.
+ * Errors: null pointers or poll_limit 0 -> KVQ_ERR_INVALID_ARG; misaligned
+ * pointers -> KVQ_ERR_UNSUPPORTED.  No page counterpart: library plumbing.
+ */
+KVQ_API kvq_status kvq_debug_wait_timeout(const void *src, uint32_t poll_limit, int32_t *status,
+                                          int32_t *result, void *stream);
+
 /* Options of kvq_decode_attention_ex. */
 #define KVQ_DECODE_OUT_ROTATED 1u  /* out = o_rot: the caller applies R_v^T (or the inverse
                                       permutation + FWHT) itself, e.g. folded into W_O */

@@ -15,7 +15,8 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_rotate_quantize_append, lib, kvq_prerope_append, kvq_prerope_decode,
                   kvq_append_decode, kvq_append_decode_host, kvq_step_workspace_size,
                   step_workspace,
-                  kvq_prerope_workspace_size, prerope_workspace, kvq_debug_rotate_group_f32)
+                  kvq_prerope_workspace_size, prerope_workspace, kvq_debug_rotate_group_f32,
+                  kvq_debug_wait_timeout)
 
 __all__ = [
     "KVCache", "PagedKVCache", "KvqError", "KVQ_DEV_BAD_TABLE", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
@@ -28,4 +29,5 @@ __all__ = [
     "kvq_rotate_quantize_append", "lib", "kvq_prerope_append", "kvq_prerope_decode",
     "kvq_append_decode", "kvq_append_decode_host", "kvq_step_workspace_size", "step_workspace",
     "kvq_prerope_workspace_size", "prerope_workspace", "kvq_debug_rotate_group_f32",
+    "kvq_debug_wait_timeout",
 ]

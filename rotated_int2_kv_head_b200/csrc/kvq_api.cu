@@ -440,6 +440,15 @@ kvq_status kvq_debug_quantize_f32(const float *Xrot, int32_t N, uint8_t *codes, 
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+kvq_status kvq_debug_wait_timeout(const void *src, uint32_t poll_limit, int32_t *status,
+                                  int32_t *result, void *stream) {
+    if (!src || !status || !result || poll_limit == 0) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(src, 16) || !aligned(status, 4) || !aligned(result, 4)) return KVQ_ERR_UNSUPPORTED;
+    cudaError_t e = launch_debug_wait_timeout(static_cast<const uint8_t *>(src), poll_limit, status,
+                                              result, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 const char *kvq_status_string(kvq_status s) {
     switch (s) {
         case KVQ_OK: return "ok";

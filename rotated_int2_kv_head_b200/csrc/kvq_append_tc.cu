@@ -250,8 +250,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             // no copy may still be landing when the CTA exits (after an abort
             // the last stages may not have been consumed): bounded waits
-            for (int d = max(0, i - A_STAGES); d < i; d++)
-                mbar_wait_bounded(&bar[BAR_FULL + d % A_STAGES], (d / A_STAGES) & 1, 1u << 10);
+            drain_ring(&bar[BAR_FULL], A_STAGES, max(0, i - A_STAGES), i);
         }
     } else if (warp == 1) {
         // ---- MMA issuer
@@ -291,8 +290,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             // the accumulators are freed below: the last MMAs must have completed
             if (i > 0)
-                mbar_wait_bounded(&bar[BAR_ACCF + (i - 1) % EPI_GROUPS], ((i - 1) / EPI_GROUPS) & 1,
-                                  1u << 10);
+                mbar_wait_bounded(&bar[BAR_ACCF + (i - 1) % EPI_GROUPS], ((i - 1) / EPI_GROUPS) & 1);
         }
     } else {
         // ---- epilogue groups

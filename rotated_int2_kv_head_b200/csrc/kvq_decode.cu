@@ -980,10 +980,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         }
     }
     if (aborted) {
-        // leave no copy in flight into this CTA's shared memory: wait (briefly,
-        // bounded) for every stage issued from this iteration on
-        if (leader)
-            for (int j = it; j < issued; j++) mbar_wait_bounded(&full[j % NS], (j / NS) & 1, 1u << 8);
+        // leave no copy in flight into this CTA's shared memory: wait (with
+        // the full bound) for every stage issued from this iteration on
+        if (leader) drain_ring(full, NS, it, issued);
         return;
     }
     if (cur_unit >= 0) flush(part_slot(blockIdx.x, cur_unit, grp));
@@ -1338,6 +1337,46 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     if (e != cudaSuccess) return e;
     if (ev_end && (e = cudaEventRecord(ev_end, st)) != cudaSuccess) return e;
     return launch_pdl(decode_merge_kernel, dim3(Hq, cd.B), dim3(MRG_THREADS), 0, st, a);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Test kernel for the give-up path of the bounded waits.  One thread runs the
+// split kernel's ring protocol on a two-slot ring: stage 0 is a real 1536-byte
+// bulk copy of `src`; slot 1 is never filled (a flag nothing sets), so the
+// wait on it runs out after poll_limit polls.  The thread then flags
+// KVQ_DEV_TIMEOUT and drains the ring with drain_ring - the same call the
+// split kernel makes before an aborted CTA returns - and reports:
+//   result[0] = 1 if the wait on the empty slot gave up, result[1] = stages
+//   drain_ring could not see land (0 expected), result[2] = the sum of the
+//   copied bytes as they sit in shared memory (the copy landed before the
+//   CTA returned).
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) debug_wait_timeout_kernel(const uint8_t *src,
+                                                                 uint32_t poll_limit,
+                                                                 int32_t *status, int32_t *result) {
+    __shared__ __align__(128) uint8_t ring[2][BLK_BYTES];
+    __shared__ __align__(8) uint64_t full[2];
+    if (threadIdx.x != 0) return;
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&full[0], BLK_BYTES);
+    bulk_g2s(ring[0], src, BLK_BYTES, &full[0]);
+    const int issued = 1;                       // slot 1: nothing is ever issued
+    const bool ok = mbar_wait_bounded(&full[1], 0u, poll_limit);
+    if (!ok) set_status(status, KVQ_DEV_TIMEOUT);
+    const int lost = drain_ring(full, 2, 0, issued);
+    int sum = 0;
+    for (int i = 0; i < BLK_BYTES; i++) sum += ring[0][i];
+    result[0] = ok ? 0 : 1;
+    result[1] = lost;
+    result[2] = sum;
+}
+
+cudaError_t launch_debug_wait_timeout(const uint8_t *src, uint32_t poll_limit, int32_t *status,
+                                      int32_t *result, cudaStream_t st) {
+    debug_wait_timeout_kernel<<<1, 32, 0, st>>>(src, poll_limit, status, result);
+    return cudaGetLastError();
 }
 
 }  // namespace kvq

@@ -267,6 +267,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return false;
 }
 
+// After a bounded wait has given up: wait, with the same bound, for the
+// stages [from, issued) of a ring of ns slots (stage j fills slot j % ns,
+// phase j / ns) to land, so that no bulk copy still targets this CTA's
+// shared memory when it returns.  A stage whose phase is already complete
+// (or that was closed by a plain arrive) passes at once.  Returns the number
+// of stages that did not land within the bound (0 unless a copy itself is
+// lost); the caller has already set KVQ_DEV_TIMEOUT.
+__device__ __forceinline__ int drain_ring(uint64_t *full, int ns, int from, int issued) {
+    int lost = 0;
+    for (int j = from; j < issued; j++)
+        if (!mbar_wait_bounded(&full[j % ns], (uint32_t)(j / ns) & 1u)) ++lost;
+    return lost;
+}
+
 // 1-D bulk copy global -> shared, completion reported on `bar` as tx bytes.
 // Both addresses 16-B aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes,
@@ -363,6 +377,8 @@ cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, const float *R, flo
                                    cudaStream_t st);
 cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
                                   cudaStream_t st);
+cudaError_t launch_debug_wait_timeout(const uint8_t *src, uint32_t poll_limit, int32_t *status,
+                                      int32_t *result, cudaStream_t st);
 cudaError_t launch_identify_sinks(const float *act, int T, float tau, const kvq_cache_desc &cd,
                                   const int32_t *seq_lens, cudaStream_t st);
 // pre-RoPE grouped-head key rotation (kvq_append.cu / kvq_prerope.cu)

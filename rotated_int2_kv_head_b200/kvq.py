@@ -103,6 +103,8 @@ def lib():
     L.kvq_debug_rotate_f32.argtypes = [p, i32, C.c_int, p, p, i32, p, p]
     L.kvq_debug_quantize_f32.restype = C.c_int
     L.kvq_debug_quantize_f32.argtypes = [p, i32, p, p, p]
+    L.kvq_debug_wait_timeout.restype = C.c_int
+    L.kvq_debug_wait_timeout.argtypes = [p, C.c_uint32, p, p, p]
     L.kvq_status_string.restype = C.c_char_p
     L.kvq_status_string.argtypes = [C.c_int]
     _lib = L
@@ -135,15 +137,38 @@ def _check(fn, code):
         raise KvqError(fn, code)
 
 
+def _need_shape(t, dtype, name, shape=None):
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and t.shape != shape:
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
 def _need(t, dtype, name, shape=None):
     if t is None:
         return
-    if t.dtype != dtype:
-        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    _need_shape(t, dtype, name, shape)
     if not (t.is_cuda and t.is_contiguous()):
         raise ValueError("%s must be a contiguous CUDA tensor" % name)
-    if shape is not None and t.shape != shape:
-        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _need_rotation(mode, R_k, R_v, perm, Hkv):
+    """The rotation inputs of `mode`: dense R_k, R_v fp32 [Hkv][128][128], or
+    perm int32 [2][Hkv][128].  The C ABI cannot see their sizes, so an
+    undersized tensor would be read out of bounds on the device."""
+    if mode == KVQ_ROT_DENSE:
+        if R_k is None or R_v is None:
+            raise ValueError("dense rotation needs R_k and R_v")
+        _need_shape(R_k, torch.float32, "R_k", (Hkv, D, D))
+        _need_shape(R_v, torch.float32, "R_v", (Hkv, D, D))
+        _need(R_k, torch.float32, "R_k", (Hkv, D, D))
+        _need(R_v, torch.float32, "R_v", (Hkv, D, D))
+    elif mode == KVQ_ROT_PERM_FWHT:
+        if perm is None:
+            raise ValueError("permutation + FWHT rotation needs perm")
+        _need(perm, torch.int32, "perm", (2, Hkv, D))
+    else:
+        raise ValueError("unknown rotation mode %r" % (mode,))
 
 
 def _sink_arrays(cache, B, Hkv, sink_fp16, identified_sinks, device):
@@ -225,15 +250,11 @@ def kvq_cache_bytes(B, Hkv, capacity):
 
 def kvq_rotate_quantize_append(K, V, mode, R_k, R_v, perm, cache, seq_lens, stream=None):
     """K, V fp16 [B][T][Hkv][128]; seq_lens int32 [B] (updated in place)."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, T, Hkv, d = K.shape
     _need(K, torch.float16, "K", (cache.B, T, cache.Hkv, D))
     _need(V, torch.float16, "V", K.shape)
     _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
-    if mode == KVQ_ROT_DENSE:
-        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
-        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
-    else:
-        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
     _check("kvq_rotate_quantize_append",
            lib().kvq_rotate_quantize_append(_ptr(K), _ptr(V), T, mode, _ptr(R_k), _ptr(R_v),
                                             _ptr(perm), C.byref(cache.desc), _ptr(seq_lens),
@@ -277,16 +298,12 @@ def decode_workspace(B, Hq, Hkv, max_ctx, device="cuda"):
 def kvq_decode_attention(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
                          workspace, out, stream=None):
     """Q fp16 [B][Hq][128] -> out fp16 [B][Hq][128]; seq_lens int32 [B] on device."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, Hq, d = Q.shape
     _need(Q, torch.float16, "Q", (cache.B, Hq, D))
     _need(out, torch.float16, "out", Q.shape)
     _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
     _need(workspace, torch.uint8, "workspace")
-    if mode == KVQ_ROT_DENSE:
-        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
-        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
-    else:
-        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
     _check("kvq_decode_attention",
            lib().kvq_decode_attention(_ptr(Q), Hq, C.byref(cache.desc), mode, _ptr(R_k), _ptr(R_v),
                                       _ptr(perm), _ptr(seq_lens), sink_fp16, max_ctx,
@@ -299,6 +316,7 @@ def kvq_append_decode(K, V, Q, cache, mode, R_k, R_v, perm, seq_lens, max_ctx, w
     """One serving step: append K, V fp16 [B][T][Hkv][128] (seq_lens int32 [B]
     advance by T on the device), then decode Q fp16 [B][Hq][128] into out over
     the updated cache."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, T, Hkv, d = K.shape
     _need(K, torch.float16, "K", (cache.B, T, cache.Hkv, D))
     _need(V, torch.float16, "V", K.shape)
@@ -308,11 +326,6 @@ def kvq_append_decode(K, V, Q, cache, mode, R_k, R_v, perm, seq_lens, max_ctx, w
     _need(workspace, torch.uint8, "workspace")
     if Q.dim() != 3 or Q.shape[0] != cache.B or Q.shape[2] != D:
         raise ValueError("Q must have shape (B, Hq, 128)")
-    if mode == KVQ_ROT_DENSE:
-        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
-        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
-    else:
-        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
     _check("kvq_append_decode",
            lib().kvq_append_decode(_ptr(K), _ptr(V), T, _ptr(Q), Q.shape[1], C.byref(cache.desc),
                                    mode, _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
@@ -350,6 +363,7 @@ def kvq_append_decode_host(K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, 
     reading out_host).  K, V and Q that are consecutive views of one buffer
     (V right after K, Q right after V) go in with a single copy.
     workspace: step_workspace(...) on the device."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, T, Hkv, d = K_host.shape
     _need_host(K_host, torch.float16, "K_host", (cache.B, T, cache.Hkv, D))
     _need_host(V_host, torch.float16, "V_host", K_host.shape)
@@ -359,11 +373,6 @@ def kvq_append_decode_host(K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, 
     _need(workspace, torch.uint8, "workspace")
     if Q_host.dim() != 3 or Q_host.shape[0] != cache.B or Q_host.shape[2] != D:
         raise ValueError("Q_host must have shape (B, Hq, 128)")
-    if mode == KVQ_ROT_DENSE:
-        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
-        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
-    else:
-        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
     _check("kvq_append_decode_host",
            lib().kvq_append_decode_host(_ptr(K_host), _ptr(V_host), T, _ptr(Q_host),
                                         Q_host.shape[1], C.byref(cache.desc), mode, _ptr(R_k),
@@ -379,16 +388,12 @@ def kvq_decode_attention_ex(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
                             workspace, out, flags=0, stream=None):
     """Q fp16 [B][Hq][q_len][128] -> out fp16 [B][Hq][q_len][128]: q_len new tokens
     per sequence, each attending causally; flags: KVQ_DECODE_OUT_ROTATED."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, Hq, q_len, d = Q.shape
     _need(Q, torch.float16, "Q", (cache.B, Hq, q_len, D))
     _need(out, torch.float16, "out", Q.shape)
     _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
     _need(workspace, torch.uint8, "workspace")
-    if mode == KVQ_ROT_DENSE:
-        _need(R_k, torch.float32, "R_k", (cache.Hkv, D, D))
-        _need(R_v, torch.float32, "R_v", (cache.Hkv, D, D))
-    else:
-        _need(perm, torch.int32, "perm", (2, cache.Hkv, D))
     _check("kvq_decode_attention_ex",
            lib().kvq_decode_attention_ex(_ptr(Q), Hq, q_len, flags, C.byref(cache.desc), mode,
                                          _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
@@ -401,6 +406,7 @@ def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp
     """kvq_decode_attention that also records torch.cuda.Events ev_begin /
     ev_end (already recorded once, so they exist) around the kernel that
     streams the packed cache."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, Hq, d = Q.shape
     _need(Q, torch.float16, "Q", (cache.B, Hq, D))
     _need(out, torch.float16, "out", Q.shape)
@@ -419,6 +425,7 @@ def kvq_decode_attention_noalloc(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_
     """kvq_decode_attention for callers that cannot allocate device memory:
     no workspace argument, the library's fixed device array serves instead
     (see include/kvq.h for its size and the sharing rules)."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
     B, Hq, d = Q.shape
     _need(Q, torch.float16, "Q", (cache.B, Hq, D))
     _need(out, torch.float16, "out", Q.shape)
@@ -518,3 +525,17 @@ def kvq_debug_rotate_group_f32(X, group_heads, perm, stream=None):
            lib().kvq_debug_rotate_group_f32(_ptr(X), N, group_heads, _ptr(perm), _ptr(out),
                                             _stream(stream, X)))
     return out
+
+
+def kvq_debug_wait_timeout(src, poll_limit, status, stream=None):
+    """Runs the bounded-wait failure path once: src uint8 [1536] on the device,
+    status int32 device word(s) (KVQ_DEV_TIMEOUT is ORed into status[0]).
+    Returns int32 [3] on the device: gave up (1), stages lost by the drain,
+    byte sum of the copy as it landed in shared memory."""
+    _need(src, torch.uint8, "src", (BLOCK_BYTES,))
+    _need(status, torch.int32, "status")
+    result = torch.full((3,), -1, dtype=torch.int32, device=src.device)
+    _check("kvq_debug_wait_timeout",
+           lib().kvq_debug_wait_timeout(_ptr(src), int(poll_limit), _ptr(status), _ptr(result),
+                                        _stream(stream, src)))
+    return result

@@ -195,3 +195,59 @@ def test_prerope_and_sink_calls_reject_bad_arguments_on_host(L):
     assert ident(d, T=65) == 1                   # T > capacity
     d.sink_count = None
     assert ident(d) == 1                         # a sink list without its counts
+
+
+def test_binding_checks_rotation_shapes_before_calling_the_library(L):
+    """Every binding that passes rotations to the library checks their dtype
+    and shape first: the C ABI receives bare pointers, so an undersized R_k,
+    R_v or perm would otherwise be read out of bounds by the kernels.  Runs on
+    CPU: the check fires before any tensor reaches the library."""
+    import torch
+    cache = kvq.KVCache(1, 2, 64, device="cpu")
+    good = torch.zeros((2, 128, 128), dtype=torch.float32)
+    short = torch.zeros((1, 128, 128), dtype=torch.float32)
+    half = torch.zeros((2, 128, 128), dtype=torch.float16)
+    perm_short = torch.zeros((2, 1, 128), dtype=torch.int32)
+    Q = torch.zeros((1, 2, 128), dtype=torch.float16)
+    sl = torch.zeros(1, dtype=torch.int32)
+    ws = torch.zeros(64, dtype=torch.uint8)
+    ev = object()
+    calls = {
+        "decode": lambda rk, rv, pm, mode: kvq.kvq_decode_attention(
+            Q, cache, mode, rk, rv, pm, sl, 0, 64, ws, Q),
+        "decode_ex": lambda rk, rv, pm, mode: kvq.kvq_decode_attention_ex(
+            Q[:, :, None], cache, mode, rk, rv, pm, sl, 0, 64, ws, Q[:, :, None]),
+        "decode_timed": lambda rk, rv, pm, mode: kvq.kvq_decode_attention_timed(
+            Q, cache, mode, rk, rv, pm, sl, 0, 64, ws, Q, ev, ev),
+        "decode_noalloc": lambda rk, rv, pm, mode: kvq.kvq_decode_attention_noalloc(
+            Q, cache, mode, rk, rv, pm, sl, 0, 64, Q),
+        "append": lambda rk, rv, pm, mode: kvq.kvq_rotate_quantize_append(
+            Q[:, None], Q[:, None], mode, rk, rv, pm, cache, sl),
+        "append_decode": lambda rk, rv, pm, mode: kvq.kvq_append_decode(
+            Q[:, None], Q[:, None], Q, cache, mode, rk, rv, pm, sl, 64, ws, Q),
+        "append_decode_host": lambda rk, rv, pm, mode: kvq.kvq_append_decode_host(
+            Q[:, None], Q[:, None], Q, cache, mode, rk, rv, pm, sl, 64, ws, Q),
+    }
+    for name, call in calls.items():
+        with pytest.raises(ValueError, match="R_k must have shape"):
+            call(short, good, None, 0)
+        with pytest.raises(ValueError, match="R_v must have shape"):
+            call(good, short, None, 0)
+        with pytest.raises(TypeError, match="R_k must be torch.float32"):
+            call(half, good, None, 0)
+        with pytest.raises(ValueError, match="needs R_k and R_v"):
+            call(None, good, None, 0)
+        with pytest.raises(ValueError, match="perm must have shape"):
+            call(None, None, perm_short, 1)
+        with pytest.raises(ValueError, match="needs perm"):
+            call(None, None, None, 1)
+        with pytest.raises(ValueError, match="unknown rotation mode"):
+            call(good, good, None, 2)
+
+
+def test_debug_wait_timeout_rejects_bad_calls(L):
+    ok = C.c_void_p(4096)
+    assert L.kvq_debug_wait_timeout(None, 8, ok, ok, None) == 1
+    assert L.kvq_debug_wait_timeout(ok, 0, ok, ok, None) == 1
+    assert L.kvq_debug_wait_timeout(ok, 8, None, ok, None) == 1
+    assert L.kvq_debug_wait_timeout(C.c_void_p(4104), 8, ok, ok, None) == 2
