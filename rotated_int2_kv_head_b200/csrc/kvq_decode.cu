@@ -48,10 +48,13 @@ constexpr int GROUP_WARPS = 4;
 constexpr int GROUP_THREADS = 32 * GROUP_WARPS;           // 128
 constexpr int DEC_THREADS = DEC_GROUPS * GROUP_THREADS;   // 512
 constexpr int DEC_WARPS = DEC_GROUPS * GROUP_WARPS;       // 16
-constexpr int STAGE_BLKS = 2 * GROUP_WARPS;               // 8 blocks = 128 tokens
-constexpr int STAGE_BYTES = STAGE_BLKS * BLK_BYTES;       // 12 KB
-// ring slots per group (the flush scratch grows with G)
-__host__ __device__ constexpr int nstage_for(int G) { return G >= 4 ? 3 : 4; }
+// Blocks per warp per stage and ring slots per group: four blocks (a 24 KB
+// stage of 256 tokens, two in the ring) for G <= 4; two (12 KB, three in
+// the ring) for G = 8, whose flush scratch leaves no room for 24 KB stages.
+__host__ __device__ constexpr int bpw_for(int G) { return G >= 8 ? 2 : 4; }
+__host__ __device__ constexpr int nstage_for(int G) { return G >= 8 ? 3 : 2; }
+__host__ __device__ constexpr int stage_blks_for(int G) { return bpw_for(G) * GROUP_WARPS; }
+__host__ __device__ constexpr int stage_bytes_for(int G) { return stage_blks_for(G) * BLK_BYTES; }
 // Prepared query per query head, QB bytes:
 //   int8 hi[128], int8 lo[128]  with q_s ~= sq_g * (hi + lo/254) per group g
 //   float kap[4] = sq_g / 4^g,  float qsum[4] = sum of q_s over group g
@@ -253,9 +256,9 @@ __device__ bool sched_init_cta(Sched &s, const DecodeArgs &a, int *scratch) {
     return true;
 }
 
-// Next stage of a group's own range (up to STAGE_BLKS blocks, never crossing
+// Next stage of a group's own range (up to max_blks blocks, never crossing
 // a unit); false when the range is exhausted.  Leader thread only.
-__device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &unit, int &b,
+__device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int max_blks, int &unit, int &b,
                                            int &h, int &kblk, int &n) {
     if (ps.cur >= ps.end) return false;
     sched_fix_unit(ps, a);
@@ -264,7 +267,7 @@ __device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int &
         ps.cur = first;
         if (ps.cur >= ps.end) return false;
     }
-    n = min(min(STAGE_BLKS, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
+    n = min(min(max_blks, ps.end - ps.cur), ps.ustart + ps.nb - ps.cur);
     unit = ps.b * a.Hkv + ps.h;
     b = ps.b;
     h = ps.h;
@@ -434,7 +437,7 @@ __host__ __device__ constexpr unsigned smem_up16(unsigned x) { return (x + 15u) 
 __host__ __device__ inline SplitSmem split_smem_layout(int G) {
     const unsigned ns = nstage_for(G);
     SplitSmem L{};
-    L.full = ns * STAGE_BYTES;                                   // ring at offset 0
+    L.full = ns * (unsigned)stage_bytes_for(G);                  // ring at offset 0
     L.desc = smem_up16(L.full + ns * 8u);
     L.fo = smem_up16(L.desc + 2u * ns * 16u);
     L.fm = smem_up16(L.fo + 4u * GROUP_WARPS * G * D);
@@ -457,6 +460,9 @@ template <int G, bool PAGED>
 __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs a) {
     using C = Cfg<G>;
     constexpr int NS = nstage_for(G);
+    constexpr int BPW = bpw_for(G);
+    constexpr int STAGE_BLKS = stage_blks_for(G);
+    constexpr int STAGE_BYTES = stage_bytes_for(G);
     constexpr int NW = G;                              // weight registers per lane per block
     constexpr int NGL = G == 1 ? 1 : (G == 2 ? 2 : 4); // V-meta groups a lane reads
     extern __shared__ __align__(128) uint8_t smem[];
@@ -509,7 +515,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     auto issue_next = [&](int slot) {
         if (ended) return;
         int unit = 0, b = 0, h = 0, kblk = 0, n = 0;
-        if (sched_take(sc, a, unit, b, h, kblk, n)) {
+        if (sched_take(sc, a, STAGE_BLKS, unit, b, h, kblk, n)) {
             if (lane == 0) {
                 desc[2 * slot] = make_int4(unit, b, h, fb + kblk);
                 desc[2 * slot + 1] = make_int4(n, 0, 0, 0);
@@ -674,13 +680,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         bar_group();
     };
 
-    // Scores, part 1: the K codes of a warp's two blocks of a stage through
-    // the integer tensor cores (one IMMA per group and block; the second
-    // block may be a phantom).
-    // Blocks b_lo .. b_hi-1 of the pair (G = 8 takes them one at a time: the
-    // accumulators of both would not fit the 128 registers).
-    auto k_mma = [&](const uint8_t *blk0, int (&dk)[2][C::NTK][4], int b_lo, int b_hi) {
-        uint4 kq[2];
+    // Scores, part 1: the K codes of blocks b_lo .. b_hi-1 of the warp's
+    // BPW blocks of a stage through the integer tensor cores (one IMMA per
+    // group and block; blocks past the stage's end are masked later).
+    auto k_mma = [&](const uint8_t *blk0, int (&dk)[BPW][C::NTK][4], int b_lo, int b_hi) {
+        uint4 kq[BPW];
 #pragma unroll
         for (int bi = b_lo; bi < b_hi; bi++)
             kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
@@ -709,8 +713,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     // Scores, part 2: integer dots -> fp32 scores (group scale and zero,
     // query scale), summed over the groups; positions outside [S, L) and
     // phantom blocks are masked to -inf.
-    auto k_combine = [&](const uint8_t *blk0, const int (&dk)[2][C::NTK][4], int tok0, int nmine,
-                         float (&sco)[2][2][C::HPL], bool (&edge)[2], int b_lo, int b_hi) {
+    auto k_combine = [&](const uint8_t *blk0, const int (&dk)[BPW][C::NTK][4], int tok0, int nmine,
+                         float (&sco)[BPW][2][C::HPL], bool (&edge)[BPW], int b_lo, int b_hi) {
         // a block needs masking if it is a phantom or crosses [S, L)
 #pragma unroll
         for (int bi = b_lo; bi < b_hi; bi++)
@@ -759,13 +763,13 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         }
     };
     // Online softmax and P.V of one stage.
-    auto v_side = [&](const uint8_t *blk0, const float (&sco)[2][2][C::HPL], const bool (&edge)[2]) {
+    auto v_side = [&](const uint8_t *blk0, const float (&sco)[BPW][2][C::HPL], const bool (&edge)[BPW]) {
         // ---- online softmax.  The running max only moves when a score of
         // this stage exceeds it (rare after the first stages), so the
         // common path is one vote; the branch is uniform over the warp.
         bool over = false;
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++)
+        for (int bi = 0; bi < BPW; bi++)
 #pragma unroll
             for (int st = 0; st < 2; st++)
 #pragma unroll
@@ -775,7 +779,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         float mt[C::HPL];
 #pragma unroll
         for (int hh = 0; hh < C::HPL; hh++) {
-            float v = fmaxf(fmaxf(sco[0][0][hh], sco[0][1][hh]), fmaxf(sco[1][0][hh], sco[1][1][hh]));
+            float v = NEG_INF;
+#pragma unroll
+            for (int bi = 0; bi < BPW; bi++) v = fmaxf(v, fmaxf(sco[bi][0][hh], sco[bi][1][hh]));
             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
@@ -816,9 +822,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                 }
         }
         }
-        float P[2][2][C::HPL];
+        float P[BPW][2][C::HPL];
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++)
+        for (int bi = 0; bi < BPW; bi++)
 #pragma unroll
             for (int st = 0; st < 2; st++)
 #pragma unroll
@@ -835,7 +841,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                 }
         // ---- P.V
 #pragma unroll
-        for (int bi = 0; bi < 2; bi++) {
+        for (int bi = 0; bi < BPW; bi++) {
             const uint8_t *blk = blk0 + bi * BLK_BYTES;
             // weights w = p * s_v in the score layout, as half2 (token r, token r+8):
             // p packed to fp16 times the two tokens' fp16 scales (one HMUL2)
@@ -936,7 +942,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         }
         return false;
     };
-    auto wblk = [&](int slot) { return ring + slot * STAGE_BYTES + (2 * warp) * BLK_BYTES; };
+    auto wblk = [&](int slot) { return ring + slot * STAGE_BYTES + (BPW * warp) * BLK_BYTES; };
 
     reset_state();
     bool aborted = false;
@@ -956,20 +962,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             cur_unit = unit;
         }
         const bool ok = mbar_wait_bounded(&full[s], (it / NS) & 1);
-        const int nmine = min(2, max(0, n - 2 * warp));
+        const int nmine = min(BPW, max(0, n - BPW * warp));
         if (ok && nmine > 0) {
-            int dk[2][C::NTK][4];
-            float sco[2][2][C::HPL];
-            bool edge[2];
-            const int tok0 = (d0.w + 2 * warp) * BLK_TOK;
-            if constexpr (G >= 8) {
-                k_mma(wblk(s), dk, 0, 1);
-                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 0, 1);
-                k_mma(wblk(s), dk, 1, 2);
-                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 1, 2);
-            } else {
-                k_mma(wblk(s), dk, 0, 2);
-                k_combine(wblk(s), dk, tok0, nmine, sco, edge, 0, 2);
+            int dk[BPW][C::NTK][4];
+            float sco[BPW][2][C::HPL];
+            bool edge[BPW];
+            const int tok0 = (d0.w + BPW * warp) * BLK_TOK;
+            // the K side in pairs of blocks (G = 8 one block at a time: the
+            // integer accumulators of two would not fit the registers)
+            constexpr int KSTEP = G >= 8 ? 1 : 2;
+#pragma unroll
+            for (int b0 = 0; b0 < BPW; b0 += KSTEP) {
+                k_mma(wblk(s), dk, b0, b0 + KSTEP);
+                k_combine(wblk(s), dk, tok0, nmine, sco, edge, b0, b0 + KSTEP);
             }
             v_side(wblk(s), sco, edge);
         }
