@@ -284,10 +284,12 @@ KVQ_API kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream);
  * kvq_debug_rotate_f32: X fp16 [N][128] rows, all rotated by one head's
  *   rotation (R fp32 [128][128] in dense mode, perm int32 [128] in FWHT mode)
  *   -> Xrot fp32 [N][128].  `variant` selects the append kernel whose
- *   rotation is exercised: 0 = the small-batch kernel (CUDA cores), 1 = the
- *   bulk kernel (dense mode: tcgen05 tensor cores with R split into fp16
- *   hi + lo, used by appends of T >= 256 rows with 16-byte aligned K and V;
- *   FWHT mode: the same kernel as 0).  Other values: KVQ_ERR_INVALID_ARG.
+ *   rotation is exercised: 0 = the small-batch kernels (CUDA cores), 1 = the
+ *   bulk kernel on the tcgen05 tensor cores, used by appends with 16-byte
+ *   aligned K and V of T >= 256 rows in dense mode (R split into fp16
+ *   hi + lo) and of T >= 128 rows in FWHT mode (the product with the
+ *   permuted +-1 Hadamard matrix, scaled by 1/sqrt(128) in fp32).  Other
+ *   values: KVQ_ERR_INVALID_ARG.
  * kvq_debug_quantize_f32: Xrot fp32 [N][128] -> codes [N][32] in the logical
  *   packing, meta [N][4] as {s, z} fp16 pairs (uint16 [N][4][2]).
  */

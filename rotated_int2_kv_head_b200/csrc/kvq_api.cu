@@ -112,8 +112,8 @@ kvq_status append_launch(const uint16_t *K, const uint16_t *V, int32_t T, kvq_ro
                          const kvq_cache_desc *cache, int32_t *seq_lens, void *stream) {
     if (T == 0) return KVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = (mode == KVQ_ROT_DENSE && append_tc_eligible(K, V, T))
-                        ? launch_append_tc(K, V, T, R_k, R_v, *cache, seq_lens, st)
+    cudaError_t e = append_tc_eligible(mode, K, V, T)
+                        ? launch_append_tc(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st)
                         : launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
@@ -425,8 +425,8 @@ kvq_status kvq_debug_rotate_f32(const uint16_t *X, int32_t N, kvq_rot_mode mode,
     if (variant != 0 && variant != 1) return KVQ_ERR_INVALID_ARG;
     if (N == 0) return KVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = (variant == 1 && mode == KVQ_ROT_DENSE)
-                        ? launch_debug_rotate_tc(X, N, R, Xrot, st)
+    cudaError_t e = variant == 1
+                        ? launch_debug_rotate_tc(X, N, mode, R, perm, Xrot, st)
                         : launch_debug_rotate_small(X, N, mode, R, perm, Xrot, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }

@@ -20,12 +20,24 @@
 //     packed four per byte) and writes the row into the packed cache (or
 //     the fp16 sink rows, or fp32 rows for the test export).
 //
-// One persistent CTA per SM walks a contiguous range of tiles.  R's fp16
-// halves live in shared memory in the MMA's K-major swizzled layout; when
-// the range moves to another (sequence, head, K|V) job, the epilogue group
-// that finished the job's last tile rewrites them (every MMA before it has
-// completed by then) and releases the MMA warp.  Every wait is bounded: a
-// wait that gives up sets KVQ_DEV_TIMEOUT and the CTA stops.
+// One persistent CTA per SM walks a contiguous range of tiles.  Jobs are
+// ordered (head, K|V) first and sequence last, so consecutive jobs share
+// their rotation.  R's fp16 halves live in shared memory in the MMA's
+// K-major swizzled layout; when the range moves to a job with another
+// rotation, the epilogue group that finished the previous job's last tile
+// rewrites them (every MMA before it has completed by then) and releases
+// the MMA warp.  Every wait is bounded: a wait that gives up sets
+// KVQ_DEV_TIMEOUT and the CTA stops.
+//
+// Permutation + FWHT rotation ("RotateKV", abstract item (i); "KVLinC",
+// abstract: Hadamard rotation) is the same contraction with
+// R = P . H / sqrt(128): y = x[perm] transformed by the Sylvester Hadamard
+// matrix H is x . B with B[m][j] = H[pinv[m]][j] = (-1)^popcount(pinv[m] & j),
+// pinv the inverse permutation.  B's entries are +-1, exact in fp16, so one
+// MMA pass (no lo part) gives the transform exactly up to fp32 accumulation,
+// and the epilogue multiplies by 1/sqrt(128) in fp32 like the CUDA-core
+// FWHT does.  B is built in shared memory from the permutation (no R in
+// memory).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -135,13 +147,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
 
 }  // namespace tc
 
-// Work of one launch.  Cache mode: job j = (b*Hkv + h)*2 + kind over
-// x = K (kind 0) or V (kind 1), rows t in [0, T).  Test mode (out_f32 set):
-// one job, x = [N][128], R = R0, fp32 rows out.
+// Work of one launch.  Cache mode: job j = (2h + kind)*B + b over
+// x = K (kind 0) or V (kind 1) of sequence b, rows t in [0, T); its
+// rotation key is j / B = 2h + kind.  Test mode (out_f32 set): one job,
+// x = [N][128], R = R0 (or perm = one plane of 128), fp32 rows out.
 struct TcArgs {
-    const float *R0, *R1;   // R_k, R_v [Hkv][128][128]
+    const float *R0, *R1;   // dense: R_k, R_v [Hkv][128][128]
+    const int32_t *perm;    // FWHT: [2][Hkv][128] (cache) or [128] (test); else nullptr
     float *out_f32;         // test mode output [T][128], else nullptr
     int T;                  // rows per job
+    int B;                  // sequences (1 in test mode)
+    int Hkv;
     int tiles_per_job, ntiles, tiles_per_cta;
 };
 
@@ -173,10 +189,57 @@ __device__ __forceinline__ void convert_r(const float *R, uint8_t *bhi, uint8_t 
     }
 }
 
+// P . H of one job in the same B layout (row j, K index m), entries
+// (-1)^popcount(pinv[m] & j) as fp16 +-1, pinv the inverse permutation.
+// Called by the 128 threads of one epilogue group, thread tt = row j.  Each
+// warp inverts the permutation into its own 128 bytes of scratch (pinv_w),
+// so only warp-level synchronisation is needed.  Entries of a permutation
+// outside [0, 128) are wrapped.
+__device__ __forceinline__ void build_fwht_b(const int32_t *perm, uint8_t *bhi, uint8_t *pinv_w,
+                                             int tt) {
+    const int lane = tt & 31;
+#pragma unroll
+    for (int k = 0; k < 4; k++) pinv_w[perm[lane + 32 * k] & (D - 1)] = (uint8_t)(lane + 32 * k);
+    __syncwarp();
+    const int j = tt;
+#pragma unroll 4
+    for (int cc = 0; cc < 16; cc++) {
+        const int m0 = 8 * cc;
+        const uint2 pw = *reinterpret_cast<const uint2 *>(pinv_w + m0);   // pinv[m0 .. m0+7]
+        uint32_t hw[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const uint32_t w = e < 2 ? pw.x : pw.y;
+            const uint32_t p0 = (w >> (16 * (e & 1))) & 0xffu, p1 = (w >> (16 * (e & 1) + 8)) & 0xffu;
+            const uint32_t s0 = __popc(p0 & (uint32_t)j) & 1u, s1 = __popc(p1 & (uint32_t)j) & 1u;
+            hw[e] = (0x3C00u | (s0 << 15)) | ((0x3C00u | (s1 << 15)) << 16);
+        }
+        const int kb = m0 >> 6, ch = (m0 & 63) >> 3;
+        const int off = kb * tc::B_HALF + j * 128 + ((ch ^ (j & 7)) << 4);
+        *reinterpret_cast<uint4 *>(bhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+    // every lane has read pinv_w before a later build rewrites it
+    __syncwarp();
+}
+
+// The B operand of rotation key hk (cache: 2h + kind; test: 0) by the 128
+// threads of epilogue group eg.
+__device__ __forceinline__ void load_b(const TcArgs &a, bool to_cache, int hk, uint8_t *bhi,
+                                       uint8_t *blo, int gt, int eg) {
+    if (a.perm) {
+        const int32_t *pm = to_cache ? a.perm + ((size_t)(hk & 1) * a.Hkv + (hk >> 1)) * D : a.perm;
+        // per-warp scratch in the lo part, unused by this rotation
+        build_fwht_b(pm, bhi, blo + 128 * (4 * eg + (gt >> 5)), gt);
+    } else {
+        const float *R = to_cache ? ((hk & 1) ? a.R1 : a.R0) + (size_t)(hk >> 1) * D * D : a.R0;
+        convert_r(R, bhi, blo, gt);
+    }
+}
+
 // The epilogue quantizes one row per thread with quantize_group_thread
 // (kvq_internal.cuh), group by group.
 
-template <bool TO_CACHE>
+template <bool TO_CACHE, bool FWHT>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     append_dense_tc_kernel(const __grid_constant__ CUtensorMap mapK,
                            const __grid_constant__ CUtensorMap mapV, TcArgs a, CacheDst c) {
@@ -193,6 +256,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int k0 = blockIdx.x * a.tiles_per_cta;
     const int nmy = max(0, min(a.ntiles, k0 + a.tiles_per_cta) - k0);
     auto job_of = [&](int k) { return k / a.tiles_per_job; };
+    auto rot_of = [&](int k) { return job_of(k) / a.B; };     // rotation key 2h + kind
+    // tile k takes another rotation than tile k - 1 (divisions only at job
+    // boundaries)
+    auto new_rot = [&](int k) { return job_of(k) != job_of(k - 1) && rot_of(k) != rot_of(k - 1); };
     auto fail = [&]() {
         set_status(c.status, KVQ_DEV_TIMEOUT);
         *abort_flag = 1;
@@ -238,9 +305,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 }
                 int kind = 0, h = 0, row = (k - j * a.tiles_per_job) * TILE_M;
                 if (TO_CACHE) {
-                    kind = j & 1;
-                    h = (j >> 1) % c.Hkv;
-                    row += (j >> 1) / c.Hkv * a.T;     // + b * T
+                    const int hk = j / a.B;
+                    kind = hk & 1;
+                    h = hk >> 1;
+                    row += (j - hk * a.B) * a.T;       // + b * T
                 }
                 const CUtensorMap *map = kind == 0 ? &mapK : &mapV;
                 uint8_t *dst = smem + OFF_A + s * A_BYTES;
@@ -259,7 +327,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             int i = 0;
             for (; i < nmy && !*abort_flag; i++) {
                 const int k = k0 + i, s = i % A_STAGES, buf = i % EPI_GROUPS;
-                if (i == 0 || job_of(k) != job_of(k - 1)) {
+                if (i == 0 || new_rot(k)) {
                     if (!mbar_wait_bounded(&bar[BAR_BREADY], nb & 1)) { fail(); break; }
                     ++nb;
                 }
@@ -274,7 +342,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 const uint32_t abase = smem_u32(smem + OFF_A + s * A_BYTES);
                 uint32_t acc = 0;
 #pragma unroll
-                for (int part = 0; part < 2; part++) {
+                for (int part = 0; part < (FWHT ? 1 : 2); part++) {
                     const uint32_t bbase = smem_u32(part == 0 ? bhi : blo);
 #pragma unroll
                     for (int kb = 0; kb < 2; kb++)
@@ -299,10 +367,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int q = warp & 3;                         // TMEM lane quarter this warp may read
         const int row = 32 * q + lane;                  // accumulator row = tile row
         if (eg == 0 && nmy > 0) {                       // R for the first job
-            const int j = job_of(k0);
-            const float *R = TO_CACHE ? ((j & 1) ? a.R1 : a.R0) + (size_t)((j >> 1) % c.Hkv) * D * D
-                                      : a.R0;
-            convert_r(R, bhi, blo, gt);
+            load_b(a, TO_CACHE, rot_of(k0), bhi, blo, gt, eg);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
@@ -320,22 +385,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             tc_fence_after();
             // this tile's MMAs (and all earlier ones) are done: if the next tile
-            // starts another job, its R goes into the B operand now
-            if (i + 1 < nmy && job_of(k + 1) != j) {
-                const int jn = j + 1;
-                const float *R = TO_CACHE ? ((jn & 1) ? a.R1 : a.R0) +
-                                                (size_t)((jn >> 1) % c.Hkv) * D * D
-                                          : a.R0;
-                convert_r(R, bhi, blo, gt);
+            // takes another rotation, it goes into the B operand now
+            if (i + 1 < nmy && new_rot(k + 1)) {
+                load_b(a, TO_CACHE, rot_of(k + 1), bhi, blo, gt, eg);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
             }
             int b = 0, h = 0, kind = 0;
             if (TO_CACHE) {
-                kind = j & 1;
-                h = (j >> 1) % c.Hkv;
-                b = (j >> 1) / c.Hkv;
+                const int hk = j / a.B;
+                kind = hk & 1;
+                h = hk >> 1;
+                b = j - hk * a.B;
                 if (j != cur_job) {
                     L0 = start_len_thread(c, b, kind == 0 && h == 0 && gt == 0);
                     sink_list_end(c, b, s_n, s_last);
@@ -353,6 +415,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             for (int g = 0; g < NG; g++) {
                 float v[32];
                 tmem_ld32(taddr + 32 * g, v);
+                if (FWHT) {                             // the FWHT's 1/sqrt(128), in fp32
+#pragma unroll
+                    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
+                }
                 if (g == NG - 1) {
                     // the accumulator is no longer needed: free it for the tile after next
                     tc_fence_before();
@@ -453,7 +519,7 @@ bool make_map(CUtensorMap *m, const uint16_t *X, int Hkv, long long rows) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool TO_CACHE>
+template <bool TO_CACHE, bool FWHT>
 cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, TcArgs a, const CacheDst &c,
                       cudaStream_t st) {
     int dev = 0, sms = 0;
@@ -462,23 +528,24 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, TcArgs a, co
     if (e != cudaSuccess) return e;
     const int grid = std::max(1, std::min(sms, a.ntiles));
     a.tiles_per_cta = (a.ntiles + grid - 1) / grid;
-    e = cudaFuncSetAttribute(append_dense_tc_kernel<TO_CACHE>,
+    e = cudaFuncSetAttribute(append_dense_tc_kernel<TO_CACHE, FWHT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    return launch_pdl(append_dense_tc_kernel<TO_CACHE>, dim3(grid), dim3(tc::THREADS),
+    return launch_pdl(append_dense_tc_kernel<TO_CACHE, FWHT>, dim3(grid), dim3(tc::THREADS),
                       (size_t)tc::SMEM_BYTES, st, mk, mv, a, c);
 }
 
 }  // namespace
 
-bool append_tc_eligible(const uint16_t *K, const uint16_t *V, int T) {
+bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T) {
     const auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    return T >= TC_MIN_T && al(K) && al(V) && encode_fn() != nullptr;
+    return T >= (mode == KVQ_ROT_DENSE ? TC_MIN_T : TC_MIN_T_FWHT) && al(K) && al(V) &&
+           encode_fn() != nullptr;
 }
 
-cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const float *R_k,
-                             const float *R_v, const kvq_cache_desc &cd, int32_t *seq_lens,
-                             cudaStream_t st) {
+cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, int mode,
+                             const float *R_k, const float *R_v, const int32_t *perm,
+                             const kvq_cache_desc &cd, int32_t *seq_lens, cudaStream_t st) {
     CUtensorMap mk, mv;
     const long long rows = (long long)cd.B * T;
     if (!make_map(&mk, K, cd.Hkv, rows) || !make_map(&mv, V, cd.Hkv, rows)) return cudaErrorInvalidValue;
@@ -486,27 +553,33 @@ cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const 
     TcArgs a;
     a.R0 = R_k;
     a.R1 = R_v;
+    a.perm = mode == KVQ_ROT_DENSE ? nullptr : perm;
     a.out_f32 = nullptr;
     a.T = T;
+    a.B = cd.B;
+    a.Hkv = cd.Hkv;
     a.tiles_per_job = (T + tc::TILE_M - 1) / tc::TILE_M;
     a.ntiles = a.tiles_per_job * cd.B * cd.Hkv * 2;
     a.tiles_per_cta = 0;
-    return launch_tc<true>(mk, mv, a, c, st);
+    return a.perm ? launch_tc<true, true>(mk, mv, a, c, st) : launch_tc<true, false>(mk, mv, a, c, st);
 }
 
-cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, const float *R, float *out,
-                                   cudaStream_t st) {
+cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, int mode, const float *R,
+                                   const int32_t *perm, float *out, cudaStream_t st) {
     CUtensorMap m;
     if (!make_map(&m, X, 1, N)) return cudaErrorInvalidValue;
     CacheDst c{};
     TcArgs a;
     a.R0 = a.R1 = R;
+    a.perm = mode == KVQ_ROT_DENSE ? nullptr : perm;
     a.out_f32 = out;
     a.T = N;
+    a.B = 1;
+    a.Hkv = 1;
     a.tiles_per_job = (N + tc::TILE_M - 1) / tc::TILE_M;
     a.ntiles = a.tiles_per_job;
     a.tiles_per_cta = 0;
-    return launch_tc<false>(m, m, a, c, st);
+    return a.perm ? launch_tc<false, true>(m, m, a, c, st) : launch_tc<false, false>(m, m, a, c, st);
 }
 
 }  // namespace kvq

@@ -366,15 +366,16 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
                                 cudaStream_t st);
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
                                       const int32_t *perm, float *out, cudaStream_t st);
-// Bulk dense appends (T >= TC_MIN_T, 16-byte aligned K and V) run the
-// rotation on the tensor cores.
+// Bulk appends (T >= TC_MIN_T dense, T >= TC_MIN_T_FWHT permutation +
+// FWHT; 16-byte aligned K and V) run the rotation on the tensor cores.
 constexpr int TC_MIN_T = 256;
-bool append_tc_eligible(const uint16_t *K, const uint16_t *V, int T);
-cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, const float *R_k,
-                             const float *R_v, const kvq_cache_desc &cd, int32_t *seq_lens,
-                             cudaStream_t st);
-cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, const float *R, float *out,
-                                   cudaStream_t st);
+constexpr int TC_MIN_T_FWHT = 128;
+bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T);
+cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, int mode,
+                             const float *R_k, const float *R_v, const int32_t *perm,
+                             const kvq_cache_desc &cd, int32_t *seq_lens, cudaStream_t st);
+cudaError_t launch_debug_rotate_tc(const uint16_t *X, int N, int mode, const float *R,
+                                   const int32_t *perm, float *out, cudaStream_t st);
 cudaError_t launch_debug_quantize(const float *X, int N, uint8_t *codes, uint16_t *meta,
                                   cudaStream_t st);
 cudaError_t launch_debug_wait_timeout(const uint8_t *src, uint32_t poll_limit, int32_t *status,

@@ -21,6 +21,13 @@ def rot_tensors(w, device="cuda"):
     return (None, None, torch.from_numpy(perm).to(device)), (None, None, perm)
 
 
+def append_variant(mode, T):
+    """The rotation variant of kvq_debug_rotate_f32 that an append of T rows
+    runs: 1 = the tensor-core bulk kernel (dense T >= 256, permutation +
+    FWHT T >= 128), else 0."""
+    return 1 if T >= (256 if mode == 0 else 128) else 0
+
+
 def gpu_append(cache, K, V, w, rt, seq_lens):
     kvq.kvq_rotate_quantize_append(K.contiguous(), V.contiguous(), w.mode, rt[0], rt[1], rt[2],
                                    cache, seq_lens)

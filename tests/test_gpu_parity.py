@@ -18,8 +18,8 @@ import rotated_int2_kv_head_b200 as kvq
 import workloads as W
 from oracle import oracle as orc
 
-from kvq_testlib import (D, download_cache, f16bits, gpu_append, gpu_decode, logical,
-                         near_tie_ok, rel_err, rot_tensors, upload_oracle_cache)
+from kvq_testlib import (D, append_variant, download_cache, f16bits, gpu_append, gpu_decode,
+                         logical, near_tie_ok, rel_err, rot_tensors, upload_oracle_cache)
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quantizer_worked.json")
@@ -120,6 +120,12 @@ def run_append(w, L0, T, device="cuda"):
     # tiles, so CTAs cross (sequence, head, K|V) boundaries mid-range
     (0, 20, 520, [0, 2, 31]),
     (0, 0, 2400, [0, 7, 16]),
+    # bulk permutation + FWHT appends (T >= 128): the same tensor-core kernel
+    # with B built from the permutation; one full tile, and ragged tiles
+    # across rotation changes
+    (1, 0, 128, [0, 5, 16]),
+    (1, 20, 300, [0, 2, 31]),
+    (1, 0, 2400, [0, 7, 16]),
 ])
 def test_append_matches_oracle(mode, S, T, L0):
     w = W.custom(seed=10 + T, B=3, Hkv=2, mode=mode, sink=S, k_outliers=4,
@@ -135,13 +141,14 @@ def test_append_matches_oracle(mode, S, T, L0):
             rows = X[:, :, h].reshape(-1, D).cuda()
             if mode == 0:
                 R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
-                variant = 1 if T >= 256 else 0     # the kernel the append used
+                variant = append_variant(0, T)     # the kernel the append used
                 grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=variant).cpu().numpy()
                 orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 0,
                                       R=(rn[0] if kind == 0 else rn[1])[h])
             else:
                 pm = rt[2][kind, h].contiguous()
-                grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=pm).cpu().numpy()
+                grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=pm,
+                                                variant=append_variant(1, T)).cpu().numpy()
                 orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 1,
                                       perm=rn[2][kind, h])
             grot = grot.reshape(w.B, T, D)
@@ -189,18 +196,19 @@ def code_mismatches(blocks_a, blocks_b):
 
 
 @pytest.mark.parametrize("path", ["dense_cuda_cores", "dense_tensor_cores", "fwht_step",
-                                  "fwht_chunk", "prerope_gh4"])
+                                  "fwht_chunk", "fwht_tensor_cores", "prerope_gh4"])
 def test_near_tie_rate_over_a_million_codes(path):
     """Codes that differ between the packed cache and the oracle's append of
     the same rows (its fp64 rotation) come only from near ties: at most 1e-4
     of the codes, counted over 2,097,152 codes (2048 tokens x 4 heads x K and
     V) for every append kernel - the CUDA-core dense append (T < 256), the
-    tensor-core bulk append, the FWHT append one token at a time and in
-    chunks, and the pre-RoPE group rotation."""
+    tensor-core bulk append (dense, and permutation + FWHT), the CUDA-core
+    FWHT append a few tokens at a time and in chunks, and the pre-RoPE group
+    rotation."""
     Hkv, T = 4, 2048
     mode = 0 if path.startswith("dense") else 1
     chunk = {"dense_cuda_cores": 128, "dense_tensor_cores": T, "fwht_step": 8,
-             "fwht_chunk": 128, "prerope_gh4": 256}[path]
+             "fwht_chunk": 64, "fwht_tensor_cores": T, "prerope_gh4": 256}[path]
     w = W.custom(seed=540 + len(path), B=1, Hq=Hkv, Hkv=Hkv, mode=mode, context=T,
                  k_outliers=8, channel_scale=(0.5, 20.0) if mode == 1 else None)
     rt, rn = rot_tensors(w)

@@ -16,7 +16,7 @@ import rotated_int2_kv_head_b200 as kvq
 import workloads as W
 from oracle import oracle as orc
 
-from kvq_testlib import (D, f16bits, gpu_append, gpu_decode, rel_err, rot_tensors,
+from kvq_testlib import (D, append_variant, f16bits, gpu_append, gpu_decode, rel_err, rot_tensors,
                          upload_oracle_cache)
 
 pytestmark = pytest.mark.gpu
@@ -81,13 +81,14 @@ def _grot(w, rt, X, h, kind, variant):
     if w.mode == 0:
         R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
         return kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=variant).cpu().numpy()
-    return kvq.kvq_debug_rotate_f32(rows, 1, perm=rt[2][kind, h].contiguous()).cpu().numpy()
+    return kvq.kvq_debug_rotate_f32(rows, 1, perm=rt[2][kind, h].contiguous(),
+                                    variant=variant).cpu().numpy()
 
 
 @pytest.mark.parametrize("mode,chunks,paged", [
     (0, [37, 1, 70], False),           # CUDA-core dense kernel
     (0, [300, 1, 520], False),         # tensor-core bulk kernel
-    (1, [37, 1, 130], False),          # permutation + FWHT kernel
+    (1, [37, 1, 130], False),          # permutation + FWHT: CUDA-core, then tensor-core kernel
     (0, [300, 37, 1], True),           # both dense kernels on a paged cache
 ])
 def test_append_identified_sinks(mode, chunks, paged):
@@ -123,7 +124,7 @@ def test_append_identified_sinks(mode, chunks, paged):
         gpu_append(plain, K.cuda(), V.cuda(), w, rt, sl_p)
         orc.identify_sinks(oc, act, TAU, osl)
         assert orc.append(oc, f16bits(K), f16bits(V), w.mode, rn[0], rn[1], rn[2], osl) == 0
-        rows.append((list(pos), K, V, 1 if (mode == 0 and T >= 256) else 0))
+        rows.append((list(pos), K, V, append_variant(mode, T)))
         pos = [p + T for p in pos]
     torch.cuda.synchronize()
     assert kvq.kvq_get_status(ic) == 0 and kvq.kvq_get_status(plain) == 0

@@ -3,9 +3,10 @@
 It exists for callers that cannot allocate device memory: it takes no
 workspace and uses a fixed device array inside the library instead.  These
 tests call it through the C ABI, twice in a row on the same inputs, and
-check each result against the regular entry point (caller workspace) within
-the decode tolerance the other tests use.  They also check that a shape too
-large for the fixed array is refused on the host.  The file is named so that
+check each result against the regular entry point (caller workspace) and
+against the CPU oracle, within the decode tolerance the other tests use.
+They also check that a shape too large for the fixed array is refused on
+the host.  The file is named so that
 pytest collects it last, and it builds its own inputs, so it passes both on
 its own in a fresh process and after the rest of the suite.
 """
@@ -22,7 +23,7 @@ DEC_TOL = 2e-3
 
 def rows_close(a, b):
     a = a.float().cpu().numpy().astype(np.float64).reshape(-1, 128)
-    b = b.float().cpu().numpy().astype(np.float64).reshape(-1, 128)
+    b = b.double().cpu().numpy().reshape(-1, 128)
     err = np.abs(a - b).max(axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-30)
     return err.max()
 
@@ -51,12 +52,26 @@ def test_noalloc_matches_workspace_decode_twice(G, mode, S):
     ref = torch.empty_like(Q)
     kvq.kvq_decode_attention(Q, cache, mode, rk, rv, pm, lens_t, S, max(lens), ws, ref)
 
+    # the CPU oracle's decode over the same cache bytes, as a check
+    # independent of the library (the bytes, not the oracle's own append: a
+    # near-tie code that differs would move a one-token context by a whole
+    # quantization step)
+    from oracle import oracle as orc
+    oc = orc.Cache(w.B, Hkv, cap, S)
+    oc.blocks[:] = cache.block_view().cpu().numpy()
+    if S:
+        oc.k_sink[:] = W.f16_bits(cache.k_sink)
+        oc.v_sink[:] = W.f16_bits(cache.v_sink)
+    ref_o, _ = orc.decode(oc, W.f16_bits(Q), mode, Rk, Rv, perm, np.array(lens, np.int32))
+    ref_o = torch.from_numpy(ref_o)
+
     for _ in range(2):                      # two calls in a row share the array
         out = torch.full_like(Q, float("nan"))
         kvq.kvq_decode_attention_noalloc(Q, cache, mode, rk, rv, pm, lens_t, S, max(lens), out)
         torch.cuda.synchronize()
         assert torch.isfinite(out).all()
         assert rows_close(out, ref) <= DEC_TOL
+        assert rows_close(out, ref_o) <= DEC_TOL
     assert kvq.kvq_get_status(cache) == 0
 
 
