@@ -22,7 +22,9 @@
  *     sinks, singled out by massive activations, are protected from 2-bit
  *     quantization.
  *   - "KVLinC : KV Cache Quantization with Hadamard Rotation and Linear
- *     Correction", abstract: a Hadamard rotation of the values.
+ *     Correction", abstract: a Hadamard rotation of the values, and
+ *     lightweight linear correction adapters that compensate for the errors
+ *     the quantized keys introduce (decode_one's adapter, below).
  * The pages fix the 2-bit width only.  The group of 32 along head_dim, the
  * asymmetric min/max grid with an fp16 scale and fp16 zero per group, and the
  * packed cache layout are this library's format; they are restated here as
@@ -435,24 +437,56 @@ static void dequant_token(const uint8_t *unit_blocks, const uint16_t *ksink_u,
     }
 }
 
+/* KVLinC's key correction adapter ("KVLinC : KV Cache Quantization with
+ * Hadamard Rotation and Linear Correction", abstract: lightweight linear
+ * correction adapters compensate for the errors introduced by quantized
+ * keys).  The page gives no formula; the reading taken: a linear map of the
+ * dequantised key in the model's (unrotated) basis, of rank r,
+ *     k~ = k^ + (k^ . U) . V^T,      U, V: [128][r] (row-major, fp32),
+ * applied to every INT2 key; fp16 sink keys carry no quantization error and
+ * are used as stored.  U = 0 or V = 0 is the plain decode. */
+static void adapt_key(const double *k_un, const float *U, const float *V, int r, double *out) {
+    double kU[D];
+    for (int j = 0; j < r; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < D; i++) acc += k_un[i] * (double)U[i * r + j];
+        kU[j] = acc;
+    }
+    for (int i = 0; i < D; i++) {
+        double acc = 0.0;
+        for (int j = 0; j < r; j++) acc += kU[j] * (double)V[i * r + j];
+        out[i] = k_un[i] + acc;
+    }
+}
+
 /* One (b, query head): q_rot = q . R_k, scores s_t = q_rot . k_t / sqrt(128)
  * over t in [0, L), softmax, o_rot = sum p_t v_t, out = o_rot . R_v^T.
- * Query head h uses KV head h / G (contiguous GQA grouping). */
+ * Query head h uses KV head h / G (contiguous GQA grouping).  With an
+ * adapter (U != NULL), an INT2 key is taken back to the model's basis
+ * (k^ = k_rot . R_k^T), corrected (adapt_key), and scored against the
+ * unrotated query: s_t = q . k~ / sqrt(128). */
 static void decode_one(const uint16_t *q, int mode, const float *Rk, const float *Rv,
                        const int32_t *pk, const int32_t *pv, const uint8_t *unit_blocks,
                        const uint16_t *ksink_u, const uint16_t *vsink_u, int S,
                        const int32_t *sink_pos, const int32_t *sink_count, int b, int L,
-                       double *out) {
-    double qin[D], qr[D], k[D], v[D], o[D];
+                       const float *U, const float *V, int r, double *out) {
+    double qin[D], qr[D], k[D], v[D], o[D], kun[D], kad[D];
     for (int i = 0; i < D; i++) qin[i] = (double)orc_f16_to_f32(q[i]);
     rotate_f64(qin, mode, Rk, pk, qr);
     double *s = (double *)malloc(sizeof(double) * (size_t)L);
     const double scale = 1.0 / sqrt((double)D);
     double m = -INFINITY;
     for (int t = 0; t < L; t++) {
-        dequant_token(unit_blocks, ksink_u, vsink_u, sink_row(S, sink_pos, sink_count, b, t), t, k, v);
+        const int row = sink_row(S, sink_pos, sink_count, b, t);
+        dequant_token(unit_blocks, ksink_u, vsink_u, row, t, k, v);
         double acc = 0.0;
-        for (int i = 0; i < D; i++) acc += qr[i] * k[i];
+        if (U && row < 0) {
+            unrotate_f64(k, mode, Rk, pk, kun);
+            adapt_key(kun, U, V, r, kad);
+            for (int i = 0; i < D; i++) acc += qin[i] * kad[i];
+        } else {
+            for (int i = 0; i < D; i++) acc += qr[i] * k[i];
+        }
         s[t] = acc * scale;
         if (s[t] > m) m = s[t];
     }
@@ -476,11 +510,12 @@ static void decode_one(const uint16_t *q, int mode, const float *Rk, const float
  * only_b / only_h >= 0 restrict the work to one sequence / KV head (used to
  * sample large workloads); other outputs are left untouched.
  * n_threads > 1 runs (b, query head) pairs on that many OpenMP threads. */
-int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
-               const float *R_v, const int32_t *perm, int capacity, int S,
-               const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
-               const int32_t *seq_lens, const int32_t *sink_pos, const int32_t *sink_count,
-               int only_b, int only_h, int n_threads, double *out) {
+static int decode_all(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
+                      const float *R_v, const int32_t *perm, int capacity, int S,
+                      const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
+                      const int32_t *seq_lens, const int32_t *sink_pos,
+                      const int32_t *sink_count, const float *U, const float *V, int r,
+                      int only_b, int only_h, int n_threads, double *out) {
     int status = 0;
     const int G = Hq / Hkv;
     const int nblk = capacity / BLK_TOK;
@@ -507,9 +542,32 @@ int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float 
                    mode == 1 ? perm + ((size_t)Hkv + h) * D : NULL,
                    blocks + u * (size_t)nblk * BLK_BYTES,
                    S > 0 ? k_sink + u * (size_t)S * D : NULL,
-                   S > 0 ? v_sink + u * (size_t)S * D : NULL, S, sink_pos, sink_count, b, L, o);
+                   S > 0 ? v_sink + u * (size_t)S * D : NULL, S, sink_pos, sink_count, b, L,
+                   U ? U + (size_t)h * D * r : NULL, U ? V + (size_t)h * D * r : NULL, r, o);
     }
     return status;
+}
+
+int orc_decode(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
+               const float *R_v, const int32_t *perm, int capacity, int S,
+               const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
+               const int32_t *seq_lens, const int32_t *sink_pos, const int32_t *sink_count,
+               int only_b, int only_h, int n_threads, double *out) {
+    return decode_all(Q, B, Hq, Hkv, mode, R_k, R_v, perm, capacity, S, blocks, k_sink, v_sink,
+                      seq_lens, sink_pos, sink_count, NULL, NULL, 0, only_b, only_h, n_threads,
+                      out);
+}
+
+/* orc_decode with KVLinC key correction adapters U, V: fp32 [Hkv][128][r]
+ * (adapt_key, per KV head). */
+int orc_decode_adapter(const uint16_t *Q, int B, int Hq, int Hkv, int mode, const float *R_k,
+                       const float *R_v, const int32_t *perm, int capacity, int S,
+                       const uint8_t *blocks, const uint16_t *k_sink, const uint16_t *v_sink,
+                       const int32_t *seq_lens, const int32_t *sink_pos,
+                       const int32_t *sink_count, const float *U, const float *V, int r,
+                       int n_threads, double *out) {
+    return decode_all(Q, B, Hq, Hkv, mode, R_k, R_v, perm, capacity, S, blocks, k_sink, v_sink,
+                      seq_lens, sink_pos, sink_count, U, V, r, -1, -1, n_threads, out);
 }
 
 /* Attention over explicit fp64 rows (no cache, no quantization), used by the

@@ -50,6 +50,9 @@ def lib():
         L.orc_decode.restype = ci
         L.orc_decode.argtypes = [p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, p, p, ci, ci,
                                  ci, p]
+        L.orc_decode_adapter.restype = ci
+        L.orc_decode_adapter.argtypes = [p, ci, ci, ci, ci, p, p, p, ci, ci, p, p, p, p, p, p, p, p,
+                                         ci, ci, p]
         L.orc_attention_f64.argtypes = [p, p, p, ci, p]
         L.orc_rope_f64.argtypes = [p, i64, C.c_double]
         L.orc_rotate_group_f64.argtypes = [p, ci, p, p]
@@ -232,6 +235,29 @@ def decode(cache, Q, mode, R_k=None, R_v=None, perm=None, seq_lens=None,
                           cache.capacity, cache.S, _p(cache.blocks), _p(cache.k_sink),
                           _p(cache.v_sink), _p(sl), _p(cache.sink_pos), _p(cache.sink_count),
                           only_b, only_h, n_threads, _p(out))
+    return out, st
+
+
+def decode_adapter(cache, Q, mode, R_k, R_v, perm, seq_lens, U, V, n_threads=1):
+    """decode with KVLinC key correction adapters: U, V fp32 [Hkv][128][r];
+    every INT2 key k^ (model basis) is scored as k^ + (k^ . U) . V^T.
+    Returns (out fp64 [B][Hq][128], status)."""
+    Q = _c(Q, np.uint16)
+    B, Hq, d = Q.shape
+    assert d == D and B == cache.B and Hq % cache.Hkv == 0
+    Rk = _c(R_k, np.float32) if mode == 0 else None
+    Rv = _c(R_v, np.float32) if mode == 0 else None
+    pc = _c(perm, np.int32) if mode == 1 else None
+    U = _c(U, np.float32)
+    V = _c(V, np.float32)
+    assert U.shape == V.shape and U.shape[:2] == (cache.Hkv, D)
+    r = U.shape[2]
+    sl = _c(seq_lens, np.int32)
+    out = np.zeros((B, Hq, D), np.float64)
+    st = lib().orc_decode_adapter(_p(Q), B, Hq, cache.Hkv, mode, _p(Rk), _p(Rv), _p(pc),
+                                  cache.capacity, cache.S, _p(cache.blocks), _p(cache.k_sink),
+                                  _p(cache.v_sink), _p(sl), _p(cache.sink_pos),
+                                  _p(cache.sink_count), _p(U), _p(V), r, n_threads, _p(out))
     return out, st
 
 

@@ -824,3 +824,82 @@ def test_prerope_identified_sinks_match_numpy_mini_oracle():
         keys = {t: K[0, t, h].astype(np.float64) for t in sinks}
         ref = np_mini.decode_prerope_one(Q[0, h], khat, h, perm[0], base, vhat, pv, keys)
         assert np.allclose(out[0, h], ref, rtol=0, atol=1e-12)
+
+
+# --- KVLinC key correction adapters --------------------------------------------------------
+
+def _adapter_case(mode, S, G, r, seed, T=45):
+    rng = np.random.default_rng(seed)
+    B, Hkv = 2, 2
+    K = (rng.standard_normal((B, T, Hkv, D)) * 2).astype(np.float16)
+    V = rng.standard_normal((B, T, Hkv, D)).astype(np.float16)
+    if mode == 0:
+        Rk = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        Rv = np.stack([rand_orth(rng) for _ in range(Hkv)])
+        perm = None
+    else:
+        Rk = Rv = None
+        perm = np.stack([np.stack([rng.permutation(D) for _ in range(Hkv)])
+                         for _ in range(2)]).astype(np.int32)
+    cache = orc.Cache(B, Hkv, 48, S)
+    sl = np.zeros(B, np.int32)
+    assert orc.append(cache, K.view(np.uint16), V.view(np.uint16), mode, Rk, Rv, perm, sl) == 0
+    lens = np.array([T, T - 7], np.int32)
+    Q = rng.standard_normal((B, Hkv * G, D)).astype(np.float16)
+    U = (rng.standard_normal((Hkv, D, r)) * 0.1).astype(np.float32)
+    Vd = (rng.standard_normal((Hkv, D, r)) * 0.1).astype(np.float32)
+    return K, V, Q, cache, lens, Rk, Rv, perm, U, Vd
+
+
+@pytest.mark.parametrize("mode,S,G,r", [(0, 0, 1, 8), (0, 4, 2, 128), (1, 0, 1, 1), (1, 3, 4, 16)])
+def test_adapter_decode_equals_attention_with_corrected_keys(mode, S, G, r):
+    """The key correction adapter, written out with explicit matrices in
+    numpy: every INT2 key, dequantised (numpy mini-oracle) and taken back to
+    the model's basis, becomes k^ + (k^ . U) . V^T; fp16 sink keys stay as
+    stored; then plain softmax attention and the value rotation removed.  A
+    swapped U and V, a correction in the rotated basis or one applied to the
+    sinks would each fail this."""
+    K, V, Q, cache, lens, Rk, Rv, perm, U, Vd = _adapter_case(mode, S, G, r, 60 + r + S)
+    out, st = orc.decode_adapter(cache, Q.view(np.uint16), mode, Rk, Rv, perm, lens, U, Vd)
+    assert st == 0
+    B, T, Hkv = K.shape[:3]
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(Hkv):
+            kw = (lambda kind: dict(R=(Rk if kind == 0 else Rv)[h])) if mode == 0 else \
+                (lambda kind: dict(perm=perm[kind, h]))
+            Mk = np_mini.rotation_matrix(mode, **kw(0))
+            Mv = np_mini.rotation_matrix(mode, **kw(1))
+            kr = np_mini.rotate_rows_f32(K[b, :L, h], mode, **kw(0))
+            vr = np_mini.rotate_rows_f32(V[b, :L, h], mode, **kw(1))
+            kc, ks, kz = np_mini.quantize_rows(kr)
+            vc, vs, vz = np_mini.quantize_rows(vr)
+            khat = np_mini.dequant(kc, ks, kz)
+            vhat = np_mini.dequant(vc, vs, vz)
+            sink = np.arange(L) < S
+            khat[sink] = kr[sink].astype(np.float16).astype(np.float64)
+            vhat[sink] = vr[sink].astype(np.float16).astype(np.float64)
+            kmodel = khat @ Mk.T                           # back to the model's basis
+            kcorr = kmodel + (kmodel @ U[h].astype(np.float64)) @ Vd[h].astype(np.float64).T
+            kcorr[sink] = kmodel[sink]
+            for hq in range(h * G, (h + 1) * G):
+                q = Q[b, hq].astype(np.float64)
+                s = kcorr @ q / np.sqrt(D)
+                p = np.exp(s - s.max())
+                ref = (p / p.sum()) @ vhat @ Mv.T
+                assert np.allclose(out[b, hq], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_zero_adapter_is_the_plain_decode(mode):
+    K, V, Q, cache, lens, Rk, Rv, perm, U, Vd = _adapter_case(mode, 4, 2, 8, 71)
+    plain, _ = orc.decode(cache, Q.view(np.uint16), mode, Rk, Rv, perm, lens)
+    for zu, zv in ((np.zeros_like(U), Vd), (U, np.zeros_like(Vd))):
+        out, st = orc.decode_adapter(cache, Q.view(np.uint16), mode, Rk, Rv, perm, lens, zu, zv)
+        assert st == 0
+        assert np.allclose(out, plain, rtol=0, atol=1e-12)
+    # a context made of fp16 sinks only has no quantized key to correct
+    short = np.array([3, 2], np.int32)
+    plain, _ = orc.decode(cache, Q.view(np.uint16), mode, Rk, Rv, perm, short)
+    out, _ = orc.decode_adapter(cache, Q.view(np.uint16), mode, Rk, Rv, perm, short, U, Vd)
+    assert np.array_equal(out, plain)
