@@ -62,20 +62,25 @@ __device__ __forceinline__ void cache_epilogue(const CacheDst &c, int b, int t, 
 
 // ---- dense rotation on CUDA cores ---------------------------------------------------------
 // 256 threads.  Warp w owns rows 16w..16w+15 of R, lane l columns 4l..4l+3:
-// a 16x4 register tile, reused for every token of the CTA.  Tokens go in
+// a 16x4 register tile, reused for every row of the CTA.  Rows go in
 // batches of 8: every warp forms its partial dot products for all 8, the
 // partials are summed in a fixed order through shared memory, and warp k
-// finishes token k of the batch (quantize + store, or fp32 store).
+// finishes row k of the batch (quantize + store, or fp32 store).  In cache
+// mode a CTA takes one (head, K|V) and the rows (b, t) of `bpc` consecutive
+// sequences b times a chunk of `tchunk` tokens t: appends of a few tokens
+// to many sequences (a decode step) share one fetch of R between
+// sequences.
 constexpr int DENSE_THREADS = 256;
 constexpr int DENSE_BATCH = 8;
 
 struct DenseRows {
-    // cache mode: grid (tchunks, Hkv, 2*B); debug mode: grid (chunks, 1, 1)
+    // cache mode: grid (tchunks, Hkv, 2*ceil(B/bpc)); debug mode: grid (chunks, 1, 1)
     const uint16_t *X0, *X1;   // K, V (cache) or X (debug)
     const float *R0, *R1;      // R_k, R_v [Hkv][128][128] (cache) or R (debug)
     float *out_f32;            // debug output or nullptr
     int n_rows;                // debug: N
-    int tchunk;                // tokens (rows) per CTA
+    int tchunk;                // tokens (rows) per CTA and sequence
+    int bpc;                   // cache mode: sequences per CTA (1..DENSE_BATCH)
 };
 
 template <bool TO_CACHE>
@@ -83,14 +88,16 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     append_dense_kernel(DenseRows a, CacheDst c) {
     __shared__ __align__(16) uint16_t xs[DENSE_BATCH][D];
     __shared__ __align__(16) float red[DENSE_BATCH][8][D];
+    __shared__ int L0s[DENSE_BATCH];            // cache mode: start length per sequence
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int b = 0, h = 0, kind = 0, L0 = 0, row0, nrows;
+    int b0 = 0, nseq = 1, h = 0, kind = 0, row0;
     const uint16_t *X;
     const float *R;
     if (TO_CACHE) {
         h = blockIdx.y;
         kind = blockIdx.z & 1;
-        b = blockIdx.z >> 1;
+        b0 = (int)(blockIdx.z >> 1) * a.bpc;
+        nseq = min(a.bpc, c.B - b0);
         X = (kind == 0 ? a.X0 : a.X1);
         R = (kind == 0 ? a.R0 : a.R1) + (size_t)h * D * D;
     } else {
@@ -112,9 +119,12 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     pdl_trigger();
     row0 = blockIdx.x * a.tchunk;
     const int avail = min(a.tchunk, (TO_CACHE ? c.T : a.n_rows) - row0);   // >= 1 by the grid
+    // row i of the CTA: sequence b0 + i / avail, token row0 + i % avail
+    const int nrows = nseq * avail;
     // thread t stages 16 B of row (base + t/16) of a batch: 8 rows x 256 B
     const int rr = threadIdx.x >> 4, piece = threadIdx.x & 15;
-    auto piece_ptr = [&](int row) -> const uint4 * {
+    auto piece_ptr = [&](int i) -> const uint4 * {
+        const int b = b0 + i / avail, row = row0 + i % avail;
         const uint16_t *src = TO_CACHE ? X + (((size_t)b * c.T + row) * c.Hkv + h) * D
                                        : X + (size_t)row * D;
         return reinterpret_cast<const uint4 *>(src + piece * 8);
@@ -122,25 +132,22 @@ __global__ void __launch_bounds__(DENSE_THREADS)
     // the first batch's input is loaded before seq_lens is examined: the two
     // loads are independent and overlap
     uint4 first = make_uint4(0u, 0u, 0u, 0u);
-    if (rr < min(DENSE_BATCH, avail)) first = *piece_ptr(row0 + rr);
+    if (rr < min(DENSE_BATCH, nrows)) first = *piece_ptr(rr);
     unsigned claim = 0u;
     if (TO_CACHE) {
-        L0 = start_len(c, b);
-        nrows = L0 < 0 ? 0 : avail;                          // skipped sequence: no rows
+        // a skipped sequence (no room, negative length) stores no rows; the
+        // first column of CTAs reports it
+        if (threadIdx.x < nseq)
+            L0s[threadIdx.x] = start_len_thread(c, b0 + threadIdx.x,
+                                                blockIdx.x == 0 && blockIdx.y == 0 && kind == 0);
         claim = append_claim(c);                             // seq_lens is not read again
-    } else {
-        nrows = avail;
-    }
-    if (nrows <= 0) {
-        if (TO_CACHE) append_finish(c, claim);
-        return;
     }
 
     for (int base = 0; base < nrows; base += DENSE_BATCH) {
         const int nb = min(DENSE_BATCH, nrows - base);
         if (rr < nb)
             *reinterpret_cast<uint4 *>(&xs[rr][piece * 8]) =
-                base == 0 ? first : *piece_ptr(row0 + base + rr);
+                base == 0 ? first : *piece_ptr(base + rr);
         __syncthreads();
         for (int k = 0; k < nb; k++) {
             const uint4 u0 = *reinterpret_cast<const uint4 *>(&xs[k][16 * warp]);
@@ -170,12 +177,15 @@ __global__ void __launch_bounds__(DENSE_THREADS)
                 v[2] += p4.z;
                 v[3] += p4.w;
             }
-            const int row = row0 + base + warp;
-            if (TO_CACHE)
-                cache_epilogue(c, b, row, h, kind, L0, v);
-            else
+            const int i = base + warp;
+            if (TO_CACHE) {
+                const int L0 = L0s[i / avail];               // uniform over the warp
+                if (L0 >= 0) cache_epilogue(c, b0 + i / avail, row0 + i % avail, h, kind, L0, v);
+            } else {
+                const int row = row0 + i;
                 *reinterpret_cast<float4 *>(a.out_f32 + (size_t)row * D + 4 * lane) =
                     make_float4(v[0], v[1], v[2], v[3]);
+            }
         }
         __syncthreads();
     }
@@ -707,7 +717,9 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
         a.out_f32 = nullptr;
         a.n_rows = 0;
         a.tchunk = T <= 64 ? T : 64;
-        dim3 grid((T + a.tchunk - 1) / a.tchunk, cd.Hkv, 2 * cd.B);
+        // fewer than DENSE_BATCH tokens: one CTA takes several sequences
+        a.bpc = T >= DENSE_BATCH ? 1 : std::min(cd.B, DENSE_BATCH / T);
+        dim3 grid((T + a.tchunk - 1) / a.tchunk, cd.Hkv, 2 * ((cd.B + a.bpc - 1) / a.bpc));
         return launch_pdl(append_dense_kernel<true>, grid, dim3(DENSE_THREADS), 0, st, a, c);
     } else {
         FwhtRows a;
@@ -736,6 +748,7 @@ cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const 
         a.out_f32 = out;
         a.n_rows = N;
         a.tchunk = 64;
+        a.bpc = 1;
         append_dense_kernel<false><<<(N + 63) / 64, DENSE_THREADS, 0, st>>>(a, c);
     } else {
         FwhtRows a;
