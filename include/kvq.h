@@ -348,6 +348,34 @@ KVQ_API kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_
                                    size_t ws_bytes, uint16_t *out, void *stream);
 
 /*
+ * Decode with KVLinC key correction adapters ("KVLinC : KV Cache
+ * Quantization with Hadamard Rotation and Linear Correction", abstract:
+ * lightweight linear correction adapters compensate for the errors that the
+ * quantized keys introduce; with the values Hadamard-rotated and the keys
+ * unrotated - dense mode with R_k = I, R_v = H/sqrt(128) - this is KVLinC's
+ * configuration).  The page gives no formula; the library's reading: a
+ * rank-r linear map of every dequantised INT2 key in the model's
+ * (unrotated) basis,
+ *     k~ = k^ + (k^ . U) . V^T,
+ * scored as q . k~ / sqrt(128); fp16 sink keys (no quantization error) are
+ * scored as stored.  The map is folded into the query once per call
+ * (q . k~ = k^ . (q + (q . V) . U^T)), so the streaming over the cache is
+ * that of kvq_decode_attention_ex.
+ *   U_k, V_k  device fp32 [Hkv][128][rank], row-major, caller-owned.
+ *   rank      1..128.
+ * Other arguments, layouts and errors as kvq_decode_attention_ex.  Null
+ * U_k / V_k or rank outside [1, 128] -> KVQ_ERR_INVALID_ARG; U_k or V_k not
+ * 4-byte aligned -> KVQ_ERR_UNSUPPORTED.
+ */
+KVQ_API kvq_status kvq_decode_attention_adapter(const uint16_t *Q, int32_t Hq, int32_t q_len,
+                                        uint32_t flags, const kvq_cache_desc *cache,
+                                        kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                        const int32_t *perm, const float *U_k, const float *V_k,
+                                        int32_t rank, const int32_t *seq_lens,
+                                        int32_t sink_fp16, int32_t max_ctx, void *workspace,
+                                        size_t ws_bytes, uint16_t *out, void *stream);
+
+/*
  * Pre-RoPE grouped-head key rotation (RotateKV abstract, item (ii): the
  * outlier-aware rotation applied to the keys before RoPE and across heads).
  * The keys of group_heads (gh) consecutive KV heads form one row of

@@ -10,6 +10,7 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   decode_workspace,
                   kvq_cache_bytes, kvq_clear_status, kvq_debug_quantize_f32, kvq_debug_rotate_f32,
                   kvq_decode_attention, kvq_decode_attention_ex, kvq_decode_attention_noalloc,
+                  kvq_decode_attention_adapter,
                   kvq_decode_attention_timed,
                   kvq_decode_workspace_size, kvq_get_status, kvq_identify_sinks,
                   kvq_rotate_quantize_append, lib, kvq_prerope_append, kvq_prerope_decode,
@@ -24,6 +25,7 @@ __all__ = [
     "KVQ_DEV_BAD_LEN", "KVQ_DEV_TIMEOUT", "decode_workspace", "kvq_cache_bytes",
     "kvq_clear_status", "kvq_debug_quantize_f32", "kvq_debug_rotate_f32",
     "kvq_decode_attention", "kvq_decode_attention_ex", "kvq_decode_attention_noalloc",
+    "kvq_decode_attention_adapter",
     "kvq_decode_attention_timed",
     "kvq_decode_workspace_size", "kvq_get_status", "kvq_identify_sinks",
     "kvq_rotate_quantize_append", "lib", "kvq_prerope_append", "kvq_prerope_decode",

@@ -253,7 +253,8 @@ kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t fl
                        const kvq_cache_desc *cache, kvq_rot_mode mode, const float *R_k,
                        const float *R_v, const int32_t *perm, const int32_t *seq_lens,
                        int32_t sink_fp16, int32_t max_ctx, void *workspace, size_t ws_bytes,
-                       uint16_t *out, void *stream, void *ev_begin, void *ev_end) {
+                       uint16_t *out, void *stream, void *ev_begin, void *ev_end,
+                       const KeyAdapter &ad = KeyAdapter()) {
     int C = 0;
     const kvq_status s = decode_check(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens,
                                       sink_fp16, max_ctx, workspace, ws_bytes, out, C);
@@ -261,7 +262,7 @@ kvq_status decode_impl(const uint16_t *Q, int32_t Hq, int32_t q_len, uint32_t fl
     cudaError_t e = launch_decode(Q, Hq * q_len, *cache, mode, R_k, R_v, perm, seq_lens, C,
                                   workspace, out, static_cast<cudaStream_t>(stream),
                                   static_cast<cudaEvent_t>(ev_begin), static_cast<cudaEvent_t>(ev_end),
-                                  q_len, (flags & KVQ_DECODE_OUT_ROTATED) ? 1 : 0);
+                                  q_len, (flags & KVQ_DECODE_OUT_ROTATED) ? 1 : 0, ad);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -286,6 +287,23 @@ kvq_status kvq_decode_attention_ex(const uint16_t *Q, int32_t Hq, int32_t q_len,
                                    size_t ws_bytes, uint16_t *out, void *stream) {
     return decode_impl(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
                        max_ctx, workspace, ws_bytes, out, stream, nullptr, nullptr);
+}
+
+kvq_status kvq_decode_attention_adapter(const uint16_t *Q, int32_t Hq, int32_t q_len,
+                                        uint32_t flags, const kvq_cache_desc *cache,
+                                        kvq_rot_mode mode, const float *R_k, const float *R_v,
+                                        const int32_t *perm, const float *U_k, const float *V_k,
+                                        int32_t rank, const int32_t *seq_lens, int32_t sink_fp16,
+                                        int32_t max_ctx, void *workspace, size_t ws_bytes,
+                                        uint16_t *out, void *stream) {
+    if (!U_k || !V_k || rank < 1 || rank > 128) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(U_k, 4) || !aligned(V_k, 4)) return KVQ_ERR_UNSUPPORTED;
+    KeyAdapter ad;
+    ad.U = U_k;
+    ad.V = V_k;
+    ad.r = rank;
+    return decode_impl(Q, Hq, q_len, flags, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
+                       max_ctx, workspace, ws_bytes, out, stream, nullptr, nullptr, ad);
 }
 
 kvq_status kvq_append_decode(const uint16_t *K, const uint16_t *V, int32_t T, const uint16_t *Q,

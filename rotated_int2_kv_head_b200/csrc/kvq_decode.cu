@@ -88,6 +88,9 @@ struct DecodeArgs {
     // query i = hq % qlen of its head and sees positions < L - (qlen-1-i)
     int qlen;
     int out_rotated;   // 1: out = o_rot (the caller folds R_v^T into its projection)
+    // KVLinC key correction adapter (or null): U, V fp32 [Hkv][128][adr]
+    const float *adU, *adV;
+    int adr;
 };
 
 // Blocks of 16 tokens that hold codes for a sequence of length L: positions
@@ -284,11 +287,20 @@ __device__ __forceinline__ bool sched_take(Sched &ps, const DecodeArgs &a, int m
 // qsum[4]}.  R_k (64 KB per head, the bulk of what it reads) is fetched
 // before the dependency wait, alongside a preceding append; Q after it.
 // ---------------------------------------------------------------------------------------------
+// With a key correction adapter ("KVLinC : KV Cache Quantization with
+// Hadamard Rotation and Linear Correction", abstract: lightweight linear
+// adapters compensate for the errors of the quantized keys), every INT2 key
+// k^ (model basis) is scored as k^ + (k^ . U) . V^T.  Its score against q is
+// k^ . qc with qc = q + (q . V) . U^T, so the correction is folded into the
+// query once per call: qc replaces q before the rotation, and the streaming
+// kernel is unchanged.  The fp16 sinks (no quantization error) are scored by
+// the merge kernel against the query as given.
 constexpr int QP_THREADS = 256;
 
 __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) {
     __shared__ __align__(16) float red[QP_THREADS / 32][D];
     __shared__ __align__(16) float qr_s[D];
+    __shared__ __align__(16) float qa_s[D], tv_s[D], qadj_s[D];   // adapter: q, q . V, qc
     const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int G = a.G;
@@ -316,6 +328,24 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
         const int hq = h * G + hd;
         const uint16_t *q = a.Q + ((size_t)b * a.Hq + hq) * D;
         __syncthreads();
+        const bool adapt = a.adU != nullptr;
+        if (adapt) {                                   // qc = q + (q . V) . U^T, fp32
+            const float *U = a.adU + (size_t)h * D * a.adr, *V = a.adV + (size_t)h * D * a.adr;
+            if (t < D) qa_s[t] = __half2float(__ushort_as_half(q[t]));
+            __syncthreads();
+            if (t < a.adr) {
+                float acc = 0.f;
+                for (int i = 0; i < D; i++) acc = fmaf(qa_s[i], V[(size_t)i * a.adr + t], acc);
+                tv_s[t] = acc;
+            }
+            __syncthreads();
+            if (t < D) {
+                float acc = qa_s[t];
+                for (int j = 0; j < a.adr; j++) acc = fmaf(U[(size_t)t * a.adr + j], tv_s[j], acc);
+                qadj_s[t] = acc;
+            }
+            __syncthreads();
+        }
         if (a.mode == KVQ_ROT_DENSE) {
             const uint4 u0 = *reinterpret_cast<const uint4 *>(q + 16 * warp);
             const uint4 u1 = *reinterpret_cast<const uint4 *>(q + 16 * warp + 8);
@@ -323,7 +353,9 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int ii = 0; ii < 8; ii++) {
-                const float2 x2 = unpack_half2(w8[ii]);
+                const float2 x2 = adapt ? make_float2(qadj_s[16 * warp + 2 * ii],
+                                                      qadj_s[16 * warp + 2 * ii + 1])
+                                        : unpack_half2(w8[ii]);
                 const float4 ra = rr[2 * ii], rb = rr[2 * ii + 1];
                 acc.x = fmaf(x2.x, ra.x, acc.x); acc.y = fmaf(x2.x, ra.y, acc.y);
                 acc.z = fmaf(x2.x, ra.z, acc.z); acc.w = fmaf(x2.x, ra.w, acc.w);
@@ -340,10 +372,18 @@ __global__ void __launch_bounds__(QP_THREADS) decode_qprep_kernel(DecodeArgs a) 
             }
         } else if (warp == 0) {
             const int4 pi = *reinterpret_cast<const int4 *>(a.perm + (size_t)h * D + 4 * lane);
-            float v[4] = {__half2float(__ushort_as_half(q[pi.x & (D - 1)])),
-                          __half2float(__ushort_as_half(q[pi.y & (D - 1)])),
-                          __half2float(__ushort_as_half(q[pi.z & (D - 1)])),
-                          __half2float(__ushort_as_half(q[pi.w & (D - 1)]))};
+            float v[4];
+            if (adapt) {
+                v[0] = qadj_s[pi.x & (D - 1)];
+                v[1] = qadj_s[pi.y & (D - 1)];
+                v[2] = qadj_s[pi.z & (D - 1)];
+                v[3] = qadj_s[pi.w & (D - 1)];
+            } else {
+                v[0] = __half2float(__ushort_as_half(q[pi.x & (D - 1)]));
+                v[1] = __half2float(__ushort_as_half(q[pi.y & (D - 1)]));
+                v[2] = __half2float(__ushort_as_half(q[pi.z & (D - 1)]));
+                v[3] = __half2float(__ushort_as_half(q[pi.w & (D - 1)]));
+            }
             fwht128_warp(v);
             *reinterpret_cast<float4 *>(&qr_s[4 * lane]) =
                 make_float4(v[0] * 0.08838834764831845f, v[1] * 0.08838834764831845f,
@@ -1297,7 +1337,7 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
                           cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end, int qlen,
-                          int out_rotated) {
+                          int out_rotated, const KeyAdapter &ad) {
     const WsLayout w = ws_layout(cd.B, Hq, cd.Hkv, C);
     uint8_t *base = static_cast<uint8_t *>(ws);
     DecodeArgs a;
@@ -1329,6 +1369,9 @@ cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, i
     a.C = C;
     a.qlen = qlen;
     a.out_rotated = out_rotated;
+    a.adU = ad.U;
+    a.adV = ad.V;
+    a.adr = ad.r;
     cudaError_t e = launch_pdl(decode_qprep_kernel, dim3(cd.Hkv, cd.B), dim3(QP_THREADS), 0, st, a);
     if (e != cudaSuccess) return e;
     if (ev_begin && (e = cudaEventRecord(ev_begin, st)) != cudaSuccess) return e;

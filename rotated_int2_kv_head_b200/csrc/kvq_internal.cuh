@@ -392,11 +392,17 @@ size_t prerope_ws_bytes(int B, int Hq, int Hkv, int gh, int max_ctx, int sms);
 cudaError_t launch_decode_prerope(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int gh,
                                   const int32_t *perm, float rope_base, const int32_t *seq_lens,
                                   int max_ctx, int sms, void *ws, uint16_t *out, cudaStream_t st);
+// KVLinC key correction adapter of a decode: U, V fp32 [Hkv][128][r], or
+// none (U = nullptr).
+struct KeyAdapter {
+    const float *U = nullptr, *V = nullptr;
+    int r = 0;
+};
 cudaError_t launch_decode(const uint16_t *Q, int Hq, const kvq_cache_desc &cd, int mode,
                           const float *R_k, const float *R_v, const int32_t *perm,
                           const int32_t *seq_lens, int C, void *ws, uint16_t *out,
                           cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end, int qlen,
-                          int out_rotated);
+                          int out_rotated, const KeyAdapter &ad = KeyAdapter());
 
 // Decode workspace: prepared queries and split partials.
 struct WsLayout {

@@ -92,6 +92,10 @@ def lib():
     L.kvq_decode_attention_ex.restype = C.c_int
     L.kvq_decode_attention_ex.argtypes = [p, i32, i32, C.c_uint32, C.POINTER(CacheDesc), C.c_int, p,
                                           p, p, p, i32, i32, p, sz, p, p]
+    L.kvq_decode_attention_adapter.restype = C.c_int
+    L.kvq_decode_attention_adapter.argtypes = [p, i32, i32, C.c_uint32, C.POINTER(CacheDesc),
+                                               C.c_int, p, p, p, p, p, i32, p, i32, i32, p, sz, p,
+                                               p]
     L.kvq_decode_attention_noalloc.restype = C.c_int
     L.kvq_decode_attention_noalloc.argtypes = [p, i32, C.POINTER(CacheDesc), C.c_int, p, p, p, p,
                                                i32, i32, p, p]
@@ -399,6 +403,33 @@ def kvq_decode_attention_ex(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16,
                                          _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(seq_lens),
                                          sink_fp16, max_ctx, _ptr(workspace), workspace.numel(),
                                          _ptr(out), _stream(stream, Q)))
+
+
+def kvq_decode_attention_adapter(Q, cache, mode, R_k, R_v, perm, U_k, V_k, seq_lens, sink_fp16,
+                                 max_ctx, workspace, out, flags=0, stream=None):
+    """Decode with KVLinC key correction adapters U_k, V_k fp32 [Hkv][128][r]:
+    every INT2 key k^ (model basis) is scored as k^ + (k^ . U) . V^T.
+    Q fp16 [B][Hq][128] or [B][Hq][q_len][128] -> out of the same shape."""
+    _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
+    if U_k is None or V_k is None or U_k.dim() != 3:
+        raise ValueError("U_k and V_k must be [Hkv][128][rank] tensors")
+    _need(U_k, torch.float32, "U_k", (cache.Hkv, D, U_k.shape[2]))
+    _need(V_k, torch.float32, "V_k", U_k.shape)
+    if Q.dim() == 3:
+        B, Hq, d = Q.shape
+        q_len = 1
+    else:
+        B, Hq, q_len, d = Q.shape
+    _need(Q, torch.float16, "Q", (cache.B, Hq, D) if Q.dim() == 3 else (cache.B, Hq, q_len, D))
+    _need(out, torch.float16, "out", Q.shape)
+    _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+    _need(workspace, torch.uint8, "workspace")
+    _check("kvq_decode_attention_adapter",
+           lib().kvq_decode_attention_adapter(_ptr(Q), Hq, q_len, flags, C.byref(cache.desc), mode,
+                                              _ptr(R_k), _ptr(R_v), _ptr(perm), _ptr(U_k),
+                                              _ptr(V_k), U_k.shape[2], _ptr(seq_lens), sink_fp16,
+                                              max_ctx, _ptr(workspace), workspace.numel(),
+                                              _ptr(out), _stream(stream, Q)))
 
 
 def kvq_decode_attention_timed(Q, cache, mode, R_k, R_v, perm, seq_lens, sink_fp16, max_ctx,
