@@ -535,7 +535,7 @@ def decode_rates(device, peak, reps=20):
     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     res = {"how": "decode only, cache filled first, L2 flushed before each call, median of %d"
                   % reps}
-    for name in ("tiny", "llama7b", "hadamard", "gqa_sinks", "ragged"):
+    for name in ("tiny", "llama7b", "hadamard", "gqa_sinks", "gqa8", "ragged"):
         w = W.WORKLOADS[name]
         lens_np = w.seq_lens().astype(np.int32)
         L = int(lens_np.max())

@@ -195,11 +195,14 @@ __device__ __forceinline__ void convert_r(const float *R, uint8_t *bhi, uint8_t 
 // warp inverts the permutation into its own 128 bytes of scratch (pinv_w),
 // so only warp-level synchronisation is needed.  Entries of a permutation
 // outside [0, 128) are wrapped.
-__device__ __forceinline__ void build_fwht_b(const int32_t *perm, uint8_t *bhi, uint8_t *pinv_w,
+__device__ __forceinline__ void build_fwht_b(const int4 pv, uint8_t *bhi, uint8_t *pinv_w,
                                              int tt) {
     const int lane = tt & 31;
-#pragma unroll
-    for (int k = 0; k < 4; k++) pinv_w[perm[lane + 32 * k] & (D - 1)] = (uint8_t)(lane + 32 * k);
+    // pv = perm[lane], perm[lane + 32], perm[lane + 64], perm[lane + 96]
+    pinv_w[pv.x & (D - 1)] = (uint8_t)lane;
+    pinv_w[pv.y & (D - 1)] = (uint8_t)(lane + 32);
+    pinv_w[pv.z & (D - 1)] = (uint8_t)(lane + 64);
+    pinv_w[pv.w & (D - 1)] = (uint8_t)(lane + 96);
     __syncwarp();
     const int j = tt;
 #pragma unroll 4
@@ -222,14 +225,21 @@ __device__ __forceinline__ void build_fwht_b(const int32_t *perm, uint8_t *bhi, 
     __syncwarp();
 }
 
+// The permutation entries of rotation key hk (cache: 2h + kind; test: 0)
+// that lane `lane` of a building warp needs (FWHT mode); loaded ahead of the
+// wait that precedes the build.
+__device__ __forceinline__ int4 fwht_perm_regs(const TcArgs &a, bool to_cache, int hk, int lane) {
+    const int32_t *pm = to_cache ? a.perm + ((size_t)(hk & 1) * a.Hkv + (hk >> 1)) * D : a.perm;
+    return make_int4(pm[lane], pm[lane + 32], pm[lane + 64], pm[lane + 96]);
+}
+
 // The B operand of rotation key hk (cache: 2h + kind; test: 0) by the 128
-// threads of epilogue group eg.
-__device__ __forceinline__ void load_b(const TcArgs &a, bool to_cache, int hk, uint8_t *bhi,
-                                       uint8_t *blo, int gt, int eg) {
+// threads of epilogue group eg; pv: fwht_perm_regs of hk (FWHT mode).
+__device__ __forceinline__ void load_b(const TcArgs &a, bool to_cache, int hk, int4 pv,
+                                       uint8_t *bhi, uint8_t *blo, int gt, int eg) {
     if (a.perm) {
-        const int32_t *pm = to_cache ? a.perm + ((size_t)(hk & 1) * a.Hkv + (hk >> 1)) * D : a.perm;
         // per-warp scratch in the lo part, unused by this rotation
-        build_fwht_b(pm, bhi, blo + 128 * (4 * eg + (gt >> 5)), gt);
+        build_fwht_b(pv, bhi, blo + 128 * (4 * eg + (gt >> 5)), gt);
     } else {
         const float *R = to_cache ? ((hk & 1) ? a.R1 : a.R0) + (size_t)(hk >> 1) * D * D : a.R0;
         convert_r(R, bhi, blo, gt);
@@ -367,7 +377,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int q = warp & 3;                         // TMEM lane quarter this warp may read
         const int row = 32 * q + lane;                  // accumulator row = tile row
         if (eg == 0 && nmy > 0) {                       // R for the first job
-            load_b(a, TO_CACHE, rot_of(k0), bhi, blo, gt, eg);
+            load_b(a, TO_CACHE, rot_of(k0),
+                   FWHT ? fwht_perm_regs(a, TO_CACHE, rot_of(k0), lane) : make_int4(0, 0, 0, 0),
+                   bhi, blo, gt, eg);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
@@ -378,20 +390,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             // decisions stay warp-uniform: tcgen05.ld below is .sync.aligned
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const int k = k0 + i, j = job_of(k), buf = i % EPI_GROUPS;     // = eg
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait_bounded(&bar[BAR_ACCF + buf], (i / EPI_GROUPS) & 1))) {
-                fail();
-                break;
-            }
-            tc_fence_after();
-            // this tile's MMAs (and all earlier ones) are done: if the next tile
-            // takes another rotation, it goes into the B operand now
-            if (i + 1 < nmy && new_rot(k + 1)) {
-                load_b(a, TO_CACHE, rot_of(k + 1), bhi, blo, gt, eg);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
-            }
+            // global reads this tile needs, issued before the wait on its
+            // accumulator: the next rotation's permutation entries and the
+            // job's start length
+            const bool rebuild = i + 1 < nmy && new_rot(k + 1);
+            int4 pv = make_int4(0, 0, 0, 0);
+            if (FWHT && rebuild) pv = fwht_perm_regs(a, TO_CACHE, rot_of(k + 1), lane);
             int b = 0, h = 0, kind = 0;
             if (TO_CACHE) {
                 const int hk = j / a.B;
@@ -403,6 +407,20 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     sink_list_end(c, b, s_n, s_last);
                     cur_job = j;
                 }
+            }
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_bounded(&bar[BAR_ACCF + buf], (i / EPI_GROUPS) & 1))) {
+                fail();
+                break;
+            }
+            tc_fence_after();
+            // this tile's MMAs (and all earlier ones) are done: if the next tile
+            // takes another rotation, it goes into the B operand now
+            if (rebuild) {
+                load_b(a, TO_CACHE, rot_of(k + 1), pv, bhi, blo, gt, eg);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
             }
             const int t = (k - j * a.tiles_per_job) * TILE_M + row;
             const bool valid = t < a.T && (!TO_CACHE || L0 >= 0);

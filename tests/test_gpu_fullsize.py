@@ -1,4 +1,4 @@
-"""The five workloads at full size, in the launch configuration bench.py
+"""The workloads at full size, in the launch configuration bench.py
 uses, checked against the CPU oracle on sampled (sequence, KV head) units.
 
 The GPU fills the whole cache from inputs drawn on the GPU; the rows of the
@@ -112,6 +112,10 @@ def test_hadamard_full():
 
 def test_gqa_sinks_full():
     check(W.WORKLOADS["gqa_sinks"], [(0, 0), (7, 7)])
+
+
+def test_gqa8_full():
+    check(W.WORKLOADS["gqa8"], [(0, 0), (3, 7)])
 
 
 def test_ragged_full():

@@ -17,6 +17,8 @@ The five workloads (head_dim 128, INT2 groups of 32 along head_dim):
   ragged      B=64, 32 heads, context lengths uniform in [1024, 65536],
               dense rotation, 8 key outlier channels x20; plus a separate
               bulk append of 32768 prefill tokens x 32 heads for B=4.
+  gqa8        B=4, 64 query heads over 8 KV heads (G = 8), context 65536,
+              dense rotation, 8 key outlier channels x20.
   ragged_b8   the first 8 sequences of ragged (for profiler captures).
   gqa_sinks_identified
               gqa_sinks, but the 4 fp16 rows go to the tokens picked by their
@@ -87,6 +89,9 @@ WORKLOADS = {
                           context=131072, sink_key_scale=50.0),
     "ragged": Workload("ragged", 1005, B=64, Hq=32, Hkv=32, mode=0, ragged=(1024, 65536),
                        k_outliers=8, extra={"prefill_B": 4, "prefill_T": 32768}),
+    # eight query heads per KV head (64 over 8), the widest GQA grouping the
+    # library takes
+    "gqa8": Workload("gqa8", 1007, B=4, Hq=64, Hkv=8, mode=0, context=65536, k_outliers=8),
     # the first 8 sequences of ragged (same seed, so the same lengths): a
     # cache of 1.6 GB, small enough for a full profiler capture of the
     # decode kernels, whose counters scale to ragged by the bytes read
