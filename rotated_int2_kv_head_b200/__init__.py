@@ -5,7 +5,7 @@ hand-written CUDA kernels behind a C ABI (include/kvq.h).  This package holds
 the CUDA sources (csrc/), the in-tree build (build.py) and a thin ctypes
 binding (kvq.py) with the same function names as the C ABI.
 """
-from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ_DEV_TIMEOUT,
+from .kvq import (HostStep, KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ_DEV_TIMEOUT,
                   KVQ_DEV_BAD_TABLE, KVQ_ROT_DENSE, KVQ_ROT_PERM_FWHT, KVCache, KvqError, PagedKVCache,
                   decode_workspace,
                   kvq_cache_bytes, kvq_clear_status, kvq_debug_quantize_f32, kvq_debug_rotate_f32,
@@ -20,7 +20,7 @@ from .kvq import (KVQ_DECODE_OUT_ROTATED, KVQ_DEV_BAD_LEN, KVQ_DEV_CAPACITY, KVQ
                   kvq_debug_wait_timeout)
 
 __all__ = [
-    "KVCache", "PagedKVCache", "KvqError", "KVQ_DEV_BAD_TABLE", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
+    "HostStep", "KVCache", "PagedKVCache", "KvqError", "KVQ_DEV_BAD_TABLE", "KVQ_DECODE_OUT_ROTATED", "KVQ_ROT_DENSE", "KVQ_ROT_PERM_FWHT",
     "KVQ_DEV_CAPACITY",
     "KVQ_DEV_BAD_LEN", "KVQ_DEV_TIMEOUT", "decode_workspace", "kvq_cache_bytes",
     "kvq_clear_status", "kvq_debug_quantize_f32", "kvq_debug_rotate_f32",

@@ -392,12 +392,17 @@ kvq_status kvq_append_decode_host(const uint16_t *K_host, const uint16_t *V_host
     const bool one = reinterpret_cast<const uint8_t *>(V_host) == hk + kv &&
                      reinterpret_cast<const uint8_t *>(Q_host) == hk + 2 * kv && l.v == l.k + kv &&
                      l.q == l.v + kv;
+    // Adjacent host inputs may still be separate allocations (a caching host
+    // allocator can place them back to back): if the single copy is refused,
+    // the three copies are made instead.
+    bool copied = false;
     if (one) {
-        if (cudaMemcpyAsync(K, K_host, 2 * kv + qb, cudaMemcpyHostToDevice, st) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-    } else if (cudaMemcpyAsync(K, K_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-               cudaMemcpyAsync(V, V_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-               cudaMemcpyAsync(Q, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+        copied = cudaMemcpyAsync(K, K_host, 2 * kv + qb, cudaMemcpyHostToDevice, st) == cudaSuccess;
+        if (!copied) (void)cudaGetLastError();
+    }
+    if (!copied && (cudaMemcpyAsync(K, K_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                    cudaMemcpyAsync(V, V_host, kv, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                    cudaMemcpyAsync(Q, Q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess)) {
         return KVQ_ERR_CUDA;
     }
     if ((s = append_launch(K, V, T, mode, R_k, R_v, perm, cache, seq_lens, stream)) != KVQ_OK) return s;

@@ -385,6 +385,50 @@ def kvq_append_decode_host(K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, 
                                         _stream(stream, workspace)))
 
 
+class HostStep:
+    """kvq_append_decode_host prepared once: every argument is checked here,
+    and run() queues the step (copies in, append, decode, copy out) with one
+    C call and no per-call Python checks, for a serving loop whose buffers
+    stay the same from step to step (their contents change: new K/V rows,
+    new queries).  The tensors must stay alive and keep their shapes; the
+    stream is the one given (or current) at construction.  run() may name
+    another int32 [B] device tensor of lengths for that step."""
+
+    def __init__(self, K_host, V_host, Q_host, cache, mode, R_k, R_v, perm, seq_lens, max_ctx,
+                 workspace, out_host, stream=None):
+        _need_rotation(mode, R_k, R_v, perm, cache.Hkv)
+        B, T, Hkv, d = K_host.shape
+        _need_host(K_host, torch.float16, "K_host", (cache.B, T, cache.Hkv, D))
+        _need_host(V_host, torch.float16, "V_host", K_host.shape)
+        _need_host(Q_host, torch.float16, "Q_host")
+        _need_host(out_host, torch.float16, "out_host", Q_host.shape)
+        _need(seq_lens, torch.int32, "seq_lens", (cache.B,))
+        _need(workspace, torch.uint8, "workspace")
+        if Q_host.dim() != 3 or Q_host.shape[0] != cache.B or Q_host.shape[2] != D:
+            raise ValueError("Q_host must have shape (B, Hq, 128)")
+        self._keep = (K_host, V_host, Q_host, cache, R_k, R_v, perm, seq_lens, workspace,
+                      out_host)
+        self._fn = lib().kvq_append_decode_host
+        self._sl_shape = seq_lens.shape
+        self._sl_dev = seq_lens.device
+        self._args = [_ptr(K_host), _ptr(V_host), T, _ptr(Q_host), Q_host.shape[1],
+                      C.byref(cache.desc), mode, _ptr(R_k), _ptr(R_v), _ptr(perm),
+                      _ptr(seq_lens), max_ctx, _ptr(workspace), workspace.numel(),
+                      _ptr(out_host), _stream(stream, workspace)]
+
+    def run(self, seq_lens=None):
+        args = self._args
+        if seq_lens is not None:
+            if (seq_lens.dtype is not torch.int32 or seq_lens.shape != self._sl_shape or
+                    seq_lens.device != self._sl_dev or not seq_lens.is_contiguous()):
+                raise ValueError("seq_lens must be a contiguous int32 tensor like the plan's")
+            args = list(args)
+            args[10] = seq_lens.data_ptr()
+        code = self._fn(*args)
+        if code:
+            raise KvqError("kvq_append_decode_host", code)
+
+
 KVQ_DECODE_OUT_ROTATED = 1
 
 

@@ -669,3 +669,51 @@ def test_append_decode_host_rejects_bad_calls():
         kvq.kvq_append_decode_host(K1.cuda(), K1, Q, cache, 0, *rt, sl, 64, ws, hO)
     torch.cuda.synchronize()
     assert list(sl.cpu().numpy()) == [0] and kvq.kvq_get_status(cache) == 0
+
+
+@pytest.mark.parametrize("layout", ["one buffer", "separate"])
+def test_host_step_plan_equals_the_host_call(layout):
+    """HostStep checks its arguments once and then runs kvq_append_decode_host
+    with one C call per step: the same cache bytes, lengths and output bits as
+    the plain call, also when each run names its own row of lengths; a
+    lengths tensor of the wrong shape is refused."""
+    w = W.custom(seed=330, B=2, Hq=4, Hkv=2, mode=0, k_outliers=4)
+    rt, _ = rot_tensors(w)
+    cap, T = 256, 2
+    K = torch.stack([W.kv_rows(w, b, 0, 100, "cpu")[0] for b in range(2)])
+    V = torch.stack([W.kv_rows(w, b, 0, 100, "cpu")[1] for b in range(2)])
+    Q = W.queries(w, "cpu")
+    res = []
+    for use_plan in (False, True):
+        cache = kvq.KVCache(2, 2, cap)
+        sl = torch.zeros(2, dtype=torch.int32, device="cuda")
+        gpu_append(cache, K[:, :90].contiguous().cuda(), V[:, :90].contiguous().cuda(), w, rt, sl)
+        Kn, Vn = K[:, 90:90 + T].contiguous(), V[:, 90:90 + T].contiguous()
+        if layout == "one buffer":     # views of one pinned buffer, as a serving loop keeps them
+            buf = torch.cat([Kn.reshape(-1), Vn.reshape(-1), Q.reshape(-1)]).pin_memory()
+            n = Kn.numel()
+            hk, hv = buf[:n].view(Kn.shape), buf[n:2 * n].view(Vn.shape)
+            hq = buf[2 * n:].view(Q.shape)
+        else:                          # three pinned allocations (possibly adjacent)
+            hk, hv, hq = Kn.pin_memory(), Vn.pin_memory(), Q.pin_memory()
+        hO = torch.zeros(Q.shape, dtype=torch.float16).pin_memory()
+        ws = kvq.step_workspace(2, T, 4, 2, cap)
+        rows = torch.tensor([[90, 90], [92, 92]], dtype=torch.int32, device="cuda")
+        outs = []
+        plan = kvq.HostStep(hk, hv, hq, cache, 0, *rt, rows[0], cap, ws, hO) if use_plan else None
+        for i in range(2):
+            if use_plan:
+                plan.run(rows[i])
+            else:
+                kvq.kvq_append_decode_host(hk, hv, hq, cache, 0, *rt, rows[i], cap, ws, hO)
+            torch.cuda.synchronize()
+            outs.append(hO.clone())
+        assert kvq.kvq_get_status(cache) == 0
+        res.append((cache.blocks.clone(), rows.clone(), outs))
+        if use_plan:
+            with pytest.raises(ValueError):
+                plan.run(rows)                       # [2][2]: not int32 [B]
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    for a, b in zip(res[0][2], res[1][2]):
+        assert torch.equal(a, b)
+    assert list(res[1][1].cpu().numpy().ravel()) == [92, 92, 94, 94]
