@@ -242,8 +242,7 @@ __device__ __forceinline__ void fwht_row_quarter(const uint16_t *xrow, const int
             v[e] = fmaf(sgn, v[e], o);
         }
     }
-#pragma unroll
-    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
+    scale_group(v, 0.08838834764831845f);
 }
 
 // Four threads per row.  Thread q (0..3) owns elements 32q..32q+31 of the

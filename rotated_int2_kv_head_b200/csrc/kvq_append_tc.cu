@@ -26,7 +26,11 @@
 // K-major swizzled layout; when the range moves to a job with another
 // rotation, the epilogue group that finished the previous job's last tile
 // rewrites them (every MMA before it has completed by then) and releases
-// the MMA warp.  Every wait is bounded: a wait that gives up sets
+// the MMA warp.  The FWHT operand needs half the room, so there two are
+// resident: the first two rotations of the range are written at the start
+// by two groups at once, and the group that finishes rotation n's last tile
+// writes rotation n + 2 into the buffer n used, a whole rotation ahead of
+// its first MMA.  Every wait is bounded: a wait that gives up sets
 // KVQ_DEV_TIMEOUT and the CTA stops.
 //
 // Permutation + FWHT rotation ("RotateKV", abstract item (i); "KVLinC",
@@ -63,12 +67,13 @@ constexpr uint32_t TMEM_COLS = 128 * EPI_GROUPS;   // one 128-column fp32 accumu
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + A_STAGES * A_BYTES;
-constexpr int OFF_BAR = OFF_B + 2 * B_PART;
+constexpr int OFF_PINV = OFF_B + 2 * B_PART;  // FWHT: per epilogue warp, 128 B of scratch
 // barriers: full_a[A_STAGES], empty_a[A_STAGES], acc_full[EPI_GROUPS],
-// acc_empty[EPI_GROUPS], b_ready
+// acc_empty[EPI_GROUPS], b_ready[2] (one per B buffer)
 constexpr int BAR_FULL = 0, BAR_EMPTY = A_STAGES, BAR_ACCF = 2 * A_STAGES,
               BAR_ACCE = 2 * A_STAGES + EPI_GROUPS, BAR_BREADY = 2 * A_STAGES + 2 * EPI_GROUPS,
-              NBAR = 2 * A_STAGES + 2 * EPI_GROUPS + 1;
+              NBAR = 2 * A_STAGES + 2 * EPI_GROUPS + 2;
+constexpr int OFF_BAR = OFF_PINV + 128 * EPI_WARPS;
 constexpr int OFF_TMEMPTR = OFF_BAR + 8 * NBAR;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
 constexpr int SMEM_USED = OFF_ABORT + 16;
@@ -233,16 +238,18 @@ __device__ __forceinline__ int4 fwht_perm_regs(const TcArgs &a, bool to_cache, i
     return make_int4(pm[lane], pm[lane + 32], pm[lane + 64], pm[lane + 96]);
 }
 
-// The B operand of rotation key hk (cache: 2h + kind; test: 0) by the 128
-// threads of epilogue group eg; pv: fwht_perm_regs of hk (FWHT mode).
+// The B operand of rotation key hk (cache: 2h + kind; test: 0), written by
+// the 128 threads of one epilogue group (gt = thread in the group) into the
+// buffer at dst: dense, R_hi at dst and R_lo at dst + B_PART; FWHT, the +-1
+// matrix at dst.  pv: fwht_perm_regs of hk; pinv_w: the warp's 128 bytes of
+// scratch (FWHT mode).
 __device__ __forceinline__ void load_b(const TcArgs &a, bool to_cache, int hk, int4 pv,
-                                       uint8_t *bhi, uint8_t *blo, int gt, int eg) {
+                                       uint8_t *dst, uint8_t *pinv_w, int gt) {
     if (a.perm) {
-        // per-warp scratch in the lo part, unused by this rotation
-        build_fwht_b(pv, bhi, blo + 128 * (4 * eg + (gt >> 5)), gt);
+        build_fwht_b(pv, dst, pinv_w, gt);
     } else {
         const float *R = to_cache ? ((hk & 1) ? a.R1 : a.R0) + (size_t)(hk >> 1) * D * D : a.R0;
-        convert_r(R, bhi, blo, gt);
+        convert_r(R, dst, dst + tc::B_PART, gt);
     }
 }
 
@@ -260,7 +267,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
-    uint8_t *bhi = smem + OFF_B, *blo = smem + OFF_B + B_PART;
+    // B buffers: the dense operand (hi + lo) fills both halves of the B
+    // region; the FWHT operand (hi only) takes one half, so two rotations
+    // can be resident and the next one is built ahead of its first tile.
+    constexpr int NBUF = FWHT ? 2 : 1;
+    auto bbuf = [&](int x) { return smem + OFF_B + x * B_PART; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int k0 = blockIdx.x * a.tiles_per_cta;
@@ -270,6 +281,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     // tile k takes another rotation than tile k - 1 (divisions only at job
     // boundaries)
     auto new_rot = [&](int k) { return job_of(k) != job_of(k - 1) && rot_of(k) != rot_of(k - 1); };
+    // this CTA's rotations are rk0 .. rk_last, consecutive keys; the n-th
+    // (key rk0 + n) lives in B buffer n % NBUF, whose b_ready barrier
+    // completes its phase n / NBUF when the operand is written
+    const int rk0 = nmy > 0 ? rot_of(k0) : 0, rk_last = nmy > 0 ? rot_of(k0 + nmy - 1) : -1;
     auto fail = [&]() {
         set_status(c.status, KVQ_DEV_TIMEOUT);
         *abort_flag = 1;
@@ -284,7 +299,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_init(&bar[BAR_ACCF + i], 1);
             mbar_init(&bar[BAR_ACCE + i], 4);       // the four warps of an epilogue group
         }
-        mbar_init(&bar[BAR_BREADY], 4);
+        for (int i = 0; i < 2; i++) mbar_init(&bar[BAR_BREADY + i], 4);   // one group's 4 warps
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -333,13 +348,16 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     } else if (warp == 1) {
         // ---- MMA issuer
         if (lane == 0) {
-            int nb = 0;   // B-operand versions consumed
+            int nr = -1;   // rotation index (rot - rk0) of the current tile
             int i = 0;
             for (; i < nmy && !*abort_flag; i++) {
                 const int k = k0 + i, s = i % A_STAGES, buf = i % EPI_GROUPS;
                 if (i == 0 || new_rot(k)) {
-                    if (!mbar_wait_bounded(&bar[BAR_BREADY], nb & 1)) { fail(); break; }
-                    ++nb;
+                    ++nr;
+                    if (!mbar_wait_bounded(&bar[BAR_BREADY + nr % NBUF], (nr / NBUF) & 1)) {
+                        fail();
+                        break;
+                    }
                 }
                 if (i >= EPI_GROUPS &&
                     !mbar_wait_bounded(&bar[BAR_ACCE + buf], ((i / EPI_GROUPS) - 1) & 1)) {
@@ -353,7 +371,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 uint32_t acc = 0;
 #pragma unroll
                 for (int part = 0; part < (FWHT ? 1 : 2); part++) {
-                    const uint32_t bbase = smem_u32(part == 0 ? bhi : blo);
+                    const uint32_t bbase = smem_u32(bbuf(nr % NBUF) + part * B_PART);
 #pragma unroll
                     for (int kb = 0; kb < 2; kb++)
 #pragma unroll
@@ -376,13 +394,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int gt = threadIdx.x - 64 - 128 * eg;     // 0..127 within the group
         const int q = warp & 3;                         // TMEM lane quarter this warp may read
         const int row = 32 * q + lane;                  // accumulator row = tile row
-        if (eg == 0 && nmy > 0) {                       // R for the first job
-            load_b(a, TO_CACHE, rot_of(k0),
-                   FWHT ? fwht_perm_regs(a, TO_CACHE, rot_of(k0), lane) : make_int4(0, 0, 0, 0),
-                   bhi, blo, gt, eg);
+        uint8_t *pinv_w = smem + OFF_PINV + 128 * (warp - 2);
+        // the first NBUF rotations: group n writes rotation n
+        if (eg < NBUF && rk0 + eg <= rk_last) {
+            const int hk = rk0 + eg;
+            load_b(a, TO_CACHE, hk, FWHT ? fwht_perm_regs(a, TO_CACHE, hk, lane) : make_int4(0, 0, 0, 0),
+                   bbuf(eg), pinv_w, gt);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
+            if (lane == 0) mbar_arrive(&bar[BAR_BREADY + eg]);
         }
         int cur_job = -1, L0 = -1;
         int s_n = 0, s_last = -1;                       // identified sinks of the job's sequence
@@ -391,11 +411,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const int k = k0 + i, j = job_of(k), buf = i % EPI_GROUPS;     // = eg
             // global reads this tile needs, issued before the wait on its
-            // accumulator: the next rotation's permutation entries and the
-            // job's start length
-            const bool rebuild = i + 1 < nmy && new_rot(k + 1);
+            // accumulator: the permutation entries of the rotation it
+            // writes next (when it is its rotation's last tile and one more
+            // rotation follows beyond the resident ones) and the job's
+            // start length
+            const bool rebuild = i + 1 < nmy && new_rot(k + 1) && rot_of(k) + NBUF <= rk_last;
+            const int hk_next = rot_of(k) + NBUF;
             int4 pv = make_int4(0, 0, 0, 0);
-            if (FWHT && rebuild) pv = fwht_perm_regs(a, TO_CACHE, rot_of(k + 1), lane);
+            if (FWHT && rebuild) pv = fwht_perm_regs(a, TO_CACHE, hk_next, lane);
             int b = 0, h = 0, kind = 0;
             if (TO_CACHE) {
                 const int hk = j / a.B;
@@ -414,13 +437,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            // this tile's MMAs (and all earlier ones) are done: if the next tile
-            // takes another rotation, it goes into the B operand now
+            // this tile's MMAs (and all earlier ones) are done, so no MMA reads
+            // its rotation's buffer any more: the rotation NBUF further on
+            // goes into it now
             if (rebuild) {
-                load_b(a, TO_CACHE, rot_of(k + 1), pv, bhi, blo, gt, eg);
+                const int x = (rot_of(k) - rk0) % NBUF;
+                load_b(a, TO_CACHE, hk_next, pv, bbuf(x), pinv_w, gt);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[BAR_BREADY]);
+                if (lane == 0) mbar_arrive(&bar[BAR_BREADY + x]);
             }
             const int t = (k - j * a.tiles_per_job) * TILE_M + row;
             const bool valid = t < a.T && (!TO_CACHE || L0 >= 0);
@@ -433,10 +458,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             for (int g = 0; g < NG; g++) {
                 float v[32];
                 tmem_ld32(taddr + 32 * g, v);
-                if (FWHT) {                             // the FWHT's 1/sqrt(128), in fp32
-#pragma unroll
-                    for (int e = 0; e < 32; e++) v[e] *= 0.08838834764831845f;
-                }
+                if (FWHT) scale_group(v, 0.08838834764831845f);   // the FWHT's 1/sqrt(128), in fp32
                 if (g == NG - 1) {
                     // the accumulator is no longer needed: free it for the tile after next
                     tc_fence_before();

@@ -112,6 +112,40 @@ __device__ __forceinline__ QuantWord quantize_row_warp(const float v[4]) {
     return q;
 }
 
+// Two fp32 values in one 64-bit register, for sm_100's paired fp32
+// sub / mul: each lane is rounded to nearest even exactly as the
+// scalar instruction rounds it.  Unlike a scalar add.rn / mul.rn, a paired
+// product followed by a paired sum may be contracted into one fused
+// multiply-add by the assembler (one rounding instead of two; seen on
+// sm_100a), so where the exact two-step result matters a paired product
+// only ever feeds a scalar .rn operation.
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t x, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// v[e] *= c for the 32 values of a group, one rounding per value (scalar
+// mul.rn, never contracted with the subtraction that follows it in the
+// quantizer).
+__device__ __forceinline__ void scale_group(float (&v)[32], float c) {
+#pragma unroll
+    for (int e = 0; e < 32; e++) v[e] = __fmul_rn(v[e], c);
+}
+
 // One thread quantizes one group g of one row: v holds the group's 32
 // rotated values.  The codes are added into the 8 logical code words of the
 // row (word w = bytes 4w..4w+3; element e of the group at byte e, bits 2g)
@@ -145,21 +179,48 @@ __device__ __forceinline__ uint32_t quantize_group_thread(const float (&v)[32], 
     const float inv = (sF == 0.0f) ? 0.0f : __frcp_rn(sF);   // = the IEEE quotient 1/s
     constexpr float MAGIC = 12582912.0f;                     // 1.5 * 2^23
     constexpr uint32_t MAGIC_BITS = 0x4B400000u;
+    // sum_j (MAGIC_BITS << (8j + 2g)) (mod 2^32), taken out of every word
+    const uint32_t magic_sum = (MAGIC_BITS << (2 * g)) + (MAGIC_BITS << (8 + 2 * g)) +
+                               (MAGIC_BITS << (16 + 2 * g)) + (MAGIC_BITS << (24 + 2 * g));
+    // Every t = (x - z) * inv of the group lies in [t(min), t(max)]: the
+    // rounded difference and its rounded product with inv >= 0 are monotone
+    // in x.  When that interval lies in [-0.5, 3.5), rounding alone already
+    // gives every code the clamped value (t in [-0.5, 0) rounds to 0, the
+    // tie -0.5 to even 0; t in (3, 3.5) rounds to 3), so the clamp is
+    // skipped and x - z and its product with inv run two elements per
+    // instruction (the magic-constant sum stays a scalar add.rn, which is
+    // never fused with the product).  A NaN or infinite bound fails the
+    // test and takes the clamped path.
+    const float tlo = __fmul_rn(__fsub_rn(mn[0], zF), inv);
+    const float thi = __fmul_rn(__fsub_rn(mx[0], zF), inv);
+    if (tlo >= -0.5f && thi < 3.5f) {
+        const uint64_t z2 = f2_make(zF, zF), i2 = f2_make(inv, inv);
 #pragma unroll
-    for (int w = 0; w < 8; w++) {
-        uint32_t acc = words[w];
+        for (int w = 0; w < 8; w++) {
+            uint32_t acc = words[w];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int e = 4 * w + j;
-            float t = __fmul_rn(__fsub_rn(v[e], zF), inv);
-            t = fminf(fmaxf(t, 0.0f), 3.0f);
-            const uint32_t bits = __float_as_uint(__fadd_rn(t, MAGIC));
-            acc += bits << (8 * j + 2 * g);
+            for (int j = 0; j < 4; j += 2) {
+                const int e = 4 * w + j;
+                float a, b;
+                f2_split(f2_mul(f2_sub(f2_make(v[e], v[e + 1]), z2), i2), a, b);
+                acc += __float_as_uint(__fadd_rn(a, MAGIC)) << (8 * j + 2 * g);
+                acc += __float_as_uint(__fadd_rn(b, MAGIC)) << (8 * (j + 1) + 2 * g);
+            }
+            words[w] = acc - magic_sum;
         }
-        // remove sum_j (MAGIC_BITS << (8j + 2g)) (mod 2^32)
-        acc -= (MAGIC_BITS << (2 * g)) + (MAGIC_BITS << (8 + 2 * g)) + (MAGIC_BITS << (16 + 2 * g)) +
-               (MAGIC_BITS << (24 + 2 * g));
-        words[w] = acc;
+    } else {
+#pragma unroll
+        for (int w = 0; w < 8; w++) {
+            uint32_t acc = words[w];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int e = 4 * w + j;
+                float t = __fmul_rn(__fsub_rn(v[e], zF), inv);
+                t = fminf(fmaxf(t, 0.0f), 3.0f);
+                acc += __float_as_uint(__fadd_rn(t, MAGIC)) << (8 * j + 2 * g);
+            }
+            words[w] = acc - magic_sum;
+        }
     }
     return (uint32_t)__half_as_ushort(s) | ((uint32_t)__half_as_ushort(z) << 16);
 }
