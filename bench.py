@@ -376,7 +376,48 @@ def append_rates(device, peak, reps=5):
                      "ms": t * 1e3, "GB_per_s": nbytes / t / 1e9, "frac_of_hbm_peak": nbytes / t / 1e9 / peak,
                      "bytes": nbytes}
         del K, V, cache
+        if nbytes < 3 * L2_BYTES:
+            out[name].update(append_back_to_back(w, T, nbytes, rk, rv, pm, device, peak))
     return out
+
+
+def append_back_to_back(w, T, nbytes, rk, rv, pm, device, peak, calls=40):
+    """An append small enough for L2 timed as a serving loop runs it: `calls`
+    appends back to back between one pair of events (no flush, no host gap),
+    cycling over independent input sets and caches (distinct memory, at least
+    3x L2 of traffic between two uses of one set), each append at the next
+    position of its cache."""
+    import rotated_int2_kv_head_b200 as kvq
+    nset = -(-3 * L2_BYTES // nbytes) + 1
+    per = -(-calls // nset)
+    sets = []
+    for i in range(nset):
+        K, V = W.kv_batch(w, i * T, (i + 1) * T, device)
+        cache = kvq.KVCache(w.B, w.Hkv, T * per, w.sink, device=device)
+        sets.append((K, V, cache, torch.zeros(w.B, dtype=torch.int32, device=device)))
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def run():
+        for _, _, _, sl in sets:
+            sl.zero_()
+        host_ahead(500e-6)
+        ev[0].record()
+        for k in range(calls):
+            K, V, cache, sl = sets[k % nset]
+            kvq.kvq_rotate_quantize_append(K, V, w.mode, rk, rv, pm, cache, sl)
+        ev[1].record()
+        torch.cuda.synchronize(device)
+        return ev[0].elapsed_time(ev[1]) * 1e-3 / calls
+
+    run()                                   # warm-up
+    t = sorted(run() for _ in range(3))[1]
+    if max(kvq.kvq_get_status(c) for _, _, c, _ in sets) != 0:
+        raise RuntimeError("append status (back to back)")
+    del sets
+    torch.cuda.empty_cache()
+    return {"back_to_back_us": t * 1e6, "back_to_back_frac_of_hbm_peak": nbytes / t / 1e9 / peak,
+            "back_to_back_how": "%d appends between one event pair over %d independent input sets "
+                                "and caches, no flush; median of 3" % (calls, nset)}
 
 
 def extension_rates(device, reps=50):
@@ -533,8 +574,9 @@ def decode_rates(device, peak, reps=20):
     import rotated_int2_kv_head_b200 as kvq
     flush = L2Flush(device)
     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    res = {"how": "decode only, cache filled first, L2 flushed before each call, median of %d"
-                  % reps}
+    res = {"how": "decode only, cache filled first, L2 flushed before each call, median of %d; "
+                  "back_to_back_*: 40 decodes between one event pair over independent copies of "
+                  "the cache (no flush, no host gap), median of 3" % reps}
     for name in ("tiny", "llama7b", "hadamard", "gqa_sinks", "gqa8", "ragged"):
         w = W.WORKLOADS[name]
         lens_np = w.seq_lens().astype(np.int32)
@@ -576,9 +618,49 @@ def decode_rates(device, peak, reps=20):
                      "context_tokens_per_s": float(lens_np.astype(np.int64).sum()) * w.Hkv / t,
                      "packed_kv_bytes": kv, "packed_kv_gbs": kv / t / 1e9,
                      "frac_of_hbm_peak": kv / t / 1e9 / peak, "total_bytes_gbs": total / t / 1e9}
+        n_layers = layers_for(cache.blocks.numel())
+        if n_layers > 0:
+            tb = decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device)
+            res[name].update({"back_to_back_us": tb * 1e6,
+                              "back_to_back_frac_of_hbm_peak": kv / tb / 1e9 / peak,
+                              "back_to_back_layers": n_layers})
         del cache, ws
         torch.cuda.empty_cache()
     return res
+
+
+def decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device, calls=40):
+    """Decode as a serving loop runs it: `calls` decodes back to back between
+    one pair of events (no flush, no host gap), cycling over n_layers
+    independent copies of the cache (at least 3x L2 of other cache traffic
+    between two uses of one copy).  Median of 3 runs, seconds per decode."""
+    import rotated_int2_kv_head_b200 as kvq
+    layers = [cache]
+    for _ in range(1, n_layers):
+        c2 = kvq.KVCache(w.B, w.Hkv, cache.capacity, w.sink, device=device)
+        c2.blocks.copy_(cache.blocks)
+        if cache.k_sink is not None:
+            c2.k_sink.copy_(cache.k_sink)
+            c2.v_sink.copy_(cache.v_sink)
+        layers.append(c2)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def run():
+        host_ahead(500e-6)
+        ev[0].record()
+        for k in range(calls):
+            kvq.kvq_decode_attention(Q, layers[k % n_layers], w.mode, rk, rv, pm, lens, w.sink, L,
+                                     ws, out)
+        ev[1].record()
+        torch.cuda.synchronize(device)
+        return ev[0].elapsed_time(ev[1]) * 1e-3 / calls
+
+    run()                                   # warm-up
+    t = sorted(run() for _ in range(3))[1]
+    if max(kvq.kvq_get_status(c) for c in layers) != 0:
+        raise RuntimeError("decode status (back to back)")
+    del layers
+    return t
 
 
 def prerope_rates(device, reps=20):
