@@ -595,15 +595,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     uint32_t qB[4][C::NTK_STEP][2];
     float qsum[C::NTK], kap2[C::NTK];
     int Lcur = 0;
-    // online-softmax state
-    float m_run[G], l_run[C::HPL], O[8][4], Z[NW];
+    // online-softmax state; m_lane[hh] = m_run of the head this lane's
+    // scores in slot hh belong to (refreshed when the maxima move)
+    float m_run[G], m_lane[C::HPL], l_run[C::HPL], O[8][4], Z[NW];
     int cur_unit = -1;
 
     auto reset_state = [&]() {
 #pragma unroll
         for (int i = 0; i < G; i++) m_run[i] = NEG_INF;
 #pragma unroll
-        for (int i = 0; i < C::HPL; i++) l_run[i] = 0.f;
+        for (int i = 0; i < C::HPL; i++) {
+            l_run[i] = 0.f;
+            m_lane[i] = NEG_INF;
+        }
 #pragma unroll
         for (int i = 0; i < 8; i++)
 #pragma unroll
@@ -728,24 +732,24 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
         for (int bi = b_lo; bi < b_hi; bi++)
             kq[bi] = *reinterpret_cast<const uint4 *>(blk0 + bi * BLK_BYTES + 16 * (4 * r + c));
-#pragma unroll
-        for (int bi = b_lo; bi < b_hi; bi++)
-#pragma unroll
-            for (int nu = 0; nu < C::NTK; nu++)
-#pragma unroll
-                for (int k = 0; k < 4; k++) dk[bi][nu][k] = 0;
-        // one IMMA per group: the masked bytes are u8 codes c * 4^g
+        // one IMMA per group: the masked bytes are u8 codes c * 4^g.  The
+        // first group feeding an N tile starts its accumulator from zero.
 #pragma unroll
         for (int g = 0; g < 4; g++) {
             const uint32_t msk = 0x03030303u << (2 * g);
+            const bool first = g == 0 || (g * 2 * G) / 8 != ((g - 1) * 2 * G) / 8;
 #pragma unroll
             for (int bi = b_lo; bi < b_hi; bi++) {
                 const uint4 q4 = kq[bi];
 #pragma unroll
                 for (int j = 0; j < C::NTK_STEP; j++) {
                     const int nu = (g * 2 * G) / 8 + j;
-                    imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
-                              qB[g][j][0], qB[g][j][1]);
+                    if (first)
+                        imma16832_zc(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
+                                     qB[g][j][0], qB[g][j][1]);
+                    else
+                        imma16832(dk[bi][nu], q4.x & msk, q4.z & msk, q4.y & msk, q4.w & msk,
+                                  qB[g][j][0], qB[g][j][1]);
                 }
             }
         }
@@ -767,18 +771,25 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             for (int st = 0; st < 2; st++)
 #pragma unroll
                 for (int hh = 0; hh < C::HPL; hh++) part_sc[st][hh] = 0.f;
+            // the K-side N tiles of one group share the tokens' scale / zero:
+            // one tile per group for G <= 4, the group's two head halves for G = 8
+            constexpr int TPG = G >= 8 ? 2 : 1;
 #pragma unroll
-            for (int nu = 0; nu < C::NTK; nu++) {
-                const int g = ktile_group<G>(nu, c);
+            for (int gi = 0; gi < C::NTK / TPG; gi++) {
+                const int g = ktile_group<G>(gi * TPG, c);
                 const uint2 mk = *reinterpret_cast<const uint2 *>(blk0 + bi * BLK_BYTES + OFF_KM +
                                                                   8 * (4 * r + g));
                 const float2 sz0 = unpack_half2(mk.x), sz1 = unpack_half2(mk.y);
-                const int hh = ktile_slot<G>(nu);
-                // hi*254 + lo is exact in int32 (|.| < 2^28)
-                const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
-                const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
-                part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
-                part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
+#pragma unroll
+                for (int j = 0; j < TPG; j++) {
+                    const int nu = gi * TPG + j;
+                    const int hh = ktile_slot<G>(nu);
+                    // hi*254 + lo is exact in int32 (|.| < 2^28)
+                    const float d0 = __int2float_rn(dk[bi][nu][0] * 254 + dk[bi][nu][1]) * kap2[nu];
+                    const float d1 = __int2float_rn(dk[bi][nu][2] * 254 + dk[bi][nu][3]) * kap2[nu];
+                    part_sc[0][hh] = fmaf(sz0.x, d0, fmaf(sz0.y, qsum[nu], part_sc[0][hh]));
+                    part_sc[1][hh] = fmaf(sz1.x, d1, fmaf(sz1.y, qsum[nu], part_sc[1][hh]));
+                }
             }
 #pragma unroll
             for (int st = 0; st < 2; st++)
@@ -814,7 +825,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             for (int st = 0; st < 2; st++)
 #pragma unroll
                 for (int hh = 0; hh < C::HPL; hh++)
-                    over |= sco[bi][st][hh] > pick<G>(m_run, lane_head<G>(c, hh));
+                    over |= sco[bi][st][hh] > m_lane[hh];
         if (__any_sync(0xffffffffu, over)) {
         float mt[C::HPL];
 #pragma unroll
@@ -844,6 +855,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                 m_run[hd] = mnew[hd];
             }
 #pragma unroll
+            for (int hh = 0; hh < C::HPL; hh++) m_lane[hh] = pick<G>(m_run, lane_head<G>(c, hh));
+#pragma unroll
             for (int hh = 0; hh < C::HPL; hh++) l_run[hh] *= pick<G>(al, lane_head<G>(c, hh));
 #pragma unroll
             for (int k = 0; k < NW; k++) {
@@ -870,7 +883,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int hh = 0; hh < C::HPL; hh++) {
                     const float v = sco[bi][st][hh];
-                    const float mr = pick<G>(m_run, lane_head<G>(c, hh));
+                    const float mr = m_lane[hh];
                     // a masked score (-inf) must give exactly 0: with several
                     // queries per sequence a head can have seen no valid
                     // position yet (mr = -inf), so subtract 0 then

@@ -373,6 +373,16 @@ __device__ __forceinline__ void imma16832(int d[4], uint32_t a0, uint32_t a1, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same product into a fresh accumulator (C = 0, no zero-fill of d).
+__device__ __forceinline__ void imma16832_zc(int d[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
 // 2^x by the SFU's ex2.approx (max relative error about 2^-22; results
 // below 2^-126 flush to 0, which a softmax weight may do).
 __device__ __forceinline__ float fast_exp2(float x) {
