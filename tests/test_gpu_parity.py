@@ -195,6 +195,44 @@ def code_mismatches(blocks_a, blocks_b):
     return int(_NONZERO_CODES[x].sum())
 
 
+@pytest.mark.parametrize("mode,T", [(0, 37), (0, 300), (1, 37), (1, 200)])
+def test_gpu_cache_reads_as_documented(mode, T):
+    """The GPU's cache bytes read through the documented block format
+    (tests/block_format.py: no oracle or kernel offset code): every appended
+    position holds the codes and fp16 scale / zero that the oracle's
+    quantizer gives for the GPU's own rotated row, and every other position
+    of the cache is zero.  CUDA-core and tensor-core appends, both
+    rotations."""
+    from tests import block_format as bf
+    w = W.custom(seed=60 + T + mode, B=2, Hkv=2, mode=mode, k_outliers=4,
+                 channel_scale=(0.5, 20.0) if mode == 1 else None)
+    L0 = [3, 16]
+    cache, oc, K, V, rt, rn = run_append(w, L0, T)
+    got = bf.read_blocks(cache.block_view().cpu().numpy())      # [B][Hkv][nblk][16] ...
+    written = np.zeros(got["k"].shape[:4], bool)
+    for kind, X in ((0, K), (1, V)):
+        for h in range(w.Hkv):
+            rows = X[:, :, h].reshape(-1, D).cuda()
+            if mode == 0:
+                R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
+                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=append_variant(0, T))
+            else:
+                grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=rt[2][kind, h].contiguous(),
+                                                variant=append_variant(1, T))
+            grot = grot.cpu().numpy().reshape(w.B, T, D)
+            for b in range(w.B):
+                c, s, z = orc.quantize_rows(grot[b])
+                p = np.arange(L0[b], L0[b] + T)
+                blk, tau = p // 16, p % 16
+                key = ("k", "ks", "kz") if kind == 0 else ("v", "vs", "vz")
+                assert np.array_equal(got[key[0]][b, h, blk, tau], c)
+                assert np.array_equal(got[key[1]][b, h, blk, tau], s)
+                assert np.array_equal(got[key[2]][b, h, blk, tau], z)
+                written[b, h, blk, tau] = True
+    for name in ("k", "v", "ks", "kz", "vs", "vz"):
+        assert not got[name][~written].any()
+
+
 @pytest.mark.parametrize("path", ["dense_cuda_cores", "dense_tensor_cores", "fwht_step",
                                   "fwht_chunk", "fwht_tensor_cores", "prerope_gh4"])
 def test_near_tie_rate_over_a_million_codes(path):
