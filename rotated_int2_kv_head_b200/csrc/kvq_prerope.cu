@@ -328,6 +328,298 @@ __global__ void __launch_bounds__(PR_THREADS) prerope_split_kernel(PreRopeArgs a
     }
 }
 
+// ---- one KV head per group and one query per KV head (gh = G = 1) --------------------------
+// The same CTA ranges, warp runs and partials as prerope_split_kernel, but a
+// warp step takes four positions at once, eight lanes per position: lane
+// (p, j) = (lane >> 3, lane & 7) holds, of position tb + p, the elements
+// e = 32g + 4j + k (g, k < 4) of the stored (rotated) key and value, which
+// in the block layout are logical code word j: one 4-byte load per row.
+// The FWHT's index bits 0, 1 (k) and 5, 6 (g) are butterflies inside the
+// lane, bits 2, 3, 4 (j) across the position's eight lanes.  The
+// un-rotated key goes through shared memory in channel order (the
+// permutation scatter), and lane j takes back channels 8j..8j+7 and their
+// RoPE partners 64+8j..64+8j+7, so RoPE needs no shuffle; the dot product
+// is reduced over eight lanes; the online softmax runs once per step for
+// four positions; P.V accumulates the lane's 16 elements of the rotated
+// value.  RoPE angles: the lane's eight frequencies at its position, reduced
+// in fp64 at the warp's first step and every 64 steps, advanced by 4*theta_f
+// per step in between.
+constexpr int PRQ_POS = 4;              // positions per warp step
+constexpr int PRQ_REANCHOR = 64;        // steps between fp64 angle reductions
+// Row stride (floats) of a position's channel-order key in shared memory:
+// the four positions of a step scatter to the same channels, and the pad
+// of 8 puts them in four different bank octets.
+constexpr int PRQ_ROW = D + 8;
+
+__device__ __forceinline__ void prq_angles(const PreRopeArgs &a, int t, int j, float (&cs)[8],
+                                           float (&sn)[8]) {
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+        const double u = (double)t * a.phi[8 * j + m];
+        sincospif((float)(2.0 * (u - floor(u))), &sn[m], &cs[m]);
+    }
+}
+
+// The codes and {s, z} of one position that a lane reads: its logical K
+// word, its two V pieces and the four groups' K and V metadata.
+struct PrqLoad {
+    uint32_t kw, vw, km[4], vm[4];
+};
+
+__device__ __forceinline__ void prq_load(const PreRopeArgs &a, int b, int h, int t, int j,
+                                         PrqLoad &d) {
+    const long long bi = cache_block_index(a.table, a.num_blocks, a.nblk, a.Hkv, b, h, t / BLK_TOK);
+    if (bi < 0 && j == 0) set_status(a.status, KVQ_DEV_BAD_TABLE);
+    const uint8_t *bp = a.blocks + (size_t)(bi < 0 ? 0 : bi) * BLK_BYTES;
+    const int tau = t % BLK_TOK, r = tau & 7, th = tau >> 3, q2 = tau >> 1;
+    d.kw = *reinterpret_cast<const uint32_t *>(bp + 16 * (4 * r + (j & 3)) + 4 * (2 * th + (j >> 2)));
+    const int vo = 512 + 16 * (q2 & 3) + 4 * (2 * (q2 >> 2) + (j >> 2)) + 2 * (tau & 1);
+    const uint32_t v0 = *reinterpret_cast<const uint16_t *>(bp + vo + 64 * ((2 * j) & 7));
+    const uint32_t v1 = *reinterpret_cast<const uint16_t *>(bp + vo + 64 * ((2 * j + 1) & 7));
+    d.vw = v0 | (v1 << 16);
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+        d.km[g] = *reinterpret_cast<const uint32_t *>(bp + 1024 + 8 * (4 * r + g) + 4 * th);
+        d.vm[g] = *reinterpret_cast<const uint32_t *>(bp + 1280 + 8 * (4 * r + g) + 4 * th);
+    }
+}
+
+__global__ void __launch_bounds__(PR_THREADS) prerope_split_q_kernel(PreRopeArgs a) {
+    // Tables laid out so that the eight lanes of a position (j = 0..7) read
+    // consecutive words: no bank conflicts.
+    __shared__ __align__(16) float kb_s[PR_WARPS][PRQ_POS][PRQ_ROW];   // keys, channel order
+    __shared__ __align__(16) float2 step_s[8][8];     // [m][j]: cos, sin of 4 theta_(8j+m)
+    __shared__ __align__(16) float4 q_s[4][8];        // [quarter][j]: the query, exp2 domain
+    __shared__ __align__(16) uint4 off_s[2][8];       // [half][j]: lane j's scatter offsets
+    __shared__ float m_s[PR_WARPS], l_s[PR_WARPS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pp = lane >> 3, j = lane & 7;                     // position slot, lane in position
+    const int split = blockIdx.x;
+    const int b = blockIdx.y / a.Hkv, h = blockIdx.y % a.Hkv;
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x < D) {
+        // channel c: quarter (c >= 64) * 2 + (c % 8) / 4 of lane j = (c % 64) / 8
+        const int c = threadIdx.x, jj = (c & 63) >> 3, qu = 2 * (c >> 6) + ((c & 7) >> 2);
+        reinterpret_cast<float *>(&q_s[qu][jj])[c & 3] =
+            __half2float(__ushort_as_half(a.Q[((size_t)b * a.Hq + h) * D + c])) *
+            (PR_LOG2E * 0.08838834764831845f);
+        if (c < D / 2) {
+            float sn4, cs4;
+            const double u = 4.0 * a.phi[c];
+            sincospif((float)(2.0 * (u - floor(u))), &sn4, &cs4);
+            step_s[c & 7][c >> 3] = make_float2(cs4, sn4);
+        }
+    } else if (threadIdx.x < D + 64) {
+        // word w = 2g + k/2 of lane jj (k = 0, 2): perm[32g + 4jj + k] |
+        // perm[32g + 4jj + k + 1] << 16, where two elements of a position's
+        // un-rotated key go in its channel-order row
+        const int i = threadIdx.x - D, jj = i >> 3, w = i & 7, g = w >> 1, k = 2 * (w & 1);
+        const int32_t *pm = a.perm + (size_t)h * D + 32 * g + 4 * jj + k;
+        reinterpret_cast<uint32_t *>(&off_s[w >> 2][jj])[w & 3] =
+            (uint32_t)(pm[0] & (D - 1)) | ((uint32_t)(pm[1] & (D - 1)) << 16);
+    }
+    const int L = a.seq_lens[b];
+    const bool lok = L >= 1 && L <= a.capacity;
+    const int nb = lok ? (L + BLK_TOK - 1) / BLK_TOK : 0;
+    const int blk0 = split * a.bps, blk1 = min(nb, blk0 + a.bps);
+    __syncthreads();                                   // q_s, step_s, off_s
+    float *krow = &kb_s[warp][pp][0];
+
+    // the CTA's tokens in PR_WARPS contiguous, equal runs, one per warp
+    const int t_beg = min(L, max(a.S, blk0 * BLK_TOK)), t_end = max(t_beg, min(L, blk1 * BLK_TOK));
+    const int per = (t_end - t_beg + PR_WARPS - 1) / PR_WARPS;
+    const int w0 = min(t_end, t_beg + warp * per), w1 = min(t_end, w0 + per);
+
+    float m_run = PR_M0, l_run = 0.f, o[16], zacc[4];
+#pragma unroll
+    for (int i = 0; i < 16; i++) o[i] = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; g++) zacc[g] = 0.f;
+    float cs[8], sn[8];
+    PrqLoad cur, nxt;
+    if (w0 < w1) prq_load(a, b, h, min(w0 + pp, w1 - 1), j, cur);
+    int step = 0;
+    for (int tb = w0; tb < w1; tb += PRQ_POS, ++step) {
+        const int t = tb + pp;
+        const bool valid = t < w1;
+        // the next step's loads in flight during this one (positions past
+        // the run reload the run's last position)
+        if (tb + PRQ_POS < w1) prq_load(a, b, h, min(tb + PRQ_POS + pp, w1 - 1), j, nxt);
+        // the block two ahead into L2 (its 1536 bytes are 12 lines)
+        if ((tb & (BLK_TOK - 1)) < PRQ_POS && pp == 0 && tb + 2 * BLK_TOK < w1) {
+            const long long bn = cache_block_index(a.table, a.num_blocks, a.nblk, a.Hkv, b, h,
+                                                   tb / BLK_TOK + 2);
+            if (bn >= 0) {
+                const uint8_t *pf = a.blocks + (size_t)bn * BLK_BYTES + 128 * j;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(pf));
+                if (j < 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(pf + 1024));
+            }
+        }
+        if (step % PRQ_REANCHOR == 0) {
+            prq_angles(a, valid ? t : tb, j, cs, sn);
+        } else {
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                const float2 st = step_s[m][j];
+                const float c2 = cs[m] * st.x - sn[m] * st.y;
+                sn[m] = fmaf(sn[m], st.x, cs[m] * st.y);
+                cs[m] = c2;
+            }
+        }
+        // ---- key: dequantise (1/sqrt(128) folded into s and z), FWHT, scatter
+        float v[16];
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+            const float2 sz = unpack_half2(cur.km[g]);
+            const float s = sz.x * 0.08838834764831845f, z = sz.y * 0.08838834764831845f;
+            float c[4];
+            unpack4(cur.kw, g, c);
+#pragma unroll
+            for (int k = 0; k < 4; k++) v[4 * g + k] = fmaf(c[k], s, z);
+        }
+        // in-lane stages: v[4g + k] holds element 32g + 4j + k, so the
+        // strides 1, 2 are index bits 0, 1 (k) and 4, 8 are bits 5, 6 (g)
+#pragma unroll
+        for (int st = 1; st < 16; st <<= 1)
+#pragma unroll
+            for (int i = 0; i < 16; i++)
+                if ((i & st) == 0) {
+                    const float x0 = v[i], x1 = v[i + st];
+                    v[i] = x0 + x1;
+                    v[i + st] = x0 - x1;
+                }
+        // cross-lane stages: index bits 2, 3, 4 (j)
+#pragma unroll
+        for (int mk = 1; mk < 8; mk <<= 1) {
+            const float sgn = (j & mk) ? -1.f : 1.f;
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const float o2 = __shfl_xor_sync(0xffffffffu, v[i], mk);
+                v[i] = fmaf(sgn, v[i], o2);
+            }
+        }
+        // k_pre[perm[e]] = y[e]
+        {
+            const uint4 oa = off_s[0][j];
+            const uint4 ob4 = off_s[1][j];
+            const uint32_t off2[8] = {oa.x, oa.y, oa.z, oa.w, ob4.x, ob4.y, ob4.z, ob4.w};
+#pragma unroll
+            for (int w = 0; w < 8; w++) {
+                krow[off2[w] & 0xffffu] = v[2 * w];
+                krow[off2[w] >> 16] = v[2 * w + 1];
+            }
+        }
+        __syncwarp();
+        float x[8], xp[8];
+        {
+            const float4 a0 = *reinterpret_cast<const float4 *>(krow + 8 * j);
+            const float4 a1 = *reinterpret_cast<const float4 *>(krow + 8 * j + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(krow + 64 + 8 * j);
+            const float4 b1 = *reinterpret_cast<const float4 *>(krow + 64 + 8 * j + 4);
+            x[0] = a0.x; x[1] = a0.y; x[2] = a0.z; x[3] = a0.w;
+            x[4] = a1.x; x[5] = a1.y; x[6] = a1.z; x[7] = a1.w;
+            xp[0] = b0.x; xp[1] = b0.y; xp[2] = b0.z; xp[3] = b0.w;
+            xp[4] = b1.x; xp[5] = b1.y; xp[6] = b1.z; xp[7] = b1.w;
+        }
+        __syncwarp();
+        // RoPE at position t (channel c < 64 with its partner c + 64) and the
+        // dot with the query over this lane's 16 channels
+        float d = 0.f;
+        {
+            const float4 qa0 = q_s[0][j], qa1 = q_s[1][j], qb0 = q_s[2][j], qb1 = q_s[3][j];
+            const float qa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
+            const float qb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                const float xr = fmaf(-xp[m], sn[m], x[m] * cs[m]);
+                const float xpr = fmaf(x[m], sn[m], xp[m] * cs[m]);
+                d = fmaf(qa[m], xr, d);
+                d = fmaf(qb[m], xpr, d);
+            }
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        // an identified sink's slot (NaN scale) scores NaN: fmax with -inf
+        // makes it -inf, weight 0 (m_run starts at PR_M0, finite)
+        d = valid ? fmaxf(d, PR_NEG_INF) : PR_NEG_INF;
+        // ---- online softmax over the step's four positions
+        float mx = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (mx > m_run) {                              // uniform over the warp
+            const float al = fast_exp2(m_run - mx);
+            l_run *= al;
+#pragma unroll
+            for (int i = 0; i < 16; i++) o[i] *= al;
+#pragma unroll
+            for (int g = 0; g < 4; g++) zacc[g] *= al;
+            m_run = mx;
+        }
+        const float p = fast_exp2(d - m_run);
+        l_run += p;
+        // ---- P.V on the rotated value: o += (p s) c, zacc += p z per group
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+            const float2 sz = unpack_half2(cur.vm[g]);
+            float c[4];
+            unpack4(cur.vw, g, c);
+            const float ps = p * sz.x;
+#pragma unroll
+            for (int k = 0; k < 4; k++) o[4 * g + k] = fmaf(ps, c[k], o[4 * g + k]);
+            zacc[g] = fmaf(p, sz.y, zacc[g]);
+        }
+        cur = nxt;
+    }
+    // the four position slots hold partial sums over different positions
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        o[i] += __shfl_xor_sync(0xffffffffu, o[i], 8);
+        o[i] += __shfl_xor_sync(0xffffffffu, o[i], 16);
+    }
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+        zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 8);
+        zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 16);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+
+    // combine the warps through kb_s, reused as [PR_WARPS][128]
+    __syncthreads();
+    float *ob = &kb_s[0][0][0];
+    static_assert(PR_WARPS * D <= PR_WARPS * PRQ_POS * PRQ_ROW, "combine area");
+    if (pp == 0) {
+#pragma unroll
+        for (int g = 0; g < 4; g++)
+#pragma unroll
+            for (int k = 0; k < 4; k++) ob[warp * D + 32 * g + 4 * j + k] = o[4 * g + k] + zacc[g];
+        if (j == 0) {
+            m_s[warp] = m_run;
+            l_s[warp] = l_run;
+        }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += PR_THREADS) {
+        float mx = PR_NEG_INF;
+#pragma unroll
+        for (int w = 0; w < PR_WARPS; w++) mx = fmaxf(mx, m_s[w]);
+        float lt = 0.f, ot = 0.f;
+#pragma unroll
+        for (int w = 0; w < PR_WARPS; w++) {
+            const float f = exp2f(m_s[w] - mx);        // PR_M0 runs (no tokens): l = 0, o = 0
+            lt = fmaf(f, l_s[w], lt);
+            ot = fmaf(f, ob[w * D + c], ot);
+        }
+        float *pp2 = a.part + (((size_t)b * a.Hq + h) * a.nsplit + split) * PR_PART;
+        pp2[4 + c] = ot;
+        if (c == 0) {
+            pp2[0] = mx;
+            pp2[1] = lt;
+        }
+    }
+}
+
 // Merge of the splits and the inverse value rotation, one CTA of 128
 // threads per (b, query head).
 __global__ void __launch_bounds__(D) prerope_merge_kernel(PreRopeArgs a) {
@@ -461,7 +753,10 @@ cudaError_t launch_decode_prerope(const uint16_t *Q, int Hq, const kvq_cache_des
     const int G = Hq / cd.Hkv;
     cudaError_t e;
     switch (gh * 16 + G) {
-        case 1 * 16 + 1: e = launch_split_pr<1, 1>(a, st); break;
+        case 1 * 16 + 1:
+            e = launch_pdl(prerope_split_q_kernel, dim3(a.nsplit, a.B * a.Hkv), dim3(PR_THREADS), 0,
+                           st, a);
+            break;
         case 1 * 16 + 2: e = launch_split_pr<1, 2>(a, st); break;
         case 1 * 16 + 4: e = launch_split_pr<1, 4>(a, st); break;
         case 1 * 16 + 8: e = launch_split_pr<1, 8>(a, st); break;

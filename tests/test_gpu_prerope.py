@@ -140,8 +140,10 @@ def gpu_prerope_decode(cache, Q, gh, perm_t, lens_t, max_ctx):
 
 
 PR_DECODE_CASES = [
-    # gh, G, Hkv, lengths
+    # gh, G, Hkv, lengths (gh = G = 1 runs the four-positions-per-step kernel)
     (1, 1, 2, [1, 15, 16, 17, 300, 1000]),
+    (1, 1, 3, [2, 3, 4, 5, 7, 64, 65, 259, 4099]),
+    (1, 1, 1, [8191]),
     (2, 1, 4, [33, 512, 2047]),
     (2, 2, 2, [5, 19, 800]),
     (4, 2, 4, [4, 257, 1500]),
@@ -171,30 +173,34 @@ def test_prerope_decode_matches_oracle(gh, G, Hkv, lens):
     assert err.max() <= DEC_TOL, err.max()
 
 
-def test_prerope_decode_long_context():
-    """Positions up to 131071: the RoPE angles are reduced in fp64 per block."""
+@pytest.mark.parametrize("gh", [2, 1])
+def test_prerope_decode_long_context(gh):
+    """Positions up to 131071: the RoPE angles are reduced in fp64 (per block,
+    or every 64 steps of four positions for gh = 1) and advanced in fp32 in
+    between."""
     L = 131072
     w = _wl(251, 1, 2, 1)
-    perm = W.prerope_perm(w, 2)
-    oc = oracle_prerope_cache(w, 2, perm, [L], L)
+    perm = W.prerope_perm(w, gh)
+    oc = oracle_prerope_cache(w, gh, perm, [L], L)
     Q = W.queries(w, "cpu")
     sl = np.array([L], np.int32)
-    ref, st = orc.decode_prerope(oc, f16bits(Q), 2, perm, BASE, sl, n_threads=8)
+    ref, st = orc.decode_prerope(oc, f16bits(Q), gh, perm, BASE, sl, n_threads=8)
     assert st == 0
     cache = kvq.KVCache(1, 2, L)
     cache.blocks.copy_(torch.from_numpy(oc.blocks.reshape(-1)))
-    out = gpu_prerope_decode(cache, Q.cuda(), 2, torch.from_numpy(perm).cuda(),
+    out = gpu_prerope_decode(cache, Q.cuda(), gh, torch.from_numpy(perm).cuda(),
                              torch.from_numpy(sl).cuda(), L)
     err = rel_err(out.cpu().numpy(), ref)
     assert err.max() <= DEC_TOL, err.max()
 
 
+@pytest.mark.parametrize("gh,G", [(2, 2), (1, 1)])
 @pytest.mark.parametrize("paged", [False, True])
-def test_prerope_append_then_decode(paged):
+def test_prerope_append_then_decode(paged, gh, G):
     """GPU appends (37, 300 and single tokens) then the GPU decode, against the
     oracle's append + decode of the same tokens."""
-    gh, G, Hkv, B = 2, 2, 4, 3
-    w = _wl(260 + paged, B, Hkv, G)
+    Hkv, B = 4, 3
+    w = _wl(260 + paged + 10 * gh, B, Hkv, G)
     perm = W.prerope_perm(w, gh)
     pt = torch.from_numpy(perm).cuda()
     L0 = [0, 5, 16]
@@ -247,15 +253,16 @@ def test_prerope_bad_length_and_unsupported():
 
 # --- with fp16 sinks (RotateKV items ii and iii together) -----------------------------------------
 
+@pytest.mark.parametrize("gh,G", [(2, 2), (1, 1)])
 @pytest.mark.parametrize("identified", [False, True])
-def test_prerope_sinks_append_and_decode(identified):
+def test_prerope_sinks_append_and_decode(identified, gh, G):
     """Leading sinks (the first 4 positions) or identified ones (massive
     tokens): sink rows hold the pre-RoPE key exactly as given and the fp16
     of the kernel's rotated value; INT2 slots zero (identified: the K-scale
     marker); the decode against the oracle over appends of 37, 300 and 1
     tokens."""
-    gh, G, Hkv, B, S = 2, 2, 4, 3, 4
-    w = W.custom(seed=280 + identified, B=B, Hq=Hkv * G, Hkv=Hkv, mode=1, sink=S, k_outliers=4,
+    Hkv, B, S = 4, 3, 4
+    w = W.custom(seed=280 + identified + 10 * gh, B=B, Hq=Hkv * G, Hkv=Hkv, mode=1, sink=S, k_outliers=4,
                  sink_key_scale=50.0, massive_rate=0.01 if identified else 0.0)
     perm = W.prerope_perm(w, gh)
     pt = torch.from_numpy(perm).cuda()
