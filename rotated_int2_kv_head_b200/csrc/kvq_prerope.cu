@@ -9,8 +9,9 @@
 // values are rotated per head as in FWHT mode and the rotation is removed
 // once, after the attention.
 //
-// Two kernels:
-//   prerope_split_kernel<GH, G>  grid (splits, B * Hkv/GH).  A CTA of 8 warps
+// Split kernels (one per group shape) and a merge kernel:
+//   prerope_split_q_kernel  GH = G = 1 (below): four positions per warp step.
+//   prerope_split_kernel<GH, G>  every other shape; grid (splits, B * Hkv/GH).  A CTA of 8 warps
 //       takes a contiguous range of 16-token cache blocks of one (b, group),
 //       split into 8 equal token runs, one per warp, taken in order.  Per
 //       token: the GH heads' K codes are dequantised (4 elements
