@@ -619,22 +619,30 @@ def decode_rates(device, peak, reps=20):
                      "packed_kv_bytes": kv, "packed_kv_gbs": kv / t / 1e9,
                      "frac_of_hbm_peak": kv / t / 1e9 / peak, "total_bytes_gbs": total / t / 1e9}
         n_layers = layers_for(cache.blocks.numel())
-        if n_layers > 0:
-            tb = decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device)
-            res[name].update({"back_to_back_us": tb * 1e6,
-                              "back_to_back_frac_of_hbm_peak": kv / tb / 1e9 / peak,
-                              "back_to_back_layers": n_layers})
+        if n_layers == 0:
+            # too small to cycle out of L2: one distinct copy per call, L2 flushed
+            # once before each timed run, so every call still reads a cold cache
+            n_layers = -40
+        tb = decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device,
+                                 flush=flush if n_layers < 0 else None)
+        res[name].update({"back_to_back_us": tb * 1e6,
+                          "back_to_back_frac_of_hbm_peak": kv / tb / 1e9 / peak,
+                          "back_to_back_layers": abs(n_layers)})
         del cache, ws
         torch.cuda.empty_cache()
     return res
 
 
-def decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device, calls=40):
+def decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, device, calls=40,
+                        flush=None):
     """Decode as a serving loop runs it: `calls` decodes back to back between
-    one pair of events (no flush, no host gap), cycling over n_layers
-    independent copies of the cache (at least 3x L2 of other cache traffic
-    between two uses of one copy).  Median of 3 runs, seconds per decode."""
+    one pair of events (no host gap), cycling over n_layers independent
+    copies of the cache (at least 3x L2 of other cache traffic between two
+    uses of one copy).  A cache too small for that passes n_layers = -calls
+    and an L2 flush: one copy per call, L2 flushed once before each run
+    (outside the events).  Median of 3 runs, seconds per decode."""
     import rotated_int2_kv_head_b200 as kvq
+    n_layers = abs(n_layers)
     layers = [cache]
     for _ in range(1, n_layers):
         c2 = kvq.KVCache(w.B, w.Hkv, cache.capacity, w.sink, device=device)
@@ -646,6 +654,8 @@ def decode_back_to_back(w, cache, Q, rk, rv, pm, lens, L, ws, out, n_layers, dev
     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
 
     def run():
+        if flush is not None:
+            flush(0)
         host_ahead(500e-6)
         ev[0].record()
         for k in range(calls):
