@@ -756,14 +756,18 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     };
     // Scores, part 2: integer dots -> fp32 scores (group scale and zero,
     // query scale), summed over the groups; positions outside [S, L) and
-    // phantom blocks are masked to -inf.
-    auto k_combine = [&](const uint8_t *blk0, const int (&dk)[BPW][C::NTK][4], int tok0, int nmine,
-                         float (&sco)[BPW][2][C::HPL], bool (&edge)[BPW], int b_lo, int b_hi) {
+    // phantom blocks are masked to -inf.  A plain stage (every block of the
+    // warp's share real and inside [S, L), no identified sinks in the cache)
+    // needs neither the masks nor the NaN guard; PLAIN is a constant at
+    // each inlined call.
+    auto k_combine = [&](const bool PLAIN, const uint8_t *blk0, const int (&dk)[BPW][C::NTK][4],
+                         int tok0, int nmine, float (&sco)[BPW][2][C::HPL], bool (&edge)[BPW],
+                         int b_lo, int b_hi) {
         // a block needs masking if it is a phantom or crosses [S, L)
 #pragma unroll
         for (int bi = b_lo; bi < b_hi; bi++)
-            edge[bi] = bi >= nmine || tok0 + bi * BLK_TOK < a.S ||
-                       tok0 + (bi + 1) * BLK_TOK > Lcur - (a.qlen - 1);
+            edge[bi] = !PLAIN && (bi >= nmine || tok0 + bi * BLK_TOK < a.S ||
+                                  tok0 + (bi + 1) * BLK_TOK > Lcur - (a.qlen - 1));
 #pragma unroll
         for (int bi = b_lo; bi < b_hi; bi++) {
             float part_sc[2][C::HPL];
@@ -809,7 +813,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
                     }
                     // an identified sink's slot scores NaN (its K scale is the
                     // marker): fmax with -inf returns -inf for NaN, v otherwise
-                    sco[bi][st][hh] = fmaxf(v, NEG_INF);
+                    sco[bi][st][hh] = PLAIN ? v : fmaxf(v, NEG_INF);
                 }
         }
     };
@@ -1024,12 +1028,23 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
             // the K side in pairs of blocks (G = 8 one block at a time: the
             // integer accumulators of two would not fit the registers)
             constexpr int KSTEP = G >= 8 ? 1 : 2;
+            auto stage_body = [&](const bool PLAIN) {
 #pragma unroll
-            for (int b0 = 0; b0 < BPW; b0 += KSTEP) {
-                k_mma(wblk(s), dk, b0, b0 + KSTEP);
-                k_combine(wblk(s), dk, tok0, nmine, sco, edge, b0, b0 + KSTEP);
-            }
-            v_side(wblk(s), sco, edge);
+                for (int b0 = 0; b0 < BPW; b0 += KSTEP) {
+                    k_mma(wblk(s), dk, b0, b0 + KSTEP);
+                    k_combine(PLAIN, wblk(s), dk, tok0, nmine, sco, edge, b0, b0 + KSTEP);
+                }
+                v_side(wblk(s), sco, edge);
+            };
+            // uniform over the warp: all BPW blocks real, inside [S, L - qlen + 1),
+            // and no identified-sink markers possible.  Not for G = 8: its second
+            // copy of the stage body spills enough to cost what it saves.
+            const bool plain = G <= 4 && !a.sink_pos && nmine == BPW && tok0 >= a.S &&
+                               tok0 + BPW * BLK_TOK <= Lcur - (a.qlen - 1);
+            if (plain)
+                stage_body(true);
+            else
+                stage_body(false);
         }
         if (!ok) set_status(a.status, KVQ_DEV_TIMEOUT);
         if (release(s, ok)) {
