@@ -342,6 +342,42 @@ def test_decode_matches_oracle(G, mode, S, lens):
     assert kvq.kvq_get_status(cache) == 0
 
 
+@pytest.mark.parametrize("G,mode,q_len", [(1, 0, 1), (2, 1, 1), (4, 0, 1), (8, 1, 1), (1, 1, 4),
+                                           (4, 0, 2)])
+def test_interior_stage_shortcut_is_exact(G, mode, q_len):
+    """The split kernel skips the position masks and the NaN guard on stages
+    that lie wholly inside every query's context when the cache has no
+    identified sinks.  The same bytes in a cache that lists identified sinks
+    (none of them in use) take the general path on every stage: the two
+    decodes must agree bit for bit."""
+    Hkv = 2
+    lens = [q_len, 15, 16, 64, 65, 255, 256, 257, 1000, 2049, 4100]   # each at least q_len
+    w = W.custom(seed=70 + 10 * G + mode + q_len, B=len(lens), Hq=Hkv * G, Hkv=Hkv, mode=mode,
+                 k_outliers=4)
+    rt, _ = rot_tensors(w)
+    cap = ((max(lens) + 15) // 16) * 16
+    plain = kvq.KVCache(w.B, Hkv, cap, 0)
+    sl = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    K, V = W.kv_batch(w, 0, max(lens), "cpu")
+    gpu_append(plain, K.cuda(), V.cuda(), w, rt, sl)
+    listed = kvq.KVCache(w.B, Hkv, cap, 1, identified_sinks=True)
+    listed.blocks.copy_(plain.blocks)
+    assert not listed.sink_count.any()
+    lens_t = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    Q = torch.randn((w.B, w.Hq, q_len, D), generator=torch.Generator().manual_seed(G + q_len)).half().cuda()
+    outs = []
+    for c in (plain, listed):
+        ws = kvq.decode_workspace(w.B, w.Hq * q_len, Hkv, max(lens))
+        out = torch.empty_like(Q)
+        kvq.kvq_decode_attention_ex(Q, c, mode, rt[0], rt[1], rt[2], lens_t, c.sink_fp16, max(lens),
+                                    ws, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(plain) == 0 and kvq.kvq_get_status(listed) == 0
+    assert torch.isfinite(outs[0].float()).all()
+    assert torch.equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("G,mode,S,lens", DECODE_CASES[:3])
 def test_append_then_decode_end_to_end(G, mode, S, lens):
     """GPU append + GPU decode against oracle append + oracle decode."""
