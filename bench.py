@@ -577,6 +577,19 @@ def decode_rates(device, peak, reps=20):
     res = {"how": "decode only, cache filled first, L2 flushed before each call, median of %d; "
                   "back_to_back_*: 40 decodes between one event pair over independent copies of "
                   "the cache (no flush, no host gap), median of 3" % reps}
+    # the floor of the isolated timing itself: the same flush, spin and event
+    # pair around one trivial kernel (torch's spin of ~0 cycles)
+    fl = []
+    for k in range(reps + 3):
+        flush(k)
+        host_ahead(300e-6)
+        ev[0].record()
+        torch.cuda._sleep(1)
+        ev[1].record()
+        torch.cuda.synchronize(device)
+        if k >= 3:
+            fl.append(ev[0].elapsed_time(ev[1]))
+    res["event_pair_floor_us"] = float(np.median(fl)) * 1e3
     for name in ("tiny", "llama7b", "hadamard", "gqa_sinks", "gqa8", "ragged"):
         w = W.WORKLOADS[name]
         lens_np = w.seq_lens().astype(np.int32)
