@@ -332,8 +332,9 @@ def append_rates(device, peak, reps=5):
     """Throughput of the append alone (rotate + quantize + pack + store) on the
     bulk appends of the workload set: the llama7b prefill (B=1, 32768 tokens,
     32 heads, dense), the ragged workload's prefill (B=4, 32768 tokens, 32
-    heads, dense) and the hadamard workload's step append (B=16, 128 tokens,
-    32 heads, permutation + FWHT).  Bytes = fp16 K
+    heads, dense), the hadamard workload's step append (B=16, 128 tokens,
+    32 heads, permutation + FWHT) and a chunked-prefill append of the same
+    size with a dense rotation.  Bytes = fp16 K
     and V read (512 B per token-head) + packed codes and metadata written
     (96 B) + the rotations read once; L2 flushed before each timed call."""
     import rotated_int2_kv_head_b200 as kvq
@@ -347,7 +348,9 @@ def append_rates(device, peak, reps=5):
              ("ragged prefill", W.custom(name="ragged_prefill", seed=w0.seed + 1, B=w0.extra["prefill_B"],
                                          Hq=32, Hkv=32, mode=0, k_outliers=8,
                                          context=w0.extra["prefill_T"]), w0.extra["prefill_T"]),
-             ("hadamard step append", W.WORKLOADS["hadamard"], W.WORKLOADS["hadamard"].append_T)]
+             ("hadamard step append", W.WORKLOADS["hadamard"], W.WORKLOADS["hadamard"].append_T),
+             ("dense chunk append", W.custom(name="dense_chunk", seed=wl.seed + 2, B=16, Hq=32, Hkv=32,
+                                             mode=0, k_outliers=8, context=128), 128)]
     for name, w, T in cases:
         Rk, Rv, perm = W.rotations(w)
         rk = torch.from_numpy(Rk).to(device) if Rk is not None else None

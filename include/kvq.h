@@ -286,10 +286,11 @@ KVQ_API kvq_status kvq_clear_status(const kvq_cache_desc *cache, void *stream);
  *   -> Xrot fp32 [N][128].  `variant` selects the append kernel whose
  *   rotation is exercised: 0 = the small-batch kernels (CUDA cores), 1 = the
  *   bulk kernel on the tcgen05 tensor cores, used by appends with 16-byte
- *   aligned K and V of T >= 256 rows in dense mode (R split into fp16
- *   hi + lo) and of T >= 128 rows in FWHT mode (the product with the
- *   permuted +-1 Hadamard matrix, scaled by 1/sqrt(128) in fp32).  Other
- *   values: KVQ_ERR_INVALID_ARG.
+ *   aligned K and V of T new rows per sequence over B sequences when, in
+ *   dense mode (R split into fp16 hi + lo), T >= 32 or T >= 8 with
+ *   B*T >= 256, and in FWHT mode (the product with the permuted +-1
+ *   Hadamard matrix, scaled by 1/sqrt(128) in fp32), T >= 128 or T >= 32
+ *   with B*T >= 1024.  Other values: KVQ_ERR_INVALID_ARG.
  * kvq_debug_quantize_f32: Xrot fp32 [N][128] -> codes [N][32] in the logical
  *   packing, meta [N][4] as {s, z} fp16 pairs (uint16 [N][4][2]).
  */

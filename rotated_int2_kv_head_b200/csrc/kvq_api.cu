@@ -112,7 +112,7 @@ kvq_status append_launch(const uint16_t *K, const uint16_t *V, int32_t T, kvq_ro
                          const kvq_cache_desc *cache, int32_t *seq_lens, void *stream) {
     if (T == 0) return KVQ_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = append_tc_eligible(mode, K, V, T)
+    cudaError_t e = append_tc_eligible(mode, K, V, T, cache->B)
                         ? launch_append_tc(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st)
                         : launch_append_small(K, V, T, mode, R_k, R_v, perm, *cache, seq_lens, st);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;

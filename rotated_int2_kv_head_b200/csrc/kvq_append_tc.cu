@@ -577,10 +577,20 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, TcArgs a, co
 
 }  // namespace
 
-bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T) {
+// Which appends take this kernel rather than the CUDA-core ones, from their
+// crossovers measured on B200 (32 KV heads, L2 flushed before each call):
+// a dense rotation from 32 new tokens per sequence, or from 8 when the batch
+// brings at least 256 rows (below that the CUDA-core kernel, which shares one
+// fetch of R among several sequences, wins); the permutation + FWHT form,
+// whose CUDA-core kernels do far less arithmetic, from 128 tokens, or from
+// 32 when the batch brings at least 1024 rows.  A job shorter than a tile
+// loads 128 rows and drops those past its own T.
+bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T, int B) {
     const auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    return T >= (mode == KVQ_ROT_DENSE ? TC_MIN_T : TC_MIN_T_FWHT) && al(K) && al(V) &&
-           encode_fn() != nullptr;
+    const long long rows = (long long)B * T;
+    const bool worth = mode == KVQ_ROT_DENSE ? (T >= 32 || (T >= 8 && rows >= 256))
+                                             : (T >= 128 || (T >= 32 && rows >= 1024));
+    return worth && al(K) && al(V) && encode_fn() != nullptr;
 }
 
 cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, int mode,

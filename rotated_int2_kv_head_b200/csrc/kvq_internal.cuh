@@ -437,11 +437,10 @@ cudaError_t launch_append_small(const uint16_t *K, const uint16_t *V, int T, int
                                 cudaStream_t st);
 cudaError_t launch_debug_rotate_small(const uint16_t *X, int N, int mode, const float *R,
                                       const int32_t *perm, float *out, cudaStream_t st);
-// Bulk appends (T >= TC_MIN_T dense, T >= TC_MIN_T_FWHT permutation +
-// FWHT; 16-byte aligned K and V) run the rotation on the tensor cores.
-constexpr int TC_MIN_T = 256;
-constexpr int TC_MIN_T_FWHT = 128;
-bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T);
+// Whether an append of T rows per sequence over B sequences (16-byte aligned
+// K and V) runs its rotation on the tensor cores (the size rule is beside
+// the kernel).
+bool append_tc_eligible(int mode, const uint16_t *K, const uint16_t *V, int T, int B);
 cudaError_t launch_append_tc(const uint16_t *K, const uint16_t *V, int T, int mode,
                              const float *R_k, const float *R_v, const int32_t *perm,
                              const kvq_cache_desc &cd, int32_t *seq_lens, cudaStream_t st);

@@ -21,11 +21,15 @@ def rot_tensors(w, device="cuda"):
     return (None, None, torch.from_numpy(perm).to(device)), (None, None, perm)
 
 
-def append_variant(mode, T):
+def append_variant(mode, T, B):
     """The rotation variant of kvq_debug_rotate_f32 that an append of T rows
-    runs: 1 = the tensor-core bulk kernel (dense T >= 256, permutation +
-    FWHT T >= 128), else 0."""
-    return 1 if T >= (256 if mode == 0 else 128) else 0
+    per sequence over B sequences runs (the library's documented size rule):
+    1 = the tensor-core bulk kernel (dense: T >= 32, or T >= 8 with
+    B*T >= 256; permutation + FWHT: T >= 128, or T >= 32 with B*T >= 1024),
+    else 0."""
+    if mode == 0:
+        return 1 if T >= 32 or (T >= 8 and B * T >= 256) else 0
+    return 1 if T >= 128 or (T >= 32 and B * T >= 1024) else 0
 
 
 def gpu_append(cache, K, V, w, rt, seq_lens):

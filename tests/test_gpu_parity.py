@@ -111,13 +111,26 @@ def run_append(w, L0, T, device="cuda"):
 
 
 @pytest.mark.parametrize("mode,S,T,L0", [
+    # CUDA-core appends (dense: T < 32 and B*T < 256 or T < 8; permutation
+    # + FWHT: T < 128 and B*T < 1024 or T < 32)
     (0, 0, 1, [0, 5, 16]),
-    (0, 4, 37, [0, 3, 29]),
+    (0, 4, 16, [0, 3, 29]),
+    (0, 20, 31, [0, 2, 31]),
+    (0, 4, 7, list(range(0, 80, 2))),            # B*T = 280 rows, T < 8
+    (0, 0, 8, list(range(0, 62, 2))),            # B = 31: 248 rows
     (1, 0, 37, [0, 5, 16]),
     (1, 4, 1, [3, 0, 21]),
+    (1, 0, 31, list(range(0, 80, 2))),           # B*T = 1240 rows, T < 32
+    # tensor-core appends of a partial tile per job: dense from T = 32, and
+    # from T = 8 with B*T = 256 rows; FWHT from T = 32 with B*T = 1024
+    (0, 0, 32, [0, 5, 16]),
+    (0, 4, 37, [0, 3, 29]),
     (0, 20, 70, [0, 2, 31]),
-    # bulk dense appends (T >= 256): tensor-core kernel; T=2400 gives 228
-    # tiles, so CTAs cross (sequence, head, K|V) boundaries mid-range
+    (0, 4, 8, list(range(0, 64, 2))),            # B = 32: 256 rows
+    (1, 4, 32, list(range(0, 64, 2))),           # B = 32: 1024 rows
+    (1, 0, 64, list(range(1, 33, 2))),           # B = 16: 1024 rows
+    # bulk dense appends: T=2400 gives 228 tiles, so CTAs cross (sequence,
+    # head, K|V) boundaries mid-range
     (0, 20, 520, [0, 2, 31]),
     (0, 0, 2400, [0, 7, 16]),
     # bulk permutation + FWHT appends (T >= 128): the same tensor-core kernel
@@ -128,7 +141,7 @@ def run_append(w, L0, T, device="cuda"):
     (1, 0, 2400, [0, 7, 16]),
 ])
 def test_append_matches_oracle(mode, S, T, L0):
-    w = W.custom(seed=10 + T, B=3, Hkv=2, mode=mode, sink=S, k_outliers=4,
+    w = W.custom(seed=10 + T, B=len(L0), Hkv=2, mode=mode, sink=S, k_outliers=4,
                  channel_scale=(0.5, 20.0) if mode == 1 else None)
     cache, oc, K, V, rt, rn = run_append(w, L0, T)
     gc = download_cache(cache)
@@ -141,14 +154,14 @@ def test_append_matches_oracle(mode, S, T, L0):
             rows = X[:, :, h].reshape(-1, D).cuda()
             if mode == 0:
                 R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
-                variant = append_variant(0, T)     # the kernel the append used
+                variant = append_variant(0, T, w.B)   # the kernel the append used
                 grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=variant).cpu().numpy()
                 orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 0,
                                       R=(rn[0] if kind == 0 else rn[1])[h])
             else:
                 pm = rt[2][kind, h].contiguous()
                 grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=pm,
-                                                variant=append_variant(1, T)).cpu().numpy()
+                                                variant=append_variant(1, T, w.B)).cpu().numpy()
                 orot = orc.rotate_f64(orc.f16_bits_to_f32(f16bits(rows)).astype(np.float64), 1,
                                       perm=rn[2][kind, h])
             grot = grot.reshape(w.B, T, D)
@@ -195,7 +208,7 @@ def code_mismatches(blocks_a, blocks_b):
     return int(_NONZERO_CODES[x].sum())
 
 
-@pytest.mark.parametrize("mode,T", [(0, 37), (0, 300), (1, 37), (1, 200)])
+@pytest.mark.parametrize("mode,T", [(0, 20), (0, 37), (0, 300), (1, 37), (1, 200)])
 def test_gpu_cache_reads_as_documented(mode, T):
     """The GPU's cache bytes read through the documented block format
     (tests/block_format.py: no oracle or kernel offset code): every appended
@@ -215,10 +228,10 @@ def test_gpu_cache_reads_as_documented(mode, T):
             rows = X[:, :, h].reshape(-1, D).cuda()
             if mode == 0:
                 R = (rt[0] if kind == 0 else rt[1])[h].contiguous()
-                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=append_variant(0, T))
+                grot = kvq.kvq_debug_rotate_f32(rows, 0, R=R, variant=append_variant(0, T, w.B))
             else:
                 grot = kvq.kvq_debug_rotate_f32(rows, 1, perm=rt[2][kind, h].contiguous(),
-                                                variant=append_variant(1, T))
+                                                variant=append_variant(1, T, w.B))
             grot = grot.cpu().numpy().reshape(w.B, T, D)
             for b in range(w.B):
                 c, s, z = orc.quantize_rows(grot[b])
@@ -239,13 +252,13 @@ def test_near_tie_rate_over_a_million_codes(path):
     """Codes that differ between the packed cache and the oracle's append of
     the same rows (its fp64 rotation) come only from near ties: at most 1e-4
     of the codes, counted over 2,097,152 codes (2048 tokens x 4 heads x K and
-    V) for every append kernel - the CUDA-core dense append (T < 256), the
-    tensor-core bulk append (dense, and permutation + FWHT), the CUDA-core
-    FWHT append a few tokens at a time and in chunks, and the pre-RoPE group
-    rotation."""
+    V) for every append kernel - the CUDA-core dense append (16 tokens at a
+    time), the tensor-core bulk append (dense, and permutation + FWHT), the
+    CUDA-core FWHT append a few tokens at a time and in chunks, and the
+    pre-RoPE group rotation."""
     Hkv, T = 4, 2048
     mode = 0 if path.startswith("dense") else 1
-    chunk = {"dense_cuda_cores": 128, "dense_tensor_cores": T, "fwht_step": 8,
+    chunk = {"dense_cuda_cores": 16, "dense_tensor_cores": T, "fwht_step": 8,
              "fwht_chunk": 64, "fwht_tensor_cores": T, "prerope_gh4": 256}[path]
     w = W.custom(seed=540 + len(path), B=1, Hq=Hkv, Hkv=Hkv, mode=mode, context=T,
                  k_outliers=8, channel_scale=(0.5, 20.0) if mode == 1 else None)

@@ -124,7 +124,7 @@ def test_append_identified_sinks(mode, chunks, paged):
         gpu_append(plain, K.cuda(), V.cuda(), w, rt, sl_p)
         orc.identify_sinks(oc, act, TAU, osl)
         assert orc.append(oc, f16bits(K), f16bits(V), w.mode, rn[0], rn[1], rn[2], osl) == 0
-        rows.append((list(pos), K, V, append_variant(mode, T)))
+        rows.append((list(pos), K, V, append_variant(mode, T, B)))
         pos = [p + T for p in pos]
     torch.cuda.synchronize()
     assert kvq.kvq_get_status(ic) == 0 and kvq.kvq_get_status(plain) == 0
