@@ -543,8 +543,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     // Copies.  Ring slot `slot` is filled with the next stage of the group's
     // range, with its descriptor {unit, b, h, first cache block}, {n}; unit -1
     // marks the end (the slot's phase is completed by a plain arrive).
-    // Descriptors are written NS-1 group barriers before anyone reads them,
-    // so they are read without waiting on the copy.
+    // Descriptors are written at least one group barrier before anyone
+    // reads them, so they are read without waiting on the copy.
     // Producer: the group leader for a contiguous cache (a stage is one bulk
     // copy); the group's whole first warp for a paged one, all lanes in step
     // (the schedule state sc evolves identically in every lane), lane j
@@ -584,8 +584,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
         ++issued;
     };
     const bool producer = PAGED ? warp == 0 : leader;   // contiguous: lane 0 alone suffices
+    // A range of 3 to 8 stages (short contexts, where the start is a large
+    // part of the kernel) issues its first stage alone and the rest of the
+    // ring once that stage has landed: when every group asks for its whole
+    // ring at once, the copies issued last land over 2 us after the first
+    // (llama7b: 29 MB at once) and those groups also finish last.  With two
+    // stages the second one's later copy would end the range later; G <= 2
+    // only: the G = 4 and 8 kernels have no registers to spare for it.
+    const int span = sc.end - sc.cur;
+    const bool staged = G <= 2 && span > 2 * STAGE_BLKS && span <= 8 * STAGE_BLKS;
     if (producer)
-        for (int k = 0; k < NS; k++) issue_next(k);
+        for (int k = 0; k < (staged ? 1 : NS); k++) issue_next(k);
     bar_group();
     pdl_wait();
     pdl_trigger();
@@ -1002,6 +1011,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 1) decode_split_kernel(DecodeArgs
     auto wblk = [&](int slot) { return ring + slot * STAGE_BYTES + (BPW * warp) * BLK_BYTES; };
 
     reset_state();
+    if (staged) {
+        // staged start, before the loop so that the loop is the same for
+        // every range: the first unit's queries, then (producer) the rest of
+        // the ring once stage 0 has landed.  After a failed wait it stays
+        // unissued; the loop's own wait then fails and the group drains.
+        const int4 d0 = desc[0];
+        if (d0.x >= 0) {
+            load_unit(d0.y, d0.z);
+            cur_unit = d0.x;
+        }
+        if (producer && mbar_wait_bounded(&full[0], 0))
+            for (int k = 1; k < NS; k++) issue_next(k);
+    }
     bool aborted = false;
     int it = 0;
     for (;; ++it) {
