@@ -391,6 +391,69 @@ def test_interior_stage_shortcut_is_exact(G, mode, q_len):
     assert torch.equal(outs[0], outs[1])
 
 
+def split_group_spans(B, Hkv, max_ctx, lens, S, sms):
+    """Schedule slots of every group of the split kernel, from the library's
+    stream-K split: min(SMs, blocks / 64) CTAs over the slots of all units
+    (a non-empty unit: 8 leading slots, then one per 16-token block), each
+    CTA's share cut into four contiguous group ranges."""
+    blocks = B * Hkv * (-(-max_ctx // 16))
+    C = max(1, min(sms, -(-blocks // 64)))
+    def slots(L):
+        nb = (L - 1) // 16 - S // 16 + 1 if S < L else 0
+        return nb + 8 if nb > 0 else 0
+    N = sum(Hkv * slots(L) for L in lens)
+    W_ = max(1, -(-N // C))
+    spans = []
+    for c in range(C):
+        beg, end = c * W_, min(N, c * W_ + W_)
+        if beg >= end:
+            continue
+        wg = -(-(end - beg) // 4)
+        spans += [min(end, p + wg) - p for p in range(beg, beg + 4 * wg, wg) if p < end]
+    return spans
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_staged_start_matches_oracle(G):
+    """Short contexts, where every group of the split kernel has a range of
+    3 to 8 stages and so takes the staged ring start (its first stage alone,
+    the rest of its ring once that stage has landed), with units starting
+    inside most ranges: the decode against the oracle on the same cache
+    bytes, and through a paged copy of the cache (a random block table),
+    whose producer is a whole warp, bit for bit the same."""
+    B, Hkv = 8, 8
+    lens = [int(x) for x in np.random.default_rng(500 + G).integers(3000, 14000, B)]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    spans = split_group_spans(B, Hkv, max(lens), lens, 0, sms)
+    assert sum(32 < s <= 128 for s in spans) >= 0.9 * len(spans)       # 16 blocks per stage
+    w = W.custom(seed=510 + G, B=B, Hq=Hkv * G, Hkv=Hkv, mode=0, k_outliers=4)
+    rt, rn = rot_tensors(w)
+    cap = ((max(lens) + 15) // 16) * 16
+    cache = kvq.KVCache(B, Hkv, cap, 0)
+    sl = torch.zeros(B, dtype=torch.int32, device="cuda")
+    for t0 in range(0, max(lens), 4096):
+        K, V = W.kv_batch(w, t0, min(max(lens), t0 + 4096), "cuda")
+        gpu_append(cache, K, V, w, rt, sl)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    Q = W.queries(w, "cuda")
+    out = gpu_decode(cache, Q, w, rt, lens_t, max(lens))
+    nblk = cap // 16
+    num_blocks = B * nblk + 5
+    table = torch.randperm(num_blocks, generator=torch.Generator().manual_seed(7))[:B * nblk]
+    table = table.view(B, nblk).to(torch.int32).cuda()
+    paged = kvq.PagedKVCache(B, Hkv, cap, num_blocks, table, 0)
+    paged.block_view()[table.view(-1).long()] = cache.block_view().permute(0, 2, 1, 3).reshape(
+        B * nblk, Hkv, -1)
+    assert torch.equal(paged.logical_view(), cache.block_view())
+    out_p = gpu_decode(paged, Q, w, rt, lens_t, max(lens))
+    torch.cuda.synchronize()
+    assert kvq.kvq_get_status(cache) == 0 and kvq.kvq_get_status(paged) == 0
+    assert torch.equal(out, out_p)
+    oc = download_cache(cache)
+    ref, _ = orc.decode(oc, f16bits(Q.cpu()), 0, rn[0], rn[1], None, np.array(lens, np.int32))
+    assert rel_err(out.float().cpu().numpy(), ref).max() <= DEC_TOL
+
+
 @pytest.mark.parametrize("G,mode,S,lens", DECODE_CASES[:3])
 def test_append_then_decode_end_to_end(G, mode, S, lens):
     """GPU append + GPU decode against oracle append + oracle decode."""
